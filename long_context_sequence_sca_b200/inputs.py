@@ -1,0 +1,119 @@
+"""Seeded synthetic inputs for the Gecko SCA + AWM forward.
+
+This module is shared by the CUDA path's tests/bench and by the CPU oracle's
+tests. It holds none of the method's arithmetic: it only draws the five
+per-head input tensors (Q, K, V, Q_m, K_m) with the shapes and value
+distributions of the projections that feed the layer ("Gecko: An Efficient
+Neural Architecture ...", method step details, steps 2 and 4): a shared
+representation Z' normalised to unit L2 norm per token, per-(head, dim)
+affine maps for the queries and keys, and SiLU values.
+
+Recipe, per tensor and per (b, h, t):
+  g ~ N(0, 1)^d,  Z' = g / ||g||_2
+  Q   = kappa_q * Z' + nu_q      K   = kappa_k * Z' + nu_k
+  Q_m = eta_q   * Z' + rho_q     K_m = eta_k   * Z' + rho_k
+  scales ~ N(1, 0.1^2), offsets ~ N(0, 0.1^2) (per head and dim)
+  V = SiLU(N(0, 1)) elementwise
+Everything is drawn in fp32 and then cast (round-to-nearest-even) to the
+workload's dtype.  The small fp32 workload shares one Z' across Q, K, Q_m,
+K_m (seed 0); the others draw each tensor from its own seed
+100 * workload_id + {Q: 0, K: 1, V: 2, Q_m: 3, K_m: 4}.
+"""
+from __future__ import annotations
+
+import dataclasses
+import torch
+
+TENSORS = ("q", "k", "v", "qm", "km")
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    """One synthetic workload: shape, dtype and generator options."""
+    name: str
+    wid: int                 # workload id used in the seed formula
+    dtype: str               # "f32" or "bf16"
+    B: int
+    H: int
+    T: int
+    d: int
+    c: int
+    shared_z: bool = False   # one Z' for Q, K, Q_m, K_m (small fp32 case)
+    key_offset_std: float = 0.1  # std of nu_k and rho_k
+
+    @property
+    def S(self) -> int:
+        return self.T // self.c
+
+    @property
+    def torch_dtype(self):
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+    def with_(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+
+# The workloads: a small fp32 case, a many-chunk bf16 case, the 7B-layer-shaped
+# headline case (H=32, d=128, c=4096), the chunk-size sweep with wide key
+# offsets, and the 4M-token case.
+WORKLOADS = {
+    "fp32_small": Workload("fp32_small", 1, "f32", 1, 1, 512, 64, 64, shared_z=True),
+    "bf16_many_chunks": Workload("bf16_many_chunks", 2, "bf16", 2, 8, 4096, 64, 256),
+    "bf16_h32_c4096": Workload("bf16_h32_c4096", 3, "bf16", 1, 32, 32768, 128, 4096),
+    "bf16_sweep_c512": Workload("bf16_sweep_c512", 4, "bf16", 1, 32, 65536, 128, 512, key_offset_std=1.0),
+    "bf16_sweep_c1024": Workload("bf16_sweep_c1024", 4, "bf16", 1, 32, 65536, 128, 1024, key_offset_std=1.0),
+    "bf16_sweep_c2048": Workload("bf16_sweep_c2048", 4, "bf16", 1, 32, 65536, 128, 2048, key_offset_std=1.0),
+    "bf16_sweep_c4096": Workload("bf16_sweep_c4096", 4, "bf16", 1, 32, 65536, 128, 4096, key_offset_std=1.0),
+    "bf16_4m_tokens": Workload("bf16_4m_tokens", 5, "bf16", 1, 8, 4194304, 128, 4096),
+}
+
+
+def _unit_rows(gen: torch.Generator, n: int, d: int, device) -> torch.Tensor:
+    g = torch.randn(n, d, generator=gen, device=device, dtype=torch.float32)
+    return g / g.norm(dim=1, keepdim=True)
+
+
+def _affine(gen: torch.Generator, H: int, d: int, off_std: float, device):
+    scale = 1.0 + 0.1 * torch.randn(H, d, generator=gen, device=device, dtype=torch.float32)
+    off = off_std * torch.randn(H, d, generator=gen, device=device, dtype=torch.float32)
+    return scale, off
+
+
+def _silu(x: torch.Tensor) -> torch.Tensor:
+    return x * torch.sigmoid(x)
+
+
+def make_inputs(w: Workload, device="cpu", seed_offset: int = 0) -> dict:
+    """Draw q, k, v, qm, km as [B, H, T, d] tensors of the workload's dtype.
+
+    Large workloads are drawn one (b, h) slab at a time so the fp32
+    temporaries stay small; each slab has its own generator seeded from the
+    tensor seed and the slab index, so results do not depend on slab order.
+    """
+    B, H, T, d = w.B, w.H, w.T, w.d
+    dt = w.torch_dtype
+    out = {n: torch.empty(B, H, T, d, dtype=dt, device=device) for n in TENSORS}
+    if w.shared_z:
+        gen = torch.Generator(device=device).manual_seed(0 + seed_offset)
+        z = _unit_rows(gen, B * H * T, d, device).view(B, H, T, d)
+        for name in ("q", "k", "qm", "km"):
+            std = w.key_offset_std if name in ("k", "km") else 0.1
+            sc, off = _affine(gen, H, d, std, device)
+            out[name].copy_((sc[None, :, None, :] * z + off[None, :, None, :]).to(dt))
+        out["v"].copy_(_silu(torch.randn(B, H, T, d, generator=gen, device=device)).to(dt))
+        return out
+    for idx, name in enumerate(TENSORS):
+        seed = 100 * w.wid + idx + seed_offset
+        gen = torch.Generator(device=device).manual_seed(seed)
+        if name != "v":
+            std = w.key_offset_std if name in ("k", "km") else 0.1
+            sc, off = _affine(gen, H, d, std, device)
+        for b in range(B):
+            for h in range(H):
+                sg = torch.Generator(device=device).manual_seed(seed * 1000003 + b * H + h)
+                if name == "v":
+                    slab = _silu(torch.randn(T, d, generator=sg, device=device, dtype=torch.float32))
+                else:
+                    slab = sc[h] * _unit_rows(sg, T, d, device) + off[h]
+                out[name][b, h].copy_(slab.to(dt))
+    return out
