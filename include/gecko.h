@@ -1,0 +1,123 @@
+/*
+ * gecko.h - C ABI of the Gecko fused forward for NVIDIA B200 (sm_100a).
+ *
+ * The library computes, per (batch b, head h), the two attention parts of a
+ * Gecko layer ("Gecko: An Efficient Neural Architecture Inherently Processing
+ * Sequences with Arbitrary Lengths", arXiv 2601.06463):
+ *
+ *   Sliding Chunk Attention (SCA)  - Gecko digest (paper.rainbus.top),
+ *     method step details, step 3; paperlayer.ai summary, section 3.2:
+ *       O_s = softmax(Q_s [K_{s-1}; K_s]^T) [V_{s-1}; V_s]
+ *     for chunk s of c tokens.  Scale 1 (no 1/sqrt(d)), causal inside the
+ *     current chunk, all c keys of the previous chunk visible, and chunk 1
+ *     attends only to itself.
+ *
+ *   Adaptive Working Memory (AWM)  - digest, core method (online-softmax
+ *     kernel) and step details, steps 4-5; paperlayer.ai summary, section
+ *     3.3 and Appendix A:
+ *       z^s   = sum_{t<=s} sum_{i<=c} exp(Km_{t,i})            (per feature)
+ *       phi^s(Km_s) = exp(Km_s) / z^s,   psi(x) = softmax over features
+ *       M'_1 = 0,
+ *       M'_s = (z^{s-2}/z^{s-1}) (.) M'_{s-1}
+ *              + phi^{s-1}(Km_{s-1})^T (V_{s-1} - psi(Km_{s-1}) M'_{s-1})
+ *       O_m,s = psi(Qm_s) M'_{s-1}        (M'_0 := 0: chunks 1, 2 read 0)
+ *     The z-ratio scales row f (key feature f) of M'.
+ *
+ *   The layer output is out_sca + out_mem (digest, step 5); the two parts
+ *   are returned separately and the caller adds them.
+ *
+ * Layout: every tensor is caller-owned, contiguous, row-major [B, H, T, d]
+ * (d innermost) in device memory, all of one dtype, each base address
+ * 16-byte aligned.  The value dimension equals d.
+ *
+ * Execution is asynchronous on `stream` (a cudaStream_t; NULL means the
+ * legacy default stream).  Argument errors are detected on the host before
+ * anything is launched or written.  Faults inside a kernel surface at the
+ * caller's next synchronisation.  Every device-side wait is bounded in time;
+ * a wait that runs out sets a device status word read by
+ * gecko_device_status().
+ */
+#ifndef GECKO_H
+#define GECKO_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* dtype codes */
+#define GECKO_F32  0   /* fp32 in, fp32 out, fp32 arithmetic (SIMT FMA) */
+#define GECKO_BF16 1   /* bf16 in, bf16 out, fp32 accumulation            */
+
+/* status codes */
+#define GECKO_OK            0
+#define GECKO_ERR_ARG       1  /* null pointer, bad dtype, size < 1, mismatched state query */
+#define GECKO_ERR_SHAPE     2  /* T % c != 0, c % 64 != 0, d not in {64, 128}, size overflow */
+#define GECKO_ERR_ALIGN     3  /* a tensor base address is not 16-byte aligned              */
+#define GECKO_ERR_ALLOC     4  /* the library workspace could not be allocated              */
+#define GECKO_ERR_CUDA      5  /* a CUDA runtime call or kernel launch failed               */
+#define GECKO_ERR_NO_STATE  6  /* gecko_awm_state before any forward on this device         */
+#define GECKO_ERR_TIMEOUT   7  /* a bounded device-side wait ran out                        */
+
+/*
+ * gecko_sca_awm_forward - fused SCA + AWM forward of one layer.
+ *
+ *   q, k, v, qm, km : [B, H, T, d] inputs (device), dtype `dtype`.
+ *                     q, k feed SCA; qm, km feed AWM; v feeds both.
+ *   out_sca, out_mem: [B, H, T, d] outputs (device), dtype `dtype`;
+ *                     fully overwritten.  They must not alias an input.
+ *   B, H, T, c, d   : batch, heads, tokens, chunk size, head dim.
+ *                     Requires B, H, T >= 1, c >= 64, c % 64 == 0,
+ *                     T % c == 0, d in {64, 128}.
+ *   dtype           : GECKO_F32 or GECKO_BF16.
+ *   stream          : cudaStream_t used for every launch and copy.
+ *
+ * Ownership: the library keeps one workspace per device (log z per chunk,
+ * per-chunk memory matrices, the carried state).  It grows on demand with
+ * stream-ordered allocation on `stream` and lives until gecko_release().
+ * Concurrent forwards on one device race on that workspace and are not
+ * supported.  Every call starts from M'_1 = 0 (no initial state).
+ *
+ * Returns GECKO_OK or an error code; the message is in gecko_last_error().
+ */
+int gecko_sca_awm_forward(const void* q, const void* k, const void* v,
+                          const void* qm, const void* km,
+                          void* out_sca, void* out_mem,
+                          int64_t B, int64_t H, int64_t T, int64_t c, int64_t d,
+                          int dtype, void* stream);
+
+/*
+ * gecko_awm_state - copy the AWM state carried out of the most recent
+ * forward on the current device: M_out [B, H, d, d] fp32 = M'_{S+1} (all S
+ * chunks folded in, normalised by z^S; row = key feature) and logz_out
+ * [B, H, d] fp32 = log z^S.  Pointers may be device or host memory
+ * (cudaMemcpyDefault).  The copy is ordered on `stream`; the call returns
+ * after the copy has completed.  Returns GECKO_ERR_NO_STATE if no forward
+ * ran on this device, GECKO_ERR_ARG if B, H, d differ from that forward,
+ * and GECKO_ERR_TIMEOUT if a kernel of that forward reported a timed-out
+ * wait.
+ */
+int gecko_awm_state(float* M_out, float* logz_out,
+                    int64_t B, int64_t H, int64_t d, void* stream);
+
+/*
+ * gecko_device_status - synchronise `stream`, then read and clear the
+ * library's device status word on the current device.  Returns GECKO_OK,
+ * GECKO_ERR_TIMEOUT if a kernel gave up on a bounded wait since the last
+ * check, or GECKO_ERR_CUDA if the synchronisation failed.
+ */
+int gecko_device_status(void* stream);
+
+/* Thread-local message describing the last non-zero status of this thread. */
+const char* gecko_last_error(void);
+
+/* Free the workspace of every device the library used.  Not thread-safe
+ * against a concurrent forward. */
+void gecko_release(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GECKO_H */

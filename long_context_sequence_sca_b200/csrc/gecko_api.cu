@@ -1,0 +1,250 @@
+// C-ABI host side of the Gecko forward: argument validation, the per-device
+// workspace, the launch sequence and the state export.  See include/gecko.h
+// for the contract of each entry point.
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+
+#include "../../include/gecko.h"
+#include "common.cuh"
+#include "gecko_internal.h"
+
+namespace gecko {
+
+// The device status word (bit kStatusTimeout: a bounded wait ran out).
+__device__ int g_status_word;
+
+size_t workspace_bytes(int64_t BH, int64_t S, int64_t d) {
+  auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const size_t vec = al(sizeof(float) * BH * S * d);
+  const size_t mat = al(sizeof(float) * BH * S * d * d);
+  const size_t mst = al(sizeof(float) * BH * (S + 1) * d * d);
+  return 3 * vec + 2 * mat + mst;
+}
+
+Workspace carve_workspace(void* base, int64_t BH, int64_t S, int64_t d) {
+  auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
+  char* p = static_cast<char*>(base);
+  Workspace w;
+  const size_t vec = al(sizeof(float) * BH * S * d);
+  const size_t mat = al(sizeof(float) * BH * S * d * d);
+  w.lse = reinterpret_cast<float*>(p);
+  p += vec;
+  w.logz = reinterpret_cast<float*>(p);
+  p += vec;
+  w.ratio = reinterpret_cast<float*>(p);
+  p += vec;
+  w.Bm = reinterpret_cast<float*>(p);
+  p += mat;
+  w.Cm = reinterpret_cast<float*>(p);
+  p += mat;
+  w.Mst = reinterpret_cast<float*>(p);
+  return w;
+}
+
+namespace {
+
+thread_local std::string t_err;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  t_err = buf;
+  return code;
+}
+
+struct DeviceState {
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  int* status = nullptr;  // device address of g_status_word
+  bool have_state = false;
+  int64_t B = 0, H = 0, d = 0, S = 0;
+};
+
+std::mutex g_mu;
+std::map<int, DeviceState> g_dev;
+
+bool env_is(const char* name, const char* val) {
+  const char* e = std::getenv(name);
+  return e && std::strcmp(e, val) == 0;
+}
+
+int check_cuda(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return GECKO_OK;
+  return fail(GECKO_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Per-device set-up: resolve the status word's device address.
+int device_state(int dev, DeviceState** out) {
+  DeviceState& ds = g_dev[dev];
+  if (!ds.status) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_status_word);
+    if (e != cudaSuccess) return check_cuda(e, "cudaGetSymbolAddress(status word)");
+    ds.status = static_cast<int*>(p);
+  }
+  *out = &ds;
+  return GECKO_OK;
+}
+
+int validate(const void* const* ptrs, int n, int64_t B, int64_t H, int64_t T, int64_t c, int64_t d, int dtype) {
+  for (int i = 0; i < n; ++i)
+    if (!ptrs[i]) return fail(GECKO_ERR_ARG, "tensor argument %d is NULL", i);
+  if (dtype != GECKO_F32 && dtype != GECKO_BF16) return fail(GECKO_ERR_ARG, "unknown dtype %d", dtype);
+  if (B < 1 || H < 1 || T < 1 || c < 1 || d < 1)
+    return fail(GECKO_ERR_ARG, "sizes must be >= 1 (B=%lld H=%lld T=%lld c=%lld d=%lld)", (long long)B,
+                (long long)H, (long long)T, (long long)c, (long long)d);
+  if (d != 64 && d != 128) return fail(GECKO_ERR_SHAPE, "d must be 64 or 128 (got %lld)", (long long)d);
+  if (c % 64 != 0) return fail(GECKO_ERR_SHAPE, "c must be a multiple of 64 (got %lld)", (long long)c);
+  if (T % c != 0) return fail(GECKO_ERR_SHAPE, "T %% c != 0 (T=%lld c=%lld)", (long long)T, (long long)c);
+  // element count and byte size must fit comfortably in int64; chunk and
+  // grid indices must fit the 32-bit ranges the kernels use
+  const long double elems = (long double)B * H * T * d;
+  if (elems * 4 > 4.0e18L) return fail(GECKO_ERR_SHAPE, "tensor size overflows");
+  if (T / c > (1 << 30) || B * H > (1 << 30) || T > (int64_t(1) << 31) - 256)
+    return fail(GECKO_ERR_SHAPE, "size exceeds kernel index range");
+  for (int i = 0; i < n; ++i)
+    if (reinterpret_cast<uintptr_t>(ptrs[i]) % 16 != 0)
+      return fail(GECKO_ERR_ALIGN, "tensor argument %d is not 16-byte aligned", i);
+  return GECKO_OK;
+}
+
+}  // namespace
+}  // namespace gecko
+
+using namespace gecko;
+
+extern "C" int gecko_sca_awm_forward(const void* q, const void* k, const void* v, const void* qm, const void* km,
+                                     void* out_sca, void* out_mem, int64_t B, int64_t H, int64_t T, int64_t c,
+                                     int64_t d, int dtype, void* stream) {
+  const void* ptrs[7] = {q, k, v, qm, km, out_sca, out_mem};
+  int rc = validate(ptrs, 7, B, H, T, c, d, dtype);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int dev = 0;
+  if ((rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice"))) return rc;
+
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState* ds = nullptr;
+  if ((rc = device_state(dev, &ds))) return rc;
+
+  const int64_t S = T / c;
+  const int64_t BH = B * H;
+  const size_t need = workspace_bytes(BH, S, d);
+  if (env_is("GECKO_FAIL_ALLOC", "1")) return fail(GECKO_ERR_ALLOC, "workspace allocation failed (injected)");
+  if (need > ds->ws_bytes) {
+    if (ds->ws) {
+      cudaFreeAsync(ds->ws, st);
+      ds->ws = nullptr;
+      ds->ws_bytes = 0;
+    }
+    void* p = nullptr;
+    cudaError_t e = cudaMallocAsync(&p, need, st);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return fail(GECKO_ERR_ALLOC, "workspace of %zu bytes: %s", need, cudaGetErrorString(e));
+    }
+    ds->ws = p;
+    ds->ws_bytes = need;
+  }
+  Workspace w = carve_workspace(ds->ws, BH, S, d);
+
+  Problem p{q, k, v, qm, km, out_sca, out_mem, B, H, T, c, d, (int)S, dtype, true, ds->status};
+  // GECKO_KERNELS=simt selects the CUDA-core kernels for every dtype (a
+  // second, independent GPU implementation used to cross-check the
+  // tensor-core path).
+  const bool force_simt = env_is("GECKO_KERNELS", "simt");
+  const bool use_tc = !force_simt && tc_supported(p);
+  p.readout_simt = true;
+
+  cudaGetLastError();  // clear stale errors from the caller
+  if ((rc = check_cuda(launch_awm_simt(p, w, /*chunk_gemms=*/true, st), "awm (simt)"))) return rc;
+  if (use_tc) {
+    if ((rc = check_cuda(launch_sca_tc(p, st), "sca (tensor core)"))) return rc;
+  } else {
+    if ((rc = check_cuda(launch_sca_simt(p, st), "sca (simt)"))) return rc;
+  }
+  ds->have_state = true;
+  ds->B = B;
+  ds->H = H;
+  ds->d = d;
+  ds->S = S;
+  return GECKO_OK;
+}
+
+extern "C" int gecko_awm_state(float* M_out, float* logz_out, int64_t B, int64_t H, int64_t d, void* stream) {
+  if (!M_out || !logz_out) return fail(GECKO_ERR_ARG, "NULL output pointer");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int dev = 0, rc;
+  if ((rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice"))) return rc;
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto it = g_dev.find(dev);
+  if (it == g_dev.end() || !it->second.have_state)
+    return fail(GECKO_ERR_NO_STATE, "no forward has run on device %d", dev);
+  DeviceState& ds = it->second;
+  if (B != ds.B || H != ds.H || d != ds.d)
+    return fail(GECKO_ERR_ARG, "state is B=%lld H=%lld d=%lld, asked for B=%lld H=%lld d=%lld", (long long)ds.B,
+                (long long)ds.H, (long long)ds.d, (long long)B, (long long)H, (long long)d);
+  const int64_t BH = B * H, S = ds.S;
+  Workspace w = carve_workspace(ds.ws, BH, S, d);
+  const size_t mat = sizeof(float) * d * d;
+  // M'_{S+1} of each (b, h) sits at Mst[bh, S]; log z^S at logz[bh, S-1]
+  if ((rc = check_cuda(cudaMemcpy2DAsync(M_out, mat, w.Mst + S * d * d, mat * (S + 1), mat, BH,
+                                         cudaMemcpyDefault, st),
+                       "copy M")))
+    return rc;
+  if ((rc = check_cuda(cudaMemcpy2DAsync(logz_out, sizeof(float) * d, w.logz + (S - 1) * d,
+                                         sizeof(float) * d * S, sizeof(float) * d, BH, cudaMemcpyDefault, st),
+                       "copy log z")))
+    return rc;
+  if ((rc = check_cuda(cudaStreamSynchronize(st), "synchronize"))) return rc;
+  int word = 0;
+  if ((rc = check_cuda(cudaMemcpy(&word, ds.status, sizeof(int), cudaMemcpyDeviceToHost), "read status")))
+    return rc;
+  if (word & kStatusTimeout) return fail(GECKO_ERR_TIMEOUT, "a kernel of the last forward timed out on a wait");
+  return GECKO_OK;
+}
+
+extern "C" int gecko_device_status(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int dev = 0, rc;
+  if ((rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice"))) return rc;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState* ds = nullptr;
+  if ((rc = device_state(dev, &ds))) return rc;
+  if ((rc = check_cuda(cudaStreamSynchronize(st), "synchronize"))) return rc;
+  int word = 0;
+  if ((rc = check_cuda(cudaMemcpy(&word, ds->status, sizeof(int), cudaMemcpyDeviceToHost), "read status")))
+    return rc;
+  const int zero = 0;
+  if ((rc = check_cuda(cudaMemcpy(ds->status, &zero, sizeof(int), cudaMemcpyHostToDevice), "clear status")))
+    return rc;
+  if (word & kStatusTimeout) return fail(GECKO_ERR_TIMEOUT, "a kernel gave up on a bounded wait");
+  return GECKO_OK;
+}
+
+extern "C" const char* gecko_last_error(void) { return t_err.c_str(); }
+
+extern "C" void gecko_release(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int cur = 0;
+  cudaGetDevice(&cur);
+  for (auto& kv : g_dev) {
+    if (kv.second.ws) {
+      cudaSetDevice(kv.first);
+      cudaDeviceSynchronize();
+      cudaFree(kv.second.ws);
+    }
+    kv.second.ws = nullptr;
+    kv.second.ws_bytes = 0;
+    kv.second.have_state = false;
+  }
+  cudaSetDevice(cur);
+}

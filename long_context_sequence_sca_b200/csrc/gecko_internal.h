@@ -1,0 +1,47 @@
+// Internal interface between the C-ABI host code and the kernel launchers.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace gecko {
+
+constexpr int kF32 = 0;
+constexpr int kBF16 = 1;
+
+// One validated forward call.
+struct Problem {
+  const void *q, *k, *v, *qm, *km;
+  void *out_sca, *out_mem;
+  int64_t B, H, T, c, d;
+  int S;
+  int dtype;
+  bool readout_simt;  // readout by the SIMT kernel (else by the tensor-core one)
+  int* status;        // device status word
+};
+
+// Device workspace carved out of one allocation (all fp32).
+struct Workspace {
+  float* lse;    // [BH, S, d]  log of per-chunk exp-sums of K_m
+  float* logz;   // [BH, S, d]  log z^s
+  float* ratio;  // [BH, S, d]  z^{s-1} / z^s  (0 for s = 1)
+  float* Bm;     // [BH, S, d, d]  Phi_s^T V_s
+  float* Cm;     // [BH, S, d, d]  Phi_s^T Psi_s
+  float* Mst;    // [BH, S+1, d, d]  M'_1 .. M'_{S+1}
+};
+
+// Bytes needed by a Workspace for (BH, S, d), each region 256-byte aligned.
+size_t workspace_bytes(int64_t BH, int64_t S, int64_t d);
+Workspace carve_workspace(void* base, int64_t BH, int64_t S, int64_t d);
+
+cudaError_t launch_awm_simt(const Problem& p, const Workspace& w, bool chunk_gemms, cudaStream_t st);
+cudaError_t launch_sca_simt(const Problem& p, cudaStream_t st);
+
+// Tensor-core (tcgen05 + TMEM + TMA) kernels, bf16 with c % 128 == 0.
+bool tc_supported(const Problem& p);
+cudaError_t launch_sca_tc(const Problem& p, cudaStream_t st);
+cudaError_t launch_awm_chunk_tc(const Problem& p, const Workspace& w, cudaStream_t st);
+cudaError_t launch_awm_readout_tc(const Problem& p, const Workspace& w, cudaStream_t st);
+
+}  // namespace gecko

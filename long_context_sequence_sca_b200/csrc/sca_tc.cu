@@ -1,0 +1,465 @@
+// Sliding Chunk Attention forward on 5th-generation tensor cores (sm_100a).
+//
+// Computes, per (b, h) and chunk s of c tokens (Gecko digest,
+// paper.rainbus.top, method step details, step 3; paperlayer.ai summary,
+// section 3.2):
+//     O_s = softmax(Q_s [K_{s-1}; K_s]^T) [V_{s-1}; V_s]
+// with scale 1, a causal mask inside the current chunk, and no previous chunk
+// for chunk 1.  Requires bf16, d in {64, 128}, c % 128 == 0.
+//
+// Design (one persistent CTA per SM, 384 threads):
+//   warp 0      TMA producer: Q tiles once per work unit; K and V tiles of
+//               128 keys through a ring of shared-memory stages.
+//   warp 1      MMA issuer (one thread): S_i = Q_i K_j^T (SS form) into TMEM,
+//               O_i += P_i V_j with P_i read from TMEM (TS form).
+//   warp 2      TMEM allocator.
+//   warps 4-7   softmax for query tile 0, warps 8-11 for query tile 1; one
+//               thread per query row; online max/sum in registers; P written
+//               back to TMEM as bf16 over the S columns; epilogue O / l.
+// A work unit is two adjacent 128-row query tiles of one (b, h).  The MMA
+// warp interleaves the two tiles (PV(0), QK(0), PV(1), QK(1)) so each
+// softmax warpgroup's exp work overlaps the other tile's MMAs.  Only the
+// diagonal key tile of each query tile is masked; key tiles entirely above
+// the diagonal or before the previous chunk are never loaded.
+//
+// The running max is updated lazily: O and l are rescaled only when a new
+// tile's row max exceeds the reference by more than 8 (log2 units), which
+// keeps every exponent <= 2^8 and leaves the final O / l unchanged.
+//
+// Every wait is bounded (see mbar_wait); on a timeout the CTA drains its
+// in-flight copies and MMAs, frees TMEM and returns with the status word set.
+#include <cstdio>
+
+#include "common.cuh"
+#include "gecko_internal.h"
+
+namespace gecko {
+namespace {
+
+constexpr int kBM = 128;   // query rows per tile
+constexpr int kBN = 128;   // keys per tile
+constexpr int kThreads = 384;
+
+template <int D>
+struct ScaCfg {
+  static constexpr int kTileBytes = 128 * D * 2;       // 128 rows x D bf16, D/64 swizzled boxes
+  static constexpr int kBoxBytes = 128 * 64 * 2;       // one [128 x 64] box
+  static constexpr int kStages = D == 64 ? 4 : 2;      // K and V stages each
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = kQOff + 2 * kTileBytes;
+  static constexpr int kVOff = kKOff + kStages * kTileBytes;
+  static constexpr int kBarOff = kVOff + kStages * kTileBytes;
+  // q_full, q_empty, k_full[S], k_empty[S], v_full[S], v_empty[S],
+  // s_full[2], p_full[2], o_full[2], o_empty[2], drain
+  static constexpr int kNumBars = 2 + 4 * kStages + 8 + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kAlloc = kBytes + 1024;         // slack for 1024-byte alignment
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
+};
+
+struct Unit {
+  int64_t bh;
+  int q0;        // first query row of tile 0
+  int nt;        // tiles in the unit (1 or 2)
+  int beg[2];    // first key tile (128-key units) of each query tile
+  int end[2];    // one past the last (= diagonal tile + 1)
+};
+
+// Map a linear unit index to (bh, pair).  When c % 256 == 0 the order puts
+// the most expensive pairs first (later chunks, larger in-chunk offsets) so
+// the static round-robin over CTAs approximates longest-first scheduling.
+__device__ __forceinline__ Unit decode_unit(int u, int BH, int T, int c) {
+  const int pairs = (T + 255) / 256;
+  const int w = u / BH;
+  Unit U;
+  U.bh = u % BH;
+  int pair = w;
+  if (c % 256 == 0) {
+    const int npc = c / 256;
+    const int S = T / c;
+    const int nA = (S - 1) * npc;
+    if (w < nA) {
+      const int o = npc - 1 - w / (S - 1);
+      const int ch = 1 + w % (S - 1);
+      pair = ch * npc + o;
+    } else {
+      pair = npc - 1 - (w - nA);
+    }
+  }
+  (void)pairs;
+  U.q0 = pair * 256;
+  U.nt = (U.q0 + 128 < T) ? 2 : 1;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int r0 = U.q0 + 128 * i;
+    const int ch = r0 / c;
+    const int lo = ch >= 1 ? (ch - 1) * c : 0;
+    U.beg[i] = lo / kBN;
+    U.end[i] = r0 / kBN + 1;
+    if (i >= U.nt) { U.beg[i] = 0; U.end[i] = 0; }
+  }
+  return U;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+              const __grid_constant__ CUtensorMap map_v, __nv_bfloat16* __restrict__ out, int T, int c, int BH,
+              int n_units, int* status) {
+  using Cfg = ScaCfg<D>;
+  constexpr int KST = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + Cfg::kQOff;
+  uint8_t* sK = smem + Cfg::kKOff;
+  uint8_t* sV = smem + Cfg::kVOff;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* k_full = bars + 2;
+  uint64_t* k_empty = k_full + KST;
+  uint64_t* v_full = k_empty + KST;
+  uint64_t* v_empty = v_full + KST;
+  uint64_t* s_full = v_empty + KST;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_full = p_full + 2;
+  uint64_t* o_empty = o_full + 2;
+  uint64_t* drain = o_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
+
+  const int warp = warp_id_uniform();
+  const int lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < KST; ++s) {
+      mbar_init(k_full + s, 1);
+      mbar_init(k_empty + s, 1);
+      mbar_init(v_full + s, 1);
+      mbar_init(v_empty + s, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(s_full + i, 1);
+      mbar_init(p_full + i, 128);
+      mbar_init(o_full + i, 1);
+      mbar_init(o_empty + i, 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&map_q);
+    tma_prefetch_desc(&map_k);
+    tma_prefetch_desc(&map_v);
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer --
+    if (lane == 0) {
+      uint32_t kv_it = 0;
+      int n = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++n) {
+        const Unit U = decode_unit(u, BH, T, c);
+        const int64_t rowbase = U.bh * (int64_t)T;
+        if (n > 0 && !(ok = mbar_wait(q_empty, (n - 1) & 1, abort_flag, status))) break;
+        mbar_arrive_expect_tx(q_full, U.nt * Cfg::kTileBytes);
+        for (int i = 0; i < U.nt; ++i)
+          for (int b = 0; b < D / 64; ++b)
+            tma_load_2d(sQ + i * Cfg::kTileBytes + b * Cfg::kBoxBytes, &map_q, q_full, b * 64,
+                        (int)(rowbase + U.q0 + 128 * i));
+        const int jb = U.beg[0], je = U.nt == 2 ? U.end[1] : U.end[0];
+        for (int j = jb; j < je; ++j, ++kv_it) {
+          const int st = kv_it % KST;
+          const uint32_t ph = (kv_it / KST) & 1;
+          const int row = (int)(rowbase + (int64_t)j * kBN);
+          if (!(ok = mbar_wait(k_empty + st, ph ^ 1, abort_flag, status))) break;
+          mbar_arrive_expect_tx(k_full + st, Cfg::kTileBytes);
+          for (int b = 0; b < D / 64; ++b)
+            tma_load_2d(sK + st * Cfg::kTileBytes + b * Cfg::kBoxBytes, &map_k, k_full + st, b * 64, row);
+          if (!(ok = mbar_wait(v_empty + st, ph ^ 1, abort_flag, status))) { ++kv_it; break; }
+          mbar_arrive_expect_tx(v_full + st, Cfg::kTileBytes);
+          for (int b = 0; b < D / 64; ++b)
+            tma_load_2d(sV + st * Cfg::kTileBytes + b * Cfg::kBoxBytes, &map_v, v_full + st, b * 64, row);
+        }
+      }
+      if (!ok) {
+        // let every copy already issued land before the CTA exits
+        for (uint32_t idx = kv_it >= (uint32_t)KST ? kv_it - KST : 0; idx < kv_it; ++idx) {
+          mbar_wait_drain(k_full + idx % KST, (idx / KST) & 1);
+          mbar_wait_drain(v_full + idx % KST, (idx / KST) & 1);
+        }
+        if (n > 0) mbar_wait_drain(q_full, (n - 1) & 1);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, false, true);
+      const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK), va = smem_u32(sV);
+      uint32_t kv_it = 0, p_cnt[2] = {0, 0}, o_cnt[2] = {0, 0};
+      int n = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++n) {
+        const Unit U = decode_unit(u, BH, T, c);
+        if (!(ok = mbar_wait(q_full, n & 1, abort_flag, status))) break;
+        tc_fence_after();
+        const int jb = U.beg[0], je = U.nt == 2 ? U.end[1] : U.end[0];
+        for (int j = jb; j <= je && ok; ++j) {
+          const uint32_t stK = kv_it % KST;
+          if (j < je) {
+            if (!(ok = mbar_wait(k_full + stK, (kv_it / KST) & 1, abort_flag, status))) break;
+            tc_fence_after();
+          }
+          const uint32_t itV = kv_it - 1;  // V_{j-1}
+          const uint32_t stV = itV % KST;
+          if (j > jb) {
+            if (!(ok = mbar_wait(v_full + stV, (itV / KST) & 1, abort_flag, status))) break;
+            tc_fence_after();
+          }
+          for (int i = 0; i < U.nt && ok; ++i) {
+            const uint32_t colS = i == 0 ? Cfg::kColS0 : Cfg::kColS1;
+            const uint32_t colO = i == 0 ? Cfg::kColO0 : Cfg::kColO1;
+            if (j - 1 >= U.beg[i] && j - 1 < U.end[i]) {
+              // O_i += P_i V_{j-1}
+              if (j - 1 == U.beg[i]) {
+                if (!(ok = mbar_wait(o_empty + i, (o_cnt[i] & 1) ^ 1, abort_flag, status))) break;
+              }
+              if (!(ok = mbar_wait(p_full + i, p_cnt[i] & 1, abort_flag, status))) break;
+              ++p_cnt[i];
+              tc_fence_after();
+#pragma unroll
+              for (int kk = 0; kk < kBN / 16; ++kk) {
+                const uint64_t bdesc = sdesc_sw128(va + stV * Cfg::kTileBytes + kk * 2048, Cfg::kBoxBytes, 1024);
+                umma_ts(tmem + colO, tmem + colS + kk * 8, bdesc, idesc_pv, (j - 1 > U.beg[i] || kk > 0) ? 1u : 0u);
+              }
+              if (j - 1 == U.end[i] - 1) {
+                umma_commit(o_full + i);
+                ++o_cnt[i];
+              }
+            }
+            if (j >= U.beg[i] && j < U.end[i]) {
+              // S_i = Q_i K_j^T
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t koff = (kk / 4) * Cfg::kBoxBytes + (kk % 4) * 32;
+                const uint64_t adesc = sdesc_sw128(qa + i * Cfg::kTileBytes + koff, 16, 1024);
+                const uint64_t bdesc = sdesc_sw128(ka + stK * Cfg::kTileBytes + koff, 16, 1024);
+                umma_ss(tmem + colS, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+              }
+              umma_commit(s_full + i);
+            }
+          }
+          if (!ok) break;
+          if (j > jb) umma_commit(v_empty + stV);
+          if (j < je) {
+            umma_commit(k_empty + stK);
+            if (j == je - 1) umma_commit(q_empty);
+            ++kv_it;
+          }
+        }
+      }
+      // all issued MMAs complete before TMEM is released
+      umma_commit(drain);
+      mbar_wait_drain(drain, 0);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------ softmax warpgroups --
+    const int i = (warp - 4) / 4;           // query tile handled by this warpgroup
+    const int r = (warp % 4) * 32 + lane;   // row within the tile = TMEM lane
+    const uint32_t lane_addr = tmem + ((uint32_t)((warp % 4) * 32) << 16);
+    const uint32_t colS = i == 0 ? Cfg::kColS0 : Cfg::kColS1;
+    const uint32_t colO = i == 0 ? Cfg::kColO0 : Cfg::kColO1;
+    uint32_t s_cnt = 0, o_cnt = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const Unit U = decode_unit(u, BH, T, c);
+      if (i >= U.nt) continue;
+      float m_ref = 0.f, l = 0.f;
+      for (int j = U.beg[i]; j < U.end[i]; ++j) {
+        ok = __all_sync(0xffffffffu, mbar_wait(s_full + i, s_cnt & 1, abort_flag, status));
+        if (!ok) break;
+        ++s_cnt;
+        tc_fence_after();
+        uint32_t sr[kBN];
+#pragma unroll
+        for (int cb = 0; cb < kBN / 32; ++cb) tmem_ld32p(lane_addr + colS + cb * 32, sr + cb * 32);
+        tmem_wait_ld();
+        float s[kBN];
+#pragma unroll
+        for (int x = 0; x < kBN; ++x) s[x] = __uint_as_float(sr[x]);
+        if (j == U.end[i] - 1) {
+#pragma unroll
+          for (int x = 0; x < kBN; ++x)
+            if (x > r) s[x] = -INFINITY;
+        }
+        float mt = s[0];
+#pragma unroll
+        for (int x = 1; x < kBN; ++x) mt = fmaxf(mt, s[x]);
+        const float m2 = mt * kLog2e;
+        if (j == U.beg[i]) {
+          m_ref = m2;
+        } else if (m2 > m_ref + 8.f) {
+          const float scale = ex2(m_ref - m2);
+          l *= scale;
+          m_ref = m2;
+#pragma unroll 1
+          for (int cb = 0; cb < D / 32; ++cb) {
+            uint32_t o[32];
+            tmem_ld32(lane_addr + colO + cb * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * scale);
+            tmem_st32(lane_addr + colO + cb * 32, o);
+          }
+        }
+        float sum = 0.f;
+#pragma unroll
+        for (int cb = 0; cb < kBN / 32; ++cb) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int x = 0; x < 16; ++x) {
+            const float p0 = ex2(fmaf(s[cb * 32 + 2 * x], kLog2e, -m_ref));
+            const float p1 = ex2(fmaf(s[cb * 32 + 2 * x + 1], kLog2e, -m_ref));
+            sum += p0 + p1;
+            pk[x] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(lane_addr + colS + cb * 16, pk);
+        }
+        tmem_wait_st();
+        l += sum;
+        tc_fence_before();
+        mbar_arrive(p_full + i);
+      }
+      if (!ok) break;
+      // epilogue: O / l -> bf16 rows
+      ok = __all_sync(0xffffffffu, mbar_wait(o_full + i, o_cnt & 1, abort_flag, status));
+      if (!ok) break;
+      ++o_cnt;
+      tc_fence_after();
+      const float inv = 1.f / l;
+      __nv_bfloat16* orow = out + (U.bh * (int64_t)T + U.q0 + 128 * i + r) * D;
+#pragma unroll 1
+      for (int cb = 0; cb < D / 32; ++cb) {
+        uint32_t o[32];
+        tmem_ld32(lane_addr + colO + cb * 32, o);
+        tmem_wait_ld();
+        uint4 w[4];
+        uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
+        for (int x = 0; x < 16; ++x)
+          wp[x] = pack_bf16x2(__uint_as_float(o[2 * x]) * inv, __uint_as_float(o[2 * x + 1]) * inv);
+        uint4* dst = reinterpret_cast<uint4*>(orow + cb * 32);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) dst[x] = w[x];
+      }
+      tc_fence_before();
+      mbar_arrive(o_empty + i);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem, Cfg::kTmemCols);
+}
+
+// --------------------------------------------------------------- host --
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [rows, d] bf16 row-major viewed as a 2D tensor; box = 128 rows x 64 columns,
+// 128-byte swizzle (the canonical K-major / MN-major UMMA operand layout).
+cudaError_t make_map(CUtensorMap* m, const void* base, int64_t rows, int d) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int D>
+cudaError_t launch_sca_tc_impl(const Problem& p, cudaStream_t st) {
+  using Cfg = ScaCfg<D>;
+  const int64_t rows = p.B * p.H * p.T;
+  CUtensorMap mq, mk, mv;
+  cudaError_t e;
+  if ((e = make_map(&mq, p.q, rows, D)) != cudaSuccess) return e;
+  if ((e = make_map(&mk, p.k, rows, D)) != cudaSuccess) return e;
+  if ((e = make_map(&mv, p.v, rows, D)) != cudaSuccess) return e;
+  const int BH = (int)(p.B * p.H);
+  const int T = (int)p.T;
+  const int n_units = BH * ((T + 255) / 256);
+  const int grid = n_units < sm_count() ? n_units : sm_count();
+  if ((e = cudaFuncSetAttribute(sca_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kAlloc)) !=
+      cudaSuccess)
+    return e;
+  sca_tc_kernel<D><<<grid, kThreads, Cfg::kAlloc, st>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(p.out_sca), T,
+                                                        (int)p.c, BH, n_units, p.status);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_supported(const Problem& p) {
+  if (p.dtype != kBF16 || p.c % 128 != 0) return false;
+  // rows addressed through 32-bit TMA coordinates
+  if (p.B * p.H * p.T > (int64_t(1) << 31) - 1) return false;
+  int dev = 0, major = 0, minor = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  return major == 10 && minor == 0;
+}
+
+cudaError_t launch_sca_tc(const Problem& p, cudaStream_t st) {
+  return p.d == 64 ? launch_sca_tc_impl<64>(p, st) : launch_sca_tc_impl<128>(p, st);
+}
+
+}  // namespace gecko

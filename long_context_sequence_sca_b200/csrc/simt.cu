@@ -1,0 +1,420 @@
+// SIMT (CUDA-core, fp32 FMA) kernels of the Gecko forward.  They serve the
+// fp32 dtype (where tensor-core tf32 would miss a 1e-4 error bound) and any
+// shape the tensor-core kernels do not cover.  Inputs are float or bf16;
+// arithmetic is fp32 throughout.
+//
+// Definitions follow the Gecko digest (paper.rainbus.top): core method
+// (phi^s, z^s, psi) and method step details, steps 3-5 (SCA, the M'_s
+// update, the readout); and the paperlayer.ai summary, sections 3.2-3.3 and
+// Appendix A (M'_1 = 0).
+#include "common.cuh"
+#include "gecko_internal.h"
+
+namespace gecko {
+namespace {
+
+template <typename T> struct Vec8;  // 8 elements in one or two 16-byte words
+template <> struct Vec8<__nv_bfloat16> {
+  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&x)[8]) {
+    uint4 u = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 f = __bfloat1622float2(h[i]);
+      x[2 * i] = f.x;
+      x[2 * i + 1] = f.y;
+    }
+  }
+};
+template <> struct Vec8<float> {
+  static __device__ __forceinline__ void load(const float* p, float (&x)[8]) {
+    float4 a = reinterpret_cast<const float4*>(p)[0];
+    float4 b = reinterpret_cast<const float4*>(p)[1];
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  }
+};
+
+// ------------------------------------------------------------------------
+// Per-chunk, per-feature log of the exp-sum: lse[bh, s, f] =
+// log sum_{i in chunk s} exp(km[i, f]).  grid (S, BH), 256 threads; each
+// thread keeps a running (max, sum) for 8 features over a strided row set.
+template <typename TIn, int D>
+__global__ void __launch_bounds__(256) awm_lse_kernel(const TIn* __restrict__ km, float* __restrict__ lse,
+                                                      int64_t T, int c) {
+  constexpr int TPR = D / 8;          // threads per row
+  constexpr int RG = 256 / TPR;       // rows processed in parallel
+  const int s = blockIdx.x;
+  const int64_t bh = blockIdx.y;
+  const int lane8 = threadIdx.x % TPR;
+  const int rg = threadIdx.x / TPR;
+  const TIn* base = km + (bh * T + (int64_t)s * c) * D + lane8 * 8;
+  float m[8], acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) { m[i] = -INFINITY; acc[i] = 0.f; }
+  for (int r = rg; r < c; r += RG) {
+    float x[8];
+    Vec8<TIn>::load(base + (int64_t)r * D, x);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (x[i] > m[i]) {
+        acc[i] = acc[i] * expf(m[i] - x[i]) + 1.f;
+        m[i] = x[i];
+      } else {
+        acc[i] += expf(x[i] - m[i]);
+      }
+    }
+  }
+  __shared__ float sm[RG][D + 1];
+  __shared__ float ss[RG][D + 1];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    sm[rg][lane8 * 8 + i] = m[i];
+    ss[rg][lane8 * 8 + i] = acc[i];
+  }
+  __syncthreads();
+  for (int f = threadIdx.x; f < D; f += 256) {
+    float M = -INFINITY;
+    for (int g = 0; g < RG; ++g) M = fmaxf(M, sm[g][f]);
+    float tot = 0.f;
+    for (int g = 0; g < RG; ++g)
+      if (sm[g][f] > -INFINITY) tot += ss[g][f] * expf(sm[g][f] - M);
+    lse[(bh * gridDim.x + s) * D + f] = M + logf(tot);
+  }
+}
+
+// ------------------------------------------------------------------------
+// Prefix over chunks in fp64: log z^s = logaddexp(log z^{s-1}, lse_s), and
+// the row ratio z^{s-1}/z^s (0 for s = 1).  grid BH, D threads.
+template <int D>
+__global__ void __launch_bounds__(D) awm_prefix_kernel(const float* __restrict__ lse, float* __restrict__ logz,
+                                                       float* __restrict__ ratio, int S) {
+  const int64_t bh = blockIdx.x;
+  const int f = threadIdx.x;
+  double L = 0.0;
+  for (int s = 0; s < S; ++s) {
+    const int64_t o = (bh * S + s) * D + f;
+    const double e = lse[o];
+    double Ln;
+    if (s == 0) {
+      Ln = e;
+    } else {
+      const double hi = fmax(L, e), lo = fmin(L, e);
+      Ln = hi + log1p(exp(lo - hi));
+    }
+    logz[o] = (float)Ln;
+    ratio[o] = s == 0 ? 0.f : (float)exp(L - Ln);
+    L = Ln;
+  }
+}
+
+// ------------------------------------------------------------------------
+// Per-chunk GEMMs of the AWM update, in fp32:
+//   Bm_s = Phi_s^T V_s,   Cm_s = Phi_s^T Psi_s         (D x D each)
+// with Phi_s = exp(Km_s - log z^s) and Psi_s = rowsoftmax(Km_s).
+// grid (S, BH), 256 threads as a 16 x 16 grid of (D/16) x (D/16) tiles.
+template <typename TIn, int D>
+__global__ void __launch_bounds__(256) awm_chunk_simt_kernel(const TIn* __restrict__ km,
+                                                             const TIn* __restrict__ v,
+                                                             const float* __restrict__ logz,
+                                                             float* __restrict__ Bm, float* __restrict__ Cm,
+                                                             int64_t T, int c) {
+  constexpr int RT = 16;       // token rows per step
+  constexpr int TM = D / 16;   // outputs per thread per dim
+  const int s = blockIdx.x;
+  const int S = gridDim.x;
+  const int64_t bh = blockIdx.y;
+  __shared__ float phi_s[RT][D];
+  __shared__ float psi_s[RT][D];
+  __shared__ float v_s[RT][D];
+  __shared__ float lz[D];
+  const int tid = threadIdx.x;
+  for (int f = tid; f < D; f += 256) lz[f] = logz[(bh * S + s) * D + f];
+  const int ty = tid / 16, tx = tid % 16;
+  float accB[TM][TM], accC[TM][TM];
+#pragma unroll
+  for (int i = 0; i < TM; ++i)
+#pragma unroll
+    for (int j = 0; j < TM; ++j) { accB[i][j] = 0.f; accC[i][j] = 0.f; }
+  const int64_t row0 = bh * T + (int64_t)s * c;
+  const int warp = tid / 32, lane = tid % 32;
+  __syncthreads();
+  for (int r0 = 0; r0 < c; r0 += RT) {
+    // each warp prepares 4 rows: phi, psi (warp-wide softmax over D), v
+    for (int rr = warp; rr < RT; rr += 8) {
+      const int64_t g = (row0 + r0 + rr) * D;
+      float x[D / 32];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < D / 32; ++i) {
+        x[i] = to_f32(km[g + lane + 32 * i]);
+        mx = fmaxf(mx, x[i]);
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffff, mx, o));
+      float sum = 0.f, e[D / 32];
+#pragma unroll
+      for (int i = 0; i < D / 32; ++i) { e[i] = expf(x[i] - mx); sum += e[i]; }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffff, sum, o);
+      const float inv = 1.f / sum;
+#pragma unroll
+      for (int i = 0; i < D / 32; ++i) {
+        const int f = lane + 32 * i;
+        psi_s[rr][f] = e[i] * inv;
+        phi_s[rr][f] = expf(x[i] - lz[f]);
+        v_s[rr][f] = to_f32(v[g + f]);
+      }
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int t = 0; t < RT; ++t) {
+      float a[TM], b[TM], p[TM];
+#pragma unroll
+      for (int i = 0; i < TM; ++i) {
+        a[i] = phi_s[t][ty * TM + i];
+        b[i] = v_s[t][tx * TM + i];
+        p[i] = psi_s[t][tx * TM + i];
+      }
+#pragma unroll
+      for (int i = 0; i < TM; ++i)
+#pragma unroll
+        for (int j = 0; j < TM; ++j) {
+          accB[i][j] = fmaf(a[i], b[j], accB[i][j]);
+          accC[i][j] = fmaf(a[i], p[j], accC[i][j]);
+        }
+    }
+    __syncthreads();
+  }
+  const int64_t o = (bh * S + s) * (int64_t)D * D;
+#pragma unroll
+  for (int i = 0; i < TM; ++i)
+#pragma unroll
+    for (int j = 0; j < TM; ++j) {
+      Bm[o + (ty * TM + i) * D + tx * TM + j] = accB[i][j];
+      Cm[o + (ty * TM + i) * D + tx * TM + j] = accC[i][j];
+    }
+}
+
+// ------------------------------------------------------------------------
+// The sequential carry, one slice of JC value columns per CTA (columns of M'
+// evolve independently):
+//   M'_{s+1}[:, J] = r_s (.) M'_s[:, J] - Cm_s M'_s[:, J] + Bm_s[:, J]
+// Writes Mst[bh, s] = M'_{s+1} for s = 0..S (M'_1 = 0 first).
+// grid (D / JC, BH), 256 threads.
+template <int D, int JC>
+__global__ void __launch_bounds__(256) awm_carry_kernel(const float* __restrict__ Bm,
+                                                        const float* __restrict__ Cm,
+                                                        const float* __restrict__ ratio,
+                                                        float* __restrict__ Mst, int S) {
+  constexpr int PER = D * JC / 256;  // outputs per thread (one row f, PER columns)
+  static_assert(256 / (JC / PER) == D, "thread layout");
+  extern __shared__ float smem_carry[];
+  float* Cs = smem_carry;               // [D][D + 1]
+  float* Ms = Cs + D * (D + 1);         // [D][JC]
+  const int64_t bh = blockIdx.y;
+  const int j0 = blockIdx.x * JC;
+  const int tid = threadIdx.x;
+  const int f = tid / (JC / PER);
+  const int jj = (tid % (JC / PER)) * PER;
+  for (int i = tid; i < D * JC; i += 256) Ms[i] = 0.f;
+  const int64_t mst_stride = (int64_t)D * D;
+  float* mout = Mst + bh * (int64_t)(S + 1) * mst_stride;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) mout[f * D + j0 + jj + j] = 0.f;   // M'_1 = 0
+  for (int s = 0; s < S; ++s) {
+    const float* C = Cm + (bh * S + s) * mst_stride;
+    __syncthreads();
+    for (int i = tid; i < D * D; i += 256) Cs[(i / D) * (D + 1) + (i % D)] = C[i];
+    __syncthreads();
+    const float rf = ratio[(bh * S + s) * D + f];
+    const float* Bp = Bm + (bh * S + s) * mst_stride + f * D + j0 + jj;
+    float acc[PER];
+#pragma unroll
+    for (int j = 0; j < PER; ++j) acc[j] = rf * Ms[f * JC + jj + j] + Bp[j];
+    for (int g = 0; g < D; ++g) {
+      const float cfg = Cs[f * (D + 1) + g];
+#pragma unroll
+      for (int j = 0; j < PER; ++j) acc[j] = fmaf(-cfg, Ms[g * JC + jj + j], acc[j]);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      Ms[f * JC + jj + j] = acc[j];
+      mout[(int64_t)(s + 1) * mst_stride + f * D + j0 + jj + j] = acc[j];
+    }
+  }
+}
+
+// ------------------------------------------------------------------------
+// Readout O_m,s = psi(Qm_s) M'_{s-1} (zero for chunks 1 and 2).
+// grid (c / 64, S, BH), 256 threads; 64 rows per CTA.
+template <typename TIn, int D>
+__global__ void __launch_bounds__(256) awm_readout_simt_kernel(const TIn* __restrict__ qm,
+                                                               const float* __restrict__ Mst,
+                                                               TIn* __restrict__ out, int64_t T, int c) {
+  constexpr int R = 64;
+  constexpr int CT = D / 16;  // columns per thread
+  extern __shared__ float smem_ro[];
+  float* Ms = smem_ro;          // [D][D]
+  float* ps = Ms + D * D;       // [R][D + 1]
+  const int s = blockIdx.y;     // 0-based chunk
+  const int S = gridDim.y;
+  const int64_t bh = blockIdx.z;
+  const int64_t row0 = bh * T + (int64_t)s * c + (int64_t)blockIdx.x * R;
+  const int tid = threadIdx.x;
+  if (s < 2) {
+    for (int i = tid; i < R * D; i += 256) out[row0 * D + i] = from_f32<TIn>(0.f);
+    return;
+  }
+  // 0-based chunk s is chunk s+1; it reads M'_s = Mst[s - 1]
+  const float* M = Mst + (bh * (S + 1) + (s - 1)) * (int64_t)D * D;
+  for (int i = tid; i < D * D; i += 256) Ms[i] = M[i];
+  const int warp = tid / 32, lane = tid % 32;
+  for (int rr = warp; rr < R; rr += 8) {
+    float x[D / 32], mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) {
+      x[i] = to_f32(qm[(row0 + rr) * D + lane + 32 * i]);
+      mx = fmaxf(mx, x[i]);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffff, mx, o));
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) { x[i] = expf(x[i] - mx); sum += x[i]; }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffff, sum, o);
+    const float inv = 1.f / sum;
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) ps[rr * (D + 1) + lane + 32 * i] = x[i] * inv;
+  }
+  __syncthreads();
+  const int ty = tid / 16, tx = tid % 16;  // rows ty*4..+4, cols tx*CT..+CT
+  float acc[4][CT];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < CT; ++j) acc[i][j] = 0.f;
+  for (int f = 0; f < D; ++f) {
+    float a[4], b[CT];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[i] = ps[(ty * 4 + i) * (D + 1) + f];
+#pragma unroll
+    for (int j = 0; j < CT; ++j) b[j] = Ms[f * D + tx * CT + j];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < CT; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < CT; ++j) out[(row0 + ty * 4 + i) * D + tx * CT + j] = from_f32<TIn>(acc[i][j]);
+}
+
+// ------------------------------------------------------------------------
+// SCA with CUDA cores: 32 queries per CTA, 4 threads per query (each owns
+// D/4 dims of q and of the output), keys streamed through shared memory in
+// tiles of 32 with an online softmax.  Scale 1.  grid (T / 32, BH).
+template <typename TIn, int D>
+__global__ void __launch_bounds__(128) sca_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
+                                                       const TIn* __restrict__ v, TIn* __restrict__ out,
+                                                       int64_t T, int c) {
+  constexpr int QD = D / 4;
+  __shared__ float ks[32][D + 4];
+  __shared__ float vs[32][D + 4];
+  const int64_t bh = blockIdx.y;
+  const int64_t t0 = (int64_t)blockIdx.x * 32;
+  const int tid = threadIdx.x;
+  const int qi = tid / 4, part = tid % 4;
+  const int64_t t = t0 + qi;
+  const int64_t lo = t0 / c >= 1 ? (t0 / c - 1) * c : 0;  // all 32 rows share one chunk
+  const TIn* qrow = q + (bh * T + t) * D + part * QD;
+  float qv[QD], acc[QD];
+#pragma unroll
+  for (int i = 0; i < QD; ++i) { qv[i] = to_f32(qrow[i]); acc[i] = 0.f; }
+  float m = -INFINITY, l = 0.f;
+  const int64_t hi = t0 + 31;
+  for (int64_t k0 = lo; k0 <= hi; k0 += 32) {
+    __syncthreads();
+    for (int i = tid; i < 32 * D; i += 128) {
+      const int r = i / D, cc = i % D;
+      const int64_t g = (bh * T + k0 + r) * D + cc;
+      ks[r][cc] = to_f32(k[g]);
+      vs[r][cc] = to_f32(v[g]);
+    }
+    __syncthreads();
+    for (int j = 0; j < 32; ++j) {
+      float sc = 0.f;
+#pragma unroll
+      for (int i = 0; i < QD; ++i) sc = fmaf(qv[i], ks[j][part * QD + i], sc);
+      sc += __shfl_xor_sync(0xffffffff, sc, 1);
+      sc += __shfl_xor_sync(0xffffffff, sc, 2);
+      if (k0 + j > t) continue;  // causal inside the current chunk
+      const float mn = fmaxf(m, sc);
+      const float corr = expf(m - mn);
+      const float p = expf(sc - mn);
+      l = l * corr + p;
+#pragma unroll
+      for (int i = 0; i < QD; ++i) acc[i] = fmaf(p, vs[j][part * QD + i], acc[i] * corr);
+      m = mn;
+    }
+  }
+  const float inv = 1.f / l;
+  TIn* orow = out + (bh * T + t) * D + part * QD;
+#pragma unroll
+  for (int i = 0; i < QD; ++i) orow[i] = from_f32<TIn>(acc[i] * inv);
+}
+
+template <typename TIn, int D>
+cudaError_t launch_simt_awm_impl(const Problem& p, const Workspace& w, bool chunk_gemms, cudaStream_t st) {
+  const int S = p.S;
+  const int64_t BH = p.B * p.H;
+  const TIn* km = static_cast<const TIn*>(p.km);
+  const TIn* v = static_cast<const TIn*>(p.v);
+  const TIn* qm = static_cast<const TIn*>(p.qm);
+  awm_lse_kernel<TIn, D><<<dim3(S, BH), 256, 0, st>>>(km, w.lse, p.T, (int)p.c);
+  awm_prefix_kernel<D><<<BH, D, 0, st>>>(w.lse, w.logz, w.ratio, S);
+  if (chunk_gemms)
+    awm_chunk_simt_kernel<TIn, D><<<dim3(S, BH), 256, 0, st>>>(km, v, w.logz, w.Bm, w.Cm, p.T, (int)p.c);
+  constexpr int JC = 16;
+  const size_t carry_smem = sizeof(float) * (D * (D + 1) + D * JC);
+  cudaFuncSetAttribute(awm_carry_kernel<D, JC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)carry_smem);
+  awm_carry_kernel<D, JC><<<dim3(D / JC, BH), 256, carry_smem, st>>>(w.Bm, w.Cm, w.ratio, w.Mst, S);
+  if (p.readout_simt) {
+    const size_t ro_smem = sizeof(float) * (D * D + 64 * (D + 1));
+    cudaFuncSetAttribute(awm_readout_simt_kernel<TIn, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)ro_smem);
+    awm_readout_simt_kernel<TIn, D><<<dim3(p.c / 64, S, BH), 256, ro_smem, st>>>(
+        qm, w.Mst, static_cast<TIn*>(p.out_mem), p.T, (int)p.c);
+  }
+  return cudaGetLastError();
+}
+
+template <typename TIn, int D>
+cudaError_t launch_sca_simt_impl(const Problem& p, cudaStream_t st) {
+  sca_simt_kernel<TIn, D><<<dim3(p.T / 32, p.B * p.H), 128, 0, st>>>(
+      static_cast<const TIn*>(p.q), static_cast<const TIn*>(p.k), static_cast<const TIn*>(p.v),
+      static_cast<TIn*>(p.out_sca), p.T, (int)p.c);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_awm_simt(const Problem& p, const Workspace& w, bool chunk_gemms, cudaStream_t st) {
+  if (p.dtype == kF32)
+    return p.d == 64 ? launch_simt_awm_impl<float, 64>(p, w, chunk_gemms, st)
+                     : launch_simt_awm_impl<float, 128>(p, w, chunk_gemms, st);
+  return p.d == 64 ? launch_simt_awm_impl<__nv_bfloat16, 64>(p, w, chunk_gemms, st)
+                   : launch_simt_awm_impl<__nv_bfloat16, 128>(p, w, chunk_gemms, st);
+}
+
+cudaError_t launch_sca_simt(const Problem& p, cudaStream_t st) {
+  if (p.dtype == kF32)
+    return p.d == 64 ? launch_sca_simt_impl<float, 64>(p, st) : launch_sca_simt_impl<float, 128>(p, st);
+  return p.d == 64 ? launch_sca_simt_impl<__nv_bfloat16, 64>(p, st)
+                   : launch_sca_simt_impl<__nv_bfloat16, 128>(p, st);
+}
+
+}  // namespace gecko

@@ -1,0 +1,146 @@
+"""Thin ctypes binding of libgecko.so (the C ABI declared in include/gecko.h).
+
+Argument marshalling only: every step of the forward runs in the library's
+CUDA kernels.  PyTorch supplies device memory and the current stream.  There
+is no fallback: if the library is missing or cannot load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgecko.so")
+
+# Symbols declared in include/gecko.h
+EXPORTS = (
+    "gecko_sca_awm_forward",
+    "gecko_awm_state",
+    "gecko_device_status",
+    "gecko_last_error",
+    "gecko_release",
+)
+
+GECKO_F32, GECKO_BF16 = 0, 1
+STATUS = {
+    0: "GECKO_OK", 1: "GECKO_ERR_ARG", 2: "GECKO_ERR_SHAPE", 3: "GECKO_ERR_ALIGN",
+    4: "GECKO_ERR_ALLOC", 5: "GECKO_ERR_CUDA", 6: "GECKO_ERR_NO_STATE", 7: "GECKO_ERR_TIMEOUT",
+}
+
+_lib = None
+
+
+class GeckoError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{STATUS.get(code, code)}: {msg}")
+        self.code = code
+
+
+def load() -> ctypes.CDLL:
+    """Load libgecko.so once; raise if it is absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m long_context_sequence_sca_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    i64, vp = ctypes.c_int64, ctypes.c_void_p
+    lib.gecko_sca_awm_forward.argtypes = [vp] * 7 + [i64] * 5 + [ctypes.c_int, vp]
+    lib.gecko_sca_awm_forward.restype = ctypes.c_int
+    lib.gecko_awm_state.argtypes = [vp, vp, i64, i64, i64, vp]
+    lib.gecko_awm_state.restype = ctypes.c_int
+    lib.gecko_device_status.argtypes = [vp]
+    lib.gecko_device_status.restype = ctypes.c_int
+    lib.gecko_last_error.argtypes = []
+    lib.gecko_last_error.restype = ctypes.c_char_p
+    lib.gecko_release.argtypes = []
+    lib.gecko_release.restype = None
+    _lib = lib
+    return lib
+
+
+def _check(rc: int):
+    if rc != 0:
+        raise GeckoError(rc, load().gecko_last_error().decode())
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+# ------------------------------------------------------- raw C entry points --
+
+def gecko_sca_awm_forward(q, k, v, qm, km, out_sca, out_mem, B, H, T, c, d, dtype, stream) -> int:
+    """Direct call of the C entry point with integer pointers; returns the status."""
+    return load().gecko_sca_awm_forward(q, k, v, qm, km, out_sca, out_mem, B, H, T, c, d, dtype, stream)
+
+
+def gecko_awm_state(M_out, logz_out, B, H, d, stream) -> int:
+    return load().gecko_awm_state(M_out, logz_out, B, H, d, stream)
+
+
+def gecko_device_status(stream) -> int:
+    return load().gecko_device_status(stream)
+
+
+def gecko_last_error() -> str:
+    return load().gecko_last_error().decode()
+
+
+def gecko_release() -> None:
+    load().gecko_release()
+
+
+# ------------------------------------------------------- tensor front end --
+
+_DT = {torch.float32: GECKO_F32, torch.bfloat16: GECKO_BF16}
+
+
+def sca_awm_forward(q, k, v, qm, km, c: int, out_sca=None, out_mem=None, stream=None):
+    """Fused SCA + AWM forward on [B, H, T, d] CUDA tensors.
+
+    Returns (out_sca, out_mem); the layer output is their sum.  Outputs are
+    allocated with torch if not given.  Runs asynchronously on `stream`
+    (default: torch's current stream).
+    """
+    xs = (q, k, v, qm, km)
+    for x in xs:
+        if not (isinstance(x, torch.Tensor) and x.is_cuda and x.is_contiguous()):
+            raise ValueError("inputs must be contiguous CUDA tensors")
+        if x.shape != q.shape or x.dtype != q.dtype or x.device != q.device:
+            raise ValueError("inputs must share shape, dtype and device")
+    if q.dim() != 4 or q.dtype not in _DT:
+        raise ValueError("inputs must be [B, H, T, d] float32 or bfloat16")
+    B, H, T, d = q.shape
+    if out_sca is None:
+        out_sca = torch.empty_like(q)
+    if out_mem is None:
+        out_mem = torch.empty_like(q)
+    with torch.cuda.device(q.device):
+        rc = gecko_sca_awm_forward(*(x.data_ptr() for x in xs), out_sca.data_ptr(), out_mem.data_ptr(),
+                                   B, H, T, c, d, _DT[q.dtype], _stream_handle(stream))
+    _check(rc)
+    return out_sca, out_mem
+
+
+def awm_state(B: int, H: int, d: int, device=None, stream=None):
+    """(M'_{S+1} [B, H, d, d], log z^S [B, H, d]) of the last forward, fp32."""
+    device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    M = torch.empty(B, H, d, d, dtype=torch.float32, device=device)
+    lz = torch.empty(B, H, d, dtype=torch.float32, device=device)
+    with torch.cuda.device(device):
+        _check(gecko_awm_state(M.data_ptr(), lz.data_ptr(), B, H, d, _stream_handle(stream)))
+    return M, lz
+
+
+def device_status(stream=None) -> int:
+    """Synchronise, read and clear the device status word (0 = OK)."""
+    return gecko_device_status(_stream_handle(stream))
+
+
+def release() -> None:
+    gecko_release()

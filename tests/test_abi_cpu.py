@@ -1,0 +1,71 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function include/gecko.h declares, and rejects bad arguments on the
+host before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from long_context_sequence_sca_b200 import build as B
+from long_context_sequence_sca_b200 import lib as L
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "gecko.h")
+
+
+@pytest.fixture(scope="module")
+def so():
+    B.build()
+    return L.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gecko_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_expected_entry_points():
+    assert set(declared_functions()) == set(L.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(so):
+    for name in declared_functions():
+        assert hasattr(so, name), name
+    out = os.popen(f"nm -D --defined-only {L.LIB_PATH}").read()
+    for name in declared_functions():
+        assert re.search(rf"\bT {name}\b", out), name
+
+
+def test_no_torch_types_in_header():
+    text = open(HEADER).read()
+    assert "torch" not in text.lower().replace("pytorch", "") and "at::" not in text
+
+
+# Each case fails host validation, so nothing reaches CUDA.
+FAKE = 0x100000  # 16-byte aligned, never dereferenced
+
+
+def _call(ptrs=None, B=1, H=1, T=256, c=128, d=64, dtype=1):
+    ptrs = ptrs or [FAKE] * 7
+    return L.gecko_sca_awm_forward(*ptrs, B, H, T, c, d, dtype, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ptrs=[0] + [FAKE] * 6), 1),
+    (dict(dtype=7), 1),
+    (dict(B=0), 1),
+    (dict(T=-4), 1),
+    (dict(d=96), 2),
+    (dict(c=96, T=192), 2),
+    (dict(T=300, c=128), 2),
+    (dict(ptrs=[FAKE, FAKE + 8] + [FAKE] * 5), 3),
+    (dict(B=1 << 40, H=1 << 20), 2),
+])
+def test_host_validation_rejects(so, kw, code):
+    assert _call(**kw) == code
+    assert L.gecko_last_error()
+
+
+def test_state_query_rejects_null(so):
+    assert L.gecko_awm_state(0, 0, 1, 1, 64, None) == 1
