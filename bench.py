@@ -1,0 +1,488 @@
+#!/usr/bin/env python
+"""Throughput of the fused Gecko SCA + AWM forward (tokens/s, bf16).
+
+Default workload: the 7B-layer-shaped case B=1, H=32, d=128, c=4096,
+T=32768 (8 chunks), synthetic inputs from the seeded generator, all resident
+in HBM (1.34 GB of inputs, larger than the 126 MB L2, so no L2 flush is
+needed between steps).  One step = one forward through the C ABI
+(AWM statistics, chunk products, carry, readout, SCA).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl gecko|reference]
+
+N > 1 runs under torchrun, one rank per GPU, each rank a full replica of the
+workload on its own inputs (weak scaling; the heads and batches of the method
+are independent, so there is no data-path collective).  The timed region is
+bracketed by a barrier and a device synchronise; the step time is the max
+over ranks; rank 0 prints one JSON line.
+
+`--impl reference` times the CPU oracle (fp64 NumPy, the machine's host cores) on
+bounded samples of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from long_context_sequence_sca_b200.inputs import WORKLOADS, Workload, make_inputs  # noqa: E402
+
+DEFAULT_WORKLOAD = "bf16_h32_c4096"
+METRIC = "tokens/s fused SCA+AWM fwd (bf16,H=32,d=128,c=4096); % bf16 TC peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+SCA_PROFILE = os.path.join(ROOT, "profiles", "sca_tc_traffic.json")
+
+
+# ------------------------------------------------------- algorithmic work --
+
+def sca_pairs(w: Workload) -> int:
+    """(query, key) pairs the SCA must score per (b, h): chunk 1 is causal over
+    itself; every later chunk sees all c previous keys plus its causal part."""
+    S, c = w.S, w.c
+    return S * c * (c + 1) // 2 + (S - 1) * c * c
+
+
+def flops(w: Workload) -> dict:
+    """Algorithmic FLOPs (2 per multiply-add) of one forward."""
+    BH, c, d, S = w.B * w.H, w.c, w.d, w.S
+    f_sca = 4 * d * sca_pairs(w) * BH                    # QK^T and PV
+    # AWM: chunk products Phi^T V (all S) and Phi^T Psi (S-1 needed), the
+    # d x d carry product C M' (S-1), and the readout of chunks 3..S.
+    f_awm = (2 * c * d * d + (S - 1) * 6 * c * d * d + max(S - 2, 0) * 2 * c * d * d) * BH
+    return {"sca": f_sca, "awm": f_awm, "total": f_sca + f_awm}
+
+
+def io_bytes(w: Workload) -> int:
+    """Algorithmic HBM bytes: five inputs read once, two outputs written once."""
+    esz = 2 if w.dtype == "bf16" else 4
+    return 7 * w.B * w.H * w.T * w.d * esz
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML (read-only) in a
+    background thread while the timed region runs."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.ok = False
+        self.samples = []
+        self.period = period_s
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            self.nv = nv
+            self.h = self._handle(device_index)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.err = repr(e)
+
+    def _handle(self, idx):
+        nv = self.nv
+        props = torch.cuda.get_device_properties(idx)
+        uuid = getattr(props, "uuid", None)
+        if uuid is not None:
+            s = str(uuid)
+            for cand in (s if s.startswith("GPU-") else "GPU-" + s,):
+                try:
+                    return nv.nvmlDeviceGetHandleByUUID(cand)
+                except Exception:
+                    pass
+        bus = getattr(props, "pci_bus_id", None)
+        dom = getattr(props, "pci_domain_id", 0)
+        dev = getattr(props, "pci_device_id", 0)
+        if bus is not None:
+            return nv.nvmlDeviceGetHandleByPciBusId(f"{dom:08x}:{bus:02x}:{dev:02x}.0")
+        return nv.nvmlDeviceGetHandleByIndex(idx)
+
+    def _reasons(self):
+        nv = self.nv
+        fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        return int(fn(self.h))
+
+    def _loop(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append((self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM),
+                                     self._reasons()))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        self.samples = []
+        if not self.ok:
+            return
+        self._stop = threading.Event()
+        self._t = threading.Thread(target=self._loop, daemon=True)
+        self._t.start()
+
+    def stop(self) -> dict:
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "error": getattr(self, "err", "nvml unavailable")}
+        self._stop.set()
+        self._t.join()
+        mhz = [m for m, _ in self.samples]
+        bits = 0
+        for _, r in self.samples:
+            bits |= r
+        reasons = sorted(name for b, name in self.REASONS.items() if bits & b)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(mhz), "source": "nvml"}
+
+
+BAD_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+
+
+def clocks_rejected(ck: dict) -> bool:
+    if not ck.get("samples"):
+        return False
+    if BAD_REASONS & set(ck["reasons"]):
+        return True
+    # stuck well below max with no reason: a leftover clock lock
+    return bool(ck["sm_mhz"] and ck["sm_max_mhz"] and not ck["reasons"]
+                and ck["sm_mhz"] < 0.6 * ck["sm_max_mhz"])
+
+
+# ------------------------------------------------------------ multi-rank --
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    """Max of a per-rank scalar (the step time) over all ranks."""
+    if ws == 1:
+        return float(x)
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(ms_local: float, tokens_local: int, ws: int) -> dict:
+    """Whole-job throughput: all ranks' tokens over the slowest rank's time."""
+    ms = max_over_ranks(ms_local, ws)
+    return {"ms_per_step": ms, "value": tokens_local * ws / (ms / 1e3)}
+
+
+# ------------------------------------------------------------ CPU oracle --
+
+def oracle_sample(w: Workload, n_chunks: int, head: int = 0):
+    """A bounded sample of the workload for the CPU oracle: the first
+    n_chunks chunks of one (b, h) head, drawn by the same generator recipe
+    (shapes, c, d and distributions of the workload)."""
+    sw = w.with_(B=1, H=1, T=n_chunks * w.c, dtype="f32", name=w.name + "_sample", wid=w.wid * 10 + head)
+    x = make_inputs(sw, device="cpu")
+    return {k_: v_.to(torch.bfloat16).double().numpy() if w.dtype == "bf16" else v_.double().numpy()
+            for k_, v_ in x.items()}, sw.T
+
+
+def time_oracle(w: Workload, n_chunks: int, reps: int = 1, head: int = 0):
+    from oracle import gecko_oracle as G
+    tot_s, tot_tok = 0.0, 0
+    for r in range(reps):
+        x, tok = oracle_sample(w, n_chunks, head + r)
+        t0 = time.perf_counter()
+        G.forward(x["q"], x["k"], x["v"], x["qm"], x["km"], w.c)
+        tot_s += time.perf_counter() - t0
+        tot_tok += tok
+    return tot_tok / tot_s, tot_s, tot_tok
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# --------------------------------------------------------- traffic record --
+
+def sca_source_hash() -> str:
+    h = hashlib.sha1()
+    for f in ("sca_tc.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "long_context_sequence_sca_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+def recorded_traffic(w: Workload):
+    """DRAM bytes per SCA launch from the committed ncu record, or None if the
+    record is missing, for another workload, or older than the kernel source."""
+    if not os.path.exists(SCA_PROFILE):
+        return None
+    with open(SCA_PROFILE) as f:
+        rec = json.load(f)
+    if rec.get("source_hash") != sca_source_hash() or rec.get("workload") != w.name:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ arms --
+
+def run_gecko(args, w: Workload, ws: int, rank: int, local: int) -> dict:
+    from long_context_sequence_sca_b200 import lib as L
+    L.load()
+    x = make_inputs(w, device="cuda", seed_offset=1000 * rank)
+    o_sca = torch.empty_like(x["q"])
+    o_mem = torch.empty_like(x["q"])
+    stream = torch.cuda.current_stream()
+
+    def step():
+        L.sca_awm_forward(x["q"], x["k"], x["v"], x["qm"], x["km"], w.c, o_sca, o_mem, stream)
+
+    L.timing_enable(True)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    L.timing_read()
+    if L.device_status() != 0:
+        raise RuntimeError("device status reported a timed-out wait during warm-up")
+
+    sampler = ClockSampler(local)
+
+    def timed():
+        barrier(ws)
+        torch.cuda.synchronize()
+        L.timing_read()
+        sampler.start()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ck = sampler.stop()
+        barrier(ws)
+        stages, n = L.timing_read()
+        return e0.elapsed_time(e1) / args.steps, {k_: v_ / max(n, 1) for k_, v_ in stages.items()}, ck
+
+    ms_local, stages, ck = timed()
+    note = None
+    if clocks_rejected(ck):
+        note = f"re-measured once: first run saw clocks {ck}"
+        ms_local, stages, ck = timed()
+    if L.device_status() != 0:
+        raise RuntimeError("device status reported a timed-out wait")
+    tokens = w.B * w.T
+    agg = aggregate(ms_local, tokens, ws)
+    fl = flops(w)
+    pk, pk_kind = peaks()
+
+    # dominant kernel: the SCA launch (one per step), timed on its stream
+    sca_ms = max_over_ranks(stages["sca"], ws)
+    achieved = fl["sca"] / (sca_ms / 1e3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "sca_tc_kernel", "achieved": round(achieved, 2),
+                "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops"], 4),
+                "peak_kind": f"{pk_kind} bf16 dense (burst)",
+                "frac_of_sustained": round(achieved / pk["bf16_tflops_sustained"], 4),
+                "traffic": recorded_traffic(w), "launch_ms": round(sca_ms, 4),
+                "algorithmic_flop_per_launch": fl["sca"]}
+
+    out = {
+        "metric": METRIC, "value": round(agg["value"], 1), "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(agg["ms_per_step"], 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded Z'-affine generator; no dataset)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "c": w.c,
+                   "tokens_per_step_per_gpu": tokens,
+                   "l2": f"inputs larger than L2 ({5 * w.B * w.H * w.T * w.d * 2 / 1e9:.2f} GB), no flush",
+                   "parallelism": f"replicas x{ws} (heads/batches independent)"},
+        "tflops": round(ws * fl["total"] / (agg["ms_per_step"] / 1e3) / 1e12, 2),
+        "pct_bf16_peak": round(100 * fl["total"] / (agg["ms_per_step"] / 1e3) / 1e12 / pk["bf16_tflops"], 2),
+        "stage_ms": {k_: round(v_, 4) for k_, v_ in stages.items()},
+        "roofline": roofline,
+        "clocks": ck,
+        "gpu_launches": 7 * args.steps,  # lse partial, lse combine, prefix, chunk, carry, readout, sca
+    }
+    if note:
+        out["note"] = note
+    if not args.no_e2e:
+        out["e2e"] = run_e2e(args, w, x, ws, stream, L)
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(w)
+    return out
+
+
+def run_e2e(args, w, x, ws, stream, L) -> dict:
+    """Same metric through the public API with host buffers: every step copies
+    its five inputs from pinned host memory and reads both outputs back."""
+    names = ("q", "k", "v", "qm", "km")
+    host_in = {n: x[n].cpu().pin_memory() for n in names}
+    dev_in = {n: torch.empty_like(x[n]) for n in names}
+    host_out = [torch.empty(x["q"].shape, dtype=x["q"].dtype).pin_memory() for _ in range(2)]
+    dev_out = [torch.empty_like(x["q"]) for _ in range(2)]
+    steps = max(1, min(args.steps, 10))
+
+    def step():
+        for n in names:
+            dev_in[n].copy_(host_in[n], non_blocking=True)
+        L.sca_awm_forward(*(dev_in[n] for n in names), w.c, dev_out[0], dev_out[1], stream)
+        host_out[0].copy_(dev_out[0], non_blocking=True)
+        host_out[1].copy_(dev_out[1], non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    barrier(ws)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    L.timing_read()
+    agg = aggregate(e0.elapsed_time(e1) / steps, w.B * w.T, ws)
+    nb = x["q"].numel() * x["q"].element_size()
+    return {"value": round(agg["value"], 1), "unit": "tokens/s", "h2d_bytes_per_step": 5 * nb,
+            "d2h_bytes_per_step": 2 * nb, "steps": steps, "ms_per_step": round(agg["ms_per_step"], 3)}
+
+
+def cpu_baseline(w: Workload) -> dict:
+    n_chunks = 3 if w.S >= 3 else w.S
+    tok_s, secs, tok = time_oracle(w, n_chunks, reps=2)
+    return {"value": round(tok_s, 2), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"fp64 oracle forward on the first {n_chunks} chunks of 2 heads "
+                      f"({tok} tokens, c={w.c}, d={w.d}) in {secs:.1f} s"}
+
+
+def run_reference(args, w: Workload) -> dict:
+    """The CPU oracle as the reference arm: every step is one bounded sample
+    (the first chunks of one head), timed with perf_counter."""
+    n_chunks = 2 if w.S >= 2 else 1
+    for i in range(args.warmup):
+        time_oracle(w, n_chunks, head=i)
+    tot_s, tot_tok = 0.0, 0
+    for i in range(args.steps):
+        _, s, t = time_oracle(w, n_chunks, head=100 + i)
+        tot_s += s
+        tot_tok += t
+    val = tot_tok / tot_s
+    sample = (f"per step: fp64 oracle forward on the first {n_chunks} chunks of one head "
+              f"({n_chunks * w.c} tokens, c={w.c}, d={w.d})")
+    return {
+        "metric": METRIC, "value": round(val, 2), "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1e3 * tot_s / args.steps, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "c": w.c},
+        "impl": "reference", "host": "CPU oracle on the box's host cores (no GPU work)",
+        "cpu_baseline": {"value": round(val, 2), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(val, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def summarize_launches(path: str) -> str:
+    """Per-kernel launches, total time and share from an ncu launch-list CSV
+    (`ncu --metrics gpu__time_duration.sum --csv`)."""
+    import collections
+    import csv
+    import re
+    rows = list(csv.reader(open(path)))
+    hi = next(i for i, r in enumerate(rows) if "Kernel Name" in r)
+    hdr = rows[hi]
+    ki, mi, vi, ui = (hdr.index(k) for k in ("Kernel Name", "Metric Name", "Metric Value", "Metric Unit"))
+    scale = {"ns": 1e-3, "nsecond": 1e-3, "us": 1.0, "usecond": 1.0, "ms": 1e3, "msecond": 1e3}
+    agg = collections.OrderedDict()
+    for r in rows[hi + 1:]:
+        if len(r) <= vi or r[mi] != "gpu__time_duration.sum":
+            continue
+        name = re.sub(r"\(.*", "", r[ki]).replace("void ", "").replace("gecko::(anonymous namespace)::", "")
+        a = agg.setdefault(name, [0, 0.0])
+        a[0] += 1
+        a[1] += float(r[vi].replace(",", "")) * scale[r[ui]]
+    tot = sum(a[1] for a in agg.values()) or 1.0
+    lines = [f"{'kernel':44s} {'launches':>8s} {'total_us':>10s} {'share':>7s}"]
+    for k, (n, t) in sorted(agg.items(), key=lambda kv: -kv[1][1]):
+        lines.append(f"{k:44s} {n:8d} {t:10.1f} {100 * t / tot:6.1f}%")
+    return "\n".join(lines)
+
+
+def main(argv=None):
+    if argv is None and len(sys.argv) > 2 and sys.argv[1] == "--summarize-launches":
+        print(summarize_launches(sys.argv[2]))
+        return 0
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("gecko", "reference"), default="gecko")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, w)), flush=True)
+        return 0
+
+    ws, rank, local = dist_setup()
+    if ws != args.gpus and rank == 0:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {ws}", file=sys.stderr)
+    try:
+        out = run_gecko(args, w, ws, rank, local)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

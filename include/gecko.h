@@ -109,6 +109,24 @@ int gecko_awm_state(float* M_out, float* logz_out,
  */
 int gecko_device_status(void* stream);
 
+/*
+ * Measurement support.  gecko_timing_enable(1) makes every later forward
+ * record CUDA events on its stream around its five stages:
+ *   0 AWM statistics (per-chunk log exp-sums of K_m and the log z prefix),
+ *   1 AWM chunk products (Phi^T V and Phi^T Psi per chunk),
+ *   2 AWM carry (the sequential M' recurrence),
+ *   3 AWM readout (psi(Q_m) M'_{s-1}),
+ *   4 SCA.
+ * gecko_timing_read() waits for the recorded forwards, writes the summed
+ * milliseconds per stage into ms_per_stage[0 .. min(capacity, 5) - 1] and
+ * the number of forwards into *n_calls, and clears the record.  Returns
+ * GECKO_OK, GECKO_ERR_ARG for NULL buffers or capacity < 1, or
+ * GECKO_ERR_CUDA.  Timing is off by default; when on it costs six event
+ * records per forward.
+ */
+int gecko_timing_enable(int enable);
+int gecko_timing_read(float* ms_per_stage, int capacity, int* n_calls);
+
 /* Thread-local message describing the last non-zero status of this thread. */
 const char* gecko_last_error(void);
 

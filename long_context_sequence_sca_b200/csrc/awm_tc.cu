@@ -1,0 +1,477 @@
+// Adaptive Working Memory kernels on 5th-generation tensor cores (sm_100a).
+//
+// The AWM of the Gecko digest (paper.rainbus.top, core method and method
+// step details, steps 4-5) needs, per (b, h) and chunk s:
+//   Phi_s = exp(Km_s - log z^s)       (online-softmax kernel over time)
+//   Psi_s = rowsoftmax(Km_s)          (softmax over features)
+//   Bm_s  = Phi_s^T V_s,   Cm_s = Phi_s^T Psi_s        (d x d, fp32)
+// for the carry M'_{s+1} = r_s (.) M'_s - Cm_s M'_s + Bm_s, and the readout
+//   O_m,s = psi(Qm_s) M'_{s-1}.
+//
+// awm_chunk_tc_kernel: one CTA per (chunk, bh).  The chunk is streamed in
+// tiles of 64 tokens.  V tiles arrive by TMA; 128 threads (two per token)
+// compute Phi and Psi in fp32 and store them as bf16 next to V in one
+// 128-byte-swizzled, MN-major stage [V | Psi | Phi], so a single
+// tcgen05.mma with M = d, N = 2d accumulates [Phi^T V | Phi^T Psi] in TMEM.
+//
+// awm_readout_tc_kernel: one CTA per (chunk, bh).  M'_{s-1} is converted to
+// bf16 once into shared memory (MN-major B operand); every 128-row tile of
+// Qm_s is turned into psi rows (K-major A operand) by 128 threads, one row
+// each, and multiplied on the tensor core; the epilogue writes bf16 rows.
+#include "common.cuh"
+#include "gecko_internal.h"
+
+namespace gecko {
+namespace {
+
+// Byte offset of element (row, col) in a 128-byte-swizzled tile made of
+// 64-column boxes of `rows` rows each (the TMA SWIZZLE_128B layout).
+__device__ __forceinline__ uint32_t sw128_off(int row, int col, int rows) {
+  const int box = col >> 6, cc = col & 63;
+  return box * rows * 128 + row * 128 + ((((cc >> 3) ^ (row & 7)) << 4)) + ((cc & 7) << 1);
+}
+
+// ------------------------------------------------------------ chunk GEMMs --
+
+constexpr int kKT = 64;  // tokens per tile
+
+template <int D>
+struct ChunkCfg {
+  static constexpr int kBox = kKT * 128;                 // one [64 x 64] bf16 box
+  static constexpr int kOperand = (D / 64) * kBox;       // a [64 x D] operand
+  static constexpr int kStage = 3 * kOperand;            // [V | Psi | Phi]
+  static constexpr int kStages = 2;
+  static constexpr int kBarOff = kStages * kStage;
+  // v_full[2], op_full[2], stage_empty[2], acc_full
+  static constexpr int kNumBars = 7;
+  static constexpr int kLzOff = kBarOff + kNumBars * 8;  // D floats: log2(e) * log z^s
+  static constexpr int kMiscOff = kLzOff + D * 4;
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kAlloc = kBytes + 1024;
+  static constexpr uint32_t kTmemCols = D == 128 ? 256 : 128;
+};
+
+// 128 compute threads (warps 0-3), warp 4 = TMA producer, warp 5 = MMA issuer.
+template <int D>
+__global__ void __launch_bounds__(192, 2) awm_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_v,
+                                                           const __nv_bfloat16* __restrict__ km,
+                                                           const float* __restrict__ logz, float* __restrict__ Bm,
+                                                           float* __restrict__ Cm, int T, int c, int* status) {
+  using Cfg = ChunkCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
+  uint64_t* v_full = bars;          // [2] TMA -> MMA
+  uint64_t* op_full = bars + 2;     // [2] compute -> MMA (128 arrivals)
+  uint64_t* st_empty = bars + 4;    // [2] MMA -> TMA, compute
+  uint64_t* acc_full = bars + 6;
+  float* lz2 = reinterpret_cast<float*>(smem + Cfg::kLzOff);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
+
+  const int s = blockIdx.x, S = gridDim.x;
+  const int64_t bh = blockIdx.y;
+  const int warp = warp_id_uniform(), lane = threadIdx.x % 32;
+  const int n_tiles = c / kKT;
+  const int64_t row0 = bh * (int64_t)T + (int64_t)s * c;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(v_full + i, 1);
+      mbar_init(op_full + i, 128);
+      mbar_init(st_empty + i, 1);
+    }
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  for (int f = threadIdx.x; f < D; f += blockDim.x) lz2[f] = logz[(bh * S + s) * D + f] * kLog2e;
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ----------------------------------------------------- V tiles by TMA --
+    if (lane == 0) {
+      tma_prefetch_desc(&map_v);
+      for (int kt = 0; kt < n_tiles; ++kt) {
+        const int st = kt & 1;
+        if (!mbar_wait(st_empty + st, ((kt >> 1) & 1) ^ 1, abort_flag, status)) break;
+        mbar_arrive_expect_tx(v_full + st, Cfg::kOperand);
+        for (int b = 0; b < D / 64; ++b)
+          tma_load_2d(smem + st * Cfg::kStage + b * Cfg::kBox, &map_v, v_full + st, b * 64,
+                      (int)(row0 + (int64_t)kt * kKT));
+      }
+      if (*abort_flag) {
+        for (int st = 0; st < 2; ++st) mbar_wait_drain(v_full + st, ((n_tiles - 1 - st) >> 1) & 1);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // --------------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(D, 2 * D, true, true);
+      const uint32_t base = smem_u32(smem);
+      bool ok = true;
+      for (int kt = 0; kt < n_tiles && ok; ++kt) {
+        const int st = kt & 1;
+        const uint32_t ph = (kt >> 1) & 1;
+        if (!(ok = mbar_wait(v_full + st, ph, abort_flag, status))) break;
+        if (!(ok = mbar_wait(op_full + st, ph, abort_flag, status))) break;
+        tc_fence_after();
+        const uint32_t sb = base + st * Cfg::kStage;
+#pragma unroll
+        for (int kk = 0; kk < kKT / 16; ++kk) {
+          // A = Phi^T (M = D features, MN-major), B = [V | Psi] (N = 2D, MN-major)
+          const uint64_t adesc = sdesc_sw128(sb + 2 * Cfg::kOperand + kk * 2048, Cfg::kBox, 1024);
+          const uint64_t bdesc = sdesc_sw128(sb + kk * 2048, Cfg::kBox, 1024);
+          umma_ss(tmem, adesc, bdesc, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(st_empty + st);
+      }
+      umma_commit(acc_full);
+      mbar_wait_drain(acc_full, 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------ Phi / Psi, then epilogue --
+    const int r = threadIdx.x >> 1;       // token row within the tile
+    const int h = threadIdx.x & 1;        // which half of the features
+    constexpr int HF = D / 2;             // features per thread
+    bool ok = true;
+    uint4 cur[HF / 8], nxt[HF / 8];
+    const __nv_bfloat16* src = km + row0 * D + (int64_t)r * D + h * HF;
+#pragma unroll
+    for (int i = 0; i < HF / 8; ++i) cur[i] = reinterpret_cast<const uint4*>(src)[i];
+    for (int kt = 0; kt < n_tiles; ++kt) {
+      const int st = kt & 1;
+      if (kt + 1 < n_tiles) {
+        const __nv_bfloat16* nsrc = src + (int64_t)(kt + 1) * kKT * D;
+#pragma unroll
+        for (int i = 0; i < HF / 8; ++i) nxt[i] = reinterpret_cast<const uint4*>(nsrc)[i];
+      }
+      float x[HF];
+#pragma unroll
+      for (int i = 0; i < HF / 8; ++i) {
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&cur[i]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f2 = __bfloat1622float2(p2[j]);
+          x[8 * i + 2 * j] = f2.x;
+          x[8 * i + 2 * j + 1] = f2.y;
+        }
+      }
+      float mx = x[0];
+#pragma unroll
+      for (int i = 1; i < HF; ++i) mx = fmaxf(mx, x[i]);
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      const float mx2 = mx * kLog2e;
+      float e[HF], sum = 0.f;
+#pragma unroll
+      for (int i = 0; i < HF; ++i) {
+        e[i] = ex2(fmaf(x[i], kLog2e, -mx2));
+        sum += e[i];
+      }
+      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+      const float inv = 1.f / sum;
+      // wait until the MMAs of tile kt-2 have released this stage
+      ok = __all_sync(0xffffffffu, mbar_wait(st_empty + st, ((kt >> 1) & 1) ^ 1, abort_flag, status));
+      if (!ok) break;
+      uint8_t* stg = smem + st * Cfg::kStage;
+#pragma unroll
+      for (int i = 0; i < HF / 8; ++i) {
+        const int col = h * HF + 8 * i;
+        uint4 ps, ph;
+        uint32_t* pp = reinterpret_cast<uint32_t*>(&ps);
+        uint32_t* pf = reinterpret_cast<uint32_t*>(&ph);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          pp[j] = pack_bf16x2(e[8 * i + 2 * j] * inv, e[8 * i + 2 * j + 1] * inv);
+          pf[j] = pack_bf16x2(ex2(fmaf(x[8 * i + 2 * j], kLog2e, -lz2[col + 2 * j])),
+                              ex2(fmaf(x[8 * i + 2 * j + 1], kLog2e, -lz2[col + 2 * j + 1])));
+        }
+        const uint32_t off = sw128_off(r, col, kKT);
+        *reinterpret_cast<uint4*>(stg + Cfg::kOperand + off) = ps;
+        *reinterpret_cast<uint4*>(stg + 2 * Cfg::kOperand + off) = ph;
+      }
+      // generic-proxy writes must be visible to the tensor core (async proxy)
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(op_full + st);
+#pragma unroll
+      for (int i = 0; i < HF / 8; ++i) cur[i] = nxt[i];
+    }
+    // epilogue: accumulator row f = TMEM lane; columns [0, D) = Bm, [D, 2D) = Cm
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, status));
+    if (ok) {
+      tc_fence_after();
+      // M = 128: row f lives in lane f.  M = 64: rows 16w..16w+15 live in
+      // lanes 32w..32w+15 of warp w.
+      const bool valid = D == 128 || lane < 16;
+      const int f = D == 128 ? warp * 32 + lane : warp * 16 + lane;
+      const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
+      const int64_t o = (bh * S + s) * (int64_t)D * D + (int64_t)f * D;
+#pragma unroll 1
+      for (int cb = 0; cb < 2 * D / 32; ++cb) {
+        uint32_t v[32];
+        tmem_ld32(taddr + cb * 32, v);
+        tmem_wait_ld();
+        if (valid) {
+          float* dst = (cb * 32 < D) ? (Bm + o + cb * 32) : (Cm + o + cb * 32 - D);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            reinterpret_cast<float4*>(dst)[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                                            __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) tmem_dealloc(tmem, Cfg::kTmemCols);
+}
+
+// --------------------------------------------------------------- readout --
+
+template <int D>
+struct ReadoutCfg {
+  static constexpr int kA = 128 * D * 2;     // psi tile, K-major, D/64 boxes of [128 x 64]
+  static constexpr int kB = D * D * 2;       // M' bf16, MN-major, D/64 boxes of [D x 64]
+  static constexpr int kAOff = 0;
+  static constexpr int kBOff = 2 * kA;       // two A buffers
+  static constexpr int kBarOff = kBOff + kB;
+  static constexpr int kNumBars = 4;         // a_full[2], acc_full[2]
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kAlloc = kBytes + 1024;
+  static constexpr uint32_t kTmemCols = 2 * D;   // two accumulators
+};
+
+// 128 threads: one row each; thread 0 also issues the MMAs.  Tiles of the
+// chunk are processed two at a time (double-buffered A and accumulators).
+template <int D>
+__global__ void __launch_bounds__(128) awm_readout_tc_kernel(const __nv_bfloat16* __restrict__ qm,
+                                                             const float* __restrict__ Mst,
+                                                             __nv_bfloat16* __restrict__ out, int T, int c,
+                                                             int* status) {
+  using Cfg = ReadoutCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* a_full = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);  // [0]: drain after an abort
+  uint64_t* acc_full = a_full + 2;                                        // [2] MMA -> threads
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
+
+  const int s = blockIdx.x, S = gridDim.x;
+  const int64_t bh = blockIdx.y;
+  const int warp = warp_id_uniform(), lane = threadIdx.x % 32;
+  const int r = threadIdx.x;
+  const int n_tiles = c / 128;
+  const int64_t row0 = bh * (int64_t)T + (int64_t)s * c;
+
+  if (s < 2) {
+    // chunks 1 and 2 read M'_0 = M'_1 = 0
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    uint4* dst = reinterpret_cast<uint4*>(out + row0 * D);
+    const int64_t n = (int64_t)c * D / 8;
+    for (int64_t i = threadIdx.x; i < n; i += blockDim.x) dst[i] = z;
+    return;
+  }
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(acc_full + i, 1);
+      mbar_init(a_full + i, 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  // B operand: M'_{s-1} (0-based chunk s reads Mst[s-1]) as bf16, rows = key
+  // feature f (K), columns = value dim j (N, contiguous): MN-major.
+  const float* M = Mst + (bh * (S + 1) + (s - 1)) * (int64_t)D * D;
+  for (int i = threadIdx.x; i < D * D / 8; i += blockDim.x) {
+    const int f = (i * 8) / D, j = (i * 8) % D;
+    const float4 a = reinterpret_cast<const float4*>(M + f * D + j)[0];
+    const float4 b = reinterpret_cast<const float4*>(M + f * D + j)[1];
+    uint4 p;
+    p.x = pack_bf16x2(a.x, a.y);
+    p.y = pack_bf16x2(a.z, a.w);
+    p.z = pack_bf16x2(b.x, b.y);
+    p.w = pack_bf16x2(b.z, b.w);
+    *reinterpret_cast<uint4*>(smem + Cfg::kBOff + sw128_off(f, j, D)) = p;
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t base = smem_u32(smem);
+  constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, true);
+  const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+  bool ok = true;
+
+  auto psi_tile = [&](int kt, int buf) {
+    const uint4* src = reinterpret_cast<const uint4*>(qm + (row0 + (int64_t)kt * 128 + r) * D);
+    float x[D];
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) {
+      const uint4 u = src[i];
+      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f2 = __bfloat1622float2(p2[j]);
+        x[8 * i + 2 * j] = f2.x;
+        x[8 * i + 2 * j + 1] = f2.y;
+      }
+    }
+    float mx = x[0];
+#pragma unroll
+    for (int i = 1; i < D; ++i) mx = fmaxf(mx, x[i]);
+    const float mx2 = mx * kLog2e;
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < D; ++i) {
+      x[i] = ex2(fmaf(x[i], kLog2e, -mx2));
+      sum += x[i];
+    }
+    const float inv = 1.f / sum;
+    uint8_t* a = smem + Cfg::kAOff + buf * Cfg::kA;
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) {
+      uint4 p;
+      p.x = pack_bf16x2(x[8 * i] * inv, x[8 * i + 1] * inv);
+      p.y = pack_bf16x2(x[8 * i + 2] * inv, x[8 * i + 3] * inv);
+      p.z = pack_bf16x2(x[8 * i + 4] * inv, x[8 * i + 5] * inv);
+      p.w = pack_bf16x2(x[8 * i + 6] * inv, x[8 * i + 7] * inv);
+      *reinterpret_cast<uint4*>(a + sw128_off(r, 8 * i, 128)) = p;
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (threadIdx.x == 0) {
+      const uint32_t aa = base + Cfg::kAOff + buf * Cfg::kA;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t koff = (kk / 4) * (128 * 128) + (kk % 4) * 32;
+        const uint64_t adesc = sdesc_sw128(aa + koff, 16, 1024);
+        const uint64_t bdesc = sdesc_sw128(base + Cfg::kBOff + kk * 16 * 128, D * 128, 1024);
+        umma_ss(tmem + buf * D, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+      }
+      umma_commit(acc_full + buf);
+    }
+  };
+
+  auto store_tile = [&](int kt, int buf, uint32_t parity) -> bool {
+    if (!__all_sync(0xffffffffu, mbar_wait(acc_full + buf, parity, abort_flag, status))) return false;
+    tc_fence_after();
+    __nv_bfloat16* orow = out + (row0 + (int64_t)kt * 128 + r) * D;
+#pragma unroll 1
+    for (int cb = 0; cb < D / 32; ++cb) {
+      uint32_t v[32];
+      tmem_ld32(lane_addr + buf * D + cb * 32, v);
+      tmem_wait_ld();
+      uint4 w[4];
+      uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) wp[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+      uint4* dst = reinterpret_cast<uint4*>(orow + cb * 32);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) dst[i] = w[i];
+    }
+    tc_fence_before();
+    return true;
+  };
+
+  // software pipeline: psi of tile kt overlaps the MMA of tile kt-1; the
+  // epilogue of tile kt-1 runs once its accumulator is ready.
+  for (int kt = 0; kt < n_tiles && ok; ++kt) {
+    const int buf = kt & 1;
+    psi_tile(kt, buf);
+    if (kt > 0) ok = store_tile(kt - 1, buf ^ 1, ((kt - 1) >> 1) & 1);
+    // the next psi_tile(kt+1) writes A buffer buf^1 and accumulator buf^1;
+    // both were released by store_tile(kt-1) above (its MMA completed)
+  }
+  if (ok) ok = store_tile(n_tiles - 1, (n_tiles - 1) & 1, ((n_tiles - 1) >> 1) & 1);
+  if (!ok && threadIdx.x == 0) {
+    // make sure no MMA is still writing TMEM before it is released
+    umma_commit(a_full);
+    mbar_wait_drain(a_full, 0);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, Cfg::kTmemCols);
+}
+
+// ------------------------------------------------------------------ host --
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+template <int D>
+cudaError_t chunk_impl(const Problem& p, const Workspace& w, cudaStream_t st) {
+  using Cfg = ChunkCfg<D>;
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  CUtensorMap mv;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)(p.B * p.H * p.T)};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)kKT};
+  cuuint32_t estr[2] = {1, 1};
+  if (fn(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(p.v), dims, strides, box, estr,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(awm_chunk_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Cfg::kAlloc);
+  if (e != cudaSuccess) return e;
+  awm_chunk_tc_kernel<D><<<dim3(p.S, p.B * p.H), 192, Cfg::kAlloc, st>>>(
+      mv, static_cast<const __nv_bfloat16*>(p.km), w.logz, w.Bm, w.Cm, (int)p.T, (int)p.c, p.status);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t readout_impl(const Problem& p, const Workspace& w, cudaStream_t st) {
+  using Cfg = ReadoutCfg<D>;
+  cudaError_t e = cudaFuncSetAttribute(awm_readout_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Cfg::kAlloc);
+  if (e != cudaSuccess) return e;
+  awm_readout_tc_kernel<D><<<dim3(p.S, p.B * p.H), 128, Cfg::kAlloc, st>>>(
+      static_cast<const __nv_bfloat16*>(p.qm), w.Mst, static_cast<__nv_bfloat16*>(p.out_mem), (int)p.T,
+      (int)p.c, p.status);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_awm_chunk_tc(const Problem& p, const Workspace& w, cudaStream_t st) {
+  return p.d == 64 ? chunk_impl<64>(p, w, st) : chunk_impl<128>(p, w, st);
+}
+
+cudaError_t launch_awm_readout_tc(const Problem& p, const Workspace& w, cudaStream_t st) {
+  return p.d == 64 ? readout_impl<64>(p, w, st) : readout_impl<128>(p, w, st);
+}
+
+}  // namespace gecko

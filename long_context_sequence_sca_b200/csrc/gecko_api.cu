@@ -5,7 +5,10 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <array>
+#include <atomic>
 #include <map>
+#include <vector>
 #include <mutex>
 #include <string>
 
@@ -18,20 +21,26 @@ namespace gecko {
 // The device status word (bit kStatusTimeout: a bounded wait ran out).
 __device__ int g_status_word;
 
-size_t workspace_bytes(int64_t BH, int64_t S, int64_t d) {
+size_t workspace_bytes(int64_t BH, int64_t T, int64_t c, int64_t d) {
   auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const int64_t S = T / c;
+  const size_t part = al(sizeof(float) * 2 * BH * (T / stats_block_rows(c)) * d);
   const size_t vec = al(sizeof(float) * BH * S * d);
   const size_t mat = al(sizeof(float) * BH * S * d * d);
   const size_t mst = al(sizeof(float) * BH * (S + 1) * d * d);
-  return 3 * vec + 2 * mat + mst;
+  return part + 3 * vec + 2 * mat + mst;
 }
 
-Workspace carve_workspace(void* base, int64_t BH, int64_t S, int64_t d) {
+Workspace carve_workspace(void* base, int64_t BH, int64_t T, int64_t c, int64_t d) {
   auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
   char* p = static_cast<char*>(base);
   Workspace w;
+  const int64_t S = T / c;
+  const size_t part = al(sizeof(float) * 2 * BH * (T / stats_block_rows(c)) * d);
   const size_t vec = al(sizeof(float) * BH * S * d);
   const size_t mat = al(sizeof(float) * BH * S * d * d);
+  w.part = reinterpret_cast<float2*>(p);
+  p += part;
   w.lse = reinterpret_cast<float*>(p);
   p += vec;
   w.logz = reinterpret_cast<float*>(p);
@@ -65,7 +74,7 @@ struct DeviceState {
   size_t ws_bytes = 0;
   int* status = nullptr;  // device address of g_status_word
   bool have_state = false;
-  int64_t B = 0, H = 0, d = 0, S = 0;
+  int64_t B = 0, H = 0, d = 0, S = 0, T = 0;
 };
 
 std::mutex g_mu;
@@ -116,6 +125,51 @@ int validate(const void* const* ptrs, int n, int64_t B, int64_t H, int64_t T, in
   return GECKO_OK;
 }
 
+// Optional per-stage timing with CUDA events recorded on the caller's
+// stream around each stage of a forward; accumulated until read.
+constexpr int kStages = 5;  // awm stats, awm chunk, awm carry, awm readout, sca
+std::atomic<bool> g_timing{false};
+std::mutex g_tmu;
+std::vector<std::array<cudaEvent_t, kStages + 1>> g_pending;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t take_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+struct StageEvents {
+  cudaStream_t st;
+  bool on;
+  std::array<cudaEvent_t, kStages + 1> ev{};
+  explicit StageEvents(cudaStream_t s) : st(s), on(g_timing.load()) {
+    if (on) {
+      std::lock_guard<std::mutex> lk(g_tmu);
+      for (auto& e : ev) e = take_event();
+    }
+  }
+  void mark(int i) {
+    if (on) cudaEventRecord(ev[i], st);
+  }
+  void commit() {
+    if (!on) return;
+    std::lock_guard<std::mutex> lk(g_tmu);
+    g_pending.push_back(ev);
+    on = false;
+  }
+  ~StageEvents() {
+    if (!on) return;  // an error path: recycle the events
+    std::lock_guard<std::mutex> lk(g_tmu);
+    for (auto& e : ev) g_event_pool.push_back(e);
+  }
+};
+
 }  // namespace
 }  // namespace gecko
 
@@ -137,7 +191,7 @@ extern "C" int gecko_sca_awm_forward(const void* q, const void* k, const void* v
 
   const int64_t S = T / c;
   const int64_t BH = B * H;
-  const size_t need = workspace_bytes(BH, S, d);
+  const size_t need = workspace_bytes(BH, T, c, d);
   if (env_is("GECKO_FAIL_ALLOC", "1")) return fail(GECKO_ERR_ALLOC, "workspace allocation failed (injected)");
   if (need > ds->ws_bytes) {
     if (ds->ws) {
@@ -154,28 +208,38 @@ extern "C" int gecko_sca_awm_forward(const void* q, const void* k, const void* v
     ds->ws = p;
     ds->ws_bytes = need;
   }
-  Workspace w = carve_workspace(ds->ws, BH, S, d);
+  Workspace w = carve_workspace(ds->ws, BH, T, c, d);
 
-  Problem p{q, k, v, qm, km, out_sca, out_mem, B, H, T, c, d, (int)S, dtype, true, ds->status};
+  Problem p{q, k, v, qm, km, out_sca, out_mem, B, H, T, c, d, (int)S, dtype, ds->status};
   // GECKO_KERNELS=simt selects the CUDA-core kernels for every dtype (a
   // second, independent GPU implementation used to cross-check the
   // tensor-core path).
   const bool force_simt = env_is("GECKO_KERNELS", "simt");
   const bool use_tc = !force_simt && tc_supported(p);
-  p.readout_simt = true;
 
   cudaGetLastError();  // clear stale errors from the caller
-  if ((rc = check_cuda(launch_awm_simt(p, w, /*chunk_gemms=*/true, st), "awm (simt)"))) return rc;
-  if (use_tc) {
-    if ((rc = check_cuda(launch_sca_tc(p, st), "sca (tensor core)"))) return rc;
-  } else {
-    if ((rc = check_cuda(launch_sca_simt(p, st), "sca (simt)"))) return rc;
-  }
+  StageEvents ev(st);
+  ev.mark(0);
+  if ((rc = check_cuda(launch_awm_stats(p, w, st), "awm stats"))) return rc;
+  ev.mark(1);
+  if ((rc = check_cuda(use_tc ? launch_awm_chunk_tc(p, w, st) : launch_awm_chunk_simt(p, w, st), "awm chunk")))
+    return rc;
+  ev.mark(2);
+  if ((rc = check_cuda(launch_awm_carry(p, w, st), "awm carry"))) return rc;
+  ev.mark(3);
+  if ((rc = check_cuda(use_tc ? launch_awm_readout_tc(p, w, st) : launch_awm_readout_simt(p, w, st),
+                       "awm readout")))
+    return rc;
+  ev.mark(4);
+  if ((rc = check_cuda(use_tc ? launch_sca_tc(p, st) : launch_sca_simt(p, st), "sca"))) return rc;
+  ev.mark(5);
+  ev.commit();
   ds->have_state = true;
   ds->B = B;
   ds->H = H;
   ds->d = d;
   ds->S = S;
+  ds->T = T;
   return GECKO_OK;
 }
 
@@ -193,7 +257,7 @@ extern "C" int gecko_awm_state(float* M_out, float* logz_out, int64_t B, int64_t
     return fail(GECKO_ERR_ARG, "state is B=%lld H=%lld d=%lld, asked for B=%lld H=%lld d=%lld", (long long)ds.B,
                 (long long)ds.H, (long long)ds.d, (long long)B, (long long)H, (long long)d);
   const int64_t BH = B * H, S = ds.S;
-  Workspace w = carve_workspace(ds.ws, BH, S, d);
+  Workspace w = carve_workspace(ds.ws, BH, ds.T, ds.T / ds.S, d);
   const size_t mat = sizeof(float) * d * d;
   // M'_{S+1} of each (b, h) sits at Mst[bh, S]; log z^S at logz[bh, S-1]
   if ((rc = check_cuda(cudaMemcpy2DAsync(M_out, mat, w.Mst + S * d * d, mat * (S + 1), mat, BH,
@@ -247,4 +311,29 @@ extern "C" void gecko_release(void) {
     kv.second.have_state = false;
   }
   cudaSetDevice(cur);
+}
+
+extern "C" int gecko_timing_enable(int enable) {
+  g_timing.store(enable != 0);
+  return GECKO_OK;
+}
+
+extern "C" int gecko_timing_read(float* ms_per_stage, int capacity, int* n_calls) {
+  if (!ms_per_stage || !n_calls || capacity < 1) return fail(GECKO_ERR_ARG, "bad timing buffers");
+  std::lock_guard<std::mutex> lk(g_tmu);
+  double acc[kStages] = {0};
+  for (auto& evs : g_pending) {
+    cudaError_t e = cudaEventSynchronize(evs[kStages]);
+    if (e != cudaSuccess) return check_cuda(e, "event synchronize");
+    for (int i = 0; i < kStages; ++i) {
+      float ms = 0.f;
+      cudaEventElapsedTime(&ms, evs[i], evs[i + 1]);
+      acc[i] += ms;
+    }
+    for (auto& x : evs) g_event_pool.push_back(x);
+  }
+  *n_calls = (int)g_pending.size();
+  g_pending.clear();
+  for (int i = 0; i < kStages && i < capacity; ++i) ms_per_stage[i] = (float)acc[i];
+  return GECKO_OK;
 }

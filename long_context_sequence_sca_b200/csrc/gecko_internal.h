@@ -17,12 +17,12 @@ struct Problem {
   int64_t B, H, T, c, d;
   int S;
   int dtype;
-  bool readout_simt;  // readout by the SIMT kernel (else by the tensor-core one)
   int* status;        // device status word
 };
 
 // Device workspace carved out of one allocation (all fp32).
 struct Workspace {
+  float2* part;  // [BH, T / R, d]  (max, sum exp(x - max)) of K_m per block of R rows
   float* lse;    // [BH, S, d]  log of per-chunk exp-sums of K_m
   float* logz;   // [BH, S, d]  log z^s
   float* ratio;  // [BH, S, d]  z^{s-1} / z^s  (0 for s = 1)
@@ -31,11 +31,18 @@ struct Workspace {
   float* Mst;    // [BH, S+1, d, d]  M'_1 .. M'_{S+1}
 };
 
-// Bytes needed by a Workspace for (BH, S, d), each region 256-byte aligned.
-size_t workspace_bytes(int64_t BH, int64_t S, int64_t d);
-Workspace carve_workspace(void* base, int64_t BH, int64_t S, int64_t d);
+// Rows per block of the partial K_m statistics (divides c).
+inline int stats_block_rows(int64_t c) { return c % 256 == 0 ? 256 : 64; }
 
-cudaError_t launch_awm_simt(const Problem& p, const Workspace& w, bool chunk_gemms, cudaStream_t st);
+// Bytes needed by a Workspace, each region 256-byte aligned.
+size_t workspace_bytes(int64_t BH, int64_t T, int64_t c, int64_t d);
+Workspace carve_workspace(void* base, int64_t BH, int64_t T, int64_t c, int64_t d);
+
+// CUDA-core kernels (any dtype, any c % 64 == 0).
+cudaError_t launch_awm_stats(const Problem& p, const Workspace& w, cudaStream_t st);   // lse + log z prefix
+cudaError_t launch_awm_chunk_simt(const Problem& p, const Workspace& w, cudaStream_t st);
+cudaError_t launch_awm_carry(const Problem& p, const Workspace& w, cudaStream_t st);
+cudaError_t launch_awm_readout_simt(const Problem& p, const Workspace& w, cudaStream_t st);
 cudaError_t launch_sca_simt(const Problem& p, cudaStream_t st);
 
 // Tensor-core (tcgen05 + TMEM + TMA) kernels, bf16 with c % 128 == 0.

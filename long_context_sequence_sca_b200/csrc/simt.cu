@@ -36,33 +36,31 @@ template <> struct Vec8<float> {
 };
 
 // ------------------------------------------------------------------------
-// Per-chunk, per-feature log of the exp-sum: lse[bh, s, f] =
-// log sum_{i in chunk s} exp(km[i, f]).  grid (S, BH), 256 threads; each
-// thread keeps a running (max, sum) for 8 features over a strided row set.
+// Partial statistics of K_m per block of R rows: for each feature f the
+// block max m and sum_i exp(km[i, f] - m).  grid (T / R, BH), 256 threads;
+// each thread keeps a running (max, sum) for 8 features over a strided row
+// set, then the row groups are merged in shared memory.
 template <typename TIn, int D>
-__global__ void __launch_bounds__(256) awm_lse_kernel(const TIn* __restrict__ km, float* __restrict__ lse,
-                                                      int64_t T, int c) {
+__global__ void __launch_bounds__(256) awm_lse_partial_kernel(const TIn* __restrict__ km, float2* __restrict__ part,
+                                                              int64_t T, int R) {
   constexpr int TPR = D / 8;          // threads per row
   constexpr int RG = 256 / TPR;       // rows processed in parallel
-  const int s = blockIdx.x;
+  const int blk = blockIdx.x, nblk = gridDim.x;
   const int64_t bh = blockIdx.y;
   const int lane8 = threadIdx.x % TPR;
   const int rg = threadIdx.x / TPR;
-  const TIn* base = km + (bh * T + (int64_t)s * c) * D + lane8 * 8;
+  const TIn* base = km + (bh * T + (int64_t)blk * R) * D + lane8 * 8;
   float m[8], acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) { m[i] = -INFINITY; acc[i] = 0.f; }
-  for (int r = rg; r < c; r += RG) {
+  for (int r = rg; r < R; r += RG) {
     float x[8];
     Vec8<TIn>::load(base + (int64_t)r * D, x);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      if (x[i] > m[i]) {
-        acc[i] = acc[i] * expf(m[i] - x[i]) + 1.f;
-        m[i] = x[i];
-      } else {
-        acc[i] += expf(x[i] - m[i]);
-      }
+      const float mn = fmaxf(m[i], x[i]);
+      acc[i] = acc[i] * expf(m[i] - mn) + expf(x[i] - mn);
+      m[i] = mn;
     }
   }
   __shared__ float sm[RG][D + 1];
@@ -79,8 +77,27 @@ __global__ void __launch_bounds__(256) awm_lse_kernel(const TIn* __restrict__ km
     float tot = 0.f;
     for (int g = 0; g < RG; ++g)
       if (sm[g][f] > -INFINITY) tot += ss[g][f] * expf(sm[g][f] - M);
-    lse[(bh * gridDim.x + s) * D + f] = M + logf(tot);
+    part[(bh * nblk + blk) * D + f] = make_float2(M, tot);
   }
+}
+
+// Merge the P partials of each chunk: lse[bh, s, f] = log sum over the
+// chunk of exp(km[., f]).  grid (S, BH), D threads.
+template <int D>
+__global__ void __launch_bounds__(D) awm_lse_combine_kernel(const float2* __restrict__ part,
+                                                            float* __restrict__ lse, int P) {
+  const int s = blockIdx.x, S = gridDim.x;
+  const int64_t bh = blockIdx.y;
+  const int f = threadIdx.x;
+  const float2* p = part + (bh * (int64_t)S * P + (int64_t)s * P) * D + f;
+  float M = -INFINITY;
+  for (int i = 0; i < P; ++i) M = fmaxf(M, p[(int64_t)i * D].x);
+  float tot = 0.f;
+  for (int i = 0; i < P; ++i) {
+    const float2 v = p[(int64_t)i * D];
+    tot += v.y * expf(v.x - M);
+  }
+  lse[(bh * S + s) * D + f] = M + logf(tot);
 }
 
 // ------------------------------------------------------------------------
@@ -140,7 +157,7 @@ __global__ void __launch_bounds__(256) awm_chunk_simt_kernel(const TIn* __restri
   const int warp = tid / 32, lane = tid % 32;
   __syncthreads();
   for (int r0 = 0; r0 < c; r0 += RT) {
-    // each warp prepares 4 rows: phi, psi (warp-wide softmax over D), v
+    // each warp prepares RT/8 rows: phi, psi (warp-wide softmax over D), v
     for (int rr = warp; rr < RT; rr += 8) {
       const int64_t g = (row0 + r0 + rr) * D;
       float x[D / 32];
@@ -368,27 +385,42 @@ __global__ void __launch_bounds__(128) sca_simt_kernel(const TIn* __restrict__ q
 }
 
 template <typename TIn, int D>
-cudaError_t launch_simt_awm_impl(const Problem& p, const Workspace& w, bool chunk_gemms, cudaStream_t st) {
-  const int S = p.S;
+cudaError_t awm_stats_impl(const Problem& p, const Workspace& w, cudaStream_t st) {
   const int64_t BH = p.B * p.H;
-  const TIn* km = static_cast<const TIn*>(p.km);
-  const TIn* v = static_cast<const TIn*>(p.v);
-  const TIn* qm = static_cast<const TIn*>(p.qm);
-  awm_lse_kernel<TIn, D><<<dim3(S, BH), 256, 0, st>>>(km, w.lse, p.T, (int)p.c);
-  awm_prefix_kernel<D><<<BH, D, 0, st>>>(w.lse, w.logz, w.ratio, S);
-  if (chunk_gemms)
-    awm_chunk_simt_kernel<TIn, D><<<dim3(S, BH), 256, 0, st>>>(km, v, w.logz, w.Bm, w.Cm, p.T, (int)p.c);
+  const int R = stats_block_rows(p.c);
+  const int P = (int)(p.c / R);
+  awm_lse_partial_kernel<TIn, D><<<dim3((unsigned)(p.T / R), BH), 256, 0, st>>>(static_cast<const TIn*>(p.km),
+                                                                                 w.part, p.T, R);
+  awm_lse_combine_kernel<D><<<dim3(p.S, BH), D, 0, st>>>(w.part, w.lse, P);
+  awm_prefix_kernel<D><<<BH, D, 0, st>>>(w.lse, w.logz, w.ratio, p.S);
+  return cudaGetLastError();
+}
+
+template <typename TIn, int D>
+cudaError_t awm_chunk_simt_impl(const Problem& p, const Workspace& w, cudaStream_t st) {
+  awm_chunk_simt_kernel<TIn, D><<<dim3(p.S, p.B * p.H), 256, 0, st>>>(
+      static_cast<const TIn*>(p.km), static_cast<const TIn*>(p.v), w.logz, w.Bm, w.Cm, p.T, (int)p.c);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t awm_carry_impl(const Problem& p, const Workspace& w, cudaStream_t st) {
   constexpr int JC = 16;
-  const size_t carry_smem = sizeof(float) * (D * (D + 1) + D * JC);
-  cudaFuncSetAttribute(awm_carry_kernel<D, JC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)carry_smem);
-  awm_carry_kernel<D, JC><<<dim3(D / JC, BH), 256, carry_smem, st>>>(w.Bm, w.Cm, w.ratio, w.Mst, S);
-  if (p.readout_simt) {
-    const size_t ro_smem = sizeof(float) * (D * D + 64 * (D + 1));
-    cudaFuncSetAttribute(awm_readout_simt_kernel<TIn, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)ro_smem);
-    awm_readout_simt_kernel<TIn, D><<<dim3(p.c / 64, S, BH), 256, ro_smem, st>>>(
-        qm, w.Mst, static_cast<TIn*>(p.out_mem), p.T, (int)p.c);
-  }
+  const size_t smem = sizeof(float) * (D * (D + 1) + D * JC);
+  cudaError_t e = cudaFuncSetAttribute(awm_carry_kernel<D, JC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  awm_carry_kernel<D, JC><<<dim3(D / JC, p.B * p.H), 256, smem, st>>>(w.Bm, w.Cm, w.ratio, w.Mst, p.S);
+  return cudaGetLastError();
+}
+
+template <typename TIn, int D>
+cudaError_t awm_readout_simt_impl(const Problem& p, const Workspace& w, cudaStream_t st) {
+  const size_t smem = sizeof(float) * (D * D + 64 * (D + 1));
+  cudaError_t e =
+      cudaFuncSetAttribute(awm_readout_simt_kernel<TIn, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  awm_readout_simt_kernel<TIn, D><<<dim3(p.c / 64, p.S, p.B * p.H), 256, smem, st>>>(
+      static_cast<const TIn*>(p.qm), w.Mst, static_cast<TIn*>(p.out_mem), p.T, (int)p.c);
   return cudaGetLastError();
 }
 
@@ -402,13 +434,23 @@ cudaError_t launch_sca_simt_impl(const Problem& p, cudaStream_t st) {
 
 }  // namespace
 
-cudaError_t launch_awm_simt(const Problem& p, const Workspace& w, bool chunk_gemms, cudaStream_t st) {
-  if (p.dtype == kF32)
-    return p.d == 64 ? launch_simt_awm_impl<float, 64>(p, w, chunk_gemms, st)
-                     : launch_simt_awm_impl<float, 128>(p, w, chunk_gemms, st);
-  return p.d == 64 ? launch_simt_awm_impl<__nv_bfloat16, 64>(p, w, chunk_gemms, st)
-                   : launch_simt_awm_impl<__nv_bfloat16, 128>(p, w, chunk_gemms, st);
+#define GECKO_DISPATCH(FN)                                                              \
+  (p.dtype == kF32 ? (p.d == 64 ? FN<float, 64>(p, w, st) : FN<float, 128>(p, w, st))      \
+                   : (p.d == 64 ? FN<__nv_bfloat16, 64>(p, w, st) : FN<__nv_bfloat16, 128>(p, w, st)))
+
+cudaError_t launch_awm_stats(const Problem& p, const Workspace& w, cudaStream_t st) {
+  return GECKO_DISPATCH(awm_stats_impl);
 }
+cudaError_t launch_awm_chunk_simt(const Problem& p, const Workspace& w, cudaStream_t st) {
+  return GECKO_DISPATCH(awm_chunk_simt_impl);
+}
+cudaError_t launch_awm_carry(const Problem& p, const Workspace& w, cudaStream_t st) {
+  return p.d == 64 ? awm_carry_impl<64>(p, w, st) : awm_carry_impl<128>(p, w, st);
+}
+cudaError_t launch_awm_readout_simt(const Problem& p, const Workspace& w, cudaStream_t st) {
+  return GECKO_DISPATCH(awm_readout_simt_impl);
+}
+#undef GECKO_DISPATCH
 
 cudaError_t launch_sca_simt(const Problem& p, cudaStream_t st) {
   if (p.dtype == kF32)

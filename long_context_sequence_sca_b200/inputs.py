@@ -65,6 +65,9 @@ WORKLOADS = {
     "bf16_sweep_c2048": Workload("bf16_sweep_c2048", 4, "bf16", 1, 32, 65536, 128, 2048, key_offset_std=1.0),
     "bf16_sweep_c4096": Workload("bf16_sweep_c4096", 4, "bf16", 1, 32, 65536, 128, 4096, key_offset_std=1.0),
     "bf16_4m_tokens": Workload("bf16_4m_tokens", 5, "bf16", 1, 8, 4194304, 128, 4096),
+    # the headline shape with 4 heads: small enough for profiler captures,
+    # inputs (168 MB) still larger than L2
+    "bf16_h4_c4096": Workload("bf16_h4_c4096", 6, "bf16", 1, 4, 32768, 128, 4096),
 }
 
 

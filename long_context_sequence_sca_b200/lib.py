@@ -18,9 +18,14 @@ EXPORTS = (
     "gecko_sca_awm_forward",
     "gecko_awm_state",
     "gecko_device_status",
+    "gecko_timing_enable",
+    "gecko_timing_read",
     "gecko_last_error",
     "gecko_release",
 )
+
+# Stages timed by gecko_timing_read, in order.
+STAGES = ("awm_stats", "awm_chunk", "awm_carry", "awm_readout", "sca")
 
 GECKO_F32, GECKO_BF16 = 0, 1
 STATUS = {
@@ -53,6 +58,10 @@ def load() -> ctypes.CDLL:
     lib.gecko_awm_state.restype = ctypes.c_int
     lib.gecko_device_status.argtypes = [vp]
     lib.gecko_device_status.restype = ctypes.c_int
+    lib.gecko_timing_enable.argtypes = [ctypes.c_int]
+    lib.gecko_timing_enable.restype = ctypes.c_int
+    lib.gecko_timing_read.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
+    lib.gecko_timing_read.restype = ctypes.c_int
     lib.gecko_last_error.argtypes = []
     lib.gecko_last_error.restype = ctypes.c_char_p
     lib.gecko_release.argtypes = []
@@ -85,6 +94,14 @@ def gecko_awm_state(M_out, logz_out, B, H, d, stream) -> int:
 
 def gecko_device_status(stream) -> int:
     return load().gecko_device_status(stream)
+
+
+def gecko_timing_enable(enable: int) -> int:
+    return load().gecko_timing_enable(enable)
+
+
+def gecko_timing_read(ms_per_stage, capacity: int, n_calls) -> int:
+    return load().gecko_timing_read(ms_per_stage, capacity, n_calls)
 
 
 def gecko_last_error() -> str:
@@ -144,3 +161,15 @@ def device_status(stream=None) -> int:
 
 def release() -> None:
     gecko_release()
+
+
+def timing_enable(on: bool = True) -> None:
+    _check(gecko_timing_enable(1 if on else 0))
+
+
+def timing_read():
+    """({stage: summed ms}, number of forwards) since the last read."""
+    buf = (ctypes.c_float * len(STAGES))()
+    n = ctypes.c_int(0)
+    _check(gecko_timing_read(buf, len(STAGES), ctypes.byref(n)))
+    return {name: float(buf[i]) for i, name in enumerate(STAGES)}, int(n.value)

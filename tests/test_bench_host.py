@@ -1,0 +1,67 @@
+"""Host logic of bench.py: the algorithmic work counts and the multi-rank
+aggregation (world size 2 over gloo on CPU)."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+from long_context_sequence_sca_b200.inputs import Workload
+
+
+def test_sca_pair_count_matches_mask_enumeration():
+    for c, S in ((4, 1), (4, 3), (8, 5)):
+        w = Workload("t", 0, "bf16", 1, 1, c * S, 64, c)
+        n = sum(1 for t in range(w.T) for u in range(w.T) if u <= t and u // c >= t // c - 1)
+        assert bench.sca_pairs(w) == n
+
+
+def test_flops_and_bytes_headline():
+    w = bench.WORKLOADS["bf16_h32_c4096"]
+    f = bench.flops(w)
+    assert abs(f["sca"] / 1e12 - 3.024) < 0.01
+    assert abs(f["awm"] / 1e9 - 120.3) < 0.5
+    assert bench.io_bytes(w) == 7 * 32 * 32768 * 128 * 2
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _worker(rank, ws, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=ws)
+    try:
+        agg = bench.aggregate(ms_local=2.0 + rank, tokens_local=1000, ws=ws)
+        q.put((rank, agg))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_aggregate_max_over_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    ps = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in ps:
+        p.start()
+    got = dict(q.get(timeout=120) for _ in ps)
+    for p in ps:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for r in (0, 1):
+        assert got[r]["ms_per_step"] == 3.0
+        assert abs(got[r]["value"] - 2000 / 3e-3) < 1e-6
+
+
+def test_clock_rejection_rules():
+    assert bench.clocks_rejected({"samples": 5, "reasons": ["hw_slowdown"], "sm_mhz": 1800, "sm_max_mhz": 1965})
+    assert not bench.clocks_rejected({"samples": 5, "reasons": ["sw_power_cap"], "sm_mhz": 1300, "sm_max_mhz": 1965})
+    assert bench.clocks_rejected({"samples": 5, "reasons": [], "sm_mhz": 600, "sm_max_mhz": 1965})
