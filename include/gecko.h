@@ -59,6 +59,7 @@ extern "C" {
 #define GECKO_ERR_CUDA      5  /* a CUDA runtime call or kernel launch failed               */
 #define GECKO_ERR_NO_STATE  6  /* gecko_awm_state before any forward on this device         */
 #define GECKO_ERR_TIMEOUT   7  /* a bounded device-side wait ran out                        */
+#define GECKO_ERR_LIMIT     8  /* workspace above the fixed scratch of the no-allocation entry */
 
 /*
  * gecko_sca_awm_forward - fused SCA + AWM forward of one layer.
@@ -86,6 +87,42 @@ int gecko_sca_awm_forward(const void* q, const void* k, const void* v,
                           void* out_sca, void* out_mem,
                           int64_t B, int64_t H, int64_t T, int64_t c, int64_t d,
                           int dtype, void* stream);
+
+/*
+ * gecko_sca_awm_forward_noalloc - the same forward as gecko_sca_awm_forward
+ * (same arguments, kernels and results) for callers that must not allocate
+ * device memory themselves or through this library: for example a plugin
+ * whose host application's memory planner or pool owns all device memory,
+ * or a latency-critical loop that cannot afford cudaMalloc's implicit
+ * device-wide synchronisation.  The paper has no counterpart of this entry
+ * point; it only changes where the working memory comes from.
+ *
+ * Working memory: instead of the growable workspace, every call uses one
+ * fixed scratch array of GECKO_NOALLOC_SCRATCH_BYTES (64 MiB) that is part
+ * of the library's device image; each GPU that loads the library holds it
+ * until the process exits.  Inputs and outputs are still passed by the
+ * caller.  The scratch needs
+ *   4 * (2*BH*T/R*d + 3*BH*S*d + (3*S + 1)*BH*d*d) bytes (each of the six
+ *   regions rounded up to 256 bytes; R = 256 if c % 256 == 0 else 64,
+ *   S = T / c, BH = B * H),
+ * e.g. B*H = 32, T = 32768, c = 4096, d = 128 needs about 57 MB.  Larger
+ * problems are rejected with GECKO_ERR_LIMIT before anything is launched.
+ * The call makes no cudaMalloc, cudaFree or other allocating call.
+ *
+ * The first call on a device resolves the scratch array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls share the array and it keeps the
+ * last call's contents (every region is fully written before it is read,
+ * so nothing needs clearing); calls that overlap on the GPU race on it.
+ * This entry point does not update the state reported by gecko_awm_state,
+ * which always describes the last gecko_sca_awm_forward call.
+ */
+#define GECKO_NOALLOC_SCRATCH_BYTES (64ull << 20)
+int gecko_sca_awm_forward_noalloc(const void* q, const void* k, const void* v,
+                                  const void* qm, const void* km,
+                                  void* out_sca, void* out_mem,
+                                  int64_t B, int64_t H, int64_t T, int64_t c, int64_t d,
+                                  int dtype, void* stream);
 
 /*
  * gecko_awm_state - copy the AWM state carried out of the most recent

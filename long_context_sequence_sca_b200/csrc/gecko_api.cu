@@ -21,6 +21,11 @@ namespace gecko {
 // The device status word (bit kStatusTimeout: a bounded wait ran out).
 __device__ int g_status_word;
 
+// Fixed working memory of gecko_sca_awm_forward_noalloc.  In host code this
+// name is only a stand-in: its device address comes from
+// cudaGetSymbolAddress, resolved once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[GECKO_NOALLOC_SCRATCH_BYTES];
+
 size_t workspace_bytes(int64_t BH, int64_t T, int64_t c, int64_t d) {
   auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
   const int64_t S = T / c;
@@ -75,6 +80,7 @@ struct DeviceState {
   int* status = nullptr;  // device address of g_status_word
   bool have_state = false;
   int64_t B = 0, H = 0, d = 0, S = 0, T = 0;
+  void* noalloc_scratch = nullptr;  // device address of g_noalloc_scratch
 };
 
 std::mutex g_mu;
@@ -335,5 +341,48 @@ extern "C" int gecko_timing_read(float* ms_per_stage, int capacity, int* n_calls
   *n_calls = (int)g_pending.size();
   g_pending.clear();
   for (int i = 0; i < kStages && i < capacity; ++i) ms_per_stage[i] = (float)acc[i];
+  return GECKO_OK;
+}
+
+extern "C" int gecko_sca_awm_forward_noalloc(const void* q, const void* k, const void* v, const void* qm,
+                                             const void* km, void* out_sca, void* out_mem, int64_t B, int64_t H,
+                                             int64_t T, int64_t c, int64_t d, int dtype, void* stream) {
+  const void* ptrs[7] = {q, k, v, qm, km, out_sca, out_mem};
+  int rc = validate(ptrs, 7, B, H, T, c, d, dtype);
+  if (rc) return rc;
+  const int64_t S = T / c;
+  const int64_t BH = B * H;
+  const size_t need = workspace_bytes(BH, T, c, d);
+  if (need > GECKO_NOALLOC_SCRATCH_BYTES)
+    return fail(GECKO_ERR_LIMIT,
+                "this problem needs %zu bytes of working memory; the no-allocation entry point has a fixed "
+                "scratch of %llu bytes (use gecko_sca_awm_forward)",
+                need, (unsigned long long)GECKO_NOALLOC_SCRATCH_BYTES);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int dev = 0;
+  if ((rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice"))) return rc;
+
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState* ds = nullptr;
+  if ((rc = device_state(dev, &ds))) return rc;
+  if (!ds->noalloc_scratch) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return check_cuda(e, "cudaGetSymbolAddress(no-allocation scratch)");
+    ds->noalloc_scratch = p;
+  }
+  Workspace w = carve_workspace(ds->noalloc_scratch, BH, T, c, d);
+
+  Problem p{q, k, v, qm, km, out_sca, out_mem, B, H, T, c, d, (int)S, dtype, ds->status};
+  const bool use_tc = !env_is("GECKO_KERNELS", "simt") && tc_supported(p);
+  cudaGetLastError();
+  if ((rc = check_cuda(launch_awm_stats(p, w, st), "awm stats"))) return rc;
+  if ((rc = check_cuda(use_tc ? launch_awm_chunk_tc(p, w, st) : launch_awm_chunk_simt(p, w, st), "awm chunk")))
+    return rc;
+  if ((rc = check_cuda(launch_awm_carry(p, w, st), "awm carry"))) return rc;
+  if ((rc = check_cuda(use_tc ? launch_awm_readout_tc(p, w, st) : launch_awm_readout_simt(p, w, st),
+                       "awm readout")))
+    return rc;
+  if ((rc = check_cuda(use_tc ? launch_sca_tc(p, st) : launch_sca_simt(p, st), "sca"))) return rc;
   return GECKO_OK;
 }

@@ -16,6 +16,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgecko.so
 # Symbols declared in include/gecko.h
 EXPORTS = (
     "gecko_sca_awm_forward",
+    "gecko_sca_awm_forward_noalloc",
     "gecko_awm_state",
     "gecko_device_status",
     "gecko_timing_enable",
@@ -31,6 +32,7 @@ GECKO_F32, GECKO_BF16 = 0, 1
 STATUS = {
     0: "GECKO_OK", 1: "GECKO_ERR_ARG", 2: "GECKO_ERR_SHAPE", 3: "GECKO_ERR_ALIGN",
     4: "GECKO_ERR_ALLOC", 5: "GECKO_ERR_CUDA", 6: "GECKO_ERR_NO_STATE", 7: "GECKO_ERR_TIMEOUT",
+    8: "GECKO_ERR_LIMIT",
 }
 
 _lib = None
@@ -54,6 +56,8 @@ def load() -> ctypes.CDLL:
     i64, vp = ctypes.c_int64, ctypes.c_void_p
     lib.gecko_sca_awm_forward.argtypes = [vp] * 7 + [i64] * 5 + [ctypes.c_int, vp]
     lib.gecko_sca_awm_forward.restype = ctypes.c_int
+    lib.gecko_sca_awm_forward_noalloc.argtypes = [vp] * 7 + [i64] * 5 + [ctypes.c_int, vp]
+    lib.gecko_sca_awm_forward_noalloc.restype = ctypes.c_int
     lib.gecko_awm_state.argtypes = [vp, vp, i64, i64, i64, vp]
     lib.gecko_awm_state.restype = ctypes.c_int
     lib.gecko_device_status.argtypes = [vp]
@@ -86,6 +90,12 @@ def _stream_handle(stream) -> int:
 def gecko_sca_awm_forward(q, k, v, qm, km, out_sca, out_mem, B, H, T, c, d, dtype, stream) -> int:
     """Direct call of the C entry point with integer pointers; returns the status."""
     return load().gecko_sca_awm_forward(q, k, v, qm, km, out_sca, out_mem, B, H, T, c, d, dtype, stream)
+
+
+def gecko_sca_awm_forward_noalloc(q, k, v, qm, km, out_sca, out_mem, B, H, T, c, d, dtype, stream) -> int:
+    """The no-allocation entry point (fixed library scratch instead of a
+    growable workspace), with integer pointers; returns the status."""
+    return load().gecko_sca_awm_forward_noalloc(q, k, v, qm, km, out_sca, out_mem, B, H, T, c, d, dtype, stream)
 
 
 def gecko_awm_state(M_out, logz_out, B, H, d, stream) -> int:
