@@ -36,6 +36,65 @@ __device__ __forceinline__ float ex2(float x) {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// ------------------------------------------------ packed fp32 pairs (sm_100) --
+
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair of floats on the FMA pipe (no SFU).  Cody-Waite style range
+// reduction x = n + f with n = rint(x) (via the 1.5 * 2^23 rounding
+// constant) and f in [-1/2, 1/2], a cubic for 2^f, and n added to the
+// exponent field.  The cubic's coefficients were fitted for this library by
+// iteratively reweighted least squares (Lawson's method) on the relative
+// error over Chebyshev nodes of [-1/2, 1/2]; max relative error 7.5e-5,
+// below bf16 resolution (2^-9).  x is clamped to [-125, 126] so the exponent
+// arithmetic stays in the normal range; 2^-125 stands in for 0.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  float x0, x1;
+  unpack2(x2, x0, x1);
+  x0 = fminf(fmaxf(x0, -125.f), 126.f);
+  x1 = fminf(fmaxf(x1, -125.f), 126.f);
+  const uint64_t rnd = pack2(12582912.f, 12582912.f);    // 1.5 * 2^23
+  const uint64_t nrnd = pack2(-12582912.f, -12582912.f);
+  const uint64_t xc = pack2(x0, x1);
+  const uint64_t t = fadd2(xc, rnd);                      // n in the low mantissa bits
+  const uint64_t n = fadd2(t, nrnd);                      // rint(x)
+  float n0, n1;
+  unpack2(n, n0, n1);
+  const uint64_t f = fadd2(xc, pack2(-n0, -n1));          // x - rint(x)
+  uint64_t p = ffma2(f, pack2(0.0551716685295105f, 0.0551716685295105f),
+                     pack2(0.2426111400127411f, 0.2426111400127411f));
+  p = ffma2(p, f, pack2(0.6932609677314758f, 0.6932609677314758f));
+  p = ffma2(p, f, pack2(0.9999280571937561f, 0.9999280571937561f));
+  float p0, p1, t0, t1;
+  unpack2(p, p0, p1);
+  unpack2(t, t0, t1);
+  const uint32_t r0 = __float_as_uint(p0) + (__float_as_uint(t0) << 23);
+  const uint32_t r1 = __float_as_uint(p1) + (__float_as_uint(t1) << 23);
+  return pack2(__uint_as_float(r0), __uint_as_float(r1));
+}
+
 // ------------------------------------------------------------ status word --
 
 // Bits of the library's device status word.
@@ -149,6 +208,24 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   d |= static_cast<uint64_t>(1) << 46;  // descriptor version for sm_100
   d |= static_cast<uint64_t>(2) << 61;  // 128-byte swizzle
   return d;
+}
+
+// The same descriptor split into 32-bit halves, so a loop can advance the
+// start address with one 32-bit add on `lo` (start field = bits 0-13; tile
+// addresses stay below 256 KB, so the add never carries out of the field).
+struct SDesc {
+  uint32_t lo, hi;
+};
+__device__ __forceinline__ SDesc sdesc_sw128_split(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  SDesc d;
+  d.lo = ((saddr & 0x3FFFFu) >> 4) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+  d.hi = ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
+  return d;
+}
+__device__ __forceinline__ uint64_t sdesc_at(SDesc d, uint32_t byte_offset) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(d.lo + (byte_offset >> 4)), "r"(d.hi));
+  return r;
 }
 
 // Instruction descriptor for kind::f16 with bf16 operands and fp32 accumulate.

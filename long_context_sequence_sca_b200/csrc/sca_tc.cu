@@ -7,15 +7,16 @@
 // with scale 1, a causal mask inside the current chunk, and no previous chunk
 // for chunk 1.  Requires bf16, d in {64, 128}, c % 128 == 0.
 //
-// Design (one persistent CTA per SM, 384 threads):
+// Design (one persistent CTA per SM, 320 threads):
 //   warp 0      TMA producer: Q tiles once per work unit; K and V tiles of
 //               128 keys through a ring of shared-memory stages.
-//   warp 1      MMA issuer (one thread): S_i = Q_i K_j^T (SS form) into TMEM,
-//               O_i += P_i V_j with P_i read from TMEM (TS form).
-//   warp 2      TMEM allocator.
-//   warps 4-7   softmax for query tile 0, warps 8-11 for query tile 1; one
-//               thread per query row; online max/sum in registers; P written
-//               back to TMEM as bf16 over the S columns; epilogue O / l.
+//   warp 1      TMEM allocator and MMA issuer (one thread): S_i = Q_i K_j^T
+//               (SS form) into TMEM, O_i += P_i V_j with P_i read from TMEM
+//               (TS form).
+//   warps 2-5   softmax for query tile 0, warps 6-9 for query tile 1; one
+//               thread per query row (TMEM lane quarter = warp % 4); online
+//               max/sum in registers; P written back to TMEM as bf16 over the
+//               S columns; epilogue O / l.
 // A work unit is two adjacent 128-row query tiles of one (b, h).  The MMA
 // warp interleaves the two tiles (PV(0), QK(0), PV(1), QK(1)) so each
 // softmax warpgroup's exp work overlaps the other tile's MMAs.  Only the
@@ -38,7 +39,16 @@ namespace {
 
 constexpr int kBM = 128;   // query rows per tile
 constexpr int kBN = 128;   // keys per tile
-constexpr int kThreads = 384;
+constexpr int kThreads = 320;   // 10 warps: TMA, MMA (+TMEM allocation), 2 x 4 softmax
+// Of every 8 exponential pairs, GECKO_SFU_PAIRS are evaluated on the SFU
+// (ex2.approx) and the rest on the FMA pipe (exp2_poly2).  Measured on B200
+// with the bench workload the all-SFU setting is fastest (the polynomial
+// costs ~10 issue cycles per element against the SFU's 8-cycle warp rate),
+// so 8 is the default; other splits remain available at compile time.
+#ifndef GECKO_SFU_PAIRS
+#define GECKO_SFU_PAIRS 8
+#endif
+constexpr int kSfuPairs = GECKO_SFU_PAIRS;
 
 template <int D>
 struct ScaCfg {
@@ -157,7 +167,7 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
     tma_prefetch_desc(&map_k);
     tma_prefetch_desc(&map_v);
   }
-  if (warp == 2) {
+  if (warp == 1) {
     tmem_alloc(tmem_slot, Cfg::kTmemCols);
     tmem_relinquish();
   }
@@ -165,6 +175,7 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
@@ -243,11 +254,11 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
               if (!(ok = mbar_wait(p_full + i, p_cnt[i] & 1, abort_flag, status))) break;
               ++p_cnt[i];
               tc_fence_after();
+              const SDesc vd = sdesc_sw128_split(va + stV * Cfg::kTileBytes, Cfg::kBoxBytes, 1024);
+              umma_ts(tmem + colO, tmem + colS, sdesc_at(vd, 0), idesc_pv, j - 1 > U.beg[i] ? 1u : 0u);
 #pragma unroll
-              for (int kk = 0; kk < kBN / 16; ++kk) {
-                const uint64_t bdesc = sdesc_sw128(va + stV * Cfg::kTileBytes + kk * 2048, Cfg::kBoxBytes, 1024);
-                umma_ts(tmem + colO, tmem + colS + kk * 8, bdesc, idesc_pv, (j - 1 > U.beg[i] || kk > 0) ? 1u : 0u);
-              }
+              for (int kk = 1; kk < kBN / 16; ++kk)
+                umma_ts(tmem + colO, tmem + colS + kk * 8, sdesc_at(vd, kk * 2048), idesc_pv, 1u);
               if (j - 1 == U.end[i] - 1) {
                 umma_commit(o_full + i);
                 ++o_cnt[i];
@@ -255,12 +266,12 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
             }
             if (j >= U.beg[i] && j < U.end[i]) {
               // S_i = Q_i K_j^T
+              const SDesc qd = sdesc_sw128_split(qa + i * Cfg::kTileBytes, 16, 1024);
+              const SDesc kd = sdesc_sw128_split(ka + stK * Cfg::kTileBytes, 16, 1024);
 #pragma unroll
               for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t koff = (kk / 4) * Cfg::kBoxBytes + (kk % 4) * 32;
-                const uint64_t adesc = sdesc_sw128(qa + i * Cfg::kTileBytes + koff, 16, 1024);
-                const uint64_t bdesc = sdesc_sw128(ka + stK * Cfg::kTileBytes + koff, 16, 1024);
-                umma_ss(tmem + colS, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+                umma_ss(tmem + colS, sdesc_at(qd, koff), sdesc_at(kd, koff), idesc_qk, kk > 0 ? 1u : 0u);
               }
               umma_commit(s_full + i);
             }
@@ -279,9 +290,9 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       mbar_wait_drain(drain, 0);
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  } else {
     // ------------------------------------------------ softmax warpgroups --
-    const int i = (warp - 4) / 4;           // query tile handled by this warpgroup
+    const int i = (warp - 2) / 4;           // query tile handled by this warpgroup
     const int r = (warp % 4) * 32 + lane;   // row within the tile = TMEM lane
     const uint32_t lane_addr = tmem + ((uint32_t)((warp % 4) * 32) << 16);
     const uint32_t colS = i == 0 ? Cfg::kColS0 : Cfg::kColS1;
@@ -297,21 +308,32 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
         if (!ok) break;
         ++s_cnt;
         tc_fence_after();
-        uint32_t sr[kBN];
+        const bool diag = j == U.end[i] - 1;
+        // pass 1: row max, streaming S out of TMEM 64 columns at a time
+        float mt = -INFINITY;
 #pragma unroll
-        for (int cb = 0; cb < kBN / 32; ++cb) tmem_ld32p(lane_addr + colS + cb * 32, sr + cb * 32);
-        tmem_wait_ld();
-        float s[kBN];
+        for (int h = 0; h < kBN / 64; ++h) {
+          uint32_t sr[64];
+          tmem_ld32p(lane_addr + colS + h * 64, sr);
+          tmem_ld32p(lane_addr + colS + h * 64 + 32, sr + 32);
+          tmem_wait_ld();
+          if (diag) {
 #pragma unroll
-        for (int x = 0; x < kBN; ++x) s[x] = __uint_as_float(sr[x]);
-        if (j == U.end[i] - 1) {
+            for (int x = 0; x < 64; ++x)
+              if (h * 64 + x > r) sr[x] = __float_as_uint(-INFINITY);
+          }
+          float mp[8];
 #pragma unroll
-          for (int x = 0; x < kBN; ++x)
-            if (x > r) s[x] = -INFINITY;
+          for (int y = 0; y < 8; ++y)
+            mp[y] = fmax3(__uint_as_float(sr[y]), __uint_as_float(sr[y + 8]), __uint_as_float(sr[y + 16]));
+#pragma unroll
+          for (int x = 24; x + 16 < 64; x += 16)
+#pragma unroll
+            for (int y = 0; y < 8; ++y) mp[y] = fmax3(mp[y], __uint_as_float(sr[x + y]), __uint_as_float(sr[x + 8 + y]));
+#pragma unroll
+          for (int y = 0; y < 8; ++y) mp[y] = fmaxf(mp[y], __uint_as_float(sr[56 + y]));
+          mt = fmax3(mt, fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7])), -INFINITY);
         }
-        float mt = s[0];
-#pragma unroll
-        for (int x = 1; x < kBN; ++x) mt = fmaxf(mt, s[x]);
         const float m2 = mt * kLog2e;
         if (j == U.beg[i]) {
           m_ref = m2;
@@ -329,21 +351,55 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
             tmem_st32(lane_addr + colO + cb * 32, o);
           }
         }
-        float sum = 0.f;
+        // pass 2: p = 2^(s log2e - m_ref) in chunks of 32 columns (the next
+        // chunk's TMEM load is in flight while this one is computed).  The
+        // argument uses packed FMA; of every 8 pairs, kSfuPairs go to the SFU
+        // and the rest to the FMA pipe (exp2_poly2).  P (bf16) overwrites
+        // the already-consumed S columns.
+        const uint64_t l2e2 = pack2(kLog2e, kLog2e);
+        const uint64_t nm2 = pack2(-m_ref, -m_ref);
+        uint64_t acc2[2] = {pack2(0.f, 0.f), pack2(0.f, 0.f)};
+        uint32_t cur[32], nxt[32];
+        tmem_ld32p(lane_addr + colS, cur);
 #pragma unroll
         for (int cb = 0; cb < kBN / 32; ++cb) {
+          tmem_wait_ld();
+          if (cb + 1 < kBN / 32) tmem_ld32p(lane_addr + colS + (cb + 1) * 32, nxt);
+          if (diag) {
+#pragma unroll
+            for (int x = 0; x < 32; ++x)
+              if (cb * 32 + x > r) cur[x] = __float_as_uint(-INFINITY);
+          }
           uint32_t pk[16];
 #pragma unroll
           for (int x = 0; x < 16; ++x) {
-            const float p0 = ex2(fmaf(s[cb * 32 + 2 * x], kLog2e, -m_ref));
-            const float p1 = ex2(fmaf(s[cb * 32 + 2 * x + 1], kLog2e, -m_ref));
-            sum += p0 + p1;
+            const uint64_t a2 = ffma2(pack2(__uint_as_float(cur[2 * x]), __uint_as_float(cur[2 * x + 1])), l2e2, nm2);
+            uint64_t p2;
+            if (x % 8 < kSfuPairs) {
+              float a0, a1;
+              unpack2(a2, a0, a1);
+              p2 = pack2(ex2(a0), ex2(a1));
+            } else {
+              p2 = exp2_poly2(a2);
+            }
+            acc2[x & 1] = fadd2(acc2[x & 1], p2);
+            float p0, p1;
+            unpack2(p2, p0, p1);
             pk[x] = pack_bf16x2(p0, p1);
           }
           tmem_st16(lane_addr + colS + cb * 16, pk);
+          if (cb + 1 < kBN / 32) {
+#pragma unroll
+            for (int x = 0; x < 32; ++x) cur[x] = nxt[x];
+          }
         }
         tmem_wait_st();
-        l += sum;
+        {
+          float a0, a1, b0, b1;
+          unpack2(acc2[0], a0, a1);
+          unpack2(acc2[1], b0, b1);
+          l += (a0 + a1) + (b0 + b1);
+        }
         tc_fence_before();
         mbar_arrive(p_full + i);
       }
@@ -377,7 +433,7 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 2) tmem_dealloc(tmem, Cfg::kTmemCols);
+  if (warp == 1) tmem_dealloc(tmem, Cfg::kTmemCols);
 }
 
 // --------------------------------------------------------------- host --
