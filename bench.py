@@ -435,7 +435,8 @@ def summarize_launches(path: str) -> str:
     for r in rows[hi + 1:]:
         if len(r) <= vi or r[mi] != "gpu__time_duration.sum":
             continue
-        name = re.sub(r"\(.*", "", r[ki]).replace("void ", "").replace("gecko::(anonymous namespace)::", "")
+        name = re.sub(r"\(.*", "", r[ki]).replace("void ", "")
+        name = re.sub(r"gecko::(\(anonymous namespace\)|<unnamed>)::", "", name)
         a = agg.setdefault(name, [0, 0.0])
         a[0] += 1
         a[1] += float(r[vi].replace(",", "")) * scale[r[ui]]
