@@ -1,12 +1,17 @@
 // Adaptive Working Memory kernels on 5th-generation tensor cores (sm_100a).
 //
 // The AWM of the Gecko digest (paper.rainbus.top, core method and method
-// step details, steps 4-5) needs, per (b, h) and chunk s:
-//   Phi_s = exp(Km_s - log z^s)       (online-softmax kernel over time)
-//   Psi_s = rowsoftmax(Km_s)          (softmax over features)
-//   Bm_s  = Phi_s^T V_s,   Cm_s = Phi_s^T Psi_s        (d x d, fp32)
-// for the carry M'_{s+1} = r_s (.) M'_s - Cm_s M'_s + Bm_s, and the readout
-//   O_m,s = psi(Qm_s) M'_{s-1}.
+// step details, steps 4-5) needs, per (b, h) and chunk s, the online-softmax
+// kernel Phi_s = exp(Km_s - log z^s) and the feature softmax Psi_s.  Since
+// Phi_s = rho_s (.) Phi~_s with the chunk-local Phi~_s = exp(Km_s - lse_s)
+// (values in (0, 1], columns summing to 1) and rho_s = exp(lse_s - log z^s),
+// the chunk kernel computes
+//   Bm_s = Phi~_s^T V_s,   Cm_s = Phi~_s^T Psi_s        (d x d, fp32)
+// independently of the prefix over chunks, and the carry applies the row
+// scales: M'_{s+1} = r_s (.) M'_s + rho_s (.) (Bm_s - Cm_s M'_s).  The
+// readout is O_m,s = psi(Qm_s) M'_{s-1}.  Phi~, Psi and psi take their
+// exponentials in packed f16 (two per SFU op); they enter the tensor core as
+// bf16, whose 8-bit mantissa is coarser than f16's.
 //
 // awm_chunk_tc_kernel: one CTA per (chunk, bh).  The chunk is streamed in
 // tiles of 64 tokens.  V tiles arrive by TMA; 128 threads (two per token)
@@ -55,7 +60,7 @@ struct ChunkCfg {
 template <int D>
 __global__ void __launch_bounds__(192, 2) awm_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_v,
                                                            const __nv_bfloat16* __restrict__ km,
-                                                           const float* __restrict__ logz, float* __restrict__ Bm,
+                                                           const float* __restrict__ lse, float* __restrict__ Bm,
                                                            float* __restrict__ Cm, int T, int c, int* status) {
   using Cfg = ChunkCfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -65,7 +70,7 @@ __global__ void __launch_bounds__(192, 2) awm_chunk_tc_kernel(const __grid_const
   uint64_t* op_full = bars + 2;     // [2] compute -> MMA (128 arrivals)
   uint64_t* st_empty = bars + 4;    // [2] MMA -> TMA, compute
   uint64_t* acc_full = bars + 6;
-  float* lz2 = reinterpret_cast<float*>(smem + Cfg::kLzOff);
+  float* lz2 = reinterpret_cast<float*>(smem + Cfg::kLzOff);  // log2(e) * lse_s
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
 
@@ -85,7 +90,7 @@ __global__ void __launch_bounds__(192, 2) awm_chunk_tc_kernel(const __grid_const
     *abort_flag = 0;
     fence_mbar_init();
   }
-  for (int f = threadIdx.x; f < D; f += blockDim.x) lz2[f] = logz[(bh * S + s) * D + f] * kLog2e;
+  for (int f = threadIdx.x; f < D; f += blockDim.x) lz2[f] = lse[(bh * S + s) * D + f] * kLog2e;
   if (warp == 5) {
     tmem_alloc(tmem_slot, Cfg::kTmemCols);
     tmem_relinquish();
@@ -171,33 +176,37 @@ __global__ void __launch_bounds__(192, 2) awm_chunk_tc_kernel(const __grid_const
       for (int i = 1; i < HF; ++i) mx = fmaxf(mx, x[i]);
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
       const float mx2 = mx * kLog2e;
-      float e[HF], sum = 0.f;
-#pragma unroll
-      for (int i = 0; i < HF; ++i) {
-        e[i] = ex2(fmaf(x[i], kLog2e, -mx2));
-        sum += e[i];
-      }
-      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-      const float inv = 1.f / sum;
       // wait until the MMAs of tile kt-2 have released this stage
       ok = __all_sync(0xffffffffu, mbar_wait(st_empty + st, ((kt >> 1) & 1) ^ 1, abort_flag, status));
       if (!ok) break;
       uint8_t* stg = smem + st * Cfg::kStage;
+      float e[HF], sum = 0.f;
 #pragma unroll
       for (int i = 0; i < HF / 8; ++i) {
         const int col = h * HF + 8 * i;
-        uint4 ps, ph;
-        uint32_t* pp = reinterpret_cast<uint32_t*>(&ps);
-        uint32_t* pf = reinterpret_cast<uint32_t*>(&ph);
+        uint4 pf;
+        uint32_t* qq = reinterpret_cast<uint32_t*>(&pf);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          pp[j] = pack_bf16x2(e[8 * i + 2 * j] * inv, e[8 * i + 2 * j + 1] * inv);
-          pf[j] = pack_bf16x2(ex2(fmaf(x[8 * i + 2 * j], kLog2e, -lz2[col + 2 * j])),
-                              ex2(fmaf(x[8 * i + 2 * j + 1], kLog2e, -lz2[col + 2 * j + 1])));
+          const int a = 8 * i + 2 * j;
+          float p0, p1;
+          ex2_h2(fmaf(x[a], kLog2e, -lz2[col + 2 * j]), fmaf(x[a + 1], kLog2e, -lz2[col + 2 * j + 1]), p0, p1);
+          qq[j] = pack_bf16x2(p0, p1);
+          ex2_h2(fmaf(x[a], kLog2e, -mx2), fmaf(x[a + 1], kLog2e, -mx2), e[a], e[a + 1]);
+          sum += e[a] + e[a + 1];
         }
-        const uint32_t off = sw128_off(r, col, kKT);
-        *reinterpret_cast<uint4*>(stg + Cfg::kOperand + off) = ps;
-        *reinterpret_cast<uint4*>(stg + 2 * Cfg::kOperand + off) = ph;
+        *reinterpret_cast<uint4*>(stg + 2 * Cfg::kOperand + sw128_off(r, col, kKT)) = pf;
+      }
+      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+      const float inv = 1.f / sum;
+#pragma unroll
+      for (int i = 0; i < HF / 8; ++i) {
+        const int col = h * HF + 8 * i;
+        uint4 ps;
+        uint32_t* pp = reinterpret_cast<uint32_t*>(&ps);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) pp[j] = pack_bf16x2(e[8 * i + 2 * j] * inv, e[8 * i + 2 * j + 1] * inv);
+        *reinterpret_cast<uint4*>(stg + Cfg::kOperand + sw128_off(r, col, kKT)) = ps;
       }
       // generic-proxy writes must be visible to the tensor core (async proxy)
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -252,8 +261,13 @@ struct ReadoutCfg {
   static constexpr uint32_t kTmemCols = 2 * D;   // two accumulators
 };
 
-// 128 threads: one row each; thread 0 also issues the MMAs.  Tiles of the
-// chunk are processed two at a time (double-buffered A and accumulators).
+// 128 threads: one row each; thread 0 also issues the MMAs.  grid
+// (S, BH, G): CTA g of a chunk takes its 128-row tiles g, g + G, ...  The A
+// operand holds the unnormalised numerators exp(q - max) of each row (bf16,
+// via packed f16 exponentials); the epilogue scales row t by 1 / sum_t.  The
+// next tile's Q_m rows are loaded while the current one is processed; A and
+// the accumulator are double-buffered so a tile's MMA overlaps the next
+// tile's exponentials.
 template <int D>
 __global__ void __launch_bounds__(128) awm_readout_tc_kernel(const __nv_bfloat16* __restrict__ qm,
                                                              const float* __restrict__ Mst,
@@ -269,19 +283,23 @@ __global__ void __launch_bounds__(128) awm_readout_tc_kernel(const __nv_bfloat16
 
   const int s = blockIdx.x, S = gridDim.x;
   const int64_t bh = blockIdx.y;
-  const int warp = warp_id_uniform(), lane = threadIdx.x % 32;
+  const int g = blockIdx.z, G = gridDim.z;
+  const int warp = warp_id_uniform();
   const int r = threadIdx.x;
   const int n_tiles = c / 128;
+  const int m = n_tiles > g ? (n_tiles - g + G - 1) / G : 0;  // tiles of this CTA
   const int64_t row0 = bh * (int64_t)T + (int64_t)s * c;
 
   if (s < 2) {
     // chunks 1 and 2 read M'_0 = M'_1 = 0
     const uint4 z = make_uint4(0, 0, 0, 0);
-    uint4* dst = reinterpret_cast<uint4*>(out + row0 * D);
-    const int64_t n = (int64_t)c * D / 8;
-    for (int64_t i = threadIdx.x; i < n; i += blockDim.x) dst[i] = z;
+    for (int idx = 0; idx < m; ++idx) {
+      uint4* dst = reinterpret_cast<uint4*>(out + (row0 + (int64_t)(g + idx * G) * 128) * D);
+      for (int i = threadIdx.x; i < 128 * D / 8; i += blockDim.x) dst[i] = z;
+    }
     return;
   }
+  if (m == 0) return;
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(acc_full + i, 1);
@@ -316,61 +334,10 @@ __global__ void __launch_bounds__(128) awm_readout_tc_kernel(const __nv_bfloat16
   const uint32_t base = smem_u32(smem);
   constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, true);
   const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+  const SDesc bdesc = sdesc_sw128_split(base + Cfg::kBOff, D * 128, 1024);
   bool ok = true;
 
-  auto psi_tile = [&](int kt, int buf) {
-    const uint4* src = reinterpret_cast<const uint4*>(qm + (row0 + (int64_t)kt * 128 + r) * D);
-    float x[D];
-#pragma unroll
-    for (int i = 0; i < D / 8; ++i) {
-      const uint4 u = src[i];
-      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f2 = __bfloat1622float2(p2[j]);
-        x[8 * i + 2 * j] = f2.x;
-        x[8 * i + 2 * j + 1] = f2.y;
-      }
-    }
-    float mx = x[0];
-#pragma unroll
-    for (int i = 1; i < D; ++i) mx = fmaxf(mx, x[i]);
-    const float mx2 = mx * kLog2e;
-    float sum = 0.f;
-#pragma unroll
-    for (int i = 0; i < D; ++i) {
-      x[i] = ex2(fmaf(x[i], kLog2e, -mx2));
-      sum += x[i];
-    }
-    const float inv = 1.f / sum;
-    uint8_t* a = smem + Cfg::kAOff + buf * Cfg::kA;
-#pragma unroll
-    for (int i = 0; i < D / 8; ++i) {
-      uint4 p;
-      p.x = pack_bf16x2(x[8 * i] * inv, x[8 * i + 1] * inv);
-      p.y = pack_bf16x2(x[8 * i + 2] * inv, x[8 * i + 3] * inv);
-      p.z = pack_bf16x2(x[8 * i + 4] * inv, x[8 * i + 5] * inv);
-      p.w = pack_bf16x2(x[8 * i + 6] * inv, x[8 * i + 7] * inv);
-      *reinterpret_cast<uint4*>(a + sw128_off(r, 8 * i, 128)) = p;
-    }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (threadIdx.x == 0) {
-      const uint32_t aa = base + Cfg::kAOff + buf * Cfg::kA;
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t koff = (kk / 4) * (128 * 128) + (kk % 4) * 32;
-        const uint64_t adesc = sdesc_sw128(aa + koff, 16, 1024);
-        const uint64_t bdesc = sdesc_sw128(base + Cfg::kBOff + kk * 16 * 128, D * 128, 1024);
-        umma_ss(tmem + buf * D, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
-      }
-      umma_commit(acc_full + buf);
-    }
-  };
-
-  auto store_tile = [&](int kt, int buf, uint32_t parity) -> bool {
+  auto store_tile = [&](int kt, int buf, uint32_t parity, float inv) -> bool {
     if (!__all_sync(0xffffffffu, mbar_wait(acc_full + buf, parity, abort_flag, status))) return false;
     tc_fence_after();
     __nv_bfloat16* orow = out + (row0 + (int64_t)kt * 128 + r) * D;
@@ -382,7 +349,8 @@ __global__ void __launch_bounds__(128) awm_readout_tc_kernel(const __nv_bfloat16
       uint4 w[4];
       uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) wp[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+      for (int i = 0; i < 16; ++i)
+        wp[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * inv, __uint_as_float(v[2 * i + 1]) * inv);
       uint4* dst = reinterpret_cast<uint4*>(orow + cb * 32);
 #pragma unroll
       for (int i = 0; i < 4; ++i) dst[i] = w[i];
@@ -391,16 +359,70 @@ __global__ void __launch_bounds__(128) awm_readout_tc_kernel(const __nv_bfloat16
     return true;
   };
 
-  // software pipeline: psi of tile kt overlaps the MMA of tile kt-1; the
-  // epilogue of tile kt-1 runs once its accumulator is ready.
-  for (int kt = 0; kt < n_tiles && ok; ++kt) {
-    const int buf = kt & 1;
-    psi_tile(kt, buf);
-    if (kt > 0) ok = store_tile(kt - 1, buf ^ 1, ((kt - 1) >> 1) & 1);
-    // the next psi_tile(kt+1) writes A buffer buf^1 and accumulator buf^1;
-    // both were released by store_tile(kt-1) above (its MMA completed)
+  uint4 cur[D / 8], nxt[D / 8];
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(qm + (row0 + (int64_t)g * 128 + r) * D);
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) cur[i] = src[i];
   }
-  if (ok) ok = store_tile(n_tiles - 1, (n_tiles - 1) & 1, ((n_tiles - 1) >> 1) & 1);
+  float inv_prev = 0.f;
+  for (int idx = 0; idx < m && ok; ++idx) {
+    const int kt = g + idx * G, buf = idx & 1;
+    if (idx + 1 < m) {
+      const uint4* src = reinterpret_cast<const uint4*>(qm + (row0 + (int64_t)(kt + G) * 128 + r) * D);
+#pragma unroll
+      for (int i = 0; i < D / 8; ++i) nxt[i] = src[i];
+    }
+    // psi numerators exp(q - max) of row r -> A[buf] (K-major, swizzled)
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) {
+      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&cur[i]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f2 = __bfloat1622float2(p2[j]);
+        mx = fmax3(mx, f2.x, f2.y);
+      }
+    }
+    const float mx2 = mx * kLog2e;
+    float sum = 0.f;
+    uint8_t* a = smem + Cfg::kAOff + buf * Cfg::kA;
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) {
+      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&cur[i]);
+      uint4 p;
+      uint32_t* pp = reinterpret_cast<uint32_t*>(&p);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f2 = __bfloat1622float2(p2[j]);
+        float e0, e1;
+        ex2_h2(fmaf(f2.x, kLog2e, -mx2), fmaf(f2.y, kLog2e, -mx2), e0, e1);
+        sum += e0 + e1;
+        pp[j] = pack_bf16x2(e0, e1);
+      }
+      *reinterpret_cast<uint4*>(a + sw128_off(r, 8 * i, 128)) = p;
+    }
+    const float inv = 1.f / sum;
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (threadIdx.x == 0) {
+      const SDesc ad = sdesc_sw128_split(base + Cfg::kAOff + buf * Cfg::kA, 16, 1024);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t koff = (kk / 4) * (128 * 128) + (kk % 4) * 32;
+        umma_ss(tmem + buf * D, sdesc_at(ad, koff), sdesc_at(bdesc, kk * 16 * 128), idesc, kk > 0 ? 1u : 0u);
+      }
+      umma_commit(acc_full + buf);
+    }
+    // epilogue of the previous tile overlaps this tile's MMA
+    if (idx > 0) ok = store_tile(kt - G, buf ^ 1, ((idx - 1) >> 1) & 1, inv_prev);
+    inv_prev = inv;
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) cur[i] = nxt[i];
+  }
+  if (ok) ok = store_tile(g + (m - 1) * G, (m - 1) & 1, ((m - 1) >> 1) & 1, inv_prev);
   if (!ok && threadIdx.x == 0) {
     // make sure no MMA is still writing TMEM before it is released
     umma_commit(a_full);
@@ -448,7 +470,7 @@ cudaError_t chunk_impl(const Problem& p, const Workspace& w, cudaStream_t st) {
                                        Cfg::kAlloc);
   if (e != cudaSuccess) return e;
   awm_chunk_tc_kernel<D><<<dim3(p.S, p.B * p.H), 192, Cfg::kAlloc, st>>>(
-      mv, static_cast<const __nv_bfloat16*>(p.km), w.logz, w.Bm, w.Cm, (int)p.T, (int)p.c, p.status);
+      mv, static_cast<const __nv_bfloat16*>(p.km), w.lse, w.Bm, w.Cm, (int)p.T, (int)p.c, p.status);
   return cudaGetLastError();
 }
 
@@ -458,7 +480,10 @@ cudaError_t readout_impl(const Problem& p, const Workspace& w, cudaStream_t st) 
   cudaError_t e = cudaFuncSetAttribute(awm_readout_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Cfg::kAlloc);
   if (e != cudaSuccess) return e;
-  awm_readout_tc_kernel<D><<<dim3(p.S, p.B * p.H), 128, Cfg::kAlloc, st>>>(
+  // split each chunk's 128-row tiles over G CTAs (up to 8 tiles per CTA)
+  const int n_tiles = (int)(p.c / 128);
+  const int G = n_tiles > 8 ? (n_tiles + 7) / 8 : 1;
+  awm_readout_tc_kernel<D><<<dim3(p.S, p.B * p.H, G), 128, Cfg::kAlloc, st>>>(
       static_cast<const __nv_bfloat16*>(p.qm), w.Mst, static_cast<__nv_bfloat16*>(p.out_mem), (int)p.T,
       (int)p.c, p.status);
   return cudaGetLastError();

@@ -6,6 +6,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 namespace gecko {
@@ -35,6 +36,19 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 constexpr float kLog2e = 1.4426950408889634f;
+
+// 2^a and 2^b through one packed half-precision SFU op (ex2.approx.f16x2).
+// For arguments <= 0 whose results only feed bf16 operands: the f16 result
+// keeps more mantissa than bf16; results below 2^-24 flush to 0.
+__device__ __forceinline__ void ex2_h2(float a, float b, float& ea, float& eb) {
+  uint32_t h, r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(b), "f"(a));  // a in the low half
+  asm("ex2.approx.f16x2 %0, %1;" : "=r"(r) : "r"(h));
+  __half2 hh = *reinterpret_cast<__half2*>(&r);
+  const float2 f = __half22float2(hh);
+  ea = f.x;
+  eb = f.y;
+}
 
 // ------------------------------------------------ packed fp32 pairs (sm_100) --
 

@@ -33,7 +33,7 @@ size_t workspace_bytes(int64_t BH, int64_t T, int64_t c, int64_t d) {
   const size_t vec = al(sizeof(float) * BH * S * d);
   const size_t mat = al(sizeof(float) * BH * S * d * d);
   const size_t mst = al(sizeof(float) * BH * (S + 1) * d * d);
-  return part + 3 * vec + 2 * mat + mst;
+  return part + 4 * vec + 2 * mat + mst;
 }
 
 Workspace carve_workspace(void* base, int64_t BH, int64_t T, int64_t c, int64_t d) {
@@ -51,6 +51,8 @@ Workspace carve_workspace(void* base, int64_t BH, int64_t T, int64_t c, int64_t 
   w.logz = reinterpret_cast<float*>(p);
   p += vec;
   w.ratio = reinterpret_cast<float*>(p);
+  p += vec;
+  w.rho = reinterpret_cast<float*>(p);
   p += vec;
   w.Bm = reinterpret_cast<float*>(p);
   p += mat;

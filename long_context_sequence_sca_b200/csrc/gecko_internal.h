@@ -26,13 +26,14 @@ struct Workspace {
   float* lse;    // [BH, S, d]  log of per-chunk exp-sums of K_m
   float* logz;   // [BH, S, d]  log z^s
   float* ratio;  // [BH, S, d]  z^{s-1} / z^s  (0 for s = 1)
-  float* Bm;     // [BH, S, d, d]  Phi_s^T V_s
-  float* Cm;     // [BH, S, d, d]  Phi_s^T Psi_s
+  float* rho;    // [BH, S, d]  e_s / z^s = exp(lse_s - log z^s)
+  float* Bm;     // [BH, S, d, d]  Phi~_s^T V_s    (Phi~_s = exp(Km_s - lse_s))
+  float* Cm;     // [BH, S, d, d]  Phi~_s^T Psi_s
   float* Mst;    // [BH, S+1, d, d]  M'_1 .. M'_{S+1}
 };
 
 // Rows per block of the partial K_m statistics (divides c).
-inline int stats_block_rows(int64_t c) { return c % 256 == 0 ? 256 : 64; }
+inline int stats_block_rows(int64_t c) { return c % 128 == 0 ? 128 : 64; }
 
 // Bytes needed by a Workspace, each region 256-byte aligned.
 size_t workspace_bytes(int64_t BH, int64_t T, int64_t c, int64_t d);

@@ -38,30 +38,33 @@ template <> struct Vec8<float> {
 // ------------------------------------------------------------------------
 // Partial statistics of K_m per block of R rows: for each feature f the
 // block max m and sum_i exp(km[i, f] - m).  grid (T / R, BH), 256 threads;
-// each thread keeps a running (max, sum) for 8 features over a strided row
-// set, then the row groups are merged in shared memory.
-template <typename TIn, int D>
+// each thread holds 8 features of R / RG rows in registers, takes their max
+// and then their exp-sum (one SFU exp2 per element), then the row groups are
+// merged in shared memory.
+template <typename TIn, int D, int R>
 __global__ void __launch_bounds__(256) awm_lse_partial_kernel(const TIn* __restrict__ km, float2* __restrict__ part,
-                                                              int64_t T, int R) {
+                                                              int64_t T) {
   constexpr int TPR = D / 8;          // threads per row
   constexpr int RG = 256 / TPR;       // rows processed in parallel
+  constexpr int NR = R / RG;          // rows per thread
   const int blk = blockIdx.x, nblk = gridDim.x;
   const int64_t bh = blockIdx.y;
   const int lane8 = threadIdx.x % TPR;
   const int rg = threadIdx.x / TPR;
   const TIn* base = km + (bh * T + (int64_t)blk * R) * D + lane8 * 8;
+  float x[NR][8];
+#pragma unroll
+  for (int n = 0; n < NR; ++n) Vec8<TIn>::load(base + (int64_t)(rg + n * RG) * D, x[n]);
   float m[8], acc[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) { m[i] = -INFINITY; acc[i] = 0.f; }
-  for (int r = rg; r < R; r += RG) {
-    float x[8];
-    Vec8<TIn>::load(base + (int64_t)r * D, x);
+  for (int i = 0; i < 8; ++i) {
+    m[i] = x[0][i];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float mn = fmaxf(m[i], x[i]);
-      acc[i] = acc[i] * expf(m[i] - mn) + expf(x[i] - mn);
-      m[i] = mn;
-    }
+    for (int n = 1; n < NR; ++n) m[i] = fmaxf(m[i], x[n][i]);
+    const float m2 = m[i] * kLog2e;
+    acc[i] = 0.f;
+#pragma unroll
+    for (int n = 0; n < NR; ++n) acc[i] += ex2(fmaf(x[n][i], kLog2e, -m2));
   }
   __shared__ float sm[RG][D + 1];
   __shared__ float ss[RG][D + 1];
@@ -75,8 +78,7 @@ __global__ void __launch_bounds__(256) awm_lse_partial_kernel(const TIn* __restr
     float M = -INFINITY;
     for (int g = 0; g < RG; ++g) M = fmaxf(M, sm[g][f]);
     float tot = 0.f;
-    for (int g = 0; g < RG; ++g)
-      if (sm[g][f] > -INFINITY) tot += ss[g][f] * expf(sm[g][f] - M);
+    for (int g = 0; g < RG; ++g) tot += ss[g][f] * expf(sm[g][f] - M);
     part[(bh * nblk + blk) * D + f] = make_float2(M, tot);
   }
 }
@@ -101,11 +103,12 @@ __global__ void __launch_bounds__(D) awm_lse_combine_kernel(const float2* __rest
 }
 
 // ------------------------------------------------------------------------
-// Prefix over chunks in fp64: log z^s = logaddexp(log z^{s-1}, lse_s), and
-// the row ratio z^{s-1}/z^s (0 for s = 1).  grid BH, D threads.
+// Prefix over chunks in fp64: log z^s = logaddexp(log z^{s-1}, lse_s), the
+// row ratio r_s = z^{s-1}/z^s (0 for s = 1) and the chunk weight
+// rho_s = e_s / z^s = exp(lse_s - log z^s).  grid BH, D threads.
 template <int D>
 __global__ void __launch_bounds__(D) awm_prefix_kernel(const float* __restrict__ lse, float* __restrict__ logz,
-                                                       float* __restrict__ ratio, int S) {
+                                                       float* __restrict__ ratio, float* __restrict__ rho, int S) {
   const int64_t bh = blockIdx.x;
   const int f = threadIdx.x;
   double L = 0.0;
@@ -121,19 +124,23 @@ __global__ void __launch_bounds__(D) awm_prefix_kernel(const float* __restrict__
     }
     logz[o] = (float)Ln;
     ratio[o] = s == 0 ? 0.f : (float)exp(L - Ln);
+    rho[o] = (float)exp(e - Ln);
     L = Ln;
   }
 }
 
 // ------------------------------------------------------------------------
 // Per-chunk GEMMs of the AWM update, in fp32:
-//   Bm_s = Phi_s^T V_s,   Cm_s = Phi_s^T Psi_s         (D x D each)
-// with Phi_s = exp(Km_s - log z^s) and Psi_s = rowsoftmax(Km_s).
+//   Bm_s = Phi~_s^T V_s,   Cm_s = Phi~_s^T Psi_s       (D x D each)
+// with the chunk-local kernel Phi~_s = exp(Km_s - lse_s) (columns sum to 1)
+// and Psi_s = rowsoftmax(Km_s).  The online-softmax kernel of the update is
+// Phi_s = rho_s (.) Phi~_s with rho_s = exp(lse_s - log z^s); the carry
+// applies rho_s to the rows of Bm_s and Cm_s.
 // grid (S, BH), 256 threads as a 16 x 16 grid of (D/16) x (D/16) tiles.
 template <typename TIn, int D>
 __global__ void __launch_bounds__(256) awm_chunk_simt_kernel(const TIn* __restrict__ km,
                                                              const TIn* __restrict__ v,
-                                                             const float* __restrict__ logz,
+                                                             const float* __restrict__ lse,
                                                              float* __restrict__ Bm, float* __restrict__ Cm,
                                                              int64_t T, int c) {
   constexpr int RT = 16;       // token rows per step
@@ -146,7 +153,7 @@ __global__ void __launch_bounds__(256) awm_chunk_simt_kernel(const TIn* __restri
   __shared__ float v_s[RT][D];
   __shared__ float lz[D];
   const int tid = threadIdx.x;
-  for (int f = tid; f < D; f += 256) lz[f] = logz[(bh * S + s) * D + f];
+  for (int f = tid; f < D; f += 256) lz[f] = lse[(bh * S + s) * D + f];
   const int ty = tid / 16, tx = tid % 16;
   float accB[TM][TM], accC[TM][TM];
 #pragma unroll
@@ -216,19 +223,22 @@ __global__ void __launch_bounds__(256) awm_chunk_simt_kernel(const TIn* __restri
 // ------------------------------------------------------------------------
 // The sequential carry, one slice of JC value columns per CTA (columns of M'
 // evolve independently):
-//   M'_{s+1}[:, J] = r_s (.) M'_s[:, J] - Cm_s M'_s[:, J] + Bm_s[:, J]
-// Writes Mst[bh, s] = M'_{s+1} for s = 0..S (M'_1 = 0 first).
-// grid (D / JC, BH), 256 threads.
+//   M'_{s+1}[:, J] = r_s (.) M'_s[:, J] + rho_s (.) (Bm_s[:, J] - Cm_s M'_s[:, J])
+// (row scales r_s = z^{s-1}/z^s and rho_s = e_s/z^s).  Writes
+// Mst[bh, s] = M'_{s+1} for s = 0..S (M'_1 = 0 first).  Cm_s is staged into
+// shared memory with 16-byte loads.  grid (D / JC, BH), 256 threads.
 template <int D, int JC>
 __global__ void __launch_bounds__(256) awm_carry_kernel(const float* __restrict__ Bm,
                                                         const float* __restrict__ Cm,
                                                         const float* __restrict__ ratio,
+                                                        const float* __restrict__ rho,
                                                         float* __restrict__ Mst, int S) {
   constexpr int PER = D * JC / 256;  // outputs per thread (one row f, PER columns)
   static_assert(256 / (JC / PER) == D, "thread layout");
+  constexpr int LD = D + 4;          // padded row of Cm in shared memory (keeps 16-byte alignment)
   extern __shared__ float smem_carry[];
-  float* Cs = smem_carry;               // [D][D + 1]
-  float* Ms = Cs + D * (D + 1);         // [D][JC]
+  float* Cs = smem_carry;            // [D][LD]
+  float* Ms = Cs + D * LD;           // [D][JC]
   const int64_t bh = blockIdx.y;
   const int j0 = blockIdx.x * JC;
   const int tid = threadIdx.x;
@@ -240,20 +250,27 @@ __global__ void __launch_bounds__(256) awm_carry_kernel(const float* __restrict_
 #pragma unroll
   for (int j = 0; j < PER; ++j) mout[f * D + j0 + jj + j] = 0.f;   // M'_1 = 0
   for (int s = 0; s < S; ++s) {
-    const float* C = Cm + (bh * S + s) * mst_stride;
+    const float4* C4 = reinterpret_cast<const float4*>(Cm + (bh * S + s) * mst_stride);
     __syncthreads();
-    for (int i = tid; i < D * D; i += 256) Cs[(i / D) * (D + 1) + (i % D)] = C[i];
+    for (int i = tid; i < D * D / 4; i += 256) {
+      const int row = (i * 4) / D, col = (i * 4) % D;
+      *reinterpret_cast<float4*>(Cs + row * LD + col) = C4[i];
+    }
     __syncthreads();
     const float rf = ratio[(bh * S + s) * D + f];
+    const float pf = rho[(bh * S + s) * D + f];
     const float* Bp = Bm + (bh * S + s) * mst_stride + f * D + j0 + jj;
     float acc[PER];
 #pragma unroll
-    for (int j = 0; j < PER; ++j) acc[j] = rf * Ms[f * JC + jj + j] + Bp[j];
+    for (int j = 0; j < PER; ++j) acc[j] = Bp[j];
+#pragma unroll 4
     for (int g = 0; g < D; ++g) {
-      const float cfg = Cs[f * (D + 1) + g];
+      const float cfg = Cs[f * LD + g];
 #pragma unroll
       for (int j = 0; j < PER; ++j) acc[j] = fmaf(-cfg, Ms[g * JC + jj + j], acc[j]);
     }
+#pragma unroll
+    for (int j = 0; j < PER; ++j) acc[j] = fmaf(rf, Ms[f * JC + jj + j], pf * acc[j]);
     __syncthreads();
 #pragma unroll
     for (int j = 0; j < PER; ++j) {
@@ -389,27 +406,30 @@ cudaError_t awm_stats_impl(const Problem& p, const Workspace& w, cudaStream_t st
   const int64_t BH = p.B * p.H;
   const int R = stats_block_rows(p.c);
   const int P = (int)(p.c / R);
-  awm_lse_partial_kernel<TIn, D><<<dim3((unsigned)(p.T / R), BH), 256, 0, st>>>(static_cast<const TIn*>(p.km),
-                                                                                 w.part, p.T, R);
+  const dim3 grid((unsigned)(p.T / R), BH);
+  if (R == 128)
+    awm_lse_partial_kernel<TIn, D, 128><<<grid, 256, 0, st>>>(static_cast<const TIn*>(p.km), w.part, p.T);
+  else
+    awm_lse_partial_kernel<TIn, D, 64><<<grid, 256, 0, st>>>(static_cast<const TIn*>(p.km), w.part, p.T);
   awm_lse_combine_kernel<D><<<dim3(p.S, BH), D, 0, st>>>(w.part, w.lse, P);
-  awm_prefix_kernel<D><<<BH, D, 0, st>>>(w.lse, w.logz, w.ratio, p.S);
+  awm_prefix_kernel<D><<<BH, D, 0, st>>>(w.lse, w.logz, w.ratio, w.rho, p.S);
   return cudaGetLastError();
 }
 
 template <typename TIn, int D>
 cudaError_t awm_chunk_simt_impl(const Problem& p, const Workspace& w, cudaStream_t st) {
   awm_chunk_simt_kernel<TIn, D><<<dim3(p.S, p.B * p.H), 256, 0, st>>>(
-      static_cast<const TIn*>(p.km), static_cast<const TIn*>(p.v), w.logz, w.Bm, w.Cm, p.T, (int)p.c);
+      static_cast<const TIn*>(p.km), static_cast<const TIn*>(p.v), w.lse, w.Bm, w.Cm, p.T, (int)p.c);
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t awm_carry_impl(const Problem& p, const Workspace& w, cudaStream_t st) {
   constexpr int JC = 16;
-  const size_t smem = sizeof(float) * (D * (D + 1) + D * JC);
+  const size_t smem = sizeof(float) * (D * (D + 4) + D * JC);
   cudaError_t e = cudaFuncSetAttribute(awm_carry_kernel<D, JC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  awm_carry_kernel<D, JC><<<dim3(D / JC, p.B * p.H), 256, smem, st>>>(w.Bm, w.Cm, w.ratio, w.Mst, p.S);
+  awm_carry_kernel<D, JC><<<dim3(D / JC, p.B * p.H), 256, smem, st>>>(w.Bm, w.Cm, w.ratio, w.rho, w.Mst, p.S);
   return cudaGetLastError();
 }
 
