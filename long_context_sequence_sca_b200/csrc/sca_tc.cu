@@ -48,6 +48,11 @@ constexpr int kThreads = 320;   // 10 warps: TMA, MMA (+TMEM allocation), 2 x 4 
 #ifndef GECKO_SFU_PAIRS
 #define GECKO_SFU_PAIRS 8
 #endif
+// GECKO_SCA_H2EXP = 1 evaluates the softmax exponentials as packed f16 pairs
+// (ex2.approx.f16x2, two per SFU op) instead of fp32 SFU ops.
+#ifndef GECKO_SCA_H2EXP
+#define GECKO_SCA_H2EXP 0
+#endif
 constexpr int kSfuPairs = GECKO_SFU_PAIRS;
 
 template <int D>
@@ -59,9 +64,9 @@ struct ScaCfg {
   static constexpr int kKOff = kQOff + 2 * kTileBytes;
   static constexpr int kVOff = kKOff + kStages * kTileBytes;
   static constexpr int kBarOff = kVOff + kStages * kTileBytes;
-  // q_full, q_empty, k_full[S], k_empty[S], v_full[S], v_empty[S],
-  // s_full[2], p_full[2], o_full[2], o_empty[2], drain
-  static constexpr int kNumBars = 2 + 4 * kStages + 8 + 1;
+  // q_full, q_empty, k_full[S], kv_done[S], v_full[S], (unused)[S],
+  // s_full[2], p_full[2], o_full[2], o_empty[2], drain, seq[2]
+  static constexpr int kNumBars = 2 + 4 * kStages + 8 + 1 + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;         // slack for 1024-byte alignment
@@ -77,26 +82,36 @@ struct Unit {
   int end[2];    // one past the last (= diagonal tile + 1)
 };
 
-// Map a linear unit index to (bh, pair).  When c % 256 == 0 the order puts
-// the most expensive pairs first (later chunks, larger in-chunk offsets) so
-// the static round-robin over CTAs approximates longest-first scheduling.
+// Map a linear unit index to (bh, pair).  When c % 256 == 0 the units are
+// grouped by (bh, chunk): the c / 256 units of one group read the same K/V
+// window (previous + current chunk), so running them next to each other
+// keeps that window in L2 while the group is in flight (ordering the whole
+// grid by cost instead puts ~148 different windows in flight, far more than
+// L2 holds, and every K/V tile then comes from DRAM).  Inside a group the
+// units go from the most to the least expensive; groups of later chunks
+// come first and the cheap chunk-1 groups last, which keeps the tail short.
 __device__ __forceinline__ Unit decode_unit(int u, int BH, int T, int c) {
   const int pairs = (T + 255) / 256;
-  const int w = u / BH;
   Unit U;
-  U.bh = u % BH;
-  int pair = w;
+  int pair;
   if (c % 256 == 0) {
     const int npc = c / 256;
     const int S = T / c;
-    const int nA = (S - 1) * npc;
-    if (w < nA) {
-      const int o = npc - 1 - w / (S - 1);
-      const int ch = 1 + w % (S - 1);
-      pair = ch * npc + o;
+    const int g = u / npc;
+    const int o = npc - 1 - u % npc;
+    const int n_main = (S - 1) * BH;
+    int ch;
+    if (g < n_main) {
+      ch = S - 1 - g / BH;
+      U.bh = g % BH;
     } else {
-      pair = npc - 1 - (w - nA);
+      ch = 0;
+      U.bh = g - n_main;
     }
+    pair = ch * npc + o;
+  } else {
+    pair = u / BH;
+    U.bh = u % BH;
   }
   (void)pairs;
   U.q0 = pair * 256;
@@ -129,14 +144,16 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
   uint64_t* k_full = bars + 2;
-  uint64_t* k_empty = k_full + KST;
-  uint64_t* v_full = k_empty + KST;
-  uint64_t* v_empty = v_full + KST;
-  uint64_t* s_full = v_empty + KST;
+  // kv_done[m % KST] completes when the MMAs of K/V iteration m are done:
+  // they were the last readers of K_m and of V_{m-1}
+  uint64_t* kv_done = k_full + KST;
+  uint64_t* v_full = kv_done + KST;
+  uint64_t* s_full = v_full + 2 * KST;
   uint64_t* p_full = s_full + 2;
   uint64_t* o_full = p_full + 2;
   uint64_t* o_empty = o_full + 2;
   uint64_t* drain = o_empty + 2;
+  uint64_t* seq = drain + 1;       // [2] exp-pass tokens between the softmax warpgroups
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
 
@@ -148,9 +165,8 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
     mbar_init(q_empty, 1);
     for (int s = 0; s < KST; ++s) {
       mbar_init(k_full + s, 1);
-      mbar_init(k_empty + s, 1);
+      mbar_init(kv_done + s, 1);
       mbar_init(v_full + s, 1);
-      mbar_init(v_empty + s, 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + i, 1);
@@ -159,6 +175,8 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       mbar_init(o_empty + i, 128);
     }
     mbar_init(drain, 1);
+    mbar_init(seq, 4);             // one arrival per warp of the other warpgroup
+    mbar_init(seq + 1, 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -195,13 +213,19 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
         const int jb = U.beg[0], je = U.nt == 2 ? U.end[1] : U.end[0];
         for (int j = jb; j < je; ++j, ++kv_it) {
           const int st = kv_it % KST;
-          const uint32_t ph = (kv_it / KST) & 1;
           const int row = (int)(rowbase + (int64_t)j * kBN);
-          if (!(ok = mbar_wait(k_empty + st, ph ^ 1, abort_flag, status))) break;
+          // slot of K_n was last read by iteration n - KST
+          if (kv_it >= (uint32_t)KST &&
+              !(ok = mbar_wait(kv_done + st, ((kv_it - KST) / KST) & 1, abort_flag, status)))
+            break;
           mbar_arrive_expect_tx(k_full + st, Cfg::kTileBytes);
           for (int b = 0; b < D / 64; ++b)
             tma_load_2d(sK + st * Cfg::kTileBytes + b * Cfg::kBoxBytes, &map_k, k_full + st, b * 64, row);
-          if (!(ok = mbar_wait(v_empty + st, ph ^ 1, abort_flag, status))) { ++kv_it; break; }
+          // slot of V_n was last read by iteration n - KST + 1 (PV of V_{n-KST})
+          if (kv_it + 1 >= (uint32_t)KST) {
+            const uint32_t m = kv_it + 1 - KST;
+            if (!(ok = mbar_wait(kv_done + m % KST, (m / KST) & 1, abort_flag, status))) { ++kv_it; break; }
+          }
           mbar_arrive_expect_tx(v_full + st, Cfg::kTileBytes);
           for (int b = 0; b < D / 64; ++b)
             tma_load_2d(sV + st * Cfg::kTileBytes + b * Cfg::kBoxBytes, &map_v, v_full + st, b * 64, row);
@@ -277,9 +301,8 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
             }
           }
           if (!ok) break;
-          if (j > jb) umma_commit(v_empty + stV);
           if (j < je) {
-            umma_commit(k_empty + stK);
+            umma_commit(kv_done + stK);   // K_j and V_{j-1} (and a drained V of the previous unit)
             if (j == je - 1) umma_commit(q_empty);
             ++kv_it;
           }
@@ -297,13 +320,19 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
     const uint32_t lane_addr = tmem + ((uint32_t)((warp % 4) * 32) << 16);
     const uint32_t colS = i == 0 ? Cfg::kColS0 : Cfg::kColS1;
     const uint32_t colO = i == 0 ? Cfg::kColO0 : Cfg::kColO1;
-    uint32_t s_cnt = 0, o_cnt = 0;
+    uint32_t s_cnt = 0, o_cnt = 0, q_cnt = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const Unit U = decode_unit(u, BH, T, c);
       if (i >= U.nt) continue;
       float m_ref = 0.f, l = 0.f;
+      // Key tiles where both query tiles are active: there the exp passes of
+      // the two warpgroups alternate (tile 0, tile 1, tile 0, ...), handing a
+      // token through seq[], so they do not compete for the SFU and issue
+      // slots and each one overlaps the other tile's MMAs.
+      const int pb = U.nt == 2 ? U.beg[1] : 0, pe = U.nt == 2 ? U.end[0] : 0;
       for (int j = U.beg[i]; j < U.end[i]; ++j) {
+        const bool paired = j >= pb && j < pe;
         ok = __all_sync(0xffffffffu, mbar_wait(s_full + i, s_cnt & 1, abort_flag, status));
         if (!ok) break;
         ++s_cnt;
@@ -351,6 +380,11 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
             tmem_st32(lane_addr + colO + cb * 32, o);
           }
         }
+        if (paired && (i == 1 || j > pb)) {
+          ok = __all_sync(0xffffffffu, mbar_wait(seq + i, q_cnt & 1, abort_flag, status));
+          if (!ok) break;
+          ++q_cnt;
+        }
         // pass 2: p = 2^(s log2e - m_ref) in chunks of 32 columns (the next
         // chunk's TMEM load is in flight while this one is computed).  The
         // argument uses packed FMA; of every 8 pairs, kSfuPairs go to the SFU
@@ -375,6 +409,15 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           for (int x = 0; x < 16; ++x) {
             const uint64_t a2 = ffma2(pack2(__uint_as_float(cur[2 * x]), __uint_as_float(cur[2 * x + 1])), l2e2, nm2);
             uint64_t p2;
+#if GECKO_SCA_H2EXP
+            {
+              // one packed f16 SFU op for the pair; P is rounded to bf16 anyway
+              float a0, a1, e0, e1;
+              unpack2(a2, a0, a1);
+              ex2_h2(a0, a1, e0, e1);
+              p2 = pack2(e0, e1);
+            }
+#else
             if (x % 8 < kSfuPairs) {
               float a0, a1;
               unpack2(a2, a0, a1);
@@ -382,6 +425,7 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
             } else {
               p2 = exp2_poly2(a2);
             }
+#endif
             acc2[x & 1] = fadd2(acc2[x & 1], p2);
             float p0, p1;
             unpack2(p2, p0, p1);
@@ -394,6 +438,10 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           }
         }
         tmem_wait_st();
+        if (paired && (i == 0 || j + 1 < pe)) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(seq + (1 - i));
+        }
         {
           float a0, a1, b0, b1;
           unpack2(acc2[0], a0, a1);
