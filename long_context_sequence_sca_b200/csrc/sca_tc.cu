@@ -257,10 +257,7 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
         const int jb = U.beg[0], je = U.nt == 2 ? U.end[1] : U.end[0];
         for (int j = jb; j <= je && ok; ++j) {
           const uint32_t stK = kv_it % KST;
-          if (j < je) {
-            if (!(ok = mbar_wait(k_full + stK, (kv_it / KST) & 1, abort_flag, status))) break;
-            tc_fence_after();
-          }
+          bool k_ready = false;  // K_j is waited for only right before the first QK that reads it
           const uint32_t itV = kv_it - 1;  // V_{j-1}
           const uint32_t stV = itV % KST;
           if (j > jb) {
@@ -289,6 +286,11 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
               }
             }
             if (j >= U.beg[i] && j < U.end[i]) {
+              if (!k_ready) {
+                if (!(ok = mbar_wait(k_full + stK, (kv_it / KST) & 1, abort_flag, status))) break;
+                tc_fence_after();
+                k_ready = true;
+              }
               // S_i = Q_i K_j^T
               const SDesc qd = sdesc_sw128_split(qa + i * Cfg::kTileBytes, 16, 1024);
               const SDesc kd = sdesc_sw128_split(ka + stK * Cfg::kTileBytes, 16, 1024);
