@@ -41,7 +41,7 @@ from long_context_sequence_sca_b200.inputs import WORKLOADS, Workload, make_inpu
 DEFAULT_WORKLOAD = "bf16_h32_c4096"
 METRIC = "tokens/s fused SCA+AWM fwd (bf16,H=32,d=128,c=4096); % bf16 TC peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-SCA_PROFILE = os.path.join(ROOT, "profiles", "sca_tc_traffic.json")
+SCA_PROFILE = os.path.join(ROOT, "profiles", "sca_tc_traffic_bf16_h32_c4096.md")
 
 
 # ------------------------------------------------------- algorithmic work --
@@ -255,15 +255,24 @@ def sca_source_hash() -> str:
 
 
 def recorded_traffic(w: Workload):
-    """DRAM bytes per SCA launch from the committed ncu record, or None if the
-    record is missing, for another workload, or older than the kernel source."""
+    """DRAM bytes per SCA launch from the committed ncu summary, or None if
+    the summary is missing, for another workload, or older than the kernel
+    source.  The summary carries `key: value` lines for workload,
+    source_hash and dram_bytes_per_launch."""
     if not os.path.exists(SCA_PROFILE):
         return None
+    rec = {}
     with open(SCA_PROFILE) as f:
-        rec = json.load(f)
+        for line in f:
+            if ":" in line and not line.startswith(("#", "|", " ")):
+                k_, v_ = line.split(":", 1)
+                rec[k_.strip()] = v_.strip()
     if rec.get("source_hash") != sca_source_hash() or rec.get("workload") != w.name:
         return None
-    return rec.get("dram_bytes_per_launch")
+    try:
+        return int(rec["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
 
 
 # ------------------------------------------------------------------ arms --
@@ -388,9 +397,9 @@ def run_e2e(args, w, x, ws, stream, L) -> dict:
 
 def cpu_baseline(w: Workload) -> dict:
     n_chunks = 3 if w.S >= 3 else w.S
-    tok_s, secs, tok = time_oracle(w, n_chunks, reps=2)
+    tok_s, secs, tok = time_oracle(w, n_chunks, reps=10)
     return {"value": round(tok_s, 2), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"fp64 oracle forward on the first {n_chunks} chunks of 2 heads "
+            "sample": f"fp64 oracle forward on the first {n_chunks} chunks of 10 heads "
                       f"({tok} tokens, c={w.c}, d={w.d}) in {secs:.1f} s"}
 
 
