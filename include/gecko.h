@@ -89,6 +89,37 @@ int gecko_sca_awm_forward(const void* q, const void* k, const void* v,
                           int dtype, void* stream);
 
 /*
+ * gecko_sca_awm_forward_continue - the same forward for one segment of a
+ * longer sequence, so a sequence of any length runs in pieces whose outputs
+ * equal those of one call over the whole sequence (up to rounding).  The AWM
+ * state is what the pages carry from chunk to chunk (Gecko digest, core
+ * method: z^s accumulates over all history; method step details, step 4:
+ * M'_s is updated from M'_{s-1}; paperlayer.ai summary, section 3.3: memory
+ * updates operate chunk by chunk), and SCA needs the previous chunk's keys
+ * and values (step 3).
+ *
+ *   state_in == NULL: a fresh sequence.  k and v are [B, H, T, d]; identical
+ *     to gecko_sca_awm_forward.
+ *   state_in != NULL: a continuation.  k and v are [B, H, c + T, d]: per
+ *     (b, h), the c rows of the previous segment's last chunk followed by
+ *     this segment's T rows.  state_in is the state_out of the previous
+ *     segment.  q, qm, km, out_sca, out_mem stay [B, H, T, d].
+ *   state_out (may be NULL, may equal state_in): [B, H, 2 d^2 + d] fp32,
+ *     per (b, h) M'_S (d x d), M'_{S+1} (d x d) and log z^S (d), in this
+ *     segment's chunk numbering (S = T / c); device or host memory.
+ *
+ * Same constraints, ownership, workspace and errors as gecko_sca_awm_forward
+ * (state_in is copied into the library's memory before use).  After the
+ * call, gecko_awm_state reports this segment's state.
+ */
+int gecko_sca_awm_forward_continue(const void* q, const void* k, const void* v,
+                                   const void* qm, const void* km,
+                                   void* out_sca, void* out_mem,
+                                   const float* state_in, float* state_out,
+                                   int64_t B, int64_t H, int64_t T, int64_t c, int64_t d,
+                                   int dtype, void* stream);
+
+/*
  * gecko_sca_awm_forward_noalloc - the same forward as gecko_sca_awm_forward
  * (same arguments, kernels and results) for callers that must not allocate
  * device memory themselves or through this library: for example a plugin
@@ -126,7 +157,8 @@ int gecko_sca_awm_forward_noalloc(const void* q, const void* k, const void* v,
 
 /*
  * gecko_awm_state - copy the AWM state carried out of the most recent
- * forward on the current device: M_out [B, H, d, d] fp32 = M'_{S+1} (all S
+ * gecko_sca_awm_forward or gecko_sca_awm_forward_continue call on the
+ * current device: M_out [B, H, d, d] fp32 = M'_{S+1} (all S
  * chunks folded in, normalised by z^S; row = key feature) and logz_out
  * [B, H, d] fp32 = log z^S.  Pointers may be device or host memory
  * (cudaMemcpyDefault).  The copy is ordered on `stream`; the call returns

@@ -61,7 +61,8 @@ template <int D>
 __global__ void __launch_bounds__(192, 2) awm_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_v,
                                                            const __nv_bfloat16* __restrict__ km,
                                                            const float* __restrict__ lse, float* __restrict__ Bm,
-                                                           float* __restrict__ Cm, int T, int c, int* status) {
+                                                           float* __restrict__ Cm, int T, int c, int koff,
+                                                           int* status) {
   using Cfg = ChunkCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -79,6 +80,8 @@ __global__ void __launch_bounds__(192, 2) awm_chunk_tc_kernel(const __grid_const
   const int warp = warp_id_uniform(), lane = threadIdx.x % 32;
   const int n_tiles = c / kKT;
   const int64_t row0 = bh * (int64_t)T + (int64_t)s * c;
+  // v carries koff extra leading rows per (b, h) when a sequence is continued
+  const int64_t vrow0 = bh * (int64_t)(T + koff) + koff + (int64_t)s * c;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -110,7 +113,7 @@ __global__ void __launch_bounds__(192, 2) awm_chunk_tc_kernel(const __grid_const
         mbar_arrive_expect_tx(v_full + st, Cfg::kOperand);
         for (int b = 0; b < D / 64; ++b)
           tma_load_2d(smem + st * Cfg::kStage + b * Cfg::kBox, &map_v, v_full + st, b * 64,
-                      (int)(row0 + (int64_t)kt * kKT));
+                      (int)(vrow0 + (int64_t)kt * kKT));
       }
       if (*abort_flag) {
         for (int st = 0; st < 2; ++st) mbar_wait_drain(v_full + st, ((n_tiles - 1 - st) >> 1) & 1);
@@ -272,6 +275,7 @@ template <int D>
 __global__ void __launch_bounds__(128) awm_readout_tc_kernel(const __nv_bfloat16* __restrict__ qm,
                                                              const float* __restrict__ Mst,
                                                              __nv_bfloat16* __restrict__ out, int T, int c,
+                                                             const float* __restrict__ Mprev0, int64_t sd,
                                                              int* status) {
   using Cfg = ReadoutCfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -290,8 +294,8 @@ __global__ void __launch_bounds__(128) awm_readout_tc_kernel(const __nv_bfloat16
   const int m = n_tiles > g ? (n_tiles - g + G - 1) / G : 0;  // tiles of this CTA
   const int64_t row0 = bh * (int64_t)T + (int64_t)s * c;
 
-  if (s < 2) {
-    // chunks 1 and 2 read M'_0 = M'_1 = 0
+  if (s < 2 && Mprev0 == nullptr) {
+    // a fresh sequence: chunks 1 and 2 read M'_0 = M'_1 = 0
     const uint4 z = make_uint4(0, 0, 0, 0);
     for (int idx = 0; idx < m; ++idx) {
       uint4* dst = reinterpret_cast<uint4*>(out + (row0 + (int64_t)(g + idx * G) * 128) * D);
@@ -312,9 +316,10 @@ __global__ void __launch_bounds__(128) awm_readout_tc_kernel(const __nv_bfloat16
     tmem_alloc(tmem_slot, Cfg::kTmemCols);
     tmem_relinquish();
   }
-  // B operand: M'_{s-1} (0-based chunk s reads Mst[s-1]) as bf16, rows = key
+  // B operand: M'_{s-1} (0-based chunk s reads Mst[s-1]; a continued
+  // sequence's first chunk reads the carried M'_prev) as bf16, rows = key
   // feature f (K), columns = value dim j (N, contiguous): MN-major.
-  const float* M = Mst + (bh * (S + 1) + (s - 1)) * (int64_t)D * D;
+  const float* M = s == 0 ? Mprev0 + bh * sd : Mst + (bh * (S + 1) + (s - 1)) * (int64_t)D * D;
   for (int i = threadIdx.x; i < D * D / 8; i += blockDim.x) {
     const int f = (i * 8) / D, j = (i * 8) % D;
     const float4 a = reinterpret_cast<const float4*>(M + f * D + j)[0];
@@ -458,7 +463,7 @@ cudaError_t chunk_impl(const Problem& p, const Workspace& w, cudaStream_t st) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
   CUtensorMap mv;
-  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)(p.B * p.H * p.T)};
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)(p.B * p.H * (p.T + p.koff))};
   cuuint64_t strides[1] = {(cuuint64_t)D * 2};
   cuuint32_t box[2] = {64, (cuuint32_t)kKT};
   cuuint32_t estr[2] = {1, 1};
@@ -470,7 +475,7 @@ cudaError_t chunk_impl(const Problem& p, const Workspace& w, cudaStream_t st) {
                                        Cfg::kAlloc);
   if (e != cudaSuccess) return e;
   awm_chunk_tc_kernel<D><<<dim3(p.S, p.B * p.H), 192, Cfg::kAlloc, st>>>(
-      mv, static_cast<const __nv_bfloat16*>(p.km), w.lse, w.Bm, w.Cm, (int)p.T, (int)p.c, p.status);
+      mv, static_cast<const __nv_bfloat16*>(p.km), w.lse, w.Bm, w.Cm, (int)p.T, (int)p.c, (int)p.koff, p.status);
   return cudaGetLastError();
 }
 
@@ -485,7 +490,7 @@ cudaError_t readout_impl(const Problem& p, const Workspace& w, cudaStream_t st) 
   const int G = n_tiles > 8 ? (n_tiles + 7) / 8 : 1;
   awm_readout_tc_kernel<D><<<dim3(p.S, p.B * p.H, G), 128, Cfg::kAlloc, st>>>(
       static_cast<const __nv_bfloat16*>(p.qm), w.Mst, static_cast<__nv_bfloat16*>(p.out_mem), (int)p.T,
-      (int)p.c, p.status);
+      (int)p.c, p.state0, state_floats(D), p.status);
   return cudaGetLastError();
 }
 

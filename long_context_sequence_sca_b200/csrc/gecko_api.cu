@@ -83,6 +83,8 @@ struct DeviceState {
   bool have_state = false;
   int64_t B = 0, H = 0, d = 0, S = 0, T = 0;
   void* noalloc_scratch = nullptr;  // device address of g_noalloc_scratch
+  void* state = nullptr;             // copy of a carried state (continued sequences)
+  size_t state_bytes = 0;
 };
 
 std::mutex g_mu;
@@ -183,9 +185,34 @@ struct StageEvents {
 
 using namespace gecko;
 
-extern "C" int gecko_sca_awm_forward(const void* q, const void* k, const void* v, const void* qm, const void* km,
-                                     void* out_sca, void* out_mem, int64_t B, int64_t H, int64_t T, int64_t c,
-                                     int64_t d, int dtype, void* stream) {
+namespace gecko {
+namespace {
+
+// Grow a per-device buffer with stream-ordered allocation.
+int ensure_buffer(void** buf, size_t* have, size_t need, cudaStream_t st, const char* what) {
+  if (need <= *have) return GECKO_OK;
+  if (*buf) {
+    cudaFreeAsync(*buf, st);
+    *buf = nullptr;
+    *have = 0;
+  }
+  void* p = nullptr;
+  cudaError_t e = cudaMallocAsync(&p, need, st);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(GECKO_ERR_ALLOC, "%s of %zu bytes: %s", what, need, cudaGetErrorString(e));
+  }
+  *buf = p;
+  *have = need;
+  return GECKO_OK;
+}
+
+// The allocating forward, fresh (state_in == nullptr) or continuing a
+// sequence (k, v with c prepended rows per (b, h); state_in on the device
+// or host).  state_out, if given, receives (M'_S, M'_{S+1}, log z^S).
+int run_forward(const void* q, const void* k, const void* v, const void* qm, const void* km, void* out_sca,
+                void* out_mem, const float* state_in, float* state_out, int64_t B, int64_t H, int64_t T,
+                int64_t c, int64_t d, int dtype, void* stream) {
   const void* ptrs[7] = {q, k, v, qm, km, out_sca, out_mem};
   int rc = validate(ptrs, 7, B, H, T, c, d, dtype);
   if (rc) return rc;
@@ -199,26 +226,21 @@ extern "C" int gecko_sca_awm_forward(const void* q, const void* k, const void* v
 
   const int64_t S = T / c;
   const int64_t BH = B * H;
-  const size_t need = workspace_bytes(BH, T, c, d);
+  const int64_t sd = state_floats(d);
   if (env_is("GECKO_FAIL_ALLOC", "1")) return fail(GECKO_ERR_ALLOC, "workspace allocation failed (injected)");
-  if (need > ds->ws_bytes) {
-    if (ds->ws) {
-      cudaFreeAsync(ds->ws, st);
-      ds->ws = nullptr;
-      ds->ws_bytes = 0;
-    }
-    void* p = nullptr;
-    cudaError_t e = cudaMallocAsync(&p, need, st);
-    if (e != cudaSuccess) {
-      cudaGetLastError();
-      return fail(GECKO_ERR_ALLOC, "workspace of %zu bytes: %s", need, cudaGetErrorString(e));
-    }
-    ds->ws = p;
-    ds->ws_bytes = need;
-  }
+  if ((rc = ensure_buffer(&ds->ws, &ds->ws_bytes, workspace_bytes(BH, T, c, d), st, "workspace"))) return rc;
   Workspace w = carve_workspace(ds->ws, BH, T, c, d);
 
   Problem p{q, k, v, qm, km, out_sca, out_mem, B, H, T, c, d, (int)S, dtype, ds->status};
+  if (state_in) {
+    // private copy, so state_out may alias state_in
+    if ((rc = ensure_buffer(&ds->state, &ds->state_bytes, sizeof(float) * BH * sd, st, "state copy"))) return rc;
+    if ((rc = check_cuda(cudaMemcpyAsync(ds->state, state_in, sizeof(float) * BH * sd, cudaMemcpyDefault, st),
+                         "copy state in")))
+      return rc;
+    p.koff = c;
+    p.state0 = static_cast<const float*>(ds->state);
+  }
   // GECKO_KERNELS=simt selects the CUDA-core kernels for every dtype (a
   // second, independent GPU implementation used to cross-check the
   // tensor-core path).
@@ -242,6 +264,18 @@ extern "C" int gecko_sca_awm_forward(const void* q, const void* k, const void* v
   if ((rc = check_cuda(use_tc ? launch_sca_tc(p, st) : launch_sca_simt(p, st), "sca"))) return rc;
   ev.mark(5);
   ev.commit();
+  if (state_out) {
+    // (M'_S, M'_{S+1}, log z^S) of every (b, h): Mst[S-1], Mst[S], logz[S-1]
+    const size_t mat = sizeof(float) * d * d, rec = sizeof(float) * sd;
+    if ((rc = check_cuda(cudaMemcpy2DAsync(state_out, rec, w.Mst + (S - 1) * d * d, mat * (S + 1), 2 * mat, BH,
+                                           cudaMemcpyDefault, st),
+                         "copy state out (M)")))
+      return rc;
+    if ((rc = check_cuda(cudaMemcpy2DAsync(state_out + 2 * d * d, rec, w.logz + (S - 1) * d, sizeof(float) * d * S,
+                                           sizeof(float) * d, BH, cudaMemcpyDefault, st),
+                         "copy state out (log z)")))
+      return rc;
+  }
   ds->have_state = true;
   ds->B = B;
   ds->H = H;
@@ -249,6 +283,22 @@ extern "C" int gecko_sca_awm_forward(const void* q, const void* k, const void* v
   ds->S = S;
   ds->T = T;
   return GECKO_OK;
+}
+
+}  // namespace
+}  // namespace gecko
+
+extern "C" int gecko_sca_awm_forward(const void* q, const void* k, const void* v, const void* qm, const void* km,
+                                     void* out_sca, void* out_mem, int64_t B, int64_t H, int64_t T, int64_t c,
+                                     int64_t d, int dtype, void* stream) {
+  return run_forward(q, k, v, qm, km, out_sca, out_mem, nullptr, nullptr, B, H, T, c, d, dtype, stream);
+}
+
+extern "C" int gecko_sca_awm_forward_continue(const void* q, const void* k, const void* v, const void* qm,
+                                              const void* km, void* out_sca, void* out_mem, const float* state_in,
+                                              float* state_out, int64_t B, int64_t H, int64_t T, int64_t c,
+                                              int64_t d, int dtype, void* stream) {
+  return run_forward(q, k, v, qm, km, out_sca, out_mem, state_in, state_out, B, H, T, c, d, dtype, stream);
 }
 
 extern "C" int gecko_awm_state(float* M_out, float* logz_out, int64_t B, int64_t H, int64_t d, void* stream) {
@@ -309,13 +359,16 @@ extern "C" void gecko_release(void) {
   int cur = 0;
   cudaGetDevice(&cur);
   for (auto& kv : g_dev) {
-    if (kv.second.ws) {
+    if (kv.second.ws || kv.second.state) {
       cudaSetDevice(kv.first);
       cudaDeviceSynchronize();
-      cudaFree(kv.second.ws);
+      if (kv.second.ws) cudaFree(kv.second.ws);
+      if (kv.second.state) cudaFree(kv.second.state);
     }
     kv.second.ws = nullptr;
     kv.second.ws_bytes = 0;
+    kv.second.state = nullptr;
+    kv.second.state_bytes = 0;
     kv.second.have_state = false;
   }
   cudaSetDevice(cur);

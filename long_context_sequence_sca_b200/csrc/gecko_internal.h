@@ -18,7 +18,13 @@ struct Problem {
   int S;
   int dtype;
   int* status;        // device status word
+  // Continuation of a longer sequence (all zero for a fresh start):
+  int64_t koff = 0;              // rows of the previous chunk prepended to k and v per head (0 or c)
+  const float* state0 = nullptr; // [BH, 2 d^2 + d] carried state (device): M'_prev, M'_cur, log z
 };
+
+// Floats per (b, h) in a carried state record: M'_prev, M'_cur (d x d each), log z (d).
+inline int64_t state_floats(int64_t d) { return 2 * d * d + d; }
 
 // Device workspace carved out of one allocation (all fp32).
 struct Workspace {

@@ -90,7 +90,7 @@ struct Unit {
 // L2 holds, and every K/V tile then comes from DRAM).  Inside a group the
 // units go from the most to the least expensive; groups of later chunks
 // come first and the cheap chunk-1 groups last, which keeps the tail short.
-__device__ __forceinline__ Unit decode_unit(int u, int BH, int T, int c) {
+__device__ __forceinline__ Unit decode_unit(int u, int BH, int T, int c, int koff) {
   const int pairs = (T + 255) / 256;
   Unit U;
   int pair;
@@ -120,7 +120,8 @@ __device__ __forceinline__ Unit decode_unit(int u, int BH, int T, int c) {
   for (int i = 0; i < 2; ++i) {
     const int r0 = U.q0 + 128 * i;
     const int ch = r0 / c;
-    const int lo = ch >= 1 ? (ch - 1) * c : 0;
+    // window start; negative (the prepended previous chunk) when koff > 0
+    const int lo = (ch >= 1 || koff > 0) ? (ch - 1) * c : 0;
     U.beg[i] = lo / kBN;
     U.end[i] = r0 / kBN + 1;
     if (i >= U.nt) { U.beg[i] = 0; U.end[i] = 0; }
@@ -132,7 +133,7 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
               const __grid_constant__ CUtensorMap map_v, __nv_bfloat16* __restrict__ out, int T, int c, int BH,
-              int n_units, int* status) {
+              int n_units, int koff, int* status) {
   using Cfg = ScaCfg<D>;
   constexpr int KST = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -202,8 +203,10 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       int n = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++n) {
-        const Unit U = decode_unit(u, BH, T, c);
+        const Unit U = decode_unit(u, BH, T, c, koff);
         const int64_t rowbase = U.bh * (int64_t)T;
+        // k and v carry koff extra leading rows per (b, h) (continued sequence)
+        const int64_t kvbase = U.bh * (int64_t)(T + koff) + koff;
         if (n > 0 && !(ok = mbar_wait(q_empty, (n - 1) & 1, abort_flag, status))) break;
         mbar_arrive_expect_tx(q_full, U.nt * Cfg::kTileBytes);
         for (int i = 0; i < U.nt; ++i)
@@ -213,7 +216,7 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
         const int jb = U.beg[0], je = U.nt == 2 ? U.end[1] : U.end[0];
         for (int j = jb; j < je; ++j, ++kv_it) {
           const int st = kv_it % KST;
-          const int row = (int)(rowbase + (int64_t)j * kBN);
+          const int row = (int)(kvbase + (int64_t)j * kBN);
           // slot of K_n was last read by iteration n - KST
           if (kv_it >= (uint32_t)KST &&
               !(ok = mbar_wait(kv_done + st, ((kv_it - KST) / KST) & 1, abort_flag, status)))
@@ -251,7 +254,7 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       int n = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++n) {
-        const Unit U = decode_unit(u, BH, T, c);
+        const Unit U = decode_unit(u, BH, T, c, koff);
         if (!(ok = mbar_wait(q_full, n & 1, abort_flag, status))) break;
         tc_fence_after();
         const int jb = U.beg[0], je = U.nt == 2 ? U.end[1] : U.end[0];
@@ -325,7 +328,7 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
     uint32_t s_cnt = 0, o_cnt = 0, q_cnt = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const Unit U = decode_unit(u, BH, T, c);
+      const Unit U = decode_unit(u, BH, T, c, koff);
       if (i >= U.nt) continue;
       float m_ref = 0.f, l = 0.f;
       // Key tiles where both query tiles are active: there the exp passes of
@@ -534,11 +537,12 @@ template <int D>
 cudaError_t launch_sca_tc_impl(const Problem& p, cudaStream_t st) {
   using Cfg = ScaCfg<D>;
   const int64_t rows = p.B * p.H * p.T;
+  const int64_t kv_rows = p.B * p.H * (p.T + p.koff);
   CUtensorMap mq, mk, mv;
   cudaError_t e;
   if ((e = make_map(&mq, p.q, rows, D)) != cudaSuccess) return e;
-  if ((e = make_map(&mk, p.k, rows, D)) != cudaSuccess) return e;
-  if ((e = make_map(&mv, p.v, rows, D)) != cudaSuccess) return e;
+  if ((e = make_map(&mk, p.k, kv_rows, D)) != cudaSuccess) return e;
+  if ((e = make_map(&mv, p.v, kv_rows, D)) != cudaSuccess) return e;
   const int BH = (int)(p.B * p.H);
   const int T = (int)p.T;
   const int n_units = BH * ((T + 255) / 256);
@@ -547,7 +551,7 @@ cudaError_t launch_sca_tc_impl(const Problem& p, cudaStream_t st) {
       cudaSuccess)
     return e;
   sca_tc_kernel<D><<<grid, kThreads, Cfg::kAlloc, st>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(p.out_sca), T,
-                                                        (int)p.c, BH, n_units, p.status);
+                                                        (int)p.c, BH, n_units, (int)p.koff, p.status);
   return cudaGetLastError();
 }
 
@@ -556,7 +560,7 @@ cudaError_t launch_sca_tc_impl(const Problem& p, cudaStream_t st) {
 bool tc_supported(const Problem& p) {
   if (p.dtype != kBF16 || p.c % 128 != 0) return false;
   // rows addressed through 32-bit TMA coordinates
-  if (p.B * p.H * p.T > (int64_t(1) << 31) - 1) return false;
+  if (p.B * p.H * (p.T + p.koff) > (int64_t(1) << 31) - 1) return false;
   int dev = 0, major = 0, minor = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);

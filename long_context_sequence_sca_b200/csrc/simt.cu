@@ -105,25 +105,29 @@ __global__ void __launch_bounds__(D) awm_lse_combine_kernel(const float2* __rest
 // ------------------------------------------------------------------------
 // Prefix over chunks in fp64: log z^s = logaddexp(log z^{s-1}, lse_s), the
 // row ratio r_s = z^{s-1}/z^s (0 for s = 1) and the chunk weight
-// rho_s = e_s / z^s = exp(lse_s - log z^s).  grid BH, D threads.
+// rho_s = e_s / z^s = exp(lse_s - log z^s).  A continued sequence seeds the
+// prefix with the carried log z (logz0, stride sd per (b, h)).  grid BH, D
+// threads.
 template <int D>
 __global__ void __launch_bounds__(D) awm_prefix_kernel(const float* __restrict__ lse, float* __restrict__ logz,
-                                                       float* __restrict__ ratio, float* __restrict__ rho, int S) {
+                                                       float* __restrict__ ratio, float* __restrict__ rho, int S,
+                                                       const float* __restrict__ logz0, int64_t sd) {
   const int64_t bh = blockIdx.x;
   const int f = threadIdx.x;
-  double L = 0.0;
+  const bool seeded = logz0 != nullptr;
+  double L = seeded ? (double)logz0[bh * sd + f] : 0.0;
   for (int s = 0; s < S; ++s) {
     const int64_t o = (bh * S + s) * D + f;
     const double e = lse[o];
     double Ln;
-    if (s == 0) {
+    if (s == 0 && !seeded) {
       Ln = e;
     } else {
       const double hi = fmax(L, e), lo = fmin(L, e);
       Ln = hi + log1p(exp(lo - hi));
     }
     logz[o] = (float)Ln;
-    ratio[o] = s == 0 ? 0.f : (float)exp(L - Ln);
+    ratio[o] = (s == 0 && !seeded) ? 0.f : (float)exp(L - Ln);
     rho[o] = (float)exp(e - Ln);
     L = Ln;
   }
@@ -142,7 +146,7 @@ __global__ void __launch_bounds__(256) awm_chunk_simt_kernel(const TIn* __restri
                                                              const TIn* __restrict__ v,
                                                              const float* __restrict__ lse,
                                                              float* __restrict__ Bm, float* __restrict__ Cm,
-                                                             int64_t T, int c) {
+                                                             int64_t T, int c, int64_t koff) {
   constexpr int RT = 16;       // token rows per step
   constexpr int TM = D / 16;   // outputs per thread per dim
   const int s = blockIdx.x;
@@ -161,12 +165,15 @@ __global__ void __launch_bounds__(256) awm_chunk_simt_kernel(const TIn* __restri
 #pragma unroll
     for (int j = 0; j < TM; ++j) { accB[i][j] = 0.f; accC[i][j] = 0.f; }
   const int64_t row0 = bh * T + (int64_t)s * c;
+  // v carries koff extra leading rows per (b, h) when a sequence is continued
+  const int64_t vrow0 = bh * (T + koff) + koff + (int64_t)s * c;
   const int warp = tid / 32, lane = tid % 32;
   __syncthreads();
   for (int r0 = 0; r0 < c; r0 += RT) {
     // each warp prepares RT/8 rows: phi, psi (warp-wide softmax over D), v
     for (int rr = warp; rr < RT; rr += 8) {
       const int64_t g = (row0 + r0 + rr) * D;
+      const int64_t gv = (vrow0 + r0 + rr) * D;
       float x[D / 32];
       float mx = -INFINITY;
 #pragma unroll
@@ -187,7 +194,7 @@ __global__ void __launch_bounds__(256) awm_chunk_simt_kernel(const TIn* __restri
         const int f = lane + 32 * i;
         psi_s[rr][f] = e[i] * inv;
         phi_s[rr][f] = expf(x[i] - lz[f]);
-        v_s[rr][f] = to_f32(v[g + f]);
+        v_s[rr][f] = to_f32(v[gv + f]);
       }
     }
     __syncthreads();
@@ -225,14 +232,17 @@ __global__ void __launch_bounds__(256) awm_chunk_simt_kernel(const TIn* __restri
 // evolve independently):
 //   M'_{s+1}[:, J] = r_s (.) M'_s[:, J] + rho_s (.) (Bm_s[:, J] - Cm_s M'_s[:, J])
 // (row scales r_s = z^{s-1}/z^s and rho_s = e_s/z^s).  Writes
-// Mst[bh, s] = M'_{s+1} for s = 0..S (M'_1 = 0 first).  Cm_s is staged into
-// shared memory with 16-byte loads.  grid (D / JC, BH), 256 threads.
+// Mst[bh, s] = M'_{s+1} for s = 0..S.  M'_1 = 0 for a fresh sequence; a
+// continued one starts from the carried M' (M0, stride sd per (b, h)).
+// Cm_s is staged into shared memory with 16-byte loads.  grid (D / JC, BH),
+// 256 threads.
 template <int D, int JC>
 __global__ void __launch_bounds__(256) awm_carry_kernel(const float* __restrict__ Bm,
                                                         const float* __restrict__ Cm,
                                                         const float* __restrict__ ratio,
                                                         const float* __restrict__ rho,
-                                                        float* __restrict__ Mst, int S) {
+                                                        float* __restrict__ Mst, int S,
+                                                        const float* __restrict__ M0, int64_t sd) {
   constexpr int PER = D * JC / 256;  // outputs per thread (one row f, PER columns)
   static_assert(256 / (JC / PER) == D, "thread layout");
   constexpr int LD = D + 4;          // padded row of Cm in shared memory (keeps 16-byte alignment)
@@ -244,11 +254,13 @@ __global__ void __launch_bounds__(256) awm_carry_kernel(const float* __restrict_
   const int tid = threadIdx.x;
   const int f = tid / (JC / PER);
   const int jj = (tid % (JC / PER)) * PER;
-  for (int i = tid; i < D * JC; i += 256) Ms[i] = 0.f;
+  for (int i = tid; i < D * JC; i += 256)
+    Ms[i] = M0 ? M0[bh * sd + (i / JC) * D + j0 + i % JC] : 0.f;
   const int64_t mst_stride = (int64_t)D * D;
   float* mout = Mst + bh * (int64_t)(S + 1) * mst_stride;
+  __syncthreads();
 #pragma unroll
-  for (int j = 0; j < PER; ++j) mout[f * D + j0 + jj + j] = 0.f;   // M'_1 = 0
+  for (int j = 0; j < PER; ++j) mout[f * D + j0 + jj + j] = Ms[f * JC + jj + j];   // M'_1
   for (int s = 0; s < S; ++s) {
     const float4* C4 = reinterpret_cast<const float4*>(Cm + (bh * S + s) * mst_stride);
     __syncthreads();
@@ -281,12 +293,15 @@ __global__ void __launch_bounds__(256) awm_carry_kernel(const float* __restrict_
 }
 
 // ------------------------------------------------------------------------
-// Readout O_m,s = psi(Qm_s) M'_{s-1} (zero for chunks 1 and 2).
+// Readout O_m,s = psi(Qm_s) M'_{s-1}.  For a fresh sequence chunks 1 and 2
+// read zero; a continued one reads the carried M'_prev (Mprev0, stride sd)
+// for its first chunk and the carried M'_cur (= Mst[0]) for its second.
 // grid (c / 64, S, BH), 256 threads; 64 rows per CTA.
 template <typename TIn, int D>
 __global__ void __launch_bounds__(256) awm_readout_simt_kernel(const TIn* __restrict__ qm,
                                                                const float* __restrict__ Mst,
-                                                               TIn* __restrict__ out, int64_t T, int c) {
+                                                               TIn* __restrict__ out, int64_t T, int c,
+                                                               const float* __restrict__ Mprev0, int64_t sd) {
   constexpr int R = 64;
   constexpr int CT = D / 16;  // columns per thread
   extern __shared__ float smem_ro[];
@@ -297,12 +312,12 @@ __global__ void __launch_bounds__(256) awm_readout_simt_kernel(const TIn* __rest
   const int64_t bh = blockIdx.z;
   const int64_t row0 = bh * T + (int64_t)s * c + (int64_t)blockIdx.x * R;
   const int tid = threadIdx.x;
-  if (s < 2) {
+  if (s < 2 && Mprev0 == nullptr) {
     for (int i = tid; i < R * D; i += 256) out[row0 * D + i] = from_f32<TIn>(0.f);
     return;
   }
-  // 0-based chunk s is chunk s+1; it reads M'_s = Mst[s - 1]
-  const float* M = Mst + (bh * (S + 1) + (s - 1)) * (int64_t)D * D;
+  // 0-based chunk s is chunk s+1; it reads M'_s = Mst[s - 1] (M'_prev for s = 0)
+  const float* M = s == 0 ? Mprev0 + bh * sd : Mst + (bh * (S + 1) + (s - 1)) * (int64_t)D * D;
   for (int i = tid; i < D * D; i += 256) Ms[i] = M[i];
   const int warp = tid / 32, lane = tid % 32;
   for (int rr = warp; rr < R; rr += 8) {
@@ -350,11 +365,13 @@ __global__ void __launch_bounds__(256) awm_readout_simt_kernel(const TIn* __rest
 // ------------------------------------------------------------------------
 // SCA with CUDA cores: 32 queries per CTA, 4 threads per query (each owns
 // D/4 dims of q and of the output), keys streamed through shared memory in
-// tiles of 32 with an online softmax.  Scale 1.  grid (T / 32, BH).
+// tiles of 32 with an online softmax.  Scale 1.  k and v hold koff extra
+// leading rows per (b, h) (the previous chunk of a continued sequence, so
+// chunk 1 then has a previous chunk).  grid (T / 32, BH).
 template <typename TIn, int D>
 __global__ void __launch_bounds__(128) sca_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
                                                        const TIn* __restrict__ v, TIn* __restrict__ out,
-                                                       int64_t T, int c) {
+                                                       int64_t T, int c, int64_t koff) {
   constexpr int QD = D / 4;
   __shared__ float ks[32][D + 4];
   __shared__ float vs[32][D + 4];
@@ -363,7 +380,10 @@ __global__ void __launch_bounds__(128) sca_simt_kernel(const TIn* __restrict__ q
   const int tid = threadIdx.x;
   const int qi = tid / 4, part = tid % 4;
   const int64_t t = t0 + qi;
-  const int64_t lo = t0 / c >= 1 ? (t0 / c - 1) * c : 0;  // all 32 rows share one chunk
+  // window start in segment coordinates (negative: rows of the prepended chunk);
+  // all 32 rows share one chunk
+  const int64_t lo = (t0 / c >= 1 || koff > 0) ? (t0 / c - 1) * c : 0;
+  const int64_t kbase = bh * (T + koff) + koff;
   const TIn* qrow = q + (bh * T + t) * D + part * QD;
   float qv[QD], acc[QD];
 #pragma unroll
@@ -374,7 +394,7 @@ __global__ void __launch_bounds__(128) sca_simt_kernel(const TIn* __restrict__ q
     __syncthreads();
     for (int i = tid; i < 32 * D; i += 128) {
       const int r = i / D, cc = i % D;
-      const int64_t g = (bh * T + k0 + r) * D + cc;
+      const int64_t g = (kbase + k0 + r) * D + cc;
       ks[r][cc] = to_f32(k[g]);
       vs[r][cc] = to_f32(v[g]);
     }
@@ -412,14 +432,16 @@ cudaError_t awm_stats_impl(const Problem& p, const Workspace& w, cudaStream_t st
   else
     awm_lse_partial_kernel<TIn, D, 64><<<grid, 256, 0, st>>>(static_cast<const TIn*>(p.km), w.part, p.T);
   awm_lse_combine_kernel<D><<<dim3(p.S, BH), D, 0, st>>>(w.part, w.lse, P);
-  awm_prefix_kernel<D><<<BH, D, 0, st>>>(w.lse, w.logz, w.ratio, w.rho, p.S);
+  const int64_t sd = state_floats(D);
+  awm_prefix_kernel<D><<<BH, D, 0, st>>>(w.lse, w.logz, w.ratio, w.rho, p.S,
+                                         p.state0 ? p.state0 + 2 * D * D : nullptr, sd);
   return cudaGetLastError();
 }
 
 template <typename TIn, int D>
 cudaError_t awm_chunk_simt_impl(const Problem& p, const Workspace& w, cudaStream_t st) {
   awm_chunk_simt_kernel<TIn, D><<<dim3(p.S, p.B * p.H), 256, 0, st>>>(
-      static_cast<const TIn*>(p.km), static_cast<const TIn*>(p.v), w.lse, w.Bm, w.Cm, p.T, (int)p.c);
+      static_cast<const TIn*>(p.km), static_cast<const TIn*>(p.v), w.lse, w.Bm, w.Cm, p.T, (int)p.c, p.koff);
   return cudaGetLastError();
 }
 
@@ -429,7 +451,8 @@ cudaError_t awm_carry_impl(const Problem& p, const Workspace& w, cudaStream_t st
   const size_t smem = sizeof(float) * (D * (D + 4) + D * JC);
   cudaError_t e = cudaFuncSetAttribute(awm_carry_kernel<D, JC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  awm_carry_kernel<D, JC><<<dim3(D / JC, p.B * p.H), 256, smem, st>>>(w.Bm, w.Cm, w.ratio, w.rho, w.Mst, p.S);
+  awm_carry_kernel<D, JC><<<dim3(D / JC, p.B * p.H), 256, smem, st>>>(
+      w.Bm, w.Cm, w.ratio, w.rho, w.Mst, p.S, p.state0 ? p.state0 + D * D : nullptr, state_floats(D));
   return cudaGetLastError();
 }
 
@@ -440,7 +463,7 @@ cudaError_t awm_readout_simt_impl(const Problem& p, const Workspace& w, cudaStre
       cudaFuncSetAttribute(awm_readout_simt_kernel<TIn, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   awm_readout_simt_kernel<TIn, D><<<dim3(p.c / 64, p.S, p.B * p.H), 256, smem, st>>>(
-      static_cast<const TIn*>(p.qm), w.Mst, static_cast<TIn*>(p.out_mem), p.T, (int)p.c);
+      static_cast<const TIn*>(p.qm), w.Mst, static_cast<TIn*>(p.out_mem), p.T, (int)p.c, p.state0, state_floats(D));
   return cudaGetLastError();
 }
 
@@ -448,7 +471,7 @@ template <typename TIn, int D>
 cudaError_t launch_sca_simt_impl(const Problem& p, cudaStream_t st) {
   sca_simt_kernel<TIn, D><<<dim3(p.T / 32, p.B * p.H), 128, 0, st>>>(
       static_cast<const TIn*>(p.q), static_cast<const TIn*>(p.k), static_cast<const TIn*>(p.v),
-      static_cast<TIn*>(p.out_sca), p.T, (int)p.c);
+      static_cast<TIn*>(p.out_sca), p.T, (int)p.c, p.koff);
   return cudaGetLastError();
 }
 

@@ -16,6 +16,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgecko.so
 # Symbols declared in include/gecko.h
 EXPORTS = (
     "gecko_sca_awm_forward",
+    "gecko_sca_awm_forward_continue",
     "gecko_sca_awm_forward_noalloc",
     "gecko_awm_state",
     "gecko_device_status",
@@ -56,6 +57,8 @@ def load() -> ctypes.CDLL:
     i64, vp = ctypes.c_int64, ctypes.c_void_p
     lib.gecko_sca_awm_forward.argtypes = [vp] * 7 + [i64] * 5 + [ctypes.c_int, vp]
     lib.gecko_sca_awm_forward.restype = ctypes.c_int
+    lib.gecko_sca_awm_forward_continue.argtypes = [vp] * 9 + [i64] * 5 + [ctypes.c_int, vp]
+    lib.gecko_sca_awm_forward_continue.restype = ctypes.c_int
     lib.gecko_sca_awm_forward_noalloc.argtypes = [vp] * 7 + [i64] * 5 + [ctypes.c_int, vp]
     lib.gecko_sca_awm_forward_noalloc.restype = ctypes.c_int
     lib.gecko_awm_state.argtypes = [vp, vp, i64, i64, i64, vp]
@@ -90,6 +93,13 @@ def _stream_handle(stream) -> int:
 def gecko_sca_awm_forward(q, k, v, qm, km, out_sca, out_mem, B, H, T, c, d, dtype, stream) -> int:
     """Direct call of the C entry point with integer pointers; returns the status."""
     return load().gecko_sca_awm_forward(q, k, v, qm, km, out_sca, out_mem, B, H, T, c, d, dtype, stream)
+
+
+def gecko_sca_awm_forward_continue(q, k, v, qm, km, out_sca, out_mem, state_in, state_out, B, H, T, c, d, dtype,
+                                   stream) -> int:
+    """Forward of one segment of a longer sequence (state_in 0 = fresh)."""
+    return load().gecko_sca_awm_forward_continue(q, k, v, qm, km, out_sca, out_mem, state_in, state_out,
+                                                 B, H, T, c, d, dtype, stream)
 
 
 def gecko_sca_awm_forward_noalloc(q, k, v, qm, km, out_sca, out_mem, B, H, T, c, d, dtype, stream) -> int:
@@ -152,6 +162,33 @@ def sca_awm_forward(q, k, v, qm, km, c: int, out_sca=None, out_mem=None, stream=
                                    B, H, T, c, d, _DT[q.dtype], _stream_handle(stream))
     _check(rc)
     return out_sca, out_mem
+
+
+def sca_awm_forward_segment(q, k, v, qm, km, c: int, state_in=None, out_sca=None, out_mem=None, stream=None):
+    """One segment of a long sequence.  q, qm, km: [B, H, T, d].  Without
+    state_in, k and v are [B, H, T, d] (fresh start); with it they are
+    [B, H, c + T, d], the previous segment's last chunk first.  Returns
+    (out_sca, out_mem, state) where state [B, H, 2 d^2 + d] fp32 feeds the
+    next segment."""
+    xs = (q, k, v, qm, km)
+    for x in xs:
+        if not (isinstance(x, torch.Tensor) and x.is_cuda and x.is_contiguous() and x.dtype == q.dtype):
+            raise ValueError("inputs must be contiguous CUDA tensors of one dtype")
+    B, H, T, d = q.shape
+    kv_rows = T + (c if state_in is not None else 0)
+    if tuple(k.shape) != (B, H, kv_rows, d) or tuple(v.shape) != (B, H, kv_rows, d):
+        raise ValueError(f"k and v must be [B, H, {kv_rows}, d]")
+    if out_sca is None:
+        out_sca = torch.empty_like(q)
+    if out_mem is None:
+        out_mem = torch.empty_like(q)
+    state = torch.empty(B, H, 2 * d * d + d, dtype=torch.float32, device=q.device)
+    with torch.cuda.device(q.device):
+        rc = gecko_sca_awm_forward_continue(*(x.data_ptr() for x in xs), out_sca.data_ptr(), out_mem.data_ptr(),
+                                            0 if state_in is None else state_in.data_ptr(), state.data_ptr(),
+                                            B, H, T, c, d, _DT[q.dtype], _stream_handle(stream))
+    _check(rc)
+    return out_sca, out_mem, state
 
 
 def awm_state(B: int, H: int, d: int, device=None, stream=None):
