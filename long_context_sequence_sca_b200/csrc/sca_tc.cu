@@ -9,7 +9,9 @@
 //
 // Design (one persistent CTA per SM, 320 threads):
 //   warp 0      TMA producer: Q tiles once per work unit; K and V tiles of
-//               128 keys through a ring of shared-memory stages.
+//               128 keys through rings of shared-memory stages (K one
+//               stage deeper than V), loads issued in the order of the
+//               iterations that free their slots.
 //   warp 1      TMEM allocator and MMA issuer (one thread): S_i = Q_i K_j^T
 //               (SS form) into TMEM, O_i += P_i V_j with P_i read from TMEM
 //               (TS form).
@@ -48,28 +50,30 @@ constexpr int kThreads = 320;   // 10 warps: TMA, MMA (+TMEM allocation), 2 x 4 
 #ifndef GECKO_SFU_PAIRS
 #define GECKO_SFU_PAIRS 8
 #endif
-// GECKO_SCA_H2EXP = 1 evaluates the softmax exponentials as packed f16 pairs
-// (ex2.approx.f16x2, two per SFU op) instead of fp32 SFU ops.
-#ifndef GECKO_SCA_H2EXP
-#define GECKO_SCA_H2EXP 0
-#endif
 constexpr int kSfuPairs = GECKO_SFU_PAIRS;
 
 template <int D>
 struct ScaCfg {
   static constexpr int kTileBytes = 128 * D * 2;       // 128 rows x D bf16, D/64 swizzled boxes
   static constexpr int kBoxBytes = 128 * 64 * 2;       // one [128 x 64] box
-  static constexpr int kStages = D == 64 ? 4 : 2;      // K and V stages each
+  // K ring one stage deeper than the V ring: K_m is read at the start of
+  // iteration m, V_m only at the start of iteration m + 1, so with equal
+  // rings K would get one iteration less to arrive (at d = 128 shared
+  // memory holds Q, 3 K and 2 V tiles: 224 KB).
+  static constexpr int kKStages = D == 64 ? 5 : 3;
+  static constexpr int kVStages = D == 64 ? 4 : 2;
+  static_assert(kKStages >= kVStages, "the iteration-done ring has kKStages slots");
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + 2 * kTileBytes;
-  static constexpr int kVOff = kKOff + kStages * kTileBytes;
-  static constexpr int kBarOff = kVOff + kStages * kTileBytes;
-  // q_full, q_empty, k_full[S], kv_done[S], v_full[S], (unused)[S],
-  // s_full[2], p_full[2], o_full[2], o_empty[2], drain, seq[2]
-  static constexpr int kNumBars = 2 + 4 * kStages + 8 + 1 + 2;
+  static constexpr int kVOff = kKOff + kKStages * kTileBytes;
+  static constexpr int kBarOff = kVOff + kVStages * kTileBytes;
+  // q_full, q_empty, k_full[KS], it_done[KS], v_full[VS], s_full[2],
+  // p_full[2], o_full[2], o_empty[2], drain
+  static constexpr int kNumBars = 2 + 2 * kKStages + kVStages + 8 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;         // slack for 1024-byte alignment
+  static_assert(kAlloc <= 232448, "dynamic shared memory above the sm_100 per-block limit");
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
 };
@@ -129,13 +133,42 @@ __device__ __forceinline__ Unit decode_unit(int u, int BH, int T, int c, int kof
   return U;
 }
 
+// Walks the K/V iterations of one CTA in the order the MMA warp consumes
+// them: its units (u, u + gridDim.x, ...) one after another, and each
+// unit's key tiles in order.
+struct KvWalk {
+  int u;            // current unit (>= n_units: finished)
+  int j, je;        // current key tile of the unit, one past its last
+  int64_t kvbase;   // first K/V row of the unit's (b, h)
+  uint32_t it;      // iterations walked so far
+};
+
+__device__ __forceinline__ void kv_walk_enter(KvWalk& w, int u, int BH, int T, int c, int koff, int n_units) {
+  w.u = u;
+  if (u < n_units) {
+    const Unit U = decode_unit(u, BH, T, c, koff);
+    w.j = U.beg[0];
+    w.je = U.nt == 2 ? U.end[1] : U.end[0];
+    w.kvbase = U.bh * (int64_t)(T + koff) + koff;
+  }
+}
+
+__device__ __forceinline__ void kv_walk_next(KvWalk& w, int stride, int BH, int T, int c, int koff, int n_units) {
+  ++w.it;
+  if (++w.j == w.je) {
+    const uint32_t it = w.it;
+    kv_walk_enter(w, w.u + stride, BH, T, c, koff, n_units);
+    w.it = it;
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
               const __grid_constant__ CUtensorMap map_v, __nv_bfloat16* __restrict__ out, int T, int c, int BH,
               int n_units, int koff, int* status) {
   using Cfg = ScaCfg<D>;
-  constexpr int KST = Cfg::kStages;
+  constexpr int KS = Cfg::kKStages, VS = Cfg::kVStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + Cfg::kQOff;
@@ -145,16 +178,15 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
   uint64_t* k_full = bars + 2;
-  // kv_done[m % KST] completes when the MMAs of K/V iteration m are done:
+  // it_done[m % KS] completes when the MMAs of K/V iteration m are done:
   // they were the last readers of K_m and of V_{m-1}
-  uint64_t* kv_done = k_full + KST;
-  uint64_t* v_full = kv_done + KST;
-  uint64_t* s_full = v_full + 2 * KST;
+  uint64_t* it_done = k_full + KS;
+  uint64_t* v_full = it_done + KS;
+  uint64_t* s_full = v_full + VS;
   uint64_t* p_full = s_full + 2;
   uint64_t* o_full = p_full + 2;
   uint64_t* o_empty = o_full + 2;
   uint64_t* drain = o_empty + 2;
-  uint64_t* seq = drain + 1;       // [2] exp-pass tokens between the softmax warpgroups
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
 
@@ -164,11 +196,11 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int s = 0; s < KST; ++s) {
+    for (int s = 0; s < KS; ++s) {
       mbar_init(k_full + s, 1);
-      mbar_init(kv_done + s, 1);
-      mbar_init(v_full + s, 1);
+      mbar_init(it_done + s, 1);
     }
+    for (int s = 0; s < VS; ++s) mbar_init(v_full + s, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + i, 1);
       mbar_init(p_full + i, 128);
@@ -176,8 +208,6 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       mbar_init(o_empty + i, 128);
     }
     mbar_init(drain, 1);
-    mbar_init(seq, 4);             // one arrival per warp of the other warpgroup
-    mbar_init(seq + 1, 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -199,48 +229,65 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
     if (lane == 0) {
-      uint32_t kv_it = 0;
-      int n = 0;
+      // Three load streams, each in the order the MMA warp consumes them:
+      // Q of every unit, K_m and V_m of every K/V iteration m.  A load
+      // first waits until the previous reader of its slot is done: K_m for
+      // iteration m - KS, V_m for iteration m + 1 - VS (V_m is read by the
+      // PV MMAs of iteration m + 1), Q of a unit for the last QK of the
+      // previous unit.  Issuing the loads in the order of those iterations
+      // (not unit by unit) lets K run ahead of V by its deeper ring, and
+      // every wait is then for an iteration whose own loads were issued
+      // earlier, so the producer never waits on itself.
+      KvWalk kw{}, vw{};
+      kv_walk_enter(kw, blockIdx.x, BH, T, c, koff, n_units);
+      vw = kw;
+      int qu = blockIdx.x, qn = 0;
+      uint32_t qit0 = 0;   // first K/V iteration of unit qu
       bool ok = true;
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++n) {
-        const Unit U = decode_unit(u, BH, T, c, koff);
-        const int64_t rowbase = U.bh * (int64_t)T;
-        // k and v carry koff extra leading rows per (b, h) (continued sequence)
-        const int64_t kvbase = U.bh * (int64_t)(T + koff) + koff;
-        if (n > 0 && !(ok = mbar_wait(q_empty, (n - 1) & 1, abort_flag, status))) break;
-        mbar_arrive_expect_tx(q_full, U.nt * Cfg::kTileBytes);
-        for (int i = 0; i < U.nt; ++i)
-          for (int b = 0; b < D / 64; ++b)
-            tma_load_2d(sQ + i * Cfg::kTileBytes + b * Cfg::kBoxBytes, &map_q, q_full, b * 64,
-                        (int)(rowbase + U.q0 + 128 * i));
-        const int jb = U.beg[0], je = U.nt == 2 ? U.end[1] : U.end[0];
-        for (int j = jb; j < je; ++j, ++kv_it) {
-          const int st = kv_it % KST;
-          const int row = (int)(kvbase + (int64_t)j * kBN);
-          // slot of K_n was last read by iteration n - KST
-          if (kv_it >= (uint32_t)KST &&
-              !(ok = mbar_wait(kv_done + st, ((kv_it - KST) / KST) & 1, abort_flag, status)))
-            break;
-          mbar_arrive_expect_tx(k_full + st, Cfg::kTileBytes);
-          for (int b = 0; b < D / 64; ++b)
-            tma_load_2d(sK + st * Cfg::kTileBytes + b * Cfg::kBoxBytes, &map_k, k_full + st, b * 64, row);
-          // slot of V_n was last read by iteration n - KST + 1 (PV of V_{n-KST})
-          if (kv_it + 1 >= (uint32_t)KST) {
-            const uint32_t m = kv_it + 1 - KST;
-            if (!(ok = mbar_wait(kv_done + m % KST, (m / KST) & 1, abort_flag, status))) { ++kv_it; break; }
-          }
+      while (ok) {
+        const bool has_k = kw.u < n_units, has_v = vw.u < n_units, has_q = qu < n_units;
+        if (!has_k && !has_v && !has_q) break;
+        const int64_t tK = has_k ? (int64_t)kw.it - KS : INT64_MAX;
+        const int64_t tV = has_v ? (int64_t)vw.it + 1 - VS : INT64_MAX;
+        const int64_t tQ = has_q ? (int64_t)qit0 - 1 : INT64_MAX;
+        if (tQ <= tK && tQ <= tV) {
+          const Unit U = decode_unit(qu, BH, T, c, koff);
+          if (qn > 0 && !(ok = mbar_wait(q_empty, (qn - 1) & 1, abort_flag, status))) break;
+          mbar_arrive_expect_tx(q_full, U.nt * Cfg::kTileBytes);
+          const int64_t rowbase = U.bh * (int64_t)T;
+          for (int i = 0; i < U.nt; ++i)
+            for (int b = 0; b < D / 64; ++b)
+              tma_load_2d(sQ + i * Cfg::kTileBytes + b * Cfg::kBoxBytes, &map_q, q_full, b * 64,
+                          (int)(rowbase + U.q0 + 128 * i));
+          qit0 += (uint32_t)((U.nt == 2 ? U.end[1] : U.end[0]) - U.beg[0]);
+          qu += gridDim.x;
+          ++qn;
+        } else if (tV <= tK) {
+          if (tV >= 0 && !(ok = mbar_wait(it_done + tV % KS, (uint32_t)(tV / KS) & 1, abort_flag, status))) break;
+          const int st = vw.it % VS;
+          const int row = (int)(vw.kvbase + (int64_t)vw.j * kBN);
           mbar_arrive_expect_tx(v_full + st, Cfg::kTileBytes);
           for (int b = 0; b < D / 64; ++b)
             tma_load_2d(sV + st * Cfg::kTileBytes + b * Cfg::kBoxBytes, &map_v, v_full + st, b * 64, row);
+          kv_walk_next(vw, gridDim.x, BH, T, c, koff, n_units);
+        } else {
+          if (tK >= 0 && !(ok = mbar_wait(it_done + tK % KS, (uint32_t)(tK / KS) & 1, abort_flag, status))) break;
+          const int st = kw.it % KS;
+          const int row = (int)(kw.kvbase + (int64_t)kw.j * kBN);
+          mbar_arrive_expect_tx(k_full + st, Cfg::kTileBytes);
+          for (int b = 0; b < D / 64; ++b)
+            tma_load_2d(sK + st * Cfg::kTileBytes + b * Cfg::kBoxBytes, &map_k, k_full + st, b * 64, row);
+          kv_walk_next(kw, gridDim.x, BH, T, c, koff, n_units);
         }
       }
       if (!ok) {
-        // let every copy already issued land before the CTA exits
-        for (uint32_t idx = kv_it >= (uint32_t)KST ? kv_it - KST : 0; idx < kv_it; ++idx) {
-          mbar_wait_drain(k_full + idx % KST, (idx / KST) & 1);
-          mbar_wait_drain(v_full + idx % KST, (idx / KST) & 1);
-        }
-        if (n > 0) mbar_wait_drain(q_full, (n - 1) & 1);
+        // let every copy already issued land before the CTA exits (older
+        // copies of a slot landed before its reuse was allowed)
+        for (uint32_t idx = kw.it >= (uint32_t)KS ? kw.it - KS : 0; idx < kw.it; ++idx)
+          mbar_wait_drain(k_full + idx % KS, (idx / KS) & 1);
+        for (uint32_t idx = vw.it >= (uint32_t)VS ? vw.it - VS : 0; idx < vw.it; ++idx)
+          mbar_wait_drain(v_full + idx % VS, (idx / VS) & 1);
+        if (qn > 0) mbar_wait_drain(q_full, (qn - 1) & 1);
       }
     }
     __syncwarp();
@@ -259,12 +306,12 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
         tc_fence_after();
         const int jb = U.beg[0], je = U.nt == 2 ? U.end[1] : U.end[0];
         for (int j = jb; j <= je && ok; ++j) {
-          const uint32_t stK = kv_it % KST;
+          const uint32_t stK = kv_it % KS;
           bool k_ready = false;  // K_j is waited for only right before the first QK that reads it
           const uint32_t itV = kv_it - 1;  // V_{j-1}
-          const uint32_t stV = itV % KST;
+          const uint32_t stV = itV % VS;
           if (j > jb) {
-            if (!(ok = mbar_wait(v_full + stV, (itV / KST) & 1, abort_flag, status))) break;
+            if (!(ok = mbar_wait(v_full + stV, (itV / VS) & 1, abort_flag, status))) break;
             tc_fence_after();
           }
           for (int i = 0; i < U.nt && ok; ++i) {
@@ -290,7 +337,7 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
             }
             if (j >= U.beg[i] && j < U.end[i]) {
               if (!k_ready) {
-                if (!(ok = mbar_wait(k_full + stK, (kv_it / KST) & 1, abort_flag, status))) break;
+                if (!(ok = mbar_wait(k_full + stK, (kv_it / KS) & 1, abort_flag, status))) break;
                 tc_fence_after();
                 k_ready = true;
               }
@@ -299,15 +346,15 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
               const SDesc kd = sdesc_sw128_split(ka + stK * Cfg::kTileBytes, 16, 1024);
 #pragma unroll
               for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t koff = (kk / 4) * Cfg::kBoxBytes + (kk % 4) * 32;
-                umma_ss(tmem + colS, sdesc_at(qd, koff), sdesc_at(kd, koff), idesc_qk, kk > 0 ? 1u : 0u);
+                const uint32_t kbyte = (kk / 4) * Cfg::kBoxBytes + (kk % 4) * 32;
+                umma_ss(tmem + colS, sdesc_at(qd, kbyte), sdesc_at(kd, kbyte), idesc_qk, kk > 0 ? 1u : 0u);
               }
               umma_commit(s_full + i);
             }
           }
           if (!ok) break;
           if (j < je) {
-            umma_commit(kv_done + stK);   // K_j and V_{j-1} (and a drained V of the previous unit)
+            umma_commit(it_done + stK);   // K_j and V_{j-1} (and a drained V of the previous unit)
             if (j == je - 1) umma_commit(q_empty);
             ++kv_it;
           }
@@ -325,19 +372,13 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
     const uint32_t lane_addr = tmem + ((uint32_t)((warp % 4) * 32) << 16);
     const uint32_t colS = i == 0 ? Cfg::kColS0 : Cfg::kColS1;
     const uint32_t colO = i == 0 ? Cfg::kColO0 : Cfg::kColO1;
-    uint32_t s_cnt = 0, o_cnt = 0, q_cnt = 0;
+    uint32_t s_cnt = 0, o_cnt = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const Unit U = decode_unit(u, BH, T, c, koff);
       if (i >= U.nt) continue;
       float m_ref = 0.f, l = 0.f;
-      // Key tiles where both query tiles are active: there the exp passes of
-      // the two warpgroups alternate (tile 0, tile 1, tile 0, ...), handing a
-      // token through seq[], so they do not compete for the SFU and issue
-      // slots and each one overlaps the other tile's MMAs.
-      const int pb = U.nt == 2 ? U.beg[1] : 0, pe = U.nt == 2 ? U.end[0] : 0;
       for (int j = U.beg[i]; j < U.end[i]; ++j) {
-        const bool paired = j >= pb && j < pe;
         ok = __all_sync(0xffffffffu, mbar_wait(s_full + i, s_cnt & 1, abort_flag, status));
         if (!ok) break;
         ++s_cnt;
@@ -369,12 +410,17 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           mt = fmax3(mt, fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7])), -INFINITY);
         }
         const float m2 = mt * kLog2e;
-        if (j == U.beg[i]) {
-          m_ref = m2;
-        } else if (m2 > m_ref + 8.f) {
-          const float scale = ex2(m_ref - m2);
-          l *= scale;
-          m_ref = m2;
+        const bool grow = j != U.beg[i] && m2 > m_ref + 8.f;
+        if (j == U.beg[i]) m_ref = m2;
+        // O is rescaled with warp-collective TMEM loads and stores, so the
+        // whole warp takes this branch when any of its rows needs it (the
+        // other rows scale by 1)
+        if (__any_sync(0xffffffffu, grow)) {
+          const float scale = grow ? ex2(m_ref - m2) : 1.f;
+          if (grow) {
+            l *= scale;
+            m_ref = m2;
+          }
 #pragma unroll 1
           for (int cb = 0; cb < D / 32; ++cb) {
             uint32_t o[32];
@@ -384,11 +430,6 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
             for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * scale);
             tmem_st32(lane_addr + colO + cb * 32, o);
           }
-        }
-        if (paired && (i == 1 || j > pb)) {
-          ok = __all_sync(0xffffffffu, mbar_wait(seq + i, q_cnt & 1, abort_flag, status));
-          if (!ok) break;
-          ++q_cnt;
         }
         // pass 2: p = 2^(s log2e - m_ref) in chunks of 32 columns (the next
         // chunk's TMEM load is in flight while this one is computed).  The
@@ -414,15 +455,6 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           for (int x = 0; x < 16; ++x) {
             const uint64_t a2 = ffma2(pack2(__uint_as_float(cur[2 * x]), __uint_as_float(cur[2 * x + 1])), l2e2, nm2);
             uint64_t p2;
-#if GECKO_SCA_H2EXP
-            {
-              // one packed f16 SFU op for the pair; P is rounded to bf16 anyway
-              float a0, a1, e0, e1;
-              unpack2(a2, a0, a1);
-              ex2_h2(a0, a1, e0, e1);
-              p2 = pack2(e0, e1);
-            }
-#else
             if (x % 8 < kSfuPairs) {
               float a0, a1;
               unpack2(a2, a0, a1);
@@ -430,7 +462,6 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
             } else {
               p2 = exp2_poly2(a2);
             }
-#endif
             acc2[x & 1] = fadd2(acc2[x & 1], p2);
             float p0, p1;
             unpack2(p2, p0, p1);
@@ -443,10 +474,6 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           }
         }
         tmem_wait_st();
-        if (paired && (i == 0 || j + 1 < pe)) {
-          __syncwarp();
-          if (lane == 0) mbar_arrive(seq + (1 - i));
-        }
         {
           float a0, a1, b0, b1;
           unpack2(acc2[0], a0, a1);
