@@ -120,3 +120,58 @@ def make_inputs(w: Workload, device="cpu", seed_offset: int = 0) -> dict:
                     slab = sc[h] * _unit_rows(sg, T, d, device) + off[h]
                 out[name][b, h].copy_(slab.to(dt))
     return out
+
+
+# --------------------------------------------------------------------------
+# CEMA (the complex damped EMA that produces the layer input): seeded
+# synthetic inputs.  x is the layer input (standard normal); the per-(d, j)
+# parameters are drawn as a trained layer would hold them after its sigmoids
+# (alpha, delta in (0, 1)); document starts, where the recurrence restarts,
+# are Bernoulli with mean document length `mean_doc` (0: one document).
+# --------------------------------------------------------------------------
+
+@dataclasses.dataclass(frozen=True)
+class CemaWorkload:
+    """One synthetic CEMA workload: x [B, L, D], h hidden dimensions per feature."""
+    name: str
+    wid: int
+    dtype: str               # "f32" or "bf16"
+    B: int
+    L: int
+    D: int
+    h: int = 16
+    mean_doc: int = 0        # mean document length for resets (0 = no resets)
+
+    @property
+    def torch_dtype(self):
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+
+# small parity cases (ragged D, resets) and the 7B-width case (D = 4096, h = 16)
+# over the same 32K tokens as the attention workload
+CEMA_WORKLOADS = {
+    "cema_f32_small": CemaWorkload("cema_f32_small", 21, "f32", 2, 1000, 96, 16, mean_doc=300),
+    "cema_bf16_small": CemaWorkload("cema_bf16_small", 22, "bf16", 2, 2304, 160, 16, mean_doc=700),
+    "cema_bf16_7b_32k": CemaWorkload("cema_bf16_7b_32k", 23, "bf16", 1, 32768, 4096, 16),
+}
+
+
+def make_cema_inputs(w: CemaWorkload, device="cpu", seed_offset: int = 0) -> dict:
+    """x [B, L, D] (workload dtype); alpha, delta, theta, beta [D, h] fp32;
+    eta [D, h, 2] fp32 (real, imaginary); reset [B, L] uint8 (1 = a document
+    starts at this token)."""
+    gen = torch.Generator(device=device).manual_seed(100 * w.wid + seed_offset)
+    f32 = dict(generator=gen, device=device, dtype=torch.float32)
+    out = {
+        "x": torch.randn(w.B, w.L, w.D, **f32).to(w.torch_dtype),
+        "alpha": torch.sigmoid(torch.randn(w.D, w.h, **f32) - 2.0),
+        "delta": torch.sigmoid(torch.randn(w.D, w.h, **f32)),
+        "theta": torch.rand(w.D, w.h, **f32) * 3.141592653589793,
+        "beta": torch.randn(w.D, w.h, **f32),
+        "eta": torch.randn(w.D, w.h, 2, **f32) / w.h ** 0.5,
+    }
+    if w.mean_doc > 0:
+        out["reset"] = (torch.rand(w.B, w.L, **f32) < 1.0 / w.mean_doc).to(torch.uint8)
+    else:
+        out["reset"] = None
+    return out
