@@ -17,6 +17,11 @@ over ranks; rank 0 prints one JSON line.
 
 `--impl reference` times the CPU oracle (fp64 NumPy, the machine's host cores) on
 bounded samples of the same workload instead.
+
+`--op cema` measures the CEMA recurrence (gecko_cema_forward) instead, on
+x [1, 32768, 4096] bf16 with h = 16, and prints its own JSON line (an FP32
+ALU-bound kernel: roofline against the FP32 FMA rate of 148 SMs x 128 lanes
+at the sampled SM clock).
 """
 from __future__ import annotations
 
@@ -36,7 +41,8 @@ if ROOT not in sys.path:
 
 import torch  # noqa: E402
 
-from long_context_sequence_sca_b200.inputs import WORKLOADS, Workload, make_inputs  # noqa: E402
+from long_context_sequence_sca_b200.inputs import (  # noqa: E402
+    CEMA_WORKLOADS, WORKLOADS, CemaWorkload, Workload, make_cema_inputs, make_inputs)
 
 DEFAULT_WORKLOAD = "bf16_h32_c4096"
 METRIC = "tokens/s fused SCA+AWM fwd (bf16,H=32,d=128,c=4096); % bf16 TC peak"
@@ -429,6 +435,121 @@ def run_reference(args, w: Workload) -> dict:
     }
 
 
+# ------------------------------------------------------------------ CEMA --
+
+CEMA_METRIC = "tokens/s CEMA fwd (bf16, D=4096, h=16, 32K tokens)"
+CEMA_FLOP_PER_ELEMENT = 12 * 16   # per hidden: complex q*h (6) + alpha beta x (1) + add (1) + Re(eta h) and sum (4)
+SM_COUNT, FP32_LANES = 148, 128
+
+
+def cema_oracle_sample(w: CemaWorkload, x, n_feat: int):
+    """Time the fp64 CEMA oracle on the first n_feat features of every token."""
+    from oracle import cema_oracle as C
+    f = slice(0, n_feat)
+    xs = x["x"][:, :, f].double().cpu().numpy()
+    prm = {k: x[k][f].double().cpu().numpy() for k in ("alpha", "delta", "theta", "beta")}
+    e = x["eta"][f].double().cpu().numpy()
+    t0 = time.perf_counter()
+    C.cema_forward(xs, prm["alpha"], prm["delta"], prm["theta"], prm["beta"], e[..., 0] + 1j * e[..., 1])
+    secs = time.perf_counter() - t0
+    return w.B * w.L * n_feat / w.D / secs, secs
+
+
+def run_cema(args, ws: int, rank: int, local: int) -> dict:
+    from long_context_sequence_sca_b200 import lib as L
+    L.load()
+    w = CEMA_WORKLOADS["cema_bf16_7b_32k"]
+    x = make_cema_inputs(w, device="cuda", seed_offset=1000 * rank)
+    y = torch.empty_like(x["x"])
+    stream = torch.cuda.current_stream()
+    prm = (x["alpha"], x["delta"], x["theta"], x["beta"], x["eta"])
+
+    def step(xin, yout):
+        L.cema_forward(xin, *prm, reset=x["reset"], y=yout, stream=stream)
+
+    for _ in range(args.warmup):
+        step(x["x"], y)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+
+    def timed():
+        barrier(ws)
+        torch.cuda.synchronize()
+        sampler.start()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step(x["x"], y)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ck = sampler.stop()
+        barrier(ws)
+        return e0.elapsed_time(e1) / args.steps, ck
+
+    ms_local, ck = timed()
+    note = None
+    if clocks_rejected(ck):
+        note = f"re-measured once: first run saw clocks {ck}"
+        ms_local, ck = timed()
+    tokens = w.B * w.L
+    agg = aggregate(ms_local, tokens, ws)
+    op_ms = max_over_ranks(ms_local, ws)
+    flop = CEMA_FLOP_PER_ELEMENT * w.B * w.L * w.D
+    mhz = ck.get("sm_mhz") or ck.get("sm_max_mhz") or 1965
+    peak = SM_COUNT * FP32_LANES * 2 * mhz * 1e6 / 1e12
+    achieved = flop / (op_ms / 1e3) / 1e12
+    nb = x["x"].numel() * x["x"].element_size()
+    out = {
+        "metric": CEMA_METRIC, "value": round(agg["value"], 1), "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(agg["ms_per_step"], 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded generator; no dataset)",
+        "config": {"workload": w.name, "B": w.B, "L": w.L, "D": w.D, "h": w.h,
+                   "l2": f"x larger than L2 ({nb / 1e9:.2f} GB), no flush",
+                   "parallelism": f"replicas x{ws}"},
+        "roofline": {"bound": "alu", "kernel": "cema_local_kernel + cema_carry_kernel + cema_out_kernel (one op)",
+                     "achieved": round(achieved, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4),
+                     "peak_kind": f"derived: {SM_COUNT} SMs x {FP32_LANES} FP32 FMA/clk x 2 flop x {mhz} MHz",
+                     "traffic": None, "launch_ms": round(op_ms, 4), "algorithmic_flop_per_launch": flop},
+        "clocks": ck,
+        "gpu_launches": 3 * args.steps,
+    }
+    if note:
+        out["note"] = note
+    if not args.no_e2e:
+        hx = x["x"].cpu().pin_memory()
+        hy = torch.empty_like(hx).pin_memory()
+        dx = torch.empty_like(x["x"])
+        steps = max(1, min(args.steps, 10))
+
+        def e2e_step():
+            dx.copy_(hx, non_blocking=True)
+            step(dx, y)
+            hy.copy_(y, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(ws)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(ws)
+        ea = aggregate(e0.elapsed_time(e1) / steps, tokens, ws)
+        out["e2e"] = {"value": round(ea["value"], 1), "unit": "tokens/s", "h2d_bytes_per_step": nb,
+                      "d2h_bytes_per_step": nb, "steps": steps, "ms_per_step": round(ea["ms_per_step"], 3)}
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        n_feat = 1024
+        val, secs = cema_oracle_sample(w, x, n_feat)
+        out["cpu_baseline"] = {"value": round(val, 2), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                               "sample": f"fp64 CEMA oracle on the first {n_feat} of {w.D} features of all "
+                                         f"{w.L} tokens in {secs:.1f} s (tokens scaled by {n_feat}/{w.D})"}
+    return out
+
+
 def summarize_launches(path: str) -> str:
     """Per-kernel launches, total time and share from an ncu launch-list CSV
     (`ncu --metrics gpu__time_duration.sum --csv`)."""
@@ -468,6 +589,8 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", choices=("sca_awm", "cema"), default="sca_awm",
+                    help="sca_awm: the fused SCA + AWM forward (default); cema: the CEMA recurrence")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -484,7 +607,7 @@ def main(argv=None):
     if ws != args.gpus and rank == 0:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE {ws}", file=sys.stderr)
     try:
-        out = run_gecko(args, w, ws, rank, local)
+        out = run_cema(args, ws, rank, local) if args.op == "cema" else run_gecko(args, w, ws, rank, local)
         if rank == 0:
             print(json.dumps(out), flush=True)
     finally:

@@ -196,6 +196,43 @@ int gecko_device_status(void* stream);
 int gecko_timing_enable(int enable);
 int gecko_timing_read(float* ms_per_stage, int capacity, int* n_calls);
 
+/*
+ * gecko_cema_forward - CEMA, the complex multi-dimensional damped
+ * exponential moving average that produces the layer input X' = CEMA(X)
+ * (Gecko digest, background section on the exponential moving average;
+ * paperlayer.ai summary, section 2.1 and Appendix B.1):
+ *   u_t[d, j] = beta[d, j] x_t[d]                               (j < h = 16)
+ *   h_t[d, j] = alpha u_t + (1 - alpha delta)(cos theta + i sin theta) h_{t-1}
+ *   y_t[d]    = Re(sum_j eta[d, j] h_t[d, j])
+ * A document start at token t (reset) drops the second term: h_t = alpha u_t.
+ * The expansion by beta and the projection by eta are the plainest readings
+ * of the pages' "expands each input dimension into h dimensions" and
+ * "projected back to a one-dimensional output"; no skip term is added.
+ *
+ *   x, y          : [B, L, D] dtype `dtype` (device); y may equal x.
+ *   alpha, delta, theta, beta : [D, h] fp32 (device), as they enter the
+ *                   recurrence (alpha, delta in (0, 1]).
+ *   eta           : [D, h, 2] fp32 (device), real and imaginary parts.
+ *   reset         : [B, L] uint8 (device) or NULL; non-zero = a document
+ *                   starts at that token.
+ *   state_in      : [B, D, h, 2] fp32 (device) h_{-1}, or NULL for zero.
+ *   state_out     : [B, D, h, 2] fp32 (device) receives h_{L-1}, or NULL; may
+ *                   equal state_in.  Chaining state_out into state_in runs a
+ *                   long sequence in segments.
+ *   h must be 16.  Requires B <= 65535 and L <= 65535 * 256; every pointer
+ *   16-byte aligned.
+ *
+ * Ownership: a per-device workspace of 2 * B * ceil(L / 256) * D * h complex
+ * fp32 (chunk states), grown on demand on `stream` and freed by
+ * gecko_release().  Asynchronous on `stream`; argument errors are detected on
+ * the host before anything is launched.  Returns GECKO_OK, GECKO_ERR_ARG,
+ * GECKO_ERR_SHAPE, GECKO_ERR_ALIGN, GECKO_ERR_ALLOC or GECKO_ERR_CUDA.
+ */
+int gecko_cema_forward(const void* x, void* y, const float* alpha, const float* delta,
+                       const float* theta, const float* beta, const float* eta,
+                       const uint8_t* reset, const float* state_in, float* state_out,
+                       int64_t B, int64_t L, int64_t D, int64_t h, int dtype, void* stream);
+
 /* Thread-local message describing the last non-zero status of this thread. */
 const char* gecko_last_error(void);
 

@@ -85,6 +85,8 @@ struct DeviceState {
   void* noalloc_scratch = nullptr;  // device address of g_noalloc_scratch
   void* state = nullptr;             // copy of a carried state (continued sequences)
   size_t state_bytes = 0;
+  void* cema_ws = nullptr;           // CEMA chunk states
+  size_t cema_ws_bytes = 0;
 };
 
 std::mutex g_mu;
@@ -359,16 +361,19 @@ extern "C" void gecko_release(void) {
   int cur = 0;
   cudaGetDevice(&cur);
   for (auto& kv : g_dev) {
-    if (kv.second.ws || kv.second.state) {
+    if (kv.second.ws || kv.second.state || kv.second.cema_ws) {
       cudaSetDevice(kv.first);
       cudaDeviceSynchronize();
       if (kv.second.ws) cudaFree(kv.second.ws);
       if (kv.second.state) cudaFree(kv.second.state);
+      if (kv.second.cema_ws) cudaFree(kv.second.cema_ws);
     }
     kv.second.ws = nullptr;
     kv.second.ws_bytes = 0;
     kv.second.state = nullptr;
     kv.second.state_bytes = 0;
+    kv.second.cema_ws = nullptr;
+    kv.second.cema_ws_bytes = 0;
     kv.second.have_state = false;
   }
   cudaSetDevice(cur);
@@ -440,4 +445,36 @@ extern "C" int gecko_sca_awm_forward_noalloc(const void* q, const void* k, const
     return rc;
   if ((rc = check_cuda(use_tc ? launch_sca_tc(p, st) : launch_sca_simt(p, st), "sca"))) return rc;
   return GECKO_OK;
+}
+
+extern "C" int gecko_cema_forward(const void* x, void* y, const float* alpha, const float* delta,
+                                  const float* theta, const float* beta, const float* eta, const uint8_t* reset,
+                                  const float* state_in, float* state_out, int64_t B, int64_t L, int64_t D,
+                                  int64_t h, int dtype, void* stream) {
+  const void* ptrs[7] = {x, y, alpha, delta, theta, beta, eta};
+  for (int i = 0; i < 7; ++i)
+    if (!ptrs[i]) return fail(GECKO_ERR_ARG, "tensor argument %d is NULL", i);
+  if (dtype != GECKO_F32 && dtype != GECKO_BF16) return fail(GECKO_ERR_ARG, "unknown dtype %d", dtype);
+  if (B < 1 || L < 1 || D < 1 || h < 1)
+    return fail(GECKO_ERR_ARG, "sizes must be >= 1 (B=%lld L=%lld D=%lld h=%lld)", (long long)B, (long long)L,
+                (long long)D, (long long)h);
+  if (h != cema_hidden()) return fail(GECKO_ERR_SHAPE, "h must be %d (got %lld)", cema_hidden(), (long long)h);
+  if ((long double)B * L * D * 4 > 4.0e18L) return fail(GECKO_ERR_SHAPE, "tensor size overflows");
+  // grid: (ceil(D / 128), chunks, B) within CUDA's y and z limits
+  if (cema_chunks(L) > 65535 || B > 65535 || D > (int64_t(1) << 30))
+    return fail(GECKO_ERR_SHAPE, "size exceeds kernel index range (B <= 65535, L <= 65535 * 256)");
+  const void* all[10] = {x, y, alpha, delta, theta, beta, eta, reset, state_in, state_out};
+  for (int i = 0; i < 10; ++i)
+    if (reinterpret_cast<uintptr_t>(all[i]) % 16 != 0)
+      return fail(GECKO_ERR_ALIGN, "argument %d is not 16-byte aligned", i);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int dev = 0, rc;
+  if ((rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice"))) return rc;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState* ds = nullptr;
+  if ((rc = device_state(dev, &ds))) return rc;
+  if ((rc = ensure_buffer(&ds->cema_ws, &ds->cema_ws_bytes, cema_workspace_bytes(B, L, D), st, "CEMA workspace")))
+    return rc;
+  CemaProblem p{x, y, alpha, delta, theta, beta, eta, reset, state_in, state_out, B, L, D, dtype};
+  return check_cuda(launch_cema(p, carve_cema_workspace(ds->cema_ws, B, L, D), st), "CEMA launch");
 }

@@ -58,4 +58,32 @@ cudaError_t launch_sca_tc(const Problem& p, cudaStream_t st);
 cudaError_t launch_awm_chunk_tc(const Problem& p, const Workspace& w, cudaStream_t st);
 cudaError_t launch_awm_readout_tc(const Problem& p, const Workspace& w, cudaStream_t st);
 
+// ---------------------------------------------------------------- CEMA --
+
+// One validated CEMA call: x, y [B, L, D] (dtype); alpha, delta, theta,
+// beta [D, 16] fp32; eta [D, 16, 2] fp32; reset [B, L] uint8 or null;
+// state_in / state_out [B, D, 16, 2] fp32 or null (device).
+struct CemaProblem {
+  const void* x;
+  void* y;
+  const float *alpha, *delta, *theta, *beta, *eta;
+  const uint8_t* reset;
+  const float* state_in;
+  float* state_out;
+  int64_t B, L, D;
+  int dtype;
+};
+
+struct CemaWorkspace {
+  float2* Bc;            // [B, C, D, 16]  end state of each chunk scanned from zero
+  float2* Hin;           // [B, C, D, 16]  state entering each chunk
+  uint8_t* chunk_reset;  // [B, C]  1 if the chunk holds a document start
+};
+
+int cema_hidden();                       // hidden dimensions per feature (16)
+int64_t cema_chunks(int64_t L);          // chunks of the scan
+size_t cema_workspace_bytes(int64_t B, int64_t L, int64_t D);
+CemaWorkspace carve_cema_workspace(void* base, int64_t B, int64_t L, int64_t D);
+cudaError_t launch_cema(const CemaProblem& p, const CemaWorkspace& w, cudaStream_t st);
+
 }  // namespace gecko

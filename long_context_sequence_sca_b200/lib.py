@@ -19,6 +19,7 @@ EXPORTS = (
     "gecko_sca_awm_forward_continue",
     "gecko_sca_awm_forward_noalloc",
     "gecko_awm_state",
+    "gecko_cema_forward",
     "gecko_device_status",
     "gecko_timing_enable",
     "gecko_timing_read",
@@ -63,6 +64,8 @@ def load() -> ctypes.CDLL:
     lib.gecko_sca_awm_forward_noalloc.restype = ctypes.c_int
     lib.gecko_awm_state.argtypes = [vp, vp, i64, i64, i64, vp]
     lib.gecko_awm_state.restype = ctypes.c_int
+    lib.gecko_cema_forward.argtypes = [vp] * 10 + [i64] * 4 + [ctypes.c_int, vp]
+    lib.gecko_cema_forward.restype = ctypes.c_int
     lib.gecko_device_status.argtypes = [vp]
     lib.gecko_device_status.restype = ctypes.c_int
     lib.gecko_timing_enable.argtypes = [ctypes.c_int]
@@ -110,6 +113,13 @@ def gecko_sca_awm_forward_noalloc(q, k, v, qm, km, out_sca, out_mem, B, H, T, c,
 
 def gecko_awm_state(M_out, logz_out, B, H, d, stream) -> int:
     return load().gecko_awm_state(M_out, logz_out, B, H, d, stream)
+
+
+def gecko_cema_forward(x, y, alpha, delta, theta, beta, eta, reset, state_in, state_out, B, L, D, h, dtype,
+                       stream) -> int:
+    """Direct call of the CEMA entry point with integer pointers (0 = NULL)."""
+    return load().gecko_cema_forward(x, y, alpha, delta, theta, beta, eta, reset, state_in, state_out,
+                                     B, L, D, h, dtype, stream)
 
 
 def gecko_device_status(stream) -> int:
@@ -220,3 +230,28 @@ def timing_read():
     n = ctypes.c_int(0)
     _check(gecko_timing_read(buf, len(STAGES), ctypes.byref(n)))
     return {name: float(buf[i]) for i, name in enumerate(STAGES)}, int(n.value)
+
+
+def cema_forward(x, alpha, delta, theta, beta, eta, reset=None, state_in=None, return_state=False, y=None,
+                 stream=None):
+    """CEMA over x [B, L, D] (float32 or bfloat16 CUDA tensor).  alpha,
+    delta, theta, beta: [D, 16] float32; eta: [D, 16, 2] float32 (real,
+    imaginary); reset: [B, L] uint8 or None; state_in: [B, D, 16, 2] float32
+    or None.  Returns y (and the final state [B, D, 16, 2] if return_state)."""
+    if not (isinstance(x, torch.Tensor) and x.is_cuda and x.is_contiguous() and x.dim() == 3 and x.dtype in _DT):
+        raise ValueError("x must be a contiguous [B, L, D] float32 or bfloat16 CUDA tensor")
+    B, L, D = x.shape
+    params = (alpha, delta, theta, beta, eta)
+    for prm in params:
+        if not (isinstance(prm, torch.Tensor) and prm.is_cuda and prm.is_contiguous() and prm.dtype == torch.float32):
+            raise ValueError("parameters must be contiguous float32 CUDA tensors")
+    h = alpha.shape[-1]
+    if y is None:
+        y = torch.empty_like(x)
+    state_out = torch.empty(B, D, h, 2, dtype=torch.float32, device=x.device) if return_state else None
+    ptr = lambda t: 0 if t is None else t.data_ptr()
+    with torch.cuda.device(x.device):
+        rc = gecko_cema_forward(x.data_ptr(), y.data_ptr(), *(prm.data_ptr() for prm in params), ptr(reset),
+                                ptr(state_in), ptr(state_out), B, L, D, h, _DT[x.dtype], _stream_handle(stream))
+    _check(rc)
+    return (y, state_out) if return_state else y

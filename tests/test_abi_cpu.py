@@ -69,3 +69,27 @@ def test_host_validation_rejects(so, kw, code):
 
 def test_state_query_rejects_null(so):
     assert L.gecko_awm_state(0, 0, 1, 1, 64, None) == 1
+
+
+def _cema(ptrs=None, B=1, L=1000, D=64, h=16, dtype=1):
+    ptrs = ptrs or [FAKE] * 7 + [0, 0, 0]
+    return L_cema(ptrs, B, L, D, h, dtype)
+
+
+def L_cema(ptrs, B, Lt, D, h, dtype):
+    return L.gecko_cema_forward(*ptrs, B, Lt, D, h, dtype, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ptrs=[FAKE, 0] + [FAKE] * 5 + [0, 0, 0]), 1),   # y NULL
+    (dict(dtype=3), 1),
+    (dict(L=0), 1),
+    (dict(h=8), 2),                                         # h must be 16
+    (dict(L=65536 * 256), 2),                               # more chunks than grid.y holds
+    (dict(B=70000), 2),
+    (dict(ptrs=[FAKE] * 7 + [FAKE + 4, 0, 0]), 3),          # reset misaligned
+    (dict(ptrs=[FAKE] * 7 + [0, 0, FAKE + 8]), 3),          # state_out misaligned
+])
+def test_cema_host_validation_rejects(so, kw, code):
+    assert _cema(**kw) == code
+    assert L.gecko_last_error()
