@@ -252,28 +252,40 @@ def blas_threads() -> int:
 
 # --------------------------------------------------------- traffic record --
 
-def sca_source_hash() -> str:
+def source_hash(files=("sca_tc.cu", "common.cuh")) -> str:
     h = hashlib.sha1()
-    for f in ("sca_tc.cu", "common.cuh"):
+    for f in files:
         with open(os.path.join(ROOT, "long_context_sequence_sca_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:12]
 
 
-def recorded_traffic(w: Workload):
-    """DRAM bytes per SCA launch from the committed ncu summary, or None if
-    the summary is missing, for another workload, or older than the kernel
+def sca_source_hash() -> str:
+    return source_hash(("sca_tc.cu", "common.cuh"))
+
+
+CEMA_PROFILE = os.path.join(ROOT, "profiles", "cema_bf16_7b_32k.md")
+
+
+def cema_source_hash() -> str:
+    return source_hash(("cema.cu", "common.cuh"))
+
+
+def recorded_traffic(w: Workload, path: str = SCA_PROFILE, src_hash=None):
+    """DRAM bytes per launch from a committed ncu summary, or None if the
+    summary is missing, for another workload, or older than the kernel
     source.  The summary carries `key: value` lines for workload,
     source_hash and dram_bytes_per_launch."""
-    if not os.path.exists(SCA_PROFILE):
+    if not os.path.exists(path):
         return None
+    src_hash = src_hash or sca_source_hash()
     rec = {}
-    with open(SCA_PROFILE) as f:
+    with open(path) as f:
         for line in f:
             if ":" in line and not line.startswith(("#", "|", " ")):
                 k_, v_ = line.split(":", 1)
                 rec[k_.strip()] = v_.strip()
-    if rec.get("source_hash") != sca_source_hash() or rec.get("workload") != w.name:
+    if rec.get("source_hash") != src_hash or rec.get("workload") != w.name:
         return None
     try:
         return int(rec["dram_bytes_per_launch"])
@@ -507,11 +519,12 @@ def run_cema(args, ws: int, rank: int, local: int) -> dict:
         "config": {"workload": w.name, "B": w.B, "L": w.L, "D": w.D, "h": w.h,
                    "l2": f"x larger than L2 ({nb / 1e9:.2f} GB), no flush",
                    "parallelism": f"replicas x{ws}"},
-        "roofline": {"bound": "alu", "kernel": "cema_local_kernel + cema_carry_kernel + cema_out_kernel (one op)",
+        "roofline": {"bound": "alu", "kernel": "cema_local_tma_kernel + cema_carry_kernel + cema_out_tma_kernel (one op)",
                      "achieved": round(achieved, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4),
                      "peak_kind": f"derived: {SM_COUNT} SMs x {FP32_LANES} FP32 FMA/clk x 2 flop x {mhz} MHz",
-                     "traffic": None, "launch_ms": round(op_ms, 4), "algorithmic_flop_per_launch": flop},
+                     "traffic": recorded_traffic(w, CEMA_PROFILE, cema_source_hash()), "launch_ms": round(op_ms, 4),
+                     "algorithmic_flop_per_launch": flop},
         "clocks": ck,
         "gpu_launches": 3 * args.steps,
     }

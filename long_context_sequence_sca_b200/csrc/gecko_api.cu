@@ -475,6 +475,6 @@ extern "C" int gecko_cema_forward(const void* x, void* y, const float* alpha, co
   if ((rc = device_state(dev, &ds))) return rc;
   if ((rc = ensure_buffer(&ds->cema_ws, &ds->cema_ws_bytes, cema_workspace_bytes(B, L, D), st, "CEMA workspace")))
     return rc;
-  CemaProblem p{x, y, alpha, delta, theta, beta, eta, reset, state_in, state_out, B, L, D, dtype};
+  CemaProblem p{x, y, alpha, delta, theta, beta, eta, reset, state_in, state_out, B, L, D, dtype, ds->status};
   return check_cuda(launch_cema(p, carve_cema_workspace(ds->cema_ws, B, L, D), st), "CEMA launch");
 }

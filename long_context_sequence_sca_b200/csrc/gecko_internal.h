@@ -72,6 +72,7 @@ struct CemaProblem {
   float* state_out;
   int64_t B, L, D;
   int dtype;
+  int* status;   // device status word (bounded waits that ran out)
 };
 
 struct CemaWorkspace {

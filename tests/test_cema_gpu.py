@@ -124,3 +124,21 @@ def test_seven_b_width_sampled_features(L):
     _close(y[:, :, feats].double().cpu().numpy(), ry, TOL["bf16"], "y (sampled features)")
     got = st[:, feats].double().cpu().numpy()
     _close(got[..., 0] + 1j * got[..., 1], rst, TOL["f32"], "final state (sampled features)")
+
+
+@pytest.mark.parametrize("w,plain", [
+    (CemaWorkload("cema_bf16_d100", 34, "bf16", 2, 700, 100, mean_doc=250), False),   # D % 8 != 0: plain loads
+    (CemaWorkload("cema_bf16_plain", 35, "bf16", 1, 900, 136, mean_doc=300), True),   # plain path forced
+    (CemaWorkload("cema_bf16_tma", 36, "bf16", 3, 777, 264, mean_doc=300), False),    # TMA path, ragged L and D
+], ids=lambda v: getattr(v, "name", str(v)))
+def test_bf16_paths(L, w, plain, monkeypatch):
+    if plain:
+        monkeypatch.setenv("GECKO_CEMA_PLAIN", "1")
+    inp = make_cema_inputs(w, device="cuda")
+    y, st = _run(L, inp, return_state=True)
+    torch.cuda.synchronize()
+    assert L.device_status() == 0
+    ry, rst = _oracle(inp)
+    _close(y.double().cpu().numpy(), ry, TOL["bf16"], "y")
+    got = st.double().cpu().numpy()
+    _close(got[..., 0] + 1j * got[..., 1], rst, TOL["f32"], "final state")
