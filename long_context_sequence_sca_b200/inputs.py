@@ -175,3 +175,50 @@ def make_cema_inputs(w: CemaWorkload, device="cpu", seed_offset: int = 0) -> dic
     else:
         out["reset"] = None
     return out
+
+
+# --------------------------------------------------------------------------
+# Timestep decay normalisation: x is the layer input (standard normal with a
+# slowly drifting per-group offset and scale, so the decayed statistics have
+# something to track); gamma, bias per feature; G groups of D / G features.
+# --------------------------------------------------------------------------
+
+@dataclasses.dataclass(frozen=True)
+class NormWorkload:
+    """One synthetic timestep-decay-normalisation workload."""
+    name: str
+    wid: int
+    dtype: str
+    B: int
+    L: int
+    D: int
+    G: int
+    beta1: float = 0.99
+    beta2: float = 0.999
+    eps: float = 1e-5
+
+    @property
+    def torch_dtype(self):
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+
+NORM_WORKLOADS = {
+    "tdnorm_f32_small": NormWorkload("tdnorm_f32_small", 51, "f32", 2, 700, 96, 4),
+    "tdnorm_bf16_small": NormWorkload("tdnorm_bf16_small", 52, "bf16", 2, 1500, 256, 8, beta1=0.9, beta2=0.99),
+    "tdnorm_bf16_7b_32k": NormWorkload("tdnorm_bf16_7b_32k", 53, "bf16", 1, 32768, 4096, 32),
+}
+
+
+def make_norm_inputs(w: NormWorkload, device="cpu", seed_offset: int = 0) -> dict:
+    """x [B, L, D] (workload dtype); gamma, bias [D] fp32."""
+    gen = torch.Generator(device=device).manual_seed(100 * w.wid + seed_offset)
+    f32 = dict(generator=gen, device=device, dtype=torch.float32)
+    t = torch.arange(w.L, device=device, dtype=torch.float32)[None, :, None]
+    drift_off = 0.5 * torch.sin(t / 997.0 + torch.rand(w.B, 1, w.G, **f32) * 6.283)
+    drift_scl = 1.0 + 0.3 * torch.cos(t / 1777.0 + torch.rand(w.B, 1, w.G, **f32) * 6.283)
+    x = torch.randn(w.B, w.L, w.G, w.D // w.G, **f32) * drift_scl[..., None] + drift_off[..., None]
+    return {
+        "x": x.reshape(w.B, w.L, w.D).to(w.torch_dtype),
+        "gamma": 1.0 + 0.1 * torch.randn(w.D, **f32),
+        "bias": 0.1 * torch.randn(w.D, **f32),
+    }
