@@ -18,7 +18,8 @@ over ranks; rank 0 prints one JSON line.
 `--impl reference` times the CPU oracle (fp64 NumPy, the machine's host cores) on
 bounded samples of the same workload instead.
 
-`--op cema` measures the CEMA recurrence (gecko_cema_forward) instead, on
+`--op tdnorm` measures timestep decay normalisation on the same x shape
+(HBM roofline).  `--op cema` measures the CEMA recurrence (gecko_cema_forward) instead, on
 x [1, 32768, 4096] bf16 with h = 16, and prints its own JSON line (an FP32
 ALU-bound kernel: roofline against the FP32 FMA rate of 148 SMs x 128 lanes
 at the sampled SM clock).
@@ -42,7 +43,8 @@ if ROOT not in sys.path:
 import torch  # noqa: E402
 
 from long_context_sequence_sca_b200.inputs import (  # noqa: E402
-    CEMA_WORKLOADS, WORKLOADS, CemaWorkload, Workload, make_cema_inputs, make_inputs)
+    CEMA_WORKLOADS, NORM_WORKLOADS, WORKLOADS, CemaWorkload, NormWorkload, Workload, make_cema_inputs, make_inputs,
+    make_norm_inputs)
 
 DEFAULT_WORKLOAD = "bf16_h32_c4096"
 METRIC = "tokens/s fused SCA+AWM fwd (bf16,H=32,d=128,c=4096); % bf16 TC peak"
@@ -265,6 +267,11 @@ def sca_source_hash() -> str:
 
 
 CEMA_PROFILE = os.path.join(ROOT, "profiles", "cema_bf16_7b_32k.md")
+NORM_PROFILE = os.path.join(ROOT, "profiles", "tdnorm_bf16_7b_32k.md")
+
+
+def norm_source_hash() -> str:
+    return source_hash(("tdnorm.cu", "common.cuh"))
 
 
 def cema_source_hash() -> str:
@@ -563,6 +570,109 @@ def run_cema(args, ws: int, rank: int, local: int) -> dict:
     return out
 
 
+# ------------------------------------------------ timestep decay norm --
+
+NORM_METRIC = "tokens/s timestep-decay norm fwd (bf16, D=4096, G=32, 32K tokens)"
+
+
+def time_steps(args, ws, local, step, stream):
+    """Warm up, then time args.steps calls of step() between CUDA events on
+    `stream` (barriers and synchronisation on both sides), sampling clocks;
+    re-measure once if the clocks are rejected.  Returns (ms, clocks, note)."""
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+
+    def timed():
+        barrier(ws)
+        torch.cuda.synchronize()
+        sampler.start()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ck = sampler.stop()
+        barrier(ws)
+        return e0.elapsed_time(e1) / args.steps, ck
+
+    ms, ck = timed()
+    note = None
+    if clocks_rejected(ck):
+        note = f"re-measured once: first run saw clocks {ck}"
+        ms, ck = timed()
+    return ms, ck, note
+
+
+def run_tdnorm(args, ws: int, rank: int, local: int) -> dict:
+    from long_context_sequence_sca_b200 import lib as L
+    from oracle import tdnorm_oracle as N
+    L.load()
+    w = NORM_WORKLOADS["tdnorm_bf16_7b_32k"]
+    x = make_norm_inputs(w, device="cuda", seed_offset=1000 * rank)
+    y = torch.empty_like(x["x"])
+    stream = torch.cuda.current_stream()
+
+    def step(xin=x["x"]):
+        L.tdnorm_forward(xin, x["gamma"], x["bias"], w.G, w.beta1, w.beta2, w.eps, y=y, stream=stream)
+
+    ms_local, ck, note = time_steps(args, ws, local, step, stream)
+    tokens = w.B * w.L
+    agg = aggregate(ms_local, tokens, ws)
+    op_ms = max_over_ranks(ms_local, ws)
+    nb = x["x"].numel() * x["x"].element_size()
+    pk, pk_kind = peaks()
+    achieved = 2 * nb / (op_ms / 1e3) / 1e9
+    out = {
+        "metric": NORM_METRIC, "value": round(agg["value"], 1), "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(agg["ms_per_step"], 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded generator; no dataset)",
+        "config": {"workload": w.name, "B": w.B, "L": w.L, "D": w.D, "G": w.G, "beta1": w.beta1, "beta2": w.beta2,
+                   "l2": f"x larger than L2 ({nb / 1e9:.2f} GB), no flush", "parallelism": f"replicas x{ws}"},
+        "roofline": {"bound": "hbm", "kernel": "tdnorm_stats_kernel + tdnorm_scan_kernel + tdnorm_apply_kernel (one op)",
+                     "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(achieved / pk["hbm_gbs"], 4), "peak_kind": f"{pk_kind} HBM copy",
+                     "traffic": recorded_traffic(w, NORM_PROFILE, norm_source_hash()), "launch_ms": round(op_ms, 4),
+                     "algorithmic_bytes_per_launch": 2 * nb},
+        "clocks": ck,
+        "gpu_launches": 3 * args.steps,
+    }
+    if note:
+        out["note"] = note
+    if not args.no_e2e:
+        hx = x["x"].cpu().pin_memory()
+        hy = torch.empty_like(hx).pin_memory()
+        dx = torch.empty_like(x["x"])
+
+        def e2e_step():
+            dx.copy_(hx, non_blocking=True)
+            step(dx)
+            hy.copy_(y, non_blocking=True)
+
+        e_args = argparse.Namespace(steps=max(1, min(args.steps, 10)), warmup=3)
+        ems, _, _ = time_steps(e_args, ws, local, e2e_step, stream)
+        ea = aggregate(ems, tokens, ws)
+        out["e2e"] = {"value": round(ea["value"], 1), "unit": "tokens/s", "h2d_bytes_per_step": nb,
+                      "d2h_bytes_per_step": nb, "steps": e_args.steps, "ms_per_step": round(ea["ms_per_step"], 3)}
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        groups = 4
+        gs = w.D // w.G
+        xs = x["x"][:, :, :groups * gs].double().cpu().numpy()
+        g = x["gamma"][:groups * gs].double().cpu().numpy()
+        b = x["bias"][:groups * gs].double().cpu().numpy()
+        t0 = time.perf_counter()
+        N.tdnorm_forward(xs, groups, w.beta1, w.beta2, w.eps, g, b)
+        secs = time.perf_counter() - t0
+        out["cpu_baseline"] = {"value": round(tokens * groups / w.G / secs, 2), "unit": "tokens/s",
+                               "cores": blas_threads(), "kind": "oracle",
+                               "sample": f"fp64 oracle on the first {groups} of {w.G} groups of all {w.L} tokens "
+                                         f"in {secs:.1f} s (tokens scaled by {groups}/{w.G})"}
+    return out
+
+
 def summarize_launches(path: str) -> str:
     """Per-kernel launches, total time and share from an ncu launch-list CSV
     (`ncu --metrics gpu__time_duration.sum --csv`)."""
@@ -602,8 +712,9 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=("sca_awm", "cema"), default="sca_awm",
-                    help="sca_awm: the fused SCA + AWM forward (default); cema: the CEMA recurrence")
+    ap.add_argument("--op", choices=("sca_awm", "cema", "tdnorm"), default="sca_awm",
+                    help="sca_awm: the fused SCA + AWM forward (default); cema: the CEMA recurrence; "
+                         "tdnorm: timestep decay normalisation")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -620,7 +731,8 @@ def main(argv=None):
     if ws != args.gpus and rank == 0:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE {ws}", file=sys.stderr)
     try:
-        out = run_cema(args, ws, rank, local) if args.op == "cema" else run_gecko(args, w, ws, rank, local)
+        runner = {"cema": lambda: run_cema(args, ws, rank, local), "tdnorm": lambda: run_tdnorm(args, ws, rank, local)}
+        out = runner[args.op]() if args.op in runner else run_gecko(args, w, ws, rank, local)
         if rank == 0:
             print(json.dumps(out), flush=True)
     finally:

@@ -233,6 +233,32 @@ int gecko_cema_forward(const void* x, void* y, const float* alpha, const float* 
                        const uint8_t* reset, const float* state_in, float* state_out,
                        int64_t B, int64_t L, int64_t D, int64_t h, int dtype, void* stream);
 
+/*
+ * gecko_tdnorm_forward - timestep decay normalisation, the normalisation
+ * before the projections (Gecko digest, section on technical novelty: the
+ * decayed mean m_t = beta1 m_{t-1} + (1 - beta1) mu_t with Adam-style bias
+ * correction; paperlayer.ai summary, sections 2.2 and 3.1).  Per batch b,
+ * token t and group g of D / G contiguous features:
+ *   mu_t, s2_t = mean and biased variance of x_t over the group
+ *   m_t = beta1 m_{t-1} + (1 - beta1) mu_t,  v_t = beta2 v_{t-1} + (1 - beta2) s2_t
+ *   y_t = (x_t - m_t / (1 - beta1^t)) / sqrt(v_t / (1 - beta2^t) + eps) * gamma + bias
+ * (t from 1).  The pages print the mean update only; the variance update
+ * with beta2, the per-timestep group statistics and the per-feature affine
+ * are the plainest readings.
+ *
+ *   x, y        : [B, L, D] dtype `dtype` (device); y may equal x.
+ *   gamma, bias : [D] fp32 (device).
+ *   Requires D / G to be a whole multiple of 8, 0 <= beta1, beta2 < 1,
+ *   eps >= 0; every pointer 16-byte aligned.
+ * Workspace: 4 * B * L * G floats per device, grown on `stream`, freed by
+ * gecko_release().  Asynchronous on `stream`; argument errors are found on
+ * the host.  Returns GECKO_OK, GECKO_ERR_ARG, GECKO_ERR_SHAPE,
+ * GECKO_ERR_ALIGN, GECKO_ERR_ALLOC or GECKO_ERR_CUDA.
+ */
+int gecko_tdnorm_forward(const void* x, void* y, const float* gamma, const float* bias,
+                         int64_t B, int64_t L, int64_t D, int64_t G,
+                         float beta1, float beta2, float eps, int dtype, void* stream);
+
 /* Thread-local message describing the last non-zero status of this thread. */
 const char* gecko_last_error(void);
 

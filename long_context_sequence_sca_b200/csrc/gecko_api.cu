@@ -87,6 +87,8 @@ struct DeviceState {
   size_t state_bytes = 0;
   void* cema_ws = nullptr;           // CEMA chunk states
   size_t cema_ws_bytes = 0;
+  void* norm_ws = nullptr;           // timestep-norm group statistics
+  size_t norm_ws_bytes = 0;
 };
 
 std::mutex g_mu;
@@ -361,12 +363,13 @@ extern "C" void gecko_release(void) {
   int cur = 0;
   cudaGetDevice(&cur);
   for (auto& kv : g_dev) {
-    if (kv.second.ws || kv.second.state || kv.second.cema_ws) {
+    if (kv.second.ws || kv.second.state || kv.second.cema_ws || kv.second.norm_ws) {
       cudaSetDevice(kv.first);
       cudaDeviceSynchronize();
       if (kv.second.ws) cudaFree(kv.second.ws);
       if (kv.second.state) cudaFree(kv.second.state);
       if (kv.second.cema_ws) cudaFree(kv.second.cema_ws);
+      if (kv.second.norm_ws) cudaFree(kv.second.norm_ws);
     }
     kv.second.ws = nullptr;
     kv.second.ws_bytes = 0;
@@ -374,6 +377,8 @@ extern "C" void gecko_release(void) {
     kv.second.state_bytes = 0;
     kv.second.cema_ws = nullptr;
     kv.second.cema_ws_bytes = 0;
+    kv.second.norm_ws = nullptr;
+    kv.second.norm_ws_bytes = 0;
     kv.second.have_state = false;
   }
   cudaSetDevice(cur);
@@ -477,4 +482,36 @@ extern "C" int gecko_cema_forward(const void* x, void* y, const float* alpha, co
     return rc;
   CemaProblem p{x, y, alpha, delta, theta, beta, eta, reset, state_in, state_out, B, L, D, dtype, ds->status};
   return check_cuda(launch_cema(p, carve_cema_workspace(ds->cema_ws, B, L, D), st), "CEMA launch");
+}
+
+extern "C" int gecko_tdnorm_forward(const void* x, void* y, const float* gamma, const float* bias, int64_t B,
+                                    int64_t L, int64_t D, int64_t G, float beta1, float beta2, float eps, int dtype,
+                                    void* stream) {
+  const void* ptrs[4] = {x, y, gamma, bias};
+  for (int i = 0; i < 4; ++i) {
+    if (!ptrs[i]) return fail(GECKO_ERR_ARG, "tensor argument %d is NULL", i);
+    if (reinterpret_cast<uintptr_t>(ptrs[i]) % 16 != 0)
+      return fail(GECKO_ERR_ALIGN, "tensor argument %d is not 16-byte aligned", i);
+  }
+  if (dtype != GECKO_F32 && dtype != GECKO_BF16) return fail(GECKO_ERR_ARG, "unknown dtype %d", dtype);
+  if (B < 1 || L < 1 || D < 1 || G < 1)
+    return fail(GECKO_ERR_ARG, "sizes must be >= 1 (B=%lld L=%lld D=%lld G=%lld)", (long long)B, (long long)L,
+                (long long)D, (long long)G);
+  if (!(beta1 >= 0.f && beta1 < 1.f && beta2 >= 0.f && beta2 < 1.f && eps >= 0.f))
+    return fail(GECKO_ERR_ARG, "need 0 <= beta1, beta2 < 1 and eps >= 0");
+  if (D % G != 0 || (D / G) % 8 != 0)
+    return fail(GECKO_ERR_SHAPE, "D / G must be a whole multiple of 8 (D=%lld G=%lld)", (long long)D, (long long)G);
+  if ((long double)B * L * D * 4 > 4.0e18L || B * G > (1 << 30))
+    return fail(GECKO_ERR_SHAPE, "size exceeds kernel index range");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int dev = 0, rc;
+  if ((rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice"))) return rc;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState* ds = nullptr;
+  if ((rc = device_state(dev, &ds))) return rc;
+  if ((rc = ensure_buffer(&ds->norm_ws, &ds->norm_ws_bytes, tdnorm_workspace_bytes(B, L, G), st,
+                          "normalisation workspace")))
+    return rc;
+  NormProblem p{x, y, gamma, bias, B, L, D, G, beta1, beta2, eps, dtype};
+  return check_cuda(launch_tdnorm(p, carve_tdnorm_workspace(ds->norm_ws, B, L, G), st), "normalisation launch");
 }

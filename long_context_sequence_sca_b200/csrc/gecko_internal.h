@@ -87,4 +87,26 @@ size_t cema_workspace_bytes(int64_t B, int64_t L, int64_t D);
 CemaWorkspace carve_cema_workspace(void* base, int64_t B, int64_t L, int64_t D);
 cudaError_t launch_cema(const CemaProblem& p, const CemaWorkspace& w, cudaStream_t st);
 
+// ------------------------------------------------ timestep decay norm --
+
+// One validated call: x, y [B, L, D] (dtype); gamma, bias [D] fp32 (device);
+// G groups of D / G features.
+struct NormProblem {
+  const void* x;
+  void* y;
+  const float *gamma, *bias;
+  int64_t B, L, D, G;
+  float beta1, beta2, eps;
+  int dtype;
+};
+
+struct NormWorkspace {
+  float2* stats;    // [B, L, G]  (mean, variance) of each group
+  float2* affine;   // [B, L, G]  (scale, shift) from the decayed statistics
+};
+
+size_t tdnorm_workspace_bytes(int64_t B, int64_t L, int64_t G);
+NormWorkspace carve_tdnorm_workspace(void* base, int64_t B, int64_t L, int64_t G);
+cudaError_t launch_tdnorm(const NormProblem& p, const NormWorkspace& w, cudaStream_t st);
+
 }  // namespace gecko

@@ -20,6 +20,7 @@ EXPORTS = (
     "gecko_sca_awm_forward_noalloc",
     "gecko_awm_state",
     "gecko_cema_forward",
+    "gecko_tdnorm_forward",
     "gecko_device_status",
     "gecko_timing_enable",
     "gecko_timing_read",
@@ -66,6 +67,9 @@ def load() -> ctypes.CDLL:
     lib.gecko_awm_state.restype = ctypes.c_int
     lib.gecko_cema_forward.argtypes = [vp] * 10 + [i64] * 4 + [ctypes.c_int, vp]
     lib.gecko_cema_forward.restype = ctypes.c_int
+    f32 = ctypes.c_float
+    lib.gecko_tdnorm_forward.argtypes = [vp] * 4 + [i64] * 4 + [f32, f32, f32, ctypes.c_int, vp]
+    lib.gecko_tdnorm_forward.restype = ctypes.c_int
     lib.gecko_device_status.argtypes = [vp]
     lib.gecko_device_status.restype = ctypes.c_int
     lib.gecko_timing_enable.argtypes = [ctypes.c_int]
@@ -120,6 +124,11 @@ def gecko_cema_forward(x, y, alpha, delta, theta, beta, eta, reset, state_in, st
     """Direct call of the CEMA entry point with integer pointers (0 = NULL)."""
     return load().gecko_cema_forward(x, y, alpha, delta, theta, beta, eta, reset, state_in, state_out,
                                      B, L, D, h, dtype, stream)
+
+
+def gecko_tdnorm_forward(x, y, gamma, bias, B, L, D, G, beta1, beta2, eps, dtype, stream) -> int:
+    """Direct call of the timestep-normalisation entry point with integer pointers."""
+    return load().gecko_tdnorm_forward(x, y, gamma, bias, B, L, D, G, beta1, beta2, eps, dtype, stream)
 
 
 def gecko_device_status(stream) -> int:
@@ -255,3 +264,21 @@ def cema_forward(x, alpha, delta, theta, beta, eta, reset=None, state_in=None, r
                                 ptr(state_in), ptr(state_out), B, L, D, h, _DT[x.dtype], _stream_handle(stream))
     _check(rc)
     return (y, state_out) if return_state else y
+
+
+def tdnorm_forward(x, gamma, bias, G: int, beta1: float, beta2: float, eps: float, y=None, stream=None):
+    """Timestep decay normalisation of x [B, L, D] (float32 or bfloat16 CUDA
+    tensor) over G feature groups; gamma, bias: [D] float32.  Returns y."""
+    if not (isinstance(x, torch.Tensor) and x.is_cuda and x.is_contiguous() and x.dim() == 3 and x.dtype in _DT):
+        raise ValueError("x must be a contiguous [B, L, D] float32 or bfloat16 CUDA tensor")
+    for prm in (gamma, bias):
+        if not (isinstance(prm, torch.Tensor) and prm.is_cuda and prm.is_contiguous() and prm.dtype == torch.float32):
+            raise ValueError("gamma and bias must be contiguous float32 CUDA tensors")
+    B, L, D = x.shape
+    if y is None:
+        y = torch.empty_like(x)
+    with torch.cuda.device(x.device):
+        rc = gecko_tdnorm_forward(x.data_ptr(), y.data_ptr(), gamma.data_ptr(), bias.data_ptr(), B, L, D, G,
+                                  beta1, beta2, eps, _DT[x.dtype], _stream_handle(stream))
+    _check(rc)
+    return y

@@ -93,3 +93,24 @@ def L_cema(ptrs, B, Lt, D, h, dtype):
 def test_cema_host_validation_rejects(so, kw, code):
     assert _cema(**kw) == code
     assert L.gecko_last_error()
+
+
+def _tdnorm(ptrs=None, B=1, Lt=100, D=64, G=4, b1=0.9, b2=0.99, eps=1e-5, dtype=1):
+    ptrs = ptrs or [FAKE] * 4
+    return L.gecko_tdnorm_forward(*ptrs, B, Lt, D, G, b1, b2, eps, dtype, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ptrs=[FAKE, 0, FAKE, FAKE]), 1),
+    (dict(dtype=5), 1),
+    (dict(G=0), 1),
+    (dict(b1=1.0), 1),
+    (dict(b2=-0.1), 1),
+    (dict(eps=-1.0), 1),
+    (dict(D=60, G=4), 2),           # D / G = 15: not a multiple of 8
+    (dict(D=64, G=3), 2),           # D % G != 0
+    (dict(ptrs=[FAKE, FAKE, FAKE + 4, FAKE]), 3),
+])
+def test_tdnorm_host_validation_rejects(so, kw, code):
+    assert _tdnorm(**kw) == code
+    assert L.gecko_last_error()
