@@ -67,7 +67,21 @@ __global__ void __launch_bounds__(256) tdnorm_stats_kernel(const TIn* __restrict
   const TIn* p = x + row * D + (int64_t)g * gs;
   const float k = to_f32(p[0]);
   float s = 0.f, q = 0.f;
-  for (int i = 0; i < gs; i += 8) {
+  int i = 0;
+  for (; i + 32 <= gs; i += 32) {   // four 16-byte loads in flight
+    float v[4][8];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) load8(p + i + 8 * u, v[u]);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float dv = v[u][e] - k;
+        s += dv;
+        q = fmaf(dv, dv, q);
+      }
+  }
+  for (; i < gs; i += 8) {
     float v[8];
     load8(p + i, v);
 #pragma unroll
@@ -100,10 +114,16 @@ __global__ void __launch_bounds__(kScanThreads) tdnorm_scan_kernel(const float2*
   const int64_t t0 = (int64_t)tid * n < L ? (int64_t)tid * n : L, t1 = t0 + n < L ? t0 + n : L;
   const float2* sp = st + ((int64_t)b * L) * G + g;
   float m = 0.f, v = 0.f;
-  for (int64_t t = t0; t < t1; ++t) {
-    const float2 mv = sp[t * G];
-    m = fmaf(beta1, m, (1.f - beta1) * mv.x);
-    v = fmaf(beta2, v, (1.f - beta2) * mv.y);
+  for (int64_t t = t0; t < t1; t += 8) {
+    float2 mv[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) mv[u] = t + u < t1 ? sp[(t + u) * G] : make_float2(0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (t + u < t1) {
+        m = fmaf(beta1, m, (1.f - beta1) * mv[u].x);
+        v = fmaf(beta2, v, (1.f - beta2) * mv[u].y);
+      }
   }
   const int len = (int)(t1 - t0);
   s_e[tid] = make_float2(m, v);
@@ -125,17 +145,25 @@ __global__ void __launch_bounds__(kScanThreads) tdnorm_scan_kernel(const float2*
   // carry-in = inclusive prefix of the previous thread
   m = tid > 0 ? s_e[tid - 1].x : 0.f;
   v = tid > 0 ? s_e[tid - 1].y : 0.f;
-  const double lb1 = log((double)beta1), lb2 = log((double)beta2);
+  // beta^(t+1) as a running fp64 product from the thread's first token, so
+  // 1 - beta^(t+1) keeps its digits for small t (beta = 0 gives 1)
+  double p1 = pow((double)beta1, (double)(t0 + 1)), p2 = pow((double)beta2, (double)(t0 + 1));
   float2* ap = aff + ((int64_t)b * L) * G + g;
-  for (int64_t t = t0; t < t1; ++t) {
-    const float2 mv = sp[t * G];
-    m = fmaf(beta1, m, (1.f - beta1) * mv.x);
-    v = fmaf(beta2, v, (1.f - beta2) * mv.y);
-    // 1 - beta^(t+1) without cancellation (beta = 0 gives 1)
-    const float c1 = beta1 > 0.f ? (float)-expm1((double)(t + 1) * lb1) : 1.f;
-    const float c2 = beta2 > 0.f ? (float)-expm1((double)(t + 1) * lb2) : 1.f;
-    const float scale = rsqrtf(v / c2 + eps);
-    ap[t * G] = make_float2(scale, -(m / c1) * scale);
+  for (int64_t t = t0; t < t1; t += 8) {
+    float2 mv[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) mv[u] = t + u < t1 ? sp[(t + u) * G] : make_float2(0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (t + u < t1) {
+        m = fmaf(beta1, m, (1.f - beta1) * mv[u].x);
+        v = fmaf(beta2, v, (1.f - beta2) * mv[u].y);
+        const float c1 = (float)(1.0 - p1), c2 = (float)(1.0 - p2);
+        p1 *= beta1;
+        p2 *= beta2;
+        const float scale = rsqrtf(v / c2 + eps);
+        ap[(t + u) * G] = make_float2(scale, -(m / c1) * scale);
+      }
   }
 }
 
