@@ -19,7 +19,8 @@
 //               thread per query row (TMEM lane quarter = warp % 4); online
 //               max/sum in registers; P written back to TMEM as bf16 over the
 //               S columns; epilogue O / l.
-// A work unit is two adjacent 128-row query tiles of one (b, h).  The MMA
+// A work unit is two adjacent 128-row query tiles of one (b, h); CTAs claim
+// units from a global counter in the schedule's order (decode_unit).  The MMA
 // warp interleaves the two tiles (PV(0), QK(0), PV(1), QK(1)) so each
 // softmax warpgroup's exp work overlaps the other tile's MMAs.  Only the
 // diagonal key tile of each query tile is masked; key tiles entirely above
@@ -52,6 +53,19 @@ constexpr int kThreads = 320;   // 10 warps: TMA, MMA (+TMEM allocation), 2 x 4 
 #endif
 constexpr int kSfuPairs = GECKO_SFU_PAIRS;
 
+// Units are claimed dynamically from a global counter, in the schedule's
+// order, by each CTA's TMA thread, which publishes them to the CTA's other
+// roles through a ring of kUnitRing slots.  The producer claims at most
+// kKStages + 1 units ahead of the slowest reader (its K loads lead the MMAs
+// by at most kKStages iterations, every unit has at least one, and the
+// softmax warps trail the MMA thread by at most one unit), so 8 slots are
+// never overwritten before they are read.
+constexpr int kUnitRing = 8;
+
+// Next unit to claim (reset to 0 on the launching stream before each launch;
+// forwards on one device are not concurrent).
+__device__ unsigned g_unit_counter;
+
 template <int D>
 struct ScaCfg {
   static constexpr int kTileBytes = 128 * D * 2;       // 128 rows x D bf16, D/64 swizzled boxes
@@ -63,15 +77,17 @@ struct ScaCfg {
   static constexpr int kKStages = D == 64 ? 5 : 3;
   static constexpr int kVStages = D == 64 ? 4 : 2;
   static_assert(kKStages >= kVStages, "the iteration-done ring has kKStages slots");
+  static_assert(kKStages + 2 <= kUnitRing, "unit ring too short for the K lead");
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + 2 * kTileBytes;
   static constexpr int kVOff = kKOff + kKStages * kTileBytes;
   static constexpr int kBarOff = kVOff + kVStages * kTileBytes;
   // q_full, q_empty, k_full[KS], it_done[KS], v_full[VS], s_full[2],
-  // p_full[2], o_full[2], o_empty[2], drain
-  static constexpr int kNumBars = 2 + 2 * kKStages + kVStages + 8 + 1;
+  // p_full[2], o_full[2], o_empty[2], drain, unit_ready[kUnitRing]
+  static constexpr int kNumBars = 2 + 2 * kKStages + kVStages + 8 + 1 + kUnitRing;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kBytes = kMiscOff + 16;
+  // tmem address, abort flag, then the unit ring (kUnitRing uint32)
+  static constexpr int kBytes = kMiscOff + 8 + 4 * kUnitRing;
   static constexpr int kAlloc = kBytes + 1024;         // slack for 1024-byte alignment
   static_assert(kAlloc <= 232448, "dynamic shared memory above the sm_100 per-block limit");
   static constexpr uint32_t kTmemCols = 512;
@@ -133,31 +149,55 @@ __device__ __forceinline__ Unit decode_unit(int u, int BH, int T, int c, int kof
   return U;
 }
 
+// The TMA thread's claims: ordinal n of this CTA's work is unit
+// slot[n % kUnitRing]; a claim takes the next unit of the global counter
+// (n_units once all are taken, the end marker), writes it to its slot and
+// arrives on the slot's barrier.
+struct Claims {
+  unsigned* counter;
+  uint32_t* slot;
+  uint64_t* ready;
+  int claimed;
+  int n_units;
+
+  __device__ __forceinline__ int unit_of(int n) {
+    while (claimed <= n) {
+      const unsigned u = atomicAdd(counter, 1u);
+      const int s = claimed % kUnitRing;
+      slot[s] = u < (unsigned)n_units ? u : (unsigned)n_units;
+      mbar_arrive(ready + s);   // release: the slot write is visible to its readers
+      ++claimed;
+    }
+    return (int)slot[n % kUnitRing];
+  }
+};
+
 // Walks the K/V iterations of one CTA in the order the MMA warp consumes
-// them: its units (u, u + gridDim.x, ...) one after another, and each
-// unit's key tiles in order.
+// them: its units in the order claimed, and each unit's key tiles in order.
 struct KvWalk {
+  int n;            // ordinal of the current unit
   int u;            // current unit (>= n_units: finished)
   int j, je;        // current key tile of the unit, one past its last
   int64_t kvbase;   // first K/V row of the unit's (b, h)
   uint32_t it;      // iterations walked so far
 };
 
-__device__ __forceinline__ void kv_walk_enter(KvWalk& w, int u, int BH, int T, int c, int koff, int n_units) {
-  w.u = u;
-  if (u < n_units) {
-    const Unit U = decode_unit(u, BH, T, c, koff);
+__device__ __forceinline__ void kv_walk_enter(KvWalk& w, int n, Claims& cl, int BH, int T, int c, int koff) {
+  w.n = n;
+  w.u = cl.unit_of(n);
+  if (w.u < cl.n_units) {
+    const Unit U = decode_unit(w.u, BH, T, c, koff);
     w.j = U.beg[0];
     w.je = U.nt == 2 ? U.end[1] : U.end[0];
     w.kvbase = U.bh * (int64_t)(T + koff) + koff;
   }
 }
 
-__device__ __forceinline__ void kv_walk_next(KvWalk& w, int stride, int BH, int T, int c, int koff, int n_units) {
+__device__ __forceinline__ void kv_walk_next(KvWalk& w, Claims& cl, int BH, int T, int c, int koff) {
   ++w.it;
   if (++w.j == w.je) {
     const uint32_t it = w.it;
-    kv_walk_enter(w, w.u + stride, BH, T, c, koff, n_units);
+    kv_walk_enter(w, w.n + 1, cl, BH, T, c, koff);
     w.it = it;
   }
 }
@@ -166,7 +206,7 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
               const __grid_constant__ CUtensorMap map_v, __nv_bfloat16* __restrict__ out, int T, int c, int BH,
-              int n_units, int koff, int* status) {
+              int n_units, int koff, unsigned* unit_counter, int* status) {
   using Cfg = ScaCfg<D>;
   constexpr int KS = Cfg::kKStages, VS = Cfg::kVStages;
   extern __shared__ uint8_t smem_raw[];
@@ -187,8 +227,10 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   uint64_t* o_full = p_full + 2;
   uint64_t* o_empty = o_full + 2;
   uint64_t* drain = o_empty + 2;
+  uint64_t* unit_ready = drain + 1;   // [kUnitRing]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
+  uint32_t* unit_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff + 8);   // [kUnitRing]
 
   const int warp = warp_id_uniform();
   const int lane = threadIdx.x % 32;
@@ -208,6 +250,7 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       mbar_init(o_empty + i, 128);
     }
     mbar_init(drain, 1);
+    for (int r = 0; r < kUnitRing; ++r) mbar_init(unit_ready + r, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -238,10 +281,12 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       // (not unit by unit) lets K run ahead of V by its deeper ring, and
       // every wait is then for an iteration whose own loads were issued
       // earlier, so the producer never waits on itself.
+      Claims cl{unit_counter, unit_slot, unit_ready, 0, n_units};
       KvWalk kw{}, vw{};
-      kv_walk_enter(kw, blockIdx.x, BH, T, c, koff, n_units);
+      kv_walk_enter(kw, 0, cl, BH, T, c, koff);
       vw = kw;
-      int qu = blockIdx.x, qn = 0;
+      int qn = 0;
+      int qu = cl.unit_of(0);
       uint32_t qit0 = 0;   // first K/V iteration of unit qu
       bool ok = true;
       while (ok) {
@@ -260,8 +305,8 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
               tma_load_2d(sQ + i * Cfg::kTileBytes + b * Cfg::kBoxBytes, &map_q, q_full, b * 64,
                           (int)(rowbase + U.q0 + 128 * i));
           qit0 += (uint32_t)((U.nt == 2 ? U.end[1] : U.end[0]) - U.beg[0]);
-          qu += gridDim.x;
           ++qn;
+          qu = cl.unit_of(qn);
         } else if (tV <= tK) {
           if (tV >= 0 && !(ok = mbar_wait(it_done + tV % KS, (uint32_t)(tV / KS) & 1, abort_flag, status))) break;
           const int st = vw.it % VS;
@@ -269,7 +314,7 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           mbar_arrive_expect_tx(v_full + st, Cfg::kTileBytes);
           for (int b = 0; b < D / 64; ++b)
             tma_load_2d(sV + st * Cfg::kTileBytes + b * Cfg::kBoxBytes, &map_v, v_full + st, b * 64, row);
-          kv_walk_next(vw, gridDim.x, BH, T, c, koff, n_units);
+          kv_walk_next(vw, cl, BH, T, c, koff);
         } else {
           if (tK >= 0 && !(ok = mbar_wait(it_done + tK % KS, (uint32_t)(tK / KS) & 1, abort_flag, status))) break;
           const int st = kw.it % KS;
@@ -277,7 +322,7 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           mbar_arrive_expect_tx(k_full + st, Cfg::kTileBytes);
           for (int b = 0; b < D / 64; ++b)
             tma_load_2d(sK + st * Cfg::kTileBytes + b * Cfg::kBoxBytes, &map_k, k_full + st, b * 64, row);
-          kv_walk_next(kw, gridDim.x, BH, T, c, koff, n_units);
+          kv_walk_next(kw, cl, BH, T, c, koff);
         }
       }
       if (!ok) {
@@ -300,7 +345,10 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       uint32_t kv_it = 0, p_cnt[2] = {0, 0}, o_cnt[2] = {0, 0};
       int n = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++n) {
+      for (;; ++n) {
+        if (!(ok = mbar_wait(unit_ready + n % kUnitRing, (n / kUnitRing) & 1, abort_flag, status))) break;
+        const int u = (int)unit_slot[n % kUnitRing];
+        if (u >= n_units) break;
         const Unit U = decode_unit(u, BH, T, c, koff);
         if (!(ok = mbar_wait(q_full, n & 1, abort_flag, status))) break;
         tc_fence_after();
@@ -359,6 +407,7 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
             ++kv_it;
           }
         }
+        if (!ok) break;
       }
       // all issued MMAs complete before TMEM is released
       umma_commit(drain);
@@ -374,7 +423,11 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
     const uint32_t colO = i == 0 ? Cfg::kColO0 : Cfg::kColO1;
     uint32_t s_cnt = 0, o_cnt = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    for (int n = 0;; ++n) {
+      ok = __all_sync(0xffffffffu, mbar_wait(unit_ready + n % kUnitRing, (n / kUnitRing) & 1, abort_flag, status));
+      if (!ok) break;
+      const int u = (int)unit_slot[n % kUnitRing];
+      if (u >= n_units) break;
       const Unit U = decode_unit(u, BH, T, c, koff);
       if (i >= U.nt) continue;
       float m_ref = 0.f, l = 0.f;
@@ -577,8 +630,12 @@ cudaError_t launch_sca_tc_impl(const Problem& p, cudaStream_t st) {
   if ((e = cudaFuncSetAttribute(sca_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kAlloc)) !=
       cudaSuccess)
     return e;
+  // the unit counter starts from zero for every launch (stream-ordered)
+  unsigned* counter = nullptr;
+  if ((e = cudaGetSymbolAddress(reinterpret_cast<void**>(&counter), g_unit_counter)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(counter, 0, sizeof(unsigned), st)) != cudaSuccess) return e;
   sca_tc_kernel<D><<<grid, kThreads, Cfg::kAlloc, st>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(p.out_sca), T,
-                                                        (int)p.c, BH, n_units, (int)p.koff, p.status);
+                                                        (int)p.c, BH, n_units, (int)p.koff, counter, p.status);
   return cudaGetLastError();
 }
 
