@@ -252,27 +252,30 @@ __global__ void __launch_bounds__(192, 2) awm_chunk_tc_kernel(const __grid_const
 
 template <int D>
 struct ReadoutCfg {
-  static constexpr int kA = 128 * D * 2;     // psi tile, K-major, D/64 boxes of [128 x 64]
-  static constexpr int kB = D * D * 2;       // M' bf16, MN-major, D/64 boxes of [D x 64]
-  static constexpr int kAOff = 0;
-  static constexpr int kBOff = 2 * kA;       // two A buffers
+  static constexpr int kBox = 128 * 128;        // one [128 rows x 64] bf16 box, 128B-swizzled
+  static constexpr int kA = 128 * D * 2;       // a Q_m tile = the psi operand (K-major, D/64 boxes)
+  static constexpr int kB = D * D * 2;         // M' bf16, MN-major, D/64 boxes of [D x 64]
+  static constexpr int kAOff = 0;              // two tiles
+  static constexpr int kBOff = 2 * kA;
   static constexpr int kBarOff = kBOff + kB;
-  static constexpr int kNumBars = 4;         // a_full[2], acc_full[2]
+  static constexpr int kNumBars = 5;           // q_full[2], acc_full[2], drain
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;
   static constexpr uint32_t kTmemCols = 2 * D;   // two accumulators
 };
 
-// 128 threads: one row each; thread 0 also issues the MMAs.  grid
-// (S, BH, G): CTA g of a chunk takes its 128-row tiles g, g + G, ...  The A
-// operand holds the unnormalised numerators exp(q - max) of each row (bf16,
-// via packed f16 exponentials); the epilogue scales row t by 1 / sum_t.  The
-// next tile's Q_m rows are loaded while the current one is processed; A and
-// the accumulator are double-buffered so a tile's MMA overlaps the next
-// tile's exponentials.
+// 128 threads: one row each; thread 0 also issues the TMA copies and the
+// MMAs.  grid (S, BH, G): CTA g of a chunk takes its 128-row tiles g,
+// g + G, ...  Each Q_m tile arrives by TMA in the 128B-swizzled K-major
+// layout of the MMA's A operand; every thread turns its row into the
+// unnormalised numerators exp(q - max) in place (bf16, packed f16
+// exponentials), and the epilogue scales row t by 1 / sum_t.  Two tile
+// buffers and two accumulators: the next tile's copy is issued as soon as
+// the MMA that read its buffer has completed, and a tile's MMA overlaps the
+// previous tile's epilogue.
 template <int D>
-__global__ void __launch_bounds__(128) awm_readout_tc_kernel(const __nv_bfloat16* __restrict__ qm,
+__global__ void __launch_bounds__(128) awm_readout_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                                                              const float* __restrict__ Mst,
                                                              __nv_bfloat16* __restrict__ out, int T, int c,
                                                              const float* __restrict__ Mprev0, int64_t sd,
@@ -280,8 +283,9 @@ __global__ void __launch_bounds__(128) awm_readout_tc_kernel(const __nv_bfloat16
   using Cfg = ReadoutCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* a_full = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);  // [0]: drain after an abort
-  uint64_t* acc_full = a_full + 2;                                        // [2] MMA -> threads
+  uint64_t* q_full = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);  // [2] TMA -> threads
+  uint64_t* acc_full = q_full + 2;                                        // [2] MMA -> threads, TMA
+  uint64_t* drain = acc_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
 
@@ -304,13 +308,23 @@ __global__ void __launch_bounds__(128) awm_readout_tc_kernel(const __nv_bfloat16
     return;
   }
   if (m == 0) return;
+  auto load_tile = [&](int idx) {   // thread 0: tile idx into buffer idx & 1
+    const int buf = idx & 1;
+    mbar_arrive_expect_tx(q_full + buf, Cfg::kA);
+    for (int b = 0; b < D / 64; ++b)
+      tma_load_2d(smem + Cfg::kAOff + buf * Cfg::kA + b * Cfg::kBox, &map_q, q_full + buf, b * 64,
+                  (int)(row0 + (int64_t)(g + idx * G) * 128));
+  };
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
+      mbar_init(q_full + i, 1);
       mbar_init(acc_full + i, 1);
-      mbar_init(a_full + i, 1);
     }
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
+    tma_prefetch_desc(&map_q);
+    load_tile(0);
   }
   if (warp == 0) {
     tmem_alloc(tmem_slot, Cfg::kTmemCols);
@@ -364,25 +378,19 @@ __global__ void __launch_bounds__(128) awm_readout_tc_kernel(const __nv_bfloat16
     return true;
   };
 
-  uint4 cur[D / 8], nxt[D / 8];
-  {
-    const uint4* src = reinterpret_cast<const uint4*>(qm + (row0 + (int64_t)g * 128 + r) * D);
-#pragma unroll
-    for (int i = 0; i < D / 8; ++i) cur[i] = src[i];
-  }
   float inv_prev = 0.f;
+  int issued = 1;   // tiles whose copy has been issued (thread 0)
   for (int idx = 0; idx < m && ok; ++idx) {
     const int kt = g + idx * G, buf = idx & 1;
-    if (idx + 1 < m) {
-      const uint4* src = reinterpret_cast<const uint4*>(qm + (row0 + (int64_t)(kt + G) * 128 + r) * D);
-#pragma unroll
-      for (int i = 0; i < D / 8; ++i) nxt[i] = src[i];
-    }
-    // psi numerators exp(q - max) of row r -> A[buf] (K-major, swizzled)
+    ok = __all_sync(0xffffffffu, mbar_wait(q_full + buf, (idx >> 1) & 1, abort_flag, status));
+    if (!ok) break;
+    // psi numerators exp(q - max) of row r, written over the row in place
+    uint8_t* a = smem + Cfg::kAOff + buf * Cfg::kA;
     float mx = -INFINITY;
 #pragma unroll
     for (int i = 0; i < D / 8; ++i) {
-      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&cur[i]);
+      const uint4 q = *reinterpret_cast<const uint4*>(a + sw128_off(r, 8 * i, 128));
+      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&q);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const float2 f2 = __bfloat1622float2(p2[j]);
@@ -391,10 +399,11 @@ __global__ void __launch_bounds__(128) awm_readout_tc_kernel(const __nv_bfloat16
     }
     const float mx2 = mx * kLog2e;
     float sum = 0.f;
-    uint8_t* a = smem + Cfg::kAOff + buf * Cfg::kA;
 #pragma unroll
     for (int i = 0; i < D / 8; ++i) {
-      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&cur[i]);
+      uint4* qa = reinterpret_cast<uint4*>(a + sw128_off(r, 8 * i, 128));
+      const uint4 q = *qa;
+      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&q);
       uint4 p;
       uint32_t* pp = reinterpret_cast<uint32_t*>(&p);
 #pragma unroll
@@ -405,7 +414,7 @@ __global__ void __launch_bounds__(128) awm_readout_tc_kernel(const __nv_bfloat16
         sum += e0 + e1;
         pp[j] = pack_bf16x2(e0, e1);
       }
-      *reinterpret_cast<uint4*>(a + sw128_off(r, 8 * i, 128)) = p;
+      *qa = p;
     }
     const float inv = 1.f / sum;
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -420,18 +429,25 @@ __global__ void __launch_bounds__(128) awm_readout_tc_kernel(const __nv_bfloat16
         umma_ss(tmem + buf * D, sdesc_at(ad, koff), sdesc_at(bdesc, kk * 16 * 128), idesc, kk > 0 ? 1u : 0u);
       }
       umma_commit(acc_full + buf);
+      // refill the other buffer once the MMA that read it (tile idx - 1) is done
+      if (idx + 1 < m) {
+        if (idx == 0 || mbar_wait(acc_full + (buf ^ 1), ((idx - 1) >> 1) & 1, abort_flag, status)) {
+          load_tile(idx + 1);
+          ++issued;
+        }
+      }
     }
     // epilogue of the previous tile overlaps this tile's MMA
     if (idx > 0) ok = store_tile(kt - G, buf ^ 1, ((idx - 1) >> 1) & 1, inv_prev);
     inv_prev = inv;
-#pragma unroll
-    for (int i = 0; i < D / 8; ++i) cur[i] = nxt[i];
   }
   if (ok) ok = store_tile(g + (m - 1) * G, (m - 1) & 1, ((m - 1) >> 1) & 1, inv_prev);
   if (!ok && threadIdx.x == 0) {
-    // make sure no MMA is still writing TMEM before it is released
-    umma_commit(a_full);
-    mbar_wait_drain(a_full, 0);
+    // no MMA may still write TMEM, and no copy still write shared memory,
+    // when the CTA exits
+    umma_commit(drain);
+    mbar_wait_drain(drain, 0);
+    for (int t = issued > 2 ? issued - 2 : 0; t < issued; ++t) mbar_wait_drain(q_full + (t & 1), (t >> 1) & 1);
   }
   tc_fence_before();
   __syncthreads();
@@ -485,12 +501,22 @@ cudaError_t readout_impl(const Problem& p, const Workspace& w, cudaStream_t st) 
   cudaError_t e = cudaFuncSetAttribute(awm_readout_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Cfg::kAlloc);
   if (e != cudaSuccess) return e;
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  CUtensorMap mq;   // Q_m as [B H T rows, D], boxes of [128 rows x 64] bf16, 128B swizzle
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)(p.B * p.H * p.T)};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  if (fn(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(p.qm), dims, strides, box, estr,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
   // split each chunk's 128-row tiles over G CTAs (up to 8 tiles per CTA)
   const int n_tiles = (int)(p.c / 128);
   const int G = n_tiles > 8 ? (n_tiles + 7) / 8 : 1;
   awm_readout_tc_kernel<D><<<dim3(p.S, p.B * p.H, G), 128, Cfg::kAlloc, st>>>(
-      static_cast<const __nv_bfloat16*>(p.qm), w.Mst, static_cast<__nv_bfloat16*>(p.out_mem), (int)p.T,
-      (int)p.c, p.state0, state_floats(D), p.status);
+      mq, w.Mst, static_cast<__nv_bfloat16*>(p.out_mem), (int)p.T, (int)p.c, p.state0, state_floats(D), p.status);
   return cudaGetLastError();
 }
 
