@@ -59,7 +59,7 @@ struct ChunkCfg {
 // 128 compute threads (warps 0-3), warp 4 = TMA producer, warp 5 = MMA issuer.
 template <int D>
 __global__ void __launch_bounds__(192, 2) awm_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_v,
-                                                           const __nv_bfloat16* __restrict__ km,
+                                                           const __grid_constant__ CUtensorMap map_km,
                                                            const float* __restrict__ lse, float* __restrict__ Bm,
                                                            float* __restrict__ Cm, int T, int c, int koff,
                                                            int* status) {
@@ -104,16 +104,22 @@ __global__ void __launch_bounds__(192, 2) awm_chunk_tc_kernel(const __grid_const
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 4) {
-    // ----------------------------------------------------- V tiles by TMA --
+    // ------------------------------------------------ V and K_m by TMA --
+    // V into the V slot, K_m into the Psi slot (where it is turned into Psi
+    // in place), both on v_full.
     if (lane == 0) {
       tma_prefetch_desc(&map_v);
+      tma_prefetch_desc(&map_km);
       for (int kt = 0; kt < n_tiles; ++kt) {
         const int st = kt & 1;
         if (!mbar_wait(st_empty + st, ((kt >> 1) & 1) ^ 1, abort_flag, status)) break;
-        mbar_arrive_expect_tx(v_full + st, Cfg::kOperand);
-        for (int b = 0; b < D / 64; ++b)
+        mbar_arrive_expect_tx(v_full + st, 2 * Cfg::kOperand);
+        for (int b = 0; b < D / 64; ++b) {
           tma_load_2d(smem + st * Cfg::kStage + b * Cfg::kBox, &map_v, v_full + st, b * 64,
                       (int)(vrow0 + (int64_t)kt * kKT));
+          tma_load_2d(smem + st * Cfg::kStage + Cfg::kOperand + b * Cfg::kBox, &map_km, v_full + st, b * 64,
+                      (int)(row0 + (int64_t)kt * kKT));
+        }
       }
       if (*abort_flag) {
         for (int st = 0; st < 2; ++st) mbar_wait_drain(v_full + st, ((n_tiles - 1 - st) >> 1) & 1);
@@ -152,21 +158,18 @@ __global__ void __launch_bounds__(192, 2) awm_chunk_tc_kernel(const __grid_const
     const int h = threadIdx.x & 1;        // which half of the features
     constexpr int HF = D / 2;             // features per thread
     bool ok = true;
-    uint4 cur[HF / 8], nxt[HF / 8];
-    const __nv_bfloat16* src = km + row0 * D + (int64_t)r * D + h * HF;
-#pragma unroll
-    for (int i = 0; i < HF / 8; ++i) cur[i] = reinterpret_cast<const uint4*>(src)[i];
     for (int kt = 0; kt < n_tiles; ++kt) {
       const int st = kt & 1;
-      if (kt + 1 < n_tiles) {
-        const __nv_bfloat16* nsrc = src + (int64_t)(kt + 1) * kKT * D;
-#pragma unroll
-        for (int i = 0; i < HF / 8; ++i) nxt[i] = reinterpret_cast<const uint4*>(nsrc)[i];
-      }
+      // V and K_m of this tile have landed (the copy also waited for the
+      // MMAs of tile kt - 2 to release the stage)
+      ok = __all_sync(0xffffffffu, mbar_wait(v_full + st, (kt >> 1) & 1, abort_flag, status));
+      if (!ok) break;
+      uint8_t* stg = smem + st * Cfg::kStage;
       float x[HF];
 #pragma unroll
       for (int i = 0; i < HF / 8; ++i) {
-        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&cur[i]);
+        const uint4 raw = *reinterpret_cast<const uint4*>(stg + Cfg::kOperand + sw128_off(r, h * HF + 8 * i, kKT));
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const float2 f2 = __bfloat1622float2(p2[j]);
@@ -179,10 +182,6 @@ __global__ void __launch_bounds__(192, 2) awm_chunk_tc_kernel(const __grid_const
       for (int i = 1; i < HF; ++i) mx = fmaxf(mx, x[i]);
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
       const float mx2 = mx * kLog2e;
-      // wait until the MMAs of tile kt-2 have released this stage
-      ok = __all_sync(0xffffffffu, mbar_wait(st_empty + st, ((kt >> 1) & 1) ^ 1, abort_flag, status));
-      if (!ok) break;
-      uint8_t* stg = smem + st * Cfg::kStage;
       float e[HF], sum = 0.f;
 #pragma unroll
       for (int i = 0; i < HF / 8; ++i) {
@@ -214,8 +213,6 @@ __global__ void __launch_bounds__(192, 2) awm_chunk_tc_kernel(const __grid_const
       // generic-proxy writes must be visible to the tensor core (async proxy)
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       mbar_arrive(op_full + st);
-#pragma unroll
-      for (int i = 0; i < HF / 8; ++i) cur[i] = nxt[i];
     }
     // epilogue: accumulator row f = TMEM lane; columns [0, D) = Bm, [D, 2D) = Cm
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, status));
@@ -478,20 +475,24 @@ cudaError_t chunk_impl(const Problem& p, const Workspace& w, cudaStream_t st) {
   using Cfg = ChunkCfg<D>;
   EncodeTiledFn fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
-  CUtensorMap mv;
-  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)(p.B * p.H * (p.T + p.koff))};
-  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)kKT};
-  cuuint32_t estr[2] = {1, 1};
-  if (fn(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(p.v), dims, strides, box, estr,
-         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
+  // V and K_m as [rows, D], boxes of [64 rows x 64] bf16, 128B swizzle (V
+  // carries koff extra leading rows per (b, h) for a continued sequence)
+  auto map = [&](CUtensorMap* m, const void* base, int64_t rows) {
+    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)kKT};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  };
+  CUtensorMap mv, mkm;
+  if (!map(&mv, p.v, p.B * p.H * (p.T + p.koff)) || !map(&mkm, p.km, p.B * p.H * p.T)) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(awm_chunk_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Cfg::kAlloc);
   if (e != cudaSuccess) return e;
   awm_chunk_tc_kernel<D><<<dim3(p.S, p.B * p.H), 192, Cfg::kAlloc, st>>>(
-      mv, static_cast<const __nv_bfloat16*>(p.km), w.lse, w.Bm, w.Cm, (int)p.T, (int)p.c, (int)p.koff, p.status);
+      mv, mkm, w.lse, w.Bm, w.Cm, (int)p.T, (int)p.c, (int)p.koff, p.status);
   return cudaGetLastError();
 }
 
