@@ -402,7 +402,8 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           }
           if (!ok) break;
           if (j < je) {
-            umma_commit(it_done + stK);   // K_j and V_{j-1} (and a drained V of the previous unit)
+            // no commit for it_done: the softmax warpgroup of the iteration's
+            // last active tile arrives on it once that tile's S is complete
             if (j == je - 1) umma_commit(q_empty);
             ++kv_it;
           }
@@ -423,17 +424,26 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
     const uint32_t colO = i == 0 ? Cfg::kColO0 : Cfg::kColO1;
     uint32_t s_cnt = 0, o_cnt = 0;
     bool ok = true;
+    uint32_t it_base = 0;   // K/V iterations of this CTA's earlier units (both warpgroups see every unit)
     for (int n = 0;; ++n) {
       ok = __all_sync(0xffffffffu, mbar_wait(unit_ready + n % kUnitRing, (n / kUnitRing) & 1, abort_flag, status));
       if (!ok) break;
       const int u = (int)unit_slot[n % kUnitRing];
       if (u >= n_units) break;
       const Unit U = decode_unit(u, BH, T, c, koff);
+      const int jb = U.beg[0], je = U.nt == 2 ? U.end[1] : U.end[0];
+      const uint32_t unit_it0 = it_base;
+      it_base += (uint32_t)(je - jb);
       if (i >= U.nt) continue;
       float m_ref = 0.f, l = 0.f;
       for (int j = U.beg[i]; j < U.end[i]; ++j) {
         ok = __all_sync(0xffffffffu, mbar_wait(s_full + i, s_cnt & 1, abort_flag, status));
         if (!ok) break;
+        // The QK of the iteration's last active tile is its last MMA, so its
+        // completion (just observed) means K_j and V_{j-1} are no longer read:
+        // one thread of that tile's warpgroup releases them to the producer.
+        if ((i == 1 || !(U.nt == 2 && j >= U.beg[1])) && warp % 4 == 2 && lane == 0)
+          mbar_arrive(it_done + (unit_it0 + (uint32_t)(j - jb)) % KS);
         ++s_cnt;
         tc_fence_after();
         const bool diag = j == U.end[i] - 1;
