@@ -89,6 +89,55 @@ int gecko_sca_awm_forward(const void* q, const void* k, const void* v,
                           int dtype, void* stream);
 
 /*
+ * gecko_sca_awm_forward_train - gecko_sca_awm_forward that also keeps what
+ * the backward needs from SCA: the natural-log sum of exp of each query
+ * row's visible scores (the softmax normaliser of SCA, Gecko digest, method
+ * step details, step 3).
+ *
+ *   lse : [B, H, T] fp32 (device), 16-byte aligned; fully overwritten.
+ *
+ * Everything else as gecko_sca_awm_forward (same outputs, bit for bit).
+ */
+int gecko_sca_awm_forward_train(const void* q, const void* k, const void* v,
+                                const void* qm, const void* km,
+                                void* out_sca, void* out_mem, float* lse,
+                                int64_t B, int64_t H, int64_t T, int64_t c, int64_t d,
+                                int dtype, void* stream);
+
+/*
+ * gecko_sca_awm_backward - gradients of one fresh-sequence forward with
+ * respect to q, k, v, qm, km, given the gradients of its two outputs.  The
+ * pages print no backward; this is the chain rule of the forward above (SCA:
+ * digest step 3; AWM: digest core method and steps 4-5, paperlayer.ai
+ * summary section 3.3 and Appendix A).  As the summary's appendix B.1
+ * (backward pass) describes, only chunk-boundary states are needed: they
+ * are rebuilt here from qm, km, v, so the forward keeps nothing but lse.
+ *
+ *   q, k, v, qm, km : the forward's inputs, [B, H, T, d] dtype (device).
+ *   out_sca, lse    : the forward's SCA output and lse
+ *                     (gecko_sca_awm_forward_train).
+ *   dout_sca, dout_mem : gradients of out_sca and out_mem, [B, H, T, d].
+ *   dq, dk, dv, dqm, dkm : [B, H, T, d] dtype (device), fully overwritten;
+ *                     dv sums the SCA and AWM parts (v feeds both).  They
+ *                     must not alias each other or any input.
+ *   All pointers 16-byte aligned; same size constraints as the forward.
+ *   The gradient of the exported state (M'_{S+1}, log z^S) is taken as zero.
+ *
+ * Ownership: a second per-device workspace (row statistics, per-chunk
+ * state gradients, the AWM part of dV in fp32) grows like the forward's
+ * and lives until gecko_release().  The call recomputes the forward's AWM
+ * workspace, so gecko_awm_state afterwards reports this sequence's state.
+ * Errors as gecko_sca_awm_forward.
+ */
+int gecko_sca_awm_backward(const void* q, const void* k, const void* v,
+                           const void* qm, const void* km,
+                           const void* out_sca, const float* lse,
+                           const void* dout_sca, const void* dout_mem,
+                           void* dq, void* dk, void* dv, void* dqm, void* dkm,
+                           int64_t B, int64_t H, int64_t T, int64_t c, int64_t d,
+                           int dtype, void* stream);
+
+/*
  * gecko_sca_awm_forward_continue - the same forward for one segment of a
  * longer sequence, so a sequence of any length runs in pieces whose outputs
  * equal those of one call over the whole sequence (up to rounding).  The AWM

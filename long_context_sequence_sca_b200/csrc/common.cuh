@@ -36,6 +36,7 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
 
 // 2^a and 2^b through one packed half-precision SFU op (ex2.approx.f16x2).
 // For arguments <= 0 whose results only feed bf16 operands: the f16 result

@@ -89,6 +89,8 @@ struct DeviceState {
   size_t cema_ws_bytes = 0;
   void* norm_ws = nullptr;           // timestep-norm group statistics
   size_t norm_ws_bytes = 0;
+  void* bwd_ws = nullptr;            // backward workspace
+  size_t bwd_ws_bytes = 0;
 };
 
 std::mutex g_mu;
@@ -216,7 +218,7 @@ int ensure_buffer(void** buf, size_t* have, size_t need, cudaStream_t st, const 
 // or host).  state_out, if given, receives (M'_S, M'_{S+1}, log z^S).
 int run_forward(const void* q, const void* k, const void* v, const void* qm, const void* km, void* out_sca,
                 void* out_mem, const float* state_in, float* state_out, int64_t B, int64_t H, int64_t T,
-                int64_t c, int64_t d, int dtype, void* stream) {
+                int64_t c, int64_t d, int dtype, void* stream, float* lse = nullptr) {
   const void* ptrs[7] = {q, k, v, qm, km, out_sca, out_mem};
   int rc = validate(ptrs, 7, B, H, T, c, d, dtype);
   if (rc) return rc;
@@ -236,6 +238,7 @@ int run_forward(const void* q, const void* k, const void* v, const void* qm, con
   Workspace w = carve_workspace(ds->ws, BH, T, c, d);
 
   Problem p{q, k, v, qm, km, out_sca, out_mem, B, H, T, c, d, (int)S, dtype, ds->status};
+  p.lse = lse;
   if (state_in) {
     // private copy, so state_out may alias state_in
     if ((rc = ensure_buffer(&ds->state, &ds->state_bytes, sizeof(float) * BH * sd, st, "state copy"))) return rc;
@@ -289,8 +292,73 @@ int run_forward(const void* q, const void* k, const void* v, const void* qm, con
   return GECKO_OK;
 }
 
+// The backward: rematerialise the AWM chunk-boundary states with the
+// forward kernels, then the AWM reverse pass, then the SCA gradients (whose
+// dV kernel adds the AWM part of dV).
+int run_backward(const void* q, const void* k, const void* v, const void* qm, const void* km, const void* out_sca,
+                 const float* lse, const void* dout_sca, const void* dout_mem, void* dq, void* dk, void* dv,
+                 void* dqm, void* dkm, int64_t B, int64_t H, int64_t T, int64_t c, int64_t d, int dtype,
+                 void* stream) {
+  const void* ptrs[14] = {q, k, v, qm, km, out_sca, lse, dout_sca, dout_mem, dq, dk, dv, dqm, dkm};
+  int rc = validate(ptrs, 14, B, H, T, c, d, dtype);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int dev = 0;
+  if ((rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice"))) return rc;
+
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState* ds = nullptr;
+  if ((rc = device_state(dev, &ds))) return rc;
+  const int64_t S = T / c;
+  const int64_t BH = B * H;
+  if ((rc = ensure_buffer(&ds->ws, &ds->ws_bytes, workspace_bytes(BH, T, c, d), st, "workspace"))) return rc;
+  if ((rc = ensure_buffer(&ds->bwd_ws, &ds->bwd_ws_bytes, bwd_workspace_bytes(BH, T, c, d), st,
+                          "backward workspace")))
+    return rc;
+  Workspace w = carve_workspace(ds->ws, BH, T, c, d);
+  BwdWorkspace bw = carve_bwd_workspace(ds->bwd_ws, BH, T, c, d);
+  BwdProblem b{Problem{q, k, v, qm, km, nullptr, nullptr, B, H, T, c, d, (int)S, dtype, ds->status},
+               out_sca, lse, dout_sca, dout_mem, dq, dk, dv, dqm, dkm};
+  const Problem& p = b.f;
+
+  cudaGetLastError();
+  if ((rc = check_cuda(launch_awm_stats(p, w, st), "awm stats"))) return rc;
+  // The chunk products are rebuilt in fp32: the rows of M' are close to one
+  // another (each is a running average of V), and the softmax gradient of
+  // the readout keeps only their differences, which bf16 operands blur.
+  if ((rc = check_cuda(launch_awm_chunk_simt(p, w, st), "awm chunk"))) return rc;
+  if ((rc = check_cuda(launch_awm_carry(p, w, st), "awm carry"))) return rc;
+  if ((rc = check_cuda(launch_awm_bwd(b, w, bw, st), "awm backward"))) return rc;
+  if ((rc = check_cuda(launch_sca_bwd_delta(b, bw, st), "sca backward delta"))) return rc;
+  if ((rc = check_cuda(launch_sca_bwd_simt(b, bw, st), "sca backward"))) return rc;
+  ds->have_state = true;  // the rematerialised states are this sequence's
+  ds->B = B;
+  ds->H = H;
+  ds->d = d;
+  ds->S = S;
+  ds->T = T;
+  return GECKO_OK;
+}
+
 }  // namespace
 }  // namespace gecko
+
+extern "C" int gecko_sca_awm_forward_train(const void* q, const void* k, const void* v, const void* qm,
+                                           const void* km, void* out_sca, void* out_mem, float* lse, int64_t B,
+                                           int64_t H, int64_t T, int64_t c, int64_t d, int dtype, void* stream) {
+  if (!lse) return fail(GECKO_ERR_ARG, "lse is NULL");
+  if (reinterpret_cast<uintptr_t>(lse) % 16 != 0) return fail(GECKO_ERR_ALIGN, "lse is not 16-byte aligned");
+  return run_forward(q, k, v, qm, km, out_sca, out_mem, nullptr, nullptr, B, H, T, c, d, dtype, stream, lse);
+}
+
+extern "C" int gecko_sca_awm_backward(const void* q, const void* k, const void* v, const void* qm, const void* km,
+                                      const void* out_sca, const float* lse, const void* dout_sca,
+                                      const void* dout_mem, void* dq, void* dk, void* dv, void* dqm, void* dkm,
+                                      int64_t B, int64_t H, int64_t T, int64_t c, int64_t d, int dtype,
+                                      void* stream) {
+  return run_backward(q, k, v, qm, km, out_sca, lse, dout_sca, dout_mem, dq, dk, dv, dqm, dkm, B, H, T, c, d, dtype,
+                      stream);
+}
 
 extern "C" int gecko_sca_awm_forward(const void* q, const void* k, const void* v, const void* qm, const void* km,
                                      void* out_sca, void* out_mem, int64_t B, int64_t H, int64_t T, int64_t c,
@@ -363,13 +431,14 @@ extern "C" void gecko_release(void) {
   int cur = 0;
   cudaGetDevice(&cur);
   for (auto& kv : g_dev) {
-    if (kv.second.ws || kv.second.state || kv.second.cema_ws || kv.second.norm_ws) {
+    if (kv.second.ws || kv.second.state || kv.second.cema_ws || kv.second.norm_ws || kv.second.bwd_ws) {
       cudaSetDevice(kv.first);
       cudaDeviceSynchronize();
       if (kv.second.ws) cudaFree(kv.second.ws);
       if (kv.second.state) cudaFree(kv.second.state);
       if (kv.second.cema_ws) cudaFree(kv.second.cema_ws);
       if (kv.second.norm_ws) cudaFree(kv.second.norm_ws);
+      if (kv.second.bwd_ws) cudaFree(kv.second.bwd_ws);
     }
     kv.second.ws = nullptr;
     kv.second.ws_bytes = 0;
@@ -379,6 +448,8 @@ extern "C" void gecko_release(void) {
     kv.second.cema_ws_bytes = 0;
     kv.second.norm_ws = nullptr;
     kv.second.norm_ws_bytes = 0;
+    kv.second.bwd_ws = nullptr;
+    kv.second.bwd_ws_bytes = 0;
     kv.second.have_state = false;
   }
   cudaSetDevice(cur);

@@ -21,6 +21,7 @@ struct Problem {
   // Continuation of a longer sequence (all zero for a fresh start):
   int64_t koff = 0;              // rows of the previous chunk prepended to k and v per head (0 or c)
   const float* state0 = nullptr; // [BH, 2 d^2 + d] carried state (device): M'_prev, M'_cur, log z
+  float* lse = nullptr;          // [BH, T] SCA row log-sum-exp (natural log), written if set
 };
 
 // Floats per (b, h) in a carried state record: M'_prev, M'_cur (d x d each), log z (d).
@@ -57,6 +58,33 @@ bool tc_supported(const Problem& p);
 cudaError_t launch_sca_tc(const Problem& p, cudaStream_t st);
 cudaError_t launch_awm_chunk_tc(const Problem& p, const Workspace& w, cudaStream_t st);
 cudaError_t launch_awm_readout_tc(const Problem& p, const Workspace& w, cudaStream_t st);
+
+// ------------------------------------------------------------ backward --
+
+// One validated backward call: the forward's inputs (f.q .. f.km, sizes,
+// dtype), the forward's SCA output and row log-sum-exp, the output
+// gradients, and the input gradients to write (all [B, H, T, d] dtype).
+struct BwdProblem {
+  Problem f;
+  const void* out_sca;
+  const float* lse;
+  const void *dout_sca, *dout_mem;
+  void *dq, *dk, *dv, *dqm, *dkm;
+};
+
+struct BwdWorkspace {
+  float* delta;   // [BH, T]  rowsum(dO * O) of SCA
+  float* E;       // [BH, S, d, d]  psi(Qm_s)^T dO_m,s
+  float* G;       // [BH, S+1, d, d]  G_s = dLoss/dM'_s, s = 1..S+1
+  float* dl;      // [BH, S, d]  dLoss/d log e_s
+  float* dv_awm;  // [BH, T, d]  AWM part of dV
+};
+
+size_t bwd_workspace_bytes(int64_t BH, int64_t T, int64_t c, int64_t d);
+BwdWorkspace carve_bwd_workspace(void* base, int64_t BH, int64_t T, int64_t c, int64_t d);
+cudaError_t launch_sca_bwd_delta(const BwdProblem& b, const BwdWorkspace& w, cudaStream_t st);
+cudaError_t launch_sca_bwd_simt(const BwdProblem& b, const BwdWorkspace& w, cudaStream_t st);
+cudaError_t launch_awm_bwd(const BwdProblem& b, const Workspace& fw, const BwdWorkspace& w, cudaStream_t st);
 
 // ---------------------------------------------------------------- CEMA --
 

@@ -205,7 +205,8 @@ __device__ __forceinline__ void kv_walk_next(KvWalk& w, Claims& cl, int BH, int 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
-              const __grid_constant__ CUtensorMap map_v, __nv_bfloat16* __restrict__ out, int T, int c, int BH,
+              const __grid_constant__ CUtensorMap map_v, __nv_bfloat16* __restrict__ out,
+              float* __restrict__ lse, int T, int c, int BH,
               int n_units, int koff, unsigned* unit_counter, int* status) {
   using Cfg = ScaCfg<D>;
   constexpr int KS = Cfg::kKStages, VS = Cfg::kVStages;
@@ -553,6 +554,8 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       ++o_cnt;
       tc_fence_after();
       const float inv = 1.f / l;
+      // row log-sum-exp (natural log) for a backward pass: p = 2^(s log2e - m_ref) / l
+      if (lse) lse[U.bh * (int64_t)T + U.q0 + 128 * i + r] = (m_ref + log2f(l)) * kLn2;
       __nv_bfloat16* orow = out + (U.bh * (int64_t)T + U.q0 + 128 * i + r) * D;
 #pragma unroll 1
       for (int cb = 0; cb < D / 32; ++cb) {
@@ -644,7 +647,7 @@ cudaError_t launch_sca_tc_impl(const Problem& p, cudaStream_t st) {
   unsigned* counter = nullptr;
   if ((e = cudaGetSymbolAddress(reinterpret_cast<void**>(&counter), g_unit_counter)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(counter, 0, sizeof(unsigned), st)) != cudaSuccess) return e;
-  sca_tc_kernel<D><<<grid, kThreads, Cfg::kAlloc, st>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(p.out_sca), T,
+  sca_tc_kernel<D><<<grid, kThreads, Cfg::kAlloc, st>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(p.out_sca), p.lse, T,
                                                         (int)p.c, BH, n_units, (int)p.koff, counter, p.status);
   return cudaGetLastError();
 }

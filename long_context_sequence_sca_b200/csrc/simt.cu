@@ -365,13 +365,14 @@ __global__ void __launch_bounds__(256) awm_readout_simt_kernel(const TIn* __rest
 // ------------------------------------------------------------------------
 // SCA with CUDA cores: 32 queries per CTA, 4 threads per query (each owns
 // D/4 dims of q and of the output), keys streamed through shared memory in
-// tiles of 32 with an online softmax.  Scale 1.  k and v hold koff extra
+// tiles of 32 with an online softmax; writes each row's log-sum-exp to lse
+// when it is given.  Scale 1.  k and v hold koff extra
 // leading rows per (b, h) (the previous chunk of a continued sequence, so
 // chunk 1 then has a previous chunk).  grid (T / 32, BH).
 template <typename TIn, int D>
 __global__ void __launch_bounds__(128) sca_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
                                                        const TIn* __restrict__ v, TIn* __restrict__ out,
-                                                       int64_t T, int c, int64_t koff) {
+                                                       float* __restrict__ lse, int64_t T, int c, int64_t koff) {
   constexpr int QD = D / 4;
   __shared__ float ks[32][D + 4];
   __shared__ float vs[32][D + 4];
@@ -416,6 +417,7 @@ __global__ void __launch_bounds__(128) sca_simt_kernel(const TIn* __restrict__ q
     }
   }
   const float inv = 1.f / l;
+  if (lse && part == 0) lse[bh * T + t] = m + logf(l);
   TIn* orow = out + (bh * T + t) * D + part * QD;
 #pragma unroll
   for (int i = 0; i < QD; ++i) orow[i] = from_f32<TIn>(acc[i] * inv);
@@ -471,7 +473,7 @@ template <typename TIn, int D>
 cudaError_t launch_sca_simt_impl(const Problem& p, cudaStream_t st) {
   sca_simt_kernel<TIn, D><<<dim3(p.T / 32, p.B * p.H), 128, 0, st>>>(
       static_cast<const TIn*>(p.q), static_cast<const TIn*>(p.k), static_cast<const TIn*>(p.v),
-      static_cast<TIn*>(p.out_sca), p.T, (int)p.c, p.koff);
+      static_cast<TIn*>(p.out_sca), p.lse, p.T, (int)p.c, p.koff);
   return cudaGetLastError();
 }
 

@@ -18,6 +18,8 @@ EXPORTS = (
     "gecko_sca_awm_forward",
     "gecko_sca_awm_forward_continue",
     "gecko_sca_awm_forward_noalloc",
+    "gecko_sca_awm_forward_train",
+    "gecko_sca_awm_backward",
     "gecko_awm_state",
     "gecko_cema_forward",
     "gecko_tdnorm_forward",
@@ -63,6 +65,10 @@ def load() -> ctypes.CDLL:
     lib.gecko_sca_awm_forward_continue.restype = ctypes.c_int
     lib.gecko_sca_awm_forward_noalloc.argtypes = [vp] * 7 + [i64] * 5 + [ctypes.c_int, vp]
     lib.gecko_sca_awm_forward_noalloc.restype = ctypes.c_int
+    lib.gecko_sca_awm_forward_train.argtypes = [vp] * 8 + [i64] * 5 + [ctypes.c_int, vp]
+    lib.gecko_sca_awm_forward_train.restype = ctypes.c_int
+    lib.gecko_sca_awm_backward.argtypes = [vp] * 14 + [i64] * 5 + [ctypes.c_int, vp]
+    lib.gecko_sca_awm_backward.restype = ctypes.c_int
     lib.gecko_awm_state.argtypes = [vp, vp, i64, i64, i64, vp]
     lib.gecko_awm_state.restype = ctypes.c_int
     lib.gecko_cema_forward.argtypes = [vp] * 10 + [i64] * 4 + [ctypes.c_int, vp]
@@ -113,6 +119,18 @@ def gecko_sca_awm_forward_noalloc(q, k, v, qm, km, out_sca, out_mem, B, H, T, c,
     """The no-allocation entry point (fixed library scratch instead of a
     growable workspace), with integer pointers; returns the status."""
     return load().gecko_sca_awm_forward_noalloc(q, k, v, qm, km, out_sca, out_mem, B, H, T, c, d, dtype, stream)
+
+
+def gecko_sca_awm_forward_train(q, k, v, qm, km, out_sca, out_mem, lse, B, H, T, c, d, dtype, stream) -> int:
+    """The forward that also writes SCA's row log-sum-exp (for the backward)."""
+    return load().gecko_sca_awm_forward_train(q, k, v, qm, km, out_sca, out_mem, lse, B, H, T, c, d, dtype, stream)
+
+
+def gecko_sca_awm_backward(q, k, v, qm, km, out_sca, lse, dout_sca, dout_mem, dq, dk, dv, dqm, dkm,
+                           B, H, T, c, d, dtype, stream) -> int:
+    """Gradients of q, k, v, qm, km with integer pointers; returns the status."""
+    return load().gecko_sca_awm_backward(q, k, v, qm, km, out_sca, lse, dout_sca, dout_mem, dq, dk, dv, dqm, dkm,
+                                         B, H, T, c, d, dtype, stream)
 
 
 def gecko_awm_state(M_out, logz_out, B, H, d, stream) -> int:
@@ -181,6 +199,68 @@ def sca_awm_forward(q, k, v, qm, km, c: int, out_sca=None, out_mem=None, stream=
                                    B, H, T, c, d, _DT[q.dtype], _stream_handle(stream))
     _check(rc)
     return out_sca, out_mem
+
+
+def _check_inputs(xs):
+    q = xs[0]
+    for x in xs:
+        if not (isinstance(x, torch.Tensor) and x.is_cuda and x.is_contiguous()):
+            raise ValueError("inputs must be contiguous CUDA tensors")
+        if x.shape != q.shape or x.dtype != q.dtype or x.device != q.device:
+            raise ValueError("inputs must share shape, dtype and device")
+    if q.dim() != 4 or q.dtype not in _DT:
+        raise ValueError("inputs must be [B, H, T, d] float32 or bfloat16")
+
+
+def sca_awm_forward_train(q, k, v, qm, km, c: int, stream=None):
+    """Forward for training: returns (out_sca, out_mem, lse) with lse the
+    [B, H, T] fp32 row log-sum-exp of SCA that sca_awm_backward needs."""
+    xs = (q, k, v, qm, km)
+    _check_inputs(xs)
+    B, H, T, d = q.shape
+    out_sca, out_mem = torch.empty_like(q), torch.empty_like(q)
+    lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
+    with torch.cuda.device(q.device):
+        rc = gecko_sca_awm_forward_train(*(x.data_ptr() for x in xs), out_sca.data_ptr(), out_mem.data_ptr(),
+                                         lse.data_ptr(), B, H, T, c, d, _DT[q.dtype], _stream_handle(stream))
+    _check(rc)
+    return out_sca, out_mem, lse
+
+
+def sca_awm_backward(q, k, v, qm, km, out_sca, lse, dout_sca, dout_mem, c: int, stream=None):
+    """Gradients (dq, dk, dv, dqm, dkm) of the fused forward for the output
+    gradients dout_sca, dout_mem; out_sca and lse come from
+    sca_awm_forward_train on the same inputs."""
+    xs = (q, k, v, qm, km, out_sca, dout_sca.contiguous(), dout_mem.contiguous())
+    _check_inputs(xs)
+    if not (lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous() and lse.shape == q.shape[:3]):
+        raise ValueError("lse must be a contiguous [B, H, T] float32 CUDA tensor")
+    B, H, T, d = q.shape
+    grads = [torch.empty_like(q) for _ in range(5)]
+    with torch.cuda.device(q.device):
+        rc = gecko_sca_awm_backward(*(x.data_ptr() for x in xs[:6]), lse.data_ptr(), xs[6].data_ptr(),
+                                    xs[7].data_ptr(), *(g.data_ptr() for g in grads), B, H, T, c, d,
+                                    _DT[q.dtype], _stream_handle(stream))
+    _check(rc)
+    return tuple(grads)
+
+
+class ScaAwmFunction(torch.autograd.Function):
+    """torch.autograd wrapper of the fused forward and backward:
+    (out_sca, out_mem) = ScaAwmFunction.apply(q, k, v, qm, km, c)."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, qm, km, c):
+        out_sca, out_mem, lse = sca_awm_forward_train(q, k, v, qm, km, c)
+        ctx.save_for_backward(q, k, v, qm, km, out_sca, lse)
+        ctx.c = c
+        return out_sca, out_mem
+
+    @staticmethod
+    def backward(ctx, dout_sca, dout_mem):
+        q, k, v, qm, km, out_sca, lse = ctx.saved_tensors
+        grads = sca_awm_backward(q, k, v, qm, km, out_sca, lse, dout_sca, dout_mem, ctx.c)
+        return (*grads, None)
 
 
 def sca_awm_forward_segment(q, k, v, qm, km, c: int, state_in=None, out_sca=None, out_mem=None, stream=None):

@@ -114,3 +114,26 @@ def _tdnorm(ptrs=None, B=1, Lt=100, D=64, G=4, b1=0.9, b2=0.99, eps=1e-5, dtype=
 def test_tdnorm_host_validation_rejects(so, kw, code):
     assert _tdnorm(**kw) == code
     assert L.gecko_last_error()
+
+
+def _bwd(ptrs=None, B=1, H=1, T=256, c=128, d=64, dtype=1):
+    ptrs = ptrs or [FAKE] * 14
+    return L.gecko_sca_awm_backward(*ptrs, B, H, T, c, d, dtype, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ptrs=[FAKE] * 6 + [0] + [FAKE] * 7), 1),     # lse NULL
+    (dict(ptrs=[FAKE] * 13 + [0]), 1),                 # dkm NULL
+    (dict(ptrs=[FAKE] * 9 + [FAKE + 4] + [FAKE] * 4), 3),
+    (dict(d=32), 2),
+    (dict(T=300), 2),
+    (dict(dtype=2), 1),
+])
+def test_backward_host_validation_rejects(so, kw, code):
+    assert _bwd(**kw) == code
+    assert L.gecko_last_error()
+
+
+def test_train_forward_rejects_bad_lse(so):
+    assert L.gecko_sca_awm_forward_train(*[FAKE] * 7, 0, 1, 1, 256, 128, 64, 1, None) == 1
+    assert L.gecko_sca_awm_forward_train(*[FAKE] * 7, FAKE + 4, 1, 1, 256, 128, 64, 1, None) == 3
