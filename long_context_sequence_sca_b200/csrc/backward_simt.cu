@@ -44,10 +44,12 @@ __device__ __forceinline__ float warp_max(float x) {
 
 // ------------------------------------------------------------------ SCA --
 
-// delta_t = sum_f dO[t, f] O[t, f], one warp per row.
+// delta_t = sum_f dO[t, f] O[t, f], and -log2(e) l_t for the exp2 form of
+// the tensor-core kernels; one warp per row.
 template <typename TIn, int D>
 __global__ void __launch_bounds__(256) sca_bwd_delta_kernel(const TIn* __restrict__ out, const TIn* __restrict__ dout,
-                                                            float* __restrict__ delta, int64_t rows) {
+                                                            const float* __restrict__ lse, float* __restrict__ delta,
+                                                            float* __restrict__ nlse2, int64_t rows) {
   const int64_t row = (int64_t)blockIdx.x * 8 + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   if (row >= rows) return;  // uniform per warp
@@ -58,7 +60,10 @@ __global__ void __launch_bounds__(256) sca_bwd_delta_kernel(const TIn* __restric
     acc = fmaf(to_f32(out[g]), to_f32(dout[g]), acc);
   }
   acc = warp_sum(acc);
-  if (lane == 0) delta[row] = acc;
+  if (lane == 0) {
+    delta[row] = acc;
+    nlse2[row] = -kLog2e * lse[row];
+  }
 }
 
 // dQ: 32 queries per CTA, 4 threads per query (each owns D/4 dims), the
@@ -572,7 +577,7 @@ cudaError_t sca_bwd_delta_impl(const BwdProblem& b, const BwdWorkspace& w, cudaS
   const Problem& p = b.f;
   const int64_t rows = p.B * p.H * p.T;
   sca_bwd_delta_kernel<TIn, D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
-      static_cast<const TIn*>(b.out_sca), static_cast<const TIn*>(b.dout_sca), w.delta, rows);
+      static_cast<const TIn*>(b.out_sca), static_cast<const TIn*>(b.dout_sca), b.lse, w.delta, w.nlse2, rows);
   return cudaGetLastError();
 }
 
@@ -627,7 +632,7 @@ cudaError_t awm_bwd_impl(const BwdProblem& b, const Workspace& fw, const BwdWork
 size_t bwd_workspace_bytes(int64_t BH, int64_t T, int64_t c, int64_t d) {
   auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
   const int64_t S = T / c;
-  return al(sizeof(float) * BH * T) + al(sizeof(float) * BH * S * d * d) + al(sizeof(float) * BH * (S + 1) * d * d) +
+  return 2 * al(sizeof(float) * BH * T) + al(sizeof(float) * BH * S * d * d) + al(sizeof(float) * BH * (S + 1) * d * d) +
          al(sizeof(float) * BH * S * d) + al(sizeof(float) * BH * T * d);
 }
 
@@ -637,6 +642,8 @@ BwdWorkspace carve_bwd_workspace(void* base, int64_t BH, int64_t T, int64_t c, i
   char* p = static_cast<char*>(base);
   BwdWorkspace w;
   w.delta = reinterpret_cast<float*>(p);
+  p += al(sizeof(float) * BH * T);
+  w.nlse2 = reinterpret_cast<float*>(p);
   p += al(sizeof(float) * BH * T);
   w.E = reinterpret_cast<float*>(p);
   p += al(sizeof(float) * BH * S * d * d);

@@ -330,7 +330,9 @@ int run_backward(const void* q, const void* k, const void* v, const void* qm, co
   if ((rc = check_cuda(launch_awm_carry(p, w, st), "awm carry"))) return rc;
   if ((rc = check_cuda(launch_awm_bwd(b, w, bw, st), "awm backward"))) return rc;
   if ((rc = check_cuda(launch_sca_bwd_delta(b, bw, st), "sca backward delta"))) return rc;
-  if ((rc = check_cuda(launch_sca_bwd_simt(b, bw, st), "sca backward"))) return rc;
+  const bool use_tc = !env_is("GECKO_KERNELS", "simt") && tc_supported(p);
+  if ((rc = check_cuda(use_tc ? launch_sca_bwd_tc(b, bw, st) : launch_sca_bwd_simt(b, bw, st), "sca backward")))
+    return rc;
   ds->have_state = true;  // the rematerialised states are this sequence's
   ds->B = B;
   ds->H = H;

@@ -74,6 +74,7 @@ struct BwdProblem {
 
 struct BwdWorkspace {
   float* delta;   // [BH, T]  rowsum(dO * O) of SCA
+  float* nlse2;   // [BH, T]  -log2(e) * (SCA row log-sum-exp)
   float* E;       // [BH, S, d, d]  psi(Qm_s)^T dO_m,s
   float* G;       // [BH, S+1, d, d]  G_s = dLoss/dM'_s, s = 1..S+1
   float* dl;      // [BH, S, d]  dLoss/d log e_s
@@ -84,6 +85,7 @@ size_t bwd_workspace_bytes(int64_t BH, int64_t T, int64_t c, int64_t d);
 BwdWorkspace carve_bwd_workspace(void* base, int64_t BH, int64_t T, int64_t c, int64_t d);
 cudaError_t launch_sca_bwd_delta(const BwdProblem& b, const BwdWorkspace& w, cudaStream_t st);
 cudaError_t launch_sca_bwd_simt(const BwdProblem& b, const BwdWorkspace& w, cudaStream_t st);
+cudaError_t launch_sca_bwd_tc(const BwdProblem& b, const BwdWorkspace& w, cudaStream_t st);   // bf16, tc_supported
 cudaError_t launch_awm_bwd(const BwdProblem& b, const Workspace& fw, const BwdWorkspace& w, cudaStream_t st);
 
 // ---------------------------------------------------------------- CEMA --
