@@ -18,6 +18,9 @@ over ranks; rank 0 prints one JSON line.
 `--impl reference` times the CPU oracle (fp64 NumPy, the machine's host cores) on
 bounded samples of the same workload instead.
 
+`--op backward` measures gecko_sca_awm_backward on the same workload (the
+gradients of q, k, v, qm, km for N(0,1) output gradients); its roofline is
+the SCA dK/dV kernel against the bf16 tensor peak.
 `--op tdnorm` measures timestep decay normalisation on the same x shape
 (HBM roofline).  `--op cema` measures the CEMA recurrence (gecko_cema_forward) instead, on
 x [1, 32768, 4096] bf16 with h = 16, and prints its own JSON line (an FP32
@@ -694,6 +697,115 @@ def run_tdnorm(args, ws: int, rank: int, local: int) -> dict:
     return out
 
 
+BWD_METRIC = "tokens/s fused SCA+AWM backward (bf16,H=32,d=128,c=4096); % bf16 TC peak"
+BWD_PROFILE = os.path.join(ROOT, "profiles", "sca_bwd_tc_bf16_h32_c4096.md")
+# launches of one backward: AWM rebuild (lse partial, combine, prefix, chunk,
+# carry), AWM reverse pass (E, carry, dl, chunk, readout), SCA delta, SCA
+# dK/dV, SCA dQ
+BWD_LAUNCHES = 13
+
+
+def bwd_source_hash() -> str:
+    return source_hash(("sca_bwd_tc.cu", "common.cuh"))
+
+
+def run_backward(args, ws: int, rank: int, local: int) -> dict:
+    """One step = one gecko_sca_awm_backward on the bench workload (the
+    forward's outputs and row statistics prepared once, outside the timed
+    region; output gradients seeded N(0, 1))."""
+    from long_context_sequence_sca_b200 import lib as L
+    L.load()
+    w = WORKLOADS[DEFAULT_WORKLOAD]
+    x = make_inputs(w, device="cuda", seed_offset=1000 * rank)
+    names = ("q", "k", "v", "qm", "km")
+    g = torch.Generator(device="cuda").manual_seed(77 + rank)
+    dos = torch.randn(x["q"].shape, generator=g, device="cuda").to(x["q"].dtype)
+    dom = torch.randn(x["q"].shape, generator=g, device="cuda").to(x["q"].dtype)
+    stream = torch.cuda.current_stream()
+    out_sca, _, lse, lo = L.sca_awm_forward_train(*(x[n] for n in names), w.c, stream=stream)
+    grads = [None]
+
+    def step():
+        grads[0] = L.sca_awm_backward(*(x[n] for n in names), out_sca, lse, dos, dom, w.c, out_sca_lo=lo,
+                                      stream=stream)
+
+    L.timing_enable(True)
+    ms_local, ck, note = time_steps(args, ws, local, step, stream)
+    stage_tot, n_calls = L.timing_read_backward()
+    L.timing_enable(False)
+    stage_ms = {k: v / max(n_calls, 1) for k, v in stage_tot.items()}
+    tokens = w.B * w.T
+    agg = aggregate(ms_local, tokens, ws)
+    f = flops(w)
+    kv_ms = max_over_ranks(stage_ms["sca_dkdv"], ws)
+    pk, pk_kind = peaks()
+    f_kv = 2 * f["sca"]            # S^T, dP^T, dV and dK: four products of the SCA pair count
+    f_bwd = 5 * f["sca"] // 2      # the minimal SCA backward: recomputed S, dP, dV, dK, dQ
+    achieved = f_kv / (kv_ms / 1e3) / 1e12
+    out = {
+        "metric": BWD_METRIC, "value": round(agg["value"], 1), "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(agg["ms_per_step"], 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded Z'-affine generator, output gradients N(0,1); no dataset)",
+        "config": {"workload": w.name + "_backward", "B": w.B, "H": w.H, "T": w.T, "d": w.d, "c": w.c,
+                   "tokens_per_step_per_gpu": tokens,
+                   "l2": "inputs larger than L2 (2.7 GB incl. output gradients), no flush",
+                   "parallelism": f"replicas x{ws} (heads/batches independent)"},
+        "tflops_sca_algorithmic": round(f_bwd / (agg["ms_per_step"] / 1e3) / 1e12, 2),
+        "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()},
+        "roofline": {"bound": "tensor", "kernel": "sca_bwd_tc_kernel<128, false> (dK/dV)",
+                     "achieved": round(achieved, 2), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(achieved / pk["bf16_tflops"], 4),
+                     "peak_kind": f"{pk_kind} bf16 dense (burst)",
+                     "frac_of_sustained": round(achieved / pk.get("bf16_tflops_sustained", pk["bf16_tflops"]), 4),
+                     "traffic": recorded_traffic(WORKLOADS[DEFAULT_WORKLOAD], BWD_PROFILE, bwd_source_hash()),
+                     "launch_ms": round(kv_ms, 4), "algorithmic_flop_per_launch": f_kv},
+        "clocks": ck,
+        "gpu_launches": BWD_LAUNCHES * args.steps,
+    }
+    if note:
+        out["note"] = note
+    if not args.no_e2e:
+        dev_in = [x[n] for n in names] + [out_sca, lse, dos, dom, lo]
+        host_in = [t.cpu().pin_memory() for t in dev_in]
+        host_out = [torch.empty_like(x["q"], device="cpu").pin_memory() for _ in range(5)]
+        staged = [torch.empty_like(t) for t in dev_in]
+
+        def e2e_step():
+            for d_, h_ in zip(staged, host_in):
+                d_.copy_(h_, non_blocking=True)
+            gr = L.sca_awm_backward(*staged[:5], staged[5], staged[6], staged[7], staged[8], w.c,
+                                    out_sca_lo=staged[9], stream=stream)
+            for h_, d_ in zip(host_out, gr):
+                h_.copy_(d_, non_blocking=True)
+
+        e_args = argparse.Namespace(steps=max(1, min(args.steps, 5)), warmup=3)
+        ems, _, _ = time_steps(e_args, ws, local, e2e_step, stream)
+        ea = aggregate(ems, tokens, ws)
+        out["e2e"] = {"value": round(ea["value"], 1), "unit": "tokens/s",
+                      "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in dev_in),
+                      "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in host_out),
+                      "steps": e_args.steps, "ms_per_step": round(ea["ms_per_step"], 3),
+                      "pipelining": "none (copy in, backward, copy out in one stream)"}
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        from oracle import gecko_backward_oracle as GB
+        n_ch = 2
+        rows = slice(0, n_ch * w.c)
+        xs = [x[n][0, 0, rows].double().cpu().numpy() for n in names]
+        do_s = dos[0, 0, rows].double().cpu().numpy()
+        do_m = dom[0, 0, rows].double().cpu().numpy()
+        t0 = time.perf_counter()
+        GB.sca_head_backward(xs[0], xs[1], xs[2], w.c, do_s)
+        GB.awm_head_backward(xs[3], xs[4], xs[2], w.c, do_m)
+        secs = time.perf_counter() - t0
+        out["cpu_baseline"] = {"value": round(n_ch * w.c / w.H / secs, 2), "unit": "tokens/s", "cores": blas_threads(),
+                               "kind": "oracle",
+                               "sample": f"fp64 gradient oracle on the first {n_ch} chunks of 1 of {w.H} heads "
+                                         f"({n_ch * w.c} rows, c={w.c}, d={w.d}) in {secs:.1f} s; tokens counted "
+                                         f"as rows / H (a token carries all H heads)"}
+    return out
+
+
 def summarize_launches(path: str) -> str:
     """Per-kernel launches, total time and share from an ncu launch-list CSV
     (`ncu --metrics gpu__time_duration.sum --csv`)."""
@@ -733,9 +845,9 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=("sca_awm", "cema", "tdnorm"), default="sca_awm",
-                    help="sca_awm: the fused SCA + AWM forward (default); cema: the CEMA recurrence; "
-                         "tdnorm: timestep decay normalisation")
+    ap.add_argument("--op", choices=("sca_awm", "backward", "cema", "tdnorm"), default="sca_awm",
+                    help="sca_awm: the fused SCA + AWM forward (default); backward: its gradients; "
+                         "cema: the CEMA recurrence; tdnorm: timestep decay normalisation")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -752,7 +864,8 @@ def main(argv=None):
     if ws != args.gpus and rank == 0:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE {ws}", file=sys.stderr)
     try:
-        runner = {"cema": lambda: run_cema(args, ws, rank, local), "tdnorm": lambda: run_tdnorm(args, ws, rank, local)}
+        runner = {"cema": lambda: run_cema(args, ws, rank, local), "tdnorm": lambda: run_tdnorm(args, ws, rank, local),
+                  "backward": lambda: run_backward(args, ws, rank, local)}
         out = runner[args.op]() if args.op in runner else run_gecko(args, w, ws, rank, local)
         if rank == 0:
             print(json.dumps(out), flush=True)

@@ -94,13 +94,18 @@ int gecko_sca_awm_forward(const void* q, const void* k, const void* v,
  * row's visible scores (the softmax normaliser of SCA, Gecko digest, method
  * step details, step 3).
  *
- *   lse : [B, H, T] fp32 (device), 16-byte aligned; fully overwritten.
+ *   lse        : [B, H, T] fp32 (device), 16-byte aligned; fully overwritten.
+ *   out_sca_lo : NULL, or [B, H, T, d] dtype (device), 16-byte aligned: the
+ *                rounding residual of out_sca (the exact output minus the
+ *                stored one, rounded to dtype; zero for GECKO_F32).  The
+ *                backward's row term rowsum(dO * O) cancels strongly at long
+ *                windows, and with bf16 O alone its error dominates dq.
  *
  * Everything else as gecko_sca_awm_forward (same outputs, bit for bit).
  */
 int gecko_sca_awm_forward_train(const void* q, const void* k, const void* v,
                                 const void* qm, const void* km,
-                                void* out_sca, void* out_mem, float* lse,
+                                void* out_sca, void* out_mem, float* lse, void* out_sca_lo,
                                 int64_t B, int64_t H, int64_t T, int64_t c, int64_t d,
                                 int dtype, void* stream);
 
@@ -114,8 +119,9 @@ int gecko_sca_awm_forward_train(const void* q, const void* k, const void* v,
  * are rebuilt here from qm, km, v, so the forward keeps nothing but lse.
  *
  *   q, k, v, qm, km : the forward's inputs, [B, H, T, d] dtype (device).
- *   out_sca, lse    : the forward's SCA output and lse
- *                     (gecko_sca_awm_forward_train).
+ *   out_sca, out_sca_lo, lse : the forward's SCA output, its residual
+ *                     (may be NULL: then O is taken as out_sca alone) and
+ *                     lse (gecko_sca_awm_forward_train).
  *   dout_sca, dout_mem : gradients of out_sca and out_mem, [B, H, T, d].
  *   dq, dk, dv, dqm, dkm : [B, H, T, d] dtype (device), fully overwritten;
  *                     dv sums the SCA and AWM parts (v feeds both).  They
@@ -131,7 +137,7 @@ int gecko_sca_awm_forward_train(const void* q, const void* k, const void* v,
  */
 int gecko_sca_awm_backward(const void* q, const void* k, const void* v,
                            const void* qm, const void* km,
-                           const void* out_sca, const float* lse,
+                           const void* out_sca, const void* out_sca_lo, const float* lse,
                            const void* dout_sca, const void* dout_mem,
                            void* dq, void* dk, void* dv, void* dqm, void* dkm,
                            int64_t B, int64_t H, int64_t T, int64_t c, int64_t d,
@@ -244,6 +250,10 @@ int gecko_device_status(void* stream);
  */
 int gecko_timing_enable(int enable);
 int gecko_timing_read(float* ms_per_stage, int capacity, int* n_calls);
+/* The same for the backward (gecko_sca_awm_backward), five stages in order:
+ * AWM state rebuild (stats, chunk products, carry), AWM reverse pass, SCA
+ * row statistics, SCA dK/dV, SCA dQ. */
+int gecko_timing_read_backward(float* ms_per_stage, int capacity, int* n_calls);
 
 /*
  * gecko_cema_forward - CEMA, the complex multi-dimensional damped

@@ -44,10 +44,12 @@ __device__ __forceinline__ float warp_max(float x) {
 
 // ------------------------------------------------------------------ SCA --
 
-// delta_t = sum_f dO[t, f] O[t, f], and -log2(e) l_t for the exp2 form of
+// delta_t = sum_f dO[t, f] O[t, f] (O = stored output + its rounding
+// residual when the forward kept it), and -log2(e) l_t for the exp2 form of
 // the tensor-core kernels; one warp per row.
 template <typename TIn, int D>
-__global__ void __launch_bounds__(256) sca_bwd_delta_kernel(const TIn* __restrict__ out, const TIn* __restrict__ dout,
+__global__ void __launch_bounds__(256) sca_bwd_delta_kernel(const TIn* __restrict__ out, const TIn* __restrict__ out_lo,
+                                                            const TIn* __restrict__ dout,
                                                             const float* __restrict__ lse, float* __restrict__ delta,
                                                             float* __restrict__ nlse2, int64_t rows) {
   const int64_t row = (int64_t)blockIdx.x * 8 + threadIdx.x / 32;
@@ -57,7 +59,8 @@ __global__ void __launch_bounds__(256) sca_bwd_delta_kernel(const TIn* __restric
 #pragma unroll
   for (int i = 0; i < D / 32; ++i) {
     const int64_t g = row * D + lane + 32 * i;
-    acc = fmaf(to_f32(out[g]), to_f32(dout[g]), acc);
+    const float o = to_f32(out[g]) + (out_lo ? to_f32(out_lo[g]) : 0.f);
+    acc = fmaf(o, to_f32(dout[g]), acc);
   }
   acc = warp_sum(acc);
   if (lane == 0) {
@@ -577,21 +580,24 @@ cudaError_t sca_bwd_delta_impl(const BwdProblem& b, const BwdWorkspace& w, cudaS
   const Problem& p = b.f;
   const int64_t rows = p.B * p.H * p.T;
   sca_bwd_delta_kernel<TIn, D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
-      static_cast<const TIn*>(b.out_sca), static_cast<const TIn*>(b.dout_sca), b.lse, w.delta, w.nlse2, rows);
+      static_cast<const TIn*>(b.out_sca), static_cast<const TIn*>(b.out_sca_lo), static_cast<const TIn*>(b.dout_sca),
+      b.lse, w.delta, w.nlse2, rows);
   return cudaGetLastError();
 }
 
 template <typename TIn, int D>
-cudaError_t sca_bwd_simt_impl(const BwdProblem& b, const BwdWorkspace& w, cudaStream_t st) {
+cudaError_t sca_bwd_simt_impl(const BwdProblem& b, const BwdWorkspace& w, cudaStream_t st, int part) {
   const Problem& p = b.f;
   const dim3 grid((unsigned)(p.T / 32), (unsigned)(p.B * p.H));
-  sca_bwd_dq_simt_kernel<TIn, D><<<grid, 128, 0, st>>>(
-      static_cast<const TIn*>(p.q), static_cast<const TIn*>(p.k), static_cast<const TIn*>(p.v),
-      static_cast<const TIn*>(b.dout_sca), b.lse, w.delta, static_cast<TIn*>(b.dq), p.T, (int)p.c);
-  sca_bwd_dkdv_simt_kernel<TIn, D><<<grid, 128, 0, st>>>(
-      static_cast<const TIn*>(p.q), static_cast<const TIn*>(p.k), static_cast<const TIn*>(p.v),
-      static_cast<const TIn*>(b.dout_sca), b.lse, w.delta, w.dv_awm, static_cast<TIn*>(b.dk),
-      static_cast<TIn*>(b.dv), p.T, (int)p.c);
+  if (part == 0)
+    sca_bwd_dkdv_simt_kernel<TIn, D><<<grid, 128, 0, st>>>(
+        static_cast<const TIn*>(p.q), static_cast<const TIn*>(p.k), static_cast<const TIn*>(p.v),
+        static_cast<const TIn*>(b.dout_sca), b.lse, w.delta, w.dv_awm, static_cast<TIn*>(b.dk),
+        static_cast<TIn*>(b.dv), p.T, (int)p.c);
+  else
+    sca_bwd_dq_simt_kernel<TIn, D><<<grid, 128, 0, st>>>(
+        static_cast<const TIn*>(p.q), static_cast<const TIn*>(p.k), static_cast<const TIn*>(p.v),
+        static_cast<const TIn*>(b.dout_sca), b.lse, w.delta, static_cast<TIn*>(b.dq), p.T, (int)p.c);
   return cudaGetLastError();
 }
 
@@ -662,8 +668,8 @@ BwdWorkspace carve_bwd_workspace(void* base, int64_t BH, int64_t T, int64_t c, i
 cudaError_t launch_sca_bwd_delta(const BwdProblem& b, const BwdWorkspace& w, cudaStream_t st) {
   return GECKO_BWD_DISPATCH(sca_bwd_delta_impl, b, w, st);
 }
-cudaError_t launch_sca_bwd_simt(const BwdProblem& b, const BwdWorkspace& w, cudaStream_t st) {
-  return GECKO_BWD_DISPATCH(sca_bwd_simt_impl, b, w, st);
+cudaError_t launch_sca_bwd_simt(const BwdProblem& b, const BwdWorkspace& w, cudaStream_t st, int part) {
+  return GECKO_BWD_DISPATCH(sca_bwd_simt_impl, b, w, st, part);
 }
 cudaError_t launch_awm_bwd(const BwdProblem& b, const Workspace& fw, const BwdWorkspace& w, cudaStream_t st) {
   return GECKO_BWD_DISPATCH(awm_bwd_impl, b, fw, w, st);

@@ -142,12 +142,19 @@ int validate(const void* const* ptrs, int n, int64_t B, int64_t H, int64_t T, in
 }
 
 // Optional per-stage timing with CUDA events recorded on the caller's
-// stream around each stage of a forward; accumulated until read.
-constexpr int kStages = 5;  // awm stats, awm chunk, awm carry, awm readout, sca
+// stream around each stage of a forward or backward; accumulated until read.
+constexpr int kStages = 5;     // forward: awm stats, awm chunk, awm carry, awm readout, sca
+constexpr int kBwdStages = 5;  // backward: awm rebuild, awm backward, sca delta, sca dK/dV, sca dQ
 std::atomic<bool> g_timing{false};
 std::mutex g_tmu;
-std::vector<std::array<cudaEvent_t, kStages + 1>> g_pending;
 std::vector<cudaEvent_t> g_event_pool;
+
+template <int N>
+struct StageLog {
+  std::vector<std::array<cudaEvent_t, N + 1>> pending;
+};
+StageLog<kStages> g_fwd_log;
+StageLog<kBwdStages> g_bwd_log;
 
 cudaEvent_t take_event() {
   if (!g_event_pool.empty()) {
@@ -160,11 +167,13 @@ cudaEvent_t take_event() {
   return e;
 }
 
-struct StageEvents {
+template <int N>
+struct StageEventsT {
   cudaStream_t st;
   bool on;
-  std::array<cudaEvent_t, kStages + 1> ev{};
-  explicit StageEvents(cudaStream_t s) : st(s), on(g_timing.load()) {
+  StageLog<N>& log;
+  std::array<cudaEvent_t, N + 1> ev{};
+  StageEventsT(cudaStream_t s, StageLog<N>& l) : st(s), on(g_timing.load()), log(l) {
     if (on) {
       std::lock_guard<std::mutex> lk(g_tmu);
       for (auto& e : ev) e = take_event();
@@ -176,15 +185,44 @@ struct StageEvents {
   void commit() {
     if (!on) return;
     std::lock_guard<std::mutex> lk(g_tmu);
-    g_pending.push_back(ev);
+    log.pending.push_back(ev);
     on = false;
   }
-  ~StageEvents() {
+  ~StageEventsT() {
     if (!on) return;  // an error path: recycle the events
     std::lock_guard<std::mutex> lk(g_tmu);
     for (auto& e : ev) g_event_pool.push_back(e);
   }
 };
+
+struct StageEvents : StageEventsT<kStages> {
+  explicit StageEvents(cudaStream_t s) : StageEventsT<kStages>(s, g_fwd_log) {}
+};
+struct BwdStageEvents : StageEventsT<kBwdStages> {
+  explicit BwdStageEvents(cudaStream_t s) : StageEventsT<kBwdStages>(s, g_bwd_log) {}
+};
+
+// Sum of each stage's time over the logged calls; the log is emptied.
+template <int N>
+int read_stage_log(StageLog<N>& log, float* ms_per_stage, int capacity, int* n_calls) {
+  if (!ms_per_stage || !n_calls || capacity < 1) return fail(GECKO_ERR_ARG, "bad timing buffers");
+  std::lock_guard<std::mutex> lk(g_tmu);
+  double acc[N] = {0};
+  for (auto& evs : log.pending) {
+    cudaError_t e = cudaEventSynchronize(evs[N]);
+    if (e != cudaSuccess) return check_cuda(e, "event synchronize");
+    for (int i = 0; i < N; ++i) {
+      float ms = 0.f;
+      cudaEventElapsedTime(&ms, evs[i], evs[i + 1]);
+      acc[i] += ms;
+    }
+    for (auto& x : evs) g_event_pool.push_back(x);
+  }
+  *n_calls = (int)log.pending.size();
+  log.pending.clear();
+  for (int i = 0; i < N && i < capacity; ++i) ms_per_stage[i] = (float)acc[i];
+  return GECKO_OK;
+}
 
 }  // namespace
 }  // namespace gecko
@@ -218,7 +256,8 @@ int ensure_buffer(void** buf, size_t* have, size_t need, cudaStream_t st, const 
 // or host).  state_out, if given, receives (M'_S, M'_{S+1}, log z^S).
 int run_forward(const void* q, const void* k, const void* v, const void* qm, const void* km, void* out_sca,
                 void* out_mem, const float* state_in, float* state_out, int64_t B, int64_t H, int64_t T,
-                int64_t c, int64_t d, int dtype, void* stream, float* lse = nullptr) {
+                int64_t c, int64_t d, int dtype, void* stream, float* lse = nullptr,
+                void* out_sca_lo = nullptr) {
   const void* ptrs[7] = {q, k, v, qm, km, out_sca, out_mem};
   int rc = validate(ptrs, 7, B, H, T, c, d, dtype);
   if (rc) return rc;
@@ -239,6 +278,7 @@ int run_forward(const void* q, const void* k, const void* v, const void* qm, con
 
   Problem p{q, k, v, qm, km, out_sca, out_mem, B, H, T, c, d, (int)S, dtype, ds->status};
   p.lse = lse;
+  p.out_sca_lo = out_sca_lo;
   if (state_in) {
     // private copy, so state_out may alias state_in
     if ((rc = ensure_buffer(&ds->state, &ds->state_bytes, sizeof(float) * BH * sd, st, "state copy"))) return rc;
@@ -296,12 +336,14 @@ int run_forward(const void* q, const void* k, const void* v, const void* qm, con
 // forward kernels, then the AWM reverse pass, then the SCA gradients (whose
 // dV kernel adds the AWM part of dV).
 int run_backward(const void* q, const void* k, const void* v, const void* qm, const void* km, const void* out_sca,
-                 const float* lse, const void* dout_sca, const void* dout_mem, void* dq, void* dk, void* dv,
+                 const void* out_sca_lo, const float* lse, const void* dout_sca, const void* dout_mem, void* dq, void* dk, void* dv,
                  void* dqm, void* dkm, int64_t B, int64_t H, int64_t T, int64_t c, int64_t d, int dtype,
                  void* stream) {
   const void* ptrs[14] = {q, k, v, qm, km, out_sca, lse, dout_sca, dout_mem, dq, dk, dv, dqm, dkm};
   int rc = validate(ptrs, 14, B, H, T, c, d, dtype);
   if (rc) return rc;
+  if (reinterpret_cast<uintptr_t>(out_sca_lo) % 16 != 0)
+    return fail(GECKO_ERR_ALIGN, "out_sca_lo is not 16-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int dev = 0;
   if ((rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice"))) return rc;
@@ -318,21 +360,31 @@ int run_backward(const void* q, const void* k, const void* v, const void* qm, co
   Workspace w = carve_workspace(ds->ws, BH, T, c, d);
   BwdWorkspace bw = carve_bwd_workspace(ds->bwd_ws, BH, T, c, d);
   BwdProblem b{Problem{q, k, v, qm, km, nullptr, nullptr, B, H, T, c, d, (int)S, dtype, ds->status},
-               out_sca, lse, dout_sca, dout_mem, dq, dk, dv, dqm, dkm};
+               out_sca, out_sca_lo, lse, dout_sca, dout_mem, dq, dk, dv, dqm, dkm};
   const Problem& p = b.f;
 
+  const bool use_tc = !env_is("GECKO_KERNELS", "simt") && tc_supported(p);
   cudaGetLastError();
+  BwdStageEvents ev(st);
+  ev.mark(0);
   if ((rc = check_cuda(launch_awm_stats(p, w, st), "awm stats"))) return rc;
   // The chunk products are rebuilt in fp32: the rows of M' are close to one
   // another (each is a running average of V), and the softmax gradient of
   // the readout keeps only their differences, which bf16 operands blur.
   if ((rc = check_cuda(launch_awm_chunk_simt(p, w, st), "awm chunk"))) return rc;
   if ((rc = check_cuda(launch_awm_carry(p, w, st), "awm carry"))) return rc;
+  ev.mark(1);
   if ((rc = check_cuda(launch_awm_bwd(b, w, bw, st), "awm backward"))) return rc;
+  ev.mark(2);
   if ((rc = check_cuda(launch_sca_bwd_delta(b, bw, st), "sca backward delta"))) return rc;
-  const bool use_tc = !env_is("GECKO_KERNELS", "simt") && tc_supported(p);
-  if ((rc = check_cuda(use_tc ? launch_sca_bwd_tc(b, bw, st) : launch_sca_bwd_simt(b, bw, st), "sca backward")))
-    return rc;
+  ev.mark(3);
+  for (int part = 0; part < 2; ++part) {   // dK/dV (with the AWM part of dV), then dQ
+    if ((rc = check_cuda(use_tc ? launch_sca_bwd_tc(b, bw, st, part) : launch_sca_bwd_simt(b, bw, st, part),
+                         "sca backward")))
+      return rc;
+    ev.mark(4 + part);
+  }
+  ev.commit();
   ds->have_state = true;  // the rematerialised states are this sequence's
   ds->B = B;
   ds->H = H;
@@ -346,20 +398,24 @@ int run_backward(const void* q, const void* k, const void* v, const void* qm, co
 }  // namespace gecko
 
 extern "C" int gecko_sca_awm_forward_train(const void* q, const void* k, const void* v, const void* qm,
-                                           const void* km, void* out_sca, void* out_mem, float* lse, int64_t B,
-                                           int64_t H, int64_t T, int64_t c, int64_t d, int dtype, void* stream) {
+                                           const void* km, void* out_sca, void* out_mem, float* lse,
+                                           void* out_sca_lo, int64_t B, int64_t H, int64_t T, int64_t c, int64_t d,
+                                           int dtype, void* stream) {
   if (!lse) return fail(GECKO_ERR_ARG, "lse is NULL");
   if (reinterpret_cast<uintptr_t>(lse) % 16 != 0) return fail(GECKO_ERR_ALIGN, "lse is not 16-byte aligned");
-  return run_forward(q, k, v, qm, km, out_sca, out_mem, nullptr, nullptr, B, H, T, c, d, dtype, stream, lse);
+  if (reinterpret_cast<uintptr_t>(out_sca_lo) % 16 != 0)
+    return fail(GECKO_ERR_ALIGN, "out_sca_lo is not 16-byte aligned");
+  return run_forward(q, k, v, qm, km, out_sca, out_mem, nullptr, nullptr, B, H, T, c, d, dtype, stream, lse,
+                     out_sca_lo);
 }
 
 extern "C" int gecko_sca_awm_backward(const void* q, const void* k, const void* v, const void* qm, const void* km,
-                                      const void* out_sca, const float* lse, const void* dout_sca,
-                                      const void* dout_mem, void* dq, void* dk, void* dv, void* dqm, void* dkm,
-                                      int64_t B, int64_t H, int64_t T, int64_t c, int64_t d, int dtype,
-                                      void* stream) {
-  return run_backward(q, k, v, qm, km, out_sca, lse, dout_sca, dout_mem, dq, dk, dv, dqm, dkm, B, H, T, c, d, dtype,
-                      stream);
+                                      const void* out_sca, const void* out_sca_lo, const float* lse,
+                                      const void* dout_sca, const void* dout_mem, void* dq, void* dk, void* dv,
+                                      void* dqm, void* dkm, int64_t B, int64_t H, int64_t T, int64_t c, int64_t d,
+                                      int dtype, void* stream) {
+  return run_backward(q, k, v, qm, km, out_sca, out_sca_lo, lse, dout_sca, dout_mem, dq, dk, dv, dqm, dkm, B, H, T,
+                      c, d, dtype, stream);
 }
 
 extern "C" int gecko_sca_awm_forward(const void* q, const void* k, const void* v, const void* qm, const void* km,
@@ -463,23 +519,11 @@ extern "C" int gecko_timing_enable(int enable) {
 }
 
 extern "C" int gecko_timing_read(float* ms_per_stage, int capacity, int* n_calls) {
-  if (!ms_per_stage || !n_calls || capacity < 1) return fail(GECKO_ERR_ARG, "bad timing buffers");
-  std::lock_guard<std::mutex> lk(g_tmu);
-  double acc[kStages] = {0};
-  for (auto& evs : g_pending) {
-    cudaError_t e = cudaEventSynchronize(evs[kStages]);
-    if (e != cudaSuccess) return check_cuda(e, "event synchronize");
-    for (int i = 0; i < kStages; ++i) {
-      float ms = 0.f;
-      cudaEventElapsedTime(&ms, evs[i], evs[i + 1]);
-      acc[i] += ms;
-    }
-    for (auto& x : evs) g_event_pool.push_back(x);
-  }
-  *n_calls = (int)g_pending.size();
-  g_pending.clear();
-  for (int i = 0; i < kStages && i < capacity; ++i) ms_per_stage[i] = (float)acc[i];
-  return GECKO_OK;
+  return read_stage_log(g_fwd_log, ms_per_stage, capacity, n_calls);
+}
+
+extern "C" int gecko_timing_read_backward(float* ms_per_stage, int capacity, int* n_calls) {
+  return read_stage_log(g_bwd_log, ms_per_stage, capacity, n_calls);
 }
 
 extern "C" int gecko_sca_awm_forward_noalloc(const void* q, const void* k, const void* v, const void* qm,

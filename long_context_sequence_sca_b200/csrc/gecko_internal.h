@@ -22,6 +22,7 @@ struct Problem {
   int64_t koff = 0;              // rows of the previous chunk prepended to k and v per head (0 or c)
   const float* state0 = nullptr; // [BH, 2 d^2 + d] carried state (device): M'_prev, M'_cur, log z
   float* lse = nullptr;          // [BH, T] SCA row log-sum-exp (natural log), written if set
+  void* out_sca_lo = nullptr;    // [BH, T, d] rounding residual of out_sca (O - rounded O), written if set
 };
 
 // Floats per (b, h) in a carried state record: M'_prev, M'_cur (d x d each), log z (d).
@@ -67,6 +68,7 @@ cudaError_t launch_awm_readout_tc(const Problem& p, const Workspace& w, cudaStre
 struct BwdProblem {
   Problem f;
   const void* out_sca;
+  const void* out_sca_lo;   // may be null
   const float* lse;
   const void *dout_sca, *dout_mem;
   void *dq, *dk, *dv, *dqm, *dkm;
@@ -84,8 +86,9 @@ struct BwdWorkspace {
 size_t bwd_workspace_bytes(int64_t BH, int64_t T, int64_t c, int64_t d);
 BwdWorkspace carve_bwd_workspace(void* base, int64_t BH, int64_t T, int64_t c, int64_t d);
 cudaError_t launch_sca_bwd_delta(const BwdProblem& b, const BwdWorkspace& w, cudaStream_t st);
-cudaError_t launch_sca_bwd_simt(const BwdProblem& b, const BwdWorkspace& w, cudaStream_t st);
-cudaError_t launch_sca_bwd_tc(const BwdProblem& b, const BwdWorkspace& w, cudaStream_t st);   // bf16, tc_supported
+// part 0: dK and dV (adding the AWM part of dV); part 1: dQ
+cudaError_t launch_sca_bwd_simt(const BwdProblem& b, const BwdWorkspace& w, cudaStream_t st, int part);
+cudaError_t launch_sca_bwd_tc(const BwdProblem& b, const BwdWorkspace& w, cudaStream_t st, int part);  // bf16, tc_supported
 cudaError_t launch_awm_bwd(const BwdProblem& b, const Workspace& fw, const BwdWorkspace& w, cudaStream_t st);
 
 // ---------------------------------------------------------------- CEMA --

@@ -384,7 +384,7 @@ cudaError_t bwd_map(CUtensorMap* m, const void* base, int64_t rows, int d) {
 }
 
 template <int D>
-cudaError_t launch_sca_bwd_tc_impl(const BwdProblem& b, const BwdWorkspace& w, cudaStream_t st) {
+cudaError_t launch_sca_bwd_tc_impl(const BwdProblem& b, const BwdWorkspace& w, cudaStream_t st, int part) {
   using Cfg = BwdCfg<D>;
   const Problem& p = b.f;
   const int64_t rows = p.B * p.H * p.T;
@@ -402,21 +402,21 @@ cudaError_t launch_sca_bwd_tc_impl(const BwdProblem& b, const BwdWorkspace& w, c
   if ((e = cudaFuncSetAttribute(sca_bwd_tc_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 Cfg::kAlloc)) != cudaSuccess)
     return e;
-  // dK, dV (the AWM part of dV is added in the epilogue)
-  sca_bwd_tc_kernel<D, false><<<grid, kBwdThreads, Cfg::kAlloc, st>>>(
-      mk, mv, mq, mdo, w.nlse2, w.delta, w.dv_awm, static_cast<__nv_bfloat16*>(b.dv),
-      static_cast<__nv_bfloat16*>(b.dk), T, c, p.status);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  // dQ
-  sca_bwd_tc_kernel<D, true><<<grid, kBwdThreads, Cfg::kAlloc, st>>>(
-      mq, mdo, mk, mv, w.nlse2, w.delta, nullptr, static_cast<__nv_bfloat16*>(b.dq), nullptr, T, c, p.status);
+  if (part == 0)
+    // dK, dV (the AWM part of dV is added in the epilogue)
+    sca_bwd_tc_kernel<D, false><<<grid, kBwdThreads, Cfg::kAlloc, st>>>(
+        mk, mv, mq, mdo, w.nlse2, w.delta, w.dv_awm, static_cast<__nv_bfloat16*>(b.dv),
+        static_cast<__nv_bfloat16*>(b.dk), T, c, p.status);
+  else
+    sca_bwd_tc_kernel<D, true><<<grid, kBwdThreads, Cfg::kAlloc, st>>>(
+        mq, mdo, mk, mv, w.nlse2, w.delta, nullptr, static_cast<__nv_bfloat16*>(b.dq), nullptr, T, c, p.status);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_sca_bwd_tc(const BwdProblem& b, const BwdWorkspace& w, cudaStream_t st) {
-  return b.f.d == 64 ? launch_sca_bwd_tc_impl<64>(b, w, st) : launch_sca_bwd_tc_impl<128>(b, w, st);
+cudaError_t launch_sca_bwd_tc(const BwdProblem& b, const BwdWorkspace& w, cudaStream_t st, int part) {
+  return b.f.d == 64 ? launch_sca_bwd_tc_impl<64>(b, w, st, part) : launch_sca_bwd_tc_impl<128>(b, w, st, part);
 }
 
 }  // namespace gecko

@@ -206,7 +206,7 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
               const __grid_constant__ CUtensorMap map_v, __nv_bfloat16* __restrict__ out,
-              float* __restrict__ lse, int T, int c, int BH,
+              float* __restrict__ lse, __nv_bfloat16* __restrict__ out_lo, int T, int c, int BH,
               int n_units, int koff, unsigned* unit_counter, int* status) {
   using Cfg = ScaCfg<D>;
   constexpr int KS = Cfg::kKStages, VS = Cfg::kVStages;
@@ -570,6 +570,18 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
         uint4* dst = reinterpret_cast<uint4*>(orow + cb * 32);
 #pragma unroll
         for (int x = 0; x < 4; ++x) dst[x] = w[x];
+        if (out_lo) {
+          // what the bf16 output dropped, for a backward that needs O more
+          // exactly (its row term rowsum(dO * O) cancels at long windows)
+#pragma unroll
+          for (int x = 0; x < 16; ++x) {
+            const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wp[x]));
+            wp[x] = pack_bf16x2(__uint_as_float(o[2 * x]) * inv - hi.x, __uint_as_float(o[2 * x + 1]) * inv - hi.y);
+          }
+          uint4* dlo = reinterpret_cast<uint4*>(out_lo + (orow - out) + cb * 32);
+#pragma unroll
+          for (int x = 0; x < 4; ++x) dlo[x] = w[x];
+        }
       }
       tc_fence_before();
       mbar_arrive(o_empty + i);
@@ -647,7 +659,8 @@ cudaError_t launch_sca_tc_impl(const Problem& p, cudaStream_t st) {
   unsigned* counter = nullptr;
   if ((e = cudaGetSymbolAddress(reinterpret_cast<void**>(&counter), g_unit_counter)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(counter, 0, sizeof(unsigned), st)) != cudaSuccess) return e;
-  sca_tc_kernel<D><<<grid, kThreads, Cfg::kAlloc, st>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(p.out_sca), p.lse, T,
+  sca_tc_kernel<D><<<grid, kThreads, Cfg::kAlloc, st>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(p.out_sca), p.lse,
+                                                        static_cast<__nv_bfloat16*>(p.out_sca_lo), T,
                                                         (int)p.c, BH, n_units, (int)p.koff, counter, p.status);
   return cudaGetLastError();
 }

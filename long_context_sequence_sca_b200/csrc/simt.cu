@@ -372,7 +372,8 @@ __global__ void __launch_bounds__(256) awm_readout_simt_kernel(const TIn* __rest
 template <typename TIn, int D>
 __global__ void __launch_bounds__(128) sca_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
                                                        const TIn* __restrict__ v, TIn* __restrict__ out,
-                                                       float* __restrict__ lse, int64_t T, int c, int64_t koff) {
+                                                       float* __restrict__ lse, TIn* __restrict__ out_lo,
+                                                       int64_t T, int c, int64_t koff) {
   constexpr int QD = D / 4;
   __shared__ float ks[32][D + 4];
   __shared__ float vs[32][D + 4];
@@ -421,6 +422,15 @@ __global__ void __launch_bounds__(128) sca_simt_kernel(const TIn* __restrict__ q
   TIn* orow = out + (bh * T + t) * D + part * QD;
 #pragma unroll
   for (int i = 0; i < QD; ++i) orow[i] = from_f32<TIn>(acc[i] * inv);
+  if (out_lo) {
+    // rounding residual of the stored output (zero for fp32)
+    TIn* lrow = out_lo + (bh * T + t) * D + part * QD;
+#pragma unroll
+    for (int i = 0; i < QD; ++i) {
+      const float x = acc[i] * inv;
+      lrow[i] = from_f32<TIn>(x - to_f32(from_f32<TIn>(x)));
+    }
+  }
 }
 
 template <typename TIn, int D>
@@ -473,7 +483,7 @@ template <typename TIn, int D>
 cudaError_t launch_sca_simt_impl(const Problem& p, cudaStream_t st) {
   sca_simt_kernel<TIn, D><<<dim3(p.T / 32, p.B * p.H), 128, 0, st>>>(
       static_cast<const TIn*>(p.q), static_cast<const TIn*>(p.k), static_cast<const TIn*>(p.v),
-      static_cast<TIn*>(p.out_sca), p.lse, p.T, (int)p.c, p.koff);
+      static_cast<TIn*>(p.out_sca), p.lse, static_cast<TIn*>(p.out_sca_lo), p.T, (int)p.c, p.koff);
   return cudaGetLastError();
 }
 

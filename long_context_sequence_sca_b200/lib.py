@@ -26,12 +26,15 @@ EXPORTS = (
     "gecko_device_status",
     "gecko_timing_enable",
     "gecko_timing_read",
+    "gecko_timing_read_backward",
     "gecko_last_error",
     "gecko_release",
 )
 
 # Stages timed by gecko_timing_read, in order.
 STAGES = ("awm_stats", "awm_chunk", "awm_carry", "awm_readout", "sca")
+# Stages timed by gecko_timing_read_backward, in order.
+BWD_STAGES = ("awm_rebuild", "awm_backward", "sca_delta", "sca_dkdv", "sca_dq")
 
 GECKO_F32, GECKO_BF16 = 0, 1
 STATUS = {
@@ -65,9 +68,9 @@ def load() -> ctypes.CDLL:
     lib.gecko_sca_awm_forward_continue.restype = ctypes.c_int
     lib.gecko_sca_awm_forward_noalloc.argtypes = [vp] * 7 + [i64] * 5 + [ctypes.c_int, vp]
     lib.gecko_sca_awm_forward_noalloc.restype = ctypes.c_int
-    lib.gecko_sca_awm_forward_train.argtypes = [vp] * 8 + [i64] * 5 + [ctypes.c_int, vp]
+    lib.gecko_sca_awm_forward_train.argtypes = [vp] * 9 + [i64] * 5 + [ctypes.c_int, vp]
     lib.gecko_sca_awm_forward_train.restype = ctypes.c_int
-    lib.gecko_sca_awm_backward.argtypes = [vp] * 14 + [i64] * 5 + [ctypes.c_int, vp]
+    lib.gecko_sca_awm_backward.argtypes = [vp] * 15 + [i64] * 5 + [ctypes.c_int, vp]
     lib.gecko_sca_awm_backward.restype = ctypes.c_int
     lib.gecko_awm_state.argtypes = [vp, vp, i64, i64, i64, vp]
     lib.gecko_awm_state.restype = ctypes.c_int
@@ -82,6 +85,8 @@ def load() -> ctypes.CDLL:
     lib.gecko_timing_enable.restype = ctypes.c_int
     lib.gecko_timing_read.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
     lib.gecko_timing_read.restype = ctypes.c_int
+    lib.gecko_timing_read_backward.argtypes = lib.gecko_timing_read.argtypes
+    lib.gecko_timing_read_backward.restype = ctypes.c_int
     lib.gecko_last_error.argtypes = []
     lib.gecko_last_error.restype = ctypes.c_char_p
     lib.gecko_release.argtypes = []
@@ -121,16 +126,19 @@ def gecko_sca_awm_forward_noalloc(q, k, v, qm, km, out_sca, out_mem, B, H, T, c,
     return load().gecko_sca_awm_forward_noalloc(q, k, v, qm, km, out_sca, out_mem, B, H, T, c, d, dtype, stream)
 
 
-def gecko_sca_awm_forward_train(q, k, v, qm, km, out_sca, out_mem, lse, B, H, T, c, d, dtype, stream) -> int:
-    """The forward that also writes SCA's row log-sum-exp (for the backward)."""
-    return load().gecko_sca_awm_forward_train(q, k, v, qm, km, out_sca, out_mem, lse, B, H, T, c, d, dtype, stream)
+def gecko_sca_awm_forward_train(q, k, v, qm, km, out_sca, out_mem, lse, out_sca_lo, B, H, T, c, d, dtype,
+                                stream) -> int:
+    """The forward that also writes SCA's row log-sum-exp and (if out_sca_lo
+    is not 0) the rounding residual of out_sca, for the backward."""
+    return load().gecko_sca_awm_forward_train(q, k, v, qm, km, out_sca, out_mem, lse, out_sca_lo, B, H, T, c, d,
+                                              dtype, stream)
 
 
-def gecko_sca_awm_backward(q, k, v, qm, km, out_sca, lse, dout_sca, dout_mem, dq, dk, dv, dqm, dkm,
+def gecko_sca_awm_backward(q, k, v, qm, km, out_sca, out_sca_lo, lse, dout_sca, dout_mem, dq, dk, dv, dqm, dkm,
                            B, H, T, c, d, dtype, stream) -> int:
     """Gradients of q, k, v, qm, km with integer pointers; returns the status."""
-    return load().gecko_sca_awm_backward(q, k, v, qm, km, out_sca, lse, dout_sca, dout_mem, dq, dk, dv, dqm, dkm,
-                                         B, H, T, c, d, dtype, stream)
+    return load().gecko_sca_awm_backward(q, k, v, qm, km, out_sca, out_sca_lo, lse, dout_sca, dout_mem, dq, dk, dv,
+                                         dqm, dkm, B, H, T, c, d, dtype, stream)
 
 
 def gecko_awm_state(M_out, logz_out, B, H, d, stream) -> int:
@@ -159,6 +167,10 @@ def gecko_timing_enable(enable: int) -> int:
 
 def gecko_timing_read(ms_per_stage, capacity: int, n_calls) -> int:
     return load().gecko_timing_read(ms_per_stage, capacity, n_calls)
+
+
+def gecko_timing_read_backward(ms_per_stage, capacity: int, n_calls) -> int:
+    return load().gecko_timing_read_backward(ms_per_stage, capacity, n_calls)
 
 
 def gecko_last_error() -> str:
@@ -212,35 +224,42 @@ def _check_inputs(xs):
         raise ValueError("inputs must be [B, H, T, d] float32 or bfloat16")
 
 
-def sca_awm_forward_train(q, k, v, qm, km, c: int, stream=None):
-    """Forward for training: returns (out_sca, out_mem, lse) with lse the
-    [B, H, T] fp32 row log-sum-exp of SCA that sca_awm_backward needs."""
+def sca_awm_forward_train(q, k, v, qm, km, c: int, stream=None, keep_residual: bool = True):
+    """Forward for training: returns (out_sca, out_mem, lse, out_sca_lo) with
+    lse the [B, H, T] fp32 row log-sum-exp of SCA and out_sca_lo the rounding
+    residual of out_sca (None if keep_residual is False), both for
+    sca_awm_backward."""
     xs = (q, k, v, qm, km)
     _check_inputs(xs)
     B, H, T, d = q.shape
     out_sca, out_mem = torch.empty_like(q), torch.empty_like(q)
     lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
+    lo = torch.empty_like(q) if keep_residual else None
     with torch.cuda.device(q.device):
         rc = gecko_sca_awm_forward_train(*(x.data_ptr() for x in xs), out_sca.data_ptr(), out_mem.data_ptr(),
-                                         lse.data_ptr(), B, H, T, c, d, _DT[q.dtype], _stream_handle(stream))
+                                         lse.data_ptr(), lo.data_ptr() if lo is not None else 0, B, H, T, c, d,
+                                         _DT[q.dtype], _stream_handle(stream))
     _check(rc)
-    return out_sca, out_mem, lse
+    return out_sca, out_mem, lse, lo
 
 
-def sca_awm_backward(q, k, v, qm, km, out_sca, lse, dout_sca, dout_mem, c: int, stream=None):
+def sca_awm_backward(q, k, v, qm, km, out_sca, lse, dout_sca, dout_mem, c: int, out_sca_lo=None, stream=None):
     """Gradients (dq, dk, dv, dqm, dkm) of the fused forward for the output
-    gradients dout_sca, dout_mem; out_sca and lse come from
+    gradients dout_sca, dout_mem; out_sca, lse and out_sca_lo come from
     sca_awm_forward_train on the same inputs."""
     xs = (q, k, v, qm, km, out_sca, dout_sca.contiguous(), dout_mem.contiguous())
     _check_inputs(xs)
+    if out_sca_lo is not None:
+        _check_inputs((q, out_sca_lo))
     if not (lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous() and lse.shape == q.shape[:3]):
         raise ValueError("lse must be a contiguous [B, H, T] float32 CUDA tensor")
     B, H, T, d = q.shape
     grads = [torch.empty_like(q) for _ in range(5)]
     with torch.cuda.device(q.device):
-        rc = gecko_sca_awm_backward(*(x.data_ptr() for x in xs[:6]), lse.data_ptr(), xs[6].data_ptr(),
-                                    xs[7].data_ptr(), *(g.data_ptr() for g in grads), B, H, T, c, d,
-                                    _DT[q.dtype], _stream_handle(stream))
+        rc = gecko_sca_awm_backward(*(x.data_ptr() for x in xs[:6]), out_sca_lo.data_ptr() if out_sca_lo is not None
+                                    else 0, lse.data_ptr(), xs[6].data_ptr(), xs[7].data_ptr(),
+                                    *(g.data_ptr() for g in grads), B, H, T, c, d, _DT[q.dtype],
+                                    _stream_handle(stream))
     _check(rc)
     return tuple(grads)
 
@@ -251,15 +270,15 @@ class ScaAwmFunction(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, q, k, v, qm, km, c):
-        out_sca, out_mem, lse = sca_awm_forward_train(q, k, v, qm, km, c)
-        ctx.save_for_backward(q, k, v, qm, km, out_sca, lse)
+        out_sca, out_mem, lse, lo = sca_awm_forward_train(q, k, v, qm, km, c)
+        ctx.save_for_backward(q, k, v, qm, km, out_sca, lse, lo)
         ctx.c = c
         return out_sca, out_mem
 
     @staticmethod
     def backward(ctx, dout_sca, dout_mem):
-        q, k, v, qm, km, out_sca, lse = ctx.saved_tensors
-        grads = sca_awm_backward(q, k, v, qm, km, out_sca, lse, dout_sca, dout_mem, ctx.c)
+        q, k, v, qm, km, out_sca, lse, lo = ctx.saved_tensors
+        grads = sca_awm_backward(q, k, v, qm, km, out_sca, lse, dout_sca, dout_mem, ctx.c, out_sca_lo=lo)
         return (*grads, None)
 
 
@@ -319,6 +338,14 @@ def timing_read():
     n = ctypes.c_int(0)
     _check(gecko_timing_read(buf, len(STAGES), ctypes.byref(n)))
     return {name: float(buf[i]) for i, name in enumerate(STAGES)}, int(n.value)
+
+
+def timing_read_backward():
+    """({stage: total ms}, n_calls) of the backwards timed since the last read."""
+    buf = (ctypes.c_float * len(BWD_STAGES))()
+    n = ctypes.c_int(0)
+    _check(gecko_timing_read_backward(buf, len(BWD_STAGES), ctypes.byref(n)))
+    return {name: float(buf[i]) for i, name in enumerate(BWD_STAGES)}, int(n.value)
 
 
 def cema_forward(x, alpha, delta, theta, beta, eta, reset=None, state_in=None, return_state=False, y=None,

@@ -44,7 +44,8 @@ import numpy as np
 
 from . import gecko_oracle as F
 
-__all__ = ["sca_lse", "sca_head_backward", "awm_head_backward", "backward"]
+__all__ = ["sca_lse", "sca_head_backward", "sca_query_rows_backward", "sca_key_rows_backward",
+           "awm_head_backward", "backward"]
 
 
 def _softmax_backward(y: np.ndarray, dy: np.ndarray) -> np.ndarray:
@@ -85,6 +86,45 @@ def sca_head_backward(q, k, v, c: int, dout):
         dk[lo:b] += dS.T @ q[a:b]
         dv[lo:b] += P.T @ dout[a:b]
     return dq, dk, dv
+
+
+def _row_softmax(q_t, k_w):
+    sc = F.SCA_SCALE * (k_w @ q_t)
+    p = np.exp(sc - sc.max())
+    return p / p.sum()
+
+
+def sca_query_rows_backward(q, k, v, dout, c: int, rows):
+    """dq of selected query rows, each from its own window (the same
+    definition row by row; used for sampled checks of full-size runs)."""
+    out = np.empty((len(rows), q.shape[1]))
+    for n, t in enumerate(rows):
+        t = int(t)
+        lo = F.window_lo(t, c)
+        p = _row_softmax(q[t], k[lo:t + 1])
+        o = p @ v[lo:t + 1]
+        ds = p * (v[lo:t + 1] @ dout[t] - dout[t] @ o) * F.SCA_SCALE
+        out[n] = ds @ k[lo:t + 1]
+    return out
+
+
+def sca_key_rows_backward(q, k, v, dout, c: int, keys):
+    """(dk, dv) of selected key rows: every query that sees the key (from
+    the key itself to the end of the next chunk), each with the softmax of
+    its own window."""
+    T = q.shape[0]
+    dk = np.zeros((len(keys), k.shape[1]))
+    dv = np.zeros((len(keys), v.shape[1]))
+    for n, u in enumerate(keys):
+        u = int(u)
+        for t in range(u, min(T, (u // c + 2) * c)):
+            lo = F.window_lo(t, c)
+            p = _row_softmax(q[t], k[lo:t + 1])
+            o = p @ v[lo:t + 1]
+            pu = p[u - lo]
+            dv[n] += pu * dout[t]
+            dk[n] += pu * (dout[t] @ v[u] - dout[t] @ o) * F.SCA_SCALE * q[t]
+    return dk, dv
 
 
 def awm_head_backward(qm, km, v, c: int, dout_mem, dM_final=None, dlogz_final=None):

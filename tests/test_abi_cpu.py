@@ -117,14 +117,15 @@ def test_tdnorm_host_validation_rejects(so, kw, code):
 
 
 def _bwd(ptrs=None, B=1, H=1, T=256, c=128, d=64, dtype=1):
-    ptrs = ptrs or [FAKE] * 14
+    ptrs = ptrs or [FAKE] * 15
     return L.gecko_sca_awm_backward(*ptrs, B, H, T, c, d, dtype, None)
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(ptrs=[FAKE] * 6 + [0] + [FAKE] * 7), 1),     # lse NULL
-    (dict(ptrs=[FAKE] * 13 + [0]), 1),                 # dkm NULL
-    (dict(ptrs=[FAKE] * 9 + [FAKE + 4] + [FAKE] * 4), 3),
+    (dict(ptrs=[FAKE] * 7 + [0] + [FAKE] * 7), 1),     # lse NULL
+    (dict(ptrs=[FAKE] * 14 + [0]), 1),                 # dkm NULL
+    (dict(ptrs=[FAKE] * 10 + [FAKE + 4] + [FAKE] * 4), 3),
+    (dict(ptrs=[FAKE] * 6 + [FAKE + 8] + [FAKE] * 8), 3),   # residual misaligned
     (dict(d=32), 2),
     (dict(T=300), 2),
     (dict(dtype=2), 1),
@@ -135,5 +136,6 @@ def test_backward_host_validation_rejects(so, kw, code):
 
 
 def test_train_forward_rejects_bad_lse(so):
-    assert L.gecko_sca_awm_forward_train(*[FAKE] * 7, 0, 1, 1, 256, 128, 64, 1, None) == 1
-    assert L.gecko_sca_awm_forward_train(*[FAKE] * 7, FAKE + 4, 1, 1, 256, 128, 64, 1, None) == 3
+    assert L.gecko_sca_awm_forward_train(*[FAKE] * 7, 0, 0, 1, 1, 256, 128, 64, 1, None) == 1
+    assert L.gecko_sca_awm_forward_train(*[FAKE] * 7, FAKE + 4, 0, 1, 1, 256, 128, 64, 1, None) == 3
+    assert L.gecko_sca_awm_forward_train(*[FAKE] * 7, FAKE, FAKE + 8, 1, 1, 256, 128, 64, 1, None) == 3

@@ -6,10 +6,13 @@ Tolerances: the gradients are sums of many terms of either sign, so the
 absolute bars of the forward are scaled by the size of the reference
 gradient: fp32 max-abs <= 1e-4 * max(1, max|ref|); bf16 max-abs <=
 2e-2 * max(1, max|ref|) and rel-L2 <= 1e-2.  The bf16 rel-L2 bar is twice
-the forward's because the backward takes the forward's bf16 output O: the
-row term delta = rowsum(dO * O) then carries O's rounding, which alone moves
-the oracle's own dq by ~6e-3 rel-L2 (pinned on the CPU in
-test_backward_tolerance_cpu.py).  The SCA row log-sum-exp is compared
+the forward's: P and dS enter the MMAs as bf16, and the dq of a row is a
+strongly cancelling sum (its dS terms sum to zero).  The backward takes the
+forward's output together with its rounding residual; with the bf16 output
+alone, the row term delta = rowsum(dO * O) would carry O's rounding, which
+by itself moves the oracle's own dq by several 1e-3 (pinned on the CPU in
+test_backward_tolerance_cpu.py) and by several 1e-2 at 8K-key windows;
+test_backward_without_residual keeps that path covered.  The SCA row log-sum-exp is compared
 against the oracle's as a forward quantity (fp32 1e-4, bf16 2e-2)."""
 import numpy as np
 import pytest
@@ -56,8 +59,8 @@ def _check_backward(L, w: Workload, seed=1234, env=None, monkeypatch=None):
             monkeypatch.setenv(k, v)
     x = make_inputs(w, device="cuda")
     dos, dom = _douts(x["q"], seed)
-    out_sca, out_mem, lse = L.sca_awm_forward_train(*(x[n] for n in NAMES), w.c)
-    grads = L.sca_awm_backward(*(x[n] for n in NAMES), out_sca, lse, dos, dom, w.c)
+    out_sca, out_mem, lse, lo = L.sca_awm_forward_train(*(x[n] for n in NAMES), w.c)
+    grads = L.sca_awm_backward(*(x[n] for n in NAMES), out_sca, lse, dos, dom, w.c, out_sca_lo=lo)
     torch.cuda.synchronize()
     assert L.device_status() == 0
     xs = [x[n].double().cpu().numpy() for n in NAMES]
@@ -98,6 +101,10 @@ def test_train_forward_outputs_equal_plain_forward(L):
     b = L.sca_awm_forward_train(*(x[n] for n in NAMES), w.c)
     torch.cuda.synchronize()
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+    # the residual is what the rounding to bf16 dropped: |lo| <= half an ulp of out
+    lo, hi = b[3].float(), b[0].float()
+    assert torch.all(lo.abs() <= hi.abs() * 2.0 ** -8 + 1e-30)
+    assert lo.abs().max() > 0
 
 
 def test_autograd_function_uses_the_same_kernels(L):
@@ -107,8 +114,23 @@ def test_autograd_function_uses_the_same_kernels(L):
     o_sca, o_mem = L.ScaAwmFunction.apply(*ins, w.c)
     dos, dom = _douts(x["q"], 7)
     torch.autograd.backward((o_sca, o_mem), (dos, dom))
-    out_sca, _, lse = L.sca_awm_forward_train(*(x[n] for n in NAMES), w.c)
-    want = L.sca_awm_backward(*(x[n] for n in NAMES), out_sca, lse, dos, dom, w.c)
+    out_sca, _, lse, lo = L.sca_awm_forward_train(*(x[n] for n in NAMES), w.c)
+    want = L.sca_awm_backward(*(x[n] for n in NAMES), out_sca, lse, dos, dom, w.c, out_sca_lo=lo)
     torch.cuda.synchronize()
     for t, g in zip(ins, want):
         assert torch.equal(t.grad, g)
+
+
+def test_backward_without_residual(L):
+    """out_sca_lo = NULL: delta from the bf16 output alone (still within the
+    bar at this window size, see the note at the top)."""
+    w = WORKLOADS["bf16_many_chunks"]
+    x = make_inputs(w, device="cuda")
+    dos, dom = _douts(x["q"], 99)
+    out_sca, _, lse, _ = L.sca_awm_forward_train(*(x[n] for n in NAMES), w.c, keep_residual=False)
+    grads = L.sca_awm_backward(*(x[n] for n in NAMES), out_sca, lse, dos, dom, w.c)
+    torch.cuda.synchronize()
+    xs = [x[n].double().cpu().numpy() for n in NAMES]
+    ref = GB.backward(*xs, w.c, dos.double().cpu().numpy(), dom.double().cpu().numpy())
+    for n, g, r in zip(NAMES, grads, ref):
+        _close(g, r, w.dtype, "d" + n)

@@ -140,3 +140,15 @@ def test_planted_mistakes_fail_finite_differences(mistake, monkeypatch):
         monkeypatch.setattr(GB, "_softmax_backward", lambda y, dy: y * dy)
     got = _grads(x["q"], x["k"], x["v"], x["qm"], x["km"], c, W)
     assert any(not np.allclose(got[n], want[n], rtol=1e-6, atol=1e-8) for n in x)
+
+
+def test_row_by_row_sca_gradients_agree_with_whole_head():
+    T, c, d = 40, 8, 4
+    q, k, v, _, _ = _inputs(T, d)
+    do = RNG.normal(size=(T, d))
+    dq, dk, dv = GB.sca_head_backward(q, k, v, c, do)
+    rows = [0, 7, 8, 15, 16, 23, 39]
+    np.testing.assert_allclose(GB.sca_query_rows_backward(q, k, v, do, c, rows), dq[rows], rtol=1e-10, atol=1e-12)
+    kr, vr = GB.sca_key_rows_backward(q, k, v, do, c, rows)
+    np.testing.assert_allclose(kr, dk[rows], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(vr, dv[rows], rtol=1e-10, atol=1e-12)
