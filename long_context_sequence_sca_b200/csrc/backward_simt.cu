@@ -602,7 +602,8 @@ cudaError_t sca_bwd_simt_impl(const BwdProblem& b, const BwdWorkspace& w, cudaSt
 }
 
 template <typename TIn, int D>
-cudaError_t awm_bwd_impl(const BwdProblem& b, const Workspace& fw, const BwdWorkspace& w, cudaStream_t st) {
+cudaError_t awm_bwd_impl(const BwdProblem& b, const Workspace& fw, const BwdWorkspace& w, cudaStream_t st,
+                         bool tc) {
   const Problem& p = b.f;
   const int64_t BH = p.B * p.H;
   const int S = p.S;
@@ -616,13 +617,18 @@ cudaError_t awm_bwd_impl(const BwdProblem& b, const Workspace& fw, const BwdWork
   awm_bwd_carry_kernel<D, JC><<<dim3(D / JC, (unsigned)BH), 256, smc, st>>>(w.E, fw.Cm, fw.ratio, fw.rho, w.G, S);
   const int64_t nw = BH * D;
   awm_bwd_dl_kernel<D><<<(unsigned)((nw + 7) / 8), 256, 0, st>>>(w.G, fw.Mst, fw.ratio, fw.rho, w.dl, S, nw);
-  const size_t smk = sizeof(float) * (2 * D * (D + 1) + 8 * 4 * D);
-  e = cudaFuncSetAttribute(awm_bwd_chunk_simt_kernel<TIn, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smk);
-  if (e != cudaSuccess) return e;
   const dim3 grid((unsigned)(p.c / 32), (unsigned)S, (unsigned)BH);
-  awm_bwd_chunk_simt_kernel<TIn, D><<<grid, 256, smk, st>>>(
-      static_cast<const TIn*>(p.km), static_cast<const TIn*>(p.v), w.G, fw.Mst, fw.lse, fw.logz, w.dl,
-      static_cast<TIn*>(b.dkm), w.dv_awm, p.T, (int)p.c);
+  if (tc) {
+    if ((e = launch_awm_bwd_chunk_tc(b, fw, w, st)) != cudaSuccess) return e;
+  } else {
+    const size_t smk = sizeof(float) * (2 * D * (D + 1) + 8 * 4 * D);
+    e = cudaFuncSetAttribute(awm_bwd_chunk_simt_kernel<TIn, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smk);
+    if (e != cudaSuccess) return e;
+    awm_bwd_chunk_simt_kernel<TIn, D><<<grid, 256, smk, st>>>(
+        static_cast<const TIn*>(p.km), static_cast<const TIn*>(p.v), w.G, fw.Mst, fw.lse, fw.logz, w.dl,
+        static_cast<TIn*>(b.dkm), w.dv_awm, p.T, (int)p.c);
+  }
   const size_t smr = sizeof(float) * (D * (D + 1) + 8 * 4 * D);
   e = cudaFuncSetAttribute(awm_bwd_readout_simt_kernel<TIn, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smr);
@@ -638,8 +644,8 @@ cudaError_t awm_bwd_impl(const BwdProblem& b, const Workspace& fw, const BwdWork
 size_t bwd_workspace_bytes(int64_t BH, int64_t T, int64_t c, int64_t d) {
   auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
   const int64_t S = T / c;
-  return 2 * al(sizeof(float) * BH * T) + al(sizeof(float) * BH * S * d * d) + al(sizeof(float) * BH * (S + 1) * d * d) +
-         al(sizeof(float) * BH * S * d) + al(sizeof(float) * BH * T * d);
+  return 2 * al(sizeof(float) * BH * T) + 2 * al(sizeof(float) * BH * S * d * d) +
+         al(sizeof(float) * BH * (S + 1) * d * d) + al(sizeof(float) * BH * S * d) + al(sizeof(float) * BH * T * d);
 }
 
 BwdWorkspace carve_bwd_workspace(void* base, int64_t BH, int64_t T, int64_t c, int64_t d) {
@@ -658,6 +664,8 @@ BwdWorkspace carve_bwd_workspace(void* base, int64_t BH, int64_t T, int64_t c, i
   w.dl = reinterpret_cast<float*>(p);
   p += al(sizeof(float) * BH * S * d);
   w.dv_awm = reinterpret_cast<float*>(p);
+  p += al(sizeof(float) * BH * T * d);
+  w.W = reinterpret_cast<float*>(p);
   return w;
 }
 
@@ -671,8 +679,9 @@ cudaError_t launch_sca_bwd_delta(const BwdProblem& b, const BwdWorkspace& w, cud
 cudaError_t launch_sca_bwd_simt(const BwdProblem& b, const BwdWorkspace& w, cudaStream_t st, int part) {
   return GECKO_BWD_DISPATCH(sca_bwd_simt_impl, b, w, st, part);
 }
-cudaError_t launch_awm_bwd(const BwdProblem& b, const Workspace& fw, const BwdWorkspace& w, cudaStream_t st) {
-  return GECKO_BWD_DISPATCH(awm_bwd_impl, b, fw, w, st);
+cudaError_t launch_awm_bwd(const BwdProblem& b, const Workspace& fw, const BwdWorkspace& w, cudaStream_t st,
+                           bool tc) {
+  return GECKO_BWD_DISPATCH(awm_bwd_impl, b, fw, w, st, tc && b.f.dtype == kBF16);
 }
 #undef GECKO_BWD_DISPATCH
 

@@ -374,7 +374,7 @@ int run_backward(const void* q, const void* k, const void* v, const void* qm, co
   if ((rc = check_cuda(launch_awm_chunk_simt(p, w, st), "awm chunk"))) return rc;
   if ((rc = check_cuda(launch_awm_carry(p, w, st), "awm carry"))) return rc;
   ev.mark(1);
-  if ((rc = check_cuda(launch_awm_bwd(b, w, bw, st), "awm backward"))) return rc;
+  if ((rc = check_cuda(launch_awm_bwd(b, w, bw, st, use_tc), "awm backward"))) return rc;
   ev.mark(2);
   if ((rc = check_cuda(launch_sca_bwd_delta(b, bw, st), "sca backward delta"))) return rc;
   ev.mark(3);

@@ -81,6 +81,7 @@ struct BwdWorkspace {
   float* G;       // [BH, S+1, d, d]  G_s = dLoss/dM'_s, s = 1..S+1
   float* dl;      // [BH, S, d]  dLoss/d log e_s
   float* dv_awm;  // [BH, T, d]  AWM part of dV
+  float* W;       // [BH, S, d, d]  W_s = M'_s G_{s+1}^T
 };
 
 size_t bwd_workspace_bytes(int64_t BH, int64_t T, int64_t c, int64_t d);
@@ -89,7 +90,11 @@ cudaError_t launch_sca_bwd_delta(const BwdProblem& b, const BwdWorkspace& w, cud
 // part 0: dK and dV (adding the AWM part of dV); part 1: dQ
 cudaError_t launch_sca_bwd_simt(const BwdProblem& b, const BwdWorkspace& w, cudaStream_t st, int part);
 cudaError_t launch_sca_bwd_tc(const BwdProblem& b, const BwdWorkspace& w, cudaStream_t st, int part);  // bf16, tc_supported
-cudaError_t launch_awm_bwd(const BwdProblem& b, const Workspace& fw, const BwdWorkspace& w, cudaStream_t st);
+// tc: the per-chunk K_m / V gradients on the tensor cores (bf16, tc_supported)
+cudaError_t launch_awm_bwd(const BwdProblem& b, const Workspace& fw, const BwdWorkspace& w, cudaStream_t st,
+                           bool tc);
+cudaError_t launch_awm_bwd_chunk_tc(const BwdProblem& b, const Workspace& fw, const BwdWorkspace& w,
+                                    cudaStream_t st);
 
 // ---------------------------------------------------------------- CEMA --
 
