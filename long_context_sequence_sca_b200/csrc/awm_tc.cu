@@ -40,11 +40,24 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int col, int rows) {
 
 constexpr int kKT = 64;  // tokens per tile
 
-template <int D>
+// What a chunk-kernel launch computes.
+//   kChunkFwd    Bm = Phi~^T V, Cm = Phi~^T Psi with bf16 operands (f16
+//                exponentials): stage [V | Psi | Phi].
+//   kChunkSplit  the same products with each computed operand carried as two
+//                bf16 parts (hi + lo, fp32 exponentials), for a backward whose
+//                softmax gradients keep only the small differences between
+//                the rows of M': stage [V | Psi_hi | Psi_lo | Phi_hi | Phi_lo];
+//                D += Phi_hi^T [V | Psi_hi] + Phi_lo^T [V | Psi_hi], Cm += Phi_hi^T Psi_lo.
+//   kChunkE      E = psi(Q_m)^T dO_m for the backward (Q_m arrives in the
+//                K_m slot, dO_m in the V slot): stage [dO | psi_hi | psi_lo].
+enum ChunkMode { kChunkFwd = 0, kChunkSplit = 1, kChunkE = 2 };
+
+template <int D, int Mode = kChunkFwd>
 struct ChunkCfg {
   static constexpr int kBox = kKT * 128;                 // one [64 x 64] bf16 box
   static constexpr int kOperand = (D / 64) * kBox;       // a [64 x D] operand
-  static constexpr int kStage = 3 * kOperand;            // [V | Psi | Phi]
+  static constexpr int kSlots = Mode == kChunkSplit ? 5 : 3;
+  static constexpr int kStage = kSlots * kOperand;
   static constexpr int kStages = 2;
   static constexpr int kBarOff = kStages * kStage;
   // v_full[2], op_full[2], stage_empty[2], acc_full
@@ -53,17 +66,17 @@ struct ChunkCfg {
   static constexpr int kMiscOff = kLzOff + D * 4;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;
-  static constexpr uint32_t kTmemCols = D == 128 ? 256 : 128;
+  static constexpr uint32_t kTmemCols = Mode == kChunkE ? D : (D == 128 ? 256 : 128);
 };
 
 // 128 compute threads (warps 0-3), warp 4 = TMA producer, warp 5 = MMA issuer.
-template <int D>
+template <int D, int Mode = kChunkFwd>
 __global__ void __launch_bounds__(192, 2) awm_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_v,
                                                            const __grid_constant__ CUtensorMap map_km,
                                                            const float* __restrict__ lse, float* __restrict__ Bm,
                                                            float* __restrict__ Cm, int T, int c, int koff,
                                                            int* status) {
-  using Cfg = ChunkCfg<D>;
+  using Cfg = ChunkCfg<D, Mode>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
@@ -77,6 +90,8 @@ __global__ void __launch_bounds__(192, 2) awm_chunk_tc_kernel(const __grid_const
 
   const int s = blockIdx.x, S = gridDim.x;
   const int64_t bh = blockIdx.y;
+  // the readouts of chunks 1 and 2 read a zero state: their E is never used
+  if (Mode == kChunkE && s < 2) return;
   const int warp = warp_id_uniform(), lane = threadIdx.x % 32;
   const int n_tiles = c / kKT;
   const int64_t row0 = bh * (int64_t)T + (int64_t)s * c;
@@ -93,7 +108,8 @@ __global__ void __launch_bounds__(192, 2) awm_chunk_tc_kernel(const __grid_const
     *abort_flag = 0;
     fence_mbar_init();
   }
-  for (int f = threadIdx.x; f < D; f += blockDim.x) lz2[f] = lse[(bh * S + s) * D + f] * kLog2e;
+  if (Mode != kChunkE)
+    for (int f = threadIdx.x; f < D; f += blockDim.x) lz2[f] = lse[(bh * S + s) * D + f] * kLog2e;
   if (warp == 5) {
     tmem_alloc(tmem_slot, Cfg::kTmemCols);
     tmem_relinquish();
@@ -130,6 +146,7 @@ __global__ void __launch_bounds__(192, 2) awm_chunk_tc_kernel(const __grid_const
     // --------------------------------------------------------- MMA issuer --
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(D, 2 * D, true, true);
+      constexpr uint32_t idesc1 = idesc_bf16_f32(D, D, true, true);
       const uint32_t base = smem_u32(smem);
       bool ok = true;
       for (int kt = 0; kt < n_tiles && ok; ++kt) {
@@ -139,12 +156,21 @@ __global__ void __launch_bounds__(192, 2) awm_chunk_tc_kernel(const __grid_const
         if (!(ok = mbar_wait(op_full + st, ph, abort_flag, status))) break;
         tc_fence_after();
         const uint32_t sb = base + st * Cfg::kStage;
+        auto desc = [&](int slot, int kk) { return sdesc_sw128(sb + slot * Cfg::kOperand + kk * 2048, Cfg::kBox, 1024); };
 #pragma unroll
         for (int kk = 0; kk < kKT / 16; ++kk) {
-          // A = Phi^T (M = D features, MN-major), B = [V | Psi] (N = 2D, MN-major)
-          const uint64_t adesc = sdesc_sw128(sb + 2 * Cfg::kOperand + kk * 2048, Cfg::kBox, 1024);
-          const uint64_t bdesc = sdesc_sw128(sb + kk * 2048, Cfg::kBox, 1024);
-          umma_ss(tmem, adesc, bdesc, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+          const uint32_t acc = (kt > 0 || kk > 0) ? 1u : 0u;
+          if (Mode == kChunkFwd) {
+            // A = Phi^T (M = D features, MN-major), B = [V | Psi] (N = 2D, MN-major)
+            umma_ss(tmem, desc(2, kk), desc(0, kk), idesc, acc);
+          } else if (Mode == kChunkSplit) {
+            umma_ss(tmem, desc(3, kk), desc(0, kk), idesc, acc);        // Phi_hi^T [V | Psi_hi]
+            umma_ss(tmem, desc(4, kk), desc(0, kk), idesc, 1u);         // Phi_lo^T [V | Psi_hi]
+            umma_ss(tmem + D, desc(3, kk), desc(2, kk), idesc1, 1u);    // Phi_hi^T Psi_lo
+          } else {
+            umma_ss(tmem, desc(1, kk), desc(0, kk), idesc1, acc);       // psi_hi^T dO
+            umma_ss(tmem, desc(2, kk), desc(0, kk), idesc1, 1u);        // psi_lo^T dO
+          }
         }
         umma_commit(st_empty + st);
       }
@@ -183,32 +209,70 @@ __global__ void __launch_bounds__(192, 2) awm_chunk_tc_kernel(const __grid_const
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
       const float mx2 = mx * kLog2e;
       float e[HF], sum = 0.f;
+      if (Mode == kChunkFwd) {
 #pragma unroll
-      for (int i = 0; i < HF / 8; ++i) {
-        const int col = h * HF + 8 * i;
-        uint4 pf;
-        uint32_t* qq = reinterpret_cast<uint32_t*>(&pf);
+        for (int i = 0; i < HF / 8; ++i) {
+          const int col = h * HF + 8 * i;
+          uint4 pf;
+          uint32_t* qq = reinterpret_cast<uint32_t*>(&pf);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int a = 8 * i + 2 * j;
-          float p0, p1;
-          ex2_h2(fmaf(x[a], kLog2e, -lz2[col + 2 * j]), fmaf(x[a + 1], kLog2e, -lz2[col + 2 * j + 1]), p0, p1);
-          qq[j] = pack_bf16x2(p0, p1);
-          ex2_h2(fmaf(x[a], kLog2e, -mx2), fmaf(x[a + 1], kLog2e, -mx2), e[a], e[a + 1]);
-          sum += e[a] + e[a + 1];
+          for (int j = 0; j < 4; ++j) {
+            const int a = 8 * i + 2 * j;
+            float p0, p1;
+            ex2_h2(fmaf(x[a], kLog2e, -lz2[col + 2 * j]), fmaf(x[a + 1], kLog2e, -lz2[col + 2 * j + 1]), p0, p1);
+            qq[j] = pack_bf16x2(p0, p1);
+            ex2_h2(fmaf(x[a], kLog2e, -mx2), fmaf(x[a + 1], kLog2e, -mx2), e[a], e[a + 1]);
+            sum += e[a] + e[a + 1];
+          }
+          *reinterpret_cast<uint4*>(stg + 2 * Cfg::kOperand + sw128_off(r, col, kKT)) = pf;
         }
-        *reinterpret_cast<uint4*>(stg + 2 * Cfg::kOperand + sw128_off(r, col, kKT)) = pf;
+      } else {
+        // fp32 exponentials; Phi (split mode only) as bf16 hi and lo parts
+#pragma unroll
+        for (int i = 0; i < HF / 8; ++i) {
+          const int col = h * HF + 8 * i;
+          uint4 fh, fl;
+          uint32_t* fhp = reinterpret_cast<uint32_t*>(&fh);
+          uint32_t* flp = reinterpret_cast<uint32_t*>(&fl);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int a = 8 * i + 2 * j;
+            if (Mode == kChunkSplit) {
+              const float p0 = ex2(fmaf(x[a], kLog2e, -lz2[col + 2 * j]));
+              const float p1 = ex2(fmaf(x[a + 1], kLog2e, -lz2[col + 2 * j + 1]));
+              fhp[j] = pack_bf16x2(p0, p1);
+              const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&fhp[j]));
+              flp[j] = pack_bf16x2(p0 - hi.x, p1 - hi.y);
+            }
+            e[a] = ex2(fmaf(x[a], kLog2e, -mx2));
+            e[a + 1] = ex2(fmaf(x[a + 1], kLog2e, -mx2));
+            sum += e[a] + e[a + 1];
+          }
+          if (Mode == kChunkSplit) {
+            *reinterpret_cast<uint4*>(stg + 3 * Cfg::kOperand + sw128_off(r, col, kKT)) = fh;
+            *reinterpret_cast<uint4*>(stg + 4 * Cfg::kOperand + sw128_off(r, col, kKT)) = fl;
+          }
+        }
       }
       sum += __shfl_xor_sync(0xffffffffu, sum, 1);
       const float inv = 1.f / sum;
 #pragma unroll
       for (int i = 0; i < HF / 8; ++i) {
         const int col = h * HF + 8 * i;
-        uint4 ps;
+        uint4 ps, pl;
         uint32_t* pp = reinterpret_cast<uint32_t*>(&ps);
+        uint32_t* plp = reinterpret_cast<uint32_t*>(&pl);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) pp[j] = pack_bf16x2(e[8 * i + 2 * j] * inv, e[8 * i + 2 * j + 1] * inv);
+        for (int j = 0; j < 4; ++j) {
+          const float a0 = e[8 * i + 2 * j] * inv, a1 = e[8 * i + 2 * j + 1] * inv;
+          pp[j] = pack_bf16x2(a0, a1);
+          if (Mode != kChunkFwd) {
+            const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pp[j]));
+            plp[j] = pack_bf16x2(a0 - hi.x, a1 - hi.y);
+          }
+        }
         *reinterpret_cast<uint4*>(stg + Cfg::kOperand + sw128_off(r, col, kKT)) = ps;
+        if (Mode != kChunkFwd) *reinterpret_cast<uint4*>(stg + 2 * Cfg::kOperand + sw128_off(r, col, kKT)) = pl;
       }
       // generic-proxy writes must be visible to the tensor core (async proxy)
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -225,7 +289,7 @@ __global__ void __launch_bounds__(192, 2) awm_chunk_tc_kernel(const __grid_const
       const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
       const int64_t o = (bh * S + s) * (int64_t)D * D + (int64_t)f * D;
 #pragma unroll 1
-      for (int cb = 0; cb < 2 * D / 32; ++cb) {
+      for (int cb = 0; cb < (Mode == kChunkE ? D : 2 * D) / 32; ++cb) {
         uint32_t v[32];
         tmem_ld32(taddr + cb * 32, v);
         tmem_wait_ld();
@@ -470,9 +534,10 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-template <int D>
-cudaError_t chunk_impl(const Problem& p, const Workspace& w, cudaStream_t st) {
-  using Cfg = ChunkCfg<D>;
+template <int D, int Mode>
+cudaError_t chunk_impl(const Problem& p, const void* vsrc, const void* ksrc, const float* lse, float* out0,
+                       float* out1, cudaStream_t st) {
+  using Cfg = ChunkCfg<D, Mode>;
   EncodeTiledFn fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
   // V and K_m as [rows, D], boxes of [64 rows x 64] bf16, 128B swizzle (V
@@ -486,13 +551,14 @@ cudaError_t chunk_impl(const Problem& p, const Workspace& w, cudaStream_t st) {
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
   };
+  const int64_t koff = Mode == kChunkE ? 0 : p.koff;
   CUtensorMap mv, mkm;
-  if (!map(&mv, p.v, p.B * p.H * (p.T + p.koff)) || !map(&mkm, p.km, p.B * p.H * p.T)) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(awm_chunk_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (!map(&mv, vsrc, p.B * p.H * (p.T + koff)) || !map(&mkm, ksrc, p.B * p.H * p.T)) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(awm_chunk_tc_kernel<D, Mode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Cfg::kAlloc);
   if (e != cudaSuccess) return e;
-  awm_chunk_tc_kernel<D><<<dim3(p.S, p.B * p.H), 192, Cfg::kAlloc, st>>>(
-      mv, mkm, w.lse, w.Bm, w.Cm, (int)p.T, (int)p.c, (int)p.koff, p.status);
+  awm_chunk_tc_kernel<D, Mode><<<dim3(p.S, p.B * p.H), 192, Cfg::kAlloc, st>>>(
+      mv, mkm, lse, out0, out1, (int)p.T, (int)p.c, (int)koff, p.status);
   return cudaGetLastError();
 }
 
@@ -524,7 +590,18 @@ cudaError_t readout_impl(const Problem& p, const Workspace& w, cudaStream_t st) 
 }  // namespace
 
 cudaError_t launch_awm_chunk_tc(const Problem& p, const Workspace& w, cudaStream_t st) {
-  return p.d == 64 ? chunk_impl<64>(p, w, st) : chunk_impl<128>(p, w, st);
+  return p.d == 64 ? chunk_impl<64, kChunkFwd>(p, p.v, p.km, w.lse, w.Bm, w.Cm, st)
+                   : chunk_impl<128, kChunkFwd>(p, p.v, p.km, w.lse, w.Bm, w.Cm, st);
+}
+
+cudaError_t launch_awm_chunk_tc_split(const Problem& p, const Workspace& w, cudaStream_t st) {
+  return p.d == 64 ? chunk_impl<64, kChunkSplit>(p, p.v, p.km, w.lse, w.Bm, w.Cm, st)
+                   : chunk_impl<128, kChunkSplit>(p, p.v, p.km, w.lse, w.Bm, w.Cm, st);
+}
+
+cudaError_t launch_awm_bwd_e_tc(const Problem& p, const void* dout_mem, float* E, cudaStream_t st) {
+  return p.d == 64 ? chunk_impl<64, kChunkE>(p, dout_mem, p.qm, nullptr, E, nullptr, st)
+                   : chunk_impl<128, kChunkE>(p, dout_mem, p.qm, nullptr, E, nullptr, st);
 }
 
 cudaError_t launch_awm_readout_tc(const Problem& p, const Workspace& w, cudaStream_t st) {

@@ -607,8 +607,13 @@ cudaError_t awm_bwd_impl(const BwdProblem& b, const Workspace& fw, const BwdWork
   const Problem& p = b.f;
   const int64_t BH = p.B * p.H;
   const int S = p.S;
-  awm_bwd_e_simt_kernel<TIn, D><<<dim3(S, (unsigned)BH), 256, 0, st>>>(
-      static_cast<const TIn*>(p.qm), static_cast<const TIn*>(b.dout_mem), w.E, p.T, (int)p.c);
+  if (tc) {
+    cudaError_t e0 = launch_awm_bwd_e_tc(p, b.dout_mem, w.E, st);
+    if (e0 != cudaSuccess) return e0;
+  } else {
+    awm_bwd_e_simt_kernel<TIn, D><<<dim3(S, (unsigned)BH), 256, 0, st>>>(
+        static_cast<const TIn*>(p.qm), static_cast<const TIn*>(b.dout_mem), w.E, p.T, (int)p.c);
+  }
   constexpr int JC = 16;
   const size_t smc = sizeof(float) * (D * (D + 4) + D * JC);
   cudaError_t e = cudaFuncSetAttribute(awm_bwd_carry_kernel<D, JC>, cudaFuncAttributeMaxDynamicSharedMemorySize,

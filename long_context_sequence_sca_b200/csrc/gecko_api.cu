@@ -368,10 +368,13 @@ int run_backward(const void* q, const void* k, const void* v, const void* qm, co
   BwdStageEvents ev(st);
   ev.mark(0);
   if ((rc = check_cuda(launch_awm_stats(p, w, st), "awm stats"))) return rc;
-  // The chunk products are rebuilt in fp32: the rows of M' are close to one
-  // another (each is a running average of V), and the softmax gradient of
-  // the readout keeps only their differences, which bf16 operands blur.
-  if ((rc = check_cuda(launch_awm_chunk_simt(p, w, st), "awm chunk"))) return rc;
+  // The chunk products are rebuilt to near fp32 (fp32 on the CUDA cores, or
+  // bf16 hi + lo operands on the tensor cores): the rows of M' are close to
+  // one another (each is a running average of V), and the softmax gradients
+  // keep only their differences, which plain bf16 operands blur.
+  if ((rc = check_cuda(use_tc ? launch_awm_chunk_tc_split(p, w, st) : launch_awm_chunk_simt(p, w, st),
+                       "awm chunk")))
+    return rc;
   if ((rc = check_cuda(launch_awm_carry(p, w, st), "awm carry"))) return rc;
   ev.mark(1);
   if ((rc = check_cuda(launch_awm_bwd(b, w, bw, st, use_tc), "awm backward"))) return rc;

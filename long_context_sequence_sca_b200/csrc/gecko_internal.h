@@ -59,6 +59,10 @@ bool tc_supported(const Problem& p);
 cudaError_t launch_sca_tc(const Problem& p, cudaStream_t st);
 cudaError_t launch_awm_chunk_tc(const Problem& p, const Workspace& w, cudaStream_t st);
 cudaError_t launch_awm_readout_tc(const Problem& p, const Workspace& w, cudaStream_t st);
+// Bm, Cm with each computed operand as bf16 hi + lo (near-fp32 products for the backward)
+cudaError_t launch_awm_chunk_tc_split(const Problem& p, const Workspace& w, cudaStream_t st);
+// E_s = psi(Qm_s)^T dO_m,s for chunks 3..S, hi + lo operands
+cudaError_t launch_awm_bwd_e_tc(const Problem& p, const void* dout_mem, float* E, cudaStream_t st);
 
 // ------------------------------------------------------------ backward --
 
