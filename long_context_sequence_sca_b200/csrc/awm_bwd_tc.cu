@@ -357,6 +357,221 @@ __global__ void __launch_bounds__(160, 1) awm_bwd_chunk_tc_kernel(
   if (warp == 4) tmem_dealloc(tmem, Cfg::kTmemCols);
 }
 
+// ------------------------------------------------------ readout gradient --
+//
+// O_m,s = psi(Qm_s) M'_{s-1} (digest, method step details, step 5) gives
+//     dQm_i = psi_i * (g_i - <g_i, psi_i>),   g_i = dO_m,i M'_{s-1}^T,
+// zero for chunks 1 and 2 (they read M'_0 = M'_1 = 0).  g is one tensor-core
+// product per 128-row tile with M' in two bf16 parts (the centring keeps
+// only the differences between the rows of M').  grid (S, BH, G), 160
+// threads: warps 0-3 one row each, warp 4 TMEM, TMA and MMA issue.
+
+template <int D>
+struct ReadoutBwdCfg {
+  static constexpr int kTile = 128 * D * 2;
+  static constexpr int kMat = D * D * 2;
+  static constexpr int kDoOff = 0;
+  static constexpr int kQmOff = kTile;
+  static constexpr int kMhiOff = 2 * kTile;
+  static constexpr int kMloOff = kMhiOff + kMat;
+  static constexpr int kBarOff = kMloOff + kMat;
+  // ld_full, acc_full, tile_done, drain
+  static constexpr int kNumBars = 4;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kAlloc = kBytes + 1024;
+  static_assert(kAlloc <= 232448, "dynamic shared memory above the sm_100 per-block limit");
+  static constexpr uint32_t kTmemCols = D;
+};
+
+template <int D>
+__global__ void __launch_bounds__(160, 1) awm_bwd_readout_tc_kernel(
+    const __grid_constant__ CUtensorMap map_do, const __grid_constant__ CUtensorMap map_qm,
+    const float* __restrict__ Mst, __nv_bfloat16* __restrict__ dqm, int T, int c, int* status) {
+  using Cfg = ReadoutBwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
+  uint64_t* ld_full = bars;
+  uint64_t* acc_full = bars + 1;
+  uint64_t* tile_done = bars + 2;
+  uint64_t* drain = bars + 3;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
+
+  const int z = blockIdx.x, S = gridDim.x;
+  const int64_t bh = blockIdx.y;
+  const int g = blockIdx.z, GG = gridDim.z;
+  const int warp = warp_id_uniform(), lane = threadIdx.x % 32;
+  const int n_tiles = c / 128;
+  const int m = n_tiles > g ? (n_tiles - g + GG - 1) / GG : 0;
+  const int64_t row0 = bh * (int64_t)T + (int64_t)z * c;
+  if (m == 0) return;
+  if (z < 2) {
+    const uint4 zero = make_uint4(0, 0, 0, 0);
+    for (int idx = 0; idx < m; ++idx) {
+      uint4* dst = reinterpret_cast<uint4*>(dqm + (row0 + (int64_t)(g + idx * GG) * 128) * D);
+      for (int i = threadIdx.x; i < 128 * D / 8; i += blockDim.x) dst[i] = zero;
+    }
+    return;
+  }
+
+  if (threadIdx.x == 0) {
+    mbar_init(ld_full, 1);
+    mbar_init(acc_full, 1);
+    mbar_init(tile_done, 128);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  // B operand: M'_{s-1} (0-based chunk z reads Mst[z - 1]) as bf16 hi + lo,
+  // stored [f][j]; read K-major (N = f rows, K = j) it is M'^T.
+  {
+    const float* M = Mst + (bh * (S + 1) + z - 1) * (int64_t)D * D;
+    for (int i = threadIdx.x; i < D * D / 8; i += blockDim.x) {
+      const int f = (i * 8) / D, j = (i * 8) % D;
+      const float4 a = reinterpret_cast<const float4*>(M + f * D + j)[0];
+      const float4 b = reinterpret_cast<const float4*>(M + f * D + j)[1];
+      const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      uint4 ph, pl;
+      uint32_t* php = reinterpret_cast<uint32_t*>(&ph);
+      uint32_t* plp = reinterpret_cast<uint32_t*>(&pl);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        php[q] = pack_bf16x2(v[2 * q], v[2 * q + 1]);
+        const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&php[q]));
+        plp[q] = pack_bf16x2(v[2 * q] - hi.x, v[2 * q + 1] - hi.y);
+      }
+      const uint32_t o = bsw128_off(f, j, D);
+      *reinterpret_cast<uint4*>(smem + Cfg::kMhiOff + o) = ph;
+      *reinterpret_cast<uint4*>(smem + Cfg::kMloOff + o) = pl;
+    }
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t base = smem_u32(smem);
+
+  if (warp == 4) {
+    // ------------------------------------------------- TMA and MMA issue --
+    if (lane == 0) {
+      tma_prefetch_desc(&map_do);
+      tma_prefetch_desc(&map_qm);
+      constexpr uint32_t idesc_k = idesc_bf16_f32(128, D, false, false);
+      constexpr int kBox = 128 * 128;
+      const SDesc a_do = sdesc_sw128_split(base + Cfg::kDoOff, 16, 1024);
+      const SDesc mhi = sdesc_sw128_split(base + Cfg::kMhiOff, 16, 1024);
+      const SDesc mlo = sdesc_sw128_split(base + Cfg::kMloOff, 16, 1024);
+      bool ok = true;
+      int issued = -1;
+      for (int idx = 0; idx < m && ok; ++idx) {
+        const int kt = g + idx * GG;
+        if (idx > 0 && !(ok = mbar_wait(tile_done, (uint32_t)(idx - 1) & 1, abort_flag, status))) break;
+        issued = idx;
+        mbar_arrive_expect_tx(ld_full, 2 * Cfg::kTile);
+        for (int b = 0; b < D / 64; ++b) {
+          tma_load_2d(smem + Cfg::kDoOff + b * kBox, &map_do, ld_full, b * 64, (int)(row0 + (int64_t)kt * 128));
+          tma_load_2d(smem + Cfg::kQmOff + b * kBox, &map_qm, ld_full, b * 64, (int)(row0 + (int64_t)kt * 128));
+        }
+        if (!(ok = mbar_wait(ld_full, (uint32_t)idx & 1, abort_flag, status))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t kb_tile = (kk / 4) * kBox + (kk % 4) * 32;
+          const uint32_t kb_mat = (kk / 4) * (D * 128) + (kk % 4) * 32;
+          umma_ss(tmem, sdesc_at(a_do, kb_tile), sdesc_at(mhi, kb_mat), idesc_k, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t kb_tile = (kk / 4) * kBox + (kk % 4) * 32;
+          const uint32_t kb_mat = (kk / 4) * (D * 128) + (kk % 4) * 32;
+          umma_ss(tmem, sdesc_at(a_do, kb_tile), sdesc_at(mlo, kb_mat), idesc_k, 1u);
+        }
+        umma_commit(acc_full);
+      }
+      if (!ok && issued >= 0) mbar_wait_drain(ld_full, (uint32_t)issued & 1);
+      umma_commit(drain);
+      mbar_wait_drain(drain, 0);
+    }
+    __syncwarp();
+  } else {
+    // --------------------------------------------------- row threads --
+    const int r = threadIdx.x;
+    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint8_t* qm = smem + Cfg::kQmOff;
+    auto xval = [&](int col) -> float2 {
+      const uint32_t raw = *reinterpret_cast<const uint32_t*>(qm + bsw128_off(r, col, 128));
+      return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw));
+    };
+    bool ok = true;
+    for (int idx = 0; idx < m; ++idx) {
+      const int kt = g + idx * GG;
+      ok = __all_sync(0xffffffffu, mbar_wait(ld_full, (uint32_t)idx & 1, abort_flag, status));
+      if (!ok) break;
+      float mx = -INFINITY;
+#pragma unroll 8
+      for (int col = 0; col < D; col += 2) {
+        const float2 x = xval(col);
+        mx = fmax3(mx, x.x, x.y);
+      }
+      const float mx2 = mx * kLog2e;
+      float sum = 0.f;
+#pragma unroll 8
+      for (int col = 0; col < D; col += 2) {
+        const float2 x = xval(col);
+        sum += ex2(fmaf(x.x, kLog2e, -mx2)) + ex2(fmaf(x.y, kLog2e, -mx2));
+      }
+      const float inv = 1.f / sum;
+      ok = __all_sync(0xffffffffu, mbar_wait(acc_full, (uint32_t)idx & 1, abort_flag, status));
+      if (!ok) break;
+      tc_fence_after();
+      float dot = 0.f;
+#pragma unroll 1
+      for (int cb = 0; cb < D / 32; ++cb) {
+        uint32_t a[32];
+        tmem_ld32(lane_addr + cb * 32, a);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const float2 x = xval(cb * 32 + 2 * q);
+          dot = fmaf(__uint_as_float(a[2 * q]), ex2(fmaf(x.x, kLog2e, -mx2)), dot);
+          dot = fmaf(__uint_as_float(a[2 * q + 1]), ex2(fmaf(x.y, kLog2e, -mx2)), dot);
+        }
+      }
+      dot *= inv;
+      __nv_bfloat16* orow = dqm + (row0 + (int64_t)kt * 128 + r) * D;
+#pragma unroll 1
+      for (int cb = 0; cb < D / 32; ++cb) {
+        uint32_t a[32];
+        tmem_ld32(lane_addr + cb * 32, a);
+        tmem_wait_ld();
+        uint32_t out[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const float2 x = xval(cb * 32 + 2 * q);
+          const float p0 = ex2(fmaf(x.x, kLog2e, -mx2)) * inv, p1 = ex2(fmaf(x.y, kLog2e, -mx2)) * inv;
+          out[q] = pack_bf16x2(p0 * (__uint_as_float(a[2 * q]) - dot), p1 * (__uint_as_float(a[2 * q + 1]) - dot));
+        }
+        uint4* dst = reinterpret_cast<uint4*>(orow + cb * 32);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) dst[q] = make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
+      }
+      tc_fence_before();
+      mbar_arrive(tile_done);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 4) tmem_dealloc(tmem, Cfg::kTmemCols);
+}
+
 // --------------------------------------------------------------- host --
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -413,7 +628,30 @@ cudaError_t awm_bwd_chunk_tc_impl(const BwdProblem& b, const Workspace& fw, cons
   return cudaGetLastError();
 }
 
+template <int D>
+cudaError_t awm_bwd_readout_tc_impl(const BwdProblem& b, const Workspace& fw, cudaStream_t st) {
+  using Cfg = ReadoutBwdCfg<D>;
+  const Problem& p = b.f;
+  const int64_t BH = p.B * p.H;
+  CUtensorMap mdo, mqm;
+  cudaError_t e;
+  if ((e = awm_bwd_map(&mdo, b.dout_mem, BH * p.T, D)) != cudaSuccess) return e;
+  if ((e = awm_bwd_map(&mqm, p.qm, BH * p.T, D)) != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(awm_bwd_readout_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Cfg::kAlloc)) != cudaSuccess)
+    return e;
+  const int n_tiles = (int)(p.c / 128);
+  const int G = n_tiles > 8 ? (n_tiles + 7) / 8 : 1;
+  awm_bwd_readout_tc_kernel<D><<<dim3(p.S, (unsigned)BH, G), 160, Cfg::kAlloc, st>>>(
+      mdo, mqm, fw.Mst, static_cast<__nv_bfloat16*>(b.dqm), (int)p.T, (int)p.c, p.status);
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_awm_bwd_readout_tc(const BwdProblem& b, const Workspace& fw, cudaStream_t st) {
+  return b.f.d == 64 ? awm_bwd_readout_tc_impl<64>(b, fw, st) : awm_bwd_readout_tc_impl<128>(b, fw, st);
+}
 
 cudaError_t launch_awm_bwd_chunk_tc(const BwdProblem& b, const Workspace& fw, const BwdWorkspace& w,
                                     cudaStream_t st) {

@@ -634,13 +634,17 @@ cudaError_t awm_bwd_impl(const BwdProblem& b, const Workspace& fw, const BwdWork
         static_cast<const TIn*>(p.km), static_cast<const TIn*>(p.v), w.G, fw.Mst, fw.lse, fw.logz, w.dl,
         static_cast<TIn*>(b.dkm), w.dv_awm, p.T, (int)p.c);
   }
-  const size_t smr = sizeof(float) * (D * (D + 1) + 8 * 4 * D);
-  e = cudaFuncSetAttribute(awm_bwd_readout_simt_kernel<TIn, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smr);
-  if (e != cudaSuccess) return e;
-  awm_bwd_readout_simt_kernel<TIn, D><<<grid, 256, smr, st>>>(
-      static_cast<const TIn*>(p.qm), static_cast<const TIn*>(b.dout_mem), fw.Mst, static_cast<TIn*>(b.dqm), p.T,
-      (int)p.c);
+  if (tc) {
+    if ((e = launch_awm_bwd_readout_tc(b, fw, st)) != cudaSuccess) return e;
+  } else {
+    const size_t smr = sizeof(float) * (D * (D + 1) + 8 * 4 * D);
+    e = cudaFuncSetAttribute(awm_bwd_readout_simt_kernel<TIn, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smr);
+    if (e != cudaSuccess) return e;
+    awm_bwd_readout_simt_kernel<TIn, D><<<grid, 256, smr, st>>>(
+        static_cast<const TIn*>(p.qm), static_cast<const TIn*>(b.dout_mem), fw.Mst, static_cast<TIn*>(b.dqm), p.T,
+        (int)p.c);
+  }
   return cudaGetLastError();
 }
 

@@ -99,6 +99,7 @@ cudaError_t launch_awm_bwd(const BwdProblem& b, const Workspace& fw, const BwdWo
                            bool tc);
 cudaError_t launch_awm_bwd_chunk_tc(const BwdProblem& b, const Workspace& fw, const BwdWorkspace& w,
                                     cudaStream_t st);
+cudaError_t launch_awm_bwd_readout_tc(const BwdProblem& b, const Workspace& fw, cudaStream_t st);
 
 // ---------------------------------------------------------------- CEMA --
 
