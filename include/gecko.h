@@ -318,6 +318,46 @@ int gecko_tdnorm_forward(const void* x, void* y, const float* gamma, const float
                          int64_t B, int64_t L, int64_t D, int64_t G,
                          float beta1, float beta2, float eps, int dtype, void* stream);
 
+/*
+ * Context parallelism: one sequence split into P consecutive segments of
+ * T tokens each (one per rank, T % c == 0), run so that the outputs equal a
+ * single call over the whole sequence (up to rounding).  The AWM carry is
+ * affine in the state once log z is known (Gecko digest, method step
+ * details, step 4: M'_{s+1} = A_s M'_s + b_s with A_s = diag(r_s) -
+ * diag(rho_s) C~_s), and log z is a prefix of exp-sums (core method), so a
+ * rank needs from the ranks before it only their log-exp-sums and their
+ * composed segment maps; SCA needs the previous segment's last chunk of K
+ * and V (step 3).  A rank r:
+ *   1. gecko_awm_segment_logsum(km_r) -> lsum_r; all-gather lsum (P x [B,H,d]);
+ *   2. gecko_awm_cp_logz(lsum_all, P, r) -> logz_in_r;
+ *      gecko_awm_segment_maps(km_r, v_r, logz_in_r) -> maps_r; all-gather maps;
+ *   3. gecko_awm_cp_state(lsum_all, maps_all, P, r) -> state_in_r, then
+ *      gecko_sca_awm_forward_continue with k, v prefixed by the previous
+ *      segment's last c rows (rank 0: a fresh gecko_sca_awm_forward).
+ * All buffers are device memory, fp32 unless stated, 16-byte aligned.
+ */
+/* lsum_out [B,H,d]: log sum over the segment's tokens of exp(km) per feature.
+ * km [B,H,T,d] dtype.  Same size rules and errors as the forward. */
+int gecko_awm_segment_logsum(const void* km, float* lsum_out,
+                             int64_t B, int64_t H, int64_t T, int64_t c, int64_t d,
+                             int dtype, void* stream);
+/* maps_out [B,H,4,d,d] = (A, b, A', b'): with log z entering the segment at
+ * logz_in [B,H,d] (-inf entries for the first segment), the segment maps its
+ * incoming state M'_in to M'_out = A M'_in + b (after its last chunk) and
+ * to A' M'_in + b' (before its last chunk).  km, v [B,H,T,d] dtype. */
+int gecko_awm_segment_maps(const void* km, const void* v, const float* logz_in, float* maps_out,
+                           int64_t B, int64_t H, int64_t T, int64_t c, int64_t d,
+                           int dtype, void* stream);
+/* logz_out [B,H,d] = logsumexp over the segments j < rank of lsum_all[j]
+ * (lsum_all [P,B,H,d]); -inf for rank 0. */
+int gecko_awm_cp_logz(const float* lsum_all, int P, int rank, float* logz_out,
+                      int64_t B, int64_t H, int64_t d, void* stream);
+/* state_out [B,H,2d^2+d] = (M'_prev, M'_in, log z) for segment `rank`, the
+ * state_in of gecko_sca_awm_forward_continue, from every rank's lsum
+ * [P,B,H,d] and maps [P,B,H,4,d,d] (zeros and -inf for rank 0). */
+int gecko_awm_cp_state(const float* lsum_all, const float* maps_all, int P, int rank, float* state_out,
+                       int64_t B, int64_t H, int64_t d, void* stream);
+
 /* Thread-local message describing the last non-zero status of this thread. */
 const char* gecko_last_error(void);
 

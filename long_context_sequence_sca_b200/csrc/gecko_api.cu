@@ -421,6 +421,106 @@ extern "C" int gecko_sca_awm_backward(const void* q, const void* k, const void* 
                       c, d, dtype, stream);
 }
 
+// ----------------------------------------------------- context parallelism
+
+extern "C" int gecko_awm_segment_logsum(const void* km, float* lsum_out, int64_t B, int64_t H, int64_t T, int64_t c,
+                                        int64_t d, int dtype, void* stream) {
+  const void* ptrs[2] = {km, lsum_out};
+  int rc = validate(ptrs, 2, B, H, T, c, d, dtype);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int dev = 0;
+  if ((rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice"))) return rc;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState* ds = nullptr;
+  if ((rc = device_state(dev, &ds))) return rc;
+  const int64_t S = T / c, BH = B * H;
+  if ((rc = ensure_buffer(&ds->ws, &ds->ws_bytes, workspace_bytes(BH, T, c, d), st, "workspace"))) return rc;
+  Workspace w = carve_workspace(ds->ws, BH, T, c, d);
+  Problem p{nullptr, nullptr, nullptr, nullptr, km, nullptr, nullptr, B, H, T, c, d, (int)S, dtype, ds->status};
+  cudaGetLastError();
+  if ((rc = check_cuda(launch_awm_stats(p, w, st), "awm stats"))) return rc;
+  // log z^S of the segment started from zero = the log-sum of all its tokens
+  return check_cuda(cudaMemcpy2DAsync(lsum_out, sizeof(float) * d, w.logz + (S - 1) * d, sizeof(float) * d * S,
+                                      sizeof(float) * d, BH, cudaMemcpyDeviceToDevice, st),
+                    "copy log-sum");
+}
+
+extern "C" int gecko_awm_segment_maps(const void* km, const void* v, const float* logz_in, float* maps_out,
+                                      int64_t B, int64_t H, int64_t T, int64_t c, int64_t d, int dtype,
+                                      void* stream) {
+  const void* ptrs[4] = {km, v, logz_in, maps_out};
+  int rc = validate(ptrs, 4, B, H, T, c, d, dtype);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int dev = 0;
+  if ((rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice"))) return rc;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState* ds = nullptr;
+  if ((rc = device_state(dev, &ds))) return rc;
+  const int64_t S = T / c, BH = B * H, sd = state_floats(d), mat = d * d;
+  if ((rc = ensure_buffer(&ds->ws, &ds->ws_bytes, workspace_bytes(BH, T, c, d), st, "workspace"))) return rc;
+  if ((rc = ensure_buffer(&ds->state, &ds->state_bytes, sizeof(float) * BH * sd, st, "state"))) return rc;
+  Workspace w = carve_workspace(ds->ws, BH, T, c, d);
+  float* state = static_cast<float*>(ds->state);
+  Problem p{nullptr, nullptr, v, nullptr, km, nullptr, nullptr, B, H, T, c, d, (int)S, dtype, ds->status};
+  p.state0 = state;   // log z seed and the carry's starting state; no prepended K/V rows (koff = 0)
+  const bool use_tc = !env_is("GECKO_KERNELS", "simt") && tc_supported(p);
+  cudaGetLastError();
+  if ((rc = check_cuda(cudaMemsetAsync(state, 0, sizeof(float) * BH * sd, st), "clear state"))) return rc;
+  if ((rc = check_cuda(cudaMemcpy2DAsync(state + 2 * mat, sizeof(float) * sd, logz_in, sizeof(float) * d,
+                                         sizeof(float) * d, BH, cudaMemcpyDeviceToDevice, st),
+                       "seed log z")))
+    return rc;
+  if ((rc = check_cuda(launch_awm_stats(p, w, st), "awm stats"))) return rc;
+  if ((rc = check_cuda(use_tc ? launch_awm_chunk_tc(p, w, st) : launch_awm_chunk_simt(p, w, st), "awm chunk")))
+    return rc;
+  // maps_out[bh] = (A, b, A', b'): the carry from M'_in = 0 gives b (after the
+  // last chunk) and b' (before it); with the chunk terms zeroed and M'_in = I
+  // it gives A and A'.
+  auto take = [&](int slot_last, int slot_prev) -> int {
+    const size_t m4 = sizeof(float) * mat;
+    int r = check_cuda(cudaMemcpy2DAsync(maps_out + slot_last * mat, 4 * m4, w.Mst + S * mat, (S + 1) * m4, m4, BH,
+                                         cudaMemcpyDeviceToDevice, st),
+                       "copy map");
+    if (r) return r;
+    return check_cuda(cudaMemcpy2DAsync(maps_out + slot_prev * mat, 4 * m4, w.Mst + (S - 1) * mat, (S + 1) * m4,
+                                        m4, BH, cudaMemcpyDeviceToDevice, st),
+                      "copy map");
+  };
+  if ((rc = check_cuda(launch_awm_carry(p, w, st), "awm carry"))) return rc;
+  if ((rc = take(1, 3))) return rc;
+  if ((rc = check_cuda(cudaMemsetAsync(w.Bm, 0, sizeof(float) * BH * S * mat, st), "clear chunk terms"))) return rc;
+  if ((rc = check_cuda(launch_set_identity(state + mat, sd, (int)d, BH, st), "identity"))) return rc;
+  if ((rc = check_cuda(launch_awm_carry(p, w, st), "awm carry"))) return rc;
+  return take(0, 2);
+}
+
+extern "C" int gecko_awm_cp_logz(const float* lsum_all, int P, int rank, float* logz_out, int64_t B, int64_t H,
+                                 int64_t d, void* stream) {
+  if (!lsum_all || !logz_out) return fail(GECKO_ERR_ARG, "NULL pointer");
+  if (P < 1 || rank < 0 || rank >= P) return fail(GECKO_ERR_ARG, "rank %d of %d", rank, P);
+  if (B < 1 || H < 1 || (d != 64 && d != 128)) return fail(GECKO_ERR_SHAPE, "bad B, H or d");
+  cudaGetLastError();
+  return check_cuda(launch_cp_logz(lsum_all, logz_out, rank, B * H, (int)d, d, static_cast<cudaStream_t>(stream)),
+                    "cp log z");
+}
+
+extern "C" int gecko_awm_cp_state(const float* lsum_all, const float* maps_all, int P, int rank, float* state_out,
+                                  int64_t B, int64_t H, int64_t d, void* stream) {
+  if (!lsum_all || !maps_all || !state_out) return fail(GECKO_ERR_ARG, "NULL pointer");
+  if (P < 1 || rank < 0 || rank >= P) return fail(GECKO_ERR_ARG, "rank %d of %d", rank, P);
+  if (B < 1 || H < 1 || (d != 64 && d != 128)) return fail(GECKO_ERR_SHAPE, "bad B, H or d");
+  if (reinterpret_cast<uintptr_t>(maps_all) % 16 != 0) return fail(GECKO_ERR_ALIGN, "maps not 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t BH = B * H, sd = state_floats(d);
+  cudaGetLastError();
+  int rc;
+  if ((rc = check_cuda(launch_cp_logz(lsum_all, state_out + 2 * d * d, rank, BH, (int)d, sd, st), "cp log z")))
+    return rc;
+  return check_cuda(launch_cp_compose(maps_all, state_out, rank, BH, (int)d, sd, st), "cp compose");
+}
+
 extern "C" int gecko_sca_awm_forward(const void* q, const void* k, const void* v, const void* qm, const void* km,
                                      void* out_sca, void* out_mem, int64_t B, int64_t H, int64_t T, int64_t c,
                                      int64_t d, int dtype, void* stream) {

@@ -101,6 +101,15 @@ cudaError_t launch_awm_bwd_chunk_tc(const BwdProblem& b, const Workspace& fw, co
                                     cudaStream_t st);
 cudaError_t launch_awm_bwd_readout_tc(const BwdProblem& b, const Workspace& fw, cudaStream_t st);
 
+// -------------------------------------------------- context parallelism --
+
+cudaError_t launch_set_identity(float* dst, int64_t stride, int d, int64_t BH, cudaStream_t st);
+// out[bh * sd + f] = logsumexp_{j < rank} lsum[j, bh, f]  (-inf for rank 0)
+cudaError_t launch_cp_logz(const float* lsum, float* out, int rank, int64_t BH, int d, int64_t sd, cudaStream_t st);
+// out[bh * sd] = M'_prev, out[bh * sd + d*d] = M'_in from the maps of ranks < rank
+cudaError_t launch_cp_compose(const float* maps, float* out, int rank, int64_t BH, int d, int64_t sd,
+                              cudaStream_t st);
+
 // ---------------------------------------------------------------- CEMA --
 
 // One validated CEMA call: x, y [B, L, D] (dtype); alpha, delta, theta,

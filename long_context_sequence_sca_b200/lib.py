@@ -23,6 +23,10 @@ EXPORTS = (
     "gecko_awm_state",
     "gecko_cema_forward",
     "gecko_tdnorm_forward",
+    "gecko_awm_segment_logsum",
+    "gecko_awm_segment_maps",
+    "gecko_awm_cp_logz",
+    "gecko_awm_cp_state",
     "gecko_device_status",
     "gecko_timing_enable",
     "gecko_timing_read",
@@ -79,6 +83,15 @@ def load() -> ctypes.CDLL:
     f32 = ctypes.c_float
     lib.gecko_tdnorm_forward.argtypes = [vp] * 4 + [i64] * 4 + [f32, f32, f32, ctypes.c_int, vp]
     lib.gecko_tdnorm_forward.restype = ctypes.c_int
+    ci = ctypes.c_int
+    lib.gecko_awm_segment_logsum.argtypes = [vp, vp] + [i64] * 5 + [ci, vp]
+    lib.gecko_awm_segment_logsum.restype = ci
+    lib.gecko_awm_segment_maps.argtypes = [vp] * 4 + [i64] * 5 + [ci, vp]
+    lib.gecko_awm_segment_maps.restype = ci
+    lib.gecko_awm_cp_logz.argtypes = [vp, ci, ci, vp, i64, i64, i64, vp]
+    lib.gecko_awm_cp_logz.restype = ci
+    lib.gecko_awm_cp_state.argtypes = [vp, vp, ci, ci, vp, i64, i64, i64, vp]
+    lib.gecko_awm_cp_state.restype = ci
     lib.gecko_device_status.argtypes = [vp]
     lib.gecko_device_status.restype = ctypes.c_int
     lib.gecko_timing_enable.argtypes = [ctypes.c_int]
@@ -155,6 +168,22 @@ def gecko_cema_forward(x, y, alpha, delta, theta, beta, eta, reset, state_in, st
 def gecko_tdnorm_forward(x, y, gamma, bias, B, L, D, G, beta1, beta2, eps, dtype, stream) -> int:
     """Direct call of the timestep-normalisation entry point with integer pointers."""
     return load().gecko_tdnorm_forward(x, y, gamma, bias, B, L, D, G, beta1, beta2, eps, dtype, stream)
+
+
+def gecko_awm_segment_logsum(km, lsum_out, B, H, T, c, d, dtype, stream) -> int:
+    return load().gecko_awm_segment_logsum(km, lsum_out, B, H, T, c, d, dtype, stream)
+
+
+def gecko_awm_segment_maps(km, v, logz_in, maps_out, B, H, T, c, d, dtype, stream) -> int:
+    return load().gecko_awm_segment_maps(km, v, logz_in, maps_out, B, H, T, c, d, dtype, stream)
+
+
+def gecko_awm_cp_logz(lsum_all, P, rank, logz_out, B, H, d, stream) -> int:
+    return load().gecko_awm_cp_logz(lsum_all, P, rank, logz_out, B, H, d, stream)
+
+
+def gecko_awm_cp_state(lsum_all, maps_all, P, rank, state_out, B, H, d, stream) -> int:
+    return load().gecko_awm_cp_state(lsum_all, maps_all, P, rank, state_out, B, H, d, stream)
 
 
 def gecko_device_status(stream) -> int:
@@ -389,3 +418,53 @@ def tdnorm_forward(x, gamma, bias, G: int, beta1: float, beta2: float, eps: floa
                                   beta1, beta2, eps, _DT[x.dtype], _stream_handle(stream))
     _check(rc)
     return y
+
+
+# ------------------------------------------------ context parallelism -----
+
+def awm_segment_logsum(km, c: int, stream=None):
+    """[B, H, d] fp32: log sum over the segment's tokens of exp(km)."""
+    _check_inputs((km,))
+    B, H, T, d = km.shape
+    out = torch.empty((B, H, d), dtype=torch.float32, device=km.device)
+    with torch.cuda.device(km.device):
+        rc = gecko_awm_segment_logsum(km.data_ptr(), out.data_ptr(), B, H, T, c, d, _DT[km.dtype],
+                                      _stream_handle(stream))
+    _check(rc)
+    return out
+
+
+def awm_segment_maps(km, v, logz_in, c: int, stream=None):
+    """[B, H, 4, d, d] fp32 maps (A, b, A', b') of the segment for the log z
+    entering it (logz_in [B, H, d] fp32)."""
+    _check_inputs((km, v))
+    B, H, T, d = km.shape
+    out = torch.empty((B, H, 4, d, d), dtype=torch.float32, device=km.device)
+    with torch.cuda.device(km.device):
+        rc = gecko_awm_segment_maps(km.data_ptr(), v.data_ptr(), logz_in.contiguous().data_ptr(), out.data_ptr(),
+                                    B, H, T, c, d, _DT[km.dtype], _stream_handle(stream))
+    _check(rc)
+    return out
+
+
+def awm_cp_logz(lsum_all, rank: int, stream=None):
+    """log z entering segment `rank` from every rank's log-sum [P, B, H, d]."""
+    P, B, H, d = lsum_all.shape
+    out = torch.empty((B, H, d), dtype=torch.float32, device=lsum_all.device)
+    with torch.cuda.device(lsum_all.device):
+        rc = gecko_awm_cp_logz(lsum_all.contiguous().data_ptr(), P, rank, out.data_ptr(), B, H, d,
+                               _stream_handle(stream))
+    _check(rc)
+    return out
+
+
+def awm_cp_state(lsum_all, maps_all, rank: int, stream=None):
+    """state_in [B, H, 2 d^2 + d] of segment `rank` (M'_prev, M'_in, log z)."""
+    P, B, H, d = lsum_all.shape
+    out = torch.empty((B, H, 2 * d * d + d), dtype=torch.float32, device=lsum_all.device)
+    with torch.cuda.device(lsum_all.device):
+        rc = gecko_awm_cp_state(lsum_all.contiguous().data_ptr(), maps_all.contiguous().data_ptr(), P, rank,
+                                out.data_ptr(), B, H, d, _stream_handle(stream))
+    _check(rc)
+    return out
+
