@@ -16,13 +16,16 @@
 //                dK += dS^T Q_i read them from TMEM (TS form).
 //   kDQ = true   rows are queries: S = Q K_j^T and dP = dO V_j^T for the key
 //                tiles of the window; dQ += dS K_j.
-// Roles (320 threads): warp 0 TMA producer (the CTA's two fixed tiles once,
+// Roles (576 threads): warp 0 TMA producer (the CTA's two fixed tiles once,
 // then a ring of two-tile stages for the loop operands, with the loop rows'
 // statistics for kDQ = false), warp 1 TMEM allocator and MMA issuer, warps
-// 2-9 two element-wise warpgroups, each owning 64 of the 128 loop columns
+// 2-17 four element-wise warpgroups, each owning 32 of the 128 loop columns
 // (warpgroup w writes its packed bf16 results over the S columns it has
-// consumed, at column 64 w, and the TS MMAs read each 16-column K step from
-// where its warpgroup put it).  Only the diagonal tile is masked.
+// consumed, at column 32 w, and the TS MMAs read each 16-column K step from
+// where its warpgroup put it).  Four warps per sub-partition, one 32-column
+// TMEM round trip each, keep the TMEM latency of the element-wise pass
+// hidden (with two warpgroups of 64 columns it took 2.4x its SFU time).
+// Only the diagonal tile is masked.
 //
 // Requires bf16, d in {64, 128}, c % 128 == 0.  Every wait is bounded; on a
 // timeout the CTA drains its copies and MMAs, frees TMEM and returns with
@@ -34,7 +37,19 @@ namespace gecko {
 namespace {
 
 constexpr int kRows = 128;          // rows per tile (keys or queries)
-constexpr int kBwdThreads = 320;
+constexpr int kEW = 4;                   // element-wise warpgroups
+constexpr int kCW = kRows / kEW;         // loop columns per warpgroup
+constexpr int kBwdThreads = 64 + 128 * kEW;
+static_assert(kCW % 32 == 0, "whole 32-column TMEM loads per warpgroup");
+// Of every 8 exponential pairs of P, GECKO_BWD_SFU_PAIRS go to the SFU and the
+// rest to the FMA pipe (exp2_poly2).  Measured on B200 (bench workload):
+// 8/8 on the SFU is fastest (dK/dV 5.80 ms against 7.06 ms at 6/8, where the
+// polynomial's registers push the 96-register budget into spills), so 8 is
+// the default and other splits remain a compile-time option.
+#ifndef GECKO_BWD_SFU_PAIRS
+#define GECKO_BWD_SFU_PAIRS 8
+#endif
+constexpr int kBwdSfuPairs = GECKO_BWD_SFU_PAIRS;
 
 template <int D>
 struct BwdCfg {
@@ -46,16 +61,20 @@ struct BwdCfg {
   static constexpr int kFixOff = 0;
   static constexpr int kStageOff = 2 * kTileBytes;
   static constexpr int kBarOff = kStageOff + kStages * kStageBytes;
-  // fix_full, ld_full[NS], ld_empty[NS], s_full, p_full, acc_full, drain
-  static constexpr int kNumBars = 1 + 2 * kStages + 4;
+  // fix_full, ld_full[NS], ld_empty[NS], s_ready, dp_ready, p_done, ds_done, acc_full, drain
+  static constexpr int kNumBars = 1 + 2 * kStages + 6;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;
   static_assert(kStageBytes % 1024 == 0 && kStageOff % 1024 == 0, "1024-byte aligned operand tiles");
   static_assert(kAlloc <= 232448, "dynamic shared memory above the sm_100 per-block limit");
   static constexpr uint32_t kTmemCols = 512;
-  // S (then P or dS, packed), dP (then dS, packed), accumulators A and B
+  // S (then P, packed), dP (then dS, packed; dK/dV kernel), accumulators A
+  // and B, and (dQ kernel) two buffers for packed dS in the spare columns
   static constexpr uint32_t kColS = 0, kColP = 128, kColA = 256, kColB = 256 + D;
+  static constexpr uint32_t kColF = 384;   // + 64 * (step % 2), 64 packed columns each
+  // the dK/dV kernel uses accumulators A and B, the dQ kernel A and the dS buffers
+  static_assert(kColF + 128 <= kTmemCols && kColA + D <= kColF && kColB + D <= kTmemCols, "TMEM columns");
 };
 
 // Tile coordinates of CTA `bid`.  CTAs of one (b, h, chunk) are adjacent
@@ -103,9 +122,14 @@ sca_bwd_tc_kernel(const __grid_constant__ CUtensorMap map_fix0, const __grid_con
   uint64_t* fix_full = bars;
   uint64_t* ld_full = bars + 1;
   uint64_t* ld_empty = ld_full + NS;
-  uint64_t* s_full = ld_empty + NS;
-  uint64_t* p_full = s_full + 1;
-  uint64_t* acc_full = p_full + 1;
+  // S and dP are committed separately, so the exponentials of P overlap the
+  // dP product and the previous step's dK product; P (dK/dV kernel) and dS
+  // are handed back separately for the same reason.
+  uint64_t* s_ready = ld_empty + NS;
+  uint64_t* dp_ready = s_ready + 1;
+  uint64_t* p_done = dp_ready + 1;
+  uint64_t* ds_done = p_done + 1;
+  uint64_t* acc_full = ds_done + 1;
   uint64_t* drain = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
@@ -122,8 +146,10 @@ sca_bwd_tc_kernel(const __grid_constant__ CUtensorMap map_fix0, const __grid_con
       mbar_init(ld_full + s, 1);
       mbar_init(ld_empty + s, 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(p_full, 256);
+    mbar_init(s_ready, 1);
+    mbar_init(dp_ready, 1);
+    mbar_init(p_done, 128 * kEW);
+    mbar_init(ds_done, 128 * kEW);
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -185,47 +211,83 @@ sca_bwd_tc_kernel(const __grid_constant__ CUtensorMap map_fix0, const __grid_con
       const uint32_t fa = smem_u32(sFix), sa = smem_u32(sStage);
       bool ok = mbar_wait(fix_full, 0, abort_flag, status);
       tc_fence_after();
+      const SDesc a0 = sdesc_sw128_split(fa, 16, 1024), a1 = sdesc_sw128_split(fa + Cfg::kTileBytes, 16, 1024);
+      // Per step n the order is: the P-side product of step n - 1 (dV; dQ's
+      // only product), S(n), the dS-side product of step n - 1 (dK), dP(n).
+      // Each product overwrites a TMEM region only after the product that
+      // read it was issued (the tensor pipe runs them in order).
+      auto ts_products = [&](int m, bool p_side) {
+        const uint32_t pb = sa + (m % NS) * Cfg::kStageBytes;
+        const SDesc b0 = sdesc_sw128_split(pb, Cfg::kBoxBytes, 1024);                     // st0, MN-major
+        const SDesc b1 = sdesc_sw128_split(pb + Cfg::kTileBytes, Cfg::kBoxBytes, 1024);   // st1, MN-major
+#pragma unroll
+        for (int kk = 0; kk < kRows / 16; ++kk) {
+          // K step kk covers loop columns 16 kk .. 16 kk + 15, packed by
+          // warpgroup (16 kk) / kCW at its own column offset
+          const uint32_t acol = (uint32_t)((16 * kk / kCW) * kCW + (16 * kk % kCW) / 2);
+          const uint32_t acc = (m > 0 || kk > 0) ? 1u : 0u;
+          if (kDQ)
+            // dS buffers are packed compactly: loop column q at column q / 2
+            umma_ts(tmem + Cfg::kColA, tmem + Cfg::kColF + 64 * (m % 2) + 8 * kk, sdesc_at(b0, kk * 2048), idesc_ts,
+                    acc);  // dQ += dS K
+          else if (p_side)
+            umma_ts(tmem + Cfg::kColA, tmem + Cfg::kColS + acol, sdesc_at(b1, kk * 2048), idesc_ts, acc);  // dV += P^T dO
+          else
+            umma_ts(tmem + Cfg::kColB, tmem + Cfg::kColP + acol, sdesc_at(b0, kk * 2048), idesc_ts, acc);  // dK += dS^T Q
+        }
+      };
+      auto ss_product = [&](int m, uint32_t col, const SDesc& a, int tile) {
+        const SDesc bq = sdesc_sw128_split(sa + (m % NS) * Cfg::kStageBytes + tile * Cfg::kTileBytes, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t kbyte = (kk / 4) * Cfg::kBoxBytes + (kk % 4) * 32;
+          umma_ss(tmem + col, sdesc_at(a, kbyte), sdesc_at(bq, kbyte), idesc_ss, kk > 0 ? 1u : 0u);
+        }
+      };
       for (int n = 0; n <= N && ok; ++n) {
+        if (kDQ) {
+          // dQ kernel: S(n) as soon as P(n - 1) has been read out of S, so
+          // the exponentials of step n overlap dQ(n - 1) and dP(n); dS lives
+          // in its own double buffer
+          if (n < N) {
+            if (n > 0 && !(ok = mbar_wait(p_done, (uint32_t)(n - 1) & 1, abort_flag, status))) break;
+            if (!(ok = mbar_wait(ld_full + n % NS, (uint32_t)(n / NS) & 1, abort_flag, status))) break;
+            tc_fence_after();
+            ss_product(n, Cfg::kColS, a0, 0);   // S = fix0 st0^T
+            umma_commit(s_ready);
+          }
+          if (n > 0) {
+            if (!(ok = mbar_wait(ds_done, (uint32_t)(n - 1) & 1, abort_flag, status))) break;
+            tc_fence_after();
+            ts_products(n - 1, true);
+            umma_commit(ld_empty + (n - 1) % NS);
+          }
+          if (n < N) {
+            ss_product(n, Cfg::kColP, a1, 1);   // dP = fix1 st1^T
+            umma_commit(dp_ready);
+          }
+          continue;
+        }
+        if (n > 0) {
+          if (!(ok = mbar_wait(p_done, (uint32_t)(n - 1) & 1, abort_flag, status))) break;
+          tc_fence_after();
+          ts_products(n - 1, true);
+        }
         if (n < N) {
           if (!(ok = mbar_wait(ld_full + n % NS, (uint32_t)(n / NS) & 1, abort_flag, status))) break;
           tc_fence_after();
+          ss_product(n, Cfg::kColS, a0, 0);   // S = fix0 st0^T
+          umma_commit(s_ready);
         }
         if (n > 0) {
-          // the products of step n - 1 with the element-wise results in TMEM
-          if (!(ok = mbar_wait(p_full, (uint32_t)(n - 1) & 1, abort_flag, status))) break;
+          if (!(ok = mbar_wait(ds_done, (uint32_t)(n - 1) & 1, abort_flag, status))) break;
           tc_fence_after();
-          const uint32_t pb = sa + ((n - 1) % NS) * Cfg::kStageBytes;
-          const SDesc b0 = sdesc_sw128_split(pb, Cfg::kBoxBytes, 1024);                     // st0, MN-major
-          const SDesc b1 = sdesc_sw128_split(pb + Cfg::kTileBytes, Cfg::kBoxBytes, 1024);   // st1, MN-major
-#pragma unroll
-          for (int kk = 0; kk < kRows / 16; ++kk) {
-            const uint32_t acol = (kk / 4) * 64 + (kk % 4) * 8;
-            const uint32_t acc = (n - 1 > 0 || kk > 0) ? 1u : 0u;
-            if (!kDQ) {
-              umma_ts(tmem + Cfg::kColA, tmem + Cfg::kColS + acol, sdesc_at(b1, kk * 2048), idesc_ts, acc);  // dV += P^T dO
-              umma_ts(tmem + Cfg::kColB, tmem + Cfg::kColP + acol, sdesc_at(b0, kk * 2048), idesc_ts, acc);  // dK += dS^T Q
-            } else {
-              umma_ts(tmem + Cfg::kColA, tmem + Cfg::kColS + acol, sdesc_at(b0, kk * 2048), idesc_ts, acc);  // dQ += dS K
-            }
-          }
+          ts_products(n - 1, false);
           umma_commit(ld_empty + (n - 1) % NS);
         }
         if (n < N) {
-          // S = fix0 st0^T, dP = fix1 st1^T  (K-major operands)
-          const uint32_t sb = sa + (n % NS) * Cfg::kStageBytes;
-          const SDesc a0 = sdesc_sw128_split(fa, 16, 1024), a1 = sdesc_sw128_split(fa + Cfg::kTileBytes, 16, 1024);
-          const SDesc c0 = sdesc_sw128_split(sb, 16, 1024), c1 = sdesc_sw128_split(sb + Cfg::kTileBytes, 16, 1024);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t kbyte = (kk / 4) * Cfg::kBoxBytes + (kk % 4) * 32;
-            umma_ss(tmem + Cfg::kColS, sdesc_at(a0, kbyte), sdesc_at(c0, kbyte), idesc_ss, kk > 0 ? 1u : 0u);
-          }
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t kbyte = (kk / 4) * Cfg::kBoxBytes + (kk % 4) * 32;
-            umma_ss(tmem + Cfg::kColP, sdesc_at(a1, kbyte), sdesc_at(c1, kbyte), idesc_ss, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(s_full);
+          ss_product(n, Cfg::kColP, a1, 1);   // dP = fix1 st1^T
+          umma_commit(dp_ready);
         }
       }
       if (ok) umma_commit(acc_full);
@@ -236,7 +298,7 @@ sca_bwd_tc_kernel(const __grid_constant__ CUtensorMap map_fix0, const __grid_con
     __syncwarp();
   } else {
     // ------------------------------------------- element-wise warpgroups --
-    const int w = (warp - 2) / 4;             // loop columns 64 w .. 64 w + 63
+    const int w = (warp - 2) / 4;             // loop columns kCW w .. kCW w + kCW - 1
     const int r = (warp % 4) * 32 + lane;     // row within the tile = TMEM lane
     const uint32_t lane_addr = tmem + ((uint32_t)((warp % 4) * 32) << 16);
     const uint64_t l2e2 = pack2(kLog2e, kLog2e);
@@ -247,7 +309,7 @@ sca_bwd_tc_kernel(const __grid_constant__ CUtensorMap map_fix0, const __grid_con
     }
     bool ok = true;
     for (int n = 0; n < N; ++n) {
-      ok = __all_sync(0xffffffffu, mbar_wait(s_full, (uint32_t)n & 1, abort_flag, status));
+      ok = __all_sync(0xffffffffu, mbar_wait(s_ready, (uint32_t)n & 1, abort_flag, status));
       if (!ok) break;
       if (!kDQ) {
         // the loop rows' statistics came with the stage's copies
@@ -258,65 +320,108 @@ sca_bwd_tc_kernel(const __grid_constant__ CUtensorMap map_fix0, const __grid_con
       const bool diag = tile.beg + n == tile.row;
       const float* st_nl = reinterpret_cast<const float*>(sStage + (n % NS) * Cfg::kStageBytes + 2 * Cfg::kTileBytes);
       const float* st_dl = st_nl + kRows;
+      // P = 2^(S log2 e - log2(e) l), kept in fp32 for dS; the dK/dV kernel
+      // also hands P (bf16) to the dV product
+      float pf[kCW];
 #pragma unroll
-      for (int cb = 0; cb < 2; ++cb) {
-        const int col0 = 64 * w + 32 * cb;
-        uint32_t sv[32], pv[32];
+      for (int cb = 0; cb < kCW / 32; ++cb) {
+        const int col0 = kCW * w + 32 * cb;
+        uint32_t sv[32];
         tmem_ld32p(lane_addr + Cfg::kColS + col0, sv);
-        tmem_ld32p(lane_addr + Cfg::kColP + col0, pv);
         tmem_wait_ld();
-        uint32_t pkP[16], pkD[16];
+        uint32_t pkP[16];
 #pragma unroll
         for (int x = 0; x < 16; ++x) {
           const int cc = col0 + 2 * x;
-          uint64_t nl2, dl2;
+          uint64_t nl2;
           if (kDQ) {
             nl2 = pack2(my_nl, my_nl);
-            dl2 = pack2(-my_dl, -my_dl);
           } else {
             const float2 a = reinterpret_cast<const float2*>(st_nl)[cc / 2];
-            const float2 b = reinterpret_cast<const float2*>(st_dl)[cc / 2];
             nl2 = pack2(a.x, a.y);
-            dl2 = pack2(-b.x, -b.y);
           }
-          float a0, a1;
-          unpack2(ffma2(pack2(__uint_as_float(sv[2 * x]), __uint_as_float(sv[2 * x + 1])), l2e2, nl2), a0, a1);
-          float p0 = ex2(a0), p1 = ex2(a1);
+          const uint64_t a2 = ffma2(pack2(__uint_as_float(sv[2 * x]), __uint_as_float(sv[2 * x + 1])), l2e2, nl2);
+          float p0, p1;
+          if (x % 8 < kBwdSfuPairs) {
+            float a0, a1;
+            unpack2(a2, a0, a1);
+            p0 = ex2(a0);
+            p1 = ex2(a1);
+          } else {
+            unpack2(exp2_poly2(a2), p0, p1);
+          }
           if (diag) {
             // dK/dV: rows are keys, a query before the key sees nothing;
             // dQ: rows are queries, keys after the query are masked
             if (kDQ ? (cc > r) : (cc < r)) p0 = 0.f;
             if (kDQ ? (cc + 1 > r) : (cc + 1 < r)) p1 = 0.f;
           }
-          const uint64_t p2 = pack2(p0, p1);
-          float d0, d1;
-          unpack2(fmul2(p2, fadd2(pack2(__uint_as_float(pv[2 * x]), __uint_as_float(pv[2 * x + 1])), dl2)), d0, d1);
+          pf[32 * cb + 2 * x] = p0;
+          pf[32 * cb + 2 * x + 1] = p1;
           pkP[x] = pack_bf16x2(p0, p1);
-          pkD[x] = pack_bf16x2(d0, d1);
         }
-        if (!kDQ) {
-          tmem_st16(lane_addr + Cfg::kColS + 64 * w + 16 * cb, pkP);
-          tmem_st16(lane_addr + Cfg::kColP + 64 * w + 16 * cb, pkD);
-        } else {
-          tmem_st16(lane_addr + Cfg::kColS + 64 * w + 16 * cb, pkD);
+        if (!kDQ) tmem_st16(lane_addr + Cfg::kColS + kCW * w + 16 * cb, pkP);
+      }
+      // S has been read (and, for dK/dV, P written): the MMA thread may go on
+      if (!kDQ) tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_done);
+      // dS = P (dP - delta)
+      ok = __all_sync(0xffffffffu, mbar_wait(dp_ready, (uint32_t)n & 1, abort_flag, status));
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int cb = 0; cb < kCW / 32; ++cb) {
+        const int col0 = kCW * w + 32 * cb;
+        uint32_t pkD[16];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {   // 16 columns of dP at a time (register budget)
+          uint32_t pv[16];
+          tmem_ld16p(lane_addr + Cfg::kColP + col0 + 16 * hh, pv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int x = 0; x < 8; ++x) {
+            const int cc = col0 + 16 * hh + 2 * x;
+            uint64_t dl2;
+            if (kDQ) {
+              dl2 = pack2(-my_dl, -my_dl);
+            } else {
+              const float2 b = reinterpret_cast<const float2*>(st_dl)[cc / 2];
+              dl2 = pack2(-b.x, -b.y);
+            }
+            const int pi = 32 * cb + 16 * hh + 2 * x;
+            float d0, d1;
+            unpack2(fmul2(pack2(pf[pi], pf[pi + 1]),
+                          fadd2(pack2(__uint_as_float(pv[2 * x]), __uint_as_float(pv[2 * x + 1])), dl2)),
+                    d0, d1);
+            pkD[8 * hh + x] = pack_bf16x2(d0, d1);
+          }
         }
+        tmem_st16(lane_addr + (kDQ ? Cfg::kColF + 64 * (n % 2) + (kCW / 2) * w : Cfg::kColP + kCW * w) + 16 * cb,
+                  pkD);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(ds_done);
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, status));
     if (ok) {
       tc_fence_after();
       const int64_t grow = rowbase + (int64_t)tile.row * kRows + r;
-      // dK/dV: warpgroup 0 writes dV (+ the AWM part), warpgroup 1 dK;
-      // dQ: warpgroup w writes columns [w D/2, (w+1) D/2)
-      const uint32_t col = kDQ ? Cfg::kColA + (uint32_t)(w * D / 2) : (w == 0 ? Cfg::kColA : Cfg::kColB);
-      __nv_bfloat16* orow = (kDQ || w == 0 ? out_a : out_b) + grow * D + (kDQ ? w * D / 2 : 0);
-      const float* add = (!kDQ && w == 0 && dv_add) ? dv_add + grow * D : nullptr;
-      constexpr int NCB = kDQ ? D / 64 : D / 32;
+      // dK/dV: the 2D output columns of a row (dV, with the AWM part added,
+      // then dK) split evenly over the warpgroups; dQ: 32 columns per
+      // warpgroup (those past D have none).  `active` is warp-uniform.
+      constexpr int OW = kDQ ? 32 : 2 * D / kEW;
+      static_assert(OW % 32 == 0, "whole 32-column TMEM loads in the epilogue");
+      const int c0 = w * OW;
+      const bool active = !kDQ || c0 < D;
+      const bool is_dk = !kDQ && c0 >= D;
+      const int cc0 = is_dk ? c0 - D : c0;
+      const uint32_t col = (is_dk ? Cfg::kColB : Cfg::kColA) + (uint32_t)cc0;
+      __nv_bfloat16* orow = (is_dk ? out_b : out_a) + grow * D + cc0;
+      const float* add = (!kDQ && !is_dk && dv_add) ? dv_add + grow * D + cc0 : nullptr;
 #pragma unroll 1
-      for (int cb = 0; cb < NCB; ++cb) {
+      for (int cb = 0; cb < (active ? OW / 32 : 0); ++cb) {
         uint32_t o[32];
         tmem_ld32(lane_addr + col + cb * 32, o);
         tmem_wait_ld();
