@@ -21,6 +21,9 @@ bounded samples of the same workload instead.
 `--op backward` measures gecko_sca_awm_backward on the same workload (the
 gradients of q, k, v, qm, km for N(0,1) output gradients); its roofline is
 the SCA dK/dV kernel against the bf16 tensor peak.
+`--op cp` runs the forward as context-parallel segments (--segments, every
+rank's phases emulated in one process on one GPU) and reports the whole-
+sequence forward of the same run beside it.
 `--op tdnorm` measures timestep decay normalisation on the same x shape
 (HBM roofline).  `--op cema` measures the CEMA recurrence (gecko_cema_forward) instead, on
 x [1, 32768, 4096] bf16 with h = 16, and prints its own JSON line (an FP32
@@ -806,6 +809,103 @@ def run_backward(args, ws: int, rank: int, local: int) -> dict:
     return out
 
 
+CP_METRIC = "tokens/s SCA+AWM fwd, sequence split into context-parallel segments (bf16,H=32,d=128,c=4096)"
+
+
+def run_cp(args, ws: int, rank: int, local: int) -> dict:
+    """Context parallelism on one GPU: the bench sequence is split into
+    --segments segments and every rank's phases (log-sums, cp log z, segment
+    maps, composed states, continued forwards) run in this process, so the
+    line measures the work context parallelism adds per rank.  The
+    whole-sequence forward is timed in the same run for comparison."""
+    from long_context_sequence_sca_b200 import cp
+    from long_context_sequence_sca_b200 import lib as L
+    L.load()
+    w = WORKLOADS[DEFAULT_WORKLOAD]
+    P = args.segments
+    if w.T % (P * w.c) != 0:
+        raise SystemExit(f"T={w.T} does not split into {P} segments of whole chunks (c={w.c})")
+    x = make_inputs(w, device="cuda", seed_offset=1000 * rank)
+    names = ("q", "k", "v", "qm", "km")
+    Tr = w.T // P
+    segs = [{n: x[n][:, :, r * Tr:(r + 1) * Tr].contiguous() for n in names} for r in range(P)]
+    stream = torch.cuda.current_stream()
+
+    def step():
+        cp.cp_forward_emulated(segs, w.c)
+
+    L.timing_enable(True)
+    ms_local, ck, note = time_steps(args, ws, local, step, stream)
+    stage_tot, n_calls = L.timing_read()
+    L.timing_enable(False)
+    # the library logs every segment forward (warm-up included): P per step
+    sca_ms = stage_tot["sca"] / max(n_calls / P, 1)
+
+    # what one rank does on its own GPU, phase by phase (no exchange time)
+    def timed(fn, reps=5):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    seg = segs[min(1, P - 1)]
+    lz = L.awm_segment_logsum(seg["km"], w.c)
+    lsum_all = torch.stack([L.awm_segment_logsum(sg["km"], w.c) for sg in segs])
+    maps_all = torch.stack([L.awm_segment_maps(sg["km"], sg["v"], L.awm_cp_logz(lsum_all, r), w.c)
+                            for r, sg in enumerate(segs)])
+    state = L.awm_cp_state(lsum_all, maps_all, 1)
+    halo = cp.halo_of(segs[0], w.c)
+    k1 = torch.cat([halo[0], seg["k"]], dim=2).contiguous()
+    v1 = torch.cat([halo[1], seg["v"]], dim=2).contiguous()
+    rank_phases = {
+        "segment_logsum": timed(lambda: L.awm_segment_logsum(seg["km"], w.c)),
+        "cp_logz": timed(lambda: L.awm_cp_logz(lsum_all, 1)),
+        "segment_maps": timed(lambda: L.awm_segment_maps(seg["km"], seg["v"], lz, w.c)),
+        "cp_state": timed(lambda: L.awm_cp_state(lsum_all, maps_all, 1)),
+        "continued_forward": timed(lambda: L.sca_awm_forward_segment(seg["q"], k1, v1, seg["qm"], seg["km"], w.c,
+                                                                     state_in=state)),
+    }
+
+    def whole():
+        L.sca_awm_forward(*(x[n] for n in names), w.c)
+
+    whole_ms, _, _ = time_steps(args, ws, local, whole, stream)
+    tokens = w.B * w.T
+    agg = aggregate(ms_local, tokens, ws)
+    f = flops(w)
+    pk, pk_kind = peaks()
+    achieved = f["sca"] / (max_over_ranks(sca_ms, ws) / 1e3) / 1e12
+    out = {
+        "metric": CP_METRIC, "value": round(agg["value"], 1), "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(agg["ms_per_step"], 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded Z'-affine generator; no dataset)",
+        "config": {"workload": f"{w.name}_cp{P}", "B": w.B, "H": w.H, "T": w.T, "d": w.d, "c": w.c,
+                   "segments": P, "ranks": f"{P} emulated on one GPU (exchanges are tensor indexing)",
+                   "l2": "inputs larger than L2 (1.34 GB), no flush",
+                   "parallelism": f"replicas x{ws}"},
+        "whole_sequence_ms": round(whole_ms, 4),
+        "cp_overhead_ms": round(ms_local - whole_ms, 4),
+        "one_rank_phase_ms": {k: round(v, 4) for k, v in rank_phases.items()},
+        "roofline": {"bound": "tensor", "kernel": "sca_tc_kernel (the P segment launches of a step)",
+                     "achieved": round(achieved, 2), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(achieved / pk["bf16_tflops"], 4), "peak_kind": f"{pk_kind} bf16 dense (burst)",
+                     "traffic": None, "launch_ms": round(sca_ms / P, 4),
+                     "algorithmic_flop_per_launch": f["sca"] // P},
+        "clocks": ck,
+        # per segment: log-sum 3, maps 7, cp log z 1, forward 7; cp state 2 for every segment but the first
+        "gpu_launches": (18 * P + 2 * (P - 1)) * args.steps,
+    }
+    if note:
+        out["note"] = note
+    return out
+
+
 def summarize_launches(path: str) -> str:
     """Per-kernel launches, total time and share from an ncu launch-list CSV
     (`ncu --metrics gpu__time_duration.sum --csv`)."""
@@ -845,9 +945,11 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=("sca_awm", "backward", "cema", "tdnorm"), default="sca_awm",
+    ap.add_argument("--op", choices=("sca_awm", "backward", "cp", "cema", "tdnorm"), default="sca_awm",
                     help="sca_awm: the fused SCA + AWM forward (default); backward: its gradients; "
+                         "cp: the forward as context-parallel segments (emulated ranks on one GPU); "
                          "cema: the CEMA recurrence; tdnorm: timestep decay normalisation")
+    ap.add_argument("--segments", type=int, default=4, help="segments of --op cp")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -865,7 +967,8 @@ def main(argv=None):
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE {ws}", file=sys.stderr)
     try:
         runner = {"cema": lambda: run_cema(args, ws, rank, local), "tdnorm": lambda: run_tdnorm(args, ws, rank, local),
-                  "backward": lambda: run_backward(args, ws, rank, local)}
+                  "backward": lambda: run_backward(args, ws, rank, local),
+                  "cp": lambda: run_cp(args, ws, rank, local)}
         out = runner[args.op]() if args.op in runner else run_gecko(args, w, ws, rank, local)
         if rank == 0:
             print(json.dumps(out), flush=True)

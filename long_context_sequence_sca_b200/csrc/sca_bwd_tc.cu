@@ -37,7 +37,10 @@ namespace gecko {
 namespace {
 
 constexpr int kRows = 128;          // rows per tile (keys or queries)
-constexpr int kEW = 4;                   // element-wise warpgroups
+#ifndef GECKO_BWD_EW
+#define GECKO_BWD_EW 4
+#endif
+constexpr int kEW = GECKO_BWD_EW;        // element-wise warpgroups
 constexpr int kCW = kRows / kEW;         // loop columns per warpgroup
 constexpr int kBwdThreads = 64 + 128 * kEW;
 static_assert(kCW % 32 == 0, "whole 32-column TMEM loads per warpgroup");
