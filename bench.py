@@ -602,10 +602,12 @@ def run_cema(args, ws: int, rank: int, local: int) -> dict:
 NORM_METRIC = "tokens/s timestep-decay norm fwd (bf16, D=4096, G=32, 32K tokens)"
 
 
-def time_steps(args, ws, local, step, stream):
+def time_steps(args, ws, local, step, stream, drain=None):
     """Warm up, then time args.steps calls of step() between CUDA events on
     `stream` (barriers and synchronisation on both sides), sampling clocks;
-    re-measure once if the clocks are rejected.  Returns (ms, clocks, note)."""
+    re-measure once if the clocks are rejected.  `drain` (e.g. a read of the
+    library's stage log) runs right before the timed region, so what it
+    discards is the warm-up.  Returns (ms, clocks, note)."""
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -614,6 +616,8 @@ def time_steps(args, ws, local, step, stream):
     def timed():
         barrier(ws)
         torch.cuda.synchronize()
+        if drain is not None:
+            drain()
         sampler.start()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -733,7 +737,7 @@ def run_backward(args, ws: int, rank: int, local: int) -> dict:
                                       stream=stream)
 
     L.timing_enable(True)
-    ms_local, ck, note = time_steps(args, ws, local, step, stream)
+    ms_local, ck, note = time_steps(args, ws, local, step, stream, drain=L.timing_read_backward)
     stage_tot, n_calls = L.timing_read_backward()
     L.timing_enable(False)
     stage_ms = {k: v / max(n_calls, 1) for k, v in stage_tot.items()}
@@ -835,10 +839,10 @@ def run_cp(args, ws: int, rank: int, local: int) -> dict:
         cp.cp_forward_emulated(segs, w.c)
 
     L.timing_enable(True)
-    ms_local, ck, note = time_steps(args, ws, local, step, stream)
+    ms_local, ck, note = time_steps(args, ws, local, step, stream, drain=L.timing_read)
     stage_tot, n_calls = L.timing_read()
     L.timing_enable(False)
-    # the library logs every segment forward (warm-up included): P per step
+    # the library logs every segment forward of the timed steps: P per step
     sca_ms = stage_tot["sca"] / max(n_calls / P, 1)
 
     # what one rank does on its own GPU, phase by phase (no exchange time)
