@@ -268,19 +268,29 @@ __global__ void __launch_bounds__(256) awm_bwd_e_simt_kernel(const TIn* __restri
 // Reverse carry, one slice of JC columns of G per CTA (columns evolve
 // independently):  G_s = E_{s+1} + r_s (.) G_{s+1} - Cm_s^T (rho_s (.) G_{s+1})
 // for 1-based s = S .. 2, G_{S+1} = 0.  Writes Gst[bh, s - 1] = G_s for
-// s = 1 .. S + 1 (G_1 is never read and is written as zero).  Cm_s is
-// staged into shared memory with its rows scaled by rho_s.  grid (D/JC, BH).
+// s = 1 .. S + 1 (G_1 is never read and is written as zero).  Everything the
+// next step reads from global memory (Cm_s, the CTA's slice of E_{s+1}, r_s,
+// rho_s) is copied into shared memory with 16-byte asynchronous copies while
+// this step computes (double buffer).  grid (D/JC, BH), 256 threads.
+template <int D, int JC>
+struct BwdCarryStage {
+  static constexpr int LD = D + 4;
+  static constexpr int kC = 0, kE = D * LD, kR = kE + D * JC, kP = kR + D;
+  static constexpr int kFloats = kP + D;
+};
+
 template <int D, int JC>
 __global__ void __launch_bounds__(256) awm_bwd_carry_kernel(const float* __restrict__ E, const float* __restrict__ Cm,
                                                             const float* __restrict__ ratio,
                                                             const float* __restrict__ rho, float* __restrict__ Gst,
                                                             int S) {
+  using St = BwdCarryStage<D, JC>;
   constexpr int PER = D * JC / 256;
-  static_assert(256 / (JC / PER) == D, "thread layout");
-  constexpr int LD = D + 4;
+  static_assert(PER >= 1 && 256 / (JC / PER) == D, "thread layout");
+  constexpr int LD = St::LD;
   extern __shared__ float smem_bc[];
-  float* Cs = smem_bc;      // [D][LD]  rho_s[g] * Cm_s[g][f]
-  float* Gs = Cs + D * LD;  // [D][JC]
+  float* Sb[2] = {smem_bc, smem_bc + St::kFloats};
+  float* Gs = smem_bc + 2 * St::kFloats;          // [D][JC]
   const int64_t bh = blockIdx.y;
   const int j0 = blockIdx.x * JC;
   const int tid = threadIdx.x;
@@ -288,41 +298,54 @@ __global__ void __launch_bounds__(256) awm_bwd_carry_kernel(const float* __restr
   const int jj = (tid % (JC / PER)) * PER;
   const int64_t mat = (int64_t)D * D;
   float* gout = Gst + bh * (int64_t)(S + 1) * mat;
+  // step k handles 1-based s = S - k (k = 0 .. S - 2), 0-based chunk z = s - 1
+  auto stage = [&](int k, float* dst) {
+    const int s = S - k, z = s - 1;
+    const float4* C4 = reinterpret_cast<const float4*>(Cm + (bh * S + z) * mat);
+    for (int i = tid; i < D * D / 4; i += 256) {
+      const int row = (i * 4) / D, col = (i * 4) % D;
+      cp_async16(dst + St::kC + row * LD + col, C4 + i);
+    }
+    if (s <= S - 1) {   // E_{s+1}: 0-based chunk s (none after the last chunk)
+      const float* Es = E + (bh * S + s) * mat + j0;
+      for (int i = tid; i < D * JC / 4; i += 256) {
+        const int row = (i * 4) / JC, col = (i * 4) % JC;
+        cp_async16(dst + St::kE + row * JC + col, Es + row * D + col);
+      }
+    }
+    for (int i = tid; i < D / 4; i += 256) {
+      cp_async16(dst + St::kR + 4 * i, ratio + (bh * S + z) * D + 4 * i);
+      cp_async16(dst + St::kP + 4 * i, rho + (bh * S + z) * D + 4 * i);
+    }
+    cp_async_commit();
+  };
+  const int steps = S - 1;   // s = S .. 2
+  if (steps > 0) stage(0, Sb[0]);
   for (int i = tid; i < D * JC; i += 256) Gs[i] = 0.f;
 #pragma unroll
   for (int j = 0; j < PER; ++j) {
     gout[(int64_t)S * mat + f * D + j0 + jj + j] = 0.f;  // G_{S+1}
     gout[f * D + j0 + jj + j] = 0.f;                     // G_1
   }
-  for (int s = S; s >= 2; --s) {
-    const int z = s - 1;  // 0-based chunk of r_s, rho_s, Cm_s
-    const float4* C4 = reinterpret_cast<const float4*>(Cm + (bh * S + z) * mat);
-    const float* rz = rho + (bh * S + z) * D;
-    __syncthreads();
-    for (int i = tid; i < D * D / 4; i += 256) {
-      const int row = (i * 4) / D, col = (i * 4) % D;
-      const float sc = rz[row];
-      float4 x = C4[i];
-      x.x *= sc;
-      x.y *= sc;
-      x.z *= sc;
-      x.w *= sc;
-      *reinterpret_cast<float4*>(Cs + row * LD + col) = x;
-    }
-    __syncthreads();
-    const float rf = ratio[(bh * S + z) * D + f];
-    float acc[PER];
-    if (s <= S - 1) {
-      const float* Ep = E + (bh * S + s) * mat + f * D + j0 + jj;  // E_{s+1}: 0-based chunk s
-#pragma unroll
-      for (int j = 0; j < PER; ++j) acc[j] = Ep[j];
+  for (int k = 0; k < steps; ++k) {
+    const int s = S - k;
+    const float* sb = Sb[k & 1];
+    if (k + 1 < steps) {
+      stage(k + 1, Sb[(k + 1) & 1]);
+      cp_async_wait<1>();
     } else {
-#pragma unroll
-      for (int j = 0; j < PER; ++j) acc[j] = 0.f;
+      cp_async_wait<0>();
     }
+    __syncthreads();
+    const float* Cs = sb + St::kC;
+    const float* rz = sb + St::kP;
+    const float rf = sb[St::kR + f];
+    float acc[PER];
+#pragma unroll
+    for (int j = 0; j < PER; ++j) acc[j] = s <= S - 1 ? sb[St::kE + f * JC + jj + j] : 0.f;
 #pragma unroll 4
     for (int g = 0; g < D; ++g) {
-      const float cgf = Cs[g * LD + f];
+      const float cgf = Cs[g * LD + f] * rz[g];
 #pragma unroll
       for (int j = 0; j < PER; ++j) acc[j] = fmaf(-cgf, Gs[g * JC + jj + j], acc[j]);
     }
@@ -601,6 +624,16 @@ cudaError_t sca_bwd_simt_impl(const BwdProblem& b, const BwdWorkspace& w, cudaSt
   return cudaGetLastError();
 }
 
+template <int D, int JC>
+cudaError_t bwd_carry_launch(const Workspace& fw, const BwdWorkspace& w, int64_t BH, int S, cudaStream_t st) {
+  const size_t smc = sizeof(float) * (2 * BwdCarryStage<D, JC>::kFloats + D * JC);
+  cudaError_t e = cudaFuncSetAttribute(awm_bwd_carry_kernel<D, JC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smc);
+  if (e != cudaSuccess) return e;
+  awm_bwd_carry_kernel<D, JC><<<dim3(D / JC, (unsigned)BH), 256, smc, st>>>(w.E, fw.Cm, fw.ratio, fw.rho, w.G, S);
+  return cudaGetLastError();
+}
+
 template <typename TIn, int D>
 cudaError_t awm_bwd_impl(const BwdProblem& b, const Workspace& fw, const BwdWorkspace& w, cudaStream_t st,
                          bool tc) {
@@ -614,12 +647,10 @@ cudaError_t awm_bwd_impl(const BwdProblem& b, const Workspace& fw, const BwdWork
     awm_bwd_e_simt_kernel<TIn, D><<<dim3(S, (unsigned)BH), 256, 0, st>>>(
         static_cast<const TIn*>(p.qm), static_cast<const TIn*>(b.dout_mem), w.E, p.T, (int)p.c);
   }
-  constexpr int JC = 16;
-  const size_t smc = sizeof(float) * (D * (D + 4) + D * JC);
-  cudaError_t e = cudaFuncSetAttribute(awm_bwd_carry_kernel<D, JC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smc);
+  cudaError_t e = carry_slice(BH, D) == 32 ? bwd_carry_launch<D, 32>(fw, w, BH, S, st)
+                  : carry_slice(BH, D) == 16 ? bwd_carry_launch<D, 16>(fw, w, BH, S, st)
+                                             : bwd_carry_launch<D, 8>(fw, w, BH, S, st);
   if (e != cudaSuccess) return e;
-  awm_bwd_carry_kernel<D, JC><<<dim3(D / JC, (unsigned)BH), 256, smc, st>>>(w.E, fw.Cm, fw.ratio, fw.rho, w.G, S);
   const int64_t nw = BH * D;
   awm_bwd_dl_kernel<D><<<(unsigned)((nw + 7) / 8), 256, 0, st>>>(w.G, fw.Mst, fw.ratio, fw.rho, w.dl, S, nw);
   const dim3 grid((unsigned)(p.c / 32), (unsigned)S, (unsigned)BH);

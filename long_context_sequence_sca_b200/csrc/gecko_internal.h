@@ -40,6 +40,15 @@ struct Workspace {
   float* Mst;    // [BH, S+1, d, d]  M'_1 .. M'_{S+1}
 };
 
+// Column slices of the sequential carries: as wide as still gives about one
+// CTA per SM (every CTA runs all S steps, so a second wave would double the
+// time).
+inline int carry_slice(int64_t BH, int D) {
+  for (int jc : {32, 16})
+    if (BH * (D / jc) >= 100) return jc;
+  return 8;
+}
+
 // Rows per block of the partial K_m statistics (divides c).
 inline int stats_block_rows(int64_t c) { return c % 128 == 0 ? 128 : 64; }
 

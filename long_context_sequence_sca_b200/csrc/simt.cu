@@ -234,8 +234,17 @@ __global__ void __launch_bounds__(256) awm_chunk_simt_kernel(const TIn* __restri
 // (row scales r_s = z^{s-1}/z^s and rho_s = e_s/z^s).  Writes
 // Mst[bh, s] = M'_{s+1} for s = 0..S.  M'_1 = 0 for a fresh sequence; a
 // continued one starts from the carried M' (M0, stride sd per (b, h)).
-// Cm_s is staged into shared memory with 16-byte loads.  grid (D / JC, BH),
-// 256 threads.
+// Everything step s + 1 reads from global memory (Cm, the CTA's slice of
+// Bm, r, rho) is copied into shared memory with 16-byte asynchronous copies
+// while step s computes (double buffer), so a step's critical path holds
+// only shared-memory reads and FMAs.  grid (D / JC, BH), 256 threads.
+template <int D, int JC>
+struct CarryStage {
+  static constexpr int LD = D + 4;   // padded row of Cm (keeps 16-byte alignment)
+  static constexpr int kC = 0, kB = D * LD, kR = kB + D * JC, kP = kR + D;
+  static constexpr int kFloats = kP + D;
+};
+
 template <int D, int JC>
 __global__ void __launch_bounds__(256) awm_carry_kernel(const float* __restrict__ Bm,
                                                         const float* __restrict__ Cm,
@@ -243,38 +252,58 @@ __global__ void __launch_bounds__(256) awm_carry_kernel(const float* __restrict_
                                                         const float* __restrict__ rho,
                                                         float* __restrict__ Mst, int S,
                                                         const float* __restrict__ M0, int64_t sd) {
+  using St = CarryStage<D, JC>;
   constexpr int PER = D * JC / 256;  // outputs per thread (one row f, PER columns)
-  static_assert(256 / (JC / PER) == D, "thread layout");
-  constexpr int LD = D + 4;          // padded row of Cm in shared memory (keeps 16-byte alignment)
+  static_assert(PER >= 1 && 256 / (JC / PER) == D, "thread layout");
+  constexpr int LD = St::LD;
   extern __shared__ float smem_carry[];
-  float* Cs = smem_carry;            // [D][LD]
-  float* Ms = Cs + D * LD;           // [D][JC]
+  float* Sb[2] = {smem_carry, smem_carry + St::kFloats};
+  float* Ms = smem_carry + 2 * St::kFloats;            // [D][JC]
   const int64_t bh = blockIdx.y;
   const int j0 = blockIdx.x * JC;
   const int tid = threadIdx.x;
   const int f = tid / (JC / PER);
   const int jj = (tid % (JC / PER)) * PER;
+  const int64_t mst_stride = (int64_t)D * D;
+  auto stage = [&](int s, float* dst) {
+    const float4* C4 = reinterpret_cast<const float4*>(Cm + (bh * S + s) * mst_stride);
+    for (int i = tid; i < D * D / 4; i += 256) {
+      const int row = (i * 4) / D, col = (i * 4) % D;
+      cp_async16(dst + St::kC + row * LD + col, C4 + i);
+    }
+    const float* Bs = Bm + (bh * S + s) * mst_stride + j0;
+    for (int i = tid; i < D * JC / 4; i += 256) {
+      const int row = (i * 4) / JC, col = (i * 4) % JC;
+      cp_async16(dst + St::kB + row * JC + col, Bs + row * D + col);
+    }
+    for (int i = tid; i < D / 4; i += 256) {
+      cp_async16(dst + St::kR + 4 * i, ratio + (bh * S + s) * D + 4 * i);
+      cp_async16(dst + St::kP + 4 * i, rho + (bh * S + s) * D + 4 * i);
+    }
+    cp_async_commit();
+  };
+  if (S > 0) stage(0, Sb[0]);
   for (int i = tid; i < D * JC; i += 256)
     Ms[i] = M0 ? M0[bh * sd + (i / JC) * D + j0 + i % JC] : 0.f;
-  const int64_t mst_stride = (int64_t)D * D;
   float* mout = Mst + bh * (int64_t)(S + 1) * mst_stride;
   __syncthreads();
 #pragma unroll
   for (int j = 0; j < PER; ++j) mout[f * D + j0 + jj + j] = Ms[f * JC + jj + j];   // M'_1
   for (int s = 0; s < S; ++s) {
-    const float4* C4 = reinterpret_cast<const float4*>(Cm + (bh * S + s) * mst_stride);
-    __syncthreads();
-    for (int i = tid; i < D * D / 4; i += 256) {
-      const int row = (i * 4) / D, col = (i * 4) % D;
-      *reinterpret_cast<float4*>(Cs + row * LD + col) = C4[i];
+    const float* sb = Sb[s & 1];
+    if (s + 1 < S) {
+      stage(s + 1, Sb[(s + 1) & 1]);   // its buffer was last read by step s - 1
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
     __syncthreads();
-    const float rf = ratio[(bh * S + s) * D + f];
-    const float pf = rho[(bh * S + s) * D + f];
-    const float* Bp = Bm + (bh * S + s) * mst_stride + f * D + j0 + jj;
+    const float* Cs = sb + St::kC;
+    const float rf = sb[St::kR + f];
+    const float pf = sb[St::kP + f];
     float acc[PER];
 #pragma unroll
-    for (int j = 0; j < PER; ++j) acc[j] = Bp[j];
+    for (int j = 0; j < PER; ++j) acc[j] = sb[St::kB + f * JC + jj + j];
 #pragma unroll 4
     for (int g = 0; g < D; ++g) {
       const float cfg = Cs[f * LD + g];
@@ -457,15 +486,21 @@ cudaError_t awm_chunk_simt_impl(const Problem& p, const Workspace& w, cudaStream
   return cudaGetLastError();
 }
 
-template <int D>
-cudaError_t awm_carry_impl(const Problem& p, const Workspace& w, cudaStream_t st) {
-  constexpr int JC = 16;
-  const size_t smem = sizeof(float) * (D * (D + 4) + D * JC);
+template <int D, int JC>
+cudaError_t awm_carry_launch(const Problem& p, const Workspace& w, cudaStream_t st) {
+  const size_t smem = sizeof(float) * (2 * CarryStage<D, JC>::kFloats + D * JC);
   cudaError_t e = cudaFuncSetAttribute(awm_carry_kernel<D, JC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   awm_carry_kernel<D, JC><<<dim3(D / JC, p.B * p.H), 256, smem, st>>>(
       w.Bm, w.Cm, w.ratio, w.rho, w.Mst, p.S, p.state0 ? p.state0 + D * D : nullptr, state_floats(D));
   return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t awm_carry_impl(const Problem& p, const Workspace& w, cudaStream_t st) {
+  const int jc = carry_slice(p.B * p.H, D);
+  return jc == 32 ? awm_carry_launch<D, 32>(p, w, st)
+                  : jc == 16 ? awm_carry_launch<D, 16>(p, w, st) : awm_carry_launch<D, 8>(p, w, st);
 }
 
 template <typename TIn, int D>
