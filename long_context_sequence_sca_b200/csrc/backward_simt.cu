@@ -289,7 +289,7 @@ __global__ void __launch_bounds__(256) awm_bwd_carry_kernel(const float* __restr
   static_assert(PER >= 1 && 256 / (JC / PER) == D, "thread layout");
   constexpr int LD = St::LD;
   extern __shared__ float smem_bc[];
-  float* Sb[2] = {smem_bc, smem_bc + St::kFloats};
+  // buffer b at smem_bc + b * St::kFloats (computed, so no pointer array in local memory)
   float* Gs = smem_bc + 2 * St::kFloats;          // [D][JC]
   const int64_t bh = blockIdx.y;
   const int j0 = blockIdx.x * JC;
@@ -320,7 +320,7 @@ __global__ void __launch_bounds__(256) awm_bwd_carry_kernel(const float* __restr
     cp_async_commit();
   };
   const int steps = S - 1;   // s = S .. 2
-  if (steps > 0) stage(0, Sb[0]);
+  if (steps > 0) stage(0, smem_bc);
   for (int i = tid; i < D * JC; i += 256) Gs[i] = 0.f;
 #pragma unroll
   for (int j = 0; j < PER; ++j) {
@@ -329,9 +329,9 @@ __global__ void __launch_bounds__(256) awm_bwd_carry_kernel(const float* __restr
   }
   for (int k = 0; k < steps; ++k) {
     const int s = S - k;
-    const float* sb = Sb[k & 1];
+    const float* sb = smem_bc + (k & 1) * St::kFloats;
     if (k + 1 < steps) {
-      stage(k + 1, Sb[(k + 1) & 1]);
+      stage(k + 1, smem_bc + ((k + 1) & 1) * St::kFloats);
       cp_async_wait<1>();
     } else {
       cp_async_wait<0>();
@@ -353,9 +353,15 @@ __global__ void __launch_bounds__(256) awm_bwd_carry_kernel(const float* __restr
     for (int j = 0; j < PER; ++j) acc[j] = fmaf(rf, Gs[f * JC + jj + j], acc[j]);
     __syncthreads();
 #pragma unroll
-    for (int j = 0; j < PER; ++j) {
-      Gs[f * JC + jj + j] = acc[j];
-      gout[(int64_t)(s - 1) * mat + f * D + j0 + jj + j] = acc[j];
+    for (int j = 0; j < PER; ++j) Gs[f * JC + jj + j] = acc[j];
+    float* dst = gout + (int64_t)(s - 1) * mat + f * D + j0 + jj;
+    if (PER % 4 == 0) {
+#pragma unroll
+      for (int j = 0; j < PER; j += 4)
+        *reinterpret_cast<float4*>(dst + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < PER; ++j) dst[j] = acc[j];
     }
   }
 }

@@ -257,7 +257,7 @@ __global__ void __launch_bounds__(256) awm_carry_kernel(const float* __restrict_
   static_assert(PER >= 1 && 256 / (JC / PER) == D, "thread layout");
   constexpr int LD = St::LD;
   extern __shared__ float smem_carry[];
-  float* Sb[2] = {smem_carry, smem_carry + St::kFloats};
+  // buffer b at smem_carry + b * St::kFloats (computed, so no pointer array in local memory)
   float* Ms = smem_carry + 2 * St::kFloats;            // [D][JC]
   const int64_t bh = blockIdx.y;
   const int j0 = blockIdx.x * JC;
@@ -282,7 +282,7 @@ __global__ void __launch_bounds__(256) awm_carry_kernel(const float* __restrict_
     }
     cp_async_commit();
   };
-  if (S > 0) stage(0, Sb[0]);
+  if (S > 0) stage(0, smem_carry);
   for (int i = tid; i < D * JC; i += 256)
     Ms[i] = M0 ? M0[bh * sd + (i / JC) * D + j0 + i % JC] : 0.f;
   float* mout = Mst + bh * (int64_t)(S + 1) * mst_stride;
@@ -290,9 +290,9 @@ __global__ void __launch_bounds__(256) awm_carry_kernel(const float* __restrict_
 #pragma unroll
   for (int j = 0; j < PER; ++j) mout[f * D + j0 + jj + j] = Ms[f * JC + jj + j];   // M'_1
   for (int s = 0; s < S; ++s) {
-    const float* sb = Sb[s & 1];
+    const float* sb = smem_carry + (s & 1) * St::kFloats;
     if (s + 1 < S) {
-      stage(s + 1, Sb[(s + 1) & 1]);   // its buffer was last read by step s - 1
+      stage(s + 1, smem_carry + ((s + 1) & 1) * St::kFloats);   // its buffer was last read by step s - 1
       cp_async_wait<1>();
     } else {
       cp_async_wait<0>();
@@ -314,9 +314,15 @@ __global__ void __launch_bounds__(256) awm_carry_kernel(const float* __restrict_
     for (int j = 0; j < PER; ++j) acc[j] = fmaf(rf, Ms[f * JC + jj + j], pf * acc[j]);
     __syncthreads();
 #pragma unroll
-    for (int j = 0; j < PER; ++j) {
-      Ms[f * JC + jj + j] = acc[j];
-      mout[(int64_t)(s + 1) * mst_stride + f * D + j0 + jj + j] = acc[j];
+    for (int j = 0; j < PER; ++j) Ms[f * JC + jj + j] = acc[j];
+    float* dst = mout + (int64_t)(s + 1) * mst_stride + f * D + j0 + jj;
+    if (PER % 4 == 0) {
+#pragma unroll
+      for (int j = 0; j < PER; j += 4)
+        *reinterpret_cast<float4*>(dst + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < PER; ++j) dst[j] = acc[j];
     }
   }
 }
