@@ -253,8 +253,11 @@ __global__ void __launch_bounds__(256) awm_carry_kernel(const float* __restrict_
                                                         float* __restrict__ Mst, int S,
                                                         const float* __restrict__ M0, int64_t sd) {
   using St = CarryStage<D, JC>;
-  constexpr int PER = D * JC / 256;  // outputs per thread (one row f, PER columns)
-  static_assert(PER >= 1 && 256 / (JC / PER) == D, "thread layout");
+  // each thread owns an RB x CB block of the slice: rows f0 .. f0 + RB - 1,
+  // columns c0 .. c0 + CB - 1 (8 column groups, D / RB row groups), so that
+  // four steps of the inner product cost RB + 4 shared loads for 4 RB CB FMAs
+  constexpr int CB = JC / 8, RB = D / 32;
+  static_assert(CB >= 1 && RB * CB * 256 == D * JC, "thread layout");
   constexpr int LD = St::LD;
   extern __shared__ float smem_carry[];
   // buffer b at smem_carry + b * St::kFloats (computed, so no pointer array in local memory)
@@ -262,8 +265,7 @@ __global__ void __launch_bounds__(256) awm_carry_kernel(const float* __restrict_
   const int64_t bh = blockIdx.y;
   const int j0 = blockIdx.x * JC;
   const int tid = threadIdx.x;
-  const int f = tid / (JC / PER);
-  const int jj = (tid % (JC / PER)) * PER;
+  const int f0 = (tid / 8) * RB, c0 = (tid % 8) * CB;
   const int64_t mst_stride = (int64_t)D * D;
   auto stage = [&](int s, float* dst) {
     const float4* C4 = reinterpret_cast<const float4*>(Cm + (bh * S + s) * mst_stride);
@@ -288,7 +290,9 @@ __global__ void __launch_bounds__(256) awm_carry_kernel(const float* __restrict_
   float* mout = Mst + bh * (int64_t)(S + 1) * mst_stride;
   __syncthreads();
 #pragma unroll
-  for (int j = 0; j < PER; ++j) mout[f * D + j0 + jj + j] = Ms[f * JC + jj + j];   // M'_1
+  for (int i = 0; i < RB; ++i)
+#pragma unroll
+    for (int j = 0; j < CB; ++j) mout[(f0 + i) * D + j0 + c0 + j] = Ms[(f0 + i) * JC + c0 + j];   // M'_1
   for (int s = 0; s < S; ++s) {
     const float* sb = smem_carry + (s & 1) * St::kFloats;
     if (s + 1 < S) {
@@ -299,30 +303,44 @@ __global__ void __launch_bounds__(256) awm_carry_kernel(const float* __restrict_
     }
     __syncthreads();
     const float* Cs = sb + St::kC;
-    const float rf = sb[St::kR + f];
-    const float pf = sb[St::kP + f];
-    float acc[PER];
+    float acc[RB][CB];
 #pragma unroll
-    for (int j = 0; j < PER; ++j) acc[j] = sb[St::kB + f * JC + jj + j];
-#pragma unroll 4
-    for (int g = 0; g < D; ++g) {
-      const float cfg = Cs[f * LD + g];
+    for (int i = 0; i < RB; ++i)
 #pragma unroll
-      for (int j = 0; j < PER; ++j) acc[j] = fmaf(-cfg, Ms[g * JC + jj + j], acc[j]);
+      for (int j = 0; j < CB; ++j) acc[i][j] = sb[St::kB + (f0 + i) * JC + c0 + j];
+#pragma unroll 2
+    for (int g = 0; g < D; g += 4) {
+      float4 cr[RB];
+#pragma unroll
+      for (int i = 0; i < RB; ++i) cr[i] = *reinterpret_cast<const float4*>(Cs + (f0 + i) * LD + g);
+#pragma unroll
+      for (int gg = 0; gg < 4; ++gg) {
+        float m[CB];
+#pragma unroll
+        for (int j = 0; j < CB; ++j) m[j] = Ms[(g + gg) * JC + c0 + j];
+#pragma unroll
+        for (int i = 0; i < RB; ++i) {
+          const float c = gg == 0 ? cr[i].x : gg == 1 ? cr[i].y : gg == 2 ? cr[i].z : cr[i].w;
+#pragma unroll
+          for (int j = 0; j < CB; ++j) acc[i][j] = fmaf(-c, m[j], acc[i][j]);
+        }
+      }
     }
 #pragma unroll
-    for (int j = 0; j < PER; ++j) acc[j] = fmaf(rf, Ms[f * JC + jj + j], pf * acc[j]);
+    for (int i = 0; i < RB; ++i) {
+      const float rf = sb[St::kR + f0 + i], pf = sb[St::kP + f0 + i];
+#pragma unroll
+      for (int j = 0; j < CB; ++j) acc[i][j] = fmaf(rf, Ms[(f0 + i) * JC + c0 + j], pf * acc[i][j]);
+    }
     __syncthreads();
 #pragma unroll
-    for (int j = 0; j < PER; ++j) Ms[f * JC + jj + j] = acc[j];
-    float* dst = mout + (int64_t)(s + 1) * mst_stride + f * D + j0 + jj;
-    if (PER % 4 == 0) {
+    for (int i = 0; i < RB; ++i) {
+      float* dst = mout + (int64_t)(s + 1) * mst_stride + (f0 + i) * D + j0 + c0;
 #pragma unroll
-      for (int j = 0; j < PER; j += 4)
-        *reinterpret_cast<float4*>(dst + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
-    } else {
-#pragma unroll
-      for (int j = 0; j < PER; ++j) dst[j] = acc[j];
+      for (int j = 0; j < CB; ++j) {
+        Ms[(f0 + i) * JC + c0 + j] = acc[i][j];
+        dst[j] = acc[i][j];
+      }
     }
   }
 }
