@@ -317,10 +317,14 @@ __global__ void __launch_bounds__(160, 1) awm_bwd_chunk_tc_kernel(
       const int64_t grow = row0 + (int64_t)kt * 128 + r;
 #pragma unroll 1
       for (int cb = 0; cb < D / 32; ++cb) {
-        uint32_t aR[32], aPhi[32], aPsi[32];
+        uint32_t aR[32], aPhi[32], aPsi[32], bPhi[16], bPsi[16];
         tmem_ld32(lane_addr + Cfg::kColR + cb * 32, aR);
         tmem_ld32(lane_addr + Cfg::kColPhiAcc + cb * 32, aPhi);
         tmem_ld32(lane_addr + Cfg::kColPsiAcc + cb * 32, aPsi);
+        // Phi and Psi of this row as the MMAs used them (bf16): here they only
+        // scale terms, so their rounding stays at the output's resolution
+        tmem_ld16p(lane_addr + Cfg::kColPhi + cb * 16, bPhi);
+        tmem_ld16p(lane_addr + Cfg::kColPsi + cb * 16, bPsi);
         tmem_wait_ld();
         float4* dvp = reinterpret_cast<float4*>(dv_awm + grow * D + cb * 32);
 #pragma unroll
@@ -331,13 +335,13 @@ __global__ void __launch_bounds__(160, 1) awm_bwd_chunk_tc_kernel(
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
           const int col = cb * 32 + 2 * q;
-          const float2 x = xval(col);
+          const float2 phi2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bPhi[q]));
+          const float2 psi2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bPsi[q]));
           float res[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const float xv = e ? x.y : x.x;
-            const float phi = ex2(fmaf(xv, kLog2e, -vL2[col + e]));
-            const float psi = ex2(fmaf(xv, kLog2e, -mx2)) * inv;
+            const float phi = e ? phi2.y : phi2.x;
+            const float psi = e ? psi2.y : psi2.x;
             res[e] = __uint_as_float(aPhi[2 * q + e]) * phi + psi * (__uint_as_float(aPsi[2 * q + e]) - dot) +
                      vDl[col + e] * phi * vInvRho[col + e];
           }

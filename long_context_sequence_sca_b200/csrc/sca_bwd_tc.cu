@@ -37,13 +37,20 @@ namespace gecko {
 namespace {
 
 constexpr int kRows = 128;          // rows per tile (keys or queries)
+// Element-wise warpgroups per kernel (measured: 4 for dK/dV, 2 for dQ).
 #ifndef GECKO_BWD_EW
 #define GECKO_BWD_EW 4
 #endif
-constexpr int kEW = GECKO_BWD_EW;        // element-wise warpgroups
-constexpr int kCW = kRows / kEW;         // loop columns per warpgroup
-constexpr int kBwdThreads = 64 + 128 * kEW;
-static_assert(kCW % 32 == 0, "whole 32-column TMEM loads per warpgroup");
+#ifndef GECKO_BWD_EW_DQ
+#define GECKO_BWD_EW_DQ 2
+#endif
+template <bool kDQ>
+struct EwLayout {
+  static constexpr int n = kDQ ? GECKO_BWD_EW_DQ : GECKO_BWD_EW;   // warpgroups
+  static constexpr int cw = kRows / n;                             // loop columns per warpgroup
+  static constexpr int threads = 64 + 128 * n;
+  static_assert(cw % 32 == 0, "whole 32-column TMEM loads per warpgroup");
+};
 // Of every 8 exponential pairs of P, GECKO_BWD_SFU_PAIRS go to the SFU and the
 // rest to the FMA pipe (exp2_poly2).  Measured on B200 (bench workload):
 // 8/8 on the SFU is fastest (dK/dV 5.80 ms against 7.06 ms at 6/8, where the
@@ -109,7 +116,7 @@ __device__ __forceinline__ BwdTile bwd_tile(int bid, int T, int c, bool dq) {
 }
 
 template <int D, bool kDQ>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(EwLayout<kDQ>::threads, 1)
 sca_bwd_tc_kernel(const __grid_constant__ CUtensorMap map_fix0, const __grid_constant__ CUtensorMap map_fix1,
                   const __grid_constant__ CUtensorMap map_st0, const __grid_constant__ CUtensorMap map_st1,
                   const float* __restrict__ nlse2, const float* __restrict__ delta,
@@ -117,6 +124,7 @@ sca_bwd_tc_kernel(const __grid_constant__ CUtensorMap map_fix0, const __grid_con
                   __nv_bfloat16* __restrict__ out_b, int T, int c, int* status) {
   using Cfg = BwdCfg<D>;
   constexpr int NS = Cfg::kStages;
+  constexpr int kEW = EwLayout<kDQ>::n, kCW = EwLayout<kDQ>::cw;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sFix = smem + Cfg::kFixOff;
@@ -414,7 +422,7 @@ sca_bwd_tc_kernel(const __grid_constant__ CUtensorMap map_fix0, const __grid_con
       // dK/dV: the 2D output columns of a row (dV, with the AWM part added,
       // then dK) split evenly over the warpgroups; dQ: 32 columns per
       // warpgroup (those past D have none).  `active` is warp-uniform.
-      constexpr int OW = kDQ ? 32 : 2 * D / kEW;
+      constexpr int OW = kDQ ? (D / kEW > 32 ? D / kEW : 32) : 2 * D / kEW;
       static_assert(OW % 32 == 0, "whole 32-column TMEM loads in the epilogue");
       const int c0 = w * OW;
       const bool active = !kDQ || c0 < D;
@@ -512,11 +520,11 @@ cudaError_t launch_sca_bwd_tc_impl(const BwdProblem& b, const BwdWorkspace& w, c
     return e;
   if (part == 0)
     // dK, dV (the AWM part of dV is added in the epilogue)
-    sca_bwd_tc_kernel<D, false><<<grid, kBwdThreads, Cfg::kAlloc, st>>>(
+    sca_bwd_tc_kernel<D, false><<<grid, EwLayout<false>::threads, Cfg::kAlloc, st>>>(
         mk, mv, mq, mdo, w.nlse2, w.delta, w.dv_awm, static_cast<__nv_bfloat16*>(b.dv),
         static_cast<__nv_bfloat16*>(b.dk), T, c, p.status);
   else
-    sca_bwd_tc_kernel<D, true><<<grid, kBwdThreads, Cfg::kAlloc, st>>>(
+    sca_bwd_tc_kernel<D, true><<<grid, EwLayout<true>::threads, Cfg::kAlloc, st>>>(
         mq, mdo, mk, mv, w.nlse2, w.delta, nullptr, static_cast<__nv_bfloat16*>(b.dq), nullptr, T, c, p.status);
   return cudaGetLastError();
 }
