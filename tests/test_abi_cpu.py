@@ -139,3 +139,21 @@ def test_train_forward_rejects_bad_lse(so):
     assert L.gecko_sca_awm_forward_train(*[FAKE] * 7, 0, 0, 1, 1, 256, 128, 64, 1, None) == 1
     assert L.gecko_sca_awm_forward_train(*[FAKE] * 7, FAKE + 4, 0, 1, 1, 256, 128, 64, 1, None) == 3
     assert L.gecko_sca_awm_forward_train(*[FAKE] * 7, FAKE, FAKE + 8, 1, 1, 256, 128, 64, 1, None) == 3
+
+
+@pytest.mark.parametrize("call,code", [
+    (lambda: L.gecko_awm_segment_logsum(0, FAKE, 1, 1, 256, 128, 64, 1, None), 1),
+    (lambda: L.gecko_awm_segment_logsum(FAKE, FAKE, 1, 1, 300, 128, 64, 1, None), 2),
+    (lambda: L.gecko_awm_segment_maps(FAKE, FAKE, 0, FAKE, 1, 1, 256, 128, 64, 1, None), 1),
+    (lambda: L.gecko_awm_segment_maps(FAKE, FAKE, FAKE, FAKE + 4, 1, 1, 256, 128, 64, 1, None), 3),
+    (lambda: L.gecko_awm_cp_logz(0, 2, 0, FAKE, 1, 1, 64, None), 1),
+    (lambda: L.gecko_awm_cp_logz(FAKE, 2, 2, FAKE, 1, 1, 64, None), 1),
+    (lambda: L.gecko_awm_cp_logz(FAKE, 2, 1, FAKE, 1, 1, 96, None), 2),
+    (lambda: L.gecko_awm_cp_state(FAKE, FAKE, 3, -1, FAKE, 1, 1, 64, None), 1),
+    (lambda: L.gecko_awm_cp_state(FAKE, FAKE + 4, 3, 1, FAKE, 1, 1, 64, None), 3),
+    (lambda: L.gecko_awm_cp_state(FAKE, FAKE, 0, 0, FAKE, 1, 1, 64, None), 1),
+], ids=["logsum-null", "logsum-shape", "maps-null", "maps-align", "logz-null", "logz-rank", "logz-d",
+        "state-rank", "state-align", "state-P"])
+def test_context_parallel_host_validation_rejects(so, call, code):
+    assert call() == code
+    assert L.gecko_last_error()
