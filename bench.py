@@ -83,6 +83,30 @@ def io_bytes(w: Workload) -> int:
     return 7 * w.B * w.H * w.T * w.d * esz
 
 
+# exp2 results per clock per SM of the special-function units (the public
+# arithmetic-throughput table's figure for compute capability 10.0)
+SFU_EXP_PER_CLK_SM = 16
+N_SM = 148
+
+
+def secondary_rooflines(w: Workload, ms_per_step: float, sca_ms: float, sm_mhz, hbm_gbs: float) -> dict:
+    """The two other bounds of the forward: the step's algorithmic HBM bytes
+    over its time against the measured copy bandwidth, and the SCA kernel's
+    exponentials (one per visible (query, key) pair) over its launch time
+    against the SFU issue rate at the sampled SM clock."""
+    gbs = io_bytes(w) / (ms_per_step / 1e3) / 1e9
+    exps = sca_pairs(w) * w.B * w.H
+    out = {"hbm": {"algorithmic_bytes_per_step": io_bytes(w), "achieved_gbs": round(gbs, 1),
+                   "peak_gbs": hbm_gbs, "frac": round(gbs / hbm_gbs, 4)}}
+    if sm_mhz:
+        g_exp = exps / (sca_ms / 1e3) / 1e9
+        peak = SFU_EXP_PER_CLK_SM * N_SM * sm_mhz / 1e3
+        out["sfu"] = {"kernel": "sca_tc_kernel", "exps_per_launch": exps, "achieved_gexp_s": round(g_exp, 1),
+                      "peak_gexp_s": round(peak, 1), "frac": round(g_exp / peak, 4),
+                      "clock": f"{sm_mhz} MHz (sampled)"}
+    return out
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -380,6 +404,7 @@ def run_gecko(args, w: Workload, ws: int, rank: int, local: int) -> dict:
         "pct_bf16_peak": round(100 * fl["total"] / (agg["ms_per_step"] / 1e3) / 1e12 / pk["bf16_tflops"], 2),
         "stage_ms": {k_: round(v_, 4) for k_, v_ in stages.items()},
         "roofline": roofline,
+        "other_bounds": secondary_rooflines(w, agg["ms_per_step"], sca_ms, ck.get("sm_mhz"), pk["hbm_gbs"]),
         "clocks": ck,
         "gpu_launches": 7 * args.steps,  # lse partial, lse combine, prefix, chunk, carry, readout, sca
     }

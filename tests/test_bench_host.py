@@ -27,6 +27,19 @@ def test_flops_and_bytes_headline():
     assert bench.io_bytes(w) == 7 * 32 * 32768 * 128 * 2
 
 
+def test_secondary_rooflines_at_the_bench_workload():
+    """HBM and SFU bounds: 1.88 GB in 3.44 ms is 546 GB/s; 5.91e9
+    exponentials in 2.97 ms at 1965 MHz against 16 per clock on 148 SMs
+    (4653 G/s) is 0.43 of the SFU rate."""
+    w = bench.WORKLOADS["bf16_h32_c4096"]
+    r = bench.secondary_rooflines(w, 3.44, 2.97, 1965, 6545.3)
+    assert abs(r["hbm"]["achieved_gbs"] - 7 * 32 * 32768 * 128 * 2 / 3.44e-3 / 1e9) < 0.1
+    assert r["sfu"]["exps_per_launch"] == 32 * (8 * 4096 * 4097 // 2 + 7 * 4096 * 4096)
+    assert abs(r["sfu"]["peak_gexp_s"] - 16 * 148 * 1.965) < 0.1
+    assert 0.42 < r["sfu"]["frac"] < 0.44
+    assert "sfu" not in bench.secondary_rooflines(w, 3.44, 2.97, None, 6545.3)
+
+
 def _free_port():
     s = socket.socket()
     s.bind(("127.0.0.1", 0))
