@@ -220,7 +220,9 @@ int gecko_sca_awm_forward_noalloc(const void* q, const void* k, const void* v,
  * after the copy has completed.  Returns GECKO_ERR_NO_STATE if no forward
  * ran on this device, GECKO_ERR_ARG if B, H, d differ from that forward,
  * and GECKO_ERR_TIMEOUT if a kernel of that forward reported a timed-out
- * wait.
+ * wait.  A gecko_sca_awm_backward call rebuilds the same state and counts as
+ * such a forward; gecko_awm_segment_logsum and gecko_awm_segment_maps
+ * invalidate it (GECKO_ERR_NO_STATE).
  */
 int gecko_awm_state(float* M_out, float* logz_out,
                     int64_t B, int64_t H, int64_t d, void* stream);
@@ -335,6 +337,9 @@ int gecko_tdnorm_forward(const void* x, void* y, const float* gamma, const float
  *      gecko_sca_awm_forward_continue with k, v prefixed by the previous
  *      segment's last c rows (rank 0: a fresh gecko_sca_awm_forward).
  * All buffers are device memory, fp32 unless stated, 16-byte aligned.
+ * gecko_awm_segment_logsum and gecko_awm_segment_maps work in the forward's
+ * per-device workspace: after either, gecko_awm_state returns
+ * GECKO_ERR_NO_STATE until the next gecko_sca_awm_forward(_continue).
  */
 /* lsum_out [B,H,d]: log sum over the segment's tokens of exp(km) per feature.
  * km [B,H,T,d] dtype.  Same size rules and errors as the forward. */

@@ -273,6 +273,7 @@ int run_forward(const void* q, const void* k, const void* v, const void* qm, con
   const int64_t BH = B * H;
   const int64_t sd = state_floats(d);
   if (env_is("GECKO_FAIL_ALLOC", "1")) return fail(GECKO_ERR_ALLOC, "workspace allocation failed (injected)");
+  ds->have_state = false;  // set again once this forward is enqueued
   if ((rc = ensure_buffer(&ds->ws, &ds->ws_bytes, workspace_bytes(BH, T, c, d), st, "workspace"))) return rc;
   Workspace w = carve_workspace(ds->ws, BH, T, c, d);
 
@@ -353,6 +354,7 @@ int run_backward(const void* q, const void* k, const void* v, const void* qm, co
   if ((rc = device_state(dev, &ds))) return rc;
   const int64_t S = T / c;
   const int64_t BH = B * H;
+  ds->have_state = false;  // set again once the rebuild is enqueued
   if ((rc = ensure_buffer(&ds->ws, &ds->ws_bytes, workspace_bytes(BH, T, c, d), st, "workspace"))) return rc;
   if ((rc = ensure_buffer(&ds->bwd_ws, &ds->bwd_ws_bytes, bwd_workspace_bytes(BH, T, c, d), st,
                           "backward workspace")))
@@ -435,6 +437,7 @@ extern "C" int gecko_awm_segment_logsum(const void* km, float* lsum_out, int64_t
   DeviceState* ds = nullptr;
   if ((rc = device_state(dev, &ds))) return rc;
   const int64_t S = T / c, BH = B * H;
+  ds->have_state = false;  // the forward's workspace is overwritten below
   if ((rc = ensure_buffer(&ds->ws, &ds->ws_bytes, workspace_bytes(BH, T, c, d), st, "workspace"))) return rc;
   Workspace w = carve_workspace(ds->ws, BH, T, c, d);
   Problem p{nullptr, nullptr, nullptr, nullptr, km, nullptr, nullptr, B, H, T, c, d, (int)S, dtype, ds->status};
@@ -459,6 +462,7 @@ extern "C" int gecko_awm_segment_maps(const void* km, const void* v, const float
   DeviceState* ds = nullptr;
   if ((rc = device_state(dev, &ds))) return rc;
   const int64_t S = T / c, BH = B * H, sd = state_floats(d), mat = d * d;
+  ds->have_state = false;  // the forward's workspace is overwritten below
   if ((rc = ensure_buffer(&ds->ws, &ds->ws_bytes, workspace_bytes(BH, T, c, d), st, "workspace"))) return rc;
   if ((rc = ensure_buffer(&ds->state, &ds->state_bytes, sizeof(float) * BH * sd, st, "state"))) return rc;
   Workspace w = carve_workspace(ds->ws, BH, T, c, d);
@@ -541,7 +545,7 @@ extern "C" int gecko_awm_state(float* M_out, float* logz_out, int64_t B, int64_t
   if ((rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice"))) return rc;
   std::lock_guard<std::mutex> lk(g_mu);
   auto it = g_dev.find(dev);
-  if (it == g_dev.end() || !it->second.have_state)
+  if (it == g_dev.end() || !it->second.have_state || !it->second.ws)
     return fail(GECKO_ERR_NO_STATE, "no forward has run on device %d", dev);
   DeviceState& ds = it->second;
   if (B != ds.B || H != ds.H || d != ds.d)

@@ -79,3 +79,21 @@ def test_segment_maps_reproduce_the_continued_state(L):
     got_prev = maps[:, :, 2] @ M_in + maps[:, :, 3]
     assert torch.allclose(got_out, want_out, atol=1e-5, rtol=1e-4)
     assert torch.allclose(got_prev, want_prev, atol=1e-5, rtol=1e-4)
+
+
+def test_segment_calls_invalidate_the_reported_state(L):
+    """The segment calls work in the forward's workspace, so afterwards
+    gecko_awm_state reports no state until the next forward."""
+    w = Workload("cp_state_invalidated", 84, "f32", 1, 2, 256, 64, 64)
+    x = make_inputs(w, device="cuda")
+    L.sca_awm_forward(*(x[n] for n in NAMES), w.c)
+    L.awm_state(w.B, w.H, w.d)
+    L.awm_segment_logsum(x["km"], w.c)
+    with pytest.raises(L.GeckoError) as e:
+        L.awm_state(w.B, w.H, w.d)
+    assert e.value.code == 6
+    L.sca_awm_forward(*(x[n] for n in NAMES), w.c)
+    M, _ = L.awm_state(w.B, w.H, w.d)
+    torch.cuda.synchronize()
+    want = F.forward(*(x[n].double().cpu().numpy() for n in NAMES), w.c)
+    assert float(np.abs(M.double().cpu().numpy() - want[2]).max()) <= 1e-4
