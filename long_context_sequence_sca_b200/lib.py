@@ -231,6 +231,7 @@ def sca_awm_forward(q, k, v, qm, km, c: int, out_sca=None, out_mem=None, stream=
     if q.dim() != 4 or q.dtype not in _DT:
         raise ValueError("inputs must be [B, H, T, d] float32 or bfloat16")
     B, H, T, d = q.shape
+    _check_outputs((out_sca, out_mem), q)
     if out_sca is None:
         out_sca = torch.empty_like(q)
     if out_mem is None:
@@ -240,6 +241,19 @@ def sca_awm_forward(q, k, v, qm, km, c: int, out_sca=None, out_mem=None, stream=
                                    B, H, T, c, d, _DT[q.dtype], _stream_handle(stream))
     _check(rc)
     return out_sca, out_mem
+
+
+def _check_outputs(outs, like):
+    """Caller-given output buffers must be what the kernels write: the
+    inputs' shape, dtype and device, contiguous (a smaller buffer would be
+    written past its end)."""
+    for o in outs:
+        if o is None:
+            continue
+        if not (isinstance(o, torch.Tensor) and o.is_contiguous() and o.shape == like.shape
+                and o.dtype == like.dtype and o.device == like.device):
+            raise ValueError(f"output buffers must be contiguous {tuple(like.shape)} {like.dtype} "
+                             f"tensors on {like.device}")
 
 
 def _check_inputs(xs):
@@ -325,6 +339,14 @@ def sca_awm_forward_segment(q, k, v, qm, km, c: int, state_in=None, out_sca=None
     kv_rows = T + (c if state_in is not None else 0)
     if tuple(k.shape) != (B, H, kv_rows, d) or tuple(v.shape) != (B, H, kv_rows, d):
         raise ValueError(f"k and v must be [B, H, {kv_rows}, d]")
+    if qm.shape != q.shape or km.shape != q.shape or q.dim() != 4 or q.dtype not in _DT \
+            or any(x.device != q.device for x in xs):
+        raise ValueError("q, qm, km must be [B, H, T, d] float32 or bfloat16 tensors on one device")
+    if state_in is not None and not (isinstance(state_in, torch.Tensor) and state_in.is_contiguous()
+                                     and state_in.dtype == torch.float32
+                                     and tuple(state_in.shape) == (B, H, 2 * d * d + d)):
+        raise ValueError(f"state_in must be a contiguous [B, H, {2 * d * d + d}] float32 tensor")
+    _check_outputs((out_sca, out_mem), q)
     if out_sca is None:
         out_sca = torch.empty_like(q)
     if out_mem is None:
@@ -391,6 +413,18 @@ def cema_forward(x, alpha, delta, theta, beta, eta, reset=None, state_in=None, r
         if not (isinstance(prm, torch.Tensor) and prm.is_cuda and prm.is_contiguous() and prm.dtype == torch.float32):
             raise ValueError("parameters must be contiguous float32 CUDA tensors")
     h = alpha.shape[-1]
+    for prm, shape in zip(params, ((D, h),) * 4 + ((D, h, 2),)):
+        if tuple(prm.shape) != shape or prm.device != x.device:
+            raise ValueError(f"CEMA parameters must be [D, h] (eta [D, h, 2]) on {x.device}; got {tuple(prm.shape)}")
+    if reset is not None and not (isinstance(reset, torch.Tensor) and reset.dtype == torch.uint8
+                                  and tuple(reset.shape) == (B, L) and reset.is_contiguous()
+                                  and reset.device == x.device):
+        raise ValueError(f"reset must be a contiguous [B, L] uint8 tensor on {x.device}")
+    if state_in is not None and not (isinstance(state_in, torch.Tensor) and state_in.dtype == torch.float32
+                                     and tuple(state_in.shape) == (B, D, h, 2) and state_in.is_contiguous()
+                                     and state_in.device == x.device):
+        raise ValueError(f"state_in must be a contiguous [B, D, h, 2] float32 tensor on {x.device}")
+    _check_outputs((y,), x)
     if y is None:
         y = torch.empty_like(x)
     state_out = torch.empty(B, D, h, 2, dtype=torch.float32, device=x.device) if return_state else None
@@ -411,6 +445,9 @@ def tdnorm_forward(x, gamma, bias, G: int, beta1: float, beta2: float, eps: floa
         if not (isinstance(prm, torch.Tensor) and prm.is_cuda and prm.is_contiguous() and prm.dtype == torch.float32):
             raise ValueError("gamma and bias must be contiguous float32 CUDA tensors")
     B, L, D = x.shape
+    if gamma.shape != (D,) or bias.shape != (D,) or gamma.device != x.device or bias.device != x.device:
+        raise ValueError(f"gamma and bias must be [D] = [{D}] on {x.device}")
+    _check_outputs((y,), x)
     if y is None:
         y = torch.empty_like(x)
     with torch.cuda.device(x.device):
@@ -434,14 +471,24 @@ def awm_segment_logsum(km, c: int, stream=None):
     return out
 
 
+def _f32_on(t, shape, device, name):
+    """t as a contiguous fp32 tensor of `shape` on `device` (the caller keeps
+    the returned tensor alive until the call is enqueued)."""
+    if not (isinstance(t, torch.Tensor) and t.dtype == torch.float32 and tuple(t.shape) == tuple(shape)
+            and t.device == device):
+        raise ValueError(f"{name} must be a float32 tensor of shape {tuple(shape)} on {device}")
+    return t.contiguous()
+
+
 def awm_segment_maps(km, v, logz_in, c: int, stream=None):
     """[B, H, 4, d, d] fp32 maps (A, b, A', b') of the segment for the log z
     entering it (logz_in [B, H, d] fp32)."""
     _check_inputs((km, v))
     B, H, T, d = km.shape
+    lz = _f32_on(logz_in, (B, H, d), km.device, "logz_in")
     out = torch.empty((B, H, 4, d, d), dtype=torch.float32, device=km.device)
     with torch.cuda.device(km.device):
-        rc = gecko_awm_segment_maps(km.data_ptr(), v.data_ptr(), logz_in.contiguous().data_ptr(), out.data_ptr(),
+        rc = gecko_awm_segment_maps(km.data_ptr(), v.data_ptr(), lz.data_ptr(), out.data_ptr(),
                                     B, H, T, c, d, _DT[km.dtype], _stream_handle(stream))
     _check(rc)
     return out
@@ -450,10 +497,10 @@ def awm_segment_maps(km, v, logz_in, c: int, stream=None):
 def awm_cp_logz(lsum_all, rank: int, stream=None):
     """log z entering segment `rank` from every rank's log-sum [P, B, H, d]."""
     P, B, H, d = lsum_all.shape
+    ls = _f32_on(lsum_all, (P, B, H, d), lsum_all.device, "lsum_all")
     out = torch.empty((B, H, d), dtype=torch.float32, device=lsum_all.device)
     with torch.cuda.device(lsum_all.device):
-        rc = gecko_awm_cp_logz(lsum_all.contiguous().data_ptr(), P, rank, out.data_ptr(), B, H, d,
-                               _stream_handle(stream))
+        rc = gecko_awm_cp_logz(ls.data_ptr(), P, rank, out.data_ptr(), B, H, d, _stream_handle(stream))
     _check(rc)
     return out
 
@@ -461,10 +508,12 @@ def awm_cp_logz(lsum_all, rank: int, stream=None):
 def awm_cp_state(lsum_all, maps_all, rank: int, stream=None):
     """state_in [B, H, 2 d^2 + d] of segment `rank` (M'_prev, M'_in, log z)."""
     P, B, H, d = lsum_all.shape
+    ls = _f32_on(lsum_all, (P, B, H, d), lsum_all.device, "lsum_all")
+    mp = _f32_on(maps_all, (P, B, H, 4, d, d), lsum_all.device, "maps_all")
     out = torch.empty((B, H, 2 * d * d + d), dtype=torch.float32, device=lsum_all.device)
     with torch.cuda.device(lsum_all.device):
-        rc = gecko_awm_cp_state(lsum_all.contiguous().data_ptr(), maps_all.contiguous().data_ptr(), P, rank,
-                                out.data_ptr(), B, H, d, _stream_handle(stream))
+        rc = gecko_awm_cp_state(ls.data_ptr(), mp.data_ptr(), P, rank, out.data_ptr(), B, H, d,
+                                _stream_handle(stream))
     _check(rc)
     return out
 

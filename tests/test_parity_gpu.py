@@ -154,6 +154,25 @@ def test_state_shape_mismatch_and_release(L):
     assert e.value.code == 6
 
 
+def test_binding_rejects_mismatched_buffers(L):
+    """The binding checks caller-given buffers before the C call: an output
+    one row short, an output of another dtype, a state of the wrong size."""
+    w = SMALL["bf16_one_chunk"]
+    x = make_inputs(w, device="cuda")
+    xs = [x[n] for n in ("q", "k", "v", "qm", "km")]
+    short = torch.empty(w.B, w.H, w.T - 1, w.d, dtype=x["q"].dtype, device="cuda")
+    with pytest.raises(ValueError):
+        L.sca_awm_forward(*xs, w.c, out_sca=short)
+    with pytest.raises(ValueError):
+        L.sca_awm_forward(*xs, w.c, out_mem=torch.empty_like(x["q"], dtype=torch.float32))
+    bad_state = torch.zeros(w.B, w.H, 2 * w.d * w.d, dtype=torch.float32, device="cuda")
+    kv = [torch.cat([x[n][:, :, :w.c], x[n]], dim=2).contiguous() for n in ("k", "v")]
+    with pytest.raises(ValueError):
+        L.sca_awm_forward_segment(x["q"], kv[0], kv[1], x["qm"], x["km"], w.c, state_in=bad_state)
+    with pytest.raises(ValueError):
+        L.awm_segment_maps(x["km"], x["v"], torch.zeros(w.B, w.H, w.d, dtype=torch.float64, device="cuda"), w.c)
+
+
 def test_injected_allocation_failure(L, monkeypatch):
     L.release()
     w = SMALL["bf16_one_chunk"]
