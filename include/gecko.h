@@ -70,7 +70,9 @@ extern "C" {
  *                     fully overwritten.  They must not alias an input.
  *   B, H, T, c, d   : batch, heads, tokens, chunk size, head dim.
  *                     Requires B, H, T >= 1, c >= 64, c % 64 == 0,
- *                     T % c == 0, d in {64, 128}.
+ *                     T % c == 0, d in {64, 128}, B * H <= 65535,
+ *                     T / c <= 65535 and T < 2^31 - 256 (else
+ *                     GECKO_ERR_SHAPE).
  *   dtype           : GECKO_F32 or GECKO_BF16.
  *   stream          : cudaStream_t used for every launch and copy.
  *

@@ -119,6 +119,8 @@ int device_state(int dev, DeviceState** out) {
   return GECKO_OK;
 }
 
+constexpr int64_t kMaxGridYZ = 65535;
+
 int validate(const void* const* ptrs, int n, int64_t B, int64_t H, int64_t T, int64_t c, int64_t d, int dtype) {
   for (int i = 0; i < n; ++i)
     if (!ptrs[i]) return fail(GECKO_ERR_ARG, "tensor argument %d is NULL", i);
@@ -129,12 +131,15 @@ int validate(const void* const* ptrs, int n, int64_t B, int64_t H, int64_t T, in
   if (d != 64 && d != 128) return fail(GECKO_ERR_SHAPE, "d must be 64 or 128 (got %lld)", (long long)d);
   if (c % 64 != 0) return fail(GECKO_ERR_SHAPE, "c must be a multiple of 64 (got %lld)", (long long)c);
   if (T % c != 0) return fail(GECKO_ERR_SHAPE, "T %% c != 0 (T=%lld c=%lld)", (long long)T, (long long)c);
-  // element count and byte size must fit comfortably in int64; chunk and
-  // grid indices must fit the 32-bit ranges the kernels use
+  // element count and byte size must fit comfortably in int64; token
+  // indices must fit the 32-bit ranges the kernels use, and (b, h) pairs and
+  // chunks index grid dimensions y and z (at most 65535 each)
   const long double elems = (long double)B * H * T * d;
   if (elems * 4 > 4.0e18L) return fail(GECKO_ERR_SHAPE, "tensor size overflows");
-  if (T / c > (1 << 30) || B * H > (1 << 30) || T > (int64_t(1) << 31) - 256)
-    return fail(GECKO_ERR_SHAPE, "size exceeds kernel index range");
+  if (T > (int64_t(1) << 31) - 256) return fail(GECKO_ERR_SHAPE, "T exceeds the kernels' index range");
+  if (B * H > kMaxGridYZ || T / c > kMaxGridYZ)
+    return fail(GECKO_ERR_SHAPE, "B*H = %lld and T/c = %lld must each be at most %d", (long long)(B * H),
+                (long long)(T / c), (int)kMaxGridYZ);
   for (int i = 0; i < n; ++i)
     if (reinterpret_cast<uintptr_t>(ptrs[i]) % 16 != 0)
       return fail(GECKO_ERR_ALIGN, "tensor argument %d is not 16-byte aligned", i);
@@ -505,6 +510,7 @@ extern "C" int gecko_awm_cp_logz(const float* lsum_all, int P, int rank, float* 
   if (!lsum_all || !logz_out) return fail(GECKO_ERR_ARG, "NULL pointer");
   if (P < 1 || rank < 0 || rank >= P) return fail(GECKO_ERR_ARG, "rank %d of %d", rank, P);
   if (B < 1 || H < 1 || (d != 64 && d != 128)) return fail(GECKO_ERR_SHAPE, "bad B, H or d");
+  if (B * H > kMaxGridYZ) return fail(GECKO_ERR_SHAPE, "B*H must be at most %d", (int)kMaxGridYZ);
   cudaGetLastError();
   return check_cuda(launch_cp_logz(lsum_all, logz_out, rank, B * H, (int)d, d, static_cast<cudaStream_t>(stream)),
                     "cp log z");
@@ -515,6 +521,7 @@ extern "C" int gecko_awm_cp_state(const float* lsum_all, const float* maps_all, 
   if (!lsum_all || !maps_all || !state_out) return fail(GECKO_ERR_ARG, "NULL pointer");
   if (P < 1 || rank < 0 || rank >= P) return fail(GECKO_ERR_ARG, "rank %d of %d", rank, P);
   if (B < 1 || H < 1 || (d != 64 && d != 128)) return fail(GECKO_ERR_SHAPE, "bad B, H or d");
+  if (B * H > kMaxGridYZ) return fail(GECKO_ERR_SHAPE, "B*H must be at most %d", (int)kMaxGridYZ);
   if (reinterpret_cast<uintptr_t>(maps_all) % 16 != 0) return fail(GECKO_ERR_ALIGN, "maps not 16-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int64_t BH = B * H, sd = state_floats(d);

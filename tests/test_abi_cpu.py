@@ -61,6 +61,8 @@ def _call(ptrs=None, B=1, H=1, T=256, c=128, d=64, dtype=1):
     (dict(T=300, c=128), 2),
     (dict(ptrs=[FAKE, FAKE + 8] + [FAKE] * 5), 3),
     (dict(B=1 << 40, H=1 << 20), 2),
+    (dict(B=256, H=256), 2),                 # B*H above the grid limit
+    (dict(T=64 * 65536, c=64), 2),           # T/c above the grid limit
 ])
 def test_host_validation_rejects(so, kw, code):
     assert _call(**kw) == code
@@ -152,8 +154,10 @@ def test_train_forward_rejects_bad_lse(so):
     (lambda: L.gecko_awm_cp_state(FAKE, FAKE, 3, -1, FAKE, 1, 1, 64, None), 1),
     (lambda: L.gecko_awm_cp_state(FAKE, FAKE + 4, 3, 1, FAKE, 1, 1, 64, None), 3),
     (lambda: L.gecko_awm_cp_state(FAKE, FAKE, 0, 0, FAKE, 1, 1, 64, None), 1),
+    (lambda: L.gecko_awm_cp_logz(FAKE, 2, 1, FAKE, 256, 256, 64, None), 2),
+    (lambda: L.gecko_awm_cp_state(FAKE, FAKE, 2, 1, FAKE, 256, 256, 64, None), 2),
 ], ids=["logsum-null", "logsum-shape", "maps-null", "maps-align", "logz-null", "logz-rank", "logz-d",
-        "state-rank", "state-align", "state-P"])
+        "state-rank", "state-align", "state-P", "logz-grid", "state-grid"])
 def test_context_parallel_host_validation_rejects(so, call, code):
     assert call() == code
     assert L.gecko_last_error()
