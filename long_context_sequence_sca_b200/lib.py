@@ -474,9 +474,9 @@ def awm_segment_logsum(km, c: int, stream=None):
 def _f32_on(t, shape, device, name):
     """t as a contiguous fp32 tensor of `shape` on `device` (the caller keeps
     the returned tensor alive until the call is enqueued)."""
-    if not (isinstance(t, torch.Tensor) and t.dtype == torch.float32 and tuple(t.shape) == tuple(shape)
-            and t.device == device):
-        raise ValueError(f"{name} must be a float32 tensor of shape {tuple(shape)} on {device}")
+    if not (isinstance(t, torch.Tensor) and t.is_cuda and t.dtype == torch.float32
+            and tuple(t.shape) == tuple(shape) and t.device == device):
+        raise ValueError(f"{name} must be a float32 CUDA tensor of shape {tuple(shape)} on {device}")
     return t.contiguous()
 
 
