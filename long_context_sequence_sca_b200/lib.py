@@ -223,13 +223,7 @@ def sca_awm_forward(q, k, v, qm, km, c: int, out_sca=None, out_mem=None, stream=
     (default: torch's current stream).
     """
     xs = (q, k, v, qm, km)
-    for x in xs:
-        if not (isinstance(x, torch.Tensor) and x.is_cuda and x.is_contiguous()):
-            raise ValueError("inputs must be contiguous CUDA tensors")
-        if x.shape != q.shape or x.dtype != q.dtype or x.device != q.device:
-            raise ValueError("inputs must share shape, dtype and device")
-    if q.dim() != 4 or q.dtype not in _DT:
-        raise ValueError("inputs must be [B, H, T, d] float32 or bfloat16")
+    _check_inputs(xs)
     B, H, T, d = q.shape
     _check_outputs((out_sca, out_mem), q)
     if out_sca is None:
