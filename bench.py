@@ -15,7 +15,7 @@ are independent, so there is no data-path collective).  The timed region is
 bracketed by a barrier and a device synchronise; the step time is the max
 over ranks; rank 0 prints one JSON line.
 
-`--impl reference` times the CPU oracle (fp64 NumPy, the machine's host cores) on
+`--impl reference` times the CPU oracle (fp64 NumPy, the host's cores) on
 bounded samples of the same workload instead.
 
 `--op backward` measures gecko_sca_awm_backward on the same workload (the
@@ -499,7 +499,7 @@ def run_reference(args, w: Workload) -> dict:
         "warmup": args.warmup, "ms_per_step": round(1e3 * tot_s / args.steps, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator)",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "c": w.c},
-        "impl": "reference", "host": "CPU oracle on the box's host cores (no GPU work)",
+        "impl": "reference", "host": "CPU oracle on the host's cores (no GPU work)",
         "cpu_baseline": {"value": round(val, 2), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(val, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
