@@ -135,7 +135,7 @@ class ClockSampler:
             self.h = self._handle(device_index)
             self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
             self.ok = True
-        except Exception as e:  # pragma: no cover - depends on the box
+        except Exception as e:  # pragma: no cover - depends on the machine
             self.err = repr(e)
 
     def _handle(self, idx):
