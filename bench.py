@@ -932,6 +932,10 @@ def run_cp(args, ws: int, rank: int, local: int) -> dict:
     }
     if note:
         out["note"] = note
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        # the segmented outputs equal the whole-sequence forward, so the
+        # oracle's forward on a bounded sample is the CPU baseline
+        out["cpu_baseline"] = cpu_baseline(w)
     return out
 
 
