@@ -79,8 +79,12 @@ extern "C" {
  * Ownership: the library keeps one workspace per device (log z per chunk,
  * per-chunk memory matrices, the carried state).  It grows on demand with
  * stream-ordered allocation on `stream` and lives until gecko_release().
- * Concurrent forwards on one device race on that workspace and are not
- * supported.  Every call starts from M'_1 = 0 (no initial state).
+ * Forwards of any kind (this one, _continue, _train, _noalloc, the
+ * context-parallel segment calls, and the backward's rebuild) must not
+ * overlap on the GPU on one device: besides the workspace they share the
+ * SCA kernel's work-unit counter and the device status word, so overlapping
+ * calls lose or repeat work.  Every call starts from M'_1 = 0 (no initial
+ * state).
  *
  * Returns GECKO_OK or an error code; the message is in gecko_last_error().
  */
@@ -201,9 +205,14 @@ int gecko_sca_awm_forward_continue(const void* q, const void* k, const void* v,
  * (cudaGetSymbolAddress) with that device current; make that first call
  * before any stream capture.  All calls share the array and it keeps the
  * last call's contents (every region is fully written before it is read,
- * so nothing needs clearing); calls that overlap on the GPU race on it.
- * This entry point does not update the state reported by gecko_awm_state,
- * which always describes the last gecko_sca_awm_forward call.
+ * so nothing needs clearing).  A call must not overlap on the GPU with any
+ * other forward on the same device, this entry point's or the allocating
+ * ones: they share the array (no-allocation calls), the SCA kernel's
+ * work-unit counter, which each SCA launch resets, and the device status
+ * word, so overlapping calls lose or repeat work.
+ * This entry point leaves the state reported by gecko_awm_state unchanged:
+ * that state stays the one of the last allocating forward, continued
+ * forward, training forward or backward on the device.
  */
 #define GECKO_NOALLOC_SCRATCH_BYTES (64ull << 20)
 int gecko_sca_awm_forward_noalloc(const void* q, const void* k, const void* v,

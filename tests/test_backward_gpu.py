@@ -82,6 +82,10 @@ def test_backward_matches_oracle(L, name):
     Workload("bwd_f32_d128_c64", 62, "f32", 1, 1, 384, 128, 64),
     Workload("bwd_bf16_one_chunk", 63, "bf16", 2, 1, 256, 64, 256),
     Workload("bwd_bf16_two_chunks", 64, "bf16", 1, 2, 512, 128, 256),
+    # c an odd multiple of 128: chunk boundaries fall between 128-row tiles
+    # that are not aligned to 256 rows
+    Workload("bwd_bf16_c384", 66, "bf16", 1, 2, 1152, 128, 384),
+    Workload("bwd_bf16_c384_d64", 67, "bf16", 2, 1, 1536, 64, 384),
 ], ids=lambda w: w.name)
 def test_backward_shapes(L, w):
     _check_backward(L, w)
