@@ -83,10 +83,26 @@ def io_bytes(w: Workload) -> int:
     return 7 * w.B * w.H * w.T * w.d * esz
 
 
+def stage_bytes(w: Workload) -> dict:
+    """Algorithmic HBM bytes of each timed stage that moves the inputs or
+    outputs: the statistics read K_m, the chunk products read K_m and V, the
+    readout reads Q_m and writes out_mem, SCA reads Q, K, V and writes
+    out_sca.  The carry only touches the O(S d^2) workspace."""
+    esz = 2 if w.dtype == "bf16" else 4
+    t = w.B * w.H * w.T * w.d * esz
+    return {"awm_stats": t, "awm_chunk": 2 * t, "awm_readout": 2 * t, "sca": 4 * t}
+
+
+def hbm_bound(w: Workload, pk: dict) -> bool:
+    """Arithmetic intensity of the step below the ridge of the measured peaks."""
+    return flops(w)["total"] / io_bytes(w) < pk["bf16_tflops"] * 1e12 / (pk["hbm_gbs"] * 1e9)
+
+
 # exp2 results per clock per SM of the special-function units (the public
 # arithmetic-throughput table's figure for compute capability 10.0)
 SFU_EXP_PER_CLK_SM = 16
 N_SM = 148
+L2_BYTES = 126 * 1024 * 1024
 
 
 def secondary_rooflines(w: Workload, ms_per_step: float, sca_ms: float, sm_mhz, hbm_gbs: float) -> dict:
@@ -352,22 +368,39 @@ def run_gecko(args, w: Workload, ws: int, rank: int, local: int) -> dict:
         raise RuntimeError("device status reported a timed-out wait during warm-up")
 
     sampler = ClockSampler(local)
+    # inputs that fit in L2 would be served from it on the next step: write a
+    # buffer of twice the L2 size between timed steps and time each step alone
+    in_bytes = sum(x[n].numel() * x[n].element_size() for n in ("q", "k", "v", "qm", "km"))
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda") if in_bytes <= L2_BYTES else None
 
     def timed():
         barrier(ws)
         torch.cuda.synchronize()
         L.timing_read()
         sampler.start()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            step()
-        e1.record(stream)
-        torch.cuda.synchronize()
+        if flush is None:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.steps):
+                step()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / args.steps
+        else:
+            evs = []
+            for _ in range(args.steps):
+                flush.fill_(1.0)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                step()
+                e1.record(stream)
+                evs.append((e0, e1))
+            torch.cuda.synchronize()
+            ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
         ck = sampler.stop()
         barrier(ws)
         stages, n = L.timing_read()
-        return e0.elapsed_time(e1) / args.steps, {k_: v_ / max(n, 1) for k_, v_ in stages.items()}, ck
+        return ms, {k_: v_ / max(n, 1) for k_, v_ in stages.items()}, ck
 
     ms_local, stages, ck = timed()
     note = None
@@ -384,25 +417,45 @@ def run_gecko(args, w: Workload, ws: int, rank: int, local: int) -> dict:
     # dominant kernel: the SCA launch (one per step), timed on its stream
     sca_ms = max_over_ranks(stages["sca"], ws)
     achieved = fl["sca"] / (sca_ms / 1e3) / 1e12
-    roofline = {"bound": "tensor", "kernel": "sca_tc_kernel", "achieved": round(achieved, 2),
-                "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops"], 4),
-                "peak_kind": f"{pk_kind} bf16 dense (burst)",
-                "frac_of_sustained": round(achieved / pk["bf16_tflops_sustained"], 4),
-                "traffic": recorded_traffic(w), "launch_ms": round(sca_ms, 4),
-                "algorithmic_flop_per_launch": fl["sca"]}
+    sb = stage_bytes(w)
+    stage_hbm = {}
+    for k_, b_ in sb.items():
+        ms_ = max_over_ranks(stages[k_], ws)
+        gbs = b_ / (ms_ / 1e3) / 1e9 if ms_ > 0 else 0.0
+        stage_hbm[k_] = {"algorithmic_bytes": b_, "ms": round(ms_, 4), "achieved_gbs": round(gbs, 1),
+                         "frac": round(gbs / pk["hbm_gbs"], 4)}
+    if hbm_bound(w, pk):
+        # below the ridge the kernels are bounded by HBM: the dominant one is
+        # the stage with the longest time
+        top = max(sb, key=lambda k_: stage_hbm[k_]["ms"])
+        roofline = {"bound": "hbm", "kernel": top, "achieved": stage_hbm[top]["achieved_gbs"],
+                    "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": stage_hbm[top]["frac"],
+                    "peak_kind": f"{pk_kind} HBM copy",
+                    "traffic": recorded_traffic(w) if top == "sca" else None,
+                    "launch_ms": stage_hbm[top]["ms"], "algorithmic_bytes_per_launch": sb[top]}
+    else:
+        roofline = {"bound": "tensor", "kernel": "sca_tc_kernel", "achieved": round(achieved, 2),
+                    "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops"], 4),
+                    "peak_kind": f"{pk_kind} bf16 dense (burst)",
+                    "frac_of_sustained": round(achieved / pk["bf16_tflops_sustained"], 4),
+                    "traffic": recorded_traffic(w), "launch_ms": round(sca_ms, 4),
+                    "algorithmic_flop_per_launch": fl["sca"]}
 
     out = {
         "metric": METRIC, "value": round(agg["value"], 1), "unit": "tokens/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(agg["ms_per_step"], 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic (seeded Z'-affine generator; no dataset)",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "c": w.c,
                    "tokens_per_step_per_gpu": tokens,
-                   "l2": f"inputs larger than L2 ({5 * w.B * w.H * w.T * w.d * 2 / 1e9:.2f} GB), no flush",
+                   "l2": (f"inputs larger than L2 ({in_bytes / 1e9:.2f} GB), no flush" if flush is None else
+                          f"inputs {in_bytes / 1e6:.1f} MB fit in L2: {2 * L2_BYTES / 1e6:.0f} MB written between "
+                          f"timed steps, each step timed alone"),
                    "parallelism": f"replicas x{ws} (heads/batches independent)"},
         "tflops": round(ws * fl["total"] / (agg["ms_per_step"] / 1e3) / 1e12, 2),
         "pct_bf16_peak": round(100 * fl["total"] / (agg["ms_per_step"] / 1e3) / 1e12 / pk["bf16_tflops"], 2),
         "stage_ms": {k_: round(v_, 4) for k_, v_ in stages.items()},
+        "stage_hbm": stage_hbm,
         "roofline": roofline,
         "other_bounds": secondary_rooflines(w, agg["ms_per_step"], sca_ms, ck.get("sm_mhz"), pk["hbm_gbs"]),
         "clocks": ck,
@@ -939,37 +992,7 @@ def run_cp(args, ws: int, rank: int, local: int) -> dict:
     return out
 
 
-def summarize_launches(path: str) -> str:
-    """Per-kernel launches, total time and share from an ncu launch-list CSV
-    (`ncu --metrics gpu__time_duration.sum --csv`)."""
-    import collections
-    import csv
-    import re
-    rows = list(csv.reader(open(path)))
-    hi = next(i for i, r in enumerate(rows) if "Kernel Name" in r)
-    hdr = rows[hi]
-    ki, mi, vi, ui = (hdr.index(k) for k in ("Kernel Name", "Metric Name", "Metric Value", "Metric Unit"))
-    scale = {"ns": 1e-3, "nsecond": 1e-3, "us": 1.0, "usecond": 1.0, "ms": 1e3, "msecond": 1e3}
-    agg = collections.OrderedDict()
-    for r in rows[hi + 1:]:
-        if len(r) <= vi or r[mi] != "gpu__time_duration.sum":
-            continue
-        name = re.sub(r"\(.*", "", r[ki]).replace("void ", "")
-        name = re.sub(r"gecko::(\(anonymous namespace\)|<unnamed>)::", "", name)
-        a = agg.setdefault(name, [0, 0.0])
-        a[0] += 1
-        a[1] += float(r[vi].replace(",", "")) * scale[r[ui]]
-    tot = sum(a[1] for a in agg.values()) or 1.0
-    lines = [f"{'kernel':44s} {'launches':>8s} {'total_us':>10s} {'share':>7s}"]
-    for k, (n, t) in sorted(agg.items(), key=lambda kv: -kv[1][1]):
-        lines.append(f"{k:44s} {n:8d} {t:10.1f} {100 * t / tot:6.1f}%")
-    return "\n".join(lines)
-
-
 def main(argv=None):
-    if argv is None and len(sys.argv) > 2 and sys.argv[1] == "--summarize-launches":
-        print(summarize_launches(sys.argv[2]))
-        return 0
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
