@@ -13,28 +13,25 @@
 // exponentials in packed f16 (two per SFU op); they enter the tensor core as
 // bf16, whose 8-bit mantissa is coarser than f16's.
 //
-// awm_chunk_tc_kernel: one CTA per (chunk, bh).  The chunk is streamed in
-// tiles of 64 tokens.  V tiles arrive by TMA; 128 threads (two per token)
-// compute Phi and Psi in fp32 and store them as bf16 next to V in one
-// 128-byte-swizzled, MN-major stage [V | Psi | Phi], so a single
+// awm_chunk_tc_kernel: one CTA per (chunk, bh), two per SM.  The chunk is
+// streamed in tiles of 64 tokens; V and K_m tiles arrive by TMA; 256 threads
+// (four per token) compute Phi and Psi in fp32 and store them as bf16 next
+// to V in one 128-byte-swizzled, MN-major stage [V | Psi | Phi], so a single
 // tcgen05.mma with M = d, N = 2d accumulates [Phi^T V | Phi^T Psi] in TMEM.
 //
-// awm_readout_tc_kernel: one CTA per (chunk, bh).  M'_{s-1} is converted to
-// bf16 once into shared memory (MN-major B operand); every 128-row tile of
-// Qm_s is turned into psi rows (K-major A operand) by 128 threads, one row
-// each, and multiplied on the tensor core; the epilogue writes bf16 rows.
+// awm_carry_tc_kernel (d = 128): the sequential carry, one CTA per (b, h),
+// the product Cm_s M'_s as bf16 hi + lo MMAs; it also writes M'_s as the
+// readout's bf16 operand image.
+//
+// awm_readout_tc_kernel: persistent, a contiguous range of 128-row tiles per
+// CTA; Q_m tiles by TMA into a 4-stage ring, psi numerators formed in place
+// (K-major A operand), the operand image of M'_{s-1} by one bulk copy per
+// chunk, the output tile staged in the freed stage and stored by TMA.
 #include "common.cuh"
 #include "gecko_internal.h"
 
 namespace gecko {
 namespace {
-
-// Byte offset of element (row, col) in a 128-byte-swizzled tile made of
-// 64-column boxes of `rows` rows each (the TMA SWIZZLE_128B layout).
-__device__ __forceinline__ uint32_t sw128_off(int row, int col, int rows) {
-  const int box = col >> 6, cc = col & 63;
-  return box * rows * 128 + row * 128 + ((((cc >> 3) ^ (row & 7)) << 4)) + ((cc & 7) << 1);
-}
 
 // ------------------------------------------------------------ chunk GEMMs --
 
@@ -69,9 +66,13 @@ struct ChunkCfg {
   static constexpr uint32_t kTmemCols = Mode == kChunkE ? D : (D == 128 ? 256 : 128);
 };
 
-// 128 compute threads (warps 0-3), warp 4 = TMA producer, warp 5 = MMA issuer.
+// 128 compute threads (warps 0-3, two per token row), warp 4 = TMA
+// producer, warp 5 = MMA issuer; two CTAs per SM.  (Eight compute warps,
+// four per row, measured slower: 0.191 against 0.183 ms at the bench
+// workload.)
+constexpr int kChunkCompute = 128, kChunkThreads = 192;
 template <int D, int Mode = kChunkFwd>
-__global__ void __launch_bounds__(192, 2) awm_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_v,
+__global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_v,
                                                            const __grid_constant__ CUtensorMap map_km,
                                                            const float* __restrict__ lse, float* __restrict__ Bm,
                                                            float* __restrict__ Cm, int T, int c, int koff,
@@ -101,7 +102,7 @@ __global__ void __launch_bounds__(192, 2) awm_chunk_tc_kernel(const __grid_const
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(v_full + i, 1);
-      mbar_init(op_full + i, 128);
+      mbar_init(op_full + i, kChunkCompute);
       mbar_init(st_empty + i, 1);
     }
     mbar_init(acc_full, 1);
@@ -313,207 +314,545 @@ __global__ void __launch_bounds__(192, 2) awm_chunk_tc_kernel(const __grid_const
 
 template <int D>
 struct ReadoutCfg {
-  static constexpr int kBox = 128 * 128;        // one [128 rows x 64] bf16 box, 128B-swizzled
-  static constexpr int kA = 128 * D * 2;       // a Q_m tile = the psi operand (K-major, D/64 boxes)
-  static constexpr int kB = D * D * 2;         // M' bf16, MN-major, D/64 boxes of [D x 64]
-  static constexpr int kAOff = 0;              // two tiles
-  static constexpr int kBOff = 2 * kA;
-  static constexpr int kBarOff = kBOff + kB;
-  static constexpr int kNumBars = 5;           // q_full[2], acc_full[2], drain
+  static constexpr int kTile = 128 * D * 2;      // a 128-row tile, bf16, D / 64 swizzled boxes of 16 KB
+  static constexpr int kBox = 128 * 128;         // one [128 rows x 64] box
+  static constexpr int kStages = 4;              // Q_m tile ring, reused to stage the output tile
+  static constexpr int kImg = D * D * 2;         // one M' operand image
+  static constexpr int kImgOff = kStages * kTile;
+  static constexpr int kInvOff = kImgOff + 2 * kImg;      // [kStages][128] 1 / row sum of psi numerators
+  static constexpr int kBarOff = kInvOff + kStages * 128 * 4;
+  // q_full, op_full, st_empty, out_ready [kStages]; img_full, img_empty, acc_full, acc_empty [2]; drain
+  static constexpr int kNumBars = 4 * kStages + 8 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;
   static constexpr uint32_t kTmemCols = 2 * D;   // two accumulators
+  static constexpr int kThreads = 320;
 };
 
-// 128 threads: one row each; thread 0 also issues the TMA copies and the
-// MMAs.  grid (S, BH, G): CTA g of a chunk takes its 128-row tiles g,
-// g + G, ...  Each Q_m tile arrives by TMA in the 128B-swizzled K-major
-// layout of the MMA's A operand; every thread turns its row into the
-// unnormalised numerators exp(q - max) in place (bf16, packed f16
-// exponentials), and the epilogue scales row t by 1 / sum_t.  Two tile
-// buffers and two accumulators: the next tile's copy is issued as soon as
-// the MMA that read its buffer has completed, and a tile's MMA overlaps the
-// previous tile's epilogue.
+// The readout O_m,s = psi(Qm_s) M'_{s-1} (Gecko digest, method step details,
+// step 5).  Persistent: CTA b takes a contiguous range of the 128-row tiles
+// ordered by (b, h), chunk, tile, balanced by weight (a tile of chunks 1
+// and 2 of a fresh sequence only writes zeros: weight 1; every other tile
+// reads Q_m and writes out_mem: weight 2).  320 threads:
+//   warps 0-3  psi: each thread turns its row of the Q_m tile (TMA, K-major
+//              A operand layout) into the numerators exp(q - max) in place,
+//              bf16, and keeps 1 / sum for the epilogue;
+//   warps 4-7  epilogue: accumulator rows from TMEM scaled by 1 / sum,
+//              bf16, written over the tile's stage and stored by one TMA
+//              store; zero tiles are written directly;
+//   warp 8     TMA producer: Q_m tiles into a 4-stage ring, and the operand
+//              image of M'_{s-1} (bf16, written by the carry in the MN-major
+//              B layout) by one bulk copy whenever the chunk changes
+//              (two image buffers);
+//   warp 9     TMEM allocation and the MMAs (one thread), two accumulators.
 template <int D>
-__global__ void __launch_bounds__(128) awm_readout_tc_kernel(const __grid_constant__ CUtensorMap map_q,
-                                                             const float* __restrict__ Mst,
-                                                             __nv_bfloat16* __restrict__ out, int T, int c,
-                                                             const float* __restrict__ Mprev0, int64_t sd,
-                                                             int* status) {
+__global__ void __launch_bounds__(ReadoutCfg<D>::kThreads, 1)
+awm_readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_o,
+                      const uint16_t* __restrict__ Mimg, __nv_bfloat16* __restrict__ out, int T, int c, int S,
+                      int BH, int fresh, int* status) {
   using Cfg = ReadoutCfg<D>;
+  constexpr int NS = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* q_full = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);  // [2] TMA -> threads
-  uint64_t* acc_full = q_full + 2;                                        // [2] MMA -> threads, TMA
-  uint64_t* drain = acc_full + 2;
+  float* rinv = reinterpret_cast<float*>(smem + Cfg::kInvOff);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
+  uint64_t* q_full = bars;                // TMA -> psi warps
+  uint64_t* op_full = q_full + NS;        // psi warps (128) -> MMA
+  uint64_t* st_empty = op_full + NS;      // output store finished reading the stage -> TMA
+  uint64_t* out_ready = st_empty + NS;    // epilogue (128) wrote the output tile -> storing thread
+  uint64_t* img_full = out_ready + NS;    // [2] image copy -> MMA
+  uint64_t* img_empty = img_full + 2;     // [2] last MMA of the image's chunk -> TMA
+  uint64_t* acc_full = img_empty + 2;     // [2] MMA -> epilogue
+  uint64_t* acc_empty = acc_full + 2;     // [2] epilogue (128) -> MMA
+  uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
 
-  const int s = blockIdx.x, S = gridDim.x;
-  const int64_t bh = blockIdx.y;
-  const int g = blockIdx.z, G = gridDim.z;
-  const int warp = warp_id_uniform();
-  const int r = threadIdx.x;
-  const int n_tiles = c / 128;
-  const int m = n_tiles > g ? (n_tiles - g + G - 1) / G : 0;  // tiles of this CTA
-  const int64_t row0 = bh * (int64_t)T + (int64_t)s * c;
-
-  if (s < 2 && Mprev0 == nullptr) {
-    // a fresh sequence: chunks 1 and 2 read M'_0 = M'_1 = 0
-    const uint4 z = make_uint4(0, 0, 0, 0);
-    for (int idx = 0; idx < m; ++idx) {
-      uint4* dst = reinterpret_cast<uint4*>(out + (row0 + (int64_t)(g + idx * G) * 128) * D);
-      for (int i = threadIdx.x; i < 128 * D / 8; i += blockDim.x) dst[i] = z;
-    }
-    return;
-  }
-  if (m == 0) return;
-  auto load_tile = [&](int idx) {   // thread 0: tile idx into buffer idx & 1
-    const int buf = idx & 1;
-    mbar_arrive_expect_tx(q_full + buf, Cfg::kA);
-    for (int b = 0; b < D / 64; ++b)
-      tma_load_2d(smem + Cfg::kAOff + buf * Cfg::kA + b * Cfg::kBox, &map_q, q_full + buf, b * 64,
-                  (int)(row0 + (int64_t)(g + idx * G) * 128));
+  const int warp = warp_id_uniform(), lane = threadIdx.x % 32;
+  const int nt = c / 128;                        // tiles per chunk
+  const int zc = fresh ? (S < 2 ? S : 2) : 0;   // leading zero chunks per (b, h)
+  // weighted split: per (b, h) the zero tiles weigh 1, the others 2
+  const int64_t wbh = (int64_t)zc * nt + 2 * (int64_t)(S - zc) * nt;
+  const int64_t W = wbh * BH;
+  auto tile_at = [&](int64_t x) -> int64_t {   // first tile whose cumulative weight reaches x
+    const int64_t bh = x / wbh, r = x % wbh, z = (int64_t)zc * nt;
+    return bh * (int64_t)S * nt + (r < z ? r : z + (r - z + 1) / 2);
   };
+  const int64_t u0 = tile_at(W * blockIdx.x / gridDim.x);
+  const int64_t u1 = blockIdx.x + 1 == gridDim.x ? (int64_t)BH * S * nt : tile_at(W * (blockIdx.x + 1) / gridDim.x);
+  const int m = (int)(u1 - u0);   // tiles of this CTA
+  // the CTA's tiles are walked with counters (no 64-bit division per tile)
+  struct TileIt {
+    int bh, s, kt;
+  };
+  const TileIt first{(int)(u0 / ((int64_t)S * nt)), (int)((u0 / nt) % S), (int)(u0 % nt)};
+  auto next = [&](TileIt& t) {
+    if (++t.kt == nt) {
+      t.kt = 0;
+      if (++t.s == S) {
+        t.s = 0;
+        ++t.bh;
+      }
+    }
+  };
+  auto is_zero = [&](const TileIt& t) { return t.s < zc; };
+  auto row_of = [&](const TileIt& t) { return (int64_t)t.bh * T + (int64_t)t.s * c + t.kt * 128; };
+  auto img_of = [&](const TileIt& t) { return (int64_t)t.bh * (S + 1) + t.s; };
+
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NS; ++i) {
       mbar_init(q_full + i, 1);
+      mbar_init(op_full + i, 128);
+      mbar_init(st_empty + i, 1);
+      mbar_init(out_ready + i, 128);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(img_full + i, 1);
+      mbar_init(img_empty + i, 1);
       mbar_init(acc_full + i, 1);
+      mbar_init(acc_empty + i, 128);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&map_q);
-    load_tile(0);
   }
-  if (warp == 0) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, Cfg::kTmemCols);
     tmem_relinquish();
   }
-  // B operand: M'_{s-1} (0-based chunk s reads Mst[s-1]; a continued
-  // sequence's first chunk reads the carried M'_prev) as bf16, rows = key
-  // feature f (K), columns = value dim j (N, contiguous): MN-major.
-  const float* M = s == 0 ? Mprev0 + bh * sd : Mst + (bh * (S + 1) + (s - 1)) * (int64_t)D * D;
-  for (int i = threadIdx.x; i < D * D / 8; i += blockDim.x) {
-    const int f = (i * 8) / D, j = (i * 8) % D;
-    const float4 a = reinterpret_cast<const float4*>(M + f * D + j)[0];
-    const float4 b = reinterpret_cast<const float4*>(M + f * D + j)[1];
-    uint4 p;
-    p.x = pack_bf16x2(a.x, a.y);
-    p.y = pack_bf16x2(a.z, a.w);
-    p.z = pack_bf16x2(b.x, b.y);
-    p.w = pack_bf16x2(b.z, b.w);
-    *reinterpret_cast<uint4*>(smem + Cfg::kBOff + sw128_off(f, j, D)) = p;
-  }
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t base = smem_u32(smem);
-  constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, true);
-  const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-  const SDesc bdesc = sdesc_sw128_split(base + Cfg::kBOff, D * 128, 1024);
-  bool ok = true;
 
-  auto store_tile = [&](int kt, int buf, uint32_t parity, float inv) -> bool {
-    if (!__all_sync(0xffffffffu, mbar_wait(acc_full + buf, parity, abort_flag, status))) return false;
-    tc_fence_after();
-    __nv_bfloat16* orow = out + (row0 + (int64_t)kt * 128 + r) * D;
-#pragma unroll 1
-    for (int cb = 0; cb < D / 32; ++cb) {
-      uint32_t v[32];
-      tmem_ld32(lane_addr + buf * D + cb * 32, v);
-      tmem_wait_ld();
-      uint4 w[4];
-      uint32_t* wp = reinterpret_cast<uint32_t*>(w);
-#pragma unroll
-      for (int i = 0; i < 16; ++i)
-        wp[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * inv, __uint_as_float(v[2 * i + 1]) * inv);
-      uint4* dst = reinterpret_cast<uint4*>(orow + cb * 32);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) dst[i] = w[i];
-    }
-    tc_fence_before();
-    return true;
-  };
-
-  float inv_prev = 0.f;
-  int issued = 1;   // tiles whose copy has been issued (thread 0)
-  for (int idx = 0; idx < m && ok; ++idx) {
-    const int kt = g + idx * G, buf = idx & 1;
-    ok = __all_sync(0xffffffffu, mbar_wait(q_full + buf, (idx >> 1) & 1, abort_flag, status));
-    if (!ok) break;
-    // psi numerators exp(q - max) of row r, written over the row in place
-    uint8_t* a = smem + Cfg::kAOff + buf * Cfg::kA;
-    float mx = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < D / 8; ++i) {
-      const uint4 q = *reinterpret_cast<const uint4*>(a + sw128_off(r, 8 * i, 128));
-      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&q);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f2 = __bfloat1622float2(p2[j]);
-        mx = fmax3(mx, f2.x, f2.y);
+  if (warp == 8) {
+    // --------------------------------------------------- TMA producer --
+    if (lane == 0) {
+      tma_prefetch_desc(&map_q);
+      int n = 0, k = -1;
+      int64_t cur = -1;
+      bool ok = true;
+      TileIt t = first;
+      for (int i = 0; i < m && ok; ++i, next(t)) {
+        if (is_zero(t)) continue;
+        const int64_t im = img_of(t);
+        if (im != cur) {
+          cur = im;
+          ++k;
+          if (k >= 2 && !(ok = mbar_wait(img_empty + (k & 1), ((k >> 1) - 1) & 1, abort_flag, status))) break;
+          mbar_arrive_expect_tx(img_full + (k & 1), Cfg::kImg);
+          bulk_load_1d(smem + Cfg::kImgOff + (k & 1) * Cfg::kImg, Mimg + im * (int64_t)D * D, Cfg::kImg,
+                       img_full + (k & 1));
+        }
+        const int st = n % NS;
+        if (n >= NS && !(ok = mbar_wait(st_empty + st, ((n / NS) - 1) & 1, abort_flag, status))) break;
+        mbar_arrive_expect_tx(q_full + st, Cfg::kTile);
+        for (int b = 0; b < D / 64; ++b)
+          tma_load_2d(smem + st * Cfg::kTile + b * Cfg::kBox, &map_q, q_full + st, b * 64, (int)row_of(t));
+        ++n;
+      }
+      if (!ok) {
+        // copies already issued land before the CTA exits
+        for (int t = n > NS ? n - NS : 0; t < n; ++t) mbar_wait_drain(q_full + t % NS, (t / NS) & 1);
+        for (int t = k > 1 ? k - 1 : 0; t <= k; ++t) mbar_wait_drain(img_full + (t & 1), (t >> 1) & 1);
       }
     }
-    const float mx2 = mx * kLog2e;
-    float sum = 0.f;
+    __syncwarp();
+  } else if (warp == 9) {
+    // ------------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, true);
+      const uint32_t base = smem_u32(smem);
+      int n = 0, k = -1;
+      int64_t cur = -1;
+      bool ok = true;
+      TileIt t = first;
+      for (int i = 0; i < m && ok; ++i, next(t)) {
+        if (is_zero(t)) continue;
+        const int64_t im = img_of(t);
+        if (im != cur) {
+          cur = im;
+          ++k;
+          if (!(ok = mbar_wait(img_full + (k & 1), (k >> 1) & 1, abort_flag, status))) break;
+        }
+        const int st = n % NS, a = n & 1;
+        if (!(ok = mbar_wait(op_full + st, (n / NS) & 1, abort_flag, status))) break;
+        if (!(ok = mbar_wait(acc_empty + a, ((n >> 1) & 1) ^ 1, abort_flag, status))) break;
+        tc_fence_after();
+        const SDesc ad = sdesc_sw128_split(base + st * Cfg::kTile, 16, 1024);
+        const SDesc bd = sdesc_sw128_split(base + Cfg::kImgOff + (k & 1) * Cfg::kImg, D * 128, 1024);
 #pragma unroll
-    for (int i = 0; i < D / 8; ++i) {
-      uint4* qa = reinterpret_cast<uint4*>(a + sw128_off(r, 8 * i, 128));
-      const uint4 q = *qa;
-      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&q);
-      uint4 p;
-      uint32_t* pp = reinterpret_cast<uint32_t*>(&p);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f2 = __bfloat1622float2(p2[j]);
-        float e0, e1;
-        ex2_h2(fmaf(f2.x, kLog2e, -mx2), fmaf(f2.y, kLog2e, -mx2), e0, e1);
-        sum += e0 + e1;
-        pp[j] = pack_bf16x2(e0, e1);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk / 4) * Cfg::kBox + (kk % 4) * 32;
+          umma_ss(tmem + a * D, sdesc_at(ad, koff), sdesc_at(bd, kk * 16 * 128), idesc, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(acc_full + a);
+        // the image is released after the last tile of its chunk in this
+        // range (tiles of one chunk are consecutive; the next chunk's tiles,
+        // if any, are never zero tiles of the same image)
+        if (i + 1 == m || t.kt + 1 == nt) umma_commit(img_empty + (k & 1));
+        ++n;
       }
-      *qa = p;
+      umma_commit(drain);
+      mbar_wait_drain(drain, 0);
     }
-    const float inv = 1.f / sum;
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (threadIdx.x == 0) {
-      const SDesc ad = sdesc_sw128_split(base + Cfg::kAOff + buf * Cfg::kA, 16, 1024);
+    __syncwarp();
+  } else if (warp < 4) {
+    // -------------------------------------------------- psi numerators --
+    const int r = threadIdx.x;   // row of the tile
+    int n = 0;
+    bool ok = true;
+    TileIt t = first;
+    for (int i = 0; i < m; ++i, next(t)) {
+      if (is_zero(t)) continue;
+      const int st = n % NS;
+      ok = __all_sync(0xffffffffu, mbar_wait(q_full + st, (n / NS) & 1, abort_flag, status));
+      if (!ok) break;
+      uint8_t* tile = smem + st * Cfg::kTile;
+      float mx = -INFINITY;
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t koff = (kk / 4) * (128 * 128) + (kk % 4) * 32;
-        umma_ss(tmem + buf * D, sdesc_at(ad, koff), sdesc_at(bdesc, kk * 16 * 128), idesc, kk > 0 ? 1u : 0u);
-      }
-      umma_commit(acc_full + buf);
-      // refill the other buffer once the MMA that read it (tile idx - 1) is done
-      if (idx + 1 < m) {
-        if (idx == 0 || mbar_wait(acc_full + (buf ^ 1), ((idx - 1) >> 1) & 1, abort_flag, status)) {
-          load_tile(idx + 1);
-          ++issued;
+      for (int i = 0; i < D / 8; ++i) {
+        const uint4 q = *reinterpret_cast<const uint4*>(tile + sw128_off(r, 8 * i, 128));
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f2 = __bfloat1622float2(p2[j]);
+          mx = fmax3(mx, f2.x, f2.y);
         }
       }
+      const float mx2 = mx * kLog2e;
+      float sum = 0.f;
+#pragma unroll
+      for (int i = 0; i < D / 8; ++i) {
+        uint4* qa = reinterpret_cast<uint4*>(tile + sw128_off(r, 8 * i, 128));
+        const uint4 q = *qa;
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&q);
+        uint4 pv;
+        uint32_t* pp = reinterpret_cast<uint32_t*>(&pv);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f2 = __bfloat1622float2(p2[j]);
+          float e0, e1;
+          ex2_h2(fmaf(f2.x, kLog2e, -mx2), fmaf(f2.y, kLog2e, -mx2), e0, e1);
+          sum += e0 + e1;
+          pp[j] = pack_bf16x2(e0, e1);
+        }
+        *qa = pv;
+      }
+      rinv[st * 128 + r] = 1.f / sum;
+      fence_proxy_async_smem();   // the numerators are read by the tensor core (async proxy)
+      mbar_arrive(op_full + st);
+      ++n;
     }
-    // epilogue of the previous tile overlaps this tile's MMA
-    if (idx > 0) ok = store_tile(kt - G, buf ^ 1, ((idx - 1) >> 1) & 1, inv_prev);
-    inv_prev = inv;
-  }
-  if (ok) ok = store_tile(g + (m - 1) * G, (m - 1) & 1, ((m - 1) >> 1) & 1, inv_prev);
-  if (!ok && threadIdx.x == 0) {
-    // no MMA may still write TMEM, and no copy still write shared memory,
-    // when the CTA exits
-    umma_commit(drain);
-    mbar_wait_drain(drain, 0);
-    for (int t = issued > 2 ? issued - 2 : 0; t < issued; ++t) mbar_wait_drain(q_full + (t & 1), (t >> 1) & 1);
+  } else {
+    // --------------------------------------------------------- epilogue --
+    const int q4 = warp % 4;                       // TMEM lane quarter
+    const int r = q4 * 32 + lane;                  // row of the tile
+    const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
+    const bool leader = warp == 4 && lane == 0;   // issues the stores
+    int n = 0;
+    bool ok = true;
+    TileIt t = first;
+    for (int i = 0; i < m && ok; ++i, next(t)) {
+      if (is_zero(t)) {
+        const uint4 z = make_uint4(0, 0, 0, 0);
+        uint4* dst = reinterpret_cast<uint4*>(out + (row_of(t) + r) * D);
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) dst[i] = z;
+        continue;
+      }
+      const int st = n % NS, a = n & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(acc_full + a, (n >> 1) & 1, abort_flag, status));
+      if (!ok) break;
+      tc_fence_after();
+      const float inv = rinv[st * 128 + r];
+      uint8_t* tile = smem + st * Cfg::kTile;   // the psi operand is no longer read: stage the output here
+#pragma unroll 1
+      for (int cb = 0; cb < D / 32; ++cb) {
+        uint32_t v[32];
+        tmem_ld32(lane_addr + a * D + cb * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(v[8 * x + 0]) * inv, __uint_as_float(v[8 * x + 1]) * inv);
+          w.y = pack_bf16x2(__uint_as_float(v[8 * x + 2]) * inv, __uint_as_float(v[8 * x + 3]) * inv);
+          w.z = pack_bf16x2(__uint_as_float(v[8 * x + 4]) * inv, __uint_as_float(v[8 * x + 5]) * inv);
+          w.w = pack_bf16x2(__uint_as_float(v[8 * x + 6]) * inv, __uint_as_float(v[8 * x + 7]) * inv);
+          *reinterpret_cast<uint4*>(tile + sw128_off(r, cb * 32 + 8 * x, 128)) = w;
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(acc_empty + a);
+      fence_proxy_async_smem();   // the tile is read by the TMA store (async proxy)
+      mbar_arrive(out_ready + st);
+      if (leader) {
+        if (!(ok = mbar_wait(out_ready + st, (n / NS) & 1, abort_flag, status))) break;
+        for (int b = 0; b < D / 64; ++b) tma_store_2d(&map_o, tile + b * Cfg::kBox, b * 64, (int)row_of(t));
+        bulk_commit();
+        // the previous tile's store has finished reading its stage
+        bulk_wait_read<1>();
+        if (n > 0) mbar_arrive(st_empty + (n - 1) % NS);
+      }
+      ++n;
+    }
+    if (leader) {
+      bulk_wait_all();
+      if (n > 0) mbar_arrive(st_empty + (n - 1) % NS);
+    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) tmem_dealloc(tmem, Cfg::kTmemCols);
+  if (warp == 9) tmem_dealloc(tmem, Cfg::kTmemCols);
+}
+
+// ------------------------------------------------------------------ carry --
+
+// The sequential carry on the tensor cores, d = 128 (Gecko digest, method
+// step details, step 4, with the row scales factored out as in the SIMT
+// carry):
+//   M'_{s+1} = r_s (.) M'_s + rho_s (.) (Bm_s - Cm_s M'_s),
+// one CTA per (b, h), 128 threads, thread f owning row f of M' (an fp32
+// master copy in registers) and TMEM lane f of the product.  Per step the
+// product Cm_s M'_s runs as two bf16 MMAs, Cm M_hi + Cm M_lo with M' split
+// into hi + lo parts and fp32 accumulation (Cm rounded to bf16 once:
+// emulated over 128 chunks of 512 tokens the state stays within 2e-5 of
+// fp64).  Cm_s arrives by one bulk copy into an fp32 staging buffer one
+// step ahead and is rounded into the K-major A operand; Bm_s arrives by TMA
+// (128-byte swizzled, so each thread reads its row without bank conflicts)
+// while the step's operands are formed and multiplied.  M'_s is split from
+// the registers into the MN-major B operands, whose hi part is also the
+// readout's operand image of M'_s (bf16, same layout) and leaves by one bulk
+// store.  Writes Mst[s] = M'_{s+1} for s = 0..S like the SIMT carry.
+struct CarryTcCfg {
+  static constexpr int kD = 128;
+  static constexpr int kStage = kD * kD * 4;     // one fp32 d x d matrix
+  static constexpr int kOp = kD * kD * 2;        // one bf16 operand (two 64-column boxes of 128 rows)
+  static constexpr int kBox = 128 * 128;         // one bf16 box [128 rows x 64]
+  static constexpr int kFBox = 128 * 128;        // one fp32 box [128 rows x 32]
+  static constexpr int kCOff = 0;                // Cm_s staging, fp32 row-major
+  static constexpr int kBmOff = kCOff + kStage;  // Bm_s, fp32, four 128B-swizzled boxes of 32 columns
+  static constexpr int kAOff = kBmOff + kStage, kBhiOff = kAOff + kOp, kBloOff = kBhiOff + kOp;
+  static constexpr int kBarOff = kBloOff + kOp;  // c_full, b_full, m_done, drain
+  static constexpr int kMiscOff = kBarOff + 32;
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+
+__global__ void __launch_bounds__(128, 1)
+awm_carry_tc_kernel(const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_m,
+                    const float* __restrict__ Cm,
+                    const float* __restrict__ ratio, const float* __restrict__ rho, float* __restrict__ Mst, int S,
+                    const float* __restrict__ M0, int64_t sd, uint16_t* __restrict__ Mimg,
+                    const float* __restrict__ Mprev0, int* status) {
+  using Cfg = CarryTcCfg;
+  constexpr int D = Cfg::kD;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const float* cst = reinterpret_cast<const float*>(smem + Cfg::kCOff);
+  uint64_t* c_full = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
+  uint64_t* b_full = c_full + 1;
+  uint64_t* m_done = c_full + 2;
+  uint64_t* drain = c_full + 3;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
+  const int64_t bh = blockIdx.x;
+  const int f = threadIdx.x, warp = f / 32, lane = f % 32;
+  const int64_t mat = (int64_t)D * D;
+  float* mout = Mst + bh * (int64_t)(S + 1) * mat;
+  uint16_t* iout = Mimg ? Mimg + bh * (int64_t)(S + 1) * mat : nullptr;
+  int cloads = 0, bloads = 0;   // staging copies issued (thread 0)
+  auto load_bm = [&](int s) {   // thread 0: Bm_s into its swizzled boxes
+    mbar_arrive_expect_tx(b_full, Cfg::kStage);
+    for (int b = 0; b < D / 32; ++b)
+      tma_load_2d(smem + Cfg::kBmOff + b * Cfg::kFBox, &map_b, b_full, b * 32, (int)((bh * S + s) * D));
+    ++bloads;
+  };
+
+  if (f == 0) {
+    mbar_init(c_full, 1);
+    mbar_init(b_full, 1);
+    mbar_init(m_done, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&map_b);
+    tma_prefetch_desc(&map_m);
+    if (S > 0) {
+      cloads = 1;
+      mbar_arrive_expect_tx(c_full, Cfg::kStage);
+      bulk_load_1d(smem + Cfg::kCOff, Cm + bh * S * mat, Cfg::kStage, c_full);
+      load_bm(0);
+    }
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+  }
+  // M'_1: zero, or the carried M'_cur of a continued sequence
+  float m[D];
+#pragma unroll
+  for (int j = 0; j < D; j += 4) {
+    const float4 v = M0 ? *reinterpret_cast<const float4*>(M0 + bh * sd + (int64_t)f * D + j) : make_float4(0, 0, 0, 0);
+    m[j] = v.x; m[j + 1] = v.y; m[j + 2] = v.z; m[j + 3] = v.w;
+    *reinterpret_cast<float4*>(mout + (int64_t)f * D + j) = v;
+  }
+  if (iout && Mprev0) {
+    // image 0: the carried M'_prev, read by a continued sequence's first chunk
+    uint8_t* img = reinterpret_cast<uint8_t*>(iout);
+#pragma unroll 4
+    for (int j = 0; j < D; j += 8) {
+      const float4 a = *reinterpret_cast<const float4*>(Mprev0 + bh * sd + (int64_t)f * D + j);
+      const float4 b = *reinterpret_cast<const float4*>(Mprev0 + bh * sd + (int64_t)f * D + j + 4);
+      *reinterpret_cast<uint4*>(img + sw128_off(f, j, D)) =
+          make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+  const uint32_t base = smem_u32(smem);
+  constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, true);
+  bool ok = true;
+
+  // Every exit from the loop follows a block barrier and tests the CTA's
+  // abort flag, so all warps leave together; a wait that gives up only
+  // raises the flag.
+  float rf = 0.f, pf = 0.f;   // r_s and rho_s of this thread's row, read one step ahead
+  if (S > 0) {
+    rf = ratio[bh * S * D + f];
+    pf = rho[bh * S * D + f];
+  }
+  for (int s = 0; s < S; ++s) {
+    // the previous image store has finished reading B_hi before it is rewritten
+    if (f == 0) bulk_wait_read<0>();
+    fence_proxy_async_smem();   // the epilogue's rows of M'_s in the staging go out by TMA
+    __syncthreads();
+    if (*abort_flag) break;
+    if (f == 0 && s > 0) {
+      // M'_s (= Mst[s]), written over Bm_{s-1} in the staging, leaves by one
+      // TMA store; Bm_s may land once the store has read the staging
+      for (int b = 0; b < D / 32; ++b)
+        tma_store_2d(&map_m, smem + Cfg::kBmOff + b * Cfg::kFBox, b * 32, (int)((bh * (S + 1) + s) * D));
+      bulk_commit();
+      bulk_wait_read<0>();
+      load_bm(s);
+    }
+    // B = M'_s as hi + lo (row f = K index f, MN-major)
+#pragma unroll
+    for (int j = 0; j < D; j += 8) {
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        hi[t] = pack_bf16x2(m[j + 2 * t], m[j + 2 * t + 1]);
+        const float2 h2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi[t]));
+        lo[t] = pack_bf16x2(m[j + 2 * t] - h2.x, m[j + 2 * t + 1] - h2.y);
+      }
+      const uint32_t o = sw128_off(f, j, D);
+      *reinterpret_cast<uint4*>(smem + Cfg::kBhiOff + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(smem + Cfg::kBloOff + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+    // A = Cm_s in bf16 (K-major): warp w converts rows 32w .. 32w + 31, lane
+    // l columns 4l .. 4l + 3 of each (conflict-free staging reads)
+    ok = __all_sync(0xffffffffu, mbar_wait(c_full, s & 1, abort_flag, status));
+    if (ok) {
+#pragma unroll 4
+      for (int rr = 0; rr < 32; ++rr) {
+        const int row = warp * 32 + rr;
+        const float4 v = *reinterpret_cast<const float4*>(cst + row * D + 4 * lane);
+        *reinterpret_cast<uint2*>(smem + Cfg::kAOff + sw128_off(row, 4 * lane, D)) =
+            make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+      }
+    }
+    fence_proxy_async_smem();   // the operands are read by the tensor core and the bulk store
+    __syncthreads();
+    if (*abort_flag) break;
+    if (f == 0) {
+      // B_hi is the readout's image of M'_s (= Mst[s]), read by chunk s + 1
+      if (iout && s + 1 < S) {
+        bulk_store_1d(iout + (int64_t)(s + 1) * mat, smem + Cfg::kBhiOff, Cfg::kOp);
+        bulk_commit();
+      }
+      // the staging buffer has been converted: prefetch the next step's Cm
+      if (s + 1 < S) {
+        ++cloads;
+        mbar_arrive_expect_tx(c_full, Cfg::kStage);
+        bulk_load_1d(smem + Cfg::kCOff, Cm + (bh * S + s + 1) * mat, Cfg::kStage, c_full);
+      }
+      tc_fence_after();
+      const SDesc ad = sdesc_sw128_split(base + Cfg::kAOff, 16, 1024);
+      const SDesc bh_ = sdesc_sw128_split(base + Cfg::kBhiOff, D * 128, 1024);
+      const SDesc bl = sdesc_sw128_split(base + Cfg::kBloOff, D * 128, 1024);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t ka = (kk / 4) * Cfg::kBox + (kk % 4) * 32, kb = kk * 16 * 128;
+        umma_ss(tmem, sdesc_at(ad, ka), sdesc_at(bh_, kb), idesc, kk > 0 ? 1u : 0u);
+        umma_ss(tmem, sdesc_at(ad, ka), sdesc_at(bl, kb), idesc, 1u);
+      }
+      umma_commit(m_done);
+    }
+    float rn = 0.f, pn = 0.f;
+    if (s + 1 < S) {
+      rn = ratio[(bh * S + s + 1) * D + f];
+      pn = rho[(bh * S + s + 1) * D + f];
+    }
+    ok = __all_sync(0xffffffffu, mbar_wait(m_done, s & 1, abort_flag, status) &&
+                                     mbar_wait(b_full, s & 1, abort_flag, status));
+    tc_fence_after();
+    if (ok) {
+#pragma unroll
+      for (int cb = 0; cb < D / 32; ++cb) {
+        uint32_t acc[32];
+        tmem_ld32(lane_addr + cb * 32, acc);
+        float bv[32];
+        uint8_t* bbox = smem + Cfg::kBmOff + cb * Cfg::kFBox + f * 128;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {   // fp32 box: 16-byte chunk t of row f sits at chunk t ^ (f & 7)
+          const float4 v = *reinterpret_cast<const float4*>(bbox + ((t ^ (f & 7)) << 4));
+          bv[4 * t] = v.x; bv[4 * t + 1] = v.y; bv[4 * t + 2] = v.z; bv[4 * t + 3] = v.w;
+        }
+        tmem_wait_ld();
+#pragma unroll
+        for (int t = 0; t < 32; ++t)
+          m[cb * 32 + t] = fmaf(rf, m[cb * 32 + t], pf * (bv[t] - __uint_as_float(acc[t])));
+        // the new row goes where Bm's row was read: the staging becomes M'_{s+1}
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+          *reinterpret_cast<float4*>(bbox + ((t ^ (f & 7)) << 4)) =
+              make_float4(m[cb * 32 + 4 * t], m[cb * 32 + 4 * t + 1], m[cb * 32 + 4 * t + 2], m[cb * 32 + 4 * t + 3]);
+      }
+    }
+    rf = rn;
+    pf = pn;
+    tc_fence_before();
+  }
+  // the last state M'_{S+1} (= Mst[S]) from the staging
+  fence_proxy_async_smem();
+  __syncthreads();
+  if (f == 0 && S > 0 && !*abort_flag) {
+    for (int b = 0; b < D / 32; ++b)
+      tma_store_2d(&map_m, smem + Cfg::kBmOff + b * Cfg::kFBox, b * 32, (int)((bh * (S + 1) + S) * D));
+    bulk_commit();
+  }
+  if (f == 0) {
+    bulk_wait_all();
+    if (*abort_flag) {
+      // no MMA may still write TMEM and no copy still land when the CTA
+      // exits: the staging copies issued complete phases 0 .. n - 1
+      umma_commit(drain);
+      mbar_wait_drain(drain, 0);
+      if (cloads > 0) mbar_wait_drain(c_full, (cloads - 1) & 1);
+      if (bloads > 0) mbar_wait_drain(b_full, (bloads - 1) & 1);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 128);
 }
 
 // ------------------------------------------------------------------ host --
@@ -557,7 +896,7 @@ cudaError_t chunk_impl(const Problem& p, const void* vsrc, const void* ksrc, con
   cudaError_t e = cudaFuncSetAttribute(awm_chunk_tc_kernel<D, Mode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Cfg::kAlloc);
   if (e != cudaSuccess) return e;
-  awm_chunk_tc_kernel<D, Mode><<<dim3(p.S, p.B * p.H), 192, Cfg::kAlloc, st>>>(
+  awm_chunk_tc_kernel<D, Mode><<<dim3(p.S, p.B * p.H), kChunkThreads, Cfg::kAlloc, st>>>(
       mv, mkm, lse, out0, out1, (int)p.T, (int)p.c, (int)koff, p.status);
   return cudaGetLastError();
 }
@@ -570,24 +909,60 @@ cudaError_t readout_impl(const Problem& p, const Workspace& w, cudaStream_t st) 
   if (e != cudaSuccess) return e;
   EncodeTiledFn fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
-  CUtensorMap mq;   // Q_m as [B H T rows, D], boxes of [128 rows x 64] bf16, 128B swizzle
-  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)(p.B * p.H * p.T)};
-  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-  cuuint32_t box[2] = {64, 128};
+  // Q_m (load) and out_mem (store) as [B H T rows, D], boxes of [128 rows x 64] bf16, 128B swizzle
+  auto map = [&](CUtensorMap* m, const void* base) {
+    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)(p.B * p.H * p.T)};
+    cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  };
+  CUtensorMap mq, mo;
+  if (!map(&mq, p.qm) || !map(&mo, p.out_mem)) return cudaErrorInvalidValue;
+  const int64_t tiles = p.B * p.H * p.S * (p.c / 128);
+  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+  awm_readout_tc_kernel<D><<<grid, Cfg::kThreads, Cfg::kAlloc, st>>>(
+      mq, mo, w.Mimg, static_cast<__nv_bfloat16*>(p.out_mem), (int)p.T, (int)p.c, p.S, (int)(p.B * p.H),
+      p.state0 == nullptr ? 1 : 0, p.status);
+  return cudaGetLastError();
+}
+
+cudaError_t carry_tc_impl(const Problem& p, const Workspace& w, cudaStream_t st, bool images) {
+  using Cfg = CarryTcCfg;
+  cudaError_t e = cudaFuncSetAttribute(awm_carry_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kAlloc);
+  if (e != cudaSuccess) return e;
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  // Bm as [BH S d rows, d] fp32, boxes of [128 rows x 32] with 128B swizzle
+  CUtensorMap mb;
+  cuuint64_t dims[2] = {128, (cuuint64_t)(p.B * p.H * p.S * 128)};
+  cuuint64_t strides[1] = {128 * 4};
+  cuuint32_t box[2] = {32, 128};
   cuuint32_t estr[2] = {1, 1};
-  if (fn(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(p.qm), dims, strides, box, estr,
-         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+  if (fn(&mb, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, w.Bm, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+      CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  // split each chunk's 128-row tiles over G CTAs (up to 8 tiles per CTA)
-  const int n_tiles = (int)(p.c / 128);
-  const int G = n_tiles > 8 ? (n_tiles + 7) / 8 : 1;
-  awm_readout_tc_kernel<D><<<dim3(p.S, p.B * p.H, G), 128, Cfg::kAlloc, st>>>(
-      mq, w.Mst, static_cast<__nv_bfloat16*>(p.out_mem), (int)p.T, (int)p.c, p.state0, state_floats(D), p.status);
+  // Mst as [BH (S+1) d rows, d] fp32, the same boxes (the states leave by TMA store)
+  CUtensorMap mm;
+  cuuint64_t mdims[2] = {128, (cuuint64_t)(p.B * p.H * (p.S + 1) * 128)};
+  if (fn(&mm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, w.Mst, mdims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+      CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  awm_carry_tc_kernel<<<(unsigned)(p.B * p.H), 128, Cfg::kAlloc, st>>>(
+      mb, mm, w.Cm, w.ratio, w.rho, w.Mst, p.S, p.state0 ? p.state0 + 128 * 128 : nullptr, state_floats(128),
+      images ? w.Mimg : nullptr, p.state0, p.status);
   return cudaGetLastError();
 }
 
 }  // namespace
+
+cudaError_t launch_awm_carry_tc(const Problem& p, const Workspace& w, cudaStream_t st, bool images) {
+  return carry_tc_impl(p, w, st, images);
+}
 
 cudaError_t launch_awm_chunk_tc(const Problem& p, const Workspace& w, cudaStream_t st) {
   return p.d == 64 ? chunk_impl<64, kChunkFwd>(p, p.v, p.km, w.lse, w.Bm, w.Cm, st)

@@ -82,27 +82,30 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// 2^x for a pair of floats on the FMA pipe (no SFU).  Cody-Waite style range
-// reduction x = n + f with n = rint(x) (via the 1.5 * 2^23 rounding
-// constant) and f in [-1/2, 1/2], a cubic for 2^f, and n added to the
-// exponent field.  The cubic's coefficients were fitted for this library by
-// iteratively reweighted least squares (Lawson's method) on the relative
-// error over Chebyshev nodes of [-1/2, 1/2]; max relative error 7.5e-5,
-// below bf16 resolution (2^-9).  x is clamped to [-125, 126] so the exponent
-// arithmetic stays in the normal range; 2^-125 stands in for 0.
+__device__ __forceinline__ uint64_t fsub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for a pair of floats on the FMA pipe (no SFU), for x <= 126.  Cody-Waite
+// style range reduction x = n + f with n = rint(x) (adding and subtracting
+// the 1.5 * 2^23 rounding constant) and f in [-1/2, 1/2], a cubic for 2^f,
+// and n added to the exponent field.  The cubic's coefficients were fitted
+// for this library by iteratively reweighted least squares (Lawson's method)
+// on the relative error over Chebyshev nodes of [-1/2, 1/2]; max relative
+// error 7.5e-5, below bf16 resolution (2^-9).  x is clamped below at -125 so
+// the exponent arithmetic stays in the normal range; 2^-125 stands in for 0.
+// The softmax only passes x <= 8 (the lazy running max), so there is no
+// upper clamp.  Per pair: two scalar max, three packed add/sub, three packed
+// FMA and two shift-adds.
 __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
   float x0, x1;
   unpack2(x2, x0, x1);
-  x0 = fminf(fmaxf(x0, -125.f), 126.f);
-  x1 = fminf(fmaxf(x1, -125.f), 126.f);
   const uint64_t rnd = pack2(12582912.f, 12582912.f);    // 1.5 * 2^23
-  const uint64_t nrnd = pack2(-12582912.f, -12582912.f);
-  const uint64_t xc = pack2(x0, x1);
+  const uint64_t xc = pack2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
   const uint64_t t = fadd2(xc, rnd);                      // n in the low mantissa bits
-  const uint64_t n = fadd2(t, nrnd);                      // rint(x)
-  float n0, n1;
-  unpack2(n, n0, n1);
-  const uint64_t f = fadd2(xc, pack2(-n0, -n1));          // x - rint(x)
+  const uint64_t f = fsub2(xc, fsub2(t, rnd));            // x - rint(x)
   uint64_t p = ffma2(f, pack2(0.0551716685295105f, 0.0551716685295105f),
                      pack2(0.2426111400127411f, 0.2426111400127411f));
   p = ffma2(p, f, pack2(0.6932609677314758f, 0.6932609677314758f));
@@ -221,6 +224,21 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// 2D tiled bulk-tensor store from shared memory, tracked by the issuing
+// thread's bulk group (x the contiguous coordinate in elements, y the row).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
+               "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+               : "memory");
+}
+
+// Wait until at most N committed bulk stores of this thread are still
+// reading shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory"); }
+// Wait until every committed bulk store of this thread has completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // 3D tiled bulk-tensor store from shared memory (elements outside the
 // tensor are not written), tracked by the issuing thread's bulk group.
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* smem_src, int x, int y, int z) {
@@ -247,6 +265,14 @@ __device__ __forceinline__ void bulk_load_1d(void* smem_dst, const void* gsrc, u
                : "memory");
 }
 
+// Untiled bulk copy shared -> global, tracked by the issuing thread's bulk
+// group (16-byte aligned addresses, size a multiple of 16).
+__device__ __forceinline__ void bulk_store_1d(void* gdst, const void* smem_src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(smem_src)),
+               "r"(bytes)
+               : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until the committed bulk stores have finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
@@ -257,6 +283,14 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
+}
+
+// Byte offset of element (row, col) of a bf16 tile stored as 64-column
+// boxes of `rows` rows each with 128-byte swizzle (the TMA SWIZZLE_128B
+// layout, and the canonical K-major / MN-major UMMA operand layout).
+__device__ __forceinline__ uint32_t sw128_off(int row, int col, int rows) {
+  const int box = col >> 6, cc = col & 63;
+  return box * rows * 128 + row * 128 + ((((cc >> 3) ^ (row & 7)) << 4)) + ((cc & 7) << 1);
 }
 
 // --------------------------------------------------------------- tcgen05 --

@@ -33,7 +33,8 @@ size_t workspace_bytes(int64_t BH, int64_t T, int64_t c, int64_t d) {
   const size_t vec = al(sizeof(float) * BH * S * d);
   const size_t mat = al(sizeof(float) * BH * S * d * d);
   const size_t mst = al(sizeof(float) * BH * (S + 1) * d * d);
-  return part + 4 * vec + 2 * mat + mst;
+  const size_t img = al(sizeof(uint16_t) * BH * (S + 1) * d * d);
+  return part + 4 * vec + 2 * mat + mst + img;
 }
 
 Workspace carve_workspace(void* base, int64_t BH, int64_t T, int64_t c, int64_t d) {
@@ -59,6 +60,8 @@ Workspace carve_workspace(void* base, int64_t BH, int64_t T, int64_t c, int64_t 
   w.Cm = reinterpret_cast<float*>(p);
   p += mat;
   w.Mst = reinterpret_cast<float*>(p);
+  p += al(sizeof(float) * BH * (S + 1) * d * d);
+  w.Mimg = reinterpret_cast<uint16_t*>(p);
   return w;
 }
 
@@ -308,7 +311,9 @@ int run_forward(const void* q, const void* k, const void* v, const void* qm, con
   if ((rc = check_cuda(use_tc ? launch_awm_chunk_tc(p, w, st) : launch_awm_chunk_simt(p, w, st), "awm chunk")))
     return rc;
   ev.mark(2);
-  if ((rc = check_cuda(launch_awm_carry(p, w, st), "awm carry"))) return rc;
+  if ((rc = check_cuda(use_tc && d == 128 ? launch_awm_carry_tc(p, w, st, true) : launch_awm_carry(p, w, st, use_tc),
+                       "awm carry")))
+    return rc;
   ev.mark(3);
   if ((rc = check_cuda(use_tc ? launch_awm_readout_tc(p, w, st) : launch_awm_readout_simt(p, w, st),
                        "awm readout")))
@@ -675,7 +680,9 @@ extern "C" int gecko_sca_awm_forward_noalloc(const void* q, const void* k, const
   if ((rc = check_cuda(launch_awm_stats(p, w, st), "awm stats"))) return rc;
   if ((rc = check_cuda(use_tc ? launch_awm_chunk_tc(p, w, st) : launch_awm_chunk_simt(p, w, st), "awm chunk")))
     return rc;
-  if ((rc = check_cuda(launch_awm_carry(p, w, st), "awm carry"))) return rc;
+  if ((rc = check_cuda(use_tc && d == 128 ? launch_awm_carry_tc(p, w, st, true) : launch_awm_carry(p, w, st, use_tc),
+                       "awm carry")))
+    return rc;
   if ((rc = check_cuda(use_tc ? launch_awm_readout_tc(p, w, st) : launch_awm_readout_simt(p, w, st),
                        "awm readout")))
     return rc;

@@ -28,7 +28,7 @@ struct Problem {
 // Floats per (b, h) in a carried state record: M'_prev, M'_cur (d x d each), log z (d).
 inline int64_t state_floats(int64_t d) { return 2 * d * d + d; }
 
-// Device workspace carved out of one allocation (all fp32).
+// Device workspace carved out of one allocation (fp32 but for Mimg).
 struct Workspace {
   float2* part;  // [BH, T / R, d]  (max, sum exp(x - max)) of K_m per block of R rows
   float* lse;    // [BH, S, d]  log of per-chunk exp-sums of K_m
@@ -38,6 +38,11 @@ struct Workspace {
   float* Bm;     // [BH, S, d, d]  Phi~_s^T V_s    (Phi~_s = exp(Km_s - lse_s))
   float* Cm;     // [BH, S, d, d]  Phi~_s^T Psi_s
   float* Mst;    // [BH, S+1, d, d]  M'_1 .. M'_{S+1}
+  // [BH, S+1, d * d] bf16 bits: image s is the readout's B operand for
+  // chunk s (0-based), i.e. M'_{s-1} (1-based) = Mst[s - 1] for s >= 1 and
+  // the carried M'_prev for s = 0, as bf16 in the 128-byte-swizzled
+  // MN-major layout (64-column boxes of d rows).  Written by the carry.
+  uint16_t* Mimg;
 };
 
 // Column slices of the sequential carries: as wide as still gives about one
@@ -59,15 +64,21 @@ Workspace carve_workspace(void* base, int64_t BH, int64_t T, int64_t c, int64_t 
 // CUDA-core kernels (any dtype, any c % 64 == 0).
 cudaError_t launch_awm_stats(const Problem& p, const Workspace& w, cudaStream_t st);   // lse + log z prefix
 cudaError_t launch_awm_chunk_simt(const Problem& p, const Workspace& w, cudaStream_t st);
-cudaError_t launch_awm_carry(const Problem& p, const Workspace& w, cudaStream_t st);
+// images: also write the readout operand images (Workspace::Mimg)
+cudaError_t launch_awm_carry(const Problem& p, const Workspace& w, cudaStream_t st, bool images = false);
 cudaError_t launch_awm_readout_simt(const Problem& p, const Workspace& w, cudaStream_t st);
 cudaError_t launch_sca_simt(const Problem& p, cudaStream_t st);
+
+// Streaming multiprocessors of the current device (queried once).
+int sm_count();
 
 // Tensor-core (tcgen05 + TMEM + TMA) kernels, bf16 with c % 128 == 0.
 bool tc_supported(const Problem& p);
 cudaError_t launch_sca_tc(const Problem& p, cudaStream_t st);
 cudaError_t launch_awm_chunk_tc(const Problem& p, const Workspace& w, cudaStream_t st);
 cudaError_t launch_awm_readout_tc(const Problem& p, const Workspace& w, cudaStream_t st);
+// The carry on the tensor cores (d = 128; bf16 hi + lo operands, ~fp32 products)
+cudaError_t launch_awm_carry_tc(const Problem& p, const Workspace& w, cudaStream_t st, bool images);
 // Bm, Cm with each computed operand as bf16 hi + lo (near-fp32 products for the backward)
 cudaError_t launch_awm_chunk_tc_split(const Problem& p, const Workspace& w, cudaStream_t st);
 // E_s = psi(Qm_s)^T dO_m,s for chunks 3..S, hi + lo operands

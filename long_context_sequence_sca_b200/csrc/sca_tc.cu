@@ -7,15 +7,16 @@
 // with scale 1, a causal mask inside the current chunk, and no previous chunk
 // for chunk 1.  Requires bf16, d in {64, 128}, c % 128 == 0.
 //
-// Design (one persistent CTA per SM, 320 threads):
+// Design (one persistent CTA per SM, 384 threads in three warpgroups):
 //   warp 0      TMA producer: Q tiles once per work unit; K and V tiles of
-//               128 keys through rings of shared-memory stages (K one
-//               stage deeper than V), loads issued in the order of the
-//               iterations that free their slots.
+//               128 keys through rings of shared-memory stages, loads issued
+//               in the order of the iterations that free their slots.
 //   warp 1      TMEM allocator and MMA issuer (one thread): S_i = Q_i K_j^T
 //               (SS form) into TMEM, O_i += P_i V_j with P_i read from TMEM
 //               (TS form).
-//   warps 2-5   softmax for query tile 0, warps 6-9 for query tile 1; one
+//   warps 2-3   idle (they complete the first warpgroup, whose registers
+//               setmaxnreg hands to the softmax warpgroups).
+//   warps 4-7   softmax for query tile 0, warps 8-11 for query tile 1; one
 //               thread per query row (TMEM lane quarter = warp % 4); online
 //               max/sum in registers; P written back to TMEM as bf16 over the
 //               S columns; epilogue O / l.
@@ -42,7 +43,19 @@ namespace {
 
 constexpr int kBM = 128;   // query rows per tile
 constexpr int kBN = 128;   // keys per tile
-constexpr int kThreads = 320;   // 10 warps: TMA, MMA (+TMEM allocation), 2 x 4 softmax
+// Warp layout.  GECKO_SCA_WG3=1 (default): 12 warps in three warpgroups
+// (TMA, MMA and two idle warps; softmax of tile 0; softmax of tile 1), and
+// setmaxnreg moves registers from the first warpgroup to the softmax
+// warpgroups (88 and 2 x 208 per thread).  With 10 warps two SM
+// sub-partitions hold three warps each, which caps every thread at 168
+// registers; the 12-warp layout measured 2.76-2.77 ms against 2.86-2.90 ms
+// per launch on the bench workload.  GECKO_SCA_WG3=0 keeps the 10-warp layout.
+#ifndef GECKO_SCA_WG3
+#define GECKO_SCA_WG3 1
+#endif
+constexpr int kThreads = GECKO_SCA_WG3 ? 384 : 320;   // TMA, MMA (+TMEM allocation), [2 idle], 2 x 4 softmax
+constexpr int kSoftmaxWarp0 = GECKO_SCA_WG3 ? 4 : 2;  // first softmax warp
+constexpr int kRegsCtl = 88, kRegsSoftmax = 208;      // per-thread registers after setmaxnreg (GECKO_SCA_WG3)
 // Of every 8 exponential pairs, GECKO_SFU_PAIRS are evaluated on the SFU
 // (ex2.approx) and the rest on the FMA pipe (exp2_poly2).  Measured on B200
 // with the bench workload the all-SFU setting is fastest (the polynomial
@@ -52,14 +65,28 @@ constexpr int kThreads = 320;   // 10 warps: TMA, MMA (+TMEM allocation), 2 x 4 
 #define GECKO_SFU_PAIRS 8
 #endif
 constexpr int kSfuPairs = GECKO_SFU_PAIRS;
+// GECKO_SCA_ONEPASS=1: the softmax reads each S tile from TMEM once into
+// registers (row max and exponentials from the same registers) instead of
+// streaming it twice (needs the 12-warp layout's registers).  Measured
+// slower than two passes (2.81-2.83 against 2.76-2.77 ms), so off by default.
+#ifndef GECKO_SCA_ONEPASS
+#define GECKO_SCA_ONEPASS 0
+#endif
+// Register budget of the kernel: the default lets the compiler fit 320
+// threads on one SM; GECKO_SCA_MAXNREG caps registers per thread instead.
+#ifdef GECKO_SCA_MAXNREG
+#define SCA_BOUNDS __maxnreg__(GECKO_SCA_MAXNREG)
+#else
+#define SCA_BOUNDS __launch_bounds__(kThreads, 1)
+#endif
 
 // Units are claimed dynamically from a global counter, in the schedule's
 // order, by each CTA's TMA thread, which publishes them to the CTA's other
 // roles through a ring of kUnitRing slots.  The producer claims at most
-// kKStages + 1 units ahead of the slowest reader (its K loads lead the MMAs
-// by at most kKStages iterations, every unit has at least one, and the
-// softmax warps trail the MMA thread by at most one unit), so 8 slots are
-// never overwritten before they are read.
+// max(kKStages, kVStages) + 1 units ahead of the slowest reader (its K and V
+// loads lead the MMAs by at most that many iterations, every unit has at
+// least one, and the softmax warps trail the MMA thread by at most one
+// unit), so 8 slots are never overwritten before they are read.
 constexpr int kUnitRing = 8;
 
 // Next unit to claim (reset to 0 on the launching stream before each launch;
@@ -70,21 +97,32 @@ template <int D>
 struct ScaCfg {
   static constexpr int kTileBytes = 128 * D * 2;       // 128 rows x D bf16, D/64 swizzled boxes
   static constexpr int kBoxBytes = 128 * 64 * 2;       // one [128 x 64] box
-  // K ring one stage deeper than the V ring: K_m is read at the start of
-  // iteration m, V_m only at the start of iteration m + 1, so with equal
-  // rings K would get one iteration less to arrive (at d = 128 shared
-  // memory holds Q, 3 K and 2 V tiles: 224 KB).
-  static constexpr int kKStages = D == 64 ? 5 : 3;
-  static constexpr int kVStages = D == 64 ? 4 : 2;
-  static_assert(kKStages >= kVStages, "the iteration-done ring has kKStages slots");
-  static_assert(kKStages + 2 <= kUnitRing, "unit ring too short for the K lead");
+  // Ring depths.  At d = 128 shared memory holds Q (two tiles) and five K/V
+  // tiles (224 KB): 2 K and 3 V stages measured ~1 % faster than 3 K and 2 V
+  // on the bench workload (2.72-2.76 against 2.76-2.77 ms per launch), and a
+  // K ring of 2 alone cost nothing, so V waits were the ones worth shortening.
+  // At d = 64 tiles are half the size: 5 K and 4 V stages.
+#ifdef GECKO_SCA_KSTAGES
+  static constexpr int kKStages = D == 64 ? 5 : GECKO_SCA_KSTAGES;
+#else
+  static constexpr int kKStages = D == 64 ? 5 : 2;
+#endif
+#ifdef GECKO_SCA_VSTAGES
+  static constexpr int kVStages = D == 64 ? 4 : GECKO_SCA_VSTAGES;
+#else
+  static constexpr int kVStages = D == 64 ? 4 : 3;
+#endif
+  // it_done has one slot per K/V iteration in flight: the deeper of the two rings
+  static constexpr int kIterRing = kKStages > kVStages ? kKStages : kVStages;
+  static_assert(kIterRing + 2 <= kUnitRing, "unit ring too short for the K/V lead");
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + 2 * kTileBytes;
   static constexpr int kVOff = kKOff + kKStages * kTileBytes;
   static constexpr int kBarOff = kVOff + kVStages * kTileBytes;
-  // q_full, q_empty, k_full[KS], it_done[KS], v_full[VS], s_full[2],
+  // q_full, q_empty, k_full[KS], it_done[max(KS, VS)], v_full[VS], s_full[2],
   // p_full[2], o_full[2], o_empty[2], drain, unit_ready[kUnitRing]
-  static constexpr int kNumBars = 2 + 2 * kKStages + kVStages + 8 + 1 + kUnitRing;
+  static constexpr int kNumBars = 2 + kKStages + (kKStages > kVStages ? kKStages : kVStages) + kVStages + 8 + 1 +
+                                  kUnitRing;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   // tmem address, abort flag, then the unit ring (kUnitRing uint32)
   static constexpr int kBytes = kMiscOff + 8 + 4 * kUnitRing;
@@ -149,6 +187,11 @@ __device__ __forceinline__ Unit decode_unit(int u, int BH, int T, int c, int kof
   return U;
 }
 
+// Key-tile range of query tile i of a unit, selected by value so that a
+// runtime i does not force the unit into local memory.
+__device__ __forceinline__ int ubeg(const Unit& U, int i) { return i ? U.beg[1] : U.beg[0]; }
+__device__ __forceinline__ int uend(const Unit& U, int i) { return i ? U.end[1] : U.end[0]; }
+
 // The TMA thread's claims: ordinal n of this CTA's work is unit
 // slot[n % kUnitRing]; a claim takes the next unit of the global counter
 // (n_units once all are taken, the end marker), writes it to its slot and
@@ -202,14 +245,121 @@ __device__ __forceinline__ void kv_walk_next(KvWalk& w, Claims& cl, int BH, int 
   }
 }
 
+// Pass 2 of the softmax of one 128-key S tile for this thread's row: p =
+// 2^(s log2e - m_ref) in chunks of 32 columns (the next chunk's TMEM load is
+// in flight while this one is computed), P as bf16 written over the
+// consumed S columns, and the row sum of p returned.  The argument uses
+// packed FMA; on tiles off the diagonal, of every 8 pairs kSfuPairs go to
+// the SFU (ex2.approx) and the rest to the FMA pipe (exp2_poly2).  The
+// diagonal tile masks keys after the row (r = row in the tile) and takes
+// every exponential on the SFU, so masked keys give exactly 0.
+template <bool kDiag>
+__device__ __forceinline__ float softmax_pass2(uint32_t s_addr, float m_ref, int r) {
+  const uint64_t l2e2 = pack2(kLog2e, kLog2e);
+  const uint64_t nm2 = pack2(-m_ref, -m_ref);
+  uint64_t acc2[2] = {pack2(0.f, 0.f), pack2(0.f, 0.f)};
+  uint32_t cur[32], nxt[32];
+  tmem_ld32p(s_addr, cur);
+#pragma unroll
+  for (int cb = 0; cb < kBN / 32; ++cb) {
+    tmem_wait_ld();
+    if (cb + 1 < kBN / 32) tmem_ld32p(s_addr + (cb + 1) * 32, nxt);
+    if (kDiag) {
+#pragma unroll
+      for (int x = 0; x < 32; ++x)
+        if (cb * 32 + x > r) cur[x] = __float_as_uint(-INFINITY);
+    }
+    uint32_t pk[16];
+#pragma unroll
+    for (int x = 0; x < 16; ++x) {
+      const uint64_t a2 = ffma2(pack2(__uint_as_float(cur[2 * x]), __uint_as_float(cur[2 * x + 1])), l2e2, nm2);
+      uint64_t p2;
+      if (kDiag || x % 8 < kSfuPairs) {
+        float a0, a1;
+        unpack2(a2, a0, a1);
+        p2 = pack2(ex2(a0), ex2(a1));
+      } else {
+        p2 = exp2_poly2(a2);
+      }
+      acc2[x & 1] = fadd2(acc2[x & 1], p2);
+      float p0, p1;
+      unpack2(p2, p0, p1);
+      pk[x] = pack_bf16x2(p0, p1);
+    }
+    tmem_st16(s_addr + cb * 16, pk);
+    if (cb + 1 < kBN / 32) {
+#pragma unroll
+      for (int x = 0; x < 32; ++x) cur[x] = nxt[x];
+    }
+  }
+  tmem_wait_st();
+  float a0, a1, b0, b1;
+  unpack2(acc2[0], a0, a1);
+  unpack2(acc2[1], b0, b1);
+  return (a0 + a1) + (b0 + b1);
+}
+
+#if GECKO_SCA_ONEPASS
+// Max of a 128-column score row held in registers (8 independent chains).
+__device__ __forceinline__ float row_max128(const uint32_t* sr) {
+  float mp[8];
+#pragma unroll
+  for (int y = 0; y < 8; ++y) mp[y] = fmax3(__uint_as_float(sr[y]), __uint_as_float(sr[y + 8]), __uint_as_float(sr[y + 16]));
+#pragma unroll
+  for (int x = 24; x + 16 < 128; x += 16)
+#pragma unroll
+    for (int y = 0; y < 8; ++y) mp[y] = fmax3(mp[y], __uint_as_float(sr[x + y]), __uint_as_float(sr[x + 8 + y]));
+#pragma unroll
+  for (int y = 0; y < 8; ++y) mp[y] = fmaxf(mp[y], __uint_as_float(sr[120 + y]));
+  return fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
+}
+
+// The exponential pass of softmax_pass2 on a row already in registers
+// (masked entries set to -inf by the caller): P (bf16) written over the S
+// columns 32 scores at a time, the row sum returned.
+template <bool kDiag>
+__device__ __forceinline__ float softmax_exp_regs(const uint32_t* sr, uint32_t s_addr, float m_ref) {
+  const uint64_t l2e2 = pack2(kLog2e, kLog2e);
+  const uint64_t nm2 = pack2(-m_ref, -m_ref);
+  uint64_t acc2[2] = {pack2(0.f, 0.f), pack2(0.f, 0.f)};
+#pragma unroll
+  for (int cb = 0; cb < kBN / 32; ++cb) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int x = 0; x < 16; ++x) {
+      const uint64_t a2 = ffma2(pack2(__uint_as_float(sr[cb * 32 + 2 * x]), __uint_as_float(sr[cb * 32 + 2 * x + 1])),
+                                l2e2, nm2);
+      uint64_t p2;
+      if (kDiag || x % 8 < kSfuPairs) {
+        float a0, a1;
+        unpack2(a2, a0, a1);
+        p2 = pack2(ex2(a0), ex2(a1));
+      } else {
+        p2 = exp2_poly2(a2);
+      }
+      acc2[x & 1] = fadd2(acc2[x & 1], p2);
+      float p0, p1;
+      unpack2(p2, p0, p1);
+      pk[x] = pack_bf16x2(p0, p1);
+    }
+    tmem_st16(s_addr + cb * 16, pk);
+  }
+  tmem_wait_st();
+  float a0, a1, b0, b1;
+  unpack2(acc2[0], a0, a1);
+  unpack2(acc2[1], b0, b1);
+  return (a0 + a1) + (b0 + b1);
+}
+#endif
+
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void SCA_BOUNDS
 sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
               const __grid_constant__ CUtensorMap map_v, __nv_bfloat16* __restrict__ out,
               float* __restrict__ lse, __nv_bfloat16* __restrict__ out_lo, int T, int c, int BH,
               int n_units, int koff, unsigned* unit_counter, int* status) {
   using Cfg = ScaCfg<D>;
-  constexpr int KS = Cfg::kKStages, VS = Cfg::kVStages;
+  constexpr int KS = Cfg::kKStages, VS = Cfg::kVStages, IR = Cfg::kIterRing;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + Cfg::kQOff;
@@ -219,10 +369,10 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
   uint64_t* k_full = bars + 2;
-  // it_done[m % KS] completes when the MMAs of K/V iteration m are done:
+  // it_done[m % IR] completes when the MMAs of K/V iteration m are done:
   // they were the last readers of K_m and of V_{m-1}
   uint64_t* it_done = k_full + KS;
-  uint64_t* v_full = it_done + KS;
+  uint64_t* v_full = it_done + IR;
   uint64_t* s_full = v_full + VS;
   uint64_t* p_full = s_full + 2;
   uint64_t* o_full = p_full + 2;
@@ -239,10 +389,8 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int s = 0; s < KS; ++s) {
-      mbar_init(k_full + s, 1);
-      mbar_init(it_done + s, 1);
-    }
+    for (int s = 0; s < KS; ++s) mbar_init(k_full + s, 1);
+    for (int s = 0; s < IR; ++s) mbar_init(it_done + s, 1);
     for (int s = 0; s < VS; ++s) mbar_init(v_full + s, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + i, 1);
@@ -270,6 +418,9 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   const uint32_t tmem = *tmem_slot;
 
 
+#if GECKO_SCA_WG3
+  if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegsCtl));
+#endif
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
     if (lane == 0) {
@@ -309,7 +460,7 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           ++qn;
           qu = cl.unit_of(qn);
         } else if (tV <= tK) {
-          if (tV >= 0 && !(ok = mbar_wait(it_done + tV % KS, (uint32_t)(tV / KS) & 1, abort_flag, status))) break;
+          if (tV >= 0 && !(ok = mbar_wait(it_done + tV % IR, (uint32_t)(tV / IR) & 1, abort_flag, status))) break;
           const int st = vw.it % VS;
           const int row = (int)(vw.kvbase + (int64_t)vw.j * kBN);
           mbar_arrive_expect_tx(v_full + st, Cfg::kTileBytes);
@@ -317,7 +468,7 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
             tma_load_2d(sV + st * Cfg::kTileBytes + b * Cfg::kBoxBytes, &map_v, v_full + st, b * 64, row);
           kv_walk_next(vw, cl, BH, T, c, koff);
         } else {
-          if (tK >= 0 && !(ok = mbar_wait(it_done + tK % KS, (uint32_t)(tK / KS) & 1, abort_flag, status))) break;
+          if (tK >= 0 && !(ok = mbar_wait(it_done + tK % IR, (uint32_t)(tK / IR) & 1, abort_flag, status))) break;
           const int st = kw.it % KS;
           const int row = (int)(kw.kvbase + (int64_t)kw.j * kBN);
           mbar_arrive_expect_tx(k_full + st, Cfg::kTileBytes);
@@ -343,7 +494,8 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, false, true);
       const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK), va = smem_u32(sV);
-      uint32_t kv_it = 0, p_cnt[2] = {0, 0}, o_cnt[2] = {0, 0};
+      // bit i: the phase parity of tile i's p_full and o_empty waits
+      uint32_t kv_it = 0, p_par = 0, o_par = 0;
       int n = 0;
       bool ok = true;
       for (;; ++n) {
@@ -366,25 +518,25 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           for (int i = 0; i < U.nt && ok; ++i) {
             const uint32_t colS = i == 0 ? Cfg::kColS0 : Cfg::kColS1;
             const uint32_t colO = i == 0 ? Cfg::kColO0 : Cfg::kColO1;
-            if (j - 1 >= U.beg[i] && j - 1 < U.end[i]) {
+            if (j - 1 >= ubeg(U, i) && j - 1 < uend(U, i)) {
               // O_i += P_i V_{j-1}
-              if (j - 1 == U.beg[i]) {
-                if (!(ok = mbar_wait(o_empty + i, (o_cnt[i] & 1) ^ 1, abort_flag, status))) break;
+              if (j - 1 == ubeg(U, i)) {
+                if (!(ok = mbar_wait(o_empty + i, ((o_par >> i) & 1) ^ 1, abort_flag, status))) break;
               }
-              if (!(ok = mbar_wait(p_full + i, p_cnt[i] & 1, abort_flag, status))) break;
-              ++p_cnt[i];
+              if (!(ok = mbar_wait(p_full + i, (p_par >> i) & 1, abort_flag, status))) break;
+              p_par ^= 1u << i;
               tc_fence_after();
               const SDesc vd = sdesc_sw128_split(va + stV * Cfg::kTileBytes, Cfg::kBoxBytes, 1024);
-              umma_ts(tmem + colO, tmem + colS, sdesc_at(vd, 0), idesc_pv, j - 1 > U.beg[i] ? 1u : 0u);
+              umma_ts(tmem + colO, tmem + colS, sdesc_at(vd, 0), idesc_pv, j - 1 > ubeg(U, i) ? 1u : 0u);
 #pragma unroll
               for (int kk = 1; kk < kBN / 16; ++kk)
                 umma_ts(tmem + colO, tmem + colS + kk * 8, sdesc_at(vd, kk * 2048), idesc_pv, 1u);
-              if (j - 1 == U.end[i] - 1) {
+              if (j - 1 == uend(U, i) - 1) {
                 umma_commit(o_full + i);
-                ++o_cnt[i];
+                o_par ^= 1u << i;
               }
             }
-            if (j >= U.beg[i] && j < U.end[i]) {
+            if (j >= ubeg(U, i) && j < uend(U, i)) {
               if (!k_ready) {
                 if (!(ok = mbar_wait(k_full + stK, (kv_it / KS) & 1, abort_flag, status))) break;
                 tc_fence_after();
@@ -416,9 +568,12 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       mbar_wait_drain(drain, 0);
     }
     __syncwarp();
-  } else {
+  } else if (warp >= kSoftmaxWarp0) {
+#if GECKO_SCA_WG3
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kRegsSoftmax));
+#endif
     // ------------------------------------------------ softmax warpgroups --
-    const int i = (warp - 2) / 4;           // query tile handled by this warpgroup
+    const int i = (warp - kSoftmaxWarp0) / 4;   // query tile handled by this warpgroup
     const int r = (warp % 4) * 32 + lane;   // row within the tile = TMEM lane
     const uint32_t lane_addr = tmem + ((uint32_t)((warp % 4) * 32) << 16);
     const uint32_t colS = i == 0 ? Cfg::kColS0 : Cfg::kColS1;
@@ -437,17 +592,30 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       it_base += (uint32_t)(je - jb);
       if (i >= U.nt) continue;
       float m_ref = 0.f, l = 0.f;
-      for (int j = U.beg[i]; j < U.end[i]; ++j) {
+      for (int j = ubeg(U, i); j < uend(U, i); ++j) {
         ok = __all_sync(0xffffffffu, mbar_wait(s_full + i, s_cnt & 1, abort_flag, status));
         if (!ok) break;
         // The QK of the iteration's last active tile is its last MMA, so its
         // completion (just observed) means K_j and V_{j-1} are no longer read:
         // one thread of that tile's warpgroup releases them to the producer.
         if ((i == 1 || !(U.nt == 2 && j >= U.beg[1])) && warp % 4 == 2 && lane == 0)
-          mbar_arrive(it_done + (unit_it0 + (uint32_t)(j - jb)) % KS);
+          mbar_arrive(it_done + (unit_it0 + (uint32_t)(j - jb)) % IR);
         ++s_cnt;
         tc_fence_after();
-        const bool diag = j == U.end[i] - 1;
+        const bool diag = j == uend(U, i) - 1;
+#if GECKO_SCA_ONEPASS
+        // the whole S row in registers: one TMEM read, one wait
+        uint32_t sr[kBN];
+#pragma unroll
+        for (int h = 0; h < kBN / 32; ++h) tmem_ld32p(lane_addr + colS + h * 32, sr + h * 32);
+        tmem_wait_ld();
+        if (diag) {
+#pragma unroll
+          for (int x = 0; x < kBN; ++x)
+            if (x > r) sr[x] = __float_as_uint(-INFINITY);
+        }
+        const float mt = row_max128(sr);
+#else
         // pass 1: row max, streaming S out of TMEM 64 columns at a time
         float mt = -INFINITY;
 #pragma unroll
@@ -473,9 +641,10 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           for (int y = 0; y < 8; ++y) mp[y] = fmaxf(mp[y], __uint_as_float(sr[56 + y]));
           mt = fmax3(mt, fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7])), -INFINITY);
         }
+#endif
         const float m2 = mt * kLog2e;
-        const bool grow = j != U.beg[i] && m2 > m_ref + 8.f;
-        if (j == U.beg[i]) m_ref = m2;
+        const bool grow = j != ubeg(U, i) && m2 > m_ref + 8.f;
+        if (j == ubeg(U, i)) m_ref = m2;
         // O is rescaled with warp-collective TMEM loads and stores, so the
         // whole warp takes this branch when any of its rows needs it (the
         // other rows scale by 1)
@@ -495,55 +664,13 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
             tmem_st32(lane_addr + colO + cb * 32, o);
           }
         }
-        // pass 2: p = 2^(s log2e - m_ref) in chunks of 32 columns (the next
-        // chunk's TMEM load is in flight while this one is computed).  The
-        // argument uses packed FMA; of every 8 pairs, kSfuPairs go to the SFU
-        // and the rest to the FMA pipe (exp2_poly2).  P (bf16) overwrites
-        // the already-consumed S columns.
-        const uint64_t l2e2 = pack2(kLog2e, kLog2e);
-        const uint64_t nm2 = pack2(-m_ref, -m_ref);
-        uint64_t acc2[2] = {pack2(0.f, 0.f), pack2(0.f, 0.f)};
-        uint32_t cur[32], nxt[32];
-        tmem_ld32p(lane_addr + colS, cur);
-#pragma unroll
-        for (int cb = 0; cb < kBN / 32; ++cb) {
-          tmem_wait_ld();
-          if (cb + 1 < kBN / 32) tmem_ld32p(lane_addr + colS + (cb + 1) * 32, nxt);
-          if (diag) {
-#pragma unroll
-            for (int x = 0; x < 32; ++x)
-              if (cb * 32 + x > r) cur[x] = __float_as_uint(-INFINITY);
-          }
-          uint32_t pk[16];
-#pragma unroll
-          for (int x = 0; x < 16; ++x) {
-            const uint64_t a2 = ffma2(pack2(__uint_as_float(cur[2 * x]), __uint_as_float(cur[2 * x + 1])), l2e2, nm2);
-            uint64_t p2;
-            if (x % 8 < kSfuPairs) {
-              float a0, a1;
-              unpack2(a2, a0, a1);
-              p2 = pack2(ex2(a0), ex2(a1));
-            } else {
-              p2 = exp2_poly2(a2);
-            }
-            acc2[x & 1] = fadd2(acc2[x & 1], p2);
-            float p0, p1;
-            unpack2(p2, p0, p1);
-            pk[x] = pack_bf16x2(p0, p1);
-          }
-          tmem_st16(lane_addr + colS + cb * 16, pk);
-          if (cb + 1 < kBN / 32) {
-#pragma unroll
-            for (int x = 0; x < 32; ++x) cur[x] = nxt[x];
-          }
-        }
-        tmem_wait_st();
-        {
-          float a0, a1, b0, b1;
-          unpack2(acc2[0], a0, a1);
-          unpack2(acc2[1], b0, b1);
-          l += (a0 + a1) + (b0 + b1);
-        }
+        // pass 2: p = 2^(s log2e - m_ref), P (bf16) written over the consumed
+        // S columns, row sum into l
+#if GECKO_SCA_ONEPASS
+        l += diag ? softmax_exp_regs<true>(sr, lane_addr + colS, m_ref) : softmax_exp_regs<false>(sr, lane_addr + colS, m_ref);
+#else
+        l += diag ? softmax_pass2<true>(lane_addr + colS, m_ref, r) : softmax_pass2<false>(lane_addr + colS, m_ref, r);
+#endif
         tc_fence_before();
         mbar_arrive(p_full + i);
       }
@@ -627,16 +754,6 @@ cudaError_t make_map(CUtensorMap* m, const void* base, int64_t rows, int d) {
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-int sm_count() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
 
 template <int D>
 cudaError_t launch_sca_tc_impl(const Problem& p, cudaStream_t st) {
@@ -666,6 +783,17 @@ cudaError_t launch_sca_tc_impl(const Problem& p, cudaStream_t st) {
 }
 
 }  // namespace
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
 
 bool tc_supported(const Problem& p) {
   if (p.dtype != kBF16 || p.c % 128 != 0) return false;

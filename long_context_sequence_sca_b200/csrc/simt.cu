@@ -103,8 +103,9 @@ __global__ void __launch_bounds__(D) awm_lse_combine_kernel(const float2* __rest
 }
 
 // ------------------------------------------------------------------------
-// Prefix over chunks in fp64: log z^s = logaddexp(log z^{s-1}, lse_s), the
-// row ratio r_s = z^{s-1}/z^s (0 for s = 1) and the chunk weight
+// Prefix over chunks: log z^s = logaddexp(log z^{s-1}, lse_s) with the
+// running sum in fp64, the row ratio r_s = z^{s-1}/z^s (0 for s = 1) and the
+// chunk weight
 // rho_s = e_s / z^s = exp(lse_s - log z^s).  A continued sequence seeds the
 // prefix with the carried log z (logz0, stride sd per (b, h)).  grid BH, D
 // threads.
@@ -123,12 +124,15 @@ __global__ void __launch_bounds__(D) awm_prefix_kernel(const float* __restrict__
     if (s == 0 && !seeded) {
       Ln = e;
     } else {
+      // the running sum stays in fp64; the correction log(1 + e^(lo - hi))
+      // lies in [0, ln 2] and is accurate to fp32 rounding
       const double hi = fmax(L, e), lo = fmin(L, e);
-      Ln = hi + log1p(exp(lo - hi));
+      Ln = hi + (double)log1pf(expf((float)(lo - hi)));
     }
     logz[o] = (float)Ln;
-    ratio[o] = (s == 0 && !seeded) ? 0.f : (float)exp(L - Ln);
-    rho[o] = (float)exp(e - Ln);
+    // both exponents are <= 0 (log z is non-decreasing and >= lse)
+    ratio[o] = (s == 0 && !seeded) ? 0.f : expf((float)(L - Ln));
+    rho[o] = expf((float)(e - Ln));
     L = Ln;
   }
 }
@@ -245,13 +249,27 @@ struct CarryStage {
   static constexpr int kFloats = kP + D;
 };
 
+// The thread's RB x CB block of a d x d matrix as bf16 into a readout
+// operand image (128-byte-swizzled MN-major, 64-column boxes of D rows).
+template <int D, int RB, int CB>
+__device__ __forceinline__ void put_image(uint16_t* img, int f0, int c0, const float (&v)[RB][CB]) {
+  uint8_t* base = reinterpret_cast<uint8_t*>(img);
+#pragma unroll
+  for (int i = 0; i < RB; ++i)
+#pragma unroll
+    for (int j = 0; j < CB; ++j)
+      *reinterpret_cast<__nv_bfloat16*>(base + sw128_off(f0 + i, c0 + j, D)) = __float2bfloat16_rn(v[i][j]);
+}
+
 template <int D, int JC>
 __global__ void __launch_bounds__(256) awm_carry_kernel(const float* __restrict__ Bm,
                                                         const float* __restrict__ Cm,
                                                         const float* __restrict__ ratio,
                                                         const float* __restrict__ rho,
                                                         float* __restrict__ Mst, int S,
-                                                        const float* __restrict__ M0, int64_t sd) {
+                                                        const float* __restrict__ M0, int64_t sd,
+                                                        uint16_t* __restrict__ Mimg,
+                                                        const float* __restrict__ Mprev0) {
   using St = CarryStage<D, JC>;
   // each thread owns an RB x CB block of the slice: rows f0 .. f0 + RB - 1,
   // columns c0 .. c0 + CB - 1 (8 column groups, D / RB row groups), so that
@@ -288,11 +306,28 @@ __global__ void __launch_bounds__(256) awm_carry_kernel(const float* __restrict_
   for (int i = tid; i < D * JC; i += 256)
     Ms[i] = M0 ? M0[bh * sd + (i / JC) * D + j0 + i % JC] : 0.f;
   float* mout = Mst + bh * (int64_t)(S + 1) * mst_stride;
+  // readout operand images (if requested): image k + 1 holds Mst[k] for
+  // k < S, image 0 the carried M'_prev of a continued sequence
+  uint16_t* iout = Mimg ? Mimg + bh * (int64_t)(S + 1) * mst_stride : nullptr;
   __syncthreads();
+  {
+    float m1[RB][CB];
 #pragma unroll
-  for (int i = 0; i < RB; ++i)
+    for (int i = 0; i < RB; ++i)
 #pragma unroll
-    for (int j = 0; j < CB; ++j) mout[(f0 + i) * D + j0 + c0 + j] = Ms[(f0 + i) * JC + c0 + j];   // M'_1
+      for (int j = 0; j < CB; ++j) {
+        m1[i][j] = Ms[(f0 + i) * JC + c0 + j];
+        mout[(f0 + i) * D + j0 + c0 + j] = m1[i][j];   // M'_1
+      }
+    if (iout && S > 1) put_image<D, RB, CB>(iout + mst_stride, f0, j0 + c0, m1);
+    if (iout && Mprev0) {
+#pragma unroll
+      for (int i = 0; i < RB; ++i)
+#pragma unroll
+        for (int j = 0; j < CB; ++j) m1[i][j] = Mprev0[bh * sd + (f0 + i) * D + j0 + c0 + j];
+      put_image<D, RB, CB>(iout, f0, j0 + c0, m1);
+    }
+  }
   for (int s = 0; s < S; ++s) {
     const float* sb = smem_carry + (s & 1) * St::kFloats;
     if (s + 1 < S) {
@@ -342,6 +377,7 @@ __global__ void __launch_bounds__(256) awm_carry_kernel(const float* __restrict_
         dst[j] = acc[i][j];
       }
     }
+    if (iout && s + 2 < S) put_image<D, RB, CB>(iout + (int64_t)(s + 2) * mst_stride, f0, j0 + c0, acc);
   }
 }
 
@@ -511,20 +547,21 @@ cudaError_t awm_chunk_simt_impl(const Problem& p, const Workspace& w, cudaStream
 }
 
 template <int D, int JC>
-cudaError_t awm_carry_launch(const Problem& p, const Workspace& w, cudaStream_t st) {
+cudaError_t awm_carry_launch(const Problem& p, const Workspace& w, cudaStream_t st, bool images) {
   const size_t smem = sizeof(float) * (2 * CarryStage<D, JC>::kFloats + D * JC);
   cudaError_t e = cudaFuncSetAttribute(awm_carry_kernel<D, JC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   awm_carry_kernel<D, JC><<<dim3(D / JC, p.B * p.H), 256, smem, st>>>(
-      w.Bm, w.Cm, w.ratio, w.rho, w.Mst, p.S, p.state0 ? p.state0 + D * D : nullptr, state_floats(D));
+      w.Bm, w.Cm, w.ratio, w.rho, w.Mst, p.S, p.state0 ? p.state0 + D * D : nullptr, state_floats(D),
+      images ? w.Mimg : nullptr, p.state0);
   return cudaGetLastError();
 }
 
 template <int D>
-cudaError_t awm_carry_impl(const Problem& p, const Workspace& w, cudaStream_t st) {
+cudaError_t awm_carry_impl(const Problem& p, const Workspace& w, cudaStream_t st, bool images) {
   const int jc = carry_slice(p.B * p.H, D);
-  return jc == 32 ? awm_carry_launch<D, 32>(p, w, st)
-                  : jc == 16 ? awm_carry_launch<D, 16>(p, w, st) : awm_carry_launch<D, 8>(p, w, st);
+  return jc == 32 ? awm_carry_launch<D, 32>(p, w, st, images)
+                  : jc == 16 ? awm_carry_launch<D, 16>(p, w, st, images) : awm_carry_launch<D, 8>(p, w, st, images);
 }
 
 template <typename TIn, int D>
@@ -558,8 +595,8 @@ cudaError_t launch_awm_stats(const Problem& p, const Workspace& w, cudaStream_t 
 cudaError_t launch_awm_chunk_simt(const Problem& p, const Workspace& w, cudaStream_t st) {
   return GECKO_DISPATCH(awm_chunk_simt_impl);
 }
-cudaError_t launch_awm_carry(const Problem& p, const Workspace& w, cudaStream_t st) {
-  return p.d == 64 ? awm_carry_impl<64>(p, w, st) : awm_carry_impl<128>(p, w, st);
+cudaError_t launch_awm_carry(const Problem& p, const Workspace& w, cudaStream_t st, bool images) {
+  return p.d == 64 ? awm_carry_impl<64>(p, w, st, images) : awm_carry_impl<128>(p, w, st, images);
 }
 cudaError_t launch_awm_readout_simt(const Problem& p, const Workspace& w, cudaStream_t st) {
   return GECKO_DISPATCH(awm_readout_simt_impl);
