@@ -190,14 +190,14 @@ int gecko_sca_awm_forward_continue(const void* q, const void* k, const void* v,
  * point; it only changes where the working memory comes from.
  *
  * Working memory: instead of the growable workspace, every call uses one
- * fixed scratch array of GECKO_NOALLOC_SCRATCH_BYTES (64 MiB) that is part
+ * fixed scratch array of GECKO_NOALLOC_SCRATCH_BYTES (80 MiB) that is part
  * of the library's device image; each GPU that loads the library holds it
  * until the process exits.  Inputs and outputs are still passed by the
  * caller.  The scratch needs
- *   4 * (2*BH*T/R*d + 4*BH*S*d + (3*S + 1)*BH*d*d) bytes (each of the seven
- *   regions rounded up to 256 bytes; R = 128 if c % 128 == 0 else 64,
- *   S = T / c, BH = B * H),
- * e.g. B*H = 32, T = 32768, c = 4096, d = 128 needs about 61 MB.  Larger
+ *   4 * (2*BH*T/R*d + 4*BH*S*d + (3*S + 1)*BH*d*d) + 2*(2*S + 1)*BH*d*d
+ *   bytes (each of the nine regions rounded up to 256 bytes; R = 128 if
+ *   c % 128 == 0 else 64, S = T / c, BH = B * H),
+ * e.g. B*H = 32, T = 32768, c = 4096, d = 128 needs about 79 MB.  Larger
  * problems are rejected with GECKO_ERR_LIMIT before anything is launched.
  * The call makes no cudaMalloc, cudaFree or other allocating call.
  *
@@ -214,7 +214,7 @@ int gecko_sca_awm_forward_continue(const void* q, const void* k, const void* v,
  * that state stays the one of the last allocating forward, continued
  * forward, training forward or backward on the device.
  */
-#define GECKO_NOALLOC_SCRATCH_BYTES (64ull << 20)
+#define GECKO_NOALLOC_SCRATCH_BYTES (80ull << 20)
 int gecko_sca_awm_forward_noalloc(const void* q, const void* k, const void* v,
                                   const void* qm, const void* km,
                                   void* out_sca, void* out_mem,

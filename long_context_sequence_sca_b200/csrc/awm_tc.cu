@@ -35,7 +35,6 @@ namespace {
 
 // ------------------------------------------------------------ chunk GEMMs --
 
-constexpr int kKT = 64;  // tokens per tile
 
 // What a chunk-kernel launch computes.
 //   kChunkFwd    Bm = Phi~^T V, Cm = Phi~^T Psi with bf16 operands (f16
@@ -51,14 +50,20 @@ enum ChunkMode { kChunkFwd = 0, kChunkSplit = 1, kChunkE = 2 };
 
 template <int D, int Mode = kChunkFwd>
 struct ChunkCfg {
-  static constexpr int kBox = kKT * 128;                 // one [64 x 64] bf16 box
-  static constexpr int kOperand = (D / 64) * kBox;       // a [64 x D] operand
+  // Tokens per tile and stages.  32-token tiles through 4 stages (three
+  // loads in flight instead of one) measured slower for the forward mode
+  // (0.210 against 0.183 ms at the bench workload), so every mode streams
+  // 64-token tiles through 2 stages.
+  static constexpr int kKT = 64;
+  static constexpr int kStages = 2;
+  static constexpr int kTPR = 128 / kKT;                 // compute threads per token row
+  static constexpr int kBox = kKT * 128;                 // one [kKT x 64] bf16 box
+  static constexpr int kOperand = (D / 64) * kBox;       // a [kKT x D] operand
   static constexpr int kSlots = Mode == kChunkSplit ? 5 : 3;
   static constexpr int kStage = kSlots * kOperand;
-  static constexpr int kStages = 2;
   static constexpr int kBarOff = kStages * kStage;
-  // v_full[2], op_full[2], stage_empty[2], acc_full
-  static constexpr int kNumBars = 7;
+  // v_full[kStages], op_full[kStages], stage_empty[kStages], acc_full
+  static constexpr int kNumBars = 3 * kStages + 1;
   static constexpr int kLzOff = kBarOff + kNumBars * 8;  // D floats: log2(e) * log z^s
   static constexpr int kMiscOff = kLzOff + D * 4;
   static constexpr int kBytes = kMiscOff + 16;
@@ -75,16 +80,17 @@ template <int D, int Mode = kChunkFwd>
 __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_v,
                                                            const __grid_constant__ CUtensorMap map_km,
                                                            const float* __restrict__ lse, float* __restrict__ Bm,
-                                                           float* __restrict__ Cm, int T, int c, int koff,
-                                                           int* status) {
+                                                           float* __restrict__ Cm, uint16_t* __restrict__ Cimg,
+                                                           int T, int c, int koff, int* status) {
   using Cfg = ChunkCfg<D, Mode>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int NS = Cfg::kStages, kKT = Cfg::kKT;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
-  uint64_t* v_full = bars;          // [2] TMA -> MMA
-  uint64_t* op_full = bars + 2;     // [2] compute -> MMA (128 arrivals)
-  uint64_t* st_empty = bars + 4;    // [2] MMA -> TMA, compute
-  uint64_t* acc_full = bars + 6;
+  uint64_t* v_full = bars;          // [NS] TMA -> MMA
+  uint64_t* op_full = bars + NS;    // [NS] compute -> MMA (128 arrivals)
+  uint64_t* st_empty = bars + 2 * NS;   // [NS] MMA -> TMA, compute
+  uint64_t* acc_full = bars + 3 * NS;
   float* lz2 = reinterpret_cast<float*>(smem + Cfg::kLzOff);  // log2(e) * lse_s
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
@@ -100,7 +106,7 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
   const int64_t vrow0 = bh * (int64_t)(T + koff) + koff + (int64_t)s * c;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NS; ++i) {
       mbar_init(v_full + i, 1);
       mbar_init(op_full + i, kChunkCompute);
       mbar_init(st_empty + i, 1);
@@ -127,10 +133,12 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
     if (lane == 0) {
       tma_prefetch_desc(&map_v);
       tma_prefetch_desc(&map_km);
+      int issued = 0;
       for (int kt = 0; kt < n_tiles; ++kt) {
-        const int st = kt & 1;
-        if (!mbar_wait(st_empty + st, ((kt >> 1) & 1) ^ 1, abort_flag, status)) break;
+        const int st = kt % NS;
+        if (!mbar_wait(st_empty + st, ((kt / NS) & 1) ^ 1, abort_flag, status)) break;
         mbar_arrive_expect_tx(v_full + st, 2 * Cfg::kOperand);
+        ++issued;
         for (int b = 0; b < D / 64; ++b) {
           tma_load_2d(smem + st * Cfg::kStage + b * Cfg::kBox, &map_v, v_full + st, b * 64,
                       (int)(vrow0 + (int64_t)kt * kKT));
@@ -139,7 +147,8 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
         }
       }
       if (*abort_flag) {
-        for (int st = 0; st < 2; ++st) mbar_wait_drain(v_full + st, ((n_tiles - 1 - st) >> 1) & 1);
+        // the copies issued land before the CTA exits
+        for (int t = issued > NS ? issued - NS : 0; t < issued; ++t) mbar_wait_drain(v_full + t % NS, (t / NS) & 1);
       }
     }
     __syncwarp();
@@ -151,8 +160,8 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
       const uint32_t base = smem_u32(smem);
       bool ok = true;
       for (int kt = 0; kt < n_tiles && ok; ++kt) {
-        const int st = kt & 1;
-        const uint32_t ph = (kt >> 1) & 1;
+        const int st = kt % NS;
+        const uint32_t ph = (kt / NS) & 1;
         if (!(ok = mbar_wait(v_full + st, ph, abort_flag, status))) break;
         if (!(ok = mbar_wait(op_full + st, ph, abort_flag, status))) break;
         tc_fence_after();
@@ -181,15 +190,16 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
     __syncwarp();
   } else {
     // ------------------------------------------ Phi / Psi, then epilogue --
-    const int r = threadIdx.x >> 1;       // token row within the tile
-    const int h = threadIdx.x & 1;        // which half of the features
-    constexpr int HF = D / 2;             // features per thread
+    constexpr int TPR = Cfg::kTPR;        // threads per token row
+    const int r = threadIdx.x / TPR;      // token row within the tile
+    const int h = threadIdx.x % TPR;      // which part of the features
+    constexpr int HF = D / TPR;           // features per thread
     bool ok = true;
     for (int kt = 0; kt < n_tiles; ++kt) {
-      const int st = kt & 1;
+      const int st = kt % NS;
       // V and K_m of this tile have landed (the copy also waited for the
-      // MMAs of tile kt - 2 to release the stage)
-      ok = __all_sync(0xffffffffu, mbar_wait(v_full + st, (kt >> 1) & 1, abort_flag, status));
+      // MMAs of tile kt - NS to release the stage)
+      ok = __all_sync(0xffffffffu, mbar_wait(v_full + st, (kt / NS) & 1, abort_flag, status));
       if (!ok) break;
       uint8_t* stg = smem + st * Cfg::kStage;
       float x[HF];
@@ -207,7 +217,8 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
       float mx = x[0];
 #pragma unroll
       for (int i = 1; i < HF; ++i) mx = fmaxf(mx, x[i]);
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+#pragma unroll
+      for (int o = 1; o < TPR; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       const float mx2 = mx * kLog2e;
       float e[HF], sum = 0.f;
       if (Mode == kChunkFwd) {
@@ -255,7 +266,8 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
           }
         }
       }
-      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+#pragma unroll
+      for (int o = 1; o < TPR; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
       const float inv = 1.f / sum;
 #pragma unroll
       for (int i = 0; i < HF / 8; ++i) {
@@ -300,6 +312,17 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
           for (int i = 0; i < 8; ++i)
             reinterpret_cast<float4*>(dst)[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
                                                             __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+          if (Mode == kChunkFwd && D == 128 && Cimg && cb * 32 >= D) {
+            // Cm row f as the tensor-core carry's bf16 A operand (K-major)
+            uint8_t* img = reinterpret_cast<uint8_t*>(Cimg + (bh * S + s) * (int64_t)D * D);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              *reinterpret_cast<uint4*>(img + sw128_off(f, cb * 32 - D + 8 * i, 128)) =
+                  make_uint4(pack_bf16x2(__uint_as_float(v[8 * i]), __uint_as_float(v[8 * i + 1])),
+                             pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
+                             pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
+                             pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
+          }
         }
       }
     }
@@ -613,100 +636,98 @@ awm_readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
 // The sequential carry on the tensor cores, d = 128 (Gecko digest, method
 // step details, step 4, with the row scales factored out as in the SIMT
 // carry):
-//   M'_{s+1} = r_s (.) M'_s + rho_s (.) (Bm_s - Cm_s M'_s),
-// one CTA per (b, h), 128 threads, thread f owning row f of M' (an fp32
-// master copy in registers) and TMEM lane f of the product.  Per step the
-// product Cm_s M'_s runs as two bf16 MMAs, Cm M_hi + Cm M_lo with M' split
-// into hi + lo parts and fp32 accumulation (Cm rounded to bf16 once:
-// emulated over 128 chunks of 512 tokens the state stays within 2e-5 of
-// fp64).  Cm_s arrives by one bulk copy into an fp32 staging buffer one
-// step ahead and is rounded into the K-major A operand; Bm_s arrives by TMA
-// (128-byte swizzled, so each thread reads its row without bank conflicts)
-// while the step's operands are formed and multiplied.  M'_s is split from
-// the registers into the MN-major B operands, whose hi part is also the
-// readout's operand image of M'_s (bf16, same layout) and leaves by one bulk
-// store.  Writes Mst[s] = M'_{s+1} for s = 0..S like the SIMT carry.
+//   M'_{s+1} = r_s (.) M'_s + rho_s (.) (Bm_s - Cm_s M'_s).
+// Columns of M' evolve independently, so two CTAs share a (b, h), each
+// owning 64 columns: 128 threads, thread f holding row f of its columns in
+// fp32 registers (the master copy) and TMEM lane f of the product.  Per step
+// the product Cm_s M'_s[:, cols] runs as two bf16 MMAs (M = 128, N = 64),
+// Cm M_hi + Cm M_lo, with M' split into hi + lo parts and Cm rounded to bf16
+// once by the chunk kernel (emulated over 128 chunks of 512 tokens the state
+// stays within 2e-5 of fp64); fp32 accumulation.  Cm_s (the chunk kernel's
+// bf16 operand image, one bulk copy) and Bm_s[:, cols] (TMA, 128-byte
+// swizzled so each thread reads its row without bank conflicts) arrive two
+// steps ahead in double buffers.  The hi part of M'_s's B operand is also the
+// readout's operand image of M'_s (64 columns = one box of it) and leaves by
+// one bulk store.  Only the states the forward reads later are written in
+// fp32: Mst[0] = M'_1, and Mst[S-1], Mst[S] (the exported state).
 struct CarryTcCfg {
-  static constexpr int kD = 128;
-  static constexpr int kStage = kD * kD * 4;     // one fp32 d x d matrix
-  static constexpr int kOp = kD * kD * 2;        // one bf16 operand (two 64-column boxes of 128 rows)
-  static constexpr int kBox = 128 * 128;         // one bf16 box [128 rows x 64]
-  static constexpr int kFBox = 128 * 128;        // one fp32 box [128 rows x 32]
-  static constexpr int kCOff = 0;                // Cm_s staging, fp32 row-major
-  static constexpr int kBmOff = kCOff + kStage;  // Bm_s, fp32, four 128B-swizzled boxes of 32 columns
-  static constexpr int kAOff = kBmOff + kStage, kBhiOff = kAOff + kOp, kBloOff = kBhiOff + kOp;
-  static constexpr int kBarOff = kBloOff + kOp;  // c_full, b_full, m_done, drain
+  static constexpr int kD = 128, kN = 64;         // d, columns per CTA
+  static constexpr int kA = kD * kD * 2;          // Cm_s, bf16 K-major (two 64-column boxes of 128 rows)
+  static constexpr int kBox = 128 * 128;          // one bf16 box [128 rows x 64]
+  static constexpr int kOp = kD * kN * 2;         // one B operand: [128 K rows x 64 N] bf16, one box
+  static constexpr int kBm = kD * kN * 4;         // Bm_s[:, cols] fp32: two boxes [128 rows x 32]
+  static constexpr int kFBox = 128 * 128;         // one fp32 box [128 rows x 32]
+  static constexpr int kAOff = 0;                 // [2] A buffers
+  static constexpr int kBmOff = kAOff + 2 * kA;   // [2] Bm buffers
+  static constexpr int kBhiOff = kBmOff + 2 * kBm, kBloOff = kBhiOff + kOp;
+  static constexpr int kBarOff = kBloOff + kOp;   // in_full[2], m_done, drain
   static constexpr int kMiscOff = kBarOff + 32;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
 __global__ void __launch_bounds__(128, 1)
-awm_carry_tc_kernel(const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_m,
-                    const float* __restrict__ Cm,
+awm_carry_tc_kernel(const __grid_constant__ CUtensorMap map_b, const uint16_t* __restrict__ Cimg,
                     const float* __restrict__ ratio, const float* __restrict__ rho, float* __restrict__ Mst, int S,
                     const float* __restrict__ M0, int64_t sd, uint16_t* __restrict__ Mimg,
                     const float* __restrict__ Mprev0, int* status) {
   using Cfg = CarryTcCfg;
-  constexpr int D = Cfg::kD;
+  constexpr int D = Cfg::kD, N = Cfg::kN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const float* cst = reinterpret_cast<const float*>(smem + Cfg::kCOff);
-  uint64_t* c_full = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
-  uint64_t* b_full = c_full + 1;
-  uint64_t* m_done = c_full + 2;
-  uint64_t* drain = c_full + 3;
+  uint64_t* in_full = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);   // [2] A and Bm of a step
+  uint64_t* m_done = in_full + 2;
+  uint64_t* drain = in_full + 3;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
-  const int64_t bh = blockIdx.x;
-  const int f = threadIdx.x, warp = f / 32, lane = f % 32;
+  const int64_t bh = blockIdx.x / 2;
+  const int half = blockIdx.x % 2, j0 = half * N;
+  const int f = threadIdx.x, warp = f / 32;
   const int64_t mat = (int64_t)D * D;
   float* mout = Mst + bh * (int64_t)(S + 1) * mat;
   uint16_t* iout = Mimg ? Mimg + bh * (int64_t)(S + 1) * mat : nullptr;
-  int cloads = 0, bloads = 0;   // staging copies issued (thread 0)
-  auto load_bm = [&](int s) {   // thread 0: Bm_s into its swizzled boxes
-    mbar_arrive_expect_tx(b_full, Cfg::kStage);
-    for (int b = 0; b < D / 32; ++b)
-      tma_load_2d(smem + Cfg::kBmOff + b * Cfg::kFBox, &map_b, b_full, b * 32, (int)((bh * S + s) * D));
-    ++bloads;
+  int loads = 0;   // steps whose inputs have been requested (thread 0)
+  auto load_step = [&](int s) {   // thread 0: Cm_s and Bm_s[:, cols] into buffer s & 1
+    uint64_t* bar = in_full + (s & 1);
+    mbar_arrive_expect_tx(bar, Cfg::kA + Cfg::kBm);
+    bulk_load_1d(smem + Cfg::kAOff + (s & 1) * Cfg::kA, Cimg + (bh * S + s) * mat, Cfg::kA, bar);
+    for (int b = 0; b < N / 32; ++b)
+      tma_load_2d(smem + Cfg::kBmOff + (s & 1) * Cfg::kBm + b * Cfg::kFBox, &map_b, bar, j0 + b * 32,
+                  (int)((bh * S + s) * D));
+    ++loads;
   };
 
   if (f == 0) {
-    mbar_init(c_full, 1);
-    mbar_init(b_full, 1);
+    mbar_init(in_full, 1);
+    mbar_init(in_full + 1, 1);
     mbar_init(m_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&map_b);
-    tma_prefetch_desc(&map_m);
-    if (S > 0) {
-      cloads = 1;
-      mbar_arrive_expect_tx(c_full, Cfg::kStage);
-      bulk_load_1d(smem + Cfg::kCOff, Cm + bh * S * mat, Cfg::kStage, c_full);
-      load_bm(0);
-    }
+    for (int s = 0; s < 2 && s < S; ++s) load_step(s);
   }
   if (warp == 0) {
-    tmem_alloc(tmem_slot, 128);
+    tmem_alloc(tmem_slot, N);
     tmem_relinquish();
   }
   // M'_1: zero, or the carried M'_cur of a continued sequence
-  float m[D];
+  float m[N];
 #pragma unroll
-  for (int j = 0; j < D; j += 4) {
-    const float4 v = M0 ? *reinterpret_cast<const float4*>(M0 + bh * sd + (int64_t)f * D + j) : make_float4(0, 0, 0, 0);
+  for (int j = 0; j < N; j += 4) {
+    const float4 v =
+        M0 ? *reinterpret_cast<const float4*>(M0 + bh * sd + (int64_t)f * D + j0 + j) : make_float4(0, 0, 0, 0);
     m[j] = v.x; m[j + 1] = v.y; m[j + 2] = v.z; m[j + 3] = v.w;
-    *reinterpret_cast<float4*>(mout + (int64_t)f * D + j) = v;
+    *reinterpret_cast<float4*>(mout + (int64_t)f * D + j0 + j) = v;
   }
   if (iout && Mprev0) {
     // image 0: the carried M'_prev, read by a continued sequence's first chunk
     uint8_t* img = reinterpret_cast<uint8_t*>(iout);
 #pragma unroll 4
-    for (int j = 0; j < D; j += 8) {
-      const float4 a = *reinterpret_cast<const float4*>(Mprev0 + bh * sd + (int64_t)f * D + j);
-      const float4 b = *reinterpret_cast<const float4*>(Mprev0 + bh * sd + (int64_t)f * D + j + 4);
-      *reinterpret_cast<uint4*>(img + sw128_off(f, j, D)) =
+    for (int j = 0; j < N; j += 8) {
+      const float4 a = *reinterpret_cast<const float4*>(Mprev0 + bh * sd + (int64_t)f * D + j0 + j);
+      const float4 b = *reinterpret_cast<const float4*>(Mprev0 + bh * sd + (int64_t)f * D + j0 + j + 4);
+      *reinterpret_cast<uint4*>(img + sw128_off(f, j0 + j, D)) =
           make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
     }
   }
@@ -716,35 +737,25 @@ awm_carry_tc_kernel(const __grid_constant__ CUtensorMap map_b, const __grid_cons
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
   const uint32_t base = smem_u32(smem);
-  constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, true);
-  bool ok = true;
-
-  // Every exit from the loop follows a block barrier and tests the CTA's
-  // abort flag, so all warps leave together; a wait that gives up only
-  // raises the flag.
+  constexpr uint32_t idesc = idesc_bf16_f32(128, N, false, true);
   float rf = 0.f, pf = 0.f;   // r_s and rho_s of this thread's row, read one step ahead
   if (S > 0) {
     rf = ratio[bh * S * D + f];
     pf = rho[bh * S * D + f];
   }
+
+  // Every exit from the loop follows a block barrier and tests the CTA's
+  // abort flag, so all warps leave together; a wait that gives up only
+  // raises the flag.
   for (int s = 0; s < S; ++s) {
+    const int buf = s & 1;
     // the previous image store has finished reading B_hi before it is rewritten
     if (f == 0) bulk_wait_read<0>();
-    fence_proxy_async_smem();   // the epilogue's rows of M'_s in the staging go out by TMA
     __syncthreads();
     if (*abort_flag) break;
-    if (f == 0 && s > 0) {
-      // M'_s (= Mst[s]), written over Bm_{s-1} in the staging, leaves by one
-      // TMA store; Bm_s may land once the store has read the staging
-      for (int b = 0; b < D / 32; ++b)
-        tma_store_2d(&map_m, smem + Cfg::kBmOff + b * Cfg::kFBox, b * 32, (int)((bh * (S + 1) + s) * D));
-      bulk_commit();
-      bulk_wait_read<0>();
-      load_bm(s);
-    }
-    // B = M'_s as hi + lo (row f = K index f, MN-major)
+    // B = M'_s[:, cols] as hi + lo (row f = K index f, MN-major, one box)
 #pragma unroll
-    for (int j = 0; j < D; j += 8) {
+    for (int j = 0; j < N; j += 8) {
       uint32_t hi[4], lo[4];
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
@@ -756,60 +767,44 @@ awm_carry_tc_kernel(const __grid_constant__ CUtensorMap map_b, const __grid_cons
       *reinterpret_cast<uint4*>(smem + Cfg::kBhiOff + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
       *reinterpret_cast<uint4*>(smem + Cfg::kBloOff + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
-    // A = Cm_s in bf16 (K-major): warp w converts rows 32w .. 32w + 31, lane
-    // l columns 4l .. 4l + 3 of each (conflict-free staging reads)
-    ok = __all_sync(0xffffffffu, mbar_wait(c_full, s & 1, abort_flag, status));
-    if (ok) {
-#pragma unroll 4
-      for (int rr = 0; rr < 32; ++rr) {
-        const int row = warp * 32 + rr;
-        const float4 v = *reinterpret_cast<const float4*>(cst + row * D + 4 * lane);
-        *reinterpret_cast<uint2*>(smem + Cfg::kAOff + sw128_off(row, 4 * lane, D)) =
-            make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
-      }
-    }
     fence_proxy_async_smem();   // the operands are read by the tensor core and the bulk store
     __syncthreads();
-    if (*abort_flag) break;
     if (f == 0) {
-      // B_hi is the readout's image of M'_s (= Mst[s]), read by chunk s + 1
+      // B_hi is the readout's image of M'_s[:, cols] (box `half` of Mst[s]'s image), read by chunk s + 1
       if (iout && s + 1 < S) {
-        bulk_store_1d(iout + (int64_t)(s + 1) * mat, smem + Cfg::kBhiOff, Cfg::kOp);
+        bulk_store_1d(reinterpret_cast<uint8_t*>(iout + (int64_t)(s + 1) * mat) + half * Cfg::kBox,
+                      smem + Cfg::kBhiOff, Cfg::kOp);
         bulk_commit();
       }
-      // the staging buffer has been converted: prefetch the next step's Cm
-      if (s + 1 < S) {
-        ++cloads;
-        mbar_arrive_expect_tx(c_full, Cfg::kStage);
-        bulk_load_1d(smem + Cfg::kCOff, Cm + (bh * S + s + 1) * mat, Cfg::kStage, c_full);
-      }
-      tc_fence_after();
-      const SDesc ad = sdesc_sw128_split(base + Cfg::kAOff, 16, 1024);
-      const SDesc bh_ = sdesc_sw128_split(base + Cfg::kBhiOff, D * 128, 1024);
-      const SDesc bl = sdesc_sw128_split(base + Cfg::kBloOff, D * 128, 1024);
+      if (mbar_wait(in_full + buf, (s >> 1) & 1, abort_flag, status)) {
+        tc_fence_after();
+        const SDesc ad = sdesc_sw128_split(base + Cfg::kAOff + buf * Cfg::kA, 16, 1024);
+        const SDesc bh_ = sdesc_sw128_split(base + Cfg::kBhiOff, N * 128, 1024);
+        const SDesc bl = sdesc_sw128_split(base + Cfg::kBloOff, N * 128, 1024);
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t ka = (kk / 4) * Cfg::kBox + (kk % 4) * 32, kb = kk * 16 * 128;
-        umma_ss(tmem, sdesc_at(ad, ka), sdesc_at(bh_, kb), idesc, kk > 0 ? 1u : 0u);
-        umma_ss(tmem, sdesc_at(ad, ka), sdesc_at(bl, kb), idesc, 1u);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ka = (kk / 4) * Cfg::kBox + (kk % 4) * 32, kb = kk * 16 * 128;
+          umma_ss(tmem, sdesc_at(ad, ka), sdesc_at(bh_, kb), idesc, kk > 0 ? 1u : 0u);
+          umma_ss(tmem, sdesc_at(ad, ka), sdesc_at(bl, kb), idesc, 1u);
+        }
+        umma_commit(m_done);
       }
-      umma_commit(m_done);
     }
     float rn = 0.f, pn = 0.f;
     if (s + 1 < S) {
       rn = ratio[(bh * S + s + 1) * D + f];
       pn = rho[(bh * S + s + 1) * D + f];
     }
-    ok = __all_sync(0xffffffffu, mbar_wait(m_done, s & 1, abort_flag, status) &&
-                                     mbar_wait(b_full, s & 1, abort_flag, status));
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(m_done, s & 1, abort_flag, status) &&
+                                                mbar_wait(in_full + buf, (s >> 1) & 1, abort_flag, status));
     tc_fence_after();
     if (ok) {
 #pragma unroll
-      for (int cb = 0; cb < D / 32; ++cb) {
+      for (int cb = 0; cb < N / 32; ++cb) {
         uint32_t acc[32];
         tmem_ld32(lane_addr + cb * 32, acc);
         float bv[32];
-        uint8_t* bbox = smem + Cfg::kBmOff + cb * Cfg::kFBox + f * 128;
+        const uint8_t* bbox = smem + Cfg::kBmOff + buf * Cfg::kBm + cb * Cfg::kFBox + f * 128;
 #pragma unroll
         for (int t = 0; t < 8; ++t) {   // fp32 box: 16-byte chunk t of row f sits at chunk t ^ (f & 7)
           const float4 v = *reinterpret_cast<const float4*>(bbox + ((t ^ (f & 7)) << 4));
@@ -819,40 +814,34 @@ awm_carry_tc_kernel(const __grid_constant__ CUtensorMap map_b, const __grid_cons
 #pragma unroll
         for (int t = 0; t < 32; ++t)
           m[cb * 32 + t] = fmaf(rf, m[cb * 32 + t], pf * (bv[t] - __uint_as_float(acc[t])));
-        // the new row goes where Bm's row was read: the staging becomes M'_{s+1}
+      }
+      if (s + 2 >= S) {
+        // Mst[s + 1] is one of the last two states: the exported state
+        float* row = mout + (int64_t)(s + 1) * mat + (int64_t)f * D + j0;
 #pragma unroll
-        for (int t = 0; t < 8; ++t)
-          *reinterpret_cast<float4*>(bbox + ((t ^ (f & 7)) << 4)) =
-              make_float4(m[cb * 32 + 4 * t], m[cb * 32 + 4 * t + 1], m[cb * 32 + 4 * t + 2], m[cb * 32 + 4 * t + 3]);
+        for (int j = 0; j < N; j += 4) *reinterpret_cast<float4*>(row + j) = make_float4(m[j], m[j + 1], m[j + 2], m[j + 3]);
       }
     }
     rf = rn;
     pf = pn;
     tc_fence_before();
-  }
-  // the last state M'_{S+1} (= Mst[S]) from the staging
-  fence_proxy_async_smem();
-  __syncthreads();
-  if (f == 0 && S > 0 && !*abort_flag) {
-    for (int b = 0; b < D / 32; ++b)
-      tma_store_2d(&map_m, smem + Cfg::kBmOff + b * Cfg::kFBox, b * 32, (int)((bh * (S + 1) + S) * D));
-    bulk_commit();
+    __syncthreads();   // buffer `buf` is free: step s + 2's inputs may land there
+    if (f == 0 && s + 2 < S && !*abort_flag) load_step(s + 2);
   }
   if (f == 0) {
     bulk_wait_all();
     if (*abort_flag) {
       // no MMA may still write TMEM and no copy still land when the CTA
-      // exits: the staging copies issued complete phases 0 .. n - 1
+      // exits: the input copies issued complete phases of in_full[t & 1]
       umma_commit(drain);
       mbar_wait_drain(drain, 0);
-      if (cloads > 0) mbar_wait_drain(c_full, (cloads - 1) & 1);
-      if (bloads > 0) mbar_wait_drain(b_full, (bloads - 1) & 1);
+      for (int t = loads > 2 ? loads - 2 : 0; t < loads; ++t) mbar_wait_drain(in_full + (t & 1), (t >> 1) & 1);
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) tmem_dealloc(tmem, 128);
+  if (warp == 0) tmem_dealloc(tmem, N);
 }
 
 // ------------------------------------------------------------------ host --
@@ -875,7 +864,7 @@ EncodeTiledFn encode_fn() {
 
 template <int D, int Mode>
 cudaError_t chunk_impl(const Problem& p, const void* vsrc, const void* ksrc, const float* lse, float* out0,
-                       float* out1, cudaStream_t st) {
+                       float* out1, cudaStream_t st, uint16_t* cimg = nullptr) {
   using Cfg = ChunkCfg<D, Mode>;
   EncodeTiledFn fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
@@ -884,7 +873,7 @@ cudaError_t chunk_impl(const Problem& p, const void* vsrc, const void* ksrc, con
   auto map = [&](CUtensorMap* m, const void* base, int64_t rows) {
     cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)kKT};
+    cuuint32_t box[2] = {64, (cuuint32_t)Cfg::kKT};
     cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -897,7 +886,7 @@ cudaError_t chunk_impl(const Problem& p, const void* vsrc, const void* ksrc, con
                                        Cfg::kAlloc);
   if (e != cudaSuccess) return e;
   awm_chunk_tc_kernel<D, Mode><<<dim3(p.S, p.B * p.H), kChunkThreads, Cfg::kAlloc, st>>>(
-      mv, mkm, lse, out0, out1, (int)p.T, (int)p.c, (int)koff, p.status);
+      mv, mkm, lse, out0, out1, cimg, (int)p.T, (int)p.c, (int)koff, p.status);
   return cudaGetLastError();
 }
 
@@ -945,15 +934,8 @@ cudaError_t carry_tc_impl(const Problem& p, const Workspace& w, cudaStream_t st,
          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
       CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  // Mst as [BH (S+1) d rows, d] fp32, the same boxes (the states leave by TMA store)
-  CUtensorMap mm;
-  cuuint64_t mdims[2] = {128, (cuuint64_t)(p.B * p.H * (p.S + 1) * 128)};
-  if (fn(&mm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, w.Mst, mdims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
-      CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
-  awm_carry_tc_kernel<<<(unsigned)(p.B * p.H), 128, Cfg::kAlloc, st>>>(
-      mb, mm, w.Cm, w.ratio, w.rho, w.Mst, p.S, p.state0 ? p.state0 + 128 * 128 : nullptr, state_floats(128),
+  awm_carry_tc_kernel<<<(unsigned)(2 * p.B * p.H), 128, Cfg::kAlloc, st>>>(
+      mb, w.Cimg, w.ratio, w.rho, w.Mst, p.S, p.state0 ? p.state0 + 128 * 128 : nullptr, state_floats(128),
       images ? w.Mimg : nullptr, p.state0, p.status);
   return cudaGetLastError();
 }
@@ -966,7 +948,7 @@ cudaError_t launch_awm_carry_tc(const Problem& p, const Workspace& w, cudaStream
 
 cudaError_t launch_awm_chunk_tc(const Problem& p, const Workspace& w, cudaStream_t st) {
   return p.d == 64 ? chunk_impl<64, kChunkFwd>(p, p.v, p.km, w.lse, w.Bm, w.Cm, st)
-                   : chunk_impl<128, kChunkFwd>(p, p.v, p.km, w.lse, w.Bm, w.Cm, st);
+                   : chunk_impl<128, kChunkFwd>(p, p.v, p.km, w.lse, w.Bm, w.Cm, st, w.Cimg);
 }
 
 cudaError_t launch_awm_chunk_tc_split(const Problem& p, const Workspace& w, cudaStream_t st) {

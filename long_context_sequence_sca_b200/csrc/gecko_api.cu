@@ -34,7 +34,8 @@ size_t workspace_bytes(int64_t BH, int64_t T, int64_t c, int64_t d) {
   const size_t mat = al(sizeof(float) * BH * S * d * d);
   const size_t mst = al(sizeof(float) * BH * (S + 1) * d * d);
   const size_t img = al(sizeof(uint16_t) * BH * (S + 1) * d * d);
-  return part + 4 * vec + 2 * mat + mst + img;
+  const size_t cimg = al(sizeof(uint16_t) * BH * S * d * d);
+  return part + 4 * vec + 2 * mat + mst + img + cimg;
 }
 
 Workspace carve_workspace(void* base, int64_t BH, int64_t T, int64_t c, int64_t d) {
@@ -62,6 +63,8 @@ Workspace carve_workspace(void* base, int64_t BH, int64_t T, int64_t c, int64_t 
   w.Mst = reinterpret_cast<float*>(p);
   p += al(sizeof(float) * BH * (S + 1) * d * d);
   w.Mimg = reinterpret_cast<uint16_t*>(p);
+  p += al(sizeof(uint16_t) * BH * (S + 1) * d * d);
+  w.Cimg = reinterpret_cast<uint16_t*>(p);
   return w;
 }
 

@@ -43,6 +43,10 @@ struct Workspace {
   // the carried M'_prev for s = 0, as bf16 in the 128-byte-swizzled
   // MN-major layout (64-column boxes of d rows).  Written by the carry.
   uint16_t* Mimg;
+  // [BH, S, d * d] bf16 bits: Cm_s rounded to bf16 in the K-major
+  // 128-byte-swizzled operand layout (rows f, K = g), written by the forward
+  // chunk kernel at d = 128 and read by the tensor-core carry.
+  uint16_t* Cimg;
 };
 
 // Column slices of the sequential carries: as wide as still gives about one

@@ -104,7 +104,7 @@ def test_noalloc_creates_no_state_and_takes_no_device_memory(L):
     free1, _ = torch.cuda.mem_get_info()
     # the allocating forward would need this much working memory
     BH, S, d = w.B * w.H, w.T // w.c, w.d
-    ws = 4 * (3 * S + 1) * BH * d * d
+    ws = 4 * (3 * S + 1) * BH * d * d + 2 * (2 * S + 1) * BH * d * d
     assert free0 - free1 < ws, (free0, free1, ws)
     rc, _, _ = _state_rc(L, w)
     assert rc == 6, "gecko_awm_state must report GECKO_ERR_NO_STATE after a release"
@@ -113,8 +113,19 @@ def test_noalloc_creates_no_state_and_takes_no_device_memory(L):
     _close(o_mem, ref_mem, w.dtype, "out_mem vs oracle")
 
 
+def test_noalloc_headline_shape_fits_and_equals_the_allocating_entry(L):
+    """B=1, H=32, T=32768, c=4096, d=128 (about 79 MB of working memory) fits
+    the scratch; the same kernels give the allocating forward's outputs bit
+    for bit."""
+    w = Workload("noalloc_headline", 34, "bf16", 1, 32, 32768, 128, 4096)
+    x = make_inputs(w, device="cuda")
+    ref_sca, ref_mem = L.sca_awm_forward(*(x[n] for n in NAMES), w.c)
+    o_sca, o_mem = _noalloc(L, x, w)
+    assert torch.equal(o_sca, ref_sca) and torch.equal(o_mem, ref_mem)
+
+
 def test_noalloc_rejects_problems_above_its_scratch(L):
-    # 400 chunks of 128 tokens at d = 128 need about 77 MB of working memory
+    # 400 chunks of 128 tokens at d = 128 need about 106 MB of working memory
     w = Workload("noalloc_big", 33, "bf16", 1, 1, 128 * 400, 128, 128)
     x = {n: torch.zeros(w.B, w.H, w.T, w.d, dtype=torch.bfloat16, device="cuda")
          for n in ("q", "k", "v", "qm", "km", "o1", "o2")}
