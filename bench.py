@@ -83,14 +83,25 @@ def io_bytes(w: Workload) -> int:
     return 7 * w.B * w.H * w.T * w.d * esz
 
 
+def fused_stats(w: Workload) -> bool:
+    """The tensor-core forward at d = 128 computes each chunk's K_m
+    statistics inside the chunk kernel (no separate pass over K_m)."""
+    return w.dtype == "bf16" and w.d == 128 and w.c % 128 == 0
+
+
 def stage_bytes(w: Workload) -> dict:
     """Algorithmic HBM bytes of each timed stage that moves the inputs or
-    outputs: the statistics read K_m, the chunk products read K_m and V, the
-    readout reads Q_m and writes out_mem, SCA reads Q, K, V and writes
-    out_sca.  The carry only touches the O(S d^2) workspace."""
+    outputs: the statistics read K_m (a stage of its own unless the chunk
+    kernel computes them), the chunk products read K_m and V, the readout
+    reads Q_m and writes out_mem, SCA reads Q, K, V and writes out_sca.  The
+    carry and the prefix over chunks only touch the O(S d) and O(S d^2)
+    workspace."""
     esz = 2 if w.dtype == "bf16" else 4
     t = w.B * w.H * w.T * w.d * esz
-    return {"awm_stats": t, "awm_chunk": 2 * t, "awm_readout": 2 * t, "sca": 4 * t}
+    out = {"awm_chunk": 2 * t, "awm_readout": 2 * t, "sca": 4 * t}
+    if not fused_stats(w):
+        out["awm_stats"] = t
+    return out
 
 
 def hbm_bound(w: Workload, pk: dict) -> bool:
@@ -472,12 +483,16 @@ def run_gecko(args, w: Workload, ws: int, rank: int, local: int) -> dict:
         "pct_bf16_peak": round(100 * fl["total"] / (agg["ms_per_step"] / 1e3) / 1e12 / pk["bf16_tflops"], 2),
         "stage_ms": {k_: round(v_, 4) for k_, v_ in stages.items()},
         "stage_note": (f"stages timed in a separate pass of {n_stage} steps with CUDA events between the stages "
-                       f"(sum {serial_ms:.4f} ms)"),
+                       f"(sum {serial_ms:.4f} ms)" +
+                       ("; the chunk kernel computes the K_m statistics and awm_chunk includes the prefix over "
+                        "chunks" if fused_stats(w) else "")),
         "stage_hbm": stage_hbm,
         "roofline": roofline,
         "other_bounds": secondary_rooflines(w, agg["ms_per_step"], sca_ms, ck.get("sm_mhz"), pk["hbm_gbs"]),
         "clocks": ck,
-        "gpu_launches": 7 * args.steps,  # lse partial, lse combine, prefix, chunk, carry, readout, sca
+        # chunk (with statistics), prefix, carry, readout, sca; or lse partial,
+        # lse combine, prefix, chunk, carry, readout, sca
+        "gpu_launches": (5 if fused_stats(w) else 7) * args.steps,
     }
     if note:
         out["note"] = note

@@ -18,6 +18,12 @@
 // (four per token) compute Phi and Psi in fp32 and store them as bf16 next
 // to V in one 128-byte-swizzled, MN-major stage [V | Psi | Phi], so a single
 // tcgen05.mma with M = d, N = 2d accumulates [Phi^T V | Phi^T Psi] in TMEM.
+// In the forward at d = 128 the kernel also computes each chunk's
+// per-feature log-sum-exp lse_s: it exponentiates against a running
+// per-feature reference (the column maximum of the tiles seen so far, raised
+// lazily with a rescale of the accumulated rows), reads the column sums of
+// those exponentials off the Cm block (every row of Psi sums to 1) and
+// normalises Bm and Cm in the epilogue, so K_m is read once.
 //
 // awm_carry_tc_kernel (d = 128): the sequential carry, one CTA per (b, h),
 // the product Cm_s M'_s as bf16 hi + lo MMAs; it also writes M'_s as the
@@ -46,7 +52,12 @@ namespace {
 //                D += Phi_hi^T [V | Psi_hi] + Phi_lo^T [V | Psi_hi], Cm += Phi_hi^T Psi_lo.
 //   kChunkE      E = psi(Q_m)^T dO_m for the backward (Q_m arrives in the
 //                K_m slot, dO_m in the V slot): stage [dO | psi_hi | psi_lo].
-enum ChunkMode { kChunkFwd = 0, kChunkSplit = 1, kChunkE = 2 };
+//   kChunkFwdStats  kChunkFwd with the chunk's per-feature log-sum-exp
+//                computed in the same pass (d = 128): Phi^ = exp(Km - m_f)
+//                with a lazily raised per-feature reference m_f, the column
+//                sums read off the Cm block (rows of Psi sum to 1), and
+//                Bm, Cm normalised in the epilogue, which also writes lse.
+enum ChunkMode { kChunkFwd = 0, kChunkSplit = 1, kChunkE = 2, kChunkFwdStats = 3 };
 
 template <int D, int Mode = kChunkFwd>
 struct ChunkCfg {
@@ -66,7 +77,11 @@ struct ChunkCfg {
   static constexpr int kNumBars = 3 * kStages + 1;
   static constexpr int kLzOff = kBarOff + kNumBars * 8;  // D floats: log2(e) * log z^s
   static constexpr int kMiscOff = kLzOff + D * 4;
-  static constexpr int kBytes = kMiscOff + 16;
+  // fused statistics: per-tile column maxima of K_m from 8 groups of 8 rows
+  // ([8][D] bf16, stored 16 bytes at a time)
+  static constexpr int kPartOff = (kMiscOff + 16 + 15) / 16 * 16;
+  static_assert(kPartOff % 16 == 0, "16-byte stores of the column maxima");
+  static constexpr int kBytes = kPartOff + (Mode == kChunkFwdStats ? 8 * D * 2 : 0);
   static constexpr int kAlloc = kBytes + 1024;
   static constexpr uint32_t kTmemCols = Mode == kChunkE ? D : (D == 128 ? 256 : 128);
 };
@@ -79,10 +94,15 @@ constexpr int kChunkCompute = 128, kChunkThreads = 192;
 template <int D, int Mode = kChunkFwd>
 __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_v,
                                                            const __grid_constant__ CUtensorMap map_km,
-                                                           const float* __restrict__ lse, float* __restrict__ Bm,
+                                                           float* __restrict__ lse, float* __restrict__ Bm,
                                                            float* __restrict__ Cm, uint16_t* __restrict__ Cimg,
                                                            int T, int c, int koff, int* status) {
   using Cfg = ChunkCfg<D, Mode>;
+  // kChunkFwdStats: the forward products with the chunk's statistics
+  // computed here (d = 128): it writes lse instead of reading it
+  constexpr bool kStats = Mode == kChunkFwdStats;
+  constexpr bool kFwd = Mode == kChunkFwd || kStats;
+  static_assert(!kStats || D == 128, "fused statistics need one thread per feature");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int NS = Cfg::kStages, kKT = Cfg::kKT;
@@ -115,7 +135,7 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (Mode != kChunkE)
+  if (Mode != kChunkE && !kStats)
     for (int f = threadIdx.x; f < D; f += blockDim.x) lz2[f] = lse[(bh * S + s) * D + f] * kLog2e;
   if (warp == 5) {
     tmem_alloc(tmem_slot, Cfg::kTmemCols);
@@ -170,7 +190,7 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
 #pragma unroll
         for (int kk = 0; kk < kKT / 16; ++kk) {
           const uint32_t acc = (kt > 0 || kk > 0) ? 1u : 0u;
-          if (Mode == kChunkFwd) {
+          if (kFwd) {
             // A = Phi^T (M = D features, MN-major), B = [V | Psi] (N = 2D, MN-major)
             umma_ss(tmem, desc(2, kk), desc(0, kk), idesc, acc);
           } else if (Mode == kChunkSplit) {
@@ -195,13 +215,80 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
     const int h = threadIdx.x % TPR;      // which part of the features
     constexpr int HF = D / TPR;           // features per thread
     bool ok = true;
+    // fused statistics: this thread's feature f = threadIdx.x (TMEM lane f
+    // of the accumulator) and its reference m_f (log2 units)
+    float m_f = 0.f;
     for (int kt = 0; kt < n_tiles; ++kt) {
       const int st = kt % NS;
       // V and K_m of this tile have landed (the copy also waited for the
       // MMAs of tile kt - NS to release the stage)
-      ok = __all_sync(0xffffffffu, mbar_wait(v_full + st, (kt / NS) & 1, abort_flag, status));
+      if (kStats) {
+        // the compute warps leave the loop together (they meet at named
+        // barriers below)
+        ok = bar_and(1, kChunkCompute, mbar_wait(v_full + st, (kt / NS) & 1, abort_flag, status));
+      } else {
+        ok = __all_sync(0xffffffffu, mbar_wait(v_full + st, (kt / NS) & 1, abort_flag, status));
+      }
       if (!ok) break;
       uint8_t* stg = smem + st * Cfg::kStage;
+      if (kStats) {
+        // Column maxima of the K_m tile: thread (rg, g) takes rows
+        // 8 rg .. 8 rg + 7 of features 8 g .. 8 g + 7, then thread f
+        // combines the 8 row groups of its feature.
+        __nv_bfloat162* part = reinterpret_cast<__nv_bfloat162*>(smem + Cfg::kPartOff);
+        {
+          const int g = threadIdx.x % 16, rg = threadIdx.x / 16;
+          uint4 mx = *reinterpret_cast<const uint4*>(stg + Cfg::kOperand + sw128_off(8 * rg, 8 * g, kKT));
+          __nv_bfloat162* m2 = reinterpret_cast<__nv_bfloat162*>(&mx);
+#pragma unroll
+          for (int rr = 1; rr < 8; ++rr) {
+            uint4 v = *reinterpret_cast<const uint4*>(stg + Cfg::kOperand + sw128_off(8 * rg + rr, 8 * g, kKT));
+            const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) m2[j] = __hmax2(m2[j], v2[j]);
+          }
+          *reinterpret_cast<uint4*>(part + rg * (D / 2) + 4 * g) = mx;
+        }
+        named_bar_sync(1, kChunkCompute);
+        const int f = threadIdx.x;
+        const __nv_bfloat16* ph = reinterpret_cast<const __nv_bfloat16*>(part);
+        float mt = __bfloat162float(ph[f]);
+#pragma unroll
+        for (int q = 1; q < 8; ++q) mt = fmaxf(mt, __bfloat162float(ph[q * D + f]));
+        const float mt2 = mt * kLog2e;
+        // The reference is raised lazily, only when the tile's maximum
+        // exceeds it by more than 8 (every exponential stays <= 2^8), and
+        // the accumulated rows of feature f are then scaled to the new one.
+        const bool grow = kt > 0 && mt2 > m_f + 8.f;
+        if (kt == 0) m_f = mt2;
+        bool rok = true;
+        if (__any_sync(0xffffffffu, grow)) {
+          // TMEM rows are scaled with warp-collective loads and stores once
+          // the MMAs of tile kt - 1 are done
+          rok = __all_sync(0xffffffffu, mbar_wait(st_empty + (kt - 1) % NS, ((kt - 1) / NS) & 1, abort_flag, status));
+          if (rok) {
+            tc_fence_after();
+            const float scale = grow ? ex2(m_f - mt2) : 1.f;
+            const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
+#pragma unroll 1
+            for (int cb = 0; cb < 2 * D / 32; ++cb) {
+              uint32_t v[32];
+              tmem_ld32(taddr + cb * 32, v);
+              tmem_wait_ld();
+#pragma unroll
+              for (int x = 0; x < 32; ++x) v[x] = __float_as_uint(__uint_as_float(v[x]) * scale);
+              tmem_st32(taddr + cb * 32, v);
+            }
+            tmem_wait_st();
+          }
+        }
+        if (grow) m_f = mt2;
+        lz2[f] = m_f;
+        // every reference is in place and every column maximum was read
+        // before K_m is overwritten by Psi below
+        ok = bar_and(1, kChunkCompute, rok);
+        if (!ok) break;
+      }
       float x[HF];
 #pragma unroll
       for (int i = 0; i < HF / 8; ++i) {
@@ -221,7 +308,7 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
       for (int o = 1; o < TPR; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       const float mx2 = mx * kLog2e;
       float e[HF], sum = 0.f;
-      if (Mode == kChunkFwd) {
+      if (kFwd) {
 #pragma unroll
         for (int i = 0; i < HF / 8; ++i) {
           const int col = h * HF + 8 * i;
@@ -279,16 +366,17 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
         for (int j = 0; j < 4; ++j) {
           const float a0 = e[8 * i + 2 * j] * inv, a1 = e[8 * i + 2 * j + 1] * inv;
           pp[j] = pack_bf16x2(a0, a1);
-          if (Mode != kChunkFwd) {
+          if (!kFwd) {
             const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pp[j]));
             plp[j] = pack_bf16x2(a0 - hi.x, a1 - hi.y);
           }
         }
         *reinterpret_cast<uint4*>(stg + Cfg::kOperand + sw128_off(r, col, kKT)) = ps;
-        if (Mode != kChunkFwd) *reinterpret_cast<uint4*>(stg + 2 * Cfg::kOperand + sw128_off(r, col, kKT)) = pl;
+        if (!kFwd) *reinterpret_cast<uint4*>(stg + 2 * Cfg::kOperand + sw128_off(r, col, kKT)) = pl;
       }
       // generic-proxy writes must be visible to the tensor core (async proxy)
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      if (kStats) tc_fence_before();   // orders the TMEM rescale before the next MMA
       mbar_arrive(op_full + st);
     }
     // epilogue: accumulator row f = TMEM lane; columns [0, D) = Bm, [D, 2D) = Cm
@@ -301,18 +389,39 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
       const int f = D == 128 ? warp * 32 + lane : warp * 16 + lane;
       const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
       const int64_t o = (bh * S + s) * (int64_t)D * D + (int64_t)f * D;
+      // fused statistics: the column sum of Phi^ over the chunk is the row
+      // sum of the Cm block (every row of Psi sums to 1); Bm and Cm rows are
+      // divided by it and lse_f = ln(sum) + m_f ln 2
+      float inv = 1.f;
+      if (kStats) {
+        float sum = 0.f;
+#pragma unroll 1
+        for (int cb = D / 32; cb < 2 * D / 32; ++cb) {
+          uint32_t v[32];
+          tmem_ld32(taddr + cb * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int x = 0; x < 32; ++x) sum += __uint_as_float(v[x]);
+        }
+        inv = 1.f / sum;
+        lse[(bh * S + s) * D + f] = (m_f + log2f(sum)) * kLn2;
+      }
 #pragma unroll 1
       for (int cb = 0; cb < (Mode == kChunkE ? D : 2 * D) / 32; ++cb) {
         uint32_t v[32];
         tmem_ld32(taddr + cb * 32, v);
         tmem_wait_ld();
+        if (kStats) {
+#pragma unroll
+          for (int x = 0; x < 32; ++x) v[x] = __float_as_uint(__uint_as_float(v[x]) * inv);
+        }
         if (valid) {
           float* dst = (cb * 32 < D) ? (Bm + o + cb * 32) : (Cm + o + cb * 32 - D);
 #pragma unroll
           for (int i = 0; i < 8; ++i)
             reinterpret_cast<float4*>(dst)[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
                                                             __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-          if (Mode == kChunkFwd && D == 128 && Cimg && cb * 32 >= D) {
+          if (kFwd && D == 128 && Cimg && cb * 32 >= D) {
             // Cm row f as the tensor-core carry's bf16 A operand (K-major)
             uint8_t* img = reinterpret_cast<uint8_t*>(Cimg + (bh * S + s) * (int64_t)D * D);
 #pragma unroll
@@ -350,25 +459,34 @@ struct ReadoutCfg {
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;
   static constexpr uint32_t kTmemCols = 2 * D;   // two accumulators
-  static constexpr int kThreads = 320;
+  // psi warps (4: one thread per row; 8: two per row, measured 0.129 against
+  // 0.135 ms at the bench workload); then 4 epilogue warps, the TMA warp
+  // and the MMA warp
+#ifndef GECKO_READOUT_PSI_WARPS
+#define GECKO_READOUT_PSI_WARPS 8
+#endif
+  static constexpr int kPsiWarps = GECKO_READOUT_PSI_WARPS;
+  static constexpr int kTPR = kPsiWarps / 4;     // psi threads per row
+  static constexpr int kEpiWarp0 = kPsiWarps, kTmaWarp = kPsiWarps + 4, kMmaWarp = kPsiWarps + 5;
+  static constexpr int kThreads = (kPsiWarps + 6) * 32;
 };
 
 // The readout O_m,s = psi(Qm_s) M'_{s-1} (Gecko digest, method step details,
 // step 5).  Persistent: CTA b takes a contiguous range of the 128-row tiles
 // ordered by (b, h), chunk, tile, balanced by weight (a tile of chunks 1
 // and 2 of a fresh sequence only writes zeros: weight 1; every other tile
-// reads Q_m and writes out_mem: weight 2).  320 threads:
-//   warps 0-3  psi: each thread turns its row of the Q_m tile (TMA, K-major
-//              A operand layout) into the numerators exp(q - max) in place,
-//              bf16, and keeps 1 / sum for the epilogue;
-//   warps 4-7  epilogue: accumulator rows from TMEM scaled by 1 / sum,
+// reads Q_m and writes out_mem: weight 2).  448 threads:
+//   warps 0-7  psi: two threads per row turn it (Q_m tile by TMA, K-major A
+//              operand layout) into the numerators exp(q - max) in place,
+//              bf16, and keep 1 / sum for the epilogue;
+//   warps 8-11 epilogue: accumulator rows from TMEM scaled by 1 / sum,
 //              bf16, written over the tile's stage and stored by one TMA
 //              store; zero tiles are written directly;
-//   warp 8     TMA producer: Q_m tiles into a 4-stage ring, and the operand
+//   warp 12    TMA producer: Q_m tiles into a 4-stage ring, and the operand
 //              image of M'_{s-1} (bf16, written by the carry in the MN-major
 //              B layout) by one bulk copy whenever the chunk changes
 //              (two image buffers);
-//   warp 9     TMEM allocation and the MMAs (one thread), two accumulators.
+//   warp 13    TMEM allocation and the MMAs (one thread), two accumulators.
 template <int D>
 __global__ void __launch_bounds__(ReadoutCfg<D>::kThreads, 1)
 awm_readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_o,
@@ -426,7 +544,7 @@ awm_readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
   if (threadIdx.x == 0) {
     for (int i = 0; i < NS; ++i) {
       mbar_init(q_full + i, 1);
-      mbar_init(op_full + i, 128);
+      mbar_init(op_full + i, Cfg::kPsiWarps * 32);
       mbar_init(st_empty + i, 1);
       mbar_init(out_ready + i, 128);
     }
@@ -440,7 +558,7 @@ awm_readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == Cfg::kMmaWarp) {
     tmem_alloc(tmem_slot, Cfg::kTmemCols);
     tmem_relinquish();
   }
@@ -449,7 +567,7 @@ awm_readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == Cfg::kTmaWarp) {
     // --------------------------------------------------- TMA producer --
     if (lane == 0) {
       tma_prefetch_desc(&map_q);
@@ -482,7 +600,7 @@ awm_readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
       }
     }
     __syncwarp();
-  } else if (warp == 9) {
+  } else if (warp == Cfg::kMmaWarp) {
     // ------------------------------------------------------- MMA issuer --
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, true);
@@ -521,9 +639,11 @@ awm_readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
       mbar_wait_drain(drain, 0);
     }
     __syncwarp();
-  } else if (warp < 4) {
+  } else if (warp < Cfg::kPsiWarps) {
     // -------------------------------------------------- psi numerators --
-    const int r = threadIdx.x;   // row of the tile
+    constexpr int TPR = Cfg::kTPR, CPT = D / TPR;   // threads per row, columns per thread
+    const int r = threadIdx.x / TPR;                // row of the tile
+    const int c0 = (threadIdx.x % TPR) * CPT;
     int n = 0;
     bool ok = true;
     TileIt t = first;
@@ -535,8 +655,8 @@ awm_readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
       uint8_t* tile = smem + st * Cfg::kTile;
       float mx = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < D / 8; ++i) {
-        const uint4 q = *reinterpret_cast<const uint4*>(tile + sw128_off(r, 8 * i, 128));
+      for (int i = 0; i < CPT / 8; ++i) {
+        const uint4 q = *reinterpret_cast<const uint4*>(tile + sw128_off(r, c0 + 8 * i, 128));
         const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&q);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -544,11 +664,12 @@ awm_readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
           mx = fmax3(mx, f2.x, f2.y);
         }
       }
+      if (TPR == 2) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
       const float mx2 = mx * kLog2e;
       float sum = 0.f;
 #pragma unroll
-      for (int i = 0; i < D / 8; ++i) {
-        uint4* qa = reinterpret_cast<uint4*>(tile + sw128_off(r, 8 * i, 128));
+      for (int i = 0; i < CPT / 8; ++i) {
+        uint4* qa = reinterpret_cast<uint4*>(tile + sw128_off(r, c0 + 8 * i, 128));
         const uint4 q = *qa;
         const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&q);
         uint4 pv;
@@ -563,7 +684,8 @@ awm_readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
         }
         *qa = pv;
       }
-      rinv[st * 128 + r] = 1.f / sum;
+      if (TPR == 2) sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+      if (c0 == 0) rinv[st * 128 + r] = 1.f / sum;
       fence_proxy_async_smem();   // the numerators are read by the tensor core (async proxy)
       mbar_arrive(op_full + st);
       ++n;
@@ -573,7 +695,7 @@ awm_readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
     const int q4 = warp % 4;                       // TMEM lane quarter
     const int r = q4 * 32 + lane;                  // row of the tile
     const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
-    const bool leader = warp == 4 && lane == 0;   // issues the stores
+    const bool leader = warp == Cfg::kEpiWarp0 && lane == 0;   // issues the stores
     int n = 0;
     bool ok = true;
     TileIt t = first;
@@ -628,7 +750,7 @@ awm_readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 9) tmem_dealloc(tmem, Cfg::kTmemCols);
+  if (warp == Cfg::kMmaWarp) tmem_dealloc(tmem, Cfg::kTmemCols);
 }
 
 // ------------------------------------------------------------------ carry --
@@ -863,7 +985,7 @@ EncodeTiledFn encode_fn() {
 }
 
 template <int D, int Mode>
-cudaError_t chunk_impl(const Problem& p, const void* vsrc, const void* ksrc, const float* lse, float* out0,
+cudaError_t chunk_impl(const Problem& p, const void* vsrc, const void* ksrc, float* lse, float* out0,
                        float* out1, cudaStream_t st, uint16_t* cimg = nullptr) {
   using Cfg = ChunkCfg<D, Mode>;
   EncodeTiledFn fn = encode_fn();
@@ -949,6 +1071,11 @@ cudaError_t launch_awm_carry_tc(const Problem& p, const Workspace& w, cudaStream
 cudaError_t launch_awm_chunk_tc(const Problem& p, const Workspace& w, cudaStream_t st) {
   return p.d == 64 ? chunk_impl<64, kChunkFwd>(p, p.v, p.km, w.lse, w.Bm, w.Cm, st)
                    : chunk_impl<128, kChunkFwd>(p, p.v, p.km, w.lse, w.Bm, w.Cm, st, w.Cimg);
+}
+
+cudaError_t launch_awm_chunk_tc_stats(const Problem& p, const Workspace& w, cudaStream_t st) {
+  if (p.d != 128) return cudaErrorInvalidValue;
+  return chunk_impl<128, kChunkFwdStats>(p, p.v, p.km, w.lse, w.Bm, w.Cm, st, w.Cimg);
 }
 
 cudaError_t launch_awm_chunk_tc_split(const Problem& p, const Workspace& w, cudaStream_t st) {

@@ -262,6 +262,26 @@ int ensure_buffer(void** buf, size_t* have, size_t need, cudaStream_t st, const 
   return GECKO_OK;
 }
 
+// The forward's AWM statistics at d = 128 on the tensor cores come from the
+// chunk kernel itself (each chunk's per-feature log-sum-exp is read off its
+// Cm block), which saves a second pass over K_m; the prefix over chunks then
+// runs after it.  Elsewhere a statistics pass precedes the chunk products.
+// GECKO_FUSED_STATS=0 at build time keeps the separate pass everywhere.
+#ifndef GECKO_FUSED_STATS
+#define GECKO_FUSED_STATS 1
+#endif
+bool fused_stats(const Problem& p, bool use_tc) { return GECKO_FUSED_STATS && use_tc && p.d == 128; }
+
+// The chunk products (and, when fused, the statistics and the prefix).
+int awm_chunks(const Problem& p, const Workspace& w, cudaStream_t st, bool use_tc, bool fused) {
+  int rc;
+  if (fused) {
+    if ((rc = check_cuda(launch_awm_chunk_tc_stats(p, w, st), "awm chunk"))) return rc;
+    return check_cuda(launch_awm_prefix(p, w, st), "awm prefix");
+  }
+  return check_cuda(use_tc ? launch_awm_chunk_tc(p, w, st) : launch_awm_chunk_simt(p, w, st), "awm chunk");
+}
+
 // The allocating forward, fresh (state_in == nullptr) or continuing a
 // sequence (k, v with c prepended rows per (b, h); state_in on the device
 // or host).  state_out, if given, receives (M'_S, M'_{S+1}, log z^S).
@@ -309,10 +329,10 @@ int run_forward(const void* q, const void* k, const void* v, const void* qm, con
   cudaGetLastError();  // clear stale errors from the caller
   StageEvents ev(st);
   ev.mark(0);
-  if ((rc = check_cuda(launch_awm_stats(p, w, st), "awm stats"))) return rc;
+  const bool fused = fused_stats(p, use_tc);
+  if (!fused && (rc = check_cuda(launch_awm_stats(p, w, st), "awm stats"))) return rc;
   ev.mark(1);
-  if ((rc = check_cuda(use_tc ? launch_awm_chunk_tc(p, w, st) : launch_awm_chunk_simt(p, w, st), "awm chunk")))
-    return rc;
+  if ((rc = awm_chunks(p, w, st, use_tc, fused))) return rc;
   ev.mark(2);
   if ((rc = check_cuda(use_tc && d == 128 ? launch_awm_carry_tc(p, w, st, true) : launch_awm_carry(p, w, st, use_tc),
                        "awm carry")))
@@ -680,9 +700,9 @@ extern "C" int gecko_sca_awm_forward_noalloc(const void* q, const void* k, const
   Problem p{q, k, v, qm, km, out_sca, out_mem, B, H, T, c, d, (int)S, dtype, ds->status};
   const bool use_tc = !env_is("GECKO_KERNELS", "simt") && tc_supported(p);
   cudaGetLastError();
-  if ((rc = check_cuda(launch_awm_stats(p, w, st), "awm stats"))) return rc;
-  if ((rc = check_cuda(use_tc ? launch_awm_chunk_tc(p, w, st) : launch_awm_chunk_simt(p, w, st), "awm chunk")))
-    return rc;
+  const bool fused = fused_stats(p, use_tc);
+  if (!fused && (rc = check_cuda(launch_awm_stats(p, w, st), "awm stats"))) return rc;
+  if ((rc = awm_chunks(p, w, st, use_tc, fused))) return rc;
   if ((rc = check_cuda(use_tc && d == 128 ? launch_awm_carry_tc(p, w, st, true) : launch_awm_carry(p, w, st, use_tc),
                        "awm carry")))
     return rc;

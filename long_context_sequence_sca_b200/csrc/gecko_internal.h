@@ -67,6 +67,7 @@ Workspace carve_workspace(void* base, int64_t BH, int64_t T, int64_t c, int64_t 
 
 // CUDA-core kernels (any dtype, any c % 64 == 0).
 cudaError_t launch_awm_stats(const Problem& p, const Workspace& w, cudaStream_t st);   // lse + log z prefix
+cudaError_t launch_awm_prefix(const Problem& p, const Workspace& w, cudaStream_t st);  // log z prefix from lse
 cudaError_t launch_awm_chunk_simt(const Problem& p, const Workspace& w, cudaStream_t st);
 // images: also write the readout operand images (Workspace::Mimg)
 cudaError_t launch_awm_carry(const Problem& p, const Workspace& w, cudaStream_t st, bool images = false);
@@ -80,6 +81,8 @@ int sm_count();
 bool tc_supported(const Problem& p);
 cudaError_t launch_sca_tc(const Problem& p, cudaStream_t st);
 cudaError_t launch_awm_chunk_tc(const Problem& p, const Workspace& w, cudaStream_t st);
+// d = 128: the chunk products with each chunk's log-sum-exp (Workspace::lse) computed in the same pass
+cudaError_t launch_awm_chunk_tc_stats(const Problem& p, const Workspace& w, cudaStream_t st);
 cudaError_t launch_awm_readout_tc(const Problem& p, const Workspace& w, cudaStream_t st);
 // The carry on the tensor cores (d = 128; bf16 hi + lo operands, ~fp32 products)
 cudaError_t launch_awm_carry_tc(const Problem& p, const Workspace& w, cudaStream_t st, bool images);

@@ -539,6 +539,13 @@ cudaError_t awm_stats_impl(const Problem& p, const Workspace& w, cudaStream_t st
   return cudaGetLastError();
 }
 
+template <int D>
+cudaError_t awm_prefix_impl(const Problem& p, const Workspace& w, cudaStream_t st) {
+  awm_prefix_kernel<D><<<p.B * p.H, D, 0, st>>>(w.lse, w.logz, w.ratio, w.rho, p.S,
+                                               p.state0 ? p.state0 + 2 * D * D : nullptr, state_floats(D));
+  return cudaGetLastError();
+}
+
 template <typename TIn, int D>
 cudaError_t awm_chunk_simt_impl(const Problem& p, const Workspace& w, cudaStream_t st) {
   awm_chunk_simt_kernel<TIn, D><<<dim3(p.S, p.B * p.H), 256, 0, st>>>(
@@ -591,6 +598,9 @@ cudaError_t launch_sca_simt_impl(const Problem& p, cudaStream_t st) {
 
 cudaError_t launch_awm_stats(const Problem& p, const Workspace& w, cudaStream_t st) {
   return GECKO_DISPATCH(awm_stats_impl);
+}
+cudaError_t launch_awm_prefix(const Problem& p, const Workspace& w, cudaStream_t st) {
+  return p.d == 64 ? awm_prefix_impl<64>(p, w, st) : awm_prefix_impl<128>(p, w, st);
 }
 cudaError_t launch_awm_chunk_simt(const Problem& p, const Workspace& w, cudaStream_t st) {
   return GECKO_DISPATCH(awm_chunk_simt_impl);

@@ -194,3 +194,32 @@ def test_repeat_calls_are_deterministic(L):
     b = L.sca_awm_forward(x["q"], x["k"], x["v"], x["qm"], x["km"], w.c)
     torch.cuda.synchronize()
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("kernels", [None, "simt"])
+def test_awm_keys_growing_within_a_chunk(L, kernels, monkeypatch):
+    """K_m features whose values climb through each chunk (by up to 30 over
+    the chunk, and one late spike of +40) and others that fall: the
+    chunk-local exponentials of a feature cannot share one reference taken
+    early in the chunk, so a kernel that tracks the per-feature maximum as
+    it streams the chunk must raise it and rescale what it has accumulated.
+    The chunk's log-sum-exp, the state and the readout still match the fp64
+    oracle (step 4 of the method: Phi = exp(Km - log z), any real Km)."""
+    if kernels:
+        monkeypatch.setenv("GECKO_KERNELS", kernels)
+    w = Workload("bf16_growing_keys", 19, "bf16", 1, 2, 1536, 128, 512)
+    x = make_inputs(w, device="cuda")
+    c, d = w.c, w.d
+    t = (torch.arange(w.T, device="cuda") % c).float() / c
+    f = torch.arange(d, device="cuda")
+    slope = torch.where(f % 4 == 0, 30.0 * (f.float() / d), torch.where(f % 4 == 1, -12.0, 0.0))
+    km = x["km"].float() + t[:, None] * slope[None, :]
+    spike = (torch.arange(w.T, device="cuda") % c) == c - 70
+    km[..., spike, 2::8] += 40.0
+    x["km"] = km.to(torch.bfloat16)
+    o_sca, o_mem, M, lz = _run(L, x, w.c)
+    r_sca, r_mem, r_M, r_lz = G.forward(*(_np(x[n]) for n in ("q", "k", "v", "qm", "km")), w.c)
+    _check(_np(o_mem), r_mem, w.dtype, "out_mem")
+    _check(_np(M), r_M, w.dtype, "M state")
+    _check(_np(lz), r_lz, w.dtype, "log z")
+    _check(_np(o_sca), r_sca, w.dtype, "out_sca")
