@@ -508,13 +508,14 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
         const int jb = U.beg[0], je = U.nt == 2 ? U.end[1] : U.end[0];
         for (int j = jb; j <= je && ok; ++j) {
           const uint32_t stK = kv_it % KS;
-          bool k_ready = false;  // K_j is waited for only right before the first QK that reads it
-          const uint32_t itV = kv_it - 1;  // V_{j-1}
-          const uint32_t stV = itV % VS;
-          if (j > jb) {
-            if (!(ok = mbar_wait(v_full + stV, (itV / VS) & 1, abort_flag, status))) break;
-            tc_fence_after();
-          }
+          // K_j and V_j are waited for together, right before the first QK
+          // of iteration j (V_j is first read by the PVs of iteration j + 1).
+          // A wait placed right after a group of MMAs overlaps the tensor
+          // core's work on that group; at the top of the iteration it would
+          // add to the gap before the next PV (SCA kernel 2.68-2.74 against
+          // 2.75-2.77 ms on the bench workload).
+          bool k_ready = false;
+          const uint32_t stV = (kv_it - 1) % VS;   // V_{j-1}, waited for in iteration j - 1
           for (int i = 0; i < U.nt && ok; ++i) {
             const uint32_t colS = i == 0 ? Cfg::kColS0 : Cfg::kColS1;
             const uint32_t colO = i == 0 ? Cfg::kColO0 : Cfg::kColO1;
@@ -539,6 +540,7 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
             if (j >= ubeg(U, i) && j < uend(U, i)) {
               if (!k_ready) {
                 if (!(ok = mbar_wait(k_full + stK, (kv_it / KS) & 1, abort_flag, status))) break;
+                if (!(ok = mbar_wait(v_full + kv_it % VS, (kv_it / VS) & 1, abort_flag, status))) break;
                 tc_fence_after();
                 k_ready = true;
               }
