@@ -9,13 +9,13 @@
 //   Bm_s = Phi~_s^T V_s,   Cm_s = Phi~_s^T Psi_s        (d x d, fp32)
 // independently of the prefix over chunks, and the carry applies the row
 // scales: M'_{s+1} = r_s (.) M'_s + rho_s (.) (Bm_s - Cm_s M'_s).  The
-// readout is O_m,s = psi(Qm_s) M'_{s-1}.  Phi~, Psi and psi take their
-// exponentials in packed f16 (two per SFU op); they enter the tensor core as
-// bf16, whose 8-bit mantissa is coarser than f16's.
+// readout is O_m,s = psi(Qm_s) M'_{s-1}.  Phi~, Psi and psi take fp32
+// exponentials on the SFU (packed f16 ones give the same number of results
+// per clock on B200 and cost conversions) and enter the tensor core as bf16.
 //
 // awm_chunk_tc_kernel: one CTA per (chunk, bh), two per SM.  The chunk is
-// streamed in tiles of 64 tokens; V and K_m tiles arrive by TMA; 256 threads
-// (four per token) compute Phi and Psi in fp32 and store them as bf16 next
+// streamed in tiles of 64 tokens; V and K_m tiles arrive by TMA; 128 threads
+// (two per token) compute Phi and Psi in fp32 and store them as bf16 next
 // to V in one 128-byte-swizzled, MN-major stage [V | Psi | Phi], so a single
 // tcgen05.mma with M = d, N = 2d accumulates [Phi^T V | Phi^T Psi] in TMEM.
 // In the forward at d = 128 the kernel also computes each chunk's
@@ -43,8 +43,8 @@ namespace {
 
 
 // What a chunk-kernel launch computes.
-//   kChunkFwd    Bm = Phi~^T V, Cm = Phi~^T Psi with bf16 operands (f16
-//                exponentials): stage [V | Psi | Phi].
+//   kChunkFwd    Bm = Phi~^T V, Cm = Phi~^T Psi with bf16 operands:
+//                stage [V | Psi | Phi].
 //   kChunkSplit  the same products with each computed operand carried as two
 //                bf16 parts (hi + lo, fp32 exponentials), for a backward whose
 //                softmax gradients keep only the small differences between
@@ -75,7 +75,10 @@ struct ChunkCfg {
   static constexpr int kBarOff = kStages * kStage;
   // v_full[kStages], op_full[kStages], stage_empty[kStages], acc_full
   static constexpr int kNumBars = 3 * kStages + 1;
-  static constexpr int kLzOff = kBarOff + kNumBars * 8;  // D floats: log2(e) * log z^s
+  // D floats: -log2(e) times each feature's reference (16-byte aligned for
+  // vector loads)
+  static constexpr int kLzOff = (kBarOff + kNumBars * 8 + 15) / 16 * 16;
+  static_assert(kLzOff % 16 == 0, "vector loads of the references");
   static constexpr int kMiscOff = kLzOff + D * 4;
   // fused statistics: per-tile column maxima of K_m from 8 groups of 8 rows
   // ([8][D] bf16, stored 16 bytes at a time)
@@ -111,7 +114,8 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
   uint64_t* op_full = bars + NS;    // [NS] compute -> MMA (128 arrivals)
   uint64_t* st_empty = bars + 2 * NS;   // [NS] MMA -> TMA, compute
   uint64_t* acc_full = bars + 3 * NS;
-  float* lz2 = reinterpret_cast<float*>(smem + Cfg::kLzOff);  // log2(e) * lse_s
+  // -log2(e) * (the reference of each feature): lse_s, or m_f with the fused statistics
+  float* nref2 = reinterpret_cast<float*>(smem + Cfg::kLzOff);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
 
@@ -136,7 +140,7 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
     fence_mbar_init();
   }
   if (Mode != kChunkE && !kStats)
-    for (int f = threadIdx.x; f < D; f += blockDim.x) lz2[f] = lse[(bh * S + s) * D + f] * kLog2e;
+    for (int f = threadIdx.x; f < D; f += blockDim.x) nref2[f] = -lse[(bh * S + s) * D + f] * kLog2e;
   if (warp == 5) {
     tmem_alloc(tmem_slot, Cfg::kTmemCols);
     tmem_relinquish();
@@ -283,7 +287,7 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
           }
         }
         if (grow) m_f = mt2;
-        lz2[f] = m_f;
+        nref2[f] = -m_f;
         // every reference is in place and every column maximum was read
         // before K_m is overwritten by Psi below
         ok = bar_and(1, kChunkCompute, rok);
@@ -301,30 +305,50 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
           x[8 * i + 2 * j + 1] = f2.y;
         }
       }
-      float mx = x[0];
+      // row maximum over this thread's features (four 3-input chains)
+      float m4[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
-      for (int i = 1; i < HF; ++i) mx = fmaxf(mx, x[i]);
+      for (int i = 4; i + 8 <= HF; i += 8)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) m4[q] = fmax3(m4[q], x[i + q], x[i + 4 + q]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) m4[q] = fmaxf(m4[q], x[HF - 4 + q]);
+      float mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
 #pragma unroll
       for (int o = 1; o < TPR; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       const float mx2 = mx * kLog2e;
       float e[HF], sum = 0.f;
       if (kFwd) {
+        // fp32 exponentials on the SFU (the packed f16 form gives the same
+        // number of results per clock and costs conversions); arguments by
+        // packed FMA
+        const uint64_t l2e2 = pack2(kLog2e, kLog2e), nmx2 = pack2(-mx2, -mx2);
+        uint64_t sum2 = pack2(0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < HF / 8; ++i) {
           const int col = h * HF + 8 * i;
+          const float4 za = *reinterpret_cast<const float4*>(nref2 + col);
+          const float4 zb = *reinterpret_cast<const float4*>(nref2 + col + 4);
+          const uint64_t nz[4] = {pack2(za.x, za.y), pack2(za.z, za.w), pack2(zb.x, zb.y), pack2(zb.z, zb.w)};
           uint4 pf;
           uint32_t* qq = reinterpret_cast<uint32_t*>(&pf);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int a = 8 * i + 2 * j;
-            float p0, p1;
-            ex2_h2(fmaf(x[a], kLog2e, -lz2[col + 2 * j]), fmaf(x[a + 1], kLog2e, -lz2[col + 2 * j + 1]), p0, p1);
-            qq[j] = pack_bf16x2(p0, p1);
-            ex2_h2(fmaf(x[a], kLog2e, -mx2), fmaf(x[a + 1], kLog2e, -mx2), e[a], e[a + 1]);
-            sum += e[a] + e[a + 1];
+            const uint64_t x2 = pack2(x[a], x[a + 1]);
+            float u0, u1, v0, v1;
+            unpack2(ffma2(x2, l2e2, nz[j]), u0, u1);
+            qq[j] = pack_bf16x2(ex2(u0), ex2(u1));
+            unpack2(ffma2(x2, l2e2, nmx2), v0, v1);
+            e[a] = ex2(v0);
+            e[a + 1] = ex2(v1);
+            sum2 = fadd2(sum2, pack2(e[a], e[a + 1]));
           }
           *reinterpret_cast<uint4*>(stg + 2 * Cfg::kOperand + sw128_off(r, col, kKT)) = pf;
         }
+        float s0, s1;
+        unpack2(sum2, s0, s1);
+        sum = s0 + s1;
       } else {
         // fp32 exponentials; Phi (split mode only) as bf16 hi and lo parts
 #pragma unroll
@@ -337,8 +361,8 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
           for (int j = 0; j < 4; ++j) {
             const int a = 8 * i + 2 * j;
             if (Mode == kChunkSplit) {
-              const float p0 = ex2(fmaf(x[a], kLog2e, -lz2[col + 2 * j]));
-              const float p1 = ex2(fmaf(x[a + 1], kLog2e, -lz2[col + 2 * j + 1]));
+              const float p0 = ex2(fmaf(x[a], kLog2e, nref2[col + 2 * j]));
+              const float p1 = ex2(fmaf(x[a + 1], kLog2e, nref2[col + 2 * j + 1]));
               fhp[j] = pack_bf16x2(p0, p1);
               const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&fhp[j]));
               flp[j] = pack_bf16x2(p0 - hi.x, p1 - hi.y);
@@ -364,7 +388,8 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
         uint32_t* plp = reinterpret_cast<uint32_t*>(&pl);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const float a0 = e[8 * i + 2 * j] * inv, a1 = e[8 * i + 2 * j + 1] * inv;
+          float a0, a1;
+          unpack2(fmul2(pack2(e[8 * i + 2 * j], e[8 * i + 2 * j + 1]), pack2(inv, inv)), a0, a1);
           pp[j] = pack_bf16x2(a0, a1);
           if (!kFwd) {
             const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pp[j]));
@@ -666,7 +691,9 @@ awm_readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
       }
       if (TPR == 2) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
       const float mx2 = mx * kLog2e;
-      float sum = 0.f;
+      // fp32 exponentials on the SFU, arguments by packed FMA
+      const uint64_t l2e2 = pack2(kLog2e, kLog2e), nmx2 = pack2(-mx2, -mx2);
+      uint64_t sum2 = pack2(0.f, 0.f);
 #pragma unroll
       for (int i = 0; i < CPT / 8; ++i) {
         uint4* qa = reinterpret_cast<uint4*>(tile + sw128_off(r, c0 + 8 * i, 128));
@@ -677,13 +704,17 @@ awm_readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const float2 f2 = __bfloat1622float2(p2[j]);
-          float e0, e1;
-          ex2_h2(fmaf(f2.x, kLog2e, -mx2), fmaf(f2.y, kLog2e, -mx2), e0, e1);
-          sum += e0 + e1;
+          float u0, u1;
+          unpack2(ffma2(pack2(f2.x, f2.y), l2e2, nmx2), u0, u1);
+          const float e0 = ex2(u0), e1 = ex2(u1);
+          sum2 = fadd2(sum2, pack2(e0, e1));
           pp[j] = pack_bf16x2(e0, e1);
         }
         *qa = pv;
       }
+      float sum, s1;
+      unpack2(sum2, sum, s1);
+      sum += s1;
       if (TPR == 2) sum += __shfl_xor_sync(0xffffffffu, sum, 1);
       if (c0 == 0) rinv[st * 128 + r] = 1.f / sum;
       fence_proxy_async_smem();   // the numerators are read by the tensor core (async proxy)
