@@ -59,6 +59,11 @@ namespace {
 //                Bm, Cm normalised in the epilogue, which also writes lse.
 enum ChunkMode { kChunkFwd = 0, kChunkSplit = 1, kChunkE = 2, kChunkFwdStats = 3 };
 
+// Compute threads of the chunk kernel: two per token row of a 64-token
+// tile.  (Eight compute warps, four threads per row, measured slower: 0.228
+// against 0.219-0.224 ms at the bench workload; so did hinting the next 2-8
+// tiles into L2 ahead of the two-stage ring: no change.)
+constexpr int kChunkCompute = 128;
 template <int D, int Mode = kChunkFwd>
 struct ChunkCfg {
   // Tokens per tile and stages.  32-token tiles through 4 stages (three
@@ -67,7 +72,7 @@ struct ChunkCfg {
   // 64-token tiles through 2 stages.
   static constexpr int kKT = 64;
   static constexpr int kStages = 2;
-  static constexpr int kTPR = 128 / kKT;                 // compute threads per token row
+  static constexpr int kTPR = kChunkCompute / kKT;        // compute threads per token row
   static constexpr int kBox = kKT * 128;                 // one [kKT x 64] bf16 box
   static constexpr int kOperand = (D / 64) * kBox;       // a [kKT x D] operand
   static constexpr int kSlots = Mode == kChunkSplit ? 5 : 3;
@@ -89,11 +94,10 @@ struct ChunkCfg {
   static constexpr uint32_t kTmemCols = Mode == kChunkE ? D : (D == 128 ? 256 : 128);
 };
 
-// 128 compute threads (warps 0-3, two per token row), warp 4 = TMA
-// producer, warp 5 = MMA issuer; two CTAs per SM.  (Eight compute warps,
-// four per row, measured slower: 0.191 against 0.183 ms at the bench
-// workload.)
-constexpr int kChunkCompute = 128, kChunkThreads = 192;
+// Warps 0-3 compute, warp 4 = TMA producer, warp 5 = MMA issuer; two CTAs
+// per SM.
+constexpr int kChunkThreads = kChunkCompute + 64;
+constexpr int kChunkTmaWarp = kChunkCompute / 32, kChunkMmaWarp = kChunkTmaWarp + 1;
 template <int D, int Mode = kChunkFwd>
 __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_v,
                                                            const __grid_constant__ CUtensorMap map_km,
@@ -141,7 +145,7 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
   }
   if (Mode != kChunkE && !kStats)
     for (int f = threadIdx.x; f < D; f += blockDim.x) nref2[f] = -lse[(bh * S + s) * D + f] * kLog2e;
-  if (warp == 5) {
+  if (warp == kChunkMmaWarp) {
     tmem_alloc(tmem_slot, Cfg::kTmemCols);
     tmem_relinquish();
   }
@@ -150,7 +154,7 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == kChunkTmaWarp) {
     // ------------------------------------------------ V and K_m by TMA --
     // V into the V slot, K_m into the Psi slot (where it is turned into Psi
     // in place), both on v_full.
@@ -176,7 +180,7 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == kChunkMmaWarp) {
     // --------------------------------------------------------- MMA issuer --
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(D, 2 * D, true, true);
@@ -240,7 +244,8 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
         // 8 rg .. 8 rg + 7 of features 8 g .. 8 g + 7, then thread f
         // combines the 8 row groups of its feature.
         __nv_bfloat162* part = reinterpret_cast<__nv_bfloat162*>(smem + Cfg::kPartOff);
-        {
+        const bool feat = threadIdx.x < D;   // warps 0-3: one feature (TMEM lane) per thread
+        if (feat) {
           const int g = threadIdx.x % 16, rg = threadIdx.x / 16;
           uint4 mx = *reinterpret_cast<const uint4*>(stg + Cfg::kOperand + sw128_off(8 * rg, 8 * g, kKT));
           __nv_bfloat162* m2 = reinterpret_cast<__nv_bfloat162*>(&mx);
@@ -254,16 +259,16 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
           *reinterpret_cast<uint4*>(part + rg * (D / 2) + 4 * g) = mx;
         }
         named_bar_sync(1, kChunkCompute);
-        const int f = threadIdx.x;
+        const int f = feat ? threadIdx.x : 0;
         const __nv_bfloat16* ph = reinterpret_cast<const __nv_bfloat16*>(part);
         float mt = __bfloat162float(ph[f]);
 #pragma unroll
         for (int q = 1; q < 8; ++q) mt = fmaxf(mt, __bfloat162float(ph[q * D + f]));
-        const float mt2 = mt * kLog2e;
+        const float mt2 = feat ? mt * kLog2e : 0.f;
         // The reference is raised lazily, only when the tile's maximum
         // exceeds it by more than 8 (every exponential stays <= 2^8), and
         // the accumulated rows of feature f are then scaled to the new one.
-        const bool grow = kt > 0 && mt2 > m_f + 8.f;
+        const bool grow = feat && kt > 0 && mt2 > m_f + 8.f;
         if (kt == 0) m_f = mt2;
         bool rok = true;
         if (__any_sync(0xffffffffu, grow)) {
@@ -287,7 +292,7 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
           }
         }
         if (grow) m_f = mt2;
-        nref2[f] = -m_f;
+        if (feat) nref2[f] = -m_f;
         // every reference is in place and every column maximum was read
         // before K_m is overwritten by Psi below
         ok = bar_and(1, kChunkCompute, rok);
@@ -404,7 +409,8 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
       if (kStats) tc_fence_before();   // orders the TMEM rescale before the next MMA
       mbar_arrive(op_full + st);
     }
-    // epilogue: accumulator row f = TMEM lane; columns [0, D) = Bm, [D, 2D) = Cm
+    // epilogue (warps 0-3): accumulator row f = TMEM lane; columns [0, D) = Bm, [D, 2D) = Cm
+    if (warp >= 4) ok = false;
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, status));
     if (ok) {
       tc_fence_after();
@@ -464,7 +470,7 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem, Cfg::kTmemCols);
+  if (warp == kChunkMmaWarp) tmem_dealloc(tmem, Cfg::kTmemCols);
 }
 
 // --------------------------------------------------------------- readout --
