@@ -83,10 +83,46 @@ def io_bytes(w: Workload) -> int:
     return 7 * w.B * w.H * w.T * w.d * esz
 
 
+def awm_plan(w: Workload, sms: int = 148) -> tuple:
+    """(fused, parts) as the library chooses them for a forward: `parts` CTAs
+    per chunk of the tensor-core chunk kernel (several when the chunks are
+    too few to fill two CTAs per SM), and whether the chunk kernel computes
+    each chunk's K_m statistics itself (d = 128 with one CTA per chunk)
+    instead of a separate statistics pass."""
+    if not (w.dtype == "bf16" and w.c % 128 == 0):
+        return False, 1
+    ctas, slots, n = w.B * w.H * w.S, 2 * sms, w.c // 64
+
+    def cost(P):   # waves x (tiles per CTA + 2), times P
+        return -(-ctas * P // slots) * (n + 2 * P)
+
+    best = 1
+    for P in range(2, min(n // 4, 16) + 1):
+        if cost(P) * best < cost(best) * P:
+            best = P
+    parts = best if best > 1 and 4 * cost(best) <= 3 * cost(1) * best else 1
+    return (w.d == 128 and parts == 1), parts
+
+
+def _sms() -> int:
+    try:
+        return torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    except Exception:
+        return 148
+
+
 def fused_stats(w: Workload) -> bool:
-    """The tensor-core forward at d = 128 computes each chunk's K_m
-    statistics inside the chunk kernel (no separate pass over K_m)."""
-    return w.dtype == "bf16" and w.d == 128 and w.c % 128 == 0
+    """The chunk kernel computes each chunk's K_m statistics itself (no
+    separate pass over K_m)."""
+    return awm_plan(w, _sms())[0]
+
+
+def forward_launches(w: Workload) -> int:
+    """Kernels of one forward: [statistics partial + combine] or nothing,
+    chunk products, [Cm image when several CTAs share a chunk at d = 128],
+    prefix, carry, readout, SCA."""
+    fused, parts = awm_plan(w, _sms())
+    return (0 if fused else 2) + 1 + (1 if parts > 1 and w.d == 128 else 0) + 4
 
 
 def stage_bytes(w: Workload) -> dict:
@@ -490,9 +526,7 @@ def run_gecko(args, w: Workload, ws: int, rank: int, local: int) -> dict:
         "roofline": roofline,
         "other_bounds": secondary_rooflines(w, agg["ms_per_step"], sca_ms, ck.get("sm_mhz"), pk["hbm_gbs"]),
         "clocks": ck,
-        # chunk (with statistics), prefix, carry, readout, sca; or lse partial,
-        # lse combine, prefix, chunk, carry, readout, sca
-        "gpu_launches": (5 if fused_stats(w) else 7) * args.steps,
+        "gpu_launches": forward_launches(w) * args.steps,
     }
     if note:
         out["note"] = note

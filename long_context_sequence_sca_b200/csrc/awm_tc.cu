@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
                                                            const __grid_constant__ CUtensorMap map_km,
                                                            float* __restrict__ lse, float* __restrict__ Bm,
                                                            float* __restrict__ Cm, uint16_t* __restrict__ Cimg,
-                                                           int T, int c, int koff, int* status) {
+                                                           int T, int c, int koff, int parts, int* status) {
   using Cfg = ChunkCfg<D, Mode>;
   // kChunkFwdStats: the forward products with the chunk's statistics
   // computed here (d = 128): it writes lse instead of reading it
@@ -123,15 +123,19 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
 
-  const int s = blockIdx.x, S = gridDim.x;
+  // `parts` CTAs share a chunk (forward mode only): CTA part p takes tiles
+  // [p n / parts, (p + 1) n / parts) and adds its products into Bm, Cm
+  // (zeroed by the host) with vector reductions
+  const int s = blockIdx.x / parts, part = blockIdx.x % parts, S = gridDim.x / parts;
   const int64_t bh = blockIdx.y;
   // the readouts of chunks 1 and 2 read a zero state: their E is never used
   if (Mode == kChunkE && s < 2) return;
   const int warp = warp_id_uniform(), lane = threadIdx.x % 32;
-  const int n_tiles = c / kKT;
-  const int64_t row0 = bh * (int64_t)T + (int64_t)s * c;
+  const int t0 = part * (c / kKT) / parts;
+  const int n_tiles = (part + 1) * (c / kKT) / parts - t0;
+  const int64_t row0 = bh * (int64_t)T + (int64_t)s * c + (int64_t)t0 * kKT;
   // v carries koff extra leading rows per (b, h) when a sequence is continued
-  const int64_t vrow0 = bh * (int64_t)(T + koff) + koff + (int64_t)s * c;
+  const int64_t vrow0 = bh * (int64_t)(T + koff) + koff + (int64_t)s * c + (int64_t)t0 * kKT;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NS; ++i) {
@@ -448,11 +452,18 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
         }
         if (valid) {
           float* dst = (cb * 32 < D) ? (Bm + o + cb * 32) : (Cm + o + cb * 32 - D);
+          if (Mode == kChunkFwd && parts > 1) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            reinterpret_cast<float4*>(dst)[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                                            __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-          if (kFwd && D == 128 && Cimg && cb * 32 >= D) {
+            for (int i = 0; i < 8; ++i)
+              red_add_v4(dst + 4 * i, __uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                         __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              reinterpret_cast<float4*>(dst)[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                                              __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+          }
+          if (kFwd && D == 128 && Cimg && parts == 1 && cb * 32 >= D) {
             // Cm row f as the tensor-core carry's bf16 A operand (K-major)
             uint8_t* img = reinterpret_cast<uint8_t*>(Cimg + (bh * S + s) * (int64_t)D * D);
 #pragma unroll
@@ -471,6 +482,24 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
   __syncthreads();
   tc_fence_after();
   if (warp == kChunkMmaWarp) tmem_dealloc(tmem, Cfg::kTmemCols);
+}
+
+// Cm_s rounded to bf16 in the carry's K-major 128-byte-swizzled operand
+// layout (the image the forward chunk kernel writes itself when one CTA owns
+// the chunk), from the fp32 Cm that several CTAs accumulated.  grid B*H*S,
+// one thread per row.
+__global__ void __launch_bounds__(128) awm_cimg_kernel(const float* __restrict__ Cm, uint16_t* __restrict__ Cimg) {
+  const int64_t m = blockIdx.x;
+  const int f = threadIdx.x;
+  const float* row = Cm + m * 128 * 128 + (int64_t)f * 128;
+  uint8_t* img = reinterpret_cast<uint8_t*>(Cimg + m * 128 * 128);
+#pragma unroll 4
+  for (int cb = 0; cb < 128; cb += 8) {
+    const float4 a = *reinterpret_cast<const float4*>(row + cb);
+    const float4 b = *reinterpret_cast<const float4*>(row + cb + 4);
+    *reinterpret_cast<uint4*>(img + sw128_off(f, cb, 128)) =
+        make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+  }
 }
 
 // --------------------------------------------------------------- readout --
@@ -1023,7 +1052,7 @@ EncodeTiledFn encode_fn() {
 
 template <int D, int Mode>
 cudaError_t chunk_impl(const Problem& p, const void* vsrc, const void* ksrc, float* lse, float* out0,
-                       float* out1, cudaStream_t st, uint16_t* cimg = nullptr) {
+                       float* out1, cudaStream_t st, uint16_t* cimg = nullptr, int parts = 1) {
   using Cfg = ChunkCfg<D, Mode>;
   EncodeTiledFn fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
@@ -1044,8 +1073,8 @@ cudaError_t chunk_impl(const Problem& p, const void* vsrc, const void* ksrc, flo
   cudaError_t e = cudaFuncSetAttribute(awm_chunk_tc_kernel<D, Mode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Cfg::kAlloc);
   if (e != cudaSuccess) return e;
-  awm_chunk_tc_kernel<D, Mode><<<dim3(p.S, p.B * p.H), kChunkThreads, Cfg::kAlloc, st>>>(
-      mv, mkm, lse, out0, out1, cimg, (int)p.T, (int)p.c, (int)koff, p.status);
+  awm_chunk_tc_kernel<D, Mode><<<dim3(p.S * parts, p.B * p.H), kChunkThreads, Cfg::kAlloc, st>>>(
+      mv, mkm, lse, out0, out1, cimg, (int)p.T, (int)p.c, (int)koff, parts, p.status);
   return cudaGetLastError();
 }
 
@@ -1105,9 +1134,20 @@ cudaError_t launch_awm_carry_tc(const Problem& p, const Workspace& w, cudaStream
   return carry_tc_impl(p, w, st, images);
 }
 
-cudaError_t launch_awm_chunk_tc(const Problem& p, const Workspace& w, cudaStream_t st) {
-  return p.d == 64 ? chunk_impl<64, kChunkFwd>(p, p.v, p.km, w.lse, w.Bm, w.Cm, st)
-                   : chunk_impl<128, kChunkFwd>(p, p.v, p.km, w.lse, w.Bm, w.Cm, st, w.Cimg);
+cudaError_t launch_awm_chunk_tc(const Problem& p, const Workspace& w, cudaStream_t st, int parts) {
+  if (parts < 1 || parts > (int)(p.c / 64)) return cudaErrorInvalidValue;
+  if (parts > 1) {
+    // the CTAs of a chunk add into zeroed products
+    const size_t bytes = sizeof(float) * p.B * p.H * p.S * p.d * p.d;
+    cudaError_t e;
+    if ((e = cudaMemsetAsync(w.Bm, 0, bytes, st)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(w.Cm, 0, bytes, st)) != cudaSuccess) return e;
+  }
+  cudaError_t e = p.d == 64 ? chunk_impl<64, kChunkFwd>(p, p.v, p.km, w.lse, w.Bm, w.Cm, st, nullptr, parts)
+                            : chunk_impl<128, kChunkFwd>(p, p.v, p.km, w.lse, w.Bm, w.Cm, st, w.Cimg, parts);
+  if (e != cudaSuccess || parts == 1 || p.d != 128) return e;
+  awm_cimg_kernel<<<(unsigned)(p.B * p.H * p.S), 128, 0, st>>>(w.Cm, w.Cimg);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_awm_chunk_tc_stats(const Problem& p, const Workspace& w, cudaStream_t st) {

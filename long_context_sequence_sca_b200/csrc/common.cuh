@@ -219,6 +219,12 @@ __device__ __forceinline__ bool bar_and(int id, int n, bool v) {
   return r != 0;
 }
 
+// *p += (a, b, c, d) as one vector reduction in L2 (16-byte aligned p).
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
 // ------------------------------------------------------------------- TMA --
 
 // 2D tiled bulk-tensor load (no multicast) into shared memory, completing

@@ -262,24 +262,61 @@ int ensure_buffer(void** buf, size_t* have, size_t need, cudaStream_t st, const 
   return GECKO_OK;
 }
 
-// The forward's AWM statistics at d = 128 on the tensor cores come from the
-// chunk kernel itself (each chunk's per-feature log-sum-exp is read off its
-// Cm block), which saves a second pass over K_m; the prefix over chunks then
-// runs after it.  Elsewhere a statistics pass precedes the chunk products.
-// GECKO_FUSED_STATS=0 at build time keeps the separate pass everywhere.
+// How a forward computes the AWM statistics and chunk products.
+//   parts  CTAs per chunk.  The tensor-core chunk kernel runs two CTAs per SM
+//          and one CTA's time is that of a whole chunk, so when the chunks
+//          are too few to fill the GPU (small batches, context-parallel
+//          segments of a few chunks) several CTAs share each chunk and add
+//          their products together.  The count minimises
+//          waves x (tiles per CTA + 2); it changes only if that saves a
+//          quarter of the time.
+//   fused  at d = 128 with one CTA per chunk, the chunk kernel computes each
+//          chunk's log-sum-exp itself (read off its Cm block), which saves a
+//          second pass over K_m; the prefix over chunks then runs after it.
+//          Otherwise a statistics pass precedes the chunk products (several
+//          CTAs per chunk need the chunk's lse before they start).
+//          GECKO_FUSED_STATS=0 at build time keeps the separate pass.
 #ifndef GECKO_FUSED_STATS
 #define GECKO_FUSED_STATS 1
 #endif
-bool fused_stats(const Problem& p, bool use_tc) { return GECKO_FUSED_STATS && use_tc && p.d == 128; }
+struct AwmPlan {
+  bool fused;
+  int parts;
+};
+
+AwmPlan awm_plan(const Problem& p, bool use_tc) {
+  AwmPlan a{false, 1};
+  if (use_tc) {
+    const int64_t ctas = p.B * p.H * p.S, slots = 2 * (int64_t)sm_count(), n = p.c / 64;
+    auto cost = [&](int64_t P) { return (ctas * P + slots - 1) / slots * (n + 2 * P); };   // x P
+    int64_t best = 1;
+    for (int64_t P = 2; P <= n / 4 && P <= 16; ++P)
+      if (cost(P) * best < cost(best) * P) best = P;
+    // cost(P) / P against cost(1): switch only for a saving of a quarter
+    if (best > 1 && 4 * cost(best) <= 3 * cost(1) * best) a.parts = (int)best;
+    // GECKO_CHUNK_PARTS=k forces k CTAs per chunk (tests cover both forms)
+    if (const char* f = getenv("GECKO_CHUNK_PARTS")) {
+      const long k = strtol(f, nullptr, 10);
+      if (k >= 1 && k <= n) a.parts = (int)k;
+    }
+    a.fused = GECKO_FUSED_STATS && p.d == 128 && a.parts == 1;
+  }
+  return a;
+}
+
+// The statistics pass, when the plan has one.
+int awm_stats_pass(const Problem& p, const Workspace& w, cudaStream_t st, const AwmPlan& a) {
+  return a.fused ? GECKO_OK : check_cuda(launch_awm_stats(p, w, st), "awm stats");
+}
 
 // The chunk products (and, when fused, the statistics and the prefix).
-int awm_chunks(const Problem& p, const Workspace& w, cudaStream_t st, bool use_tc, bool fused) {
+int awm_chunks(const Problem& p, const Workspace& w, cudaStream_t st, bool use_tc, const AwmPlan& a) {
   int rc;
-  if (fused) {
+  if (a.fused) {
     if ((rc = check_cuda(launch_awm_chunk_tc_stats(p, w, st), "awm chunk"))) return rc;
     return check_cuda(launch_awm_prefix(p, w, st), "awm prefix");
   }
-  return check_cuda(use_tc ? launch_awm_chunk_tc(p, w, st) : launch_awm_chunk_simt(p, w, st), "awm chunk");
+  return check_cuda(use_tc ? launch_awm_chunk_tc(p, w, st, a.parts) : launch_awm_chunk_simt(p, w, st), "awm chunk");
 }
 
 // The allocating forward, fresh (state_in == nullptr) or continuing a
@@ -329,10 +366,10 @@ int run_forward(const void* q, const void* k, const void* v, const void* qm, con
   cudaGetLastError();  // clear stale errors from the caller
   StageEvents ev(st);
   ev.mark(0);
-  const bool fused = fused_stats(p, use_tc);
-  if (!fused && (rc = check_cuda(launch_awm_stats(p, w, st), "awm stats"))) return rc;
+  const AwmPlan plan = awm_plan(p, use_tc);
+  if ((rc = awm_stats_pass(p, w, st, plan))) return rc;
   ev.mark(1);
-  if ((rc = awm_chunks(p, w, st, use_tc, fused))) return rc;
+  if ((rc = awm_chunks(p, w, st, use_tc, plan))) return rc;
   ev.mark(2);
   if ((rc = check_cuda(use_tc && d == 128 ? launch_awm_carry_tc(p, w, st, true) : launch_awm_carry(p, w, st, use_tc),
                        "awm carry")))
@@ -509,9 +546,14 @@ extern "C" int gecko_awm_segment_maps(const void* km, const void* v, const float
                                          sizeof(float) * d, BH, cudaMemcpyDeviceToDevice, st),
                        "seed log z")))
     return rc;
-  if ((rc = check_cuda(launch_awm_stats(p, w, st), "awm stats"))) return rc;
-  if ((rc = check_cuda(use_tc ? launch_awm_chunk_tc(p, w, st) : launch_awm_chunk_simt(p, w, st), "awm chunk")))
-    return rc;
+  const AwmPlan plan = awm_plan(p, use_tc);
+  if ((rc = awm_stats_pass(p, w, st, plan))) return rc;
+  if ((rc = awm_chunks(p, w, st, use_tc, plan))) return rc;
+  // the tensor-core carry at d = 128 (its C operand image comes from the chunk products)
+  auto carry = [&]() {
+    return check_cuda(use_tc && d == 128 ? launch_awm_carry_tc(p, w, st, false) : launch_awm_carry(p, w, st),
+                      "awm carry");
+  };
   // maps_out[bh] = (A, b, A', b'): the carry from M'_in = 0 gives b (after the
   // last chunk) and b' (before it); with the chunk terms zeroed and M'_in = I
   // it gives A and A'.
@@ -525,11 +567,11 @@ extern "C" int gecko_awm_segment_maps(const void* km, const void* v, const float
                                         m4, BH, cudaMemcpyDeviceToDevice, st),
                       "copy map");
   };
-  if ((rc = check_cuda(launch_awm_carry(p, w, st), "awm carry"))) return rc;
+  if ((rc = carry())) return rc;
   if ((rc = take(1, 3))) return rc;
   if ((rc = check_cuda(cudaMemsetAsync(w.Bm, 0, sizeof(float) * BH * S * mat, st), "clear chunk terms"))) return rc;
   if ((rc = check_cuda(launch_set_identity(state + mat, sd, (int)d, BH, st), "identity"))) return rc;
-  if ((rc = check_cuda(launch_awm_carry(p, w, st), "awm carry"))) return rc;
+  if ((rc = carry())) return rc;
   return take(0, 2);
 }
 
@@ -700,9 +742,9 @@ extern "C" int gecko_sca_awm_forward_noalloc(const void* q, const void* k, const
   Problem p{q, k, v, qm, km, out_sca, out_mem, B, H, T, c, d, (int)S, dtype, ds->status};
   const bool use_tc = !env_is("GECKO_KERNELS", "simt") && tc_supported(p);
   cudaGetLastError();
-  const bool fused = fused_stats(p, use_tc);
-  if (!fused && (rc = check_cuda(launch_awm_stats(p, w, st), "awm stats"))) return rc;
-  if ((rc = awm_chunks(p, w, st, use_tc, fused))) return rc;
+  const AwmPlan plan = awm_plan(p, use_tc);
+  if ((rc = awm_stats_pass(p, w, st, plan))) return rc;
+  if ((rc = awm_chunks(p, w, st, use_tc, plan))) return rc;
   if ((rc = check_cuda(use_tc && d == 128 ? launch_awm_carry_tc(p, w, st, true) : launch_awm_carry(p, w, st, use_tc),
                        "awm carry")))
     return rc;

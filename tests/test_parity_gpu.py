@@ -196,17 +196,23 @@ def test_repeat_calls_are_deterministic(L):
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
 
-@pytest.mark.parametrize("kernels", [None, "simt"])
-def test_awm_keys_growing_within_a_chunk(L, kernels, monkeypatch):
+@pytest.mark.parametrize("kernels,parts", [(None, None), (None, "1"), ("simt", None)])
+def test_awm_keys_growing_within_a_chunk(L, kernels, parts, monkeypatch):
     """K_m features whose values climb through each chunk (by up to 30 over
     the chunk, and one late spike of +40) and others that fall: the
     chunk-local exponentials of a feature cannot share one reference taken
     early in the chunk, so a kernel that tracks the per-feature maximum as
     it streams the chunk must raise it and rescale what it has accumulated.
     The chunk's log-sum-exp, the state and the readout still match the fp64
-    oracle (step 4 of the method: Phi = exp(Km - log z), any real Km)."""
+    oracle (step 4 of the method: Phi = exp(Km - log z), any real Km).
+    parts="1" keeps one CTA per chunk, the form whose chunk kernel computes
+    the chunk statistics itself (raising its reference); by default this
+    small problem shares each chunk among several CTAs after a separate
+    statistics pass."""
     if kernels:
         monkeypatch.setenv("GECKO_KERNELS", kernels)
+    if parts:
+        monkeypatch.setenv("GECKO_CHUNK_PARTS", parts)
     w = Workload("bf16_growing_keys", 19, "bf16", 1, 2, 1536, 128, 512)
     x = make_inputs(w, device="cuda")
     c, d = w.c, w.d
@@ -223,3 +229,14 @@ def test_awm_keys_growing_within_a_chunk(L, kernels, monkeypatch):
     _check(_np(M), r_M, w.dtype, "M state")
     _check(_np(lz), r_lz, w.dtype, "log z")
     _check(_np(o_sca), r_sca, w.dtype, "out_sca")
+
+
+@pytest.mark.parametrize("name,parts", [("bf16_d128_c512", "1"), ("bf16_d128_c512", "3"), ("bf16_d128_c512", "8"),
+                                        ("bf16_d64_c128", "2"), ("bf16_c384", "1"), ("bf16_c384", "6")])
+def test_parity_chunk_parts(L, name, parts, monkeypatch):
+    """The chunk products with k CTAs per chunk (each adding its share of
+    the tiles into the products, ragged shares included) and with one CTA
+    per chunk (at d = 128 with the statistics computed in the chunk kernel)
+    against the oracle."""
+    monkeypatch.setenv("GECKO_CHUNK_PARTS", parts)
+    _full_parity(L, SMALL[name])
