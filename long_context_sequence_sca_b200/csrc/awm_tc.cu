@@ -508,16 +508,20 @@ template <int D>
 struct ReadoutCfg {
   static constexpr int kTile = 128 * D * 2;      // a 128-row tile, bf16, D / 64 swizzled boxes of 16 KB
   static constexpr int kBox = 128 * 128;         // one [128 rows x 64] box
-  static constexpr int kStages = 4;              // Q_m tile ring, reused to stage the output tile
+  // Q_m tile ring; each stage returns to the producer once the tile's MMA
+  // has read it
+  static constexpr int kStages = D == 128 ? 3 : 4;
   static constexpr int kImg = D * D * 2;         // one M' operand image
   static constexpr int kImgOff = kStages * kTile;
-  static constexpr int kInvOff = kImgOff + 2 * kImg;      // [kStages][128] 1 / row sum of psi numerators
-  static constexpr int kBarOff = kInvOff + kStages * 128 * 4;
-  // q_full, op_full, st_empty, out_ready [kStages]; img_full, img_empty, acc_full, acc_empty [2]; drain
-  static constexpr int kNumBars = 4 * kStages + 8 + 1;
+  static constexpr int kOutOff = kImgOff + 2 * kImg;      // two output staging tiles
+  static constexpr int kBarOff = kOutOff + 2 * kTile;
+  // q_full, op_full, st_empty [kStages]; img_full, img_empty, acc_full,
+  // acc_empty, out_ready, out_free [2]; drain
+  static constexpr int kNumBars = 3 * kStages + 12 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;
+  static_assert(kAlloc <= 232448, "shared memory above the per-block limit");
   static constexpr uint32_t kTmemCols = 2 * D;   // two accumulators
   // psi warps (4: one thread per row; 8: two per row, measured 0.129 against
   // 0.135 ms at the bench workload); then 4 epilogue warps, the TMA warp
@@ -537,12 +541,12 @@ struct ReadoutCfg {
 // and 2 of a fresh sequence only writes zeros: weight 1; every other tile
 // reads Q_m and writes out_mem: weight 2).  448 threads:
 //   warps 0-7  psi: two threads per row turn it (Q_m tile by TMA, K-major A
-//              operand layout) into the numerators exp(q - max) in place,
-//              bf16, and keep 1 / sum for the epilogue;
-//   warps 8-11 epilogue: accumulator rows from TMEM scaled by 1 / sum,
-//              bf16, written over the tile's stage and stored by one TMA
-//              store; zero tiles are written directly;
-//   warp 12    TMA producer: Q_m tiles into a 4-stage ring, and the operand
+//              operand layout) into psi = exp(q - max) / sum in place, bf16;
+//   warps 8-11 epilogue: accumulator rows from TMEM to bf16 in one of two
+//              output staging tiles, stored by one TMA store; zero tiles
+//              are written directly;
+//   warp 12    TMA producer: Q_m tiles into a 3-stage ring (4 at d = 64;
+//              a stage is free again once its tile's MMA has read it), and the operand
 //              image of M'_{s-1} (bf16, written by the carry in the MN-major
 //              B layout) by one bulk copy whenever the chunk changes
 //              (two image buffers);
@@ -556,17 +560,17 @@ awm_readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
   constexpr int NS = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* rinv = reinterpret_cast<float*>(smem + Cfg::kInvOff);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
   uint64_t* q_full = bars;                // TMA -> psi warps
-  uint64_t* op_full = q_full + NS;        // psi warps (128) -> MMA
-  uint64_t* st_empty = op_full + NS;      // output store finished reading the stage -> TMA
-  uint64_t* out_ready = st_empty + NS;    // epilogue (128) wrote the output tile -> storing thread
-  uint64_t* img_full = out_ready + NS;    // [2] image copy -> MMA
+  uint64_t* op_full = q_full + NS;        // psi warps -> MMA
+  uint64_t* st_empty = op_full + NS;      // the tile's MMA read the stage -> TMA
+  uint64_t* img_full = st_empty + NS;     // [2] image copy -> MMA
   uint64_t* img_empty = img_full + 2;     // [2] last MMA of the image's chunk -> TMA
   uint64_t* acc_full = img_empty + 2;     // [2] MMA -> epilogue
   uint64_t* acc_empty = acc_full + 2;     // [2] epilogue (128) -> MMA
-  uint64_t* drain = acc_empty + 2;
+  uint64_t* out_ready = acc_empty + 2;    // [2] epilogue (128) wrote the output tile -> storing thread
+  uint64_t* out_free = out_ready + 2;     // [2] the store of that tile finished reading it -> epilogue
+  uint64_t* drain = out_free + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
 
@@ -606,13 +610,14 @@ awm_readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
       mbar_init(q_full + i, 1);
       mbar_init(op_full + i, Cfg::kPsiWarps * 32);
       mbar_init(st_empty + i, 1);
-      mbar_init(out_ready + i, 128);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(img_full + i, 1);
       mbar_init(img_empty + i, 1);
       mbar_init(acc_full + i, 1);
       mbar_init(acc_empty + i, 128);
+      mbar_init(out_ready + i, 128);
+      mbar_init(out_free + i, 1);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -689,6 +694,7 @@ awm_readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
           umma_ss(tmem + a * D, sdesc_at(ad, koff), sdesc_at(bd, kk * 16 * 128), idesc, kk > 0 ? 1u : 0u);
         }
         umma_commit(acc_full + a);
+        umma_commit(st_empty + st);   // the psi operand has been read
         // the image is released after the last tile of its chunk in this
         // range (tiles of one chunk are consecutive; the next chunk's tiles,
         // if any, are never zero tiles of the same image)
@@ -726,32 +732,43 @@ awm_readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
       }
       if (TPR == 2) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
       const float mx2 = mx * kLog2e;
-      // fp32 exponentials on the SFU, arguments by packed FMA
+      // fp32 exponentials on the SFU, arguments by packed FMA; psi is
+      // normalised before it is rounded to bf16, so the MMA gives the
+      // readout rows directly
       const uint64_t l2e2 = pack2(kLog2e, kLog2e), nmx2 = pack2(-mx2, -mx2);
       uint64_t sum2 = pack2(0.f, 0.f);
+      float e[CPT];
 #pragma unroll
       for (int i = 0; i < CPT / 8; ++i) {
-        uint4* qa = reinterpret_cast<uint4*>(tile + sw128_off(r, c0 + 8 * i, 128));
-        const uint4 q = *qa;
+        const uint4 q = *reinterpret_cast<const uint4*>(tile + sw128_off(r, c0 + 8 * i, 128));
         const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&q);
-        uint4 pv;
-        uint32_t* pp = reinterpret_cast<uint32_t*>(&pv);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const float2 f2 = __bfloat1622float2(p2[j]);
           float u0, u1;
           unpack2(ffma2(pack2(f2.x, f2.y), l2e2, nmx2), u0, u1);
-          const float e0 = ex2(u0), e1 = ex2(u1);
-          sum2 = fadd2(sum2, pack2(e0, e1));
-          pp[j] = pack_bf16x2(e0, e1);
+          e[8 * i + 2 * j] = ex2(u0);
+          e[8 * i + 2 * j + 1] = ex2(u1);
+          sum2 = fadd2(sum2, pack2(e[8 * i + 2 * j], e[8 * i + 2 * j + 1]));
         }
-        *qa = pv;
       }
       float sum, s1;
       unpack2(sum2, sum, s1);
       sum += s1;
       if (TPR == 2) sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-      if (c0 == 0) rinv[st * 128 + r] = 1.f / sum;
+      const uint64_t inv2 = pack2(1.f / sum, 1.f / sum);
+#pragma unroll
+      for (int i = 0; i < CPT / 8; ++i) {
+        uint4 pv;
+        uint32_t* pp = reinterpret_cast<uint32_t*>(&pv);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float a0, a1;
+          unpack2(fmul2(pack2(e[8 * i + 2 * j], e[8 * i + 2 * j + 1]), inv2), a0, a1);
+          pp[j] = pack_bf16x2(a0, a1);
+        }
+        *reinterpret_cast<uint4*>(tile + sw128_off(r, c0 + 8 * i, 128)) = pv;
+      }
       fence_proxy_async_smem();   // the numerators are read by the tensor core (async proxy)
       mbar_arrive(op_full + st);
       ++n;
@@ -773,12 +790,14 @@ awm_readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
         for (int i = 0; i < D / 8; ++i) dst[i] = z;
         continue;
       }
-      const int st = n % NS, a = n & 1;
+      const int a = n & 1;   // accumulator and output staging tile
       ok = __all_sync(0xffffffffu, mbar_wait(acc_full + a, (n >> 1) & 1, abort_flag, status));
       if (!ok) break;
+      // the store of tile n - 2 has finished reading this staging tile
+      if (n >= 2) ok = __all_sync(0xffffffffu, mbar_wait(out_free + a, ((n >> 1) - 1) & 1, abort_flag, status));
+      if (!ok) break;
       tc_fence_after();
-      const float inv = rinv[st * 128 + r];
-      uint8_t* tile = smem + st * Cfg::kTile;   // the psi operand is no longer read: stage the output here
+      uint8_t* tile = smem + Cfg::kOutOff + a * Cfg::kTile;
 #pragma unroll 1
       for (int cb = 0; cb < D / 32; ++cb) {
         uint32_t v[32];
@@ -787,31 +806,28 @@ awm_readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
           uint4 w;
-          w.x = pack_bf16x2(__uint_as_float(v[8 * x + 0]) * inv, __uint_as_float(v[8 * x + 1]) * inv);
-          w.y = pack_bf16x2(__uint_as_float(v[8 * x + 2]) * inv, __uint_as_float(v[8 * x + 3]) * inv);
-          w.z = pack_bf16x2(__uint_as_float(v[8 * x + 4]) * inv, __uint_as_float(v[8 * x + 5]) * inv);
-          w.w = pack_bf16x2(__uint_as_float(v[8 * x + 6]) * inv, __uint_as_float(v[8 * x + 7]) * inv);
+          w.x = pack_bf16x2(__uint_as_float(v[8 * x + 0]), __uint_as_float(v[8 * x + 1]));
+          w.y = pack_bf16x2(__uint_as_float(v[8 * x + 2]), __uint_as_float(v[8 * x + 3]));
+          w.z = pack_bf16x2(__uint_as_float(v[8 * x + 4]), __uint_as_float(v[8 * x + 5]));
+          w.w = pack_bf16x2(__uint_as_float(v[8 * x + 6]), __uint_as_float(v[8 * x + 7]));
           *reinterpret_cast<uint4*>(tile + sw128_off(r, cb * 32 + 8 * x, 128)) = w;
         }
       }
       tc_fence_before();
       mbar_arrive(acc_empty + a);
       fence_proxy_async_smem();   // the tile is read by the TMA store (async proxy)
-      mbar_arrive(out_ready + st);
+      mbar_arrive(out_ready + a);
       if (leader) {
-        if (!(ok = mbar_wait(out_ready + st, (n / NS) & 1, abort_flag, status))) break;
+        if (!(ok = mbar_wait(out_ready + a, (n >> 1) & 1, abort_flag, status))) break;
         for (int b = 0; b < D / 64; ++b) tma_store_2d(&map_o, tile + b * Cfg::kBox, b * 64, (int)row_of(t));
         bulk_commit();
-        // the previous tile's store has finished reading its stage
+        // the previous tile's store has finished reading its staging tile
         bulk_wait_read<1>();
-        if (n > 0) mbar_arrive(st_empty + (n - 1) % NS);
+        if (n > 0) mbar_arrive(out_free + (a ^ 1));
       }
       ++n;
     }
-    if (leader) {
-      bulk_wait_all();
-      if (n > 0) mbar_arrive(st_empty + (n - 1) % NS);
-    }
+    if (leader) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
