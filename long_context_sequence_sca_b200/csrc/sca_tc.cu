@@ -11,19 +11,20 @@
 //   warp 0      TMA producer: Q tiles once per work unit; K and V tiles of
 //               128 keys through rings of shared-memory stages, loads issued
 //               in the order of the iterations that free their slots.
-//   warp 1      TMEM allocator and MMA issuer (one thread): S_i = Q_i K_j^T
-//               (SS form) into TMEM, O_i += P_i V_j with P_i read from TMEM
-//               (TS form).
-//   warps 2-3   idle (they complete the first warpgroup, whose registers
+//   warps 1-2   MMA issuers, one thread each, one per query tile i (warp 1
+//               also allocates TMEM): S_i = Q_i K_j^T (SS form) into TMEM,
+//               O_i += P_i V_j with P_i read from TMEM (TS form).
+//   warp 3      idle (it completes the first warpgroup, whose registers
 //               setmaxnreg hands to the softmax warpgroups).
 //   warps 4-7   softmax for query tile 0, warps 8-11 for query tile 1; one
 //               thread per query row (TMEM lane quarter = warp % 4); online
 //               max/sum in registers; P written back to TMEM as bf16 over the
 //               S columns; epilogue O / l.
 // A work unit is two adjacent 128-row query tiles of one (b, h); CTAs claim
-// units from a global counter in the schedule's order (decode_unit).  The MMA
-// warp interleaves the two tiles (PV(0), QK(0), PV(1), QK(1)) so each
-// softmax warpgroup's exp work overlaps the other tile's MMAs.  Only the
+// units from a global counter in the schedule's order (decode_unit).  The
+// two issuers alternate by turns (PV(0), QK(0) then PV(1), QK(1) for each
+// key tile) so each softmax warpgroup's exp work overlaps the other tile's
+// MMAs.  Only the
 // diagonal key tile of each query tile is masked; key tiles entirely above
 // the diagonal or before the previous chunk are never loaded.
 //
@@ -72,6 +73,17 @@ constexpr int kSfuPairs = GECKO_SFU_PAIRS;
 #ifndef GECKO_SCA_ONEPASS
 #define GECKO_SCA_ONEPASS 0
 #endif
+// GECKO_SCA_ISSUERS=2 (default): warps 1 and 2 each issue one query tile's
+// MMAs and take strict turns (tile 0's step of iteration j, then tile 1's),
+// so the barrier waits, commits and loop work of one issuer overlap the
+// other's MMAs on the tensor core (SCA kernel 2.68 against 2.73 ms over
+// eight interleaved runs on the bench workload).  Each issuer releases K_j
+// and V_{j-1} with its own commit (a commit covers only the committing
+// thread's MMAs).  GECKO_SCA_ISSUERS=1 keeps one MMA thread for both tiles.
+#ifndef GECKO_SCA_ISSUERS
+#define GECKO_SCA_ISSUERS 2
+#endif
+constexpr int kIssuers = GECKO_SCA_ISSUERS;
 // Register budget of the kernel: the default lets the compiler fit 320
 // threads on one SM; GECKO_SCA_MAXNREG caps registers per thread instead.
 #ifdef GECKO_SCA_MAXNREG
@@ -120,9 +132,9 @@ struct ScaCfg {
   static constexpr int kVOff = kKOff + kKStages * kTileBytes;
   static constexpr int kBarOff = kVOff + kVStages * kTileBytes;
   // q_full, q_empty, k_full[KS], it_done[max(KS, VS)], v_full[VS], s_full[2],
-  // p_full[2], o_full[2], o_empty[2], drain, unit_ready[kUnitRing]
+  // p_full[2], o_full[2], o_empty[2], drain, unit_ready[kUnitRing], turn_done[2]
   static constexpr int kNumBars = 2 + kKStages + (kKStages > kVStages ? kKStages : kVStages) + kVStages + 8 + 1 +
-                                  kUnitRing;
+                                  kUnitRing + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   // tmem address, abort flag, then the unit ring (kUnitRing uint32)
   static constexpr int kBytes = kMiscOff + 8 + 4 * kUnitRing;
@@ -379,6 +391,7 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   uint64_t* o_empty = o_full + 2;
   uint64_t* drain = o_empty + 2;
   uint64_t* unit_ready = drain + 1;   // [kUnitRing]
+  uint64_t* turn_done = unit_ready + kUnitRing;   // [2] two issuers: issuer i finished its turn
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
   uint32_t* unit_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff + 8);   // [kUnitRing]
@@ -388,9 +401,9 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
+    mbar_init(q_empty, kIssuers);
     for (int s = 0; s < KS; ++s) mbar_init(k_full + s, 1);
-    for (int s = 0; s < IR; ++s) mbar_init(it_done + s, 1);
+    for (int s = 0; s < IR; ++s) mbar_init(it_done + s, kIssuers);
     for (int s = 0; s < VS; ++s) mbar_init(v_full + s, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + i, 1);
@@ -398,7 +411,9 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       mbar_init(o_full + i, 1);
       mbar_init(o_empty + i, 128);
     }
-    mbar_init(drain, 1);
+    mbar_init(drain, kIssuers);
+    mbar_init(turn_done + 0, 1);
+    mbar_init(turn_done + 1, 1);
     for (int r = 0; r < kUnitRing; ++r) mbar_init(unit_ready + r, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -486,6 +501,80 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           mbar_wait_drain(v_full + idx % VS, (idx / VS) & 1);
         if (qn > 0) mbar_wait_drain(q_full, (qn - 1) & 1);
       }
+    }
+    __syncwarp();
+  } else if (kIssuers == 2 && (warp == 1 || warp == 2)) {
+    // ------------------------------------------- two MMA issuers, one per tile --
+    if (lane == 0) {
+      const int i = warp - 1;   // the query tile this thread issues for
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, false, true);
+      const uint32_t qa = smem_u32(sQ) + i * Cfg::kTileBytes, ka = smem_u32(sK), va = smem_u32(sV);
+      const uint32_t colS = i == 0 ? Cfg::kColS0 : Cfg::kColS1;
+      const uint32_t colO = i == 0 ? Cfg::kColO0 : Cfg::kColO1;
+      uint32_t kv_it = 0, p_par = 0, o_par = 0, turn = 0;
+      bool ok = true;
+      for (int n = 0;; ++n) {
+        if (!(ok = mbar_wait(unit_ready + n % kUnitRing, (n / kUnitRing) & 1, abort_flag, status))) break;
+        const int u = (int)unit_slot[n % kUnitRing];
+        if (u >= n_units) break;
+        const Unit U = decode_unit(u, BH, T, c, koff);
+        if (!(ok = mbar_wait(q_full, n & 1, abort_flag, status))) break;
+        tc_fence_after();
+        const int jb = U.beg[0], je = U.nt == 2 ? U.end[1] : U.end[0];
+        const int bi = i < U.nt ? ubeg(U, i) : 0, ei = i < U.nt ? uend(U, i) : 0;
+        for (int j = jb; j <= je && ok; ++j) {
+          // turn (j, i): after the other issuer's turn (j, 0) or (j - 1, 1)
+          if (!(i == 0 && turn == 0)) {
+            const uint32_t q = i == 0 ? turn - 1 : turn;
+            if (!(ok = mbar_wait(turn_done + (1 - i), q & 1, abort_flag, status))) break;
+          }
+          if (j - 1 >= bi && j - 1 < ei) {
+            // O_i += P_i V_{j-1} (V_{j-1} was waited for with this tile's QK of iteration j - 1)
+            if (j - 1 == bi) {
+              if (!(ok = mbar_wait(o_empty + i, (o_par & 1) ^ 1, abort_flag, status))) break;
+            }
+            if (!(ok = mbar_wait(p_full + i, p_par & 1, abort_flag, status))) break;
+            p_par ^= 1u;
+            tc_fence_after();
+            const SDesc vd = sdesc_sw128_split(va + ((kv_it - 1) % VS) * Cfg::kTileBytes, Cfg::kBoxBytes, 1024);
+            umma_ts(tmem + colO, tmem + colS, sdesc_at(vd, 0), idesc_pv, j - 1 > bi ? 1u : 0u);
+#pragma unroll
+            for (int kk = 1; kk < kBN / 16; ++kk)
+              umma_ts(tmem + colO, tmem + colS + kk * 8, sdesc_at(vd, kk * 2048), idesc_pv, 1u);
+            if (j - 1 == ei - 1) {
+              umma_commit(o_full + i);
+              o_par ^= 1u;
+            }
+          }
+          if (j >= bi && j < ei) {
+            // S_i = Q_i K_j^T; V_j (read by the PVs of iteration j + 1) is waited for here too
+            if (!(ok = mbar_wait(k_full + kv_it % KS, (kv_it / KS) & 1, abort_flag, status))) break;
+            if (!(ok = mbar_wait(v_full + kv_it % VS, (kv_it / VS) & 1, abort_flag, status))) break;
+            tc_fence_after();
+            const SDesc qd = sdesc_sw128_split(qa, 16, 1024);
+            const SDesc kd = sdesc_sw128_split(ka + (kv_it % KS) * Cfg::kTileBytes, 16, 1024);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t kbyte = (kk / 4) * Cfg::kBoxBytes + (kk % 4) * 32;
+              umma_ss(tmem + colS, sdesc_at(qd, kbyte), sdesc_at(kd, kbyte), idesc_qk, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(s_full + i);
+          }
+          mbar_arrive(turn_done + i);
+          ++turn;
+          if (j < je) {
+            // this issuer is done with K_j and V_{j-1} once its MMAs so far complete
+            umma_commit(it_done + kv_it % IR);
+            if (j == je - 1) umma_commit(q_empty);
+            ++kv_it;
+          }
+        }
+        if (!ok) break;
+      }
+      // all issued MMAs complete before TMEM is released
+      umma_commit(drain);
+      mbar_wait_drain(drain, 0);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -600,7 +689,7 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
         // The QK of the iteration's last active tile is its last MMA, so its
         // completion (just observed) means K_j and V_{j-1} are no longer read:
         // one thread of that tile's warpgroup releases them to the producer.
-        if ((i == 1 || !(U.nt == 2 && j >= U.beg[1])) && warp % 4 == 2 && lane == 0)
+        if (kIssuers == 1 && (i == 1 || !(U.nt == 2 && j >= U.beg[1])) && warp % 4 == 2 && lane == 0)
           mbar_arrive(it_done + (unit_it0 + (uint32_t)(j - jb)) % IR);
         ++s_cnt;
         tc_fence_after();
