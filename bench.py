@@ -87,8 +87,8 @@ def awm_plan(w: Workload, sms: int = 148) -> tuple:
     """(fused, parts) as the library chooses them for a forward: `parts` CTAs
     per chunk of the tensor-core chunk kernel (several when the chunks are
     too few to fill two CTAs per SM), and whether the chunk kernel computes
-    each chunk's K_m statistics itself (d = 128 with one CTA per chunk)
-    instead of a separate statistics pass."""
+    each chunk's K_m statistics itself (one CTA per chunk) instead of a
+    separate statistics pass."""
     if not (w.dtype == "bf16" and w.c % 128 == 0):
         return False, 1
     ctas, slots, n = w.B * w.H * w.S, 2 * sms, w.c // 64
@@ -101,7 +101,7 @@ def awm_plan(w: Workload, sms: int = 148) -> tuple:
         if cost(P) * best < cost(best) * P:
             best = P
     parts = best if best > 1 and 4 * cost(best) <= 3 * cost(1) * best else 1
-    return (w.d == 128 and parts == 1), parts
+    return parts == 1, parts
 
 
 def _sms() -> int:

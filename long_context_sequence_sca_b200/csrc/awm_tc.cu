@@ -18,7 +18,7 @@
 // (two per token) compute Phi and Psi in fp32 and store them as bf16 next
 // to V in one 128-byte-swizzled, MN-major stage [V | Psi | Phi], so a single
 // tcgen05.mma with M = d, N = 2d accumulates [Phi^T V | Phi^T Psi] in TMEM.
-// In the forward at d = 128 the kernel also computes each chunk's
+// In the forward (one CTA per chunk) the kernel also computes each chunk's
 // per-feature log-sum-exp lse_s: it exponentiates against a running
 // per-feature reference (the column maximum of the tiles seen so far, raised
 // lazily with a rescale of the accumulated rows), reads the column sums of
@@ -53,7 +53,7 @@ namespace {
 //   kChunkE      E = psi(Q_m)^T dO_m for the backward (Q_m arrives in the
 //                K_m slot, dO_m in the V slot): stage [dO | psi_hi | psi_lo].
 //   kChunkFwdStats  kChunkFwd with the chunk's per-feature log-sum-exp
-//                computed in the same pass (d = 128): Phi^ = exp(Km - m_f)
+//                computed in the same pass: Phi^ = exp(Km - m_f)
 //                with a lazily raised per-feature reference m_f, the column
 //                sums read off the Cm block (rows of Psi sum to 1), and
 //                Bm, Cm normalised in the epilogue, which also writes lse.
@@ -89,7 +89,8 @@ struct ChunkCfg {
   // ([8][D] bf16, stored 16 bytes at a time)
   static constexpr int kPartOff = (kMiscOff + 16 + 15) / 16 * 16;
   static_assert(kPartOff % 16 == 0, "16-byte stores of the column maxima");
-  static constexpr int kBytes = kPartOff + (Mode == kChunkFwdStats ? 8 * D * 2 : 0);
+  // [kChunkCompute / (D / 8) row groups][D] bf16 = 2 KB
+  static constexpr int kBytes = kPartOff + (Mode == kChunkFwdStats ? 2048 : 0);
   static constexpr int kAlloc = kBytes + 1024;
   static constexpr uint32_t kTmemCols = Mode == kChunkE ? D : (D == 128 ? 256 : 128);
 };
@@ -109,7 +110,9 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
   // computed here (d = 128): it writes lse instead of reading it
   constexpr bool kStats = Mode == kChunkFwdStats;
   constexpr bool kFwd = Mode == kChunkFwd || kStats;
-  static_assert(!kStats || D == 128, "fused statistics need one thread per feature");
+  // fused statistics: the column maxima of a tile come from kRG groups of
+  // kKT / kRG rows, one thread per (row group, 8 features)
+  constexpr int kFG = D / 8, kRG = kChunkCompute / kFG;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int NS = Cfg::kStages, kKT = Cfg::kKT;
@@ -244,30 +247,33 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
       if (!ok) break;
       uint8_t* stg = smem + st * Cfg::kStage;
       if (kStats) {
-        // Column maxima of the K_m tile: thread (rg, g) takes rows
-        // 8 rg .. 8 rg + 7 of features 8 g .. 8 g + 7, then thread f
-        // combines the 8 row groups of its feature.
+        // Column maxima of the K_m tile: thread (rg, g) takes the kKT / kRG
+        // rows of group rg for features 8 g .. 8 g + 7, then the thread of
+        // feature f combines the kRG row groups.  The thread of feature f
+        // is the one whose TMEM lane holds accumulator row f: lane f for
+        // M = 128, lane 16 w + (f % 16) of warp w = f / 16 for M = 64.
         __nv_bfloat162* part = reinterpret_cast<__nv_bfloat162*>(smem + Cfg::kPartOff);
-        const bool feat = threadIdx.x < D;   // warps 0-3: one feature (TMEM lane) per thread
-        if (feat) {
-          const int g = threadIdx.x % 16, rg = threadIdx.x / 16;
-          uint4 mx = *reinterpret_cast<const uint4*>(stg + Cfg::kOperand + sw128_off(8 * rg, 8 * g, kKT));
+        {
+          constexpr int kRPG = kKT / kRG;
+          const int g = threadIdx.x % kFG, rg = threadIdx.x / kFG;
+          uint4 mx = *reinterpret_cast<const uint4*>(stg + Cfg::kOperand + sw128_off(kRPG * rg, 8 * g, kKT));
           __nv_bfloat162* m2 = reinterpret_cast<__nv_bfloat162*>(&mx);
 #pragma unroll
-          for (int rr = 1; rr < 8; ++rr) {
-            uint4 v = *reinterpret_cast<const uint4*>(stg + Cfg::kOperand + sw128_off(8 * rg + rr, 8 * g, kKT));
+          for (int rr = 1; rr < kRPG; ++rr) {
+            uint4 v = *reinterpret_cast<const uint4*>(stg + Cfg::kOperand + sw128_off(kRPG * rg + rr, 8 * g, kKT));
             const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
             for (int j = 0; j < 4; ++j) m2[j] = __hmax2(m2[j], v2[j]);
           }
           *reinterpret_cast<uint4*>(part + rg * (D / 2) + 4 * g) = mx;
         }
+        const bool feat = D == 128 ? threadIdx.x < D : lane < 16;
         named_bar_sync(1, kChunkCompute);
-        const int f = feat ? threadIdx.x : 0;
+        const int f = feat ? (D == 128 ? (int)threadIdx.x : warp * 16 + lane) : 0;
         const __nv_bfloat16* ph = reinterpret_cast<const __nv_bfloat16*>(part);
         float mt = __bfloat162float(ph[f]);
 #pragma unroll
-        for (int q = 1; q < 8; ++q) mt = fmaxf(mt, __bfloat162float(ph[q * D + f]));
+        for (int q = 1; q < kRG; ++q) mt = fmaxf(mt, __bfloat162float(ph[q * D + f]));
         const float mt2 = feat ? mt * kLog2e : 0.f;
         // The reference is raised lazily, only when the tile's maximum
         // exceeds it by more than 8 (every exponential stays <= 2^8), and
@@ -439,7 +445,7 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
           for (int x = 0; x < 32; ++x) sum += __uint_as_float(v[x]);
         }
         inv = 1.f / sum;
-        lse[(bh * S + s) * D + f] = (m_f + log2f(sum)) * kLn2;
+        if (valid) lse[(bh * S + s) * D + f] = (m_f + log2f(sum)) * kLn2;
       }
 #pragma unroll 1
       for (int cb = 0; cb < (Mode == kChunkE ? D : 2 * D) / 32; ++cb) {
@@ -1174,8 +1180,8 @@ cudaError_t launch_awm_chunk_tc(const Problem& p, const Workspace& w, cudaStream
 }
 
 cudaError_t launch_awm_chunk_tc_stats(const Problem& p, const Workspace& w, cudaStream_t st) {
-  if (p.d != 128) return cudaErrorInvalidValue;
-  return chunk_impl<128, kChunkFwdStats>(p, p.v, p.km, w.lse, w.Bm, w.Cm, st, w.Cimg);
+  return p.d == 64 ? chunk_impl<64, kChunkFwdStats>(p, p.v, p.km, w.lse, w.Bm, w.Cm, st)
+                   : chunk_impl<128, kChunkFwdStats>(p, p.v, p.km, w.lse, w.Bm, w.Cm, st, w.Cimg);
 }
 
 cudaError_t launch_awm_chunk_tc_split(const Problem& p, const Workspace& w, cudaStream_t st) {

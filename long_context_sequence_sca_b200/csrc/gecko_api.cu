@@ -270,8 +270,8 @@ int ensure_buffer(void** buf, size_t* have, size_t need, cudaStream_t st, const 
 //          their products together.  The count minimises
 //          waves x (tiles per CTA + 2); it changes only if that saves a
 //          quarter of the time.
-//   fused  at d = 128 with one CTA per chunk, the chunk kernel computes each
-//          chunk's log-sum-exp itself (read off its Cm block), which saves a
+//   fused  with one CTA per chunk, the chunk kernel computes each chunk's
+//          log-sum-exp itself (read off its Cm block), which saves a
 //          second pass over K_m; the prefix over chunks then runs after it.
 //          Otherwise a statistics pass precedes the chunk products (several
 //          CTAs per chunk need the chunk's lse before they start).
@@ -299,7 +299,7 @@ AwmPlan awm_plan(const Problem& p, bool use_tc) {
       const long k = strtol(f, nullptr, 10);
       if (k >= 1 && k <= n) a.parts = (int)k;
     }
-    a.fused = GECKO_FUSED_STATS && p.d == 128 && a.parts == 1;
+    a.fused = GECKO_FUSED_STATS && a.parts == 1;
   }
   return a;
 }

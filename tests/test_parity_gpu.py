@@ -196,8 +196,8 @@ def test_repeat_calls_are_deterministic(L):
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
 
-@pytest.mark.parametrize("kernels,parts", [(None, None), (None, "1"), ("simt", None)])
-def test_awm_keys_growing_within_a_chunk(L, kernels, parts, monkeypatch):
+@pytest.mark.parametrize("kernels,parts,d", [(None, None, 128), (None, "1", 128), ("simt", None, 128), (None, "1", 64)])
+def test_awm_keys_growing_within_a_chunk(L, kernels, parts, d, monkeypatch):
     """K_m features whose values climb through each chunk (by up to 30 over
     the chunk, and one late spike of +40) and others that fall: the
     chunk-local exponentials of a feature cannot share one reference taken
@@ -213,9 +213,9 @@ def test_awm_keys_growing_within_a_chunk(L, kernels, parts, monkeypatch):
         monkeypatch.setenv("GECKO_KERNELS", kernels)
     if parts:
         monkeypatch.setenv("GECKO_CHUNK_PARTS", parts)
-    w = Workload("bf16_growing_keys", 19, "bf16", 1, 2, 1536, 128, 512)
+    w = Workload(f"bf16_growing_keys_d{d}", 19, "bf16", 1, 2, 1536, d, 512)
     x = make_inputs(w, device="cuda")
-    c, d = w.c, w.d
+    c = w.c
     t = (torch.arange(w.T, device="cuda") % c).float() / c
     f = torch.arange(d, device="cuda")
     slope = torch.where(f % 4 == 0, 30.0 * (f.float() / d), torch.where(f % 4 == 1, -12.0, 0.0))
