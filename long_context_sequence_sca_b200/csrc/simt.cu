@@ -117,9 +117,18 @@ __global__ void __launch_bounds__(D) awm_prefix_kernel(const float* __restrict__
   const int f = threadIdx.x;
   const bool seeded = logz0 != nullptr;
   double L = seeded ? (double)logz0[bh * sd + f] : 0.0;
+  // the chunk log-sum-exps are read 8 chunks ahead of the sequential chain,
+  // so their load latency is paid once per 8 steps
+  float ahead[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) ahead[k] = k < S ? lse[(bh * S + k) * D + f] : 0.f;
   for (int s = 0; s < S; ++s) {
     const int64_t o = (bh * S + s) * D + f;
-    const double e = lse[o];
+    const double e = ahead[s % 8];
+    if (s % 8 == 7) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) ahead[k] = s + 1 + k < S ? lse[(bh * S + s + 1 + k) * D + f] : 0.f;
+    }
     double Ln;
     if (s == 0 && !seeded) {
       Ln = e;
