@@ -56,7 +56,13 @@ constexpr int kBN = 128;   // keys per tile
 #endif
 constexpr int kThreads = GECKO_SCA_WG3 ? 384 : 320;   // TMA, MMA (+TMEM allocation), [2 idle], 2 x 4 softmax
 constexpr int kSoftmaxWarp0 = GECKO_SCA_WG3 ? 4 : 2;  // first softmax warp
-constexpr int kRegsCtl = 88, kRegsSoftmax = 208;      // per-thread registers after setmaxnreg (GECKO_SCA_WG3)
+// Per-thread registers after setmaxnreg (GECKO_SCA_WG3).  The split must fit
+// the registers the block was launched with: 128 x kRegsCtl + 256 x
+// kRegsSoftmax <= 384 x 168 = 64512 (a larger sum would leave setmaxnreg.inc
+// waiting for registers forever).  96 / 200 measured 2.59-2.60 against
+// 2.63-2.67 ms for 88 / 208 (the two MMA issuers live in the first warpgroup).
+constexpr int kRegsCtl = 96, kRegsSoftmax = 200;
+static_assert(128 * kRegsCtl + 256 * kRegsSoftmax <= 384 * 168, "setmaxnreg split above the launch registers");
 // Of every 8 exponential pairs, GECKO_SFU_PAIRS are evaluated on the SFU
 // (ex2.approx) and the rest on the FMA pipe (exp2_poly2).  Measured on B200
 // with the bench workload the all-SFU setting is fastest (the polynomial
@@ -863,6 +869,18 @@ cudaError_t launch_sca_tc_impl(const Problem& p, cudaStream_t st) {
   if ((e = cudaFuncSetAttribute(sca_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kAlloc)) !=
       cudaSuccess)
     return e;
+#if GECKO_SCA_WG3
+  {
+    // the setmaxnreg split must fit the registers the kernel is launched with
+    static int regs = 0;
+    if (!regs) {
+      cudaFuncAttributes fa;
+      if ((e = cudaFuncGetAttributes(&fa, sca_tc_kernel<D>)) != cudaSuccess) return e;
+      regs = fa.numRegs;
+    }
+    if (128 * kRegsCtl + 256 * kRegsSoftmax > kThreads * regs) return cudaErrorInvalidConfiguration;
+  }
+#endif
   // the unit counter starts from zero for every launch (stream-ordered)
   unsigned* counter = nullptr;
   if ((e = cudaGetSymbolAddress(reinterpret_cast<void**>(&counter), g_unit_counter)) != cudaSuccess) return e;
