@@ -103,7 +103,7 @@ constexpr int kIssuers = GECKO_SCA_ISSUERS;
 // roles through a ring of kUnitRing slots.  The producer claims at most
 // max(kKStages, kVStages) + 1 units ahead of the slowest reader (its K and V
 // loads lead the MMAs by at most that many iterations, every unit has at
-// least one, and the softmax warps trail the MMA thread by at most one
+// least one, and the softmax warps trail the MMA issuers by at most one
 // unit), so 8 slots are never overwritten before they are read.
 constexpr int kUnitRing = 8;
 
@@ -233,7 +233,7 @@ struct Claims {
   }
 };
 
-// Walks the K/V iterations of one CTA in the order the MMA warp consumes
+// Walks the K/V iterations of one CTA in the order the MMA issuers consume
 // them: its units in the order claimed, and each unit's key tiles in order.
 struct KvWalk {
   int n;            // ordinal of the current unit
@@ -445,7 +445,7 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
     if (lane == 0) {
-      // Three load streams, each in the order the MMA warp consumes them:
+      // Three load streams, each in the order the MMA issuers consume them:
       // Q of every unit, K_m and V_m of every K/V iteration m.  A load
       // first waits until the previous reader of its slot is done: K_m for
       // iteration m - KS, V_m for iteration m + 1 - VS (V_m is read by the
@@ -692,9 +692,11 @@ sca_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       for (int j = ubeg(U, i); j < uend(U, i); ++j) {
         ok = __all_sync(0xffffffffu, mbar_wait(s_full + i, s_cnt & 1, abort_flag, status));
         if (!ok) break;
-        // The QK of the iteration's last active tile is its last MMA, so its
-        // completion (just observed) means K_j and V_{j-1} are no longer read:
-        // one thread of that tile's warpgroup releases them to the producer.
+        // With one MMA thread, the QK of the iteration's last active tile is
+        // its last MMA, so its completion (just observed) means K_j and
+        // V_{j-1} are no longer read: one thread of that tile's warpgroup
+        // releases them to the producer.  (Two issuers release them with
+        // their own commits.)
         if (kIssuers == 1 && (i == 1 || !(U.nt == 2 && j >= U.beg[1])) && warp % 4 == 2 && lane == 0)
           mbar_arrive(it_done + (unit_it0 + (uint32_t)(j - jb)) % IR);
         ++s_cnt;
