@@ -36,6 +36,19 @@
  * caller's next synchronisation.  Every device-side wait is bounded in time;
  * a wait that runs out sets a device status word read by
  * gecko_device_status().
+ *
+ * Environment (read at each call; for tests and cross-checks):
+ *   GECKO_KERNELS=simt    run the CUDA-core kernels for every dtype instead of
+ *                         the tensor-core ones (a second GPU implementation).
+ *   GECKO_CHUNK_PARTS=k   use k CTAs per chunk for the AWM chunk products
+ *                         (1 <= k <= c / 64, tensor-core path only) instead
+ *                         of the library's choice;
+ *                         with one CTA per chunk the chunk kernel also computes
+ *                         the chunk's K_m statistics.
+ *   GECKO_FAIL_ALLOC=1    make every workspace allocation fail
+ *                         (GECKO_ERR_ALLOC), to test callers' error paths.
+ *   GECKO_CEMA_PLAIN=1    load the CEMA inputs with plain loads instead of TMA.
+ * Other values of these variables are ignored.
  */
 #ifndef GECKO_H
 #define GECKO_H
