@@ -119,10 +119,12 @@ def fused_stats(w: Workload) -> bool:
 
 def forward_launches(w: Workload) -> int:
     """Kernels of one forward: [statistics partial + combine] or nothing,
-    chunk products, [Cm image when several CTAs share a chunk at d = 128],
-    prefix, carry, readout, SCA."""
+    chunk products, [the fix-up pass of the fused statistics (its CTAs
+    return at once unless their chunk outgrew the first tile's reference)],
+    [Cm image when several CTAs share a chunk at d = 128], prefix, carry,
+    readout, SCA."""
     fused, parts = awm_plan(w, _sms())
-    return (0 if fused else 2) + 1 + (1 if parts > 1 and w.d == 128 else 0) + 4
+    return (1 if fused else 2) + 1 + (1 if parts > 1 and w.d == 128 else 0) + 4
 
 
 def stage_bytes(w: Workload) -> dict:

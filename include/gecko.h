@@ -207,8 +207,8 @@ int gecko_sca_awm_forward_continue(const void* q, const void* k, const void* v,
  * of the library's device image; each GPU that loads the library holds it
  * until the process exits.  Inputs and outputs are still passed by the
  * caller.  The scratch needs
- *   4 * (2*BH*T/R*d + 4*BH*S*d + (3*S + 1)*BH*d*d) + 2*(2*S + 1)*BH*d*d
- *   bytes (each of the nine regions rounded up to 256 bytes; R = 128 if
+ *   4 * (2*BH*T/R*d + 4*BH*S*d + (3*S + 1)*BH*d*d + BH*S) + 2*(2*S + 1)*BH*d*d
+ *   bytes (each of the eleven regions rounded up to 256 bytes; R = 128 if
  *   c % 128 == 0 else 64, S = T / c, BH = B * H),
  * e.g. B*H = 32, T = 32768, c = 4096, d = 128 needs about 79 MB.  Larger
  * problems are rejected with GECKO_ERR_LIMIT before anything is launched.

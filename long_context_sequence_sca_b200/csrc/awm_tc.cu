@@ -57,7 +57,20 @@ namespace {
 //                with a lazily raised per-feature reference m_f, the column
 //                sums read off the Cm block (rows of Psi sum to 1), and
 //                Bm, Cm normalised in the epilogue, which also writes lse.
-enum ChunkMode { kChunkFwd = 0, kChunkSplit = 1, kChunkE = 2, kChunkFwdStats = 3 };
+//                Given a flag array, only the chunks flagged there run (the
+//                fix-up pass of kChunkFwdStatsFirst).
+//   kChunkFwdStatsFirst  the same statistics with the reference m_f fixed at
+//                the first tile's column maximum, so the later tiles need no
+//                column maxima and no barriers; a chunk whose exponent
+//                arguments climb more than kRefSlack above that reference
+//                is flagged (its results are then unusable) and redone by
+//                kChunkFwdStats.
+enum ChunkMode { kChunkFwd = 0, kChunkSplit = 1, kChunkE = 2, kChunkFwdStats = 3, kChunkFwdStatsFirst = 4 };
+
+// Growth (log2 units) that kChunkFwdStatsFirst allows the exponentials above
+// the first tile's reference: Phi^ <= 2^32, and sums of 4096 such values
+// times V stay far inside the fp32 range.
+constexpr float kRefSlack = 32.f;
 
 // Compute threads of the chunk kernel: two per token row of a 64-token
 // tile.  (Eight compute warps, four threads per row, measured slower: 0.228
@@ -90,7 +103,7 @@ struct ChunkCfg {
   static constexpr int kPartOff = (kMiscOff + 16 + 15) / 16 * 16;
   static_assert(kPartOff % 16 == 0, "16-byte stores of the column maxima");
   // [kChunkCompute / (D / 8) row groups][D] bf16 = 2 KB
-  static constexpr int kBytes = kPartOff + (Mode == kChunkFwdStats ? 2048 : 0);
+  static constexpr int kBytes = kPartOff + (Mode == kChunkFwdStats || Mode == kChunkFwdStatsFirst ? 2048 : 0);
   static constexpr int kAlloc = kBytes + 1024;
   static constexpr uint32_t kTmemCols = Mode == kChunkE ? D : (D == 128 ? 256 : 128);
 };
@@ -104,11 +117,13 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
                                                            const __grid_constant__ CUtensorMap map_km,
                                                            float* __restrict__ lse, float* __restrict__ Bm,
                                                            float* __restrict__ Cm, uint16_t* __restrict__ Cimg,
-                                                           int T, int c, int koff, int parts, int* status) {
+                                                           int T, int c, int koff, int parts, int* flags,
+                                                           int* status) {
   using Cfg = ChunkCfg<D, Mode>;
-  // kChunkFwdStats: the forward products with the chunk's statistics
-  // computed here (d = 128): it writes lse instead of reading it
-  constexpr bool kStats = Mode == kChunkFwdStats;
+  // kChunkFwdStats / kChunkFwdStatsFirst: the forward products with the
+  // chunk's statistics computed here: it writes lse instead of reading it
+  constexpr bool kFirstRef = Mode == kChunkFwdStatsFirst;
+  constexpr bool kStats = Mode == kChunkFwdStats || kFirstRef;
   constexpr bool kFwd = Mode == kChunkFwd || kStats;
   // fused statistics: the column maxima of a tile come from kRG groups of
   // kKT / kRG rows, one thread per (row group, 8 features)
@@ -125,6 +140,8 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
   float* nref2 = reinterpret_cast<float*>(smem + Cfg::kLzOff);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 4);
+  // kChunkFwdStatsFirst: set when an exponent argument exceeded kRefSlack
+  volatile int* outgrown = reinterpret_cast<volatile int*>(smem + Cfg::kMiscOff + 8);
 
   // `parts` CTAs share a chunk (forward mode only): CTA part p takes tiles
   // [p n / parts, (p + 1) n / parts) and adds its products into Bm, Cm
@@ -133,6 +150,8 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
   const int64_t bh = blockIdx.y;
   // the readouts of chunks 1 and 2 read a zero state: their E is never used
   if (Mode == kChunkE && s < 2) return;
+  // the fix-up pass redoes only the chunks that the first-tile pass flagged
+  if (Mode == kChunkFwdStats && flags != nullptr && flags[bh * S + s] == 0) return;
   const int warp = warp_id_uniform(), lane = threadIdx.x % 32;
   const int t0 = part * (c / kKT) / parts;
   const int n_tiles = (part + 1) * (c / kKT) / parts - t0;
@@ -148,6 +167,7 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
     }
     mbar_init(acc_full, 1);
     *abort_flag = 0;
+    *outgrown = 0;
     fence_mbar_init();
   }
   if (Mode != kChunkE && !kStats)
@@ -233,11 +253,16 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
     // fused statistics: this thread's feature f = threadIdx.x (TMEM lane f
     // of the accumulator) and its reference m_f (log2 units)
     float m_f = 0.f;
+    // kChunkFwdStatsFirst: the largest exponent argument of this thread
+    float umax = -INFINITY;
     for (int kt = 0; kt < n_tiles; ++kt) {
       const int st = kt % NS;
+      // column maxima (and the barriers around them) on every tile, or on
+      // the first one only
+      const bool colmax = kStats && (!kFirstRef || kt == 0);
       // V and K_m of this tile have landed (the copy also waited for the
       // MMAs of tile kt - NS to release the stage)
-      if (kStats) {
+      if (colmax) {
         // the compute warps leave the loop together (they meet at named
         // barriers below)
         ok = bar_and(1, kChunkCompute, mbar_wait(v_full + st, (kt / NS) & 1, abort_flag, status));
@@ -246,7 +271,7 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
       }
       if (!ok) break;
       uint8_t* stg = smem + st * Cfg::kStage;
-      if (kStats) {
+      if (colmax) {
         // Column maxima of the K_m tile: thread (rg, g) takes the kKT / kRG
         // rows of group rg for features 8 g .. 8 g + 7, then the thread of
         // feature f combines the kRG row groups.  The thread of feature f
@@ -353,6 +378,7 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
             const uint64_t x2 = pack2(x[a], x[a + 1]);
             float u0, u1, v0, v1;
             unpack2(ffma2(x2, l2e2, nz[j]), u0, u1);
+            if (kFirstRef) umax = fmax3(umax, u0, u1);
             qq[j] = pack_bf16x2(ex2(u0), ex2(u1));
             unpack2(ffma2(x2, l2e2, nmx2), v0, v1);
             e[a] = ex2(v0);
@@ -419,6 +445,7 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
       if (kStats) tc_fence_before();   // orders the TMEM rescale before the next MMA
       mbar_arrive(op_full + st);
     }
+    if (kFirstRef && umax > kRefSlack) *outgrown = 1;
     // epilogue (warps 0-3): accumulator row f = TMEM lane; columns [0, D) = Bm, [D, 2D) = Cm
     if (warp >= 4) ok = false;
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, status));
@@ -488,6 +515,8 @@ __global__ void __launch_bounds__(kChunkThreads, 2) awm_chunk_tc_kernel(const __
   __syncthreads();
   tc_fence_after();
   if (warp == kChunkMmaWarp) tmem_dealloc(tmem, Cfg::kTmemCols);
+  // every chunk's flag is written, so the array needs no clearing
+  if (kFirstRef && threadIdx.x == 0) flags[bh * S + s] = *outgrown;
 }
 
 // Cm_s rounded to bf16 in the carry's K-major 128-byte-swizzled operand
@@ -1081,7 +1110,8 @@ EncodeTiledFn encode_fn() {
 
 template <int D, int Mode>
 cudaError_t chunk_impl(const Problem& p, const void* vsrc, const void* ksrc, float* lse, float* out0,
-                       float* out1, cudaStream_t st, uint16_t* cimg = nullptr, int parts = 1) {
+                       float* out1, cudaStream_t st, uint16_t* cimg = nullptr, int parts = 1,
+                       int* flags = nullptr) {
   using Cfg = ChunkCfg<D, Mode>;
   EncodeTiledFn fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
@@ -1103,7 +1133,7 @@ cudaError_t chunk_impl(const Problem& p, const void* vsrc, const void* ksrc, flo
                                        Cfg::kAlloc);
   if (e != cudaSuccess) return e;
   awm_chunk_tc_kernel<D, Mode><<<dim3(p.S * parts, p.B * p.H), kChunkThreads, Cfg::kAlloc, st>>>(
-      mv, mkm, lse, out0, out1, cimg, (int)p.T, (int)p.c, (int)koff, parts, p.status);
+      mv, mkm, lse, out0, out1, cimg, (int)p.T, (int)p.c, (int)koff, parts, flags, p.status);
   return cudaGetLastError();
 }
 
@@ -1179,9 +1209,25 @@ cudaError_t launch_awm_chunk_tc(const Problem& p, const Workspace& w, cudaStream
   return cudaGetLastError();
 }
 
+// Reference of the fused statistics: taken from each chunk's first tile,
+// with the running-reference kernel redoing the chunks that outgrow it (1),
+// or the running reference for every chunk (0).
+#ifndef GECKO_CHUNK_FIRST_REF
+#define GECKO_CHUNK_FIRST_REF 1
+#endif
+
 cudaError_t launch_awm_chunk_tc_stats(const Problem& p, const Workspace& w, cudaStream_t st) {
-  return p.d == 64 ? chunk_impl<64, kChunkFwdStats>(p, p.v, p.km, w.lse, w.Bm, w.Cm, st)
-                   : chunk_impl<128, kChunkFwdStats>(p, p.v, p.km, w.lse, w.Bm, w.Cm, st, w.Cimg);
+  uint16_t* cimg = p.d == 128 ? w.Cimg : nullptr;
+  if (!GECKO_CHUNK_FIRST_REF)
+    return p.d == 64 ? chunk_impl<64, kChunkFwdStats>(p, p.v, p.km, w.lse, w.Bm, w.Cm, st)
+                     : chunk_impl<128, kChunkFwdStats>(p, p.v, p.km, w.lse, w.Bm, w.Cm, st, cimg);
+  cudaError_t e =
+      p.d == 64 ? chunk_impl<64, kChunkFwdStatsFirst>(p, p.v, p.km, w.lse, w.Bm, w.Cm, st, cimg, 1, w.flags)
+                : chunk_impl<128, kChunkFwdStatsFirst>(p, p.v, p.km, w.lse, w.Bm, w.Cm, st, cimg, 1, w.flags);
+  if (e != cudaSuccess) return e;
+  // the fix-up pass: its CTAs of unflagged chunks return at once
+  return p.d == 64 ? chunk_impl<64, kChunkFwdStats>(p, p.v, p.km, w.lse, w.Bm, w.Cm, st, cimg, 1, w.flags)
+                   : chunk_impl<128, kChunkFwdStats>(p, p.v, p.km, w.lse, w.Bm, w.Cm, st, cimg, 1, w.flags);
 }
 
 cudaError_t launch_awm_chunk_tc_split(const Problem& p, const Workspace& w, cudaStream_t st) {

@@ -35,7 +35,8 @@ size_t workspace_bytes(int64_t BH, int64_t T, int64_t c, int64_t d) {
   const size_t mst = al(sizeof(float) * BH * (S + 1) * d * d);
   const size_t img = al(sizeof(uint16_t) * BH * (S + 1) * d * d);
   const size_t cimg = al(sizeof(uint16_t) * BH * S * d * d);
-  return part + 4 * vec + 2 * mat + mst + img + cimg;
+  const size_t flags = al(sizeof(int) * BH * S);
+  return part + 4 * vec + 2 * mat + mst + img + cimg + flags;
 }
 
 Workspace carve_workspace(void* base, int64_t BH, int64_t T, int64_t c, int64_t d) {
@@ -65,6 +66,8 @@ Workspace carve_workspace(void* base, int64_t BH, int64_t T, int64_t c, int64_t 
   w.Mimg = reinterpret_cast<uint16_t*>(p);
   p += al(sizeof(uint16_t) * BH * (S + 1) * d * d);
   w.Cimg = reinterpret_cast<uint16_t*>(p);
+  p += al(sizeof(uint16_t) * BH * S * d * d);
+  w.flags = reinterpret_cast<int*>(p);
   return w;
 }
 

@@ -47,6 +47,9 @@ struct Workspace {
   // 128-byte-swizzled operand layout (rows f, K = g), written by the forward
   // chunk kernel at d = 128 and read by the tensor-core carry.
   uint16_t* Cimg;
+  // [BH, S]: 1 where the fused statistics' first-tile reference was
+  // outgrown and the chunk has to be redone (written for every chunk).
+  int* flags;
 };
 
 // Column slices of the sequential carries: as wide as still gives about one

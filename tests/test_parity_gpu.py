@@ -206,9 +206,10 @@ def test_awm_keys_growing_within_a_chunk(L, kernels, parts, d, monkeypatch):
     The chunk's log-sum-exp, the state and the readout still match the fp64
     oracle (step 4 of the method: Phi = exp(Km - log z), any real Km).
     parts="1" keeps one CTA per chunk, the form whose chunk kernel computes
-    the chunk statistics itself (raising its reference); by default this
-    small problem shares each chunk among several CTAs after a separate
-    statistics pass."""
+    the chunk statistics itself (from the first tile's reference, every
+    chunk here outgrowing it, so each is redone by the pass that raises
+    its reference); by default this small problem shares each chunk among
+    several CTAs after a separate statistics pass."""
     if kernels:
         monkeypatch.setenv("GECKO_KERNELS", kernels)
     if parts:
@@ -222,6 +223,34 @@ def test_awm_keys_growing_within_a_chunk(L, kernels, parts, d, monkeypatch):
     km = x["km"].float() + t[:, None] * slope[None, :]
     spike = (torch.arange(w.T, device="cuda") % c) == c - 70
     km[..., spike, 2::8] += 40.0
+    x["km"] = km.to(torch.bfloat16)
+    o_sca, o_mem, M, lz = _run(L, x, w.c)
+    r_sca, r_mem, r_M, r_lz = G.forward(*(_np(x[n]) for n in ("q", "k", "v", "qm", "km")), w.c)
+    _check(_np(o_mem), r_mem, w.dtype, "out_mem")
+    _check(_np(M), r_M, w.dtype, "M state")
+    _check(_np(lz), r_lz, w.dtype, "log z")
+    _check(_np(o_sca), r_sca, w.dtype, "out_sca")
+
+
+@pytest.mark.parametrize("d", [128, 64])
+@pytest.mark.parametrize("growth", [15.0, 60.0])
+def test_awm_keys_outgrowing_the_first_tile(L, d, growth, monkeypatch):
+    """One CTA per chunk, the chunk statistics computed in the chunk kernel
+    against a reference taken from each chunk's first tile.  A third of the
+    K_m features climb by `growth` (natural-log units) through the second
+    chunk only.  A climb of 15 keeps the exponentials within the 2^32 the
+    first-tile reference allows, so no chunk is redone; a climb of 60 goes
+    past it, so that chunk alone is redone with a running reference while
+    the other chunks keep their first pass.  Either way the state, log z
+    and both outputs match the fp64 oracle."""
+    monkeypatch.setenv("GECKO_CHUNK_PARTS", "1")
+    w = Workload(f"bf16_outgrow_d{d}", 29, "bf16", 1, 2, 2048, d, 512)
+    x = make_inputs(w, device="cuda")
+    c = w.c
+    pos = torch.arange(w.T, device="cuda")
+    ramp = ((pos // c) == 1).float() * (pos % c).float() / c * growth
+    km = x["km"].float()
+    km[..., 1::3] += ramp[:, None]
     x["km"] = km.to(torch.bfloat16)
     o_sca, o_mem, M, lz = _run(L, x, w.c)
     r_sca, r_mem, r_M, r_lz = G.forward(*(_np(x[n]) for n in ("q", "k", "v", "qm", "km")), w.c)
