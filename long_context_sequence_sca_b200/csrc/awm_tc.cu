@@ -19,10 +19,11 @@
 // to V in one 128-byte-swizzled, MN-major stage [V | Psi | Phi], so a single
 // tcgen05.mma with M = d, N = 2d accumulates [Phi^T V | Phi^T Psi] in TMEM.
 // In the forward (one CTA per chunk) the kernel also computes each chunk's
-// per-feature log-sum-exp lse_s: it exponentiates against a running
-// per-feature reference (the column maximum of the tiles seen so far, raised
-// lazily with a rescale of the accumulated rows), reads the column sums of
-// those exponentials off the Cm block (every row of Psi sums to 1) and
+// per-feature log-sum-exp lse_s: it exponentiates against a per-feature
+// reference (the first tile's column maximum; a chunk whose keys climb too
+// far above it is redone with a running maximum raised lazily with a
+// rescale of the accumulated rows), reads the column sums of those
+// exponentials off the Cm block (every row of Psi sums to 1) and
 // normalises Bm and Cm in the epilogue, so K_m is read once.
 //
 // awm_carry_tc_kernel (d = 128): the sequential carry, one CTA per (b, h),

@@ -86,7 +86,9 @@ cudaError_t launch_sca_tc(const Problem& p, cudaStream_t st);
 // parts > 1: that many CTAs share each chunk and add into Bm, Cm (zeroed
 // here), and the bf16 image of Cm is made by a separate pass
 cudaError_t launch_awm_chunk_tc(const Problem& p, const Workspace& w, cudaStream_t st, int parts = 1);
-// the chunk products with each chunk's log-sum-exp (Workspace::lse) computed in the same pass
+// the chunk products with each chunk's log-sum-exp (Workspace::lse) computed
+// in the same pass (two launches: against the first tile's reference, then a
+// redo of the chunks flagged in Workspace::flags)
 cudaError_t launch_awm_chunk_tc_stats(const Problem& p, const Workspace& w, cudaStream_t st);
 cudaError_t launch_awm_readout_tc(const Problem& p, const Workspace& w, cudaStream_t st);
 // The carry on the tensor cores (d = 128; bf16 hi + lo operands, ~fp32 products)
