@@ -27,6 +27,31 @@ def test_flops_and_bytes_headline():
     assert bench.io_bytes(w) == 7 * 32 * 32768 * 128 * 2
 
 
+def test_awm_plan_and_launch_count():
+    """The plan bench.py assumes when it counts launches (the library's own
+    rule: k CTAs per chunk when that saves a quarter of waves x (tiles per
+    CTA + 2), the statistics fused only with one CTA per chunk)."""
+    sms = 148
+    # 256 chunks fill one wave of two CTAs per SM: one CTA per chunk, fused
+    # statistics (first-tile pass, redo pass, prefix, carry, readout, SCA)
+    assert bench.awm_plan(bench.WORKLOADS["bf16_h32_c4096"], sms) == (True, 1)
+    # 32 chunks of 64 tiles: nine CTAs each (288 CTAs, 7-8 tiles, one wave)
+    assert bench.awm_plan(bench.WORKLOADS["bf16_h4_c4096"], sms) == (False, 9)
+    # c = 256 has 4 tiles per chunk: never split
+    assert bench.awm_plan(bench.WORKLOADS["bf16_many_chunks"], sms) == (True, 1)
+    # fp32 takes the CUDA-core kernels: separate statistics pass
+    assert bench.awm_plan(bench.WORKLOADS["fp32_small"], sms) == (False, 1)
+    # one wave with P CTAs per chunk costs (n + 2P) / P against n + 2 for one
+    w = bench.WORKLOADS["bf16_h4_c4096"]
+    n = w.c // 64
+    assert (n + 2 * 9) / 9 <= 0.75 * (n + 2)
+    if not torch.cuda.is_available():   # the counts below assume 148 SMs
+        # fused: chunk pass, redo pass, prefix, carry, readout, SCA
+        assert bench.forward_launches(bench.WORKLOADS["bf16_h32_c4096"]) == 6
+        # split: partial + combine + prefix, chunk, Cm image, carry, readout, SCA
+        assert bench.forward_launches(bench.WORKLOADS["bf16_h4_c4096"]) == 8
+
+
 def test_secondary_rooflines_at_the_bench_workload():
     """HBM and SFU bounds: 1.88 GB in 3.44 ms is 546 GB/s; 5.91e9
     exponentials in 2.97 ms at 1965 MHz against 16 per clock on 148 SMs
