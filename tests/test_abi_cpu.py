@@ -161,3 +161,33 @@ def test_train_forward_rejects_bad_lse(so):
 def test_context_parallel_host_validation_rejects(so, call, code):
     assert call() == code
     assert L.gecko_last_error()
+
+
+def _noalloc_bytes(BH, T, c, d):
+    """Working memory of the no-allocation entry point as include/gecko.h
+    states it: eleven regions, each rounded up to 256 bytes."""
+    al = lambda x: (x + 255) // 256 * 256
+    S, R = T // c, (128 if c % 128 == 0 else 64)
+    regions = [8 * BH * (T // R) * d] + [4 * BH * S * d] * 4 + [4 * BH * S * d * d] * 2 + \
+              [4 * BH * (S + 1) * d * d, 2 * BH * (S + 1) * d * d, 2 * BH * S * d * d, 4 * BH * S]
+    return sum(al(r) for r in regions)
+
+
+# (768, 256, 64): the boundary moves if the smallest region (the per-chunk
+# flags) is left out of the count
+@pytest.mark.parametrize("T,c,d", [(32768, 4096, 128), (65536, 512, 128), (8192, 256, 64), (4096, 64, 64),
+                                   (768, 256, 64)])
+def test_noalloc_limit_follows_the_documented_size(so, T, c, d):
+    """The largest B*H whose documented working memory fits the fixed scratch
+    is accepted on the host; one more (b, h) is rejected with GECKO_ERR_LIMIT
+    before any CUDA call."""
+    import torch
+    limit = 80 << 20
+    bh = 1
+    while _noalloc_bytes(bh + 1, T, c, d) <= limit:
+        bh += 1
+    assert _noalloc_bytes(bh, T, c, d) <= limit < _noalloc_bytes(bh + 1, T, c, d)
+    assert L.gecko_sca_awm_forward_noalloc(*([FAKE] * 7), 1, bh + 1, T, c, d, 1, None) == 8
+    if not torch.cuda.is_available():
+        # passes the size check and stops at the first CUDA call (no device here)
+        assert L.gecko_sca_awm_forward_noalloc(*([FAKE] * 7), 1, bh, T, c, d, 1, None) == 5
