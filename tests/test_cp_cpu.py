@@ -162,6 +162,46 @@ def _worker_groups(rank, port, errq):
         errq.put((rank, repr(e), None))
 
 
+class FailingBackend(OracleBackend):
+    """A rank whose first phase fails on the host: it raises, or it stalls
+    (sleeps past the group's timeout before going on)."""
+
+    def __init__(self, mode):
+        self.mode = mode
+
+    def segment_logsum(self, seg, c):
+        if self.mode == "raise":
+            raise RuntimeError("injected failure")
+        import time
+        time.sleep(8)
+        return super().segment_logsum(seg, c)
+
+
+def _worker_fail(rank, P, port, fail_rank, mode, errq):
+    """Every rank runs cp_forward under a 3 s process-group timeout; rank
+    `fail_rank` fails in its first phase.  Each rank reports how its call
+    ended, then exits without tearing the group down (a peer may be gone)."""
+    from datetime import timedelta
+    try:
+        os.environ["MASTER_ADDR"] = "127.0.0.1"
+        os.environ["MASTER_PORT"] = str(port)
+        dist.init_process_group("gloo", rank=rank, world_size=P, timeout=timedelta(seconds=3))
+        x, T = _inputs(P)
+        Tr = T // P
+        seg = {n: torch.from_numpy(a[:, :, rank * Tr:(rank + 1) * Tr].copy()) for n, a in x.items()}
+        be = FailingBackend(mode) if rank == fail_rank else OracleBackend()
+        try:
+            cp.cp_forward(seg, 4, backend=be)
+            errq.put((rank, "completed"))
+        except Exception as e:
+            errq.put((rank, f"{type(e).__name__}: {e}"[:300]))
+    except Exception as e:  # pragma: no cover - reported to the parent
+        errq.put((rank, f"setup {e!r}"))
+    errq.close()
+    errq.join_thread()
+    os._exit(0)
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
@@ -207,3 +247,36 @@ def test_two_sequences_in_two_process_groups():
     res = _run(4, groups=True)
     for rank, ok_sca, ok_mem in res:
         assert ok_sca is True and ok_mem is True, res
+
+
+@pytest.mark.parametrize("fail_rank,mode", [(0, "raise"), (1, "raise"), (1, "stall")])
+def test_a_failed_rank_ends_the_others_calls(fail_rank, mode):
+    """Failure detection on the host: when one rank of a context-parallel
+    forward fails before its collectives (raises and leaves, or stalls past
+    the group's timeout), the other ranks' calls end with an error (the
+    gather's peer closed, or the timeout) instead of waiting for good."""
+    import time
+    P = 3
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_fail, args=(r, P, port, fail_rank, mode, q)) for r in range(P)]
+    t0 = time.time()
+    for p in procs:
+        p.start()
+    res = []
+    try:
+        for _ in range(P):
+            res.append(q.get(timeout=120))
+    finally:
+        for p in procs:
+            p.join(timeout=30)
+            if p.is_alive():
+                p.kill()
+    res = dict(res)
+    if mode == "raise":
+        assert "injected failure" in res[fail_rank], res
+    for r in range(P):
+        if r != fail_rank:
+            assert res[r] != "completed" and not res[r].startswith("setup"), res
+    assert time.time() - t0 < 100
