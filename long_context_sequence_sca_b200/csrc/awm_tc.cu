@@ -69,8 +69,9 @@ namespace {
 enum ChunkMode { kChunkFwd = 0, kChunkSplit = 1, kChunkE = 2, kChunkFwdStats = 3, kChunkFwdStatsFirst = 4 };
 
 // Growth (log2 units) that kChunkFwdStatsFirst allows the exponentials above
-// the first tile's reference: Phi^ <= 2^32, and sums of 4096 such values
-// times V stay far inside the fp32 range.
+// the first tile's reference: Phi^ <= 2^32, so the sums over a chunk of up
+// to 2^31 tokens stay below 2^63, and their products with values |V| < 2^64
+// inside the fp32 range.
 constexpr float kRefSlack = 32.f;
 
 // Compute threads of the chunk kernel: two per token row of a 64-token
